@@ -1,0 +1,381 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each test ties the oracle to a fact fixed by the method's definition or by
+mathematics: a hand-worked example, library routines it must reduce to
+(PyTorch's scaled_dot_product_attention in float64), a separately written
+brute-force hierarchical sum, exhaustive subset search, closed forms and
+invariants.  A dropped term, a wrong sign or index, or a transposed operand in
+the oracle fails at least one of them (see test_oracle_mutants.py).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rand_case(seed, B, L, H, Hkv, d, S, lm_scale=1.0):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((B, L, H, d))
+    K = rng.standard_normal((B, Hkv, L, d))
+    V = rng.standard_normal((B, Hkv, L, d))
+    lm = lm_scale * rng.standard_normal((B, Hkv, L // S, d))
+    return Q, K, V, lm
+
+
+def sdpa_causal(Q, K, V, G, scale=None):
+    """Causal attention per head with PyTorch's SDPA in float64 (GQA by repeat)."""
+    q = torch.from_numpy(Q).permute(0, 2, 1, 3)                  # [B,H,L,d]
+    k = torch.from_numpy(K).repeat_interleave(G, dim=1)           # [B,H,L,d]
+    v = torch.from_numpy(V).repeat_interleave(G, dim=1)
+    o = F.scaled_dot_product_attention(q, k, v, is_causal=True, scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()                           # [B,L,H,d]
+
+
+def sdpa_full(q, k, v, scale=None):
+    """Non-causal attention of query rows q [n,d] over k,v [m,d] (float64 SDPA)."""
+    o = F.scaled_dot_product_attention(torch.from_numpy(q)[None, None],
+                                       torch.from_numpy(k)[None, None],
+                                       torch.from_numpy(v)[None, None], scale=scale)
+    return o[0, 0].numpy()
+
+
+# --------------------------------------------------------------------------- hand example
+def test_hand_worked_example(oracle_lib):
+    g = json.load(open(os.path.join(GOLDEN, "hand_example.json")))
+    L, H, d = g["L"], g["H"], g["d"]
+    Q = np.broadcast_to(np.array(g["Q_per_position"]), (1, L, H, d)).copy()
+    K = np.array(g["K"])[None, None]
+    V = np.array(g["V"])[None, None]
+    lm = np.array(g["lm"])[None, None]
+    r = oracle_lib.prefill(Q, K, V, lm, g["S"], g["topk"], g["own_chunk"], g["scale"])
+    np.testing.assert_allclose(r["O"], np.array(g["expected_O"]), atol=1e-12, rtol=0)
+    np.testing.assert_array_equal(r["idx"][:, 0, :], np.array(g["expected_idx"]))
+    np.testing.assert_allclose(r["sbar"][:, 0, :], np.array(g["expected_sbar"]), atol=1e-12)
+    np.testing.assert_allclose(r["w"], np.array(g["expected_w"]), atol=1e-12)
+
+
+# --------------------------------------------------------------------------- reductions
+@pytest.mark.parametrize("L,S", [(16, 16), (13, 16), (64, 64)])
+@pytest.mark.parametrize("H,Hkv", [(4, 1), (4, 2), (2, 2)])
+def test_single_chunk_is_causal_attention(oracle_lib, L, S, H, Hkv):
+    """With one chunk (L <= S) nothing is selectable; O is textbook causal attention."""
+    d = 8
+    Q, K, V, _ = rand_case(1, 2, L, H, Hkv, d, S)
+    lm = np.zeros((2, Hkv, L // S, d))
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk=3, own_chunk=1)
+    ref = sdpa_causal(Q, K, V, H // Hkv)                          # default scale 1/sqrt(d)
+    np.testing.assert_allclose(r["O"].reshape(ref.shape), ref, atol=1e-12, rtol=0)
+    assert (r["idx"] == -1).all() and (r["w"] == 0).all()
+
+
+def test_own_chunk_matches_causal_prefix_of_every_chunk(oracle_lib):
+    """topk=1 with one visible chunk forced to be weight 1: the own term alone is
+    the causal attention restricted to the chunk (checked with SDPA per chunk)."""
+    B, L, H, Hkv, d, S = 1, 48, 2, 1, 4, 16
+    Q, K, V, lm = rand_case(2, B, L, H, Hkv, d, S)
+    r0 = oracle_lib.prefill(Q, K, V, lm, S, topk=2, own_chunk=0)
+    r1 = oracle_lib.prefill(Q, K, V, lm, S, topk=2, own_chunk=1)
+    own = (r1["O"] - r0["O"]).reshape(B, L, H, d)
+    for c in range(L // S):
+        sl = slice(c * S, (c + 1) * S)
+        ref = sdpa_causal(Q[:, sl], K[:, :, sl], V[:, :, sl], H // Hkv)
+        np.testing.assert_allclose(own[:, sl], ref, atol=1e-12)
+
+
+def test_topk1_is_attention_over_argmax_chunk(oracle_lib):
+    B, L, H, Hkv, d, S = 2, 96, 4, 2, 8, 16
+    Q, K, V, lm = rand_case(3, B, L, H, Hkv, d, S)
+    G = H // Hkv
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk=1, own_chunk=0)
+    O = r["O"].reshape(B, L, H, d)
+    scale = 1 / math.sqrt(d)
+    for b in range(B):
+        for t in range(L):
+            nvis = t // S
+            for g in range(Hkv):
+                if nvis == 0:
+                    assert r["idx"][b * L + t, g, 0] == -1
+                    assert np.all(O[b, t, g * G:(g + 1) * G] == 0)
+                    continue
+                qbar = Q[b, t, g * G:(g + 1) * G].mean(axis=0)
+                i = int(np.argmax(lm[b, g, :nvis] @ qbar))       # first maximum = lowest index
+                assert r["idx"][b * L + t, g, 0] == i
+                ref = sdpa_full(Q[b, t, g * G:(g + 1) * G], K[b, g, i * S:(i + 1) * S],
+                                V[b, g, i * S:(i + 1) * S], scale)
+                np.testing.assert_allclose(O[b, t, g * G:(g + 1) * G], ref, atol=1e-12)
+                np.testing.assert_array_equal(r["w"][b * L + t, g * G:(g + 1) * G, 0], 1.0)
+
+
+def brute_force_hierarchical(Q, K, V, lm, S, own_chunk, scale):
+    """Every visible chunk fused (no selection, no sort): written independently
+    of the oracle with vectorised numpy and SDPA for the in-chunk attention."""
+    B, L, H, d = Q.shape
+    Hkv = K.shape[1]
+    G = H // Hkv
+    O = np.zeros_like(Q)
+    for b in range(B):
+        for h in range(H):
+            g = h // G
+            # chunk outputs o[t, i] for all t and all complete chunks i
+            Nc = L // S
+            Kc = K[b, g, :Nc * S].reshape(Nc, S, d)
+            Vc = V[b, g, :Nc * S].reshape(Nc, S, d)
+            logits = np.einsum("td,isd->tis", Q[b, :, h], Kc) * scale       # [L,Nc,S]
+            p = np.exp(logits - logits.max(axis=2, keepdims=True))
+            p /= p.sum(axis=2, keepdims=True)
+            o_chunks = np.einsum("tis,isd->tid", p, Vc)                       # [L,Nc,d]
+            s = Q[b, :, h] @ lm[b, g].T * scale                               # [L,Nc]
+            for t in range(L):
+                nvis = t // S
+                if nvis:
+                    e = np.exp(s[t, :nvis] - s[t, :nvis].max())
+                    O[b, t, h] = (e / e.sum()) @ o_chunks[t, :nvis]
+        if own_chunk:
+            O[b] += sdpa_chunked_causal(Q[b:b + 1], K[b:b + 1], V[b:b + 1], S, G, scale)[0]
+    return O
+
+
+def sdpa_chunked_causal(Q, K, V, S, G, scale):
+    B, L, H, d = Q.shape
+    out = np.zeros_like(Q)
+    for c0 in range(0, L, S):
+        sl = slice(c0, min(L, c0 + S))
+        out[:, sl] = sdpa_causal(Q[:, sl], K[:, :, sl], V[:, :, sl], G, scale)
+    return out
+
+
+@pytest.mark.parametrize("own_chunk", [0, 1])
+@pytest.mark.parametrize("L", [128, 120])
+def test_topk_all_visible_matches_bruteforce_sum(oracle_lib, own_chunk, L):
+    B, H, Hkv, d, S = 2, 4, 2, 8, 16
+    Q, K, V, lm = rand_case(4, B, L, H, Hkv, d, S)
+    scale = 0.3
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk=L // S, own_chunk=own_chunk, scale=scale)
+    ref = brute_force_hierarchical(Q, K, V, lm, S, own_chunk, scale)
+    np.testing.assert_allclose(r["O"].reshape(ref.shape), ref, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- invariants
+def test_fusion_weights_sum_to_one(oracle_lib):
+    B, L, H, Hkv, d, S = 1, 256, 8, 2, 16, 16
+    Q, K, V, lm = rand_case(5, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk=4)
+    nvis = (np.arange(L) // S)
+    wsum = r["w"].sum(axis=2)
+    np.testing.assert_allclose(wsum[nvis >= 1], 1.0, atol=1e-12)
+    assert np.all(wsum[nvis == 0] == 0)
+    assert np.all(r["w"] >= 0)
+    # padded slots carry weight 0 and index -1
+    pad = r["idx"] < 0
+    assert np.all(r["w"].reshape(L, Hkv, H // Hkv, 4)[np.repeat(pad[:, :, None, :], H // Hkv, 2)] == 0)
+
+
+def test_unselected_chunks_do_not_matter(oracle_lib):
+    """Changing K/V of every chunk a query did not select leaves its output bit-identical."""
+    B, L, H, Hkv, d, S, topk = 1, 256, 4, 1, 8, 16, 3
+    Q, K, V, lm = rand_case(6, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk)
+    rng = np.random.default_rng(99)
+    for t in (40, 130, 255):
+        sel = set(int(i) for i in r["idx"][t, 0] if i >= 0)
+        K2, V2 = K.copy(), V.copy()
+        c_t = t // S
+        for i in range(L // S):
+            if i not in sel and i != c_t:
+                K2[0, 0, i * S:(i + 1) * S] = rng.standard_normal((S, d)) * 5
+                V2[0, 0, i * S:(i + 1) * S] = rng.standard_normal((S, d)) * 5
+        # keys after t inside the own chunk are causally masked too
+        K2[0, 0, t + 1:(c_t + 1) * S] = 7.0
+        V2[0, 0, t + 1:(c_t + 1) * S] = -7.0
+        r2 = oracle_lib.prefill(Q, K2, V2, lm, S, topk, rows=np.array([t]))
+        assert np.array_equal(r2["O"][0], r["O"][t])
+        assert np.array_equal(r2["idx"][0], r["idx"][t])
+
+
+def test_selection_is_best_subset_by_exhaustive_search(oracle_lib):
+    """Tiny case: the selected set maximises the summed group score over all
+    subsets of the visible chunks of size min(K, nvis), and ranks them in order."""
+    B, L, H, Hkv, d, S, topk = 1, 256, 2, 2, 4, 16, 3
+    Q, K, V, lm = rand_case(7, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk, scale=1.0)
+    for t in range(0, L, 7):
+        nvis = t // S
+        for g in range(Hkv):
+            qbar = Q[0, t, g:g + 1].mean(axis=0)            # G=1 here
+            s = lm[0, g, :nvis] @ qbar
+            m = min(topk, nvis)
+            best = max(itertools.combinations(range(nvis), m), key=lambda c: sum(s[list(c)]),
+                       default=())
+            got = [int(i) for i in r["idx"][t, g] if i >= 0]
+            assert sorted(got) == sorted(best)
+            assert all(s[got[j]] >= s[got[j + 1]] for j in range(len(got) - 1))
+
+
+def test_ties_go_to_lowest_index(oracle_lib):
+    B, L, H, Hkv, d, S, topk = 1, 128, 2, 1, 4, 16, 2
+    Q, K, V, _ = rand_case(8, B, L, H, Hkv, d, S)
+    lm = np.zeros((1, 1, L // S, d))
+    lm[0, 0, :] = np.array([1.0, 0.5, -0.25, 2.0])   # all chunks tie exactly
+    lm[0, 0, 5] *= 2.0                                 # chunk 5 strictly best when qbar.l0 > 0
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk)
+    for t in range(S, L):
+        nvis = t // S
+        qbar = Q[0, t].mean(axis=0)
+        s0 = float(lm[0, 0, 0] @ qbar)
+        got = [int(i) for i in r["idx"][t, 0] if i >= 0]
+        if nvis <= 5 or s0 == 0:
+            assert got == list(range(min(topk, nvis)))
+        elif s0 > 0:
+            assert got == [5, 0]
+        else:  # chunk 5 is the unique worst; lowest-index ties fill the set
+            assert got == [0, 1]
+
+
+# --------------------------------------------------------------------------- landmarks
+def test_dhsa_landmark_closed_form(oracle_lib):
+    S, d = 64, 8
+    K = np.zeros((1, 1, 3 * S + 5, d))
+    # dyadic constants: every partial sum is exact, so the closed form holds bit for bit
+    consts = [np.arange(d) * 0.5 - 1, np.full(d, 3.25), np.arange(d) * -0.375 + 1.125]
+    for i, c in enumerate(consts):
+        K[0, 0, i * S:(i + 1) * S] = c
+    lm = oracle_lib.landmarks(K, S)
+    assert lm.shape == (1, 1, 3, d)          # the partial tail chunk has no landmark
+    for i, c in enumerate(consts):
+        np.testing.assert_array_equal(lm[0, 0, i], 8.0 * c)   # sqrt(64) * mean of a constant
+
+
+def test_dhsa_landmark_matches_numpy_mean(oracle_lib):
+    rng = np.random.default_rng(10)
+    S = 16
+    K = rng.standard_normal((2, 3, 5 * S + 3, 8))
+    lm = oracle_lib.landmarks(K, S)
+    ref = math.sqrt(S) * K[:, :, :5 * S].reshape(2, 3, 5, S, 8).mean(axis=3)
+    np.testing.assert_allclose(lm, ref, atol=1e-13)
+
+
+def test_dhsa_mode_equals_explicit_landmarks(oracle_lib):
+    B, L, H, Hkv, d, S = 1, 160, 4, 2, 8, 16
+    Q, K, V, _ = rand_case(11, B, L, H, Hkv, d, S)
+    lm = math.sqrt(S) * K[:, :, :(L // S) * S].reshape(B, Hkv, L // S, S, d).mean(axis=3)
+    r1 = oracle_lib.prefill(Q, K, V, None, S, 3)
+    r2 = oracle_lib.prefill(Q, K, V, lm, S, 3)
+    np.testing.assert_array_equal(r1["idx"], r2["idx"])
+    np.testing.assert_allclose(r1["O"], r2["O"], atol=1e-12)
+
+
+# --------------------------------------------------------------------------- GQA
+def test_duplicated_heads_match_single_head_group(oracle_lib):
+    """G identical query heads select what one head selects, and each head's
+    output equals the G=1 output."""
+    B, L, d, S, topk = 1, 192, 8, 16, 4
+    Q1, K, V, lm = rand_case(12, B, L, 1, 1, d, S)
+    r1 = oracle_lib.prefill(Q1, K, V, lm, S, topk)
+    Q4 = np.repeat(Q1, 4, axis=2)
+    r4 = oracle_lib.prefill(Q4, K, V, lm, S, topk)
+    np.testing.assert_array_equal(r1["idx"], r4["idx"])
+    for h in range(4):
+        np.testing.assert_allclose(r4["O"][:, h], r1["O"][:, 0], atol=1e-13)
+
+
+def test_group_selection_uses_mean_of_heads(oracle_lib):
+    """Group score = mean over heads: a group whose heads disagree picks the
+    chunks best for the average, checked against a direct per-head sum."""
+    B, L, H, Hkv, d, S, topk = 1, 256, 4, 1, 8, 16, 2
+    Q, K, V, lm = rand_case(13, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk)
+    for t in range(S, L, 11):
+        nvis = t // S
+        per_head = np.stack([lm[0, 0, :nvis] @ Q[0, t, h] for h in range(H)])   # [H,nvis]
+        total = per_head.sum(axis=0)
+        order = sorted(range(nvis), key=lambda i: (-total[i], i))[:topk]
+        assert [int(i) for i in r["idx"][t, 0] if i >= 0] == order
+        np.testing.assert_allclose(r["sbar"][t, 0, :len(order)],
+                                   total[order] / H / math.sqrt(d), atol=1e-12)
+
+
+# --------------------------------------------------------------------------- needles
+def test_planted_needles_rank_first(oracle_lib):
+    from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_prefill_inputs
+    wl = WORKLOADS["long_prefill_bf16"].with_(L=4096, B=1)
+    x = make_prefill_inputs(wl, "cpu")
+    probes = np.array(x["probe_pos"][:64])
+    r = oracle_lib.prefill(x["Q"], x["K"], x["V"], None, wl.S, wl.topk, rows=probes)
+    needles = x["needle_chunks"]
+    for n, t in enumerate(probes):
+        vis = [c for c in needles if c < t // wl.S]
+        assert vis
+        for g in range(wl.Hkv):
+            top = [int(i) for i in r["idx"][n, g][:len(vis)]]
+            assert sorted(top) == sorted(vis), (t, g, top, vis)
+
+
+# --------------------------------------------------------------------------- decode
+def test_decode_equals_prefill_row_at_position_Lc(oracle_lib):
+    """Decode's query at position Lc sees all Lc/S chunks and has no own term:
+    it equals the prefill row t = Lc of a sequence one token longer with
+    own_chunk = 0."""
+    B, H, Hkv, d, S, topk = 2, 4, 2, 8, 16, 3
+    Lc = 8 * S
+    rng = np.random.default_rng(14)
+    q = rng.standard_normal((B, H, d))
+    K = rng.standard_normal((B, Hkv, Lc, d))
+    V = rng.standard_normal((B, Hkv, Lc, d))
+    lm = rng.standard_normal((B, Hkv, Lc // S, d))
+    dec = oracle_lib.decode(q, K, V, lm, S, topk)
+    Lp = Lc + 1
+    Kp = np.concatenate([K, rng.standard_normal((B, Hkv, 1, d))], axis=2)
+    Vp = np.concatenate([V, rng.standard_normal((B, Hkv, 1, d))], axis=2)
+    Qp = np.zeros((B, Lp, H, d))
+    Qp[:, Lc] = q
+    rows = np.array([b * Lp + Lc for b in range(B)])
+    pre = oracle_lib.prefill(Qp, Kp, Vp, lm, S, topk, own_chunk=0, rows=rows)
+    np.testing.assert_array_equal(dec["idx"], pre["idx"])
+    np.testing.assert_allclose(dec["O"], pre["O"], atol=1e-13)
+
+
+def test_decode_bruteforce(oracle_lib):
+    B, H, Hkv, d, S, topk = 3, 8, 2, 16, 16, 4
+    Lc = 12 * S
+    rng = np.random.default_rng(15)
+    q = rng.standard_normal((B, H, d))
+    K = rng.standard_normal((B, Hkv, Lc, d))
+    V = rng.standard_normal((B, Hkv, Lc, d))
+    lm = rng.standard_normal((B, Hkv, Lc // S, d))
+    dec = oracle_lib.decode(q, K, V, lm, S, topk)
+    G = H // Hkv
+    scale = 1 / math.sqrt(d)
+    for b in range(B):
+        for g in range(Hkv):
+            s = lm[b, g] @ q[b, g * G:(g + 1) * G].mean(axis=0)
+            order = np.lexsort((np.arange(len(s)), -s))[:topk]
+            np.testing.assert_array_equal(dec["idx"][b, g], order)
+            for h in range(g * G, (g + 1) * G):
+                logit = lm[b, g, order] @ q[b, h] * scale
+                wgt = np.exp(logit - logit.max())
+                wgt /= wgt.sum()
+                o = sum(wgt[j] * sdpa_full(q[b, h][None], K[b, g, i * S:(i + 1) * S],
+                                           V[b, g, i * S:(i + 1) * S], scale)[0]
+                        for j, i in enumerate(order))
+                np.testing.assert_allclose(dec["O"][b, h], o, atol=1e-12)
+
+
+def test_decode_fewer_chunks_than_topk(oracle_lib):
+    B, H, Hkv, d, S, topk = 1, 2, 1, 4, 16, 8
+    rng = np.random.default_rng(16)
+    q = rng.standard_normal((B, H, d))
+    K = rng.standard_normal((B, Hkv, 3 * S, d))
+    V = rng.standard_normal((B, Hkv, 3 * S, d))
+    lm = rng.standard_normal((B, Hkv, 3, d))
+    dec = oracle_lib.decode(q, K, V, lm, S, topk)
+    assert sorted(dec["idx"][0, 0, :3].tolist()) == [0, 1, 2]
+    assert (dec["idx"][0, 0, 3:] == -1).all()
+    assert np.isinf(dec["gap"][0, 0])
+    np.testing.assert_allclose(dec["w"].sum(-1), 1.0, atol=1e-12)
