@@ -1,0 +1,488 @@
+"""Benchmark: hierarchical chunk-sparse landmark attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-decode] [--no-e2e] [--no-cpu-baseline]
+
+One step = one full hsa_prefill call (landmarks when DHSA, selection, work
+list, in-chunk attention, fusion, own-chunk term) over one batch of the
+workload, inputs resident in HBM.  ``value`` is algorithmic TFLOP/s summed
+over ranks / max-over-ranks device time (weak scaling: every rank runs its own
+independent batch, seeded by rank; no collective on the data path).  The same
+JSON line carries the 32M-context decode figure (tokens/s and HBM roofline),
+the roofline of the dominant kernel timed live with CUDA events on the
+launching stream, an end-to-end figure through host buffers, the SM clocks
+sampled during the timed region and the fp64 CPU oracle timed on a bounded
+sample of the same workload.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference for this
+method) on the host cores, each step a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0, "source": "fallback"}
+L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
+SM_COUNT = 148
+
+
+# ----------------------------------------------------------------------------- work counts
+def prefill_token_counts(wl):
+    t = np.arange(wl.L, dtype=np.int64)
+    nvis = t // wl.S
+    keff = np.minimum(wl.topk, nvis)
+    own = (t - wl.S * nvis + 1) if wl.own_chunk else np.zeros_like(t)
+    return nvis, keff, own
+
+
+def prefill_flops(wl) -> dict:
+    """Algorithmic FLOPs of one prefill call (what the method must compute):
+    selection once per KV group, fusion logits, in-chunk QK^T and PV, own-chunk
+    causal attention.  Softmax exponentials and dense work avoided are not counted."""
+    nvis, keff, own = prefill_token_counts(wl)
+    d, H, Hkv, S, B = wl.d, wl.H, wl.Hkv, wl.S, wl.B
+    sel = B * float((Hkv * 2 * d * nvis).sum())
+    fuse = B * float((H * 2 * d * keff).sum())
+    chunk = B * float((H * 4 * d * S * keff).sum())
+    ownf = B * float((H * 4 * d * own).sum())
+    return {"selection": sel, "fusion": fuse, "in_chunk": chunk, "own_chunk": ownf,
+            "total": sel + fuse + chunk + ownf, "attention_kernel": chunk + ownf}
+
+
+def decode_bytes(wl, lm_elem_bytes=2) -> float:
+    """Algorithmic HBM bytes of one decode step: every visible landmark, the K
+    and V of the selected chunks, q and O.  The full cache is never read."""
+    Nc = wl.L // wl.S
+    el = 2 if wl.dtype == "bf16" else 4
+    per_seq = (wl.Hkv * Nc * wl.d * lm_elem_bytes + wl.Hkv * min(wl.topk, Nc) * wl.S * wl.d * el * 2
+               + 2 * wl.H * wl.d * el)
+    return float(wl.B * per_seq)
+
+
+# ----------------------------------------------------------------------------- environment
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.uuid:
+            cmd[1:1] = ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, src_files) -> float | None:
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current source of that kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("source_hash") != kernel_source_hash(src_files):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(dist, value_units: float, seconds: float, device=None):
+    """Whole-job throughput: units summed over ranks / max-over-ranks time."""
+    if dist is None:
+        return value_units, seconds
+    import torch
+    t = torch.tensor([value_units, seconds], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    u = t[:1].clone()
+    s = t[1:].clone()
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    dist.all_reduce(s, op=dist.ReduceOp.MAX)
+    return float(u.item()), float(s.item())
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, dist, rank, world):
+    import torch
+
+    import hierarchical_chunk_sparse_landmark_b200 as hsa
+    from hierarchical_chunk_sparse_landmark_b200.workloads import (WORKLOADS,
+                                                                   make_decode_inputs,
+                                                                   make_prefill_inputs)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    wl = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    x = make_prefill_inputs(wl, dev)
+    flops = prefill_flops(wl)
+    out = torch.empty_like(x["Q"])
+    ws = hsa.workspace(hsa.prefill_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S,
+                                                  wl.topk), dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n_ev = 5
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+                for _ in range(args.steps)]
+
+    def step():
+        hsa.prefill(x["Q"], x["K"], x["V"], x["lm"], S=wl.S, topk=wl.topk,
+                    own_chunk=wl.own_chunk, out=out, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+        flush.fill_(1)
+    hsa.check(ws)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    launches = 0
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as clk:
+        for i in range(args.steps):
+            hsa.set_stage_events(stage_ev[i])
+            step()
+            launches += hsa.last_call_launches()
+            hsa.set_stage_events([])
+            flush.fill_(1)           # L2 flush between timed steps (outside the events)
+        torch.cuda.synchronize()
+    hsa.check(ws)
+    if dist is not None:
+        dist.barrier()
+    step_ms = [stage_ev[i][0].elapsed_time(stage_ev[i][4]) for i in range(args.steps)]
+    attn_ms = [stage_ev[i][3].elapsed_time(stage_ev[i][4]) for i in range(args.steps)]
+    sel_ms = [stage_ev[i][1].elapsed_time(stage_ev[i][2]) for i in range(args.steps)]
+    total_s = sum(step_ms) / 1e3
+    units, tmax = aggregate(dist, flops["total"] * args.steps / 1e12, total_s, dev)
+    value = units / tmax
+    clocks = clk.summary()
+
+    attn_s = statistics.mean(attn_ms) / 1e3
+    attn_tf = flops["attention_kernel"] / attn_s / 1e12
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    attn_files = ["hierarchical_chunk_sparse_landmark_b200/csrc/attend_simt.cu"]
+    roofline = {"kernel": "attend_simt_kernel", "bound": "tensor", "achieved": round(attn_tf, 3),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 5),
+                "traffic": measured_traffic("attend", attn_files),
+                "peak_source": peaks["source"] + " bf16 burst",
+                "algorithmic_flops_per_launch": flops["attention_kernel"],
+                "ms_per_launch": round(attn_s * 1e3, 4)}
+
+    res = {
+        "metric": "HSA prefill TFLOP/s (train-shape workload) + 32M-ctx decode tokens/s",
+        "value": round(value, 4), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(tmax * 1e3 / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded N(0,1), per-rank seed)",
+        "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "Hkv": wl.Hkv,
+                   "d": wl.d, "S": wl.S, "topk": wl.topk, "own_chunk": wl.own_chunk,
+                   "landmarks": wl.landmarks, "parallelism": f"independent batches x{world}",
+                   "l2": "flushed between timed steps (256 MiB write)"},
+        "stage_ms": {"selection": round(statistics.mean(sel_ms), 4),
+                     "attention": round(statistics.mean(attn_ms), 4)},
+        "flops_per_step": flops,
+        "roofline": roofline, "clocks": clocks, "gpu_launches": launches,
+    }
+
+    if args.e2e:
+        res["e2e"] = e2e_prefill(args, wl, x, ws, dev, dist)
+    del x, out
+    torch.cuda.empty_cache()
+    if args.decode:
+        res["decode_32m"] = bench_decode(args, dev, peaks, rank, dist)
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(args, wl)
+    return res
+
+
+def e2e_prefill(args, wl, x, ws, dev, dist):
+    """Same metric through the public API with host buffers: pinned host ->
+    device copies of Q/K/V/landmarks, the call, and the device -> host copy of O,
+    all inside the timed region (CUDA events on the stream)."""
+    import torch
+
+    import hierarchical_chunk_sparse_landmark_b200 as hsa
+    hQ, hK, hV = (x[k].cpu().pin_memory() for k in ("Q", "K", "V"))
+    hlm = x["lm"].cpu().pin_memory() if x["lm"] is not None else None
+    dQ, dK, dV = torch.empty_like(x["Q"]), torch.empty_like(x["K"]), torch.empty_like(x["V"])
+    dlm = torch.empty_like(x["lm"]) if hlm is not None else None
+    hO = torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory()
+    dO = torch.empty_like(x["Q"])
+    steps = max(3, args.steps // 4)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+
+    def one():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        if dlm is not None:
+            dlm.copy_(hlm, non_blocking=True)
+        hsa.prefill(dQ, dK, dV, dlm, S=wl.S, topk=wl.topk, own_chunk=wl.own_chunk, out=dO, ws=ws)
+        hO.copy_(dO, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record()
+        one()
+        b.record()
+    torch.cuda.synchronize()
+    secs = sum(a.elapsed_time(b) for a, b in ev) / 1e3
+    flops = prefill_flops(wl)["total"]
+    units, tmax = aggregate(dist, flops * steps / 1e12, secs, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV) + ((hlm,) if hlm is not None else ()))
+    return {"value": round(units / tmax, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": hO.numel() * hO.element_size(), "steps": steps,
+            "ms_per_step": round(tmax * 1e3 / steps, 4)}
+
+
+def bench_decode(args, dev, peaks, rank, dist):
+    import torch
+
+    import hierarchical_chunk_sparse_landmark_b200 as hsa
+    from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_decode_inputs
+    wl = WORKLOADS["decode_32m_bf16"].with_(seed=rank)
+    x = make_decode_inputs(wl, dev)
+    out = torch.empty_like(x["q"])
+    ws = hsa.workspace(hsa.decode_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S, wl.topk),
+                       dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    steps = max(5, args.steps)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for _ in range(3):
+        hsa.decode(x["q"], x["K"], x["V"], x["lm"], topk=wl.topk, out=out, ws=ws)
+        flush.fill_(1)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        hsa.set_stage_events(ev[i])
+        hsa.decode(x["q"], x["K"], x["V"], x["lm"], topk=wl.topk, out=out, ws=ws)
+        hsa.set_stage_events([])
+        flush.fill_(1)
+    torch.cuda.synchronize()
+    hsa.check(ws)
+    secs = sum(a.elapsed_time(b) for a, b in ev) / 1e3
+    nbytes = decode_bytes(wl)
+    toks, tmax = aggregate(dist, float(wl.B * steps), secs, dev)
+    per = secs / steps
+    gbs = nbytes / per / 1e9
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    del x
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "value": round(toks / tmax, 2), "unit": "tokens/s",
+            "ms_per_step": round(per * 1e3, 4), "steps": steps,
+            "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                         "traffic": None, "algorithmic_bytes_per_launch": nbytes,
+                         "peak_source": peaks["source"] + " copy bandwidth"},
+            "l2": "flushed between timed steps"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample_rows(wl, n_rows, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(wl.B * wl.L, size=min(n_rows, wl.B * wl.L), replace=False))
+
+
+def sample_flops(wl, rows) -> float:
+    t = rows % wl.L
+    nvis = t // wl.S
+    keff = np.minimum(wl.topk, nvis)
+    own = (t - wl.S * nvis + 1) if wl.own_chunk else np.zeros_like(t)
+    d, H, Hkv, S = wl.d, wl.H, wl.Hkv, wl.S
+    return float((Hkv * 2 * d * nvis + H * 2 * d * keff + H * 4 * d * S * keff
+                  + H * 4 * d * own).sum())
+
+
+def cpu_baseline(args, wl, budget_s: float = 12.0, x_host=None):
+    """Time the fp64 oracle, as it stands, on the host cores over a bounded
+    sample of rows of the same workload; throughput in the same unit."""
+    import torch
+
+    import oracle
+    from hierarchical_chunk_sparse_landmark_b200.workloads import make_prefill_inputs
+    orc = oracle.Oracle()
+    x = x_host if x_host is not None else make_prefill_inputs(wl, "cpu")
+    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
+    K, V, lm = f64(x["K"]), f64(x["V"]), f64(x["lm"])
+    Qall = x["Q"].reshape(wl.B * wl.L, wl.H, wl.d)
+    n = 256
+    total_f, total_s, total_rows = 0.0, 0.0, 0
+    while total_s < budget_s and total_rows < wl.B * wl.L:
+        rows = oracle_sample_rows(wl, n, seed=total_rows)
+        Qr = f64(Qall[torch.as_tensor(rows)])
+        t0 = time.perf_counter()
+        orc.prefill(None, K, V, lm, wl.S, wl.topk, wl.own_chunk, rows=rows, Q_rows=Qr)
+        dt = time.perf_counter() - t0
+        total_f += sample_flops(wl, rows)
+        total_s += dt
+        total_rows += len(rows)
+        n = min(4 * n, 8192)
+    return {"value": round(total_f / total_s / 1e12, 6), "unit": "TFLOP/s",
+            "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{total_rows} random rows (all heads) of {wl.name}, fp64 C/OpenMP oracle",
+            "seconds": round(total_s, 2)}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on host cores (rank 0 only)."""
+    from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_prefill_inputs
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    x = make_prefill_inputs(wl, "cpu")
+    per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(args, wl, budget_s=per_step_budget / 4, x_host=x)
+    vals, secs = [], 0.0
+    info = None
+    for _ in range(args.steps):
+        info = cpu_baseline(args, wl, budget_s=per_step_budget, x_host=x)
+        vals.append(info["value"])
+        secs += info["seconds"]
+    value = statistics.mean(vals)
+    return {"impl": "reference", "metric": "HSA prefill TFLOP/s (train-shape workload) "
+            "+ 32M-ctx decode tokens/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "Hkv": wl.Hkv,
+                       "d": wl.d, "S": wl.S, "topk": wl.topk},
+            "cpu_baseline": {"kind": "oracle", "cores": info["cores"], "sample": info["sample"],
+                             "value": value, "unit": "TFLOP/s"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="train_prefill_bf16")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", dest="decode", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as td
+        torch.cuda.set_device(local)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    else:
+        torch.cuda.set_device(0)
+    res = run_ours(args, dist, rank, world)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,13 @@
+"""Hierarchical chunk-sparse landmark attention (HSA / HiLS / DHSA forward pass)
+for NVIDIA B200 (sm_100a).
+
+The computation runs in hand-written CUDA kernels behind a C ABI
+(``include/hsa.h``, built into ``libhsa.so``); this package is the Python
+binding (PyTorch supplies device memory and streams) plus the seeded synthetic
+workloads used by the tests and the benchmark.
+"""
+from ._binding import (HSAError, check, last_call_launches, decode, decode_workspace_size, landmarks, lib, prefill,
+                       prefill_workspace_size, set_stage_events, status_string, workspace)
+
+__all__ = ["HSAError", "check", "last_call_launches", "decode", "decode_workspace_size", "landmarks", "lib", "prefill",
+           "prefill_workspace_size", "set_stage_events", "status_string", "workspace"]

@@ -1,0 +1,218 @@
+"""ctypes binding of libhsa.so (the C ABI declared in include/hsa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  PyTorch supplies device memory and the current
+stream.  If the shared library is missing the import of the ops fails with a
+clear error; there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhsa.so")
+
+HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED = 0, 1, 2
+HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT = 3, 4, 5
+HSA_F32, HSA_BF16 = 0, 1
+
+EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
+            "hsa_decode_workspace_size", "hsa_decode", "hsa_check", "hsa_status_string",
+            "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches")
+
+
+class HSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def _declare(lib):
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    lib.hsa_landmarks.argtypes = [vp, i32, vp, i32, i32, i64, i32, i32, vp]
+    lib.hsa_prefill_workspace_size.argtypes = [i32, i32, i32, i64, i32, i32, i32]
+    lib.hsa_prefill_workspace_size.restype = sz
+    lib.hsa_prefill.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, i32,
+                                f32, vp, vp, vp, vp, sz, vp]
+    lib.hsa_decode_workspace_size.argtypes = [i32, i32, i32, i64, i32, i32, i32]
+    lib.hsa_decode_workspace_size.restype = sz
+    lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
+                               vp, vp, vp, sz, vp]
+    lib.hsa_check.argtypes = [vp, vp]
+    lib.hsa_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
+    lib.hsa_status_string.argtypes = [i32]
+    lib.hsa_status_string.restype = ctypes.c_char_p
+    for n in ("hsa_landmarks", "hsa_prefill", "hsa_decode", "hsa_check", "hsa_version",
+              "hsa_set_stage_events", "hsa_last_call_launches"):
+        getattr(lib, n).restype = i32
+    return lib
+
+
+def lib():
+    """The loaded libhsa (raises if the CUDA library was not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise ImportError(
+                        f"libhsa.so not found at {LIB_PATH}; build it with "
+                        "`python -m hierarchical_chunk_sparse_landmark_b200.build`")
+                _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().hsa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != HSA_OK:
+        raise HSAError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return HSA_F32
+    if t.dtype == torch.bfloat16:
+        return HSA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _opt(t):
+    """A tensor argument or None (flags such as ``idx_out=False`` mean "not wanted")."""
+    return t if isinstance(t, torch.Tensor) else None
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+# Workspaces are cached per (device, stream): calls on one stream are ordered,
+# so reusing the buffer there is safe.
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    device = torch.device(device)
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def landmarks(K: torch.Tensor, S: int = 64, out: torch.Tensor | None = None) -> torch.Tensor:
+    """DHSA landmarks sqrt(S) * mean of each complete chunk's keys, fp32 [B,Hkv,L//S,d]."""
+    _dev(K, "K")
+    B, Hkv, L, d = K.shape
+    if out is None:
+        out = torch.empty(B, Hkv, L // S, d, dtype=torch.float32, device=K.device)
+    _check(lib().hsa_landmarks(_ptr(K), _dtype_code(K), _ptr(out), B, Hkv, L, d, S,
+                               _stream(K.device)), "hsa_landmarks")
+    return out
+
+
+def prefill_workspace_size(B, H, Hkv, L, d, S, topk) -> int:
+    return int(lib().hsa_prefill_workspace_size(B, H, Hkv, L, d, S, topk))
+
+
+def prefill(Q, K, V, lm=None, *, S: int = 64, topk: int = 8, own_chunk: int = 1,
+            scale: float = 0.0, out=None, idx_out=None, w_out=None, ws=None):
+    """Hierarchical chunk-sparse prefill.  Returns (O, idx, w); idx/w are None
+    unless buffers are given or ``idx_out=True`` / ``w_out=True``."""
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _dev(t, n)
+    B, L, H, d = Q.shape
+    Hkv = K.shape[1]
+    if K.shape != (B, Hkv, L, d) or V.shape != K.shape:
+        raise ValueError("K and V must be [B, Hkv, L, d] matching Q [B, L, H, d]")
+    if lm is not None:
+        _dev(lm, "lm")
+        if lm.shape != (B, Hkv, L // S, d):
+            raise ValueError(f"lm must be [B, Hkv, L//S, d] = {(B, Hkv, L // S, d)}")
+    dev = Q.device
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx_out is True:
+        idx_out = torch.empty(B, L, Hkv, topk, dtype=torch.int32, device=dev)
+    if w_out is True:
+        w_out = torch.empty(B, L, H, topk, dtype=torch.float32, device=dev)
+    nbytes = prefill_workspace_size(B, H, Hkv, L, d, S, topk)
+    if ws is None:
+        ws = workspace(nbytes, dev)
+    st = lib().hsa_prefill(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(lm),
+                           _dtype_code(lm) if lm is not None else HSA_F32, B, H, Hkv, L, d, S,
+                           topk, int(own_chunk), float(scale), _ptr(out),
+                           _ptr(_opt(idx_out)), _ptr(_opt(w_out)), _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(dev))
+    _check(st, "hsa_prefill")
+    return out, _opt(idx_out), _opt(w_out)
+
+
+def decode_workspace_size(B, H, Hkv, Lc, d, S, topk) -> int:
+    return int(lib().hsa_decode_workspace_size(B, H, Hkv, Lc, d, S, topk))
+
+
+def decode(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.0, out=None,
+           idx_out=None, ws=None):
+    """One query per sequence at position Lc against a Lc-token cache.  Returns (O, idx)."""
+    for n, t in (("q", q), ("K", K), ("V", V), ("lm", lm)):
+        _dev(t, n)
+    B, H, d = q.shape
+    _, Hkv, Lc, _ = K.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is True:
+        idx_out = torch.empty(B, Hkv, topk, dtype=torch.int32, device=dev)
+    nbytes = decode_workspace_size(B, H, Hkv, Lc, d, S, topk)
+    if ws is None:
+        ws = workspace(nbytes, dev)
+    st = lib().hsa_decode(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm), _dtype_code(lm),
+                          B, H, Hkv, Lc, d, S, topk, float(scale), _ptr(out),
+                          _ptr(_opt(idx_out)), _ptr(ws), ws.numel() * ws.element_size(),
+                          _stream(dev))
+    _check(st, "hsa_decode")
+    return out, _opt(idx_out)
+
+
+def set_stage_events(events) -> None:
+    """Timing hook: record these torch.cuda.Event objects at the stage
+    boundaries of this thread's next calls (see hsa_set_stage_events); pass
+    an empty list to stop."""
+    arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event)
+                                                    for e in events])
+    _check(lib().hsa_set_stage_events(arr, len(events)), "hsa_set_stage_events")
+
+
+def last_call_launches() -> int:
+    """Kernels launched by this thread's most recent library call."""
+    return int(lib().hsa_last_call_launches())
+
+
+def check(ws=None, device=None):
+    """Synchronise the current stream and report device-side status flags."""
+    device = device if device is not None else (ws.device if ws is not None else "cuda")
+    _check(lib().hsa_check(_ptr(ws), _stream(device)), "hsa_check")

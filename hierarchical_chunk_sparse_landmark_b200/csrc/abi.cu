@@ -1,0 +1,261 @@
+// abi.cu -- the extern "C" entry points of libhsa (declared in include/hsa.h):
+// argument validation, workspace layout and kernel dispatch.
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "hsa.h"
+
+namespace hsa {
+cudaError_t launch_landmarks(const void *K, bool bf16, float *lm, int B, int Hkv, int64_t L,
+                             int d, cudaStream_t st);
+cudaError_t launch_select(const void *Q, bool q_bf16, const void *lm, bool lm_bf16, int B, int H,
+                          int Hkv, int64_t L, int d, int S, int topk, float scale, int32_t *idx,
+                          float *w, cudaStream_t st);
+cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool bf16,
+                               const int32_t *idx, const float *w, int B, int H, int Hkv,
+                               int64_t L, int d, int S, int topk, int own_chunk, float scale,
+                               void *O, cudaStream_t st);
+cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
+                          const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
+                          int S, int topk, float scale, int splits, uint64_t *cand,
+                          unsigned *tickets, void *O, int32_t *idx_out, cudaStream_t st);
+int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
+}  // namespace hsa
+
+using namespace hsa;
+
+namespace {
+
+constexpr int kChunk = 64;
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool dtype_ok(hsa_dtype_t t) { return t == HSA_F32 || t == HSA_BF16; }
+
+// Shape checks shared by every call.  INVALID_ARG for impossible requests,
+// UNSUPPORTED for valid ones this build does not implement.
+hsa_status_t check_shape(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
+    if (B < 1 || H < 1 || Hkv < 1 || L < 0 || d < 1 || S < 1 || topk < 1)
+        return HSA_ERR_INVALID_ARG;
+    if (H % Hkv != 0) return HSA_ERR_INVALID_ARG;
+    const int G = H / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return HSA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return HSA_ERR_UNSUPPORTED;
+    if (S != kChunk) return HSA_ERR_UNSUPPORTED;
+    if (topk > 32) return HSA_ERR_UNSUPPORTED;
+    if (L > (int64_t)INT32_MAX) return HSA_ERR_UNSUPPORTED;   // chunk indices are int32
+    return HSA_OK;
+}
+
+int num_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return sms;
+}
+
+struct PrefillLayout {
+    size_t idx_off, w_off, lm_off, total;
+};
+
+PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
+    PrefillLayout p;
+    size_t off = kStatusBytes;
+    p.idx_off = off;
+    off = align_up(off + sizeof(int32_t) * (size_t)B * L * Hkv * topk, 256);
+    p.w_off = off;
+    off = align_up(off + sizeof(float) * (size_t)B * L * H * topk, 256);
+    p.lm_off = off;
+    off = align_up(off + sizeof(float) * (size_t)B * Hkv * (L / S) * d, 256);
+    p.total = off;
+    return p;
+}
+
+struct DecodeLayout {
+    size_t tickets_off, cand_off, total;
+    int splits;
+};
+
+DecodeLayout decode_layout(int B, int Hkv, int64_t Lc, int S, int topk) {
+    DecodeLayout p;
+    const int64_t Nc = Lc / S;
+    p.splits = decode_splits(B, Hkv, Nc, num_sms());
+    size_t off = kStatusBytes;
+    p.tickets_off = off;
+    off = align_up(off + sizeof(unsigned) * (size_t)B * Hkv, 256);
+    p.cand_off = off;
+    off = align_up(off + sizeof(uint64_t) * (size_t)B * Hkv * p.splits * topk, 256);
+    p.total = off;
+    return p;
+}
+
+hsa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? HSA_OK : HSA_ERR_CUDA; }
+
+// Per-thread timing hook (hsa_set_stage_events).
+constexpr int kMaxStageEvents = 8;
+thread_local cudaEvent_t t_stage_events[kMaxStageEvents];
+thread_local int t_n_stage_events = 0;
+thread_local int t_launches = 0;      // kernels launched by this thread's last call
+
+inline void stage_mark(int i, cudaStream_t st) {
+    if (i < t_n_stage_events && t_stage_events[i]) cudaEventRecord(t_stage_events[i], st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hsa_version(void) { return 100; }
+
+int hsa_last_call_launches(void) { return t_launches; }
+
+hsa_status_t hsa_set_stage_events(void *const *events, int n) {
+    if (n < 0 || n > kMaxStageEvents || (n > 0 && !events)) return HSA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) t_stage_events[i] = (cudaEvent_t)events[i];
+    t_n_stage_events = n;
+    return HSA_OK;
+}
+
+const char *hsa_status_string(hsa_status_t s) {
+    switch (s) {
+    case HSA_OK: return "ok";
+    case HSA_ERR_INVALID_ARG: return "invalid argument";
+    case HSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case HSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case HSA_ERR_CUDA: return "CUDA error";
+    case HSA_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+hsa_status_t hsa_landmarks(const void *K, hsa_dtype_t k_dt, float *lm_out, int B, int Hkv,
+                           int64_t L, int d, int S, void *stream) {
+    hsa_status_t s = check_shape(B, Hkv, Hkv, L, d, S, 1);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(k_dt)) return HSA_ERR_UNSUPPORTED;
+    t_launches = 0;
+    if (L / S == 0) return HSA_OK;
+    if (!K || !lm_out || !aligned16(K) || !aligned16(lm_out)) return HSA_ERR_INVALID_ARG;
+    t_launches = 1;
+    return from_cuda(launch_landmarks(K, k_dt == HSA_BF16, lm_out, B, Hkv, L, d,
+                                      (cudaStream_t)stream));
+}
+
+size_t hsa_prefill_workspace_size(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
+    if (check_shape(B, H, Hkv, L, d, S, topk) != HSA_OK) return 0;
+    return prefill_layout(B, H, Hkv, L, d, S, topk).total;
+}
+
+hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                         const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t L,
+                         int d, int S, int topk, int own_chunk, float scale, void *O,
+                         int32_t *idx_out, float *w_out, void *workspace, size_t ws_bytes,
+                         void *stream) {
+    hsa_status_t s = check_shape(B, H, Hkv, L, d, S, topk);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
+    if (own_chunk != 0 && own_chunk != 1) return HSA_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    if (L == 0) return HSA_OK;
+    const void *ptrs[] = {Q, K, V, O, workspace};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    if ((lm && !aligned16(lm)) || (idx_out && !aligned16(idx_out)) || (w_out && !aligned16(w_out)))
+        return HSA_ERR_INVALID_ARG;
+    const PrefillLayout lay = prefill_layout(B, H, Hkv, L, d, S, topk);
+    if (ws_bytes < lay.total) return HSA_ERR_WORKSPACE;
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+
+    cudaStream_t st = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    int32_t *idx = idx_out ? idx_out : (int32_t *)(ws + lay.idx_off);
+    float *w = w_out ? w_out : (float *)(ws + lay.w_off);
+    const bool bf16 = dt == HSA_BF16;
+    const void *lm_use = lm;
+    bool lm_bf16 = lm_dt == HSA_BF16;
+    stage_mark(0, st);
+    if (!lm) {
+        float *lm_ws = (float *)(ws + lay.lm_off);
+        cudaError_t e = launch_landmarks(K, bf16, lm_ws, B, Hkv, L, d, st);
+        if (e != cudaSuccess) return HSA_ERR_CUDA;
+        t_launches += L / S > 0 ? 1 : 0;
+        lm_use = lm_ws;
+        lm_bf16 = false;
+    }
+    stage_mark(1, st);
+    cudaError_t e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
+                                  w, st);
+    if (e != cudaSuccess) return HSA_ERR_CUDA;
+    t_launches += 1;
+    stage_mark(2, st);
+    stage_mark(3, st);
+    e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale, O,
+                           st);
+    t_launches += e == cudaSuccess ? 1 : 0;
+    stage_mark(4, st);
+    return from_cuda(e);
+}
+
+size_t hsa_decode_workspace_size(int B, int H, int Hkv, int64_t Lc, int d, int S, int topk) {
+    if (check_shape(B, H, Hkv, Lc, d, S, topk) != HSA_OK) return 0;
+    if (Lc % S != 0) return 0;
+    return decode_layout(B, Hkv, Lc, S, topk).total;
+}
+
+hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                        const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t Lc,
+                        int d, int S, int topk, float scale, void *O, int32_t *idx_out,
+                        void *workspace, size_t ws_bytes, void *stream) {
+    hsa_status_t s = check_shape(B, H, Hkv, Lc, d, S, topk);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
+    if (Lc % S != 0) return HSA_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    if (!q || !O || !workspace || !aligned16(q) || !aligned16(O) || !aligned16(workspace))
+        return HSA_ERR_INVALID_ARG;
+    if (idx_out && !aligned16(idx_out)) return HSA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (Lc == 0) {   // nothing visible: O = 0, no selection
+        const size_t el = dt == HSA_BF16 ? 2 : 4;
+        if (cudaMemsetAsync(O, 0, el * (size_t)B * H * d, st) != cudaSuccess) return HSA_ERR_CUDA;
+        if (idx_out && cudaMemsetAsync(idx_out, 0xff, sizeof(int32_t) * (size_t)B * Hkv * topk,
+                                       st) != cudaSuccess)
+            return HSA_ERR_CUDA;
+        return HSA_OK;
+    }
+    const void *ptrs[] = {Kc, Vc, lm};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    const DecodeLayout lay = decode_layout(B, Hkv, Lc, S, topk);
+    if (ws_bytes < lay.total) return HSA_ERR_WORKSPACE;
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    char *ws = (char *)workspace;
+    stage_mark(0, st);
+    hsa_status_t r = from_cuda(launch_decode(q, Kc, Vc, dt == HSA_BF16, lm, lm_dt == HSA_BF16, B, H, Hkv,
+                                   Lc, d, S, topk, scale, lay.splits,
+                                   (uint64_t *)(ws + lay.cand_off),
+                                   (unsigned *)(ws + lay.tickets_off), O, idx_out, st));
+    t_launches = r == HSA_OK ? 1 : 0;
+    stage_mark(1, st);
+    return r;
+}
+
+hsa_status_t hsa_check(void *workspace, void *stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return HSA_ERR_CUDA;
+    if (!workspace) return HSA_OK;
+    unsigned flags = 0;
+    if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return HSA_ERR_CUDA;
+    if (flags & kFlagTimeout) {
+        const unsigned zero = 0;
+        cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        return HSA_ERR_TIMEOUT;
+    }
+    return HSA_OK;
+}
+
+}  // extern "C"

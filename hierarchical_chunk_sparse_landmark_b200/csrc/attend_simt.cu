@@ -1,0 +1,153 @@
+// attend_simt.cu -- in-chunk attention + score-weighted fusion on CUDA cores.
+//
+// O[t,h] = sum_k w[t,h,k] * softmax_j(scale q.k_j) V over chunk sel_k
+//          + (own_chunk ? causal softmax attention over keys c_t*S .. t : 0)
+// (HiLS Attention abstract: attention inside each retrieved chunk, outputs
+// fused by retrieval scores.)
+//
+// Query-centric: one block per (b, t, g), one warp per query head of the
+// group.  For every selected chunk the block stages the chunk's K and V rows
+// in shared memory; each warp computes its head's 64 logits (lane j: keys j
+// and j+32), the chunk softmax with warp shuffles, and P.V with lanes over
+// the head dimension, accumulating w_k * o_k in registers.  This is the fp32
+// path (fp32 accumulate end to end) and the reference layout for the
+// tensor-core path.
+#include "common.cuh"
+
+namespace hsa {
+
+template <typename T, int D>
+__global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K,
+                                   const T *__restrict__ V, const int32_t *__restrict__ idx,
+                                   const float *__restrict__ w, int H, int Hkv, int64_t L, int S,
+                                   int topk, int own_chunk, float scale, T *__restrict__ O) {
+    constexpr int VEC = Vec16<T>::N;
+    constexpr int PAD = VEC;                     // 16 bytes of padding per row
+    constexpr int RS = D + PAD;                  // row stride (elements)
+    constexpr int MAXS = 64;
+    extern __shared__ float4 smem4[];
+    float *qs = reinterpret_cast<float *>(smem4);                 // [G][D]
+    const int G = H / Hkv;
+    T *ks = reinterpret_cast<T *>(qs + G * D);                    // [S][RS]
+    T *vs = ks + MAXS * RS;                                       // [S][RS]
+
+    const int64_t t = blockIdx.x;
+    const int g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nthr = blockDim.x;
+    const int64_t row = (int64_t)b * L + t;
+
+    for (int e = threadIdx.x; e < G * D; e += nthr)
+        qs[e] = to_f32(Q[(row * H + (int64_t)g * G) * D + e]);
+
+    constexpr int R = D / 32;                    // output elements per lane
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
+
+    const int64_t c_t = t / S;
+    const T *Kbg = K + ((int64_t)b * Hkv + g) * L * D;
+    const T *Vbg = V + ((int64_t)b * Hkv + g) * L * D;
+    const int32_t *ip = idx + (row * Hkv + g) * topk;
+    const int h = g * G + warp;
+    const int n_items = topk + (own_chunk ? 1 : 0);
+    for (int it = 0; it < n_items; ++it) {
+        int64_t first;
+        int nkeys;
+        float wt;
+        if (it < topk) {
+            const int32_t ci = ip[it];
+            if (ci < 0) continue;                    // uniform across the block
+            first = (int64_t)ci * S;
+            nkeys = S;
+            wt = w[(row * H + h) * topk + it];
+        } else {
+            first = c_t * S;
+            nkeys = (int)(t - first + 1);
+            wt = 1.f;
+        }
+        __syncthreads();
+        const int vec_per_row = D / VEC;
+        for (int e = threadIdx.x; e < nkeys * vec_per_row; e += nthr) {
+            const int r = e / vec_per_row, c = (e % vec_per_row) * VEC;
+            *reinterpret_cast<uint4 *>(ks + r * RS + c) =
+                *reinterpret_cast<const uint4 *>(Kbg + (first + r) * D + c);
+            *reinterpret_cast<uint4 *>(vs + r * RS + c) =
+                *reinterpret_cast<const uint4 *>(Vbg + (first + r) * D + c);
+        }
+        __syncthreads();
+        // logits for keys lane and lane+32
+        const float *qh = qs + warp * D;
+        float lg[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = lane + 32 * u;
+            lg[u] = -INFINITY;
+            if (j < nkeys) {
+                float a = 0.f;
+#pragma unroll 4
+                for (int c = 0; c < D; c += VEC) {
+                    float f[VEC];
+                    Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(ks + j * RS + c), f);
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) a = fmaf(qh[c + e], f[e], a);
+                }
+                lg[u] = scale * a;
+            }
+        }
+        float mx = fmaxf(lg[0], lg[1]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float p[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) p[u] = (lane + 32 * u < nkeys) ? expf(lg[u] - mx) : 0.f;
+        float den = p[0] + p[1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        float o_r[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) o_r[r] = 0.f;
+        for (int j = 0; j < nkeys; ++j) {
+            const float pj = __shfl_sync(0xffffffffu, p[j >> 5], j & 31);
+#pragma unroll
+            for (int r = 0; r < R; ++r) o_r[r] = fmaf(pj, to_f32(vs[j * RS + lane + 32 * r]), o_r[r]);
+        }
+        const float f = wt / den;
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] = fmaf(f, o_r[r], acc[r]);
+    }
+    T *op = O + (row * H + h) * (int64_t)D;
+#pragma unroll
+    for (int r = 0; r < R; ++r) op[lane + 32 * r] = from_f32<T>(acc[r]);
+}
+
+template <typename T, int D>
+static cudaError_t launch_attend_simt_t(const void *Q, const void *K, const void *V,
+                                        const int32_t *idx, const float *w, int B, int H,
+                                        int Hkv, int64_t L, int S, int topk, int own_chunk,
+                                        float scale, void *O, cudaStream_t st) {
+    constexpr int VEC = Vec16<T>::N;
+    const int G = H / Hkv;
+    const size_t smem = sizeof(float) * G * D + 2 * sizeof(T) * 64 * (D + VEC);
+    auto kern = attend_simt_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)L, (unsigned)Hkv, (unsigned)B);
+    kern<<<grid, 32 * G, smem, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, w, H, Hkv,
+                                     L, S, topk, own_chunk, scale, (T *)O);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool bf16,
+                               const int32_t *idx, const float *w, int B, int H, int Hkv,
+                               int64_t L, int d, int S, int topk, int own_chunk, float scale,
+                               void *O, cudaStream_t st) {
+    if (bf16)
+        return d == 128 ? launch_attend_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st)
+                        : launch_attend_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st);
+    return d == 128 ? launch_attend_simt_t<float, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st)
+                    : launch_attend_simt_t<float, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st);
+}
+
+}  // namespace hsa

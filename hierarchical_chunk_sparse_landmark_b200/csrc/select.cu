@@ -1,0 +1,195 @@
+// select.cu -- prefill chunk selection and fusion weights.
+//
+// For each (b, t, g): group query qbar = mean of the G heads' queries, group
+// scores sbar_i = scale * qbar . l_i over the visible chunks i < floor(t/S),
+// the top-K chunks by (score desc, index asc), then per head the fusion
+// weights w = softmax over the selected chunks of scale * q_h . l_i.
+// (Per-token top-K retrieval over chunk landmarks: Understanding and Improving
+// Length Generalization in Hierarchical Sparse Attention Models, "Methodology
+// in Plain English"; fusion by retrieval scores: HiLS Attention abstract.)
+//
+// One block owns 64 consecutive tokens of one (b, g).  Their qbar rows stay
+// in shared memory while the landmark rows of the visible chunks stream
+// through shared memory 32 at a time.  Each thread scores one token against 8
+// chunks of a tile (fp32 FMA, float4 operands) into a shared score tile; then
+// each warp folds the tile into the sorted top-K lists of its 8 tokens, kept
+// warp-distributed (lane k holds a token's k-th best 64-bit key).  Only lanes
+// whose key beats the current K-th best take part in an insertion.
+#include "common.cuh"
+
+namespace hsa {
+
+constexpr int kSelTokens = 64;   // tokens per block
+constexpr int kSelChunks = 32;   // landmark rows per shared-memory tile
+constexpr int kSelThreads = 256; // 8 warps, 8 tokens per warp
+constexpr int kSelTokPerWarp = kSelTokens / (kSelThreads / 32);
+
+// Insert x into a warp-distributed sorted list (lane k < topk holds entry k).
+// Executed by the whole warp with the same x; returns this lane's new entry.
+__device__ __forceinline__ uint64_t list_insert(uint64_t v, uint64_t x, int topk, int lane) {
+    const unsigned better = __ballot_sync(0xffffffffu, lane < topk && v > x);
+    const int pos = __popc(better);
+    const uint64_t up = __shfl_up_sync(0xffffffffu, v, 1);
+    if (lane < topk) {
+        if (lane == pos) v = x;
+        else if (lane > pos) v = up;
+    }
+    return v;
+}
+
+template <typename T, typename TL, int D>
+__global__ void __launch_bounds__(kSelThreads)
+select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv, int64_t L,
+              int S, int topk, float scale, int32_t *__restrict__ idx_out,
+              float *__restrict__ w_out) {
+    extern __shared__ float4 smem4[];
+    float *qbar = reinterpret_cast<float *>(smem4);                 // [64][D+4]
+    float *lmt = qbar + kSelTokens * (D + 4);                        // [32][D+4]
+    float *sc = lmt + kSelChunks * (D + 4);                          // [64][33]
+
+    const int n_tiles = (int)((L + kSelTokens - 1) / kSelTokens);
+    const int tile = n_tiles - 1 - (int)blockIdx.x;                 // heavy tiles first
+    const int g = blockIdx.y, b = blockIdx.z;
+    const int G = H / Hkv;
+    const int64_t Nc = L / S;
+    const int64_t t0 = (int64_t)tile * kSelTokens;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // qbar for the block's tokens (rows past L are zero).
+    for (int e = tid; e < kSelTokens * D; e += kSelThreads) {
+        const int r = e / D, j = e % D;
+        const int64_t t = t0 + r;
+        float acc = 0.f;
+        if (t < L) {
+            const T *qp = Q + ((b * L + t) * H + (int64_t)g * G) * D + j;
+            for (int h = 0; h < G; ++h) acc += to_f32(qp[(int64_t)h * D]);
+            acc = acc / (float)G;
+        }
+        qbar[r * (D + 4) + j] = acc;
+    }
+    const int64_t t_last = (t0 + kSelTokens - 1 < L ? t0 + kSelTokens - 1 : L - 1);
+    const int64_t nvis_max = t_last / S;
+
+    // scoring role: token tok_s, chunks sub + 4m of each tile
+    const int tok_s = tid >> 2, sub = tid & 3;
+    // list role: this warp's tokens
+    uint64_t v[kSelTokPerWarp], thr[kSelTokPerWarp];
+#pragma unroll
+    for (int u = 0; u < kSelTokPerWarp; ++u) { v[u] = 0ull; thr[u] = 0ull; }
+
+    const TL *lm_bg = lm + ((int64_t)b * Hkv + g) * Nc * D;
+    for (int64_t c0 = 0; c0 < nvis_max; c0 += kSelChunks) {
+        __syncthreads();
+        for (int e = tid; e < kSelChunks * D; e += kSelThreads) {
+            const int r = e / D, j = e % D;
+            const int64_t i = c0 + r;
+            lmt[r * (D + 4) + j] = i < nvis_max ? to_f32(lm_bg[i * D + j]) : 0.f;
+        }
+        __syncthreads();
+        {
+            float acc[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[m] = 0.f;
+            const float4 *qv = reinterpret_cast<const float4 *>(qbar + tok_s * (D + 4));
+#pragma unroll 4
+            for (int j4 = 0; j4 < D / 4; ++j4) {
+                const float4 a = qv[j4];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const float4 l =
+                        reinterpret_cast<const float4 *>(lmt + (sub + 4 * m) * (D + 4))[j4];
+                    acc[m] = fmaf(a.x, l.x, acc[m]);
+                    acc[m] = fmaf(a.y, l.y, acc[m]);
+                    acc[m] = fmaf(a.z, l.z, acc[m]);
+                    acc[m] = fmaf(a.w, l.w, acc[m]);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) sc[tok_s * 33 + sub + 4 * m] = scale * acc[m];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kSelTokPerWarp; ++u) {
+            const int tok = warp * kSelTokPerWarp + u;
+            const int64_t t = t0 + tok;
+            const int64_t nvis = t < L ? t / S : 0;
+            const int64_t i = c0 + lane;
+            const uint64_t key = i < nvis ? make_key(sc[tok * 33 + lane], i) : 0ull;
+            unsigned m = __ballot_sync(0xffffffffu, key > thr[u]);
+            while (m) {
+                const int s = __ffs(m) - 1;
+                m &= m - 1;
+                const uint64_t x = __shfl_sync(0xffffffffu, key, s);
+                if (x > thr[u]) {
+                    v[u] = list_insert(v[u], x, topk, lane);
+                    thr[u] = __shfl_sync(0xffffffffu, v[u], topk - 1);
+                }
+            }
+        }
+    }
+
+    // outputs: idx (lane k = rank k) and per-head fusion weights
+#pragma unroll
+    for (int u = 0; u < kSelTokPerWarp; ++u) {
+        const int64_t t = t0 + warp * kSelTokPerWarp + u;
+        if (t >= L) continue;
+        const int32_t sel = lane < topk ? key_index(v[u]) : -1;
+        if (lane < topk && idx_out) idx_out[((b * L + t) * Hkv + g) * topk + lane] = sel;
+        for (int h = 0; h < G; ++h) {
+            const int hh = g * G + h;
+            const T *qh = Q + ((b * L + t) * H + hh) * (int64_t)D;
+            float s = -INFINITY;
+            if (sel >= 0) {
+                const TL *lp = lm_bg + (int64_t)sel * D;
+                float a = 0.f;
+                for (int j = 0; j < D; ++j) a = fmaf(to_f32(qh[j]), to_f32(lp[j]), a);
+                s = scale * a;
+            }
+            float mx = s;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float e = sel >= 0 ? expf(s - mx) : 0.f;
+            float den = e;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+            if (lane < topk) w_out[((b * L + t) * H + hh) * topk + lane] = den > 0.f ? e / den : 0.f;
+        }
+    }
+}
+
+template <typename T, typename TL, int D>
+static cudaError_t launch_select_t(const void *Q, const void *lm, int B, int H, int Hkv,
+                                   int64_t L, int S, int topk, float scale, int32_t *idx,
+                                   float *w, cudaStream_t st) {
+    const size_t smem =
+        sizeof(float) * ((kSelTokens + kSelChunks) * (D + 4) + kSelTokens * 33);
+    auto kern = select_kernel<T, TL, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((L + kSelTokens - 1) / kSelTokens), (unsigned)Hkv, (unsigned)B);
+    kern<<<grid, kSelThreads, smem, st>>>((const T *)Q, (const TL *)lm, H, Hkv, L, S, topk,
+                                          scale, idx, w);
+    return cudaGetLastError();
+}
+
+template <typename T, typename TL>
+static cudaError_t launch_select_l(const void *Q, const void *lm, int B, int H, int Hkv,
+                                   int64_t L, int d, int S, int topk, float scale, int32_t *idx,
+                                   float *w, cudaStream_t st) {
+    return d == 128 ? launch_select_t<T, TL, 128>(Q, lm, B, H, Hkv, L, S, topk, scale, idx, w, st)
+                    : launch_select_t<T, TL, 64>(Q, lm, B, H, Hkv, L, S, topk, scale, idx, w, st);
+}
+
+cudaError_t launch_select(const void *Q, bool q_bf16, const void *lm, bool lm_bf16, int B, int H,
+                          int Hkv, int64_t L, int d, int S, int topk, float scale, int32_t *idx,
+                          float *w, cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    if (q_bf16)
+        return lm_bf16 ? launch_select_l<bf, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st)
+                       : launch_select_l<bf, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st);
+    return lm_bf16 ? launch_select_l<float, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st)
+                   : launch_select_l<float, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st);
+}
+
+}  // namespace hsa

@@ -1,0 +1,177 @@
+/*
+ * hsa.h -- C ABI of libhsa: hierarchical chunk-sparse landmark attention
+ * (HSA / HiLS / DHSA forward pass) on NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For query token t of head h in KV group g = h / G
+ * (G = H / Hkv query heads share one KV head), with chunk size S,
+ * c_t = floor(t / S) and scale = 1/sqrt(d) unless given:
+ *
+ *   s[t,h,i]  = scale * q[t,h] . l[g,i]                 landmark score of chunk i
+ *   sbar[t,g,i] = mean over the G heads of s[t,h,i]     group score (shared selection)
+ *   sel(t,g)  = the topk chunks i < c_t with the largest sbar; equal scores go
+ *               to the lower chunk index; fewer visible chunks -> all of them
+ *   w[t,h,k]  = softmax over k in sel(t,g) of s[t,h,k]  fusion weights
+ *   o[t,h,i]  = softmax_j(scale * q[t,h] . k[g,j]) v[g,j] over the S keys of chunk i
+ *   O[t,h]    = sum_k w[t,h,k] o[t,h,sel_k]
+ *               + (own_chunk ? causal attention over keys c_t*S .. t : 0)
+ *
+ * Sources: chunk size 64, one landmark per chunk and per-token top-K
+ * retrieval are from "Understanding and Improving Length Generalization in
+ * Hierarchical Sparse Attention Models" (ai.info summary, "Methodology in
+ * Plain English" and "Main Findings"); attention inside each retrieved chunk
+ * with outputs fused by the retrieval scores is the HiLS Attention abstract
+ * (mlsift "length extrapolation" tag page); the DHSA landmark sqrt(|C|) * mean
+ * of a chunk's keys is from the Dynamic Hierarchical Sparse Attention review
+ * (pith.science, "What carries the argument").  Where the pages leave a step
+ * open the library takes the readings stated next to each call.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers, row-major and densely packed in
+ *    the layout given; they must be 16-byte aligned.  The caller owns every
+ *    buffer, the workspace included.  The library allocates no memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work on it; none synchronises except
+ *    hsa_check.
+ *  - Arguments are checked before anything is launched.  A failed check
+ *    returns HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED or HSA_ERR_WORKSPACE and
+ *    launches nothing.  A launch failure returns HSA_ERR_CUDA.
+ *  - Supported shapes: d in {64, 128}; S = 64; 1 <= topk <= 32; H % Hkv == 0
+ *    with G = H / Hkv in {1, 2, 4, 8, 16}; dtypes HSA_F32 or HSA_BF16.
+ *    Accumulation is fp32 throughout; O is written in the input dtype.
+ */
+#ifndef HSA_H_
+#define HSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HSA_OK = 0,
+    HSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, inconsistent sizes */
+    HSA_ERR_UNSUPPORTED = 2,   /* valid request outside the supported shapes/dtypes */
+    HSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than *_workspace_size */
+    HSA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+    HSA_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see hsa_check) */
+} hsa_status_t;
+
+typedef enum { HSA_F32 = 0, HSA_BF16 = 1 } hsa_dtype_t;
+
+/*
+ * hsa_landmarks -- DHSA landmarks: l[b,g,i] = sqrt(S) * mean of the S keys of
+ * chunk i (Dynamic Hierarchical Sparse Attention review, "What carries the
+ * argument": chunk representation sqrt(|C|) times the mean key).
+ *   K       [B, Hkv, L, d]  in k_dt (bf16 or fp32)
+ *   lm_out  [B, Hkv, floor(L/S), d] fp32 -- one landmark per complete chunk;
+ *           a partial tail chunk has none (it is never selectable).
+ * Kept in fp32 because bf16 rounding of a landmark (2^-9 relative) would move
+ * selection scores by more than the separation of near-tied chunks.
+ */
+hsa_status_t hsa_landmarks(const void *K, hsa_dtype_t k_dt, float *lm_out,
+                           int B, int Hkv, int64_t L, int d, int S, void *stream);
+
+/*
+ * hsa_prefill_workspace_size -- bytes of device workspace hsa_prefill needs
+ * for these sizes (0 on invalid arguments).  The workspace holds the group
+ * selection, the fusion weights, the chunk-bucketed work list, per-entry
+ * partial outputs and a status word.  A new workspace must be zero-filled
+ * once before its first use; every completed call leaves it reusable.
+ */
+size_t hsa_prefill_workspace_size(int B, int H, int Hkv, int64_t L, int d, int S, int topk);
+
+/*
+ * hsa_prefill -- causal prefill of L query tokens against their own K/V.
+ *   Q        [B, L, H, d]    dt (the G heads of a group are adjacent)
+ *   K, V     [B, Hkv, L, d]  dt (one chunk = S contiguous rows)
+ *   lm       [B, Hkv, floor(L/S), d] in lm_dt (bf16 or fp32), or NULL to use
+ *            the DHSA form computed from K (hsa_landmarks, written into the
+ *            workspace)
+ *   own_chunk 1: add causal attention over keys c_t*S .. t (query t's own,
+ *            unfinished chunk is never selectable); 0: retrieved chunks only.
+ *   scale    logit scale for landmark scores and in-chunk logits; 0 -> 1/sqrt(d)
+ *   O        [B, L, H, d]    dt, written
+ *   idx_out  [B, L, Hkv, topk] int32 or NULL: selected chunks in rank order
+ *            (best first), -1 where fewer than topk chunks are visible
+ *   w_out    [B, L, H, topk] fp32 or NULL: fusion weights (0 on padded slots)
+ * L need not be a multiple of S.  A query with no visible chunk and
+ * own_chunk = 0 gets O = 0.
+ */
+hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                         const void *lm, hsa_dtype_t lm_dt,
+                         int B, int H, int Hkv, int64_t L, int d, int S, int topk,
+                         int own_chunk, float scale,
+                         void *O, int32_t *idx_out, float *w_out,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * hsa_decode_workspace_size -- bytes of device workspace hsa_decode needs
+ * (0 on invalid arguments; the size depends on the current device's SM
+ * count).  It holds per-(sequence, group) tickets, the per-block candidate
+ * lists and a status word.  A new workspace must be zero-filled once before
+ * its first use; every completed call leaves the tickets at zero again.
+ * Calls that share a workspace must be ordered (same stream).
+ */
+size_t hsa_decode_workspace_size(int B, int H, int Hkv, int64_t Lc, int d, int S, int topk);
+
+/*
+ * hsa_decode -- one new query per sequence at position Lc against a KV cache
+ * of Lc tokens (Lc % S == 0): every one of the Lc/S chunks is visible and
+ * there is no own-chunk term (local attention around the new token belongs to
+ * the model's sliding-window layers, not to this operator).
+ *   q        [B, H, d]          dt
+ *   Kc, Vc   [B, Hkv, Lc, d]    dt; only the selected chunks are read
+ *   lm       [B, Hkv, Lc/S, d]  lm_dt (bf16 or fp32)
+ *   O        [B, H, d]          dt, written
+ *   idx_out  [B, Hkv, topk] int32 or NULL
+ * The landmark scan is split over many thread blocks; the last block of each
+ * (sequence, KV group) merges the partial top-K lists, gathers the selected
+ * chunks and writes O.  Cache offsets are 64-bit (Lc up to 2^31 - 1 tokens).
+ */
+hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                        const void *lm, hsa_dtype_t lm_dt,
+                        int B, int H, int Hkv, int64_t Lc, int d, int S, int topk, float scale,
+                        void *O, int32_t *idx_out,
+                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * hsa_check -- synchronises `stream`, then reads the status word at the head
+ * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
+ * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up (and clears
+ * the word), HSA_ERR_CUDA if the stream reports an error, HSA_OK otherwise.
+ * `workspace` may be NULL to check the stream only.
+ */
+hsa_status_t hsa_check(void *workspace, void *stream);
+
+/*
+ * hsa_set_stage_events -- timing hook for benchmarks.  Until called again
+ * with n = 0, hsa_prefill and hsa_decode calls made by the CALLING THREAD
+ * record events[i] (cudaEvent_t values passed as void*) on their stream at
+ * stage boundary i, for i < n:
+ *   hsa_prefill: 0 start, 1 after the landmark kernel (DHSA mode), 2 after
+ *                selection, 3 after the work-list build, 4 after attention
+ *                (end of the call);
+ *   hsa_decode:  0 start, 1 end.
+ * Boundaries a call does not reach are not recorded.  n must be 0..8.  The
+ * events belong to the caller.  No effect on results.
+ */
+hsa_status_t hsa_set_stage_events(void *const *events, int n);
+
+/*
+ * hsa_last_call_launches -- number of kernels the calling thread's most
+ * recent hsa_prefill / hsa_decode / hsa_landmarks call launched.
+ */
+int hsa_last_call_launches(void);
+
+/* hsa_status_string -- static, NUL-terminated description of a status. */
+const char *hsa_status_string(hsa_status_t status);
+
+/* hsa_version -- library version as major*10000 + minor*100 + patch. */
+int hsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSA_H_ */
