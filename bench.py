@@ -145,6 +145,17 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def make_events(n):
+    """CUDA events with their handles created (torch creates them lazily at
+    the first record, and the library needs the handle up front)."""
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    return evs
+
+
 def kernel_source_hash(files) -> str:
     h = hashlib.sha256()
     for f in files:
@@ -204,8 +215,7 @@ def run_ours(args, dist, rank, world):
                                                   wl.topk), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n_ev = 5
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-                for _ in range(args.steps)]
+    stage_ev = [make_events(n_ev) for _ in range(args.steps)]
 
     def step():
         hsa.prefill(x["Q"], x["K"], x["V"], x["lm"], S=wl.S, topk=wl.topk,
@@ -336,7 +346,7 @@ def bench_decode(args, dev, peaks, rank, dist):
                        dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     steps = max(5, args.steps)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    ev = [make_events(2) for _ in range(steps)]
     for _ in range(3):
         hsa.decode(x["q"], x["K"], x["V"], x["lm"], topk=wl.topk, out=out, ws=ws)
         flush.fill_(1)
@@ -396,9 +406,10 @@ def cpu_baseline(args, wl, budget_s: float = 12.0, x_host=None):
     K, V, lm = f64(x["K"]), f64(x["V"]), f64(x["lm"])
     Qall = x["Q"].reshape(wl.B * wl.L, wl.H, wl.d)
     n = 256
-    total_f, total_s, total_rows = 0.0, 0.0, 0
-    while total_s < budget_s and total_rows < wl.B * wl.L:
-        rows = oracle_sample_rows(wl, n, seed=total_rows)
+    total_f, total_s, total_rows, it = 0.0, 0.0, 0, 0
+    while total_s < budget_s:
+        rows = oracle_sample_rows(wl, n, seed=it)
+        it += 1
         Qr = f64(Qall[torch.as_tensor(rows)])
         t0 = time.perf_counter()
         orc.prefill(None, K, V, lm, wl.S, wl.topk, wl.own_chunk, rows=rows, Q_rows=Qr)
