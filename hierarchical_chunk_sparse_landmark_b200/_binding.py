@@ -22,7 +22,8 @@ HSA_F32, HSA_BF16 = 0, 1
 
 EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_decode_workspace_size", "hsa_decode", "hsa_check", "hsa_status_string",
-            "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches")
+            "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches",
+            "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch")
 
 
 class HSAError(RuntimeError):
@@ -48,11 +49,15 @@ def _declare(lib):
     lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
                                vp, vp, vp, sz, vp]
     lib.hsa_check.argtypes = [vp, vp]
+    lib.hsa_decode_noalloc.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
+                                       i32, f32, vp, vp, vp]
+    lib.hsa_decode_noalloc_max_scratch.argtypes = []
+    lib.hsa_decode_noalloc_max_scratch.restype = sz
     lib.hsa_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
     lib.hsa_status_string.argtypes = [i32]
     lib.hsa_status_string.restype = ctypes.c_char_p
     for n in ("hsa_landmarks", "hsa_prefill", "hsa_decode", "hsa_check", "hsa_version",
-              "hsa_set_stage_events", "hsa_last_call_launches"):
+              "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -195,6 +200,28 @@ def decode(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.0, out=N
                           _ptr(_opt(idx_out)), _ptr(ws), ws.numel() * ws.element_size(),
                           _stream(dev))
     _check(st, "hsa_decode")
+    return out, _opt(idx_out)
+
+
+def decode_noalloc(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.0, out=None,
+                   idx_out=None):
+    """hsa_decode for callers that cannot allocate device memory: the scratch
+    is the library's fixed device array (see hsa_decode_noalloc in hsa.h), so
+    no workspace is passed.  ``out`` and ``idx_out`` should be preallocated by
+    such callers (when omitted they are created here with torch, for tests).
+    Calls must be ordered on one stream.  Returns (O, idx)."""
+    for n, t in (("q", q), ("K", K), ("V", V), ("lm", lm)):
+        _dev(t, n)
+    B, H, d = q.shape
+    _, Hkv, Lc, _ = K.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is True:
+        idx_out = torch.empty(B, Hkv, topk, dtype=torch.int32, device=q.device)
+    st = lib().hsa_decode_noalloc(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm),
+                                  _dtype_code(lm), B, H, Hkv, Lc, d, S, topk, float(scale),
+                                  _ptr(out), _ptr(_opt(idx_out)), _stream(q.device))
+    _check(st, "hsa_decode_noalloc")
     return out, _opt(idx_out)
 
 

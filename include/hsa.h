@@ -137,6 +137,41 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
                         void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * hsa_decode_noalloc -- hsa_decode for callers that cannot allocate device
+ * memory.  (The pages describe no such call; it is an interface convenience
+ * of this library.)  Some callers cannot hand hsa_decode a workspace: a
+ * plugin inside a host program that owns all device memory (for example a
+ * serving engine that reserves the whole HBM for its KV cache at start-up and
+ * passes a plugin only its inputs and outputs), or code on a latency-critical
+ * path that must not call cudaMalloc/cudaFree because they can synchronise
+ * the device.  This entry point takes the same arguments as hsa_decode minus
+ * the workspace and allocates nothing: its scratch is one fixed array of
+ * hsa_decode_noalloc_max_scratch() bytes (1 MiB) in device global memory that
+ * the library declares statically, so every GPU that loads the library holds
+ * it until the process exits.
+ *  - Sizes whose scratch (hsa_decode_workspace_size) exceeds that array are
+ *    rejected with HSA_ERR_WORKSPACE before anything is launched; invalid
+ *    arguments return the same status hsa_decode would.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture on the device.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    previous call's contents.  Each call clears the part that must start at
+ *    zero with cudaMemsetAsync on `stream`.  Calls that can overlap on the
+ *    GPU (different streams, or several host threads without ordering) race
+ *    on the array and give wrong results: order them on one stream.
+ *  - No cudaMalloc, cudaFree or other allocating routine is called.
+ * hsa_check(NULL, stream) reports errors of a call.
+ */
+hsa_status_t hsa_decode_noalloc(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                                const void *lm, hsa_dtype_t lm_dt,
+                                int B, int H, int Hkv, int64_t Lc, int d, int S, int topk,
+                                float scale, void *O, int32_t *idx_out, void *stream);
+
+/* hsa_decode_noalloc_max_scratch -- size in bytes of hsa_decode_noalloc's array. */
+size_t hsa_decode_noalloc_max_scratch(void);
+
+/*
  * hsa_check -- synchronises `stream`, then reads the status word at the head
  * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
  * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up (and clears
