@@ -248,6 +248,8 @@ def run_ours(args, dist, rank, world):
     step_ms = [stage_ev[i][0].elapsed_time(stage_ev[i][4]) for i in range(args.steps)]
     attn_ms = [stage_ev[i][3].elapsed_time(stage_ev[i][4]) for i in range(args.steps)]
     sel_ms = [stage_ev[i][1].elapsed_time(stage_ev[i][2]) for i in range(args.steps)]
+    lm_ms = [stage_ev[i][0].elapsed_time(stage_ev[i][1]) for i in range(args.steps)]
+    bkt_ms = [stage_ev[i][2].elapsed_time(stage_ev[i][3]) for i in range(args.steps)]
     total_s = sum(step_ms) / 1e3
     units, tmax = aggregate(dist, flops["total"] * args.steps / 1e12, total_s, dev)
     value = units / tmax
@@ -256,10 +258,14 @@ def run_ours(args, dist, rank, world):
     attn_s = statistics.mean(attn_ms) / 1e3
     attn_tf = flops["attention_kernel"] / attn_s / 1e12
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    attn_files = ["hierarchical_chunk_sparse_landmark_b200/csrc/attend_simt.cu"]
-    roofline = {"kernel": "attend_simt_kernel", "bound": "tensor", "achieved": round(attn_tf, 3),
+    tc_path = wl.dtype == "bf16" and wl.G in (8, 16) and wl.d in (64, 128)
+    attn_files = ["hierarchical_chunk_sparse_landmark_b200/csrc/" +
+                  ("attend_tc.cu" if tc_path else "attend_simt.cu")]
+    kname = ("attend_tc_kernel (retrieved-chunk + own-chunk launches)" if tc_path
+             else "attend_simt_kernel")
+    roofline = {"kernel": kname, "bound": "tensor", "achieved": round(attn_tf, 3),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 5),
-                "traffic": measured_traffic("attend", attn_files),
+                "traffic": measured_traffic(attn_files[0].rsplit("/", 1)[1][:-3], attn_files),
                 "peak_source": peaks["source"] + " bf16 burst",
                 "algorithmic_flops_per_launch": flops["attention_kernel"],
                 "ms_per_launch": round(attn_s * 1e3, 4)}
@@ -274,7 +280,9 @@ def run_ours(args, dist, rank, world):
                    "d": wl.d, "S": wl.S, "topk": wl.topk, "own_chunk": wl.own_chunk,
                    "landmarks": wl.landmarks, "parallelism": f"independent batches x{world}",
                    "l2": "flushed between timed steps (256 MiB write)"},
-        "stage_ms": {"selection": round(statistics.mean(sel_ms), 4),
+        "stage_ms": {"landmarks": round(statistics.mean(lm_ms), 4),
+                     "selection": round(statistics.mean(sel_ms), 4),
+                     "work_list": round(statistics.mean(bkt_ms), 4),
                      "attention": round(statistics.mean(attn_ms), 4)},
         "flops_per_step": flops,
         "roofline": roofline, "clocks": clocks, "gpu_launches": launches,

@@ -1,6 +1,8 @@
 // abi.cu -- the extern "C" entry points of libhsa (declared in include/hsa.h):
 // argument validation, workspace layout and kernel dispatch.
+#include <cuda_fp16.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -21,6 +23,16 @@ cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf
                           int S, int topk, float scale, int splits, uint64_t *cand,
                           unsigned *tickets, void *O, int32_t *idx_out, cudaStream_t st);
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
+cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
+                          int ept, int32_t *counts, int32_t *cursor, int32_t *entries,
+                          int4 *tiles, int32_t *tile_count, cudaStream_t st);
+bool attend_tc_supported(bool bf16, int G, int d);
+cudaError_t launch_attend_tc(const void *Q, const void *K, const void *V, int B, int H, int Hkv,
+                             int64_t L, int d, int S, int topk, int own_chunk, float scale,
+                             const int32_t *idx, const float *w, const int32_t *entries,
+                             const int4 *tiles, const int32_t *tile_count, int64_t max_tiles,
+                             __half *part, void *O, unsigned *status, int num_sms,
+                             cudaStream_t st);
 }  // namespace hsa
 
 using namespace hsa;
@@ -55,21 +67,63 @@ int num_sms() {
     return sms;
 }
 
+// Shapes the chunk-bucketed tensor-core path takes (bf16 inputs are checked
+// at dispatch): G in {8, 16} so a 128-row tile holds whole KV groups, and all
+// row / entry indices fit the 32-bit fields of the work lists and TMA maps.
+bool tc_shape_ok(int B, int H, int Hkv, int64_t L, int d, int topk) {
+    const int G = H / Hkv;
+    if (!(G == 8 || G == 16) || !(d == 64 || d == 128)) return false;
+    if (L >= (int64_t(1) << 26)) return false;                      // entry code t*32+k
+    if ((int64_t)B * L * H >= INT32_MAX) return false;              // TMA row of Q
+    if ((int64_t)B * Hkv * L * topk >= INT32_MAX) return false;     // entry index
+    return true;
+}
+
 struct PrefillLayout {
     size_t idx_off, w_off, lm_off, total;
+    // tensor-core path (present when tc_shape_ok)
+    bool tc;
+    size_t counts_off, counts_bytes, cursor_off, entries_off, tiles_off, part_off;
+    int64_t max_tiles;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
     PrefillLayout p;
+    const int64_t Nc = L / S;
     size_t off = kStatusBytes;
     p.idx_off = off;
     off = align_up(off + sizeof(int32_t) * (size_t)B * L * Hkv * topk, 256);
     p.w_off = off;
     off = align_up(off + sizeof(float) * (size_t)B * L * H * topk, 256);
     p.lm_off = off;
-    off = align_up(off + sizeof(float) * (size_t)B * Hkv * (L / S) * d, 256);
+    off = align_up(off + sizeof(float) * (size_t)B * Hkv * Nc * d, 256);
+    p.tc = tc_shape_ok(B, H, Hkv, L, d, topk);
+    p.counts_off = p.cursor_off = p.entries_off = p.tiles_off = p.part_off = 0;
+    p.counts_bytes = 0;
+    p.max_tiles = 0;
+    if (p.tc) {
+        const int ept = 128 / (H / Hkv);
+        // per-(b, g, chunk) counts followed by the global tile counter: one memset
+        p.counts_off = off;
+        p.counts_bytes = sizeof(int32_t) * ((size_t)B * Hkv * Nc + 1);
+        off = align_up(off + p.counts_bytes, 256);
+        p.cursor_off = off;
+        off = align_up(off + sizeof(int32_t) * (size_t)B * Hkv * Nc, 256);
+        p.entries_off = off;
+        off = align_up(off + sizeof(int32_t) * (size_t)B * Hkv * L * topk, 256);
+        p.max_tiles = (int64_t)B * Hkv * ((L * topk + ept - 1) / ept + Nc);
+        p.tiles_off = off;
+        off = align_up(off + sizeof(int4) * (size_t)p.max_tiles, 256);
+        p.part_off = off;
+        off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
+    }
     p.total = off;
     return p;
+}
+
+bool force_simt_path() {
+    const char *v = getenv("HSA_PREFILL_PATH");
+    return v && strcmp(v, "simt") == 0;
 }
 
 struct DecodeLayout {
@@ -190,10 +244,30 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
     if (e != cudaSuccess) return HSA_ERR_CUDA;
     t_launches += 1;
     stage_mark(2, st);
-    stage_mark(3, st);
-    e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale, O,
-                           st);
-    t_launches += e == cudaSuccess ? 1 : 0;
+    const bool use_tc = bf16 && lay.tc && !force_simt_path() &&
+                        attend_tc_supported(bf16, H / Hkv, d);
+    if (use_tc) {
+        const int64_t Nc = L / S;
+        int32_t *counts = (int32_t *)(ws + lay.counts_off);
+        int32_t *tile_count = counts + (size_t)B * Hkv * Nc;
+        if (cudaMemsetAsync(counts, 0, lay.counts_bytes, st) != cudaSuccess) return HSA_ERR_CUDA;
+        e = launch_bucket(idx, B, Hkv, L, topk, Nc, 128 / (H / Hkv), counts,
+                          (int32_t *)(ws + lay.cursor_off), (int32_t *)(ws + lay.entries_off),
+                          (int4 *)(ws + lay.tiles_off), tile_count, st);
+        if (e != cudaSuccess) return HSA_ERR_CUDA;
+        t_launches += 3;
+        stage_mark(3, st);
+        e = launch_attend_tc(Q, K, V, B, H, Hkv, L, d, S, topk, own_chunk, scale, idx, w,
+                             (const int32_t *)(ws + lay.entries_off),
+                             (const int4 *)(ws + lay.tiles_off), tile_count, lay.max_tiles,
+                             (__half *)(ws + lay.part_off), O, (unsigned *)ws, num_sms(), st);
+        t_launches += e == cudaSuccess ? 2 : 0;
+    } else {
+        stage_mark(3, st);
+        e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale,
+                               O, st);
+        t_launches += e == cudaSuccess ? 1 : 0;
+    }
     stage_mark(4, st);
     return from_cuda(e);
 }
