@@ -24,15 +24,27 @@ cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf
                           unsigned *tickets, void *O, int32_t *idx_out, cudaStream_t st);
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
-                          int ept, int32_t *counts, int32_t *cursor, int32_t *entries,
-                          int4 *tiles, int32_t *tile_count, cudaStream_t st);
+                          int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
+                          int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
+                          int64_t *seg_start, cudaStream_t st);
+struct TcLaunch {
+    const void *Q, *K, *V, *lm;
+    int B, H, Hkv, S, topk, own_chunk, lm_bf16;
+    int64_t L, W, cap;
+    float scale;
+    const int32_t *idx, *entries, *wntiles;
+    const int4 *wtiles;
+    int32_t *done;
+    const int64_t *seg_start;
+    float *logits, *w_out;
+    __half *part;
+    void *O;
+    unsigned *status;
+    int num_sms;
+};
 bool attend_tc_supported(bool bf16, int G, int d);
-cudaError_t launch_attend_tc(const void *Q, const void *K, const void *V, int B, int H, int Hkv,
-                             int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                             const int32_t *idx, const float *w, const int32_t *entries,
-                             const int4 *tiles, const int32_t *tile_count, int64_t max_tiles,
-                             __half *part, void *O, unsigned *status, int num_sms,
-                             cudaStream_t st);
+int64_t attend_tc_max_windows();
+cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st);
 }  // namespace hsa
 
 using namespace hsa;
@@ -79,12 +91,27 @@ bool tc_shape_ok(int B, int H, int Hkv, int64_t L, int d, int topk) {
     return true;
 }
 
+// Token window of the tensor-core work queue: sized so that one window's fp16
+// partial outputs (W * topk * G * d * 2 bytes per (b, g)) are about 32 MB and
+// stay in L2 until that window's own tiles fuse them; a multiple of 256.
+int64_t tc_window(int B, int H, int Hkv, int64_t L, int d, int topk, int64_t max_windows) {
+    const int G = H / Hkv;
+    const int64_t per_token = (int64_t)topk * G * d * 2;
+    int64_t W = ((int64_t(32) << 20) / per_token) / 256 * 256;
+    if (W < 256) W = 256;
+    const int64_t Lr = (L + 255) / 256 * 256;
+    if (W > Lr) W = Lr;
+    while ((int64_t)B * Hkv * ((L + W - 1) / W) > max_windows) W *= 2;
+    return W;
+}
+
 struct PrefillLayout {
     size_t idx_off, w_off, lm_off, total;
     // tensor-core path (present when tc_shape_ok)
     bool tc;
-    size_t counts_off, counts_bytes, cursor_off, entries_off, tiles_off, part_off;
-    int64_t max_tiles;
+    int64_t W, NW, cap;
+    size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
+        seg_off, part_off;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
@@ -98,22 +125,29 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     p.lm_off = off;
     off = align_up(off + sizeof(float) * (size_t)B * Hkv * Nc * d, 256);
     p.tc = tc_shape_ok(B, H, Hkv, L, d, topk);
-    p.counts_off = p.cursor_off = p.entries_off = p.tiles_off = p.part_off = 0;
-    p.counts_bytes = 0;
-    p.max_tiles = 0;
+    p.W = p.NW = p.cap = 0;
+    p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
+    p.wntiles_off = p.done_off = p.seg_off = p.part_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
-        // per-(b, g, chunk) counts followed by the global tile counter: one memset
+        p.W = tc_window(B, H, Hkv, L, d, topk, attend_tc_max_windows());
+        p.NW = (int64_t)B * Hkv * ((L + p.W - 1) / p.W);
+        p.cap = (p.W * topk + ept - 1) / ept + Nc;
         p.counts_off = off;
-        p.counts_bytes = sizeof(int32_t) * ((size_t)B * Hkv * Nc + 1);
+        p.counts_bytes = sizeof(int32_t) * (size_t)(p.NW * Nc > 0 ? p.NW * Nc : 1);
         off = align_up(off + p.counts_bytes, 256);
         p.cursor_off = off;
-        off = align_up(off + sizeof(int32_t) * (size_t)B * Hkv * Nc, 256);
+        off = align_up(off + p.counts_bytes, 256);
         p.entries_off = off;
         off = align_up(off + sizeof(int32_t) * (size_t)B * Hkv * L * topk, 256);
-        p.max_tiles = (int64_t)B * Hkv * ((L * topk + ept - 1) / ept + Nc);
-        p.tiles_off = off;
-        off = align_up(off + sizeof(int4) * (size_t)p.max_tiles, 256);
+        p.wtiles_off = off;
+        off = align_up(off + sizeof(int4) * (size_t)(p.NW * p.cap), 256);
+        p.wntiles_off = off;
+        off = align_up(off + sizeof(int32_t) * (size_t)p.NW, 256);
+        p.done_off = off;
+        off = align_up(off + sizeof(int32_t) * (size_t)p.NW, 256);
+        p.seg_off = off;
+        off = align_up(off + sizeof(int64_t) * (size_t)(2 * p.NW + 1), 256);
         p.part_off = off;
         off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
     }
@@ -239,29 +273,42 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         lm_bf16 = false;
     }
     stage_mark(1, st);
+    const bool use_tc = bf16 && lay.tc && !force_simt_path() &&
+                        attend_tc_supported(bf16, H / Hkv, d);
+    // The tensor-core path computes the fusion logits inside its S tiles and
+    // the weights in its fusion epilogue; the workspace weight region then
+    // holds the logits.
+    float *w_ws = (float *)(ws + lay.w_off);
     cudaError_t e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
-                                  w, st);
+                                  use_tc ? nullptr : w, st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
     t_launches += 1;
     stage_mark(2, st);
-    const bool use_tc = bf16 && lay.tc && !force_simt_path() &&
-                        attend_tc_supported(bf16, H / Hkv, d);
     if (use_tc) {
         const int64_t Nc = L / S;
-        int32_t *counts = (int32_t *)(ws + lay.counts_off);
-        int32_t *tile_count = counts + (size_t)B * Hkv * Nc;
-        if (cudaMemsetAsync(counts, 0, lay.counts_bytes, st) != cudaSuccess) return HSA_ERR_CUDA;
-        e = launch_bucket(idx, B, Hkv, L, topk, Nc, 128 / (H / Hkv), counts,
-                          (int32_t *)(ws + lay.cursor_off), (int32_t *)(ws + lay.entries_off),
-                          (int4 *)(ws + lay.tiles_off), tile_count, st);
+        if (cudaMemsetAsync(ws + lay.counts_off, 0, lay.counts_bytes, st) != cudaSuccess)
+            return HSA_ERR_CUDA;
+        e = launch_bucket(idx, B, Hkv, L, topk, Nc, 128 / (H / Hkv), lay.W, lay.cap,
+                          (int32_t *)(ws + lay.counts_off), (int32_t *)(ws + lay.cursor_off),
+                          (int32_t *)(ws + lay.entries_off), (int4 *)(ws + lay.wtiles_off),
+                          (int32_t *)(ws + lay.wntiles_off), (int32_t *)(ws + lay.done_off),
+                          (int64_t *)(ws + lay.seg_off), st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
-        t_launches += 3;
+        t_launches += 4;
         stage_mark(3, st);
-        e = launch_attend_tc(Q, K, V, B, H, Hkv, L, d, S, topk, own_chunk, scale, idx, w,
-                             (const int32_t *)(ws + lay.entries_off),
-                             (const int4 *)(ws + lay.tiles_off), tile_count, lay.max_tiles,
-                             (__half *)(ws + lay.part_off), O, (unsigned *)ws, num_sms(), st);
-        t_launches += e == cudaSuccess ? 2 : 0;
+        TcLaunch a;
+        a.Q = Q; a.K = K; a.V = V; a.lm = lm_use; a.lm_bf16 = lm_bf16 ? 1 : 0;
+        a.B = B; a.H = H; a.Hkv = Hkv; a.S = S; a.topk = topk; a.own_chunk = own_chunk;
+        a.L = L; a.W = lay.W; a.cap = lay.cap; a.scale = scale;
+        a.idx = idx; a.entries = (const int32_t *)(ws + lay.entries_off);
+        a.wntiles = (const int32_t *)(ws + lay.wntiles_off);
+        a.wtiles = (const int4 *)(ws + lay.wtiles_off); a.done = (int32_t *)(ws + lay.done_off);
+        a.seg_start = (const int64_t *)(ws + lay.seg_off);
+        a.logits = w_ws; a.w_out = w_out;
+        a.part = (__half *)(ws + lay.part_off); a.O = O; a.status = (unsigned *)ws;
+        a.num_sms = num_sms();
+        e = launch_attend_tc(a, d, st);
+        t_launches += e == cudaSuccess ? 1 : 0;
     } else {
         stage_mark(3, st);
         e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale,

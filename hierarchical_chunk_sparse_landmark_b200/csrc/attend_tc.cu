@@ -1,27 +1,39 @@
-// attend_tc.cu -- in-chunk attention and fusion on the 5th-generation tensor
-// cores (tcgen05, TMEM accumulators, TMA tile loads), bf16 in, fp32 accumulate.
+// attend_tc.cu -- in-chunk attention and score-weighted fusion on the
+// 5th-generation tensor cores (tcgen05 MMA, TMEM accumulators, TMA tile
+// loads), bf16 in, fp32 accumulate.
 //
 // HiLS Attention abstract: every query attends independently inside each
 // retrieved chunk; the chunk outputs are fused with weights from the retrieval
 // scores.  The work is chunk-bucketed (bucket.cu): a tile is one chunk's 64
 // keys/values plus up to 128/G selected entries, each entry contributing its G
 // query-head rows (the heads of a KV group share the selection), so a tile is a
-// dense 128-row problem:
+// dense 128-row problem.  The chunk's landmark rides along as two extra "key"
+// rows (its bf16 high and low parts), so the same MMA also yields every row's
+// fusion logit scale * q_h . l_chunk:
 //
-//   S = Q_rows . K_chunk^T          M=128, N=64, K=d   (tcgen05, TMEM)
-//   P = exp(S*scale - rowmax)        per row, in registers (bf16 into smem)
-//   O = P . V_chunk                  M=128, N=d, K=64   (tcgen05, TMEM)
-//   partial[entry] = w/rowsum * O    fp16, one slot per (t, g, k)
+//   S = Q_rows . [K_chunk ; l_hi ; l_lo]^T  M=128, N=80, K=d  (tcgen05 -> TMEM)
+//   P = exp(S*scale - rowmax) / rowsum      per row in registers, bf16 -> smem
+//   O = P . V_chunk                         M=128, N=d, K=64  (tcgen05 -> TMEM)
+//   partial[t, g, k] = O (fp16), logit[t, h, k] = scale * (S[:,64] + S[:,65])
 //
-// Mode "own": tiles of 128/G consecutive tokens of one chunk against their own
-// chunk with the causal mask (keys c*S .. t); the epilogue adds the token's
-// K partial slots and writes O in bf16, so the fusion needs no extra pass.
+// Own tiles: 128/G consecutive tokens of a chunk against that chunk with the
+// causal mask (keys c*S .. t).  Their epilogue completes the fusion:
+//   w = softmax over the token's selected chunks of the logits,
+//   O = own_term + sum_k w_k * partial_k  (bf16 out).
 //
-// One tile at a time per block of 128 threads (thread r <-> tile row r <->
-// TMEM lane r); thread 0 issues TMA and MMA.  Two blocks fit per SM at d=128
-// (80 KB of shared memory and 256 TMEM columns each; four at d=64), so one block's softmax and
-// epilogue overlap the other's loads and MMAs.  Every wait is bounded; a
-// timed-out block sets the workspace status flag, frees its TMEM and exits.
+// One persistent block per SM walks the work queue (retrieved-chunk tiles of
+// window n, then own tiles of window n-1, ...) with four roles linked by
+// mbarriers and double-buffered shared memory / TMEM:
+//   warp 0      producer  (landmark rows into smem; TMA of the chunk's K and V
+//                          and, lane-parallel, of the gathered Q rows)
+//   warp 1      MMA issuer (S of tile j+1 is issued before P.V of tile j)
+//   warps 2-5   softmax   (thread = tile row = TMEM lane)
+//   warps 6-9   epilogue  (TMEM -> fp16 partials, or -> fused bf16 O)
+// Consumer roles prefetch the next tile's metadata while working on the
+// current one.  Own tiles of window n wait, in the epilogue only, until every
+// retrieved-chunk tile of window n has published its partials.  Every wait is
+// bounded; on expiry the block sets the status flag in the workspace, lets
+// in-flight copies land, frees its TMEM and exits.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -35,32 +47,41 @@ struct TcCfg {
     static constexpr int M = 128;
     static constexpr int EPT = M / G;            // entries (or tokens) per tile
     static constexpr int KB = D / 64;            // 64-element blocks of d
-    static constexpr int A_BYTES = M * D * 2;    // gathered query rows
-    static constexpr int KV_BYTES = 64 * D * 2;  // one chunk of K (or V)
+    static constexpr int NS = 80;                // S columns: 64 keys, l_hi, l_lo, pad
+    static constexpr int Q_BYTES = M * D * 2;    // gathered query rows
+    static constexpr int KBLK = NS * 128;        // one 64-wide d block of [K; l]
+    static constexpr int K_BYTES = KB * KBLK;
+    static constexpr int V_BYTES = 64 * D * 2;
     static constexpr int P_BYTES = M * 64 * 2;   // probabilities, bf16
-    static constexpr int SMEM = 1024 + A_BYTES + 2 * KV_BYTES + P_BYTES + 64;
-    // S: 64 fp32 columns at 0; O: D columns after it (power-of-two allocation)
-    static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;
-    static constexpr uint32_t O_COL = D == 128 ? 128 : 64;
+    static constexpr int STAGE = Q_BYTES + K_BYTES + V_BYTES + P_BYTES;
+    static constexpr int SMEM = 1024 + 2 * STAGE + 256;
+    // TMEM: S[2] at columns 0 / 128 (80 used), O[2] at 256 / 256 + D
+    static constexpr uint32_t S_COL = 128;
+    static constexpr uint32_t O_COL = 256;
+    static constexpr uint32_t TMEM_COLS = 512;
 };
 
 struct TcParams {
-    const int4 *tiles;
-    const int32_t *tile_count;
+    const int64_t *seg_start;     // [2 * NW + 1]
+    const int4 *wtiles;           // [NW * cap] retrieved-chunk tiles per window
+    const int32_t *wntiles;       // [NW]
+    int32_t *done;                // [NW] published retrieved-chunk tiles
     const int32_t *entries;
-    const float *w;
     const int32_t *idx;
+    const void *lm;               // [B, Hkv, Nc, D] bf16 or fp32
+    float *logits;                // [B, L, H, topk] fusion logits
+    float *w_out;                 // [B, L, H, topk] or NULL
     __half *part;
     __nv_bfloat16 *O;
     unsigned *status;
-    int64_t L;
-    int64_t n_own_tiles;
-    int H, Hkv, topk, S, own_mode;
-    int add_own;          // own mode: 1 adds the causal own-chunk term, 0 only fuses
-    float scale_log2e;
+    int64_t L, W, nwb, NW, cap, Nc;
+    int H, Hkv, topk, S, add_own, lm_bf16;
+    float scale, scale_log2e;
 };
 
-constexpr long long kWaitBudget = 4000000000LL;   // SM cycles (~2 s)
+constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
+constexpr int kThreads = 320;
+constexpr int kMaxWindows = 2048;                  // shared segment table size / 2
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -70,224 +91,409 @@ __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
     __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&v);
 }
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded mbarrier wait that also gives up when another role aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!tc::mbar_try_wait(bar, parity)) {
+        if (*abort || clock64() - t0 > kWaitBudget) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// A queue position decoded into one tile.
+struct Tile {
+    int64_t bg, first, t0;   // first entry (retrieved) or first token (own)
+    int chunk, n, own;
+    int64_t win;
+};
+
+__device__ __forceinline__ void decode_tile(const TcParams &p, const int64_t *seg, int nseg,
+                                            int64_t pos, int ept, Tile &tl) {
+    int lo = 0, hi = nseg;                  // seg[lo] <= pos < seg[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (seg[mid] <= pos) lo = mid; else hi = mid;
+    }
+    const int64_t j = pos - seg[lo];
+    if (lo == 0) { tl.own = 0; tl.win = 0; }
+    else if (lo == nseg - 1) { tl.own = 1; tl.win = p.NW - 1; }
+    else if (lo & 1) { tl.own = 0; tl.win = (lo + 1) / 2; }
+    else { tl.own = 1; tl.win = lo / 2 - 1; }
+    if (!tl.own) {
+        const int4 d = p.wtiles[tl.win * p.cap + j];
+        tl.bg = d.x; tl.chunk = d.y; tl.first = d.z; tl.n = d.w; tl.t0 = 0;
+    } else {
+        tl.bg = tl.win / p.nwb;
+        const int64_t ts = (tl.win % p.nwb) * p.W;
+        const int64_t te = ts + p.W < p.L ? ts + p.W : p.L;
+        tl.t0 = ts + j * ept;
+        tl.n = (int)(te - tl.t0 < ept ? te - tl.t0 : ept);
+        tl.chunk = (int)(tl.t0 / p.S);
+        tl.first = 0;
+    }
+}
+
+// Per-row view of a tile for the softmax and epilogue threads.
+struct RowJob {
+    Tile tl;
+    int64_t t;
+    int k;
+    bool valid;
+};
+
+__device__ __forceinline__ RowJob fetch_row(const TcParams &p, const int64_t *seg, int nseg,
+                                            int64_t pos, int ept, int e) {
+    RowJob rj;
+    decode_tile(p, seg, nseg, pos, ept, rj.tl);
+    rj.valid = e < rj.tl.n;
+    rj.t = 0;
+    rj.k = 0;
+    if (rj.valid) {
+        if (rj.tl.own) rj.t = rj.tl.t0 + e;
+        else {
+            const int32_t code = p.entries[rj.tl.first + e];
+            rj.t = code >> 5;
+            rj.k = code & 31;
+        }
+    }
+    return rj;
+}
 
 template <int D, int G>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const TcParams p) {
     using C = TcCfg<D, G>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sA = smem;                      // [KB][128 rows][128 B]
-    uint8_t *sK = sA + C::A_BYTES;           // [KB][64 rows][128 B]
-    uint8_t *sV = sK + C::KV_BYTES;          // [KB][64 rows][128 B]
-    uint8_t *sP = sV + C::KV_BYTES;          // [128 rows][128 B]
-    uint64_t *bar = (uint64_t *)(sP + C::P_BYTES);   // [0] loads, [1] mma
-    uint32_t *s_tmem = (uint32_t *)(bar + 2);
+    // stage s: [Q | K;l | V | P]
+    auto sQ = [&](int s) { return smem + s * C::STAGE; };
+    auto sK = [&](int s) { return smem + s * C::STAGE + C::Q_BYTES; };
+    auto sV = [&](int s) { return smem + s * C::STAGE + C::Q_BYTES + C::K_BYTES; };
+    auto sP = [&](int s) { return smem + s * C::STAGE + C::Q_BYTES + C::K_BYTES + C::V_BYTES; };
+    uint64_t *bars = (uint64_t *)(smem + 2 * C::STAGE);
+    uint64_t *full = bars, *empty = bars + 2, *sfull = bars + 4, *sfree = bars + 6;
+    uint64_t *pfull = bars + 8, *ofull = bars + 10, *ofree = bars + 12;
+    uint32_t *s_tmem = (uint32_t *)(bars + 14);
+    volatile int *s_abort = (volatile int *)(s_tmem + 1);
+    __shared__ int64_t seg[2 * kMaxWindows + 1];
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    if (warp == 0) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nseg = (int)(2 * p.NW);
+    for (int i = tid; i <= nseg; i += kThreads) seg[i] = p.seg_start[i];
+    if (warp == 1) {
         tc::tmem_alloc(s_tmem, C::TMEM_COLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(&bar[0], 1);
-        tc::mbar_init(&bar[1], 1);
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+            tc::mbar_init(&sfull[s], 1);
+            tc::mbar_init(&sfree[s], 128);
+            tc::mbar_init(&pfull[s], 128);
+            tc::mbar_init(&ofull[s], 1);
+            tc::mbar_init(&ofree[s], 128);
+        }
+        *s_abort = 0;
         tc::fence_barrier_init();
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tS = tmem, tO = tmem + C::O_COL;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-
-    constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, 64, false);
-    constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
+    const int64_t qlen = seg[nseg];
     const int64_t L = p.L;
-    const int S = p.S, H = p.H, Hkv = p.Hkv, topk = p.topk;
-    const int64_t n_tiles = p.own_mode ? p.n_own_tiles
-                                       : (int64_t)(*(volatile const int32_t *)p.tile_count);
-    const int64_t own_per_bg = (L + C::EPT - 1) / C::EPT;
-    uint32_t ph_load = 0, ph_mma = 0;
-    int abort = 0;
+    const int H = p.H, Hkv = p.Hkv, topk = p.topk, S = p.S;
+    constexpr int EPT = C::EPT;
+    const int64_t my_tiles = qlen > blockIdx.x ? (qlen - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        int64_t bg, first = 0, t0 = 0;
-        int chunk, n;
-        if (!p.own_mode) {
-            const int4 d = p.tiles[tile];
-            bg = d.x; chunk = d.y; first = d.z; n = d.w;
-        } else {
-            bg = tile / own_per_bg;
-            t0 = (tile % own_per_bg) * C::EPT;
-            n = (int)((L - t0) < C::EPT ? (L - t0) : C::EPT);
-            chunk = (int)(t0 / S);
-        }
-        const int64_t b = bg / Hkv;
-        const int g = (int)(bg % Hkv);
-
-        // this thread's row: entry e, head h
-        const int e = tid / G, h = tid % G;
-        const bool valid = e < n;
-        int64_t t = 0;
-        int k = 0;
-        if (valid) {
-            if (!p.own_mode) {
-                const int32_t code = p.entries[first + e];
-                t = code >> 5;
-                k = code & 31;
-            } else {
-                t = t0 + e;
-            }
-        }
-
-        if (tid == 0) {
-            tc::mbar_expect_tx(&bar[0], (uint32_t)(2 * C::KV_BYTES + n * G * D * 2));
-            const int krow = (int)(bg * L + (int64_t)chunk * S);
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            const int64_t pos = blockIdx.x + j * gridDim.x;
+            Tile tl;
+            decode_tile(p, seg, nseg, pos, EPT, tl);
+            const int s = (int)(j & 1);
+            int ok = 1;
+            if (lane == 0 && j >= 2) ok = wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int64_t b = tl.bg / Hkv;
+            const int g = (int)(tl.bg % Hkv);
+            int64_t tq = 0;
+            if (lane < tl.n) tq = tl.own ? tl.t0 + lane : (int64_t)(p.entries[tl.first + lane] >> 5);
+            if (!tl.own && lane < D / 8) {
+                // landmark row of the chunk -> rows 64 (bf16 high part) and 65 (low part)
+                float x[8];
+                const int64_t li = (tl.bg * p.Nc + tl.chunk) * D + lane * 8;
+                if (p.lm_bf16) {
+                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(
+                        (const __nv_bfloat16 *)p.lm + li), x);
+                } else {
+                    const uint4 *src = reinterpret_cast<const uint4 *>((const float *)p.lm + li);
+                    Vec16<float>::unpack(src[0], x);
+                    Vec16<float>::unpack(src[1], x + 4);
+                }
+                float hi[8], lo[8];
 #pragma unroll
-            for (int kb = 0; kb < C::KB; ++kb) {
-                tc::tma_load_2d(sK + kb * 8192, &tmK, &bar[0], kb * 64, krow);
-                tc::tma_load_2d(sV + kb * 8192, &tmV, &bar[0], kb * 64, krow);
+                for (int q = 0; q < 8; ++q) {
+                    hi[q] = __bfloat162float(__float2bfloat16_rn(x[q]));
+                    lo[q] = x[q] - hi[q];
+                }
+                const int kb = (lane * 8) / 64, c = ((lane * 8) % 64) / 8;
+                uint8_t *blk = sK(s) + kb * C::KBLK;
+                *reinterpret_cast<uint4 *>(blk + tc::sw128_offset(64, c)) =
+                    make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
+                               pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
+                *reinterpret_cast<uint4 *>(blk + tc::sw128_offset(65, c)) =
+                    make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
+                               pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
+                tc::fence_proxy_async_smem();
             }
-            for (int ee = 0; ee < n; ++ee) {
-                const int64_t tq = p.own_mode ? t0 + ee : (int64_t)(p.entries[first + ee] >> 5);
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_expect_tx(&full[s], (uint32_t)(2 * C::V_BYTES + tl.n * G * D * 2));
+                const int krow = (int)(tl.bg * L + (int64_t)tl.chunk * S);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb) {
+                    tc::tma_load_2d(sK(s) + kb * C::KBLK, &tmK, &full[s], kb * 64, krow);
+                    tc::tma_load_2d(sV(s) + kb * 8192, &tmV, &full[s], kb * 64, krow);
+                }
+            }
+            __syncwarp();
+            if (lane < tl.n) {
                 const int qrow = (int)((b * L + tq) * H + (int64_t)g * G);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tc::tma_load_2d(sA + kb * (128 * 128) + ee * G * 128, &tmQ, &bar[0], kb * 64,
-                                    qrow);
+                    tc::tma_load_2d(sQ(s) + kb * (128 * 128) + lane * G * 128, &tmQ, &full[s],
+                                    kb * 64, qrow);
             }
         }
-        if (!tc::mbar_wait(&bar[0], ph_load, kWaitBudget)) abort = 1;
-        ph_load ^= 1;
-        if (__syncthreads_or(abort)) break;
-
-        // S = Q K^T
-        if (tid == 0) {
-            tc::fence_after_sync();
-#pragma unroll
-            for (int kb = 0; kb < C::KB; ++kb)
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, C::NS, false);
+            constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
+            auto issue_pv = [&](int64_t i) -> bool {
+                const int s = (int)(i & 1);
+                if (!wait_bar(&pfull[s], (uint32_t)((i >> 1) & 1), s_abort)) return false;
+                if (i >= 2 && !wait_bar(&ofree[s], (uint32_t)(((i >> 1) + 1) & 1), s_abort)) return false;
+                tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sA + kb * 16384 + kk * 32), 16, 1024);
-                    const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sK + kb * 8192 + kk * 32), 16, 1024);
-                    tc::mma_bf16(tS, ad, bd, IDESC_S, (kb | kk) ? 1u : 0u);
+                    const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP(s) + kk * 32), 16, 1024);
+                    const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sV(s) + kk * 2048), 8192, 1024);
+                    tc::mma_bf16(tmem + C::O_COL + s * D, ad, bd, IDESC_O, kk ? 1u : 0u);
                 }
-            tc::mma_commit(&bar[1]);
-        }
-        if (!tc::mbar_wait(&bar[1], ph_mma, kWaitBudget)) abort = 1;
-        ph_mma ^= 1;
-        tc::fence_after_sync();
-
-        float s0[32], s1[32];
-        tc::tmem_ld32(tS + lane_off + 0, s0);
-        tc::tmem_ld32(tS + lane_off + 32, s1);
-        tc::tmem_wait_ld();
-        // causal limit inside the own chunk; all 64 keys of a retrieved chunk
-        const int nk = (p.own_mode && valid) ? (int)(t - (int64_t)chunk * S) + 1 : 64;
-        float mx = -INFINITY;
+                tc::mma_commit(&ofull[s]);
+                tc::mma_commit(&empty[s]);
+                return true;
+            };
+            bool ok = true;
+            int64_t j = 0;
+            for (; j < my_tiles && ok; ++j) {
+                const int s = (int)(j & 1);
+                if (!wait_bar(&full[s], (uint32_t)((j >> 1) & 1), s_abort)) { ok = false; break; }
+                if (j >= 2 && !wait_bar(&sfree[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort)) { ok = false; break; }
+                tc::fence_after_sync();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            if (j < nk) mx = fmaxf(mx, s0[j]);
-            if (j + 32 < nk) mx = fmaxf(mx, s1[j]);
-        }
-        const float ms = mx * p.scale_log2e;
-        float l = 0.f;
+                for (int kb = 0; kb < C::KB; ++kb)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            s0[j] = j < nk ? tc::ex2_approx(fmaf(s0[j], p.scale_log2e, -ms)) : 0.f;
-            s1[j] = j + 32 < nk ? tc::ex2_approx(fmaf(s1[j], p.scale_log2e, -ms)) : 0.f;
-            l += s0[j] + s1[j];
-        }
-        // P row (unnormalised, bf16) into the swizzled K-major tile
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float *src = c < 4 ? s0 + 8 * c : s1 + 8 * (c - 4);
-            const uint4 u = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                                       pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
-            *reinterpret_cast<uint4 *>(sP + tc::sw128_offset(tid, c)) = u;
-        }
-        float f = 0.f;
-        if (valid) {
-            const float wt = p.own_mode ? (float)p.add_own : p.w[((b * L + t) * H + (int64_t)g * G + h) * topk + k];
-            f = wt / l;
-        }
-        tc::fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-
-        // O = P V
-        if (tid == 0) {
-            tc::fence_after_sync();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP + kk * 32), 16, 1024);
-                const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sV + kk * 2048), 8192, 1024);
-                tc::mma_bf16(tO, ad, bd, IDESC_O, kk ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sQ(s) + kb * 16384 + kk * 32), 16, 1024);
+                        const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sK(s) + kb * C::KBLK + kk * 32), 16, 1024);
+                        tc::mma_bf16(tmem + s * C::S_COL, ad, bd, IDESC_S, (kb | kk) ? 1u : 0u);
+                    }
+                tc::mma_commit(&sfull[s]);
+                if (j >= 1) ok = issue_pv(j - 1);
             }
-            tc::mma_commit(&bar[1]);
+            if (ok && j >= 1) issue_pv(j - 1);
         }
-        if (!tc::mbar_wait(&bar[1], ph_mma, kWaitBudget)) abort = 1;
-        ph_mma ^= 1;
-        tc::fence_after_sync();
-
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            float o[32];
-            tc::tmem_ld32(tO + lane_off + c0, o);
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ softmax
+        const int q4 = warp & 3;                  // TMEM lane quarter
+        const int r = q4 * 32 + lane;             // tile row
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int e = r / G, h = r % G;
+        RowJob cur;
+        if (my_tiles > 0) cur = fetch_row(p, seg, nseg, blockIdx.x, EPT, e);
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            RowJob nxt;
+            if (j + 1 < my_tiles) nxt = fetch_row(p, seg, nseg, blockIdx.x + (j + 1) * gridDim.x, EPT, e);
+            const int s = (int)(j & 1);
+            const int64_t b = cur.tl.bg / Hkv;
+            const int g = (int)(cur.tl.bg % Hkv);
+            if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
+            tc::fence_after_sync();
+            float s0[32], s1[32], l_hi, l_lo;
+            const uint32_t ta = tmem + s * C::S_COL + lane_off;
+            tc::tmem_ld32(ta, s0);
+            tc::tmem_ld32(ta + 32, s1);
+            tc::tmem_ld2(ta + 64, l_hi, l_lo);
             tc::tmem_wait_ld();
-            if (!valid) continue;
-            if (!p.own_mode) {
-                __half *dst = p.part + ((((b * L + t) * Hkv + g) * topk + k) * G + h) * (int64_t)D + c0;
+            tc::fence_before_sync();
+            tc::mbar_arrive(&sfree[s]);
+            if (cur.valid && !cur.tl.own)
+                p.logits[((b * L + cur.t) * H + (int64_t)g * G + h) * topk + cur.k] =
+                    p.scale * (l_hi + l_lo);
+            const int nk = (cur.tl.own && cur.valid) ? (int)(cur.t - (int64_t)cur.tl.chunk * S) + 1 : 64;
+            float mx = -INFINITY;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                        pack_f16x2(o[8 * q + 0] * f, o[8 * q + 1] * f),
-                        pack_f16x2(o[8 * q + 2] * f, o[8 * q + 3] * f),
-                        pack_f16x2(o[8 * q + 4] * f, o[8 * q + 5] * f),
-                        pack_f16x2(o[8 * q + 6] * f, o[8 * q + 7] * f));
-            } else {
+            for (int c = 0; c < 32; ++c) {
+                if (c < nk) mx = fmaxf(mx, s0[c]);
+                if (c + 32 < nk) mx = fmaxf(mx, s1[c]);
+            }
+            const float ms = mx * p.scale_log2e;
+            float l = 0.f;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[j] *= f;
-                const int32_t *ip = p.idx + ((b * L + t) * Hkv + g) * topk;
-                for (int kk = 0; kk < topk; ++kk) {
-                    if (ip[kk] < 0) break;
-                    const __half *src = p.part + ((((b * L + t) * Hkv + g) * topk + kk) * G + h) * (int64_t)D + c0;
+            for (int c = 0; c < 32; ++c) {
+                s0[c] = c < nk ? tc::ex2_approx(fmaf(s0[c], p.scale_log2e, -ms)) : 0.f;
+                s1[c] = c + 32 < nk ? tc::ex2_approx(fmaf(s1[c], p.scale_log2e, -ms)) : 0.f;
+                l += s0[c] + s1[c];
+            }
+            const float f = cur.valid ? (cur.tl.own ? (float)p.add_own : 1.f) / l : 0.f;
+            if (j >= 2 && !wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort)) break;
+            uint8_t *prow = sP(s);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 u = reinterpret_cast<const uint4 *>(src)[q];
-                        const __half2 *hh = reinterpret_cast<const __half2 *>(&u);
-#pragma unroll
-                        for (int z = 0; z < 4; ++z) {
-                            const float2 v = __half22float2(hh[z]);
-                            o[8 * q + 2 * z] += v.x;
-                            o[8 * q + 2 * z + 1] += v.y;
-                        }
+            for (int c = 0; c < 8; ++c) {
+                const float *src = c < 4 ? s0 + 8 * c : s1 + 8 * (c - 4);
+                const uint4 u = make_uint4(pack_bf16x2(src[0] * f, src[1] * f),
+                                           pack_bf16x2(src[2] * f, src[3] * f),
+                                           pack_bf16x2(src[4] * f, src[5] * f),
+                                           pack_bf16x2(src[6] * f, src[7] * f));
+                *reinterpret_cast<uint4 *>(prow + tc::sw128_offset(r, c)) = u;
+            }
+            tc::fence_proxy_async_smem();
+            if (!cur.tl.own) __threadfence();        // logit visible before the tile is published
+            tc::mbar_arrive(&pfull[s]);
+            cur = nxt;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int e = r / G, h = r % G;
+        const bool leader = (warp == 6 && lane == 0);
+        constexpr int NCH = D / 32;               // 32-column chunks of a row
+        RowJob cur;
+        if (my_tiles > 0) cur = fetch_row(p, seg, nseg, blockIdx.x, EPT, e);
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            RowJob nxt;
+            if (j + 1 < my_tiles) nxt = fetch_row(p, seg, nseg, blockIdx.x + (j + 1) * gridDim.x, EPT, e);
+            const int s = (int)(j & 1);
+            const int64_t b = cur.tl.bg / Hkv;
+            const int g = (int)(cur.tl.bg % Hkv);
+            const int64_t row = (b * L + cur.t) * Hkv + g;       // (t, g) selection row
+            const int64_t hrow = (b * L + cur.t) * H + (int64_t)g * G + h;
+            float lg[32];
+            int nsel = 0;
+            float m = -INFINITY, inv_den = 0.f;
+            if (cur.tl.own) {
+                // the window's retrieved-chunk partials must all be published
+                if (leader) {
+                    const int32_t need = p.wntiles[cur.tl.win];
+                    const long long t0c = clock64();
+                    while (ld_acquire(&p.done[cur.tl.win]) < need) {
+                        if (*s_abort || clock64() - t0c > kWaitBudget) { *s_abort = 1; break; }
+                        __nanosleep(128);
                     }
                 }
-                __nv_bfloat16 *dst = p.O + ((b * L + t) * H + (int64_t)g * G + h) * D + c0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                        pack_bf16x2(o[8 * q + 0], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
-                        pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+                named_sync(1, 128);
+                if (*s_abort) break;
+                if (cur.valid) {
+                    const int32_t *ip = p.idx + row * topk;
+                    for (int kk = 0; kk < topk && ip[kk] >= 0; ++kk) {
+                        lg[kk] = __ldcg(p.logits + hrow * topk + kk);
+                        m = fmaxf(m, lg[kk]);
+                        ++nsel;
+                    }
+                    float den = 0.f;
+                    for (int kk = 0; kk < nsel; ++kk) {
+                        lg[kk] = __expf(lg[kk] - m);
+                        den += lg[kk];
+                    }
+                    inv_den = nsel ? 1.f / den : 0.f;
+                    if (p.w_out)
+                        for (int kk = 0; kk < topk; ++kk)
+                            p.w_out[hrow * topk + kk] = kk < nsel ? lg[kk] * inv_den : 0.f;
+                }
             }
+            if (!wait_bar(&ofull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
+            tc::fence_after_sync();
+#pragma unroll 1
+            for (int ch = 0; ch < NCH; ++ch) {
+                float o[32];
+                tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o);
+                tc::tmem_wait_ld();
+                if (!cur.valid) continue;
+                if (!cur.tl.own) {
+                    // partial layout [entry][d/32][head][32] (fp16)
+                    __half *dst = p.part + (((row * topk + cur.k) * NCH + ch) * G + h) * 32;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
+                            pack_f16x2(o[8 * q + 0], o[8 * q + 1]), pack_f16x2(o[8 * q + 2], o[8 * q + 3]),
+                            pack_f16x2(o[8 * q + 4], o[8 * q + 5]), pack_f16x2(o[8 * q + 6], o[8 * q + 7]));
+                } else {
+                    for (int kk = 0; kk < nsel; ++kk) {
+                        const float wk = lg[kk] * inv_den;
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            p.part + (((row * topk + kk) * NCH + ch) * G + h) * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 u = __ldcg(src + q);
+                            const __half2 *hh = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+                            for (int z = 0; z < 4; ++z) {
+                                const float2 v = __half22float2(hh[z]);
+                                o[8 * q + 2 * z] = fmaf(wk, v.x, o[8 * q + 2 * z]);
+                                o[8 * q + 2 * z + 1] = fmaf(wk, v.y, o[8 * q + 2 * z + 1]);
+                            }
+                        }
+                    }
+                    __nv_bfloat16 *dst = p.O + hrow * D + ch * 32;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
+                            pack_bf16x2(o[8 * q + 0], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                            pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+                }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&ofree[s]);
+            if (!cur.tl.own) {
+                // publish this tile's partials for the window's own tiles
+                __threadfence();
+                named_sync(2, 128);
+                if (leader) atomicAdd(&p.done[cur.tl.win], 1);
+            }
+            cur = nxt;
         }
-        tc::fence_before_sync();
-        if (__syncthreads_or(abort)) break;
     }
 
-    if (abort) {
-        // let copies and MMAs still in flight land before the block exits
-        if (tid == 0) {
-            tc::mbar_wait(&bar[0], ph_load ^ 1u, kWaitBudget);   // the phase that timed out
-            atomicOr(p.status, kFlagTimeout);
-        }
-    }
     __syncthreads();
+    if (*s_abort) {
+        if (tid == 0) atomicOr(p.status, kFlagTimeout);
+        // let copies and MMAs that may still be in flight land before exiting
+        const long long t0 = clock64();
+        while (clock64() - t0 < 20000000) { }
+    }
     tc::fence_after_sync();
-    if (warp == 0) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- host side
@@ -322,60 +528,57 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
            CUDA_SUCCESS;
 }
 
+struct TcLaunch {
+    const void *Q, *K, *V, *lm;
+    int B, H, Hkv, S, topk, own_chunk, lm_bf16;
+    int64_t L, W, cap;
+    float scale;
+    const int32_t *idx, *entries, *wntiles;
+    const int4 *wtiles;
+    int32_t *done;
+    const int64_t *seg_start;
+    float *logits, *w_out;
+    __half *part;
+    void *O;
+    unsigned *status;
+    int num_sms;
+};
+
 template <int D, int G>
-static cudaError_t launch_attend_tc_t(const void *Q, const void *K, const void *V, int B, int H,
-                                      int Hkv, int64_t L, int S, int topk, int own_chunk,
-                                      float scale, const int32_t *idx, const float *w, const int32_t *entries,
-                                      const int4 *tiles, const int32_t *tile_count, int64_t max_tiles,
-                                      __half *part, void *O, unsigned *status, int num_sms,
-                                      cudaStream_t st) {
+static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     using C = TcCfg<D, G>;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, Q, (uint64_t)B * L * H, D, G) ||
-        !make_map(&mk, K, (uint64_t)B * Hkv * L, D, 64) ||
-        !make_map(&mv, V, (uint64_t)B * Hkv * L, D, 64))
+    if (!make_map(&mq, a.Q, (uint64_t)a.B * a.L * a.H, D, G) ||
+        !make_map(&mk, a.K, (uint64_t)a.B * a.Hkv * a.L, D, 64) ||
+        !make_map(&mv, a.V, (uint64_t)a.B * a.Hkv * a.L, D, 64))
         return cudaErrorInvalidValue;
     auto kern = attend_tc_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     TcParams p;
-    p.tiles = tiles; p.tile_count = tile_count; p.entries = entries; p.w = w; p.idx = idx;
-    p.part = part; p.O = (__nv_bfloat16 *)O; p.status = status; p.L = L;
-    p.H = H; p.Hkv = Hkv; p.topk = topk; p.S = S; p.add_own = own_chunk;
-    p.scale_log2e = scale * 1.4426950408889634f;
-    p.n_own_tiles = (int64_t)B * Hkv * ((L + C::EPT - 1) / C::EPT);
-    // retrieved-chunk tiles (tile count known on the device only)
-    p.own_mode = 0;
-    int64_t grid = 2LL * num_sms;
-    if (grid > max_tiles) grid = max_tiles > 0 ? max_tiles : 1;
-    kern<<<(unsigned)grid, 128, C::SMEM, st>>>(mq, mk, mv, p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // own-chunk tiles + fusion of the partials
-    p.own_mode = 1;
-    grid = 2LL * num_sms;
-    if (grid > p.n_own_tiles) grid = p.n_own_tiles;
-    kern<<<(unsigned)grid, 128, C::SMEM, st>>>(mq, mk, mv, p);
+    p.seg_start = a.seg_start; p.wtiles = a.wtiles; p.wntiles = a.wntiles; p.done = a.done;
+    p.entries = a.entries; p.idx = a.idx; p.lm = a.lm; p.logits = a.logits; p.w_out = a.w_out;
+    p.part = a.part; p.O = (__nv_bfloat16 *)a.O; p.status = a.status;
+    p.L = a.L; p.W = a.W; p.nwb = (a.L + a.W - 1) / a.W;
+    p.NW = (int64_t)a.B * a.Hkv * p.nwb; p.cap = a.cap; p.Nc = a.L / a.S;
+    p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
+    p.lm_bf16 = a.lm_bf16;
+    p.scale = a.scale;
+    p.scale_log2e = a.scale * 1.4426950408889634f;
+    kern<<<(unsigned)a.num_sms, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
+
+int64_t attend_tc_max_windows() { return kMaxWindows; }
 
 bool attend_tc_supported(bool bf16, int G, int d) {
     return bf16 && (G == 8 || G == 16) && (d == 64 || d == 128) && encode_fn() != nullptr;
 }
 
-cudaError_t launch_attend_tc(const void *Q, const void *K, const void *V, int B, int H, int Hkv,
-                             int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                             const int32_t *idx, const float *w, const int32_t *entries,
-                             const int4 *tiles, const int32_t *tile_count, int64_t max_tiles,
-                             __half *part, void *O, unsigned *status, int num_sms,
-                             cudaStream_t st) {
-    const int G = H / Hkv;
-#define HSA_TC(DD, GG) \
-    return launch_attend_tc_t<DD, GG>(Q, K, V, B, H, Hkv, L, S, topk, own_chunk, scale, idx, w, entries, tiles, tile_count, max_tiles, part, O, status, num_sms, st)
-    if (d == 128) { if (G == 8) HSA_TC(128, 8); HSA_TC(128, 16); }
-    if (G == 8) HSA_TC(64, 8);
-    HSA_TC(64, 16);
-#undef HSA_TC
+cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st) {
+    const int G = a.H / a.Hkv;
+    if (d == 128) return G == 8 ? launch_attend_tc_t<128, 8>(a, st) : launch_attend_tc_t<128, 16>(a, st);
+    return G == 8 ? launch_attend_tc_t<64, 8>(a, st) : launch_attend_tc_t<64, 16>(a, st);
 }
 
 }  // namespace hsa

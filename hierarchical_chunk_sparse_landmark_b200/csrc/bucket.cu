@@ -1,15 +1,26 @@
-// bucket.cu -- chunk-bucketed work lists for the tensor-core prefill path.
+// bucket.cu -- chunk-bucketed, token-windowed work lists for the tensor-core
+// prefill path.
 //
 // The selection gives every (b, t, g) up to K chunks.  To run the in-chunk
 // attention as dense tensor-core tiles, entries (t, k) are grouped by the
-// chunk they selected: a tile is one chunk's K/V and up to 128/G entries
-// (G query-head rows each) that chose it, so each chunk's K/V is read once per
-// tile instead of once per query.  Three passes over the selection:
-//   count   -- entries per (b, g, chunk)               (shared-memory histogram)
-//   scan    -- bucket offsets, tile descriptors        (one block per (b, g))
-//   scatter -- entry ids into their bucket slots       (atomic cursors)
-// The order of entries inside a bucket is not fixed, which does not change any
-// result: every tile row is computed independently of the other rows.
+// chunk they selected: a tile is one chunk's K/V and up to 128/G entries (G
+// query-head rows each) that chose it, so each chunk's K/V is read once per
+// tile instead of once per query.  Grouping is done per token window (W
+// consecutive tokens of one (b, g)): the per-entry partial outputs of a window
+// are written and then fused while they are still in L2.
+//
+// Passes over the selection (all windows at once):
+//   count   -- entries per (window, chunk)                 (shared-memory histogram)
+//   scan    -- bucket offsets, tile descriptors per window (one block per window)
+//   order   -- start of every segment of the work queue    (one block)
+//   scatter -- entry codes t*32+k into their bucket slots  (atomic cursors)
+// The order of entries inside a bucket is not fixed, which does not change
+// any result: every tile row is computed independently of the other rows.
+//
+// Work queue (consumed by attend_tc.cu): segments
+//   C0, C1, O0, C2, O1, ..., C(n-1), O(n-2), O(n-1)
+// where Cn = retrieved-chunk tiles of window n and On = own-chunk/fusion tiles
+// of window n; On comes one window after Cn so that Cn has finished by then.
 #include "common.cuh"
 
 namespace hsa {
@@ -17,55 +28,71 @@ namespace hsa {
 constexpr int kBucketThreads = 256;
 constexpr int kScanThreads = 1024;
 
-// counts[bg * Nc + i] += #entries of (b, g) that selected chunk i
+struct WinGeom {
+    int64_t L, Nc, W, nwb;     // sequence length, chunks, window tokens, windows per (b, g)
+    int Hkv, topk, ept;
+    int64_t cap;               // tile capacity of one window's list
+};
+
+__device__ __forceinline__ void window_span(const WinGeom &w, int64_t n, int64_t &bg,
+                                            int64_t &t_start, int64_t &t_end) {
+    bg = n / w.nwb;
+    t_start = (n % w.nwb) * w.W;
+    t_end = t_start + w.W < w.L ? t_start + w.W : w.L;
+}
+
+// counts[n * Nc + i] += #entries of window n that selected chunk i
 __global__ void __launch_bounds__(kBucketThreads)
-bucket_count_kernel(const int32_t *__restrict__ idx, int Hkv, int64_t L, int topk, int64_t Nc,
-                    int use_smem, int32_t *__restrict__ counts) {
+bucket_count_kernel(const int32_t *__restrict__ idx, WinGeom wg, int use_smem,
+                    int32_t *__restrict__ counts) {
     extern __shared__ int32_t hist[];
     const int g = blockIdx.y, b = blockIdx.z;
-    const int64_t bg = (int64_t)b * Hkv + g;
+    const int64_t bg = (int64_t)b * wg.Hkv + g;
+    const int64_t t_blk = (int64_t)blockIdx.x * kBucketThreads;    // within one window
+    const int64_t n = bg * wg.nwb + t_blk / wg.W;
     if (use_smem) {
-        for (int64_t i = threadIdx.x; i < Nc; i += blockDim.x) hist[i] = 0;
+        for (int64_t i = threadIdx.x; i < wg.Nc; i += blockDim.x) hist[i] = 0;
         __syncthreads();
     }
-    const int64_t t = (int64_t)blockIdx.x * kBucketThreads + threadIdx.x;
-    if (t < L) {
-        const int32_t *ip = idx + (((int64_t)b * L + t) * Hkv + g) * topk;
-        for (int k = 0; k < topk; ++k) {
+    const int64_t t = t_blk + threadIdx.x;
+    if (t < wg.L) {
+        const int32_t *ip = idx + (((int64_t)b * wg.L + t) * wg.Hkv + g) * wg.topk;
+        for (int k = 0; k < wg.topk; ++k) {
             const int32_t i = ip[k];
             if (i < 0) break;                       // padding only at the end
             if (use_smem) atomicAdd(&hist[i], 1);
-            else atomicAdd(&counts[bg * Nc + i], 1);
+            else atomicAdd(&counts[n * wg.Nc + i], 1);
         }
     }
     if (use_smem) {
         __syncthreads();
-        for (int64_t i = threadIdx.x; i < Nc; i += blockDim.x)
-            if (hist[i]) atomicAdd(&counts[bg * Nc + i], hist[i]);
+        for (int64_t i = threadIdx.x; i < wg.Nc; i += blockDim.x)
+            if (hist[i]) atomicAdd(&counts[n * wg.Nc + i], hist[i]);
     }
 }
 
-// One block per (b, g): exclusive scan of the counts -> absolute bucket
-// offsets (cursor), tile descriptors appended at atomicAdd(tile_count).
-// tiles[j] = {bg, chunk, first entry, n entries}
+// One block per window: cursor = absolute entry offset of each bucket, tile
+// descriptors {bg, chunk, first entry, n entries} at wtiles[n * cap ...],
+// wntiles[n] = number of tiles, done[n] = 0.
 __global__ void __launch_bounds__(kScanThreads)
-bucket_scan_kernel(const int32_t *__restrict__ counts, int Hkv, int64_t L, int topk, int64_t Nc,
-                   int ept, int32_t *__restrict__ cursor, int4 *__restrict__ tiles,
-                   int32_t *__restrict__ tile_count) {
+bucket_scan_kernel(const int32_t *__restrict__ counts, WinGeom wg, int32_t *__restrict__ cursor,
+                   int4 *__restrict__ wtiles, int32_t *__restrict__ wntiles,
+                   int32_t *__restrict__ done) {
     __shared__ int64_t warp_e[32], warp_t[32];
-    __shared__ int64_t s_tile_base;
-    const int g = blockIdx.x, b = blockIdx.y;
-    const int64_t bg = (int64_t)b * Hkv + g;
+    const int64_t n = blockIdx.x;
+    int64_t bg, t_start, t_end;
+    window_span(wg, n, bg, t_start, t_end);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t Nc = wg.Nc;
     const int64_t per = (Nc + kScanThreads - 1) / kScanThreads;
     const int64_t i0 = tid * per, i1 = (i0 + per < Nc) ? i0 + per : Nc;
+    const int32_t *cn = counts + n * Nc;
     int64_t e_sum = 0, t_sum = 0;
     for (int64_t i = i0; i < i1; ++i) {
-        const int64_t c = counts[bg * Nc + i];
+        const int64_t c = cn[i];
         e_sum += c;
-        t_sum += (c + ept - 1) / ept;
+        t_sum += (c + wg.ept - 1) / wg.ept;
     }
-    // block exclusive scan of (e_sum, t_sum)
     int64_t e_inc = e_sum, t_inc = t_sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -85,56 +112,116 @@ bucket_scan_kernel(const int32_t *__restrict__ counts, int Hkv, int64_t L, int t
         }
         warp_e[lane] = a;
         warp_t[lane] = c;
-        if (lane == 31) s_tile_base = atomicAdd(tile_count, (int32_t)c);
+        if (lane == 31) {
+            wntiles[n] = (int32_t)c;
+            done[n] = 0;
+        }
     }
     __syncthreads();
     int64_t e_off = e_inc - e_sum + (warp ? warp_e[warp - 1] : 0);
-    int64_t t_off = t_inc - t_sum + (warp ? warp_t[warp - 1] : 0) + s_tile_base;
-    const int64_t base = bg * L * topk;
+    int64_t t_off = t_inc - t_sum + (warp ? warp_t[warp - 1] : 0);
+    const int64_t base = bg * wg.L * wg.topk + t_start * wg.topk;     // window's entry region
+    int4 *tl = wtiles + n * wg.cap;
     for (int64_t i = i0; i < i1; ++i) {
-        const int64_t c = counts[bg * Nc + i];
-        cursor[bg * Nc + i] = (int32_t)(base + e_off);
-        for (int64_t s = 0; s < c; s += ept) {
-            const int64_t n = c - s < ept ? c - s : ept;
-            tiles[t_off++] = make_int4((int)bg, (int)i, (int)(base + e_off + s), (int)n);
+        const int64_t c = cn[i];
+        cursor[n * Nc + i] = (int32_t)(base + e_off);
+        for (int64_t s = 0; s < c; s += wg.ept) {
+            const int64_t m = c - s < wg.ept ? c - s : wg.ept;
+            tl[t_off++] = make_int4((int)bg, (int)i, (int)(base + e_off + s), (int)m);
         }
         e_off += c;
     }
 }
 
-// entries[cursor[bg, i]++] = t * 32 + k
+// One block: seg_start[s] for the 2*NW queue segments (see the file comment).
+__global__ void __launch_bounds__(kScanThreads)
+queue_order_kernel(const int32_t *__restrict__ wntiles, WinGeom wg, int64_t NW,
+                   int64_t *__restrict__ seg_start) {
+    __shared__ int64_t warp_s[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t nseg = 2 * NW;
+    const int64_t per = (nseg + kScanThreads - 1) / kScanThreads;
+    const int64_t s0 = tid * per, s1 = (s0 + per < nseg) ? s0 + per : nseg;
+    auto seg_len = [&](int64_t s) -> int64_t {
+        int64_t type_own, n;
+        if (s == 0) { type_own = 0; n = 0; }
+        else if (s == nseg - 1) { type_own = 1; n = NW - 1; }
+        else if (s & 1) { type_own = 0; n = (s + 1) / 2; }
+        else { type_own = 1; n = s / 2 - 1; }
+        if (!type_own) return wntiles[n];
+        int64_t bg, ts, te;
+        window_span(wg, n, bg, ts, te);
+        return (te - ts + wg.ept - 1) / wg.ept;
+    };
+    int64_t sum = 0;
+    for (int64_t s = s0; s < s1; ++s) sum += seg_len(s);
+    int64_t inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t a = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += a;
+    }
+    if (lane == 31) warp_s[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int64_t a = warp_s[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t x = __shfl_up_sync(0xffffffffu, a, o);
+            if (lane >= o) a += x;
+        }
+        warp_s[lane] = a;
+    }
+    __syncthreads();
+    int64_t off = inc - sum + (warp ? warp_s[warp - 1] : 0);
+    for (int64_t s = s0; s < s1; ++s) {
+        seg_start[s] = off;
+        off += seg_len(s);
+    }
+    if (s1 == nseg && s0 < s1) seg_start[nseg] = off;
+    if (nseg == 0 && tid == 0) seg_start[0] = 0;
+}
+
+// entries[cursor[n, i]++] = t * 32 + k
 __global__ void __launch_bounds__(kBucketThreads)
-bucket_scatter_kernel(const int32_t *__restrict__ idx, int Hkv, int64_t L, int topk, int64_t Nc,
-                      int32_t *__restrict__ cursor, int32_t *__restrict__ entries) {
+bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int32_t *__restrict__ cursor,
+                      int32_t *__restrict__ entries) {
     const int g = blockIdx.y, b = blockIdx.z;
-    const int64_t bg = (int64_t)b * Hkv + g;
+    const int64_t bg = (int64_t)b * wg.Hkv + g;
     const int64_t t = (int64_t)blockIdx.x * kBucketThreads + threadIdx.x;
-    if (t >= L) return;
-    const int32_t *ip = idx + (((int64_t)b * L + t) * Hkv + g) * topk;
-    for (int k = 0; k < topk; ++k) {
+    if (t >= wg.L) return;
+    const int64_t n = bg * wg.nwb + t / wg.W;
+    const int32_t *ip = idx + (((int64_t)b * wg.L + t) * wg.Hkv + g) * wg.topk;
+    for (int k = 0; k < wg.topk; ++k) {
         const int32_t i = ip[k];
         if (i < 0) break;
-        const int32_t p = atomicAdd(&cursor[bg * Nc + i], 1);
+        const int32_t p = atomicAdd(&cursor[n * wg.Nc + i], 1);
         entries[p] = (int32_t)(t * 32 + k);
     }
 }
 
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
-                          int ept, int32_t *counts, int32_t *cursor, int32_t *entries,
-                          int4 *tiles, int32_t *tile_count, cudaStream_t st) {
+                          int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
+                          int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
+                          int64_t *seg_start, cudaStream_t st) {
+    WinGeom wg;
+    wg.L = L; wg.Nc = Nc; wg.W = W; wg.nwb = (L + W - 1) / W;
+    wg.Hkv = Hkv; wg.topk = topk; wg.ept = ept; wg.cap = cap;
+    const int64_t NW = (int64_t)B * Hkv * wg.nwb;
     dim3 grid((unsigned)((L + kBucketThreads - 1) / kBucketThreads), (unsigned)Hkv, (unsigned)B);
     const int use_smem = Nc <= 8192 ? 1 : 0;
-    const size_t smem = use_smem ? sizeof(int32_t) * (size_t)Nc : 0;
-    bucket_count_kernel<<<grid, kBucketThreads, smem, st>>>(idx, Hkv, L, topk, Nc, use_smem,
-                                                            counts);
+    const size_t smem = use_smem ? sizeof(int32_t) * (size_t)(Nc > 0 ? Nc : 1) : 0;
+    bucket_count_kernel<<<grid, kBucketThreads, smem, st>>>(idx, wg, use_smem, counts);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bucket_scan_kernel<<<dim3((unsigned)Hkv, (unsigned)B), kScanThreads, 0, st>>>(
-        counts, Hkv, L, topk, Nc, ept, cursor, tiles, tile_count);
+    bucket_scan_kernel<<<(unsigned)NW, kScanThreads, 0, st>>>(counts, wg, cursor, wtiles, wntiles,
+                                                            done);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bucket_scatter_kernel<<<grid, kBucketThreads, 0, st>>>(idx, Hkv, L, topk, Nc, cursor,
-                                                           entries);
+    queue_order_kernel<<<1, kScanThreads, 0, st>>>(wntiles, wg, NW, seg_start);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bucket_scatter_kernel<<<grid, kBucketThreads, 0, st>>>(idx, wg, cursor, entries);
     return cudaGetLastError();
 }
 

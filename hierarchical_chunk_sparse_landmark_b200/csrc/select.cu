@@ -2,8 +2,10 @@
 //
 // For each (b, t, g): group query qbar = mean of the G heads' queries, group
 // scores sbar_i = scale * qbar . l_i over the visible chunks i < floor(t/S),
-// the top-K chunks by (score desc, index asc), then per head the fusion
-// weights w = softmax over the selected chunks of scale * q_h . l_i.
+// the top-K chunks by (score desc, index asc), then (when w_out is given) per
+// head the fusion weights w = softmax over the selected chunks of
+// scale * q_h . l_i.  The tensor-core attention path computes those logits
+// itself, inside its S = Q K^T tiles, and passes w_out = NULL here.
 // (Per-token top-K retrieval over chunk landmarks: Understanding and Improving
 // Length Generalization in Hierarchical Sparse Attention Models, "Methodology
 // in Plain English"; fusion by retrieval scores: HiLS Attention abstract.)
@@ -128,31 +130,45 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
         }
     }
 
-    // outputs: idx (lane k = rank k) and per-head fusion weights
-#pragma unroll
+    // outputs: idx (lane k = rank k) and per-head fusion weights.  For the
+    // logits the warp is split into KP slots (KP = topk rounded up to a power
+    // of two) of PARTS = 32/KP lanes; the lanes of slot k split d and reduce
+    // with PARTS-wide shuffles, so all slots of a head are computed at once.
+    int KP = 1;
+    while (KP < topk) KP <<= 1;
+    const int PARTS = 32 / KP;
+    const int slot = lane / PARTS, part = lane % PARTS;
+    const int span = D / PARTS;                       // d elements per lane
+#pragma unroll 1
     for (int u = 0; u < kSelTokPerWarp; ++u) {
         const int64_t t = t0 + warp * kSelTokPerWarp + u;
         if (t >= L) continue;
         const int32_t sel = lane < topk ? key_index(v[u]) : -1;
         if (lane < topk && idx_out) idx_out[((b * L + t) * Hkv + g) * topk + lane] = sel;
+        if (w_out == nullptr) continue;     // weights computed downstream (tensor-core path)
+        const int32_t my_sel = __shfl_sync(0xffffffffu, sel, slot < 32 ? slot : 0);
+        const bool active = slot < topk && my_sel >= 0;
+        const TL *lp = lm_bg + (int64_t)(my_sel > 0 ? my_sel : 0) * D + part * span;
+#pragma unroll 1
         for (int h = 0; h < G; ++h) {
             const int hh = g * G + h;
-            const T *qh = Q + ((b * L + t) * H + hh) * (int64_t)D;
-            float s = -INFINITY;
-            if (sel >= 0) {
-                const TL *lp = lm_bg + (int64_t)sel * D;
-                float a = 0.f;
-                for (int j = 0; j < D; ++j) a = fmaf(to_f32(qh[j]), to_f32(lp[j]), a);
-                s = scale * a;
+            const T *qh = Q + ((b * L + t) * H + hh) * (int64_t)D + part * span;
+            float a = 0.f;
+            if (active) {
+#pragma unroll 4
+                for (int e = 0; e < span; ++e) a = fmaf(to_f32(qh[e]), to_f32(lp[e]), a);
             }
+            for (int o = PARTS / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            const float s = active ? scale * a : -INFINITY;
             float mx = s;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float e = sel >= 0 ? expf(s - mx) : 0.f;
+            const float e = (active && part == 0) ? expf(s - mx) : 0.f;
             float den = e;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-            if (lane < topk) w_out[((b * L + t) * H + hh) * topk + lane] = den > 0.f ? e / den : 0.f;
+            if (part == 0 && slot < topk)
+                w_out[((b * L + t) * H + hh) * topk + slot] = (active && den > 0.f) ? e / den : 0.f;
         }
     }
 }
