@@ -31,7 +31,9 @@
 //   warps 6-9   epilogue  (TMEM -> fp16 partials, or -> fused bf16 O)
 // Consumer roles prefetch the next tile's metadata while working on the
 // current one.  Own tiles of window n wait, in the epilogue only, until every
-// retrieved-chunk tile of window n has published its partials.  Every wait is
+// retrieved-chunk tile of window n has published its logits and partials; a
+// block publishes once per window (one fence per role when it moves past its
+// last tile of that window), not once per tile.  Every wait is
 // bounded; on expiry the block sets the status flag in the workspace, lets
 // in-flight copies land, frees its TMEM and exits.
 #include <cuda.h>
@@ -63,6 +65,7 @@ struct TcCfg {
 
 struct TcParams {
     const int64_t *seg_start;     // [2 * NW + 1]
+    const void *Q;                // [B, L, H, D] bf16 (rows gathered with cp.async)
     const int4 *wtiles;           // [NW * cap] retrieved-chunk tiles per window
     const int32_t *wntiles;       // [NW]
     int32_t *done;                // [NW] published retrieved-chunk tiles
@@ -76,11 +79,13 @@ struct TcParams {
     unsigned *status;
     int64_t L, W, nwb, NW, cap, Nc;
     int H, Hkv, topk, S, add_own, lm_bf16;
+    int q3d;                      // Q map is the 3-D (cols, rows, d-half) view
     float scale, scale_log2e;
 };
 
 constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;                       // 11 warps
+constexpr int kGatherWarp = 10;
 constexpr int kMaxWindows = 2048;                  // shared segment table size / 2
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -98,6 +103,14 @@ __device__ __forceinline__ int ld_acquire(const int32_t *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Make this role's global stores of a window visible, then count its tiles
+// of that window (128 threads of one role; `id` is the role's named barrier).
+__device__ __forceinline__ void publish(int32_t *counter, int n, int id, bool leader) {
+    __threadfence();
+    named_sync(id, 128);
+    if (leader) atomicAdd(counter, n);
 }
 
 // Bounded mbarrier wait that also gives up when another role aborted.
@@ -146,6 +159,16 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int64_t *se
     }
 }
 
+// Tile metadata the producer publishes to the softmax and epilogue roles
+// through a small shared-memory ring (so only the producer walks the global
+// work lists).  code[e] = t * 32 + k of entry e (own tiles: t * 32).
+constexpr int kRing = 4;
+struct TileInfo {
+    int64_t bg, win;
+    int chunk, n, own, pad;
+    int32_t code[16];
+};
+
 // Per-row view of a tile for the softmax and epilogue threads.
 struct RowJob {
     Tile tl;
@@ -154,21 +177,14 @@ struct RowJob {
     bool valid;
 };
 
-__device__ __forceinline__ RowJob fetch_row(const TcParams &p, const int64_t *seg, int nseg,
-                                            int64_t pos, int ept, int e) {
+__device__ __forceinline__ RowJob read_row(const TileInfo &ti, int e) {
     RowJob rj;
-    decode_tile(p, seg, nseg, pos, ept, rj.tl);
-    rj.valid = e < rj.tl.n;
-    rj.t = 0;
-    rj.k = 0;
-    if (rj.valid) {
-        if (rj.tl.own) rj.t = rj.tl.t0 + e;
-        else {
-            const int32_t code = p.entries[rj.tl.first + e];
-            rj.t = code >> 5;
-            rj.k = code & 31;
-        }
-    }
+    rj.tl.bg = ti.bg; rj.tl.win = ti.win; rj.tl.chunk = ti.chunk; rj.tl.n = ti.n;
+    rj.tl.own = ti.own; rj.tl.first = 0; rj.tl.t0 = 0;
+    rj.valid = e < ti.n;
+    const int32_t code = rj.valid ? ti.code[e] : 0;
+    rj.t = code >> 5;
+    rj.k = code & 31;
     return rj;
 }
 
@@ -187,9 +203,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     uint64_t *bars = (uint64_t *)(smem + 2 * C::STAGE);
     uint64_t *full = bars, *empty = bars + 2, *sfull = bars + 4, *sfree = bars + 6;
     uint64_t *pfull = bars + 8, *ofull = bars + 10, *ofree = bars + 12;
-    uint32_t *s_tmem = (uint32_t *)(bars + 14);
+    uint64_t *ifull = bars + 14, *ifree = bars + 14 + kRing;
+    uint32_t *s_tmem = (uint32_t *)(bars + 14 + 2 * kRing);
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
     __shared__ int64_t seg[2 * kMaxWindows + 1];
+    __shared__ TileInfo ring[kRing];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nseg = (int)(2 * p.NW);
@@ -200,13 +218,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&full[s], 2);        // K/V producer + Q gather warp
             tc::mbar_init(&empty[s], 1);
             tc::mbar_init(&sfull[s], 1);
             tc::mbar_init(&sfree[s], 128);
             tc::mbar_init(&pfull[s], 128);
             tc::mbar_init(&ofull[s], 1);
             tc::mbar_init(&ofree[s], 128);
+        }
+        for (int i = 0; i < kRing; ++i) {
+            tc::mbar_init(&ifull[i], 1);
+            tc::mbar_init(&ifree[i], 257);     // softmax + epilogue threads + gather warp
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -223,35 +245,63 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        for (int64_t j = 0; j < my_tiles; ++j) {
-            const int64_t pos = blockIdx.x + j * gridDim.x;
-            Tile tl;
-            decode_tile(p, seg, nseg, pos, EPT, tl);
-            const int s = (int)(j & 1);
-            int ok = 1;
-            if (lane == 0 && j >= 2) ok = wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const int64_t b = tl.bg / Hkv;
-            const int g = (int)(tl.bg % Hkv);
-            int64_t tq = 0;
-            if (lane < tl.n) tq = tl.own ? tl.t0 + lane : (int64_t)(p.entries[tl.first + lane] >> 5);
+        // Software-pipelined two tiles deep: in iteration j the descriptor of
+        // tile j+2 and the entry codes / landmark row of tile j+1 are loaded
+        // while tile j is published and its copies are issued.
+        auto load_rows = [&](const Tile &tl, int32_t &code, float (&x)[8]) {
+            code = 0;
+            if (lane < tl.n)
+                code = tl.own ? (int32_t)((tl.t0 + lane) * 32) : p.entries[tl.first + lane];
             if (!tl.own && lane < D / 8) {
-                // landmark row of the chunk -> rows 64 (bf16 high part) and 65 (low part)
-                float x[8];
                 const int64_t li = (tl.bg * p.Nc + tl.chunk) * D + lane * 8;
                 if (p.lm_bf16) {
-                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(
-                        (const __nv_bfloat16 *)p.lm + li), x);
+                    Vec16<__nv_bfloat16>::unpack(
+                        *reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.lm + li), x);
                 } else {
                     const uint4 *src = reinterpret_cast<const uint4 *>((const float *)p.lm + li);
                     Vec16<float>::unpack(src[0], x);
                     Vec16<float>::unpack(src[1], x + 4);
                 }
+            }
+        };
+        Tile d0, d1;
+        int32_t c0 = 0;
+        float x0[8];
+        if (my_tiles > 0) decode_tile(p, seg, nseg, blockIdx.x, EPT, d0);
+        if (my_tiles > 1) decode_tile(p, seg, nseg, blockIdx.x + gridDim.x, EPT, d1);
+        if (my_tiles > 0) load_rows(d0, c0, x0);
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            Tile d2;
+            if (j + 2 < my_tiles) decode_tile(p, seg, nseg, blockIdx.x + (j + 2) * gridDim.x, EPT, d2);
+            int32_t c1 = 0;
+            float x1[8];
+            if (j + 1 < my_tiles) load_rows(d1, c1, x1);
+
+            // publish the tile's metadata
+            const int ri = (int)(j & (kRing - 1));
+            int ok = 1;
+            if (lane == 0 && j >= kRing)
+                ok = wait_bar(&ifree[ri], (uint32_t)(((j / kRing) + 1) & 1), s_abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane < 16) ring[ri].code[lane] = c0;
+            if (lane == 0) {
+                ring[ri].bg = d0.bg; ring[ri].win = d0.win; ring[ri].chunk = d0.chunk;
+                ring[ri].n = d0.n; ring[ri].own = d0.own;
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&ifull[ri]);
+
+            // stage the tile's operands
+            const int s = (int)(j & 1);
+            if (lane == 0 && j >= 2) ok = wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (!d0.own && lane < D / 8) {
+                // landmark row of the chunk -> key rows 64 (bf16 high part), 65 (low part)
                 float hi[8], lo[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    hi[q] = __bfloat162float(__float2bfloat16_rn(x[q]));
-                    lo[q] = x[q] - hi[q];
+                    hi[q] = __bfloat162float(__float2bfloat16_rn(x0[q]));
+                    lo[q] = x0[q] - hi[q];
                 }
                 const int kb = (lane * 8) / 64, c = ((lane * 8) % 64) / 8;
                 uint8_t *blk = sK(s) + kb * C::KBLK;
@@ -265,21 +315,53 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             __syncwarp();
             if (lane == 0) {
-                tc::mbar_expect_tx(&full[s], (uint32_t)(2 * C::V_BYTES + tl.n * G * D * 2));
-                const int krow = (int)(tl.bg * L + (int64_t)tl.chunk * S);
+                // K and V of the chunk by TMA (the Q rows come from the gather warp)
+                tc::mbar_expect_tx(&full[s], (uint32_t)(2 * C::V_BYTES));
+                const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb) {
                     tc::tma_load_2d(sK(s) + kb * C::KBLK, &tmK, &full[s], kb * 64, krow);
                     tc::tma_load_2d(sV(s) + kb * 8192, &tmV, &full[s], kb * 64, krow);
                 }
             }
-            __syncwarp();
-            if (lane < tl.n) {
-                const int qrow = (int)((b * L + tq) * H + (int64_t)g * G);
+            d0 = d1;
+            d1 = d2;
+            c0 = c1;
 #pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tc::tma_load_2d(sQ(s) + kb * (128 * 128) + lane * G * 128, &tmQ, &full[s],
-                                    kb * 64, qrow);
+            for (int q = 0; q < 8; ++q) x0[q] = x1[q];
+        }
+    } else if (warp == kGatherWarp) {
+        // ------------------------------------------------------------ Q gather
+        // One TMA box per entry: all G query-head rows of the entry (both
+        // 64-wide halves of d in one box when the 3-D view is available).
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            const int ri = (int)(j & (kRing - 1));
+            const int s = (int)(j & 1);
+            int ok = 1;
+            if (lane == 0) {
+                ok = wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort);
+                if (ok && j >= 2) ok = wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort);
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const TileInfo &ti = ring[ri];
+            const int n = ti.n;
+            const int64_t b = ti.bg / Hkv;
+            const int g = (int)(ti.bg % Hkv);
+            const int32_t code = lane < n ? ti.code[lane] : 0;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&ifree[ri]);
+            if (lane == 0) tc::mbar_expect_tx(&full[s], (uint32_t)(n * G * D * 2));
+            __syncwarp();
+            if (lane < n) {
+                const int qrow = (int)((b * L + (int64_t)(code >> 5)) * H + (int64_t)g * G);
+                if (p.q3d) {
+                    tc::tma_load_3d(sQ(s) + lane * (C::KB * G * 128), &tmQ, &full[s], 0, qrow, 0);
+                } else {
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tc::tma_load_2d(sQ(s) + kb * (128 * 128) + lane * G * 128, &tmQ, &full[s],
+                                        kb * 64, qrow);
+                }
             }
         }
     } else if (warp == 1) {
@@ -313,7 +395,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 for (int kb = 0; kb < C::KB; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sQ(s) + kb * 16384 + kk * 32), 16, 1024);
+                        const uint64_t ad = p.q3d
+                            ? tc::sdesc_sw128(tc::smem_u32(sQ(s) + kb * (G * 128) + kk * 32), 16, C::KB * G * 128)
+                            : tc::sdesc_sw128(tc::smem_u32(sQ(s) + kb * 16384 + kk * 32), 16, 1024);
                         const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sK(s) + kb * C::KBLK + kk * 32), 16, 1024);
                         tc::mma_bf16(tmem + s * C::S_COL, ad, bd, IDESC_S, (kb | kk) ? 1u : 0u);
                     }
@@ -328,14 +412,23 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int r = q4 * 32 + lane;             // tile row
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
-        RowJob cur;
-        if (my_tiles > 0) cur = fetch_row(p, seg, nseg, blockIdx.x, EPT, e);
+        const bool leader = (warp == 2 && lane == 0);
+        int64_t pub_win = -1;
+        int pub_cnt = 0;
         for (int64_t j = 0; j < my_tiles; ++j) {
-            RowJob nxt;
-            if (j + 1 < my_tiles) nxt = fetch_row(p, seg, nseg, blockIdx.x + (j + 1) * gridDim.x, EPT, e);
+            const int ri = (int)(j & (kRing - 1));
+            if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
+            const RowJob cur = read_row(ring[ri], e);
+            tc::mbar_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
             const int64_t b = cur.tl.bg / Hkv;
             const int g = (int)(cur.tl.bg % Hkv);
+            if (cur.tl.own || cur.tl.win != pub_win) {
+                // leaving window pub_win: its logits from this block are published
+                if (pub_cnt) publish(p.done + pub_win, pub_cnt, 3, leader);
+                pub_win = cur.tl.own ? -1 : cur.tl.win;
+                pub_cnt = 0;
+            }
             if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
             float s0[32], s1[32], l_hi, l_lo;
@@ -377,10 +470,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 *reinterpret_cast<uint4 *>(prow + tc::sw128_offset(r, c)) = u;
             }
             tc::fence_proxy_async_smem();
-            if (!cur.tl.own) __threadfence();        // logit visible before the tile is published
             tc::mbar_arrive(&pfull[s]);
-            cur = nxt;
+            if (!cur.tl.own) ++pub_cnt;
         }
+        if (pub_cnt && !*s_abort) publish(p.done + pub_win, pub_cnt, 3, leader);
     } else {
         // ------------------------------------------------------------ epilogue
         const int q4 = warp & 3;
@@ -389,12 +482,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int e = r / G, h = r % G;
         const bool leader = (warp == 6 && lane == 0);
         constexpr int NCH = D / 32;               // 32-column chunks of a row
-        RowJob cur;
-        if (my_tiles > 0) cur = fetch_row(p, seg, nseg, blockIdx.x, EPT, e);
+        int64_t pub_win = -1;
+        int pub_cnt = 0;
         for (int64_t j = 0; j < my_tiles; ++j) {
-            RowJob nxt;
-            if (j + 1 < my_tiles) nxt = fetch_row(p, seg, nseg, blockIdx.x + (j + 1) * gridDim.x, EPT, e);
+            const int ri = (int)(j & (kRing - 1));
+            if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
+            const RowJob cur = read_row(ring[ri], e);
+            tc::mbar_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
+            if (cur.tl.own || cur.tl.win != pub_win) {
+                // leaving window pub_win: its partials from this block are published
+                if (pub_cnt) publish(p.done + pub_win, pub_cnt, 2, leader);
+                pub_win = cur.tl.own ? -1 : cur.tl.win;
+                pub_cnt = 0;
+            }
             const int64_t b = cur.tl.bg / Hkv;
             const int g = (int)(cur.tl.bg % Hkv);
             const int64_t row = (b * L + cur.t) * Hkv + g;       // (t, g) selection row
@@ -405,7 +506,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (cur.tl.own) {
                 // the window's retrieved-chunk partials must all be published
                 if (leader) {
-                    const int32_t need = p.wntiles[cur.tl.win];
+                    // both roles (softmax: logits, epilogue: partials) count every tile
+                    const int32_t need = 2 * p.wntiles[cur.tl.win];
                     const long long t0c = clock64();
                     while (ld_acquire(&p.done[cur.tl.win]) < need) {
                         if (*s_abort || clock64() - t0c > kWaitBudget) { *s_abort = 1; break; }
@@ -415,31 +517,27 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 named_sync(1, 128);
                 if (*s_abort) break;
                 if (cur.valid) {
+                    // selected slots come first; load the row's indices and logits at once
                     const int32_t *ip = p.idx + row * topk;
-                    for (int kk = 0; kk < topk && ip[kk] >= 0; ++kk) {
-                        lg[kk] = __ldcg(p.logits + hrow * topk + kk);
-                        m = fmaxf(m, lg[kk]);
-                        ++nsel;
-                    }
+                    for (int kk = 0; kk < topk; ++kk) nsel += ip[kk] >= 0 ? 1 : 0;
+                    for (int kk = 0; kk < nsel; ++kk) lg[kk] = __ldcg(p.logits + hrow * topk + kk);
+                    for (int kk = 0; kk < nsel; ++kk) m = fmaxf(m, lg[kk]);
                     float den = 0.f;
                     for (int kk = 0; kk < nsel; ++kk) {
                         lg[kk] = __expf(lg[kk] - m);
                         den += lg[kk];
                     }
                     inv_den = nsel ? 1.f / den : 0.f;
+                    for (int kk = 0; kk < nsel; ++kk) lg[kk] *= inv_den;    // fusion weights
                     if (p.w_out)
                         for (int kk = 0; kk < topk; ++kk)
-                            p.w_out[hrow * topk + kk] = kk < nsel ? lg[kk] * inv_den : 0.f;
+                            p.w_out[hrow * topk + kk] = kk < nsel ? lg[kk] : 0.f;
                 }
             }
             if (!wait_bar(&ofull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
-#pragma unroll 1
-            for (int ch = 0; ch < NCH; ++ch) {
-                float o[32];
-                tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o);
-                tc::tmem_wait_ld();
-                if (!cur.valid) continue;
+            // O chunk ch (32 columns) of this row -> partial slot or fused output
+            auto emit = [&](int ch, float (&o)[32]) {
                 if (!cur.tl.own) {
                     // partial layout [entry][d/32][head][32] (fp16)
                     __half *dst = p.part + (((row * topk + cur.k) * NCH + ch) * G + h) * 32;
@@ -449,21 +547,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             pack_f16x2(o[8 * q + 0], o[8 * q + 1]), pack_f16x2(o[8 * q + 2], o[8 * q + 3]),
                             pack_f16x2(o[8 * q + 4], o[8 * q + 5]), pack_f16x2(o[8 * q + 6], o[8 * q + 7]));
                 } else {
-                    for (int kk = 0; kk < nsel; ++kk) {
-                        const float wk = lg[kk] * inv_den;
-                        const uint4 *src = reinterpret_cast<const uint4 *>(
-                            p.part + (((row * topk + kk) * NCH + ch) * G + h) * 32);
+                    // fusion: O += sum_k w_k * partial_k, four slots' loads in flight at a time
+                    for (int k0 = 0; k0 < nsel; k0 += 4) {
+                        uint4 u[4][4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 u = __ldcg(src + q);
-                            const __half2 *hh = reinterpret_cast<const __half2 *>(&u);
+                        for (int a = 0; a < 4; ++a)
+                            if (k0 + a < nsel) {
+                                const uint4 *src = reinterpret_cast<const uint4 *>(
+                                    p.part + (((row * topk + k0 + a) * NCH + ch) * G + h) * 32);
 #pragma unroll
-                            for (int z = 0; z < 4; ++z) {
-                                const float2 v = __half22float2(hh[z]);
-                                o[8 * q + 2 * z] = fmaf(wk, v.x, o[8 * q + 2 * z]);
-                                o[8 * q + 2 * z + 1] = fmaf(wk, v.y, o[8 * q + 2 * z + 1]);
+                                for (int q = 0; q < 4; ++q) u[a][q] = __ldcg(src + q);
                             }
-                        }
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            if (k0 + a < nsel) {
+                                const float wk = lg[k0 + a];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const __half2 *hh = reinterpret_cast<const __half2 *>(&u[a][q]);
+#pragma unroll
+                                    for (int z = 0; z < 4; ++z) {
+                                        const float2 v = __half22float2(hh[z]);
+                                        o[8 * q + 2 * z] = fmaf(wk, v.x, o[8 * q + 2 * z]);
+                                        o[8 * q + 2 * z + 1] = fmaf(wk, v.y, o[8 * q + 2 * z + 1]);
+                                    }
+                                }
+                            }
                     }
                     __nv_bfloat16 *dst = p.O + hrow * D + ch * 32;
 #pragma unroll
@@ -472,17 +581,34 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             pack_bf16x2(o[8 * q + 0], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
                             pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
                 }
+            };
+            if (!cur.tl.own) {
+#pragma unroll 1
+                for (int ch = 0; ch < NCH; ch += 2) {
+                    float o0[32], o1[32];
+                    // two 32-column TMEM loads per wait
+                    tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o0);
+                    tc::tmem_ld32(tmem + C::O_COL + s * D + (ch + 1) * 32 + lane_off, o1);
+                    tc::tmem_wait_ld();
+                    if (!cur.valid) continue;
+                    emit(ch, o0);
+                    emit(ch + 1, o1);
+                }
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < NCH; ++ch) {
+                    float o0[32];
+                    tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o0);
+                    tc::tmem_wait_ld();
+                    if (!cur.valid) continue;
+                    emit(ch, o0);
+                }
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&ofree[s]);
-            if (!cur.tl.own) {
-                // publish this tile's partials for the window's own tiles
-                __threadfence();
-                named_sync(2, 128);
-                if (leader) atomicAdd(&p.done[cur.tl.win], 1);
-            }
-            cur = nxt;
+            if (!cur.tl.own) ++pub_cnt;
         }
+        if (pub_cnt && !*s_abort) publish(p.done + pub_win, pub_cnt, 2, leader);
     }
 
     __syncthreads();
@@ -528,6 +654,22 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
            CUDA_SUCCESS;
 }
 
+// 3-D bf16 view of [rows, D] (D = 128) as (64 columns, rows, 2 halves of d),
+// strides 2*D and 128 bytes: one box (64, G, 2) brings all of an entry's G
+// rows, both halves, as two 128B-swizzled [G x 128 B] blocks.
+static bool make_map_q3d(CUtensorMap *m, const void *base, uint64_t rows, int D, int G) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(D / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, 128u};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)(D / 64)};
+    const cuuint32_t es[3] = {1u, 1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 struct TcLaunch {
     const void *Q, *K, *V, *lm;
     int B, H, Hkv, S, topk, own_chunk, lm_bf16;
@@ -548,14 +690,19 @@ template <int D, int G>
 static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     using C = TcCfg<D, G>;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.Q, (uint64_t)a.B * a.L * a.H, D, G) ||
-        !make_map(&mk, a.K, (uint64_t)a.B * a.Hkv * a.L, D, 64) ||
+    // the single-box entry layout has a uniform 8-row atom stride only when an
+    // entry is exactly one atom (G = 8) and d has two halves
+    bool q3d = (G == 8 && D == 128) &&
+               make_map_q3d(&mq, a.Q, (uint64_t)a.B * a.L * a.H, D, G);
+    if (!q3d && !make_map(&mq, a.Q, (uint64_t)a.B * a.L * a.H, D, G)) return cudaErrorInvalidValue;
+    if (!make_map(&mk, a.K, (uint64_t)a.B * a.Hkv * a.L, D, 64) ||
         !make_map(&mv, a.V, (uint64_t)a.B * a.Hkv * a.L, D, 64))
         return cudaErrorInvalidValue;
     auto kern = attend_tc_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     TcParams p;
+    p.Q = a.Q;
     p.seg_start = a.seg_start; p.wtiles = a.wtiles; p.wntiles = a.wntiles; p.done = a.done;
     p.entries = a.entries; p.idx = a.idx; p.lm = a.lm; p.logits = a.logits; p.w_out = a.w_out;
     p.part = a.part; p.O = (__nv_bfloat16 *)a.O; p.status = a.status;
@@ -563,6 +710,7 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     p.NW = (int64_t)a.B * a.Hkv * p.nwb; p.cap = a.cap; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
     p.lm_bf16 = a.lm_bf16;
+    p.q3d = q3d ? 1 : 0;
     p.scale = a.scale;
     p.scale_log2e = a.scale * 1.4426950408889634f;
     kern<<<(unsigned)a.num_sms, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
