@@ -369,10 +369,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (lane == 0) {
             constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, C::NS, false);
             constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
-            auto issue_pv = [&](int64_t i) -> bool {
+            auto issue_pv = [&](int64_t i) {
                 const int s = (int)(i & 1);
-                if (!wait_bar(&pfull[s], (uint32_t)((i >> 1) & 1), s_abort)) return false;
-                if (i >= 2 && !wait_bar(&ofree[s], (uint32_t)(((i >> 1) + 1) & 1), s_abort)) return false;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -382,14 +380,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
                 tc::mma_commit(&ofull[s]);
                 tc::mma_commit(&empty[s]);
-                return true;
             };
-            bool ok = true;
-            int64_t j = 0;
-            for (; j < my_tiles && ok; ++j) {
+            // Issue S of the next tile or P.V of the oldest pending one, whichever
+            // is ready first (at most two tiles in flight, one per stage).
+            auto issue_s = [&](int64_t j) {
                 const int s = (int)(j & 1);
-                if (!wait_bar(&full[s], (uint32_t)((j >> 1) & 1), s_abort)) { ok = false; break; }
-                if (j >= 2 && !wait_bar(&sfree[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort)) { ok = false; break; }
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
@@ -402,9 +397,31 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         tc::mma_bf16(tmem + s * C::S_COL, ad, bd, IDESC_S, (kb | kk) ? 1u : 0u);
                     }
                 tc::mma_commit(&sfull[s]);
-                if (j >= 1) ok = issue_pv(j - 1);
+            };
+            auto ready_s = [&](int64_t j) -> bool {
+                const int s = (int)(j & 1);
+                return tc::mbar_try_wait(&full[s], (uint32_t)((j >> 1) & 1)) &&
+                       (j < 2 || tc::mbar_try_wait(&sfree[s], (uint32_t)(((j >> 1) + 1) & 1)));
+            };
+            auto ready_pv = [&](int64_t i) -> bool {
+                const int s = (int)(i & 1);
+                return tc::mbar_try_wait(&pfull[s], (uint32_t)((i >> 1) & 1)) &&
+                       (i < 2 || tc::mbar_try_wait(&ofree[s], (uint32_t)(((i >> 1) + 1) & 1)));
+            };
+            int64_t ns = 0, npv = 0;
+            long long t0 = clock64();
+            while (npv < my_tiles) {
+                if (ns < my_tiles && ns - npv < 2 && ready_s(ns)) {
+                    issue_s(ns++);
+                    t0 = clock64();
+                } else if (npv < ns && ready_pv(npv)) {
+                    issue_pv(npv++);
+                    t0 = clock64();
+                } else if (*s_abort || clock64() - t0 > kWaitBudget) {
+                    *s_abort = 1;
+                    break;
+                }
             }
-            if (ok && j >= 1) issue_pv(j - 1);
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ softmax
