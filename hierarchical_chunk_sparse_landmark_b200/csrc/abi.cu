@@ -32,12 +32,11 @@ struct TcLaunch {
     int B, H, Hkv, S, topk, own_chunk, lm_bf16;
     int64_t L, W, cap;
     float scale;
-    const int32_t *idx, *entries, *wntiles;
+    const int32_t *idx, *entries;
     const int4 *wtiles;
-    int32_t *done;
     const int64_t *seg_start;
     float *logits, *w_out;
-    __half *part;
+    __half *part, *own;
     void *O;
     unsigned *status;
     int num_sms;
@@ -91,16 +90,11 @@ bool tc_shape_ok(int B, int H, int Hkv, int64_t L, int d, int topk) {
     return true;
 }
 
-// Token window of the tensor-core work queue: sized so that one window's fp16
-// partial outputs (W * topk * G * d * 2 bytes per (b, g)) are about 32 MB and
-// stay in L2 until that window's own tiles fuse them; a multiple of 256.
+// Token window of the work lists: one window per (b, g) -- the tiles carry no
+// dependencies, so larger windows only make the chunk buckets fuller.
 int64_t tc_window(int B, int H, int Hkv, int64_t L, int d, int topk, int64_t max_windows) {
-    const int G = H / Hkv;
-    const int64_t per_token = (int64_t)topk * G * d * 2;
-    int64_t W = ((int64_t(32) << 20) / per_token) / 256 * 256;
-    if (W < 256) W = 256;
-    const int64_t Lr = (L + 255) / 256 * 256;
-    if (W > Lr) W = Lr;
+    (void)H; (void)d; (void)topk;
+    int64_t W = (L + 255) / 256 * 256;
     while ((int64_t)B * Hkv * ((L + W - 1) / W) > max_windows) W *= 2;
     return W;
 }
@@ -111,7 +105,7 @@ struct PrefillLayout {
     bool tc;
     int64_t W, NW, cap;
     size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
-        seg_off, part_off;
+        seg_off, part_off, own_off;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
@@ -127,7 +121,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     p.tc = tc_shape_ok(B, H, Hkv, L, d, topk);
     p.W = p.NW = p.cap = 0;
     p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
-    p.wntiles_off = p.done_off = p.seg_off = p.part_off = 0;
+    p.wntiles_off = p.done_off = p.seg_off = p.part_off = p.own_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
         p.W = tc_window(B, H, Hkv, L, d, topk, attend_tc_max_windows());
@@ -150,6 +144,8 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         off = align_up(off + sizeof(int64_t) * (size_t)(2 * p.NW + 1), 256);
         p.part_off = off;
         off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
+        p.own_off = off;
+        off = align_up(off + sizeof(__half) * (size_t)B * L * H * d, 256);
     }
     p.total = off;
     return p;
@@ -301,14 +297,14 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.B = B; a.H = H; a.Hkv = Hkv; a.S = S; a.topk = topk; a.own_chunk = own_chunk;
         a.L = L; a.W = lay.W; a.cap = lay.cap; a.scale = scale;
         a.idx = idx; a.entries = (const int32_t *)(ws + lay.entries_off);
-        a.wntiles = (const int32_t *)(ws + lay.wntiles_off);
-        a.wtiles = (const int4 *)(ws + lay.wtiles_off); a.done = (int32_t *)(ws + lay.done_off);
+        a.wtiles = (const int4 *)(ws + lay.wtiles_off);
         a.seg_start = (const int64_t *)(ws + lay.seg_off);
         a.logits = w_ws; a.w_out = w_out;
-        a.part = (__half *)(ws + lay.part_off); a.O = O; a.status = (unsigned *)ws;
+        a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
+        a.O = O; a.status = (unsigned *)ws;
         a.num_sms = num_sms();
         e = launch_attend_tc(a, d, st);
-        t_launches += e == cudaSuccess ? 1 : 0;
+        t_launches += e == cudaSuccess ? 2 : 0;
     } else {
         stage_mark(3, st);
         e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale,

@@ -1,6 +1,6 @@
-// attend_tc.cu -- in-chunk attention and score-weighted fusion on the
-// 5th-generation tensor cores (tcgen05 MMA, TMEM accumulators, TMA tile
-// loads), bf16 in, fp32 accumulate.
+// attend_tc.cu -- in-chunk attention on the 5th-generation tensor cores
+// (tcgen05 MMA, TMEM accumulators, TMA tile loads), bf16 in, fp32 accumulate,
+// and the score-weighted fusion of the chunk outputs.
 //
 // HiLS Attention abstract: every query attends independently inside each
 // retrieved chunk; the chunk outputs are fused with weights from the retrieval
@@ -17,23 +17,21 @@
 //   partial[t, g, k] = O (fp16), logit[t, h, k] = scale * (S[:,64] + S[:,65])
 //
 // Own tiles: 128/G consecutive tokens of a chunk against that chunk with the
-// causal mask (keys c*S .. t).  Their epilogue completes the fusion:
+// causal mask (keys c*S .. t); their output (the own-chunk term) goes to an
+// fp16 array.  fuse_kernel then completes the method, one warp per (t, h):
 //   w = softmax over the token's selected chunks of the logits,
 //   O = own_term + sum_k w_k * partial_k  (bf16 out).
 //
-// One persistent block per SM walks the work queue (retrieved-chunk tiles of
-// window n, then own tiles of window n-1, ...) with four roles linked by
-// mbarriers and double-buffered shared memory / TMEM:
-//   warp 0      producer  (landmark rows into smem; TMA of the chunk's K and V
-//                          and, lane-parallel, of the gathered Q rows)
-//   warp 1      MMA issuer (S of tile j+1 is issued before P.V of tile j)
+// attend_tc_kernel: one persistent block per SM walks the tile queue with
+// four roles linked by mbarriers and double-buffered shared memory / TMEM:
+//   warp 0      producer  (tile metadata into a shared ring, landmark rows
+//                          into smem, TMA of the chunk's K and V)
+//   warp 10     Q gather  (one TMA box per entry: its G query-head rows)
+//   warp 1      MMA issuer (S of the next tile or P.V of the oldest pending
+//                          one, whichever is ready)
 //   warps 2-5   softmax   (thread = tile row = TMEM lane)
-//   warps 6-9   epilogue  (TMEM -> fp16 partials, or -> fused bf16 O)
-// Consumer roles prefetch the next tile's metadata while working on the
-// current one.  Own tiles of window n wait, in the epilogue only, until every
-// retrieved-chunk tile of window n has published its logits and partials; a
-// block publishes once per window (one fence per role when it moves past its
-// last tile of that window), not once per tile.  Every wait is
+//   warps 6-9   epilogue  (TMEM -> fp16 partial slots / own-chunk term)
+// Tiles are independent, so no block waits on another.  Every wait is
 // bounded; on expiry the block sets the status flag in the workspace, lets
 // in-flight copies land, frees its TMEM and exits.
 #include <cuda.h>
@@ -65,17 +63,12 @@ struct TcCfg {
 
 struct TcParams {
     const int64_t *seg_start;     // [2 * NW + 1]
-    const void *Q;                // [B, L, H, D] bf16 (rows gathered with cp.async)
     const int4 *wtiles;           // [NW * cap] retrieved-chunk tiles per window
-    const int32_t *wntiles;       // [NW]
-    int32_t *done;                // [NW] published retrieved-chunk tiles
     const int32_t *entries;
-    const int32_t *idx;
     const void *lm;               // [B, Hkv, Nc, D] bf16 or fp32
     float *logits;                // [B, L, H, topk] fusion logits
-    float *w_out;                 // [B, L, H, topk] or NULL
-    __half *part;
-    __nv_bfloat16 *O;
+    __half *part;                 // [B*L*Hkv*topk entries][D/32][G][32] chunk outputs
+    __half *own;                  // [B, L, H, D] own-chunk term
     unsigned *status;
     int64_t L, W, nwb, NW, cap, Nc;
     int H, Hkv, topk, S, add_own, lm_bf16;
@@ -95,22 +88,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
     __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&v);
-}
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int32_t *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Make this role's global stores of a window visible, then count its tiles
-// of that window (128 threads of one role; `id` is the role's named barrier).
-__device__ __forceinline__ void publish(int32_t *counter, int n, int id, bool leader) {
-    __threadfence();
-    named_sync(id, 128);
-    if (leader) atomicAdd(counter, n);
 }
 
 // Bounded mbarrier wait that also gives up when another role aborted.
@@ -429,9 +406,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int r = q4 * 32 + lane;             // tile row
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
-        const bool leader = (warp == 2 && lane == 0);
-        int64_t pub_win = -1;
-        int pub_cnt = 0;
         for (int64_t j = 0; j < my_tiles; ++j) {
             const int ri = (int)(j & (kRing - 1));
             if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
@@ -440,12 +414,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const int s = (int)(j & 1);
             const int64_t b = cur.tl.bg / Hkv;
             const int g = (int)(cur.tl.bg % Hkv);
-            if (cur.tl.own || cur.tl.win != pub_win) {
-                // leaving window pub_win: its logits from this block are published
-                if (pub_cnt) publish(p.done + pub_win, pub_cnt, 3, leader);
-                pub_win = cur.tl.own ? -1 : cur.tl.win;
-                pub_cnt = 0;
-            }
             if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
             float s0[32], s1[32], l_hi, l_lo;
@@ -488,144 +456,50 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&pfull[s]);
-            if (!cur.tl.own) ++pub_cnt;
         }
-        if (pub_cnt && !*s_abort) publish(p.done + pub_win, pub_cnt, 3, leader);
     } else {
         // ------------------------------------------------------------ epilogue
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
-        const bool leader = (warp == 6 && lane == 0);
         constexpr int NCH = D / 32;               // 32-column chunks of a row
-        int64_t pub_win = -1;
-        int pub_cnt = 0;
         for (int64_t j = 0; j < my_tiles; ++j) {
             const int ri = (int)(j & (kRing - 1));
             if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
             const RowJob cur = read_row(ring[ri], e);
             tc::mbar_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
-            if (cur.tl.own || cur.tl.win != pub_win) {
-                // leaving window pub_win: its partials from this block are published
-                if (pub_cnt) publish(p.done + pub_win, pub_cnt, 2, leader);
-                pub_win = cur.tl.own ? -1 : cur.tl.win;
-                pub_cnt = 0;
-            }
             const int64_t b = cur.tl.bg / Hkv;
             const int g = (int)(cur.tl.bg % Hkv);
             const int64_t row = (b * L + cur.t) * Hkv + g;       // (t, g) selection row
             const int64_t hrow = (b * L + cur.t) * H + (int64_t)g * G + h;
-            float lg[32];
-            int nsel = 0;
-            float m = -INFINITY, inv_den = 0.f;
-            if (cur.tl.own) {
-                // the window's retrieved-chunk partials must all be published
-                if (leader) {
-                    // both roles (softmax: logits, epilogue: partials) count every tile
-                    const int32_t need = 2 * p.wntiles[cur.tl.win];
-                    const long long t0c = clock64();
-                    while (ld_acquire(&p.done[cur.tl.win]) < need) {
-                        if (*s_abort || clock64() - t0c > kWaitBudget) { *s_abort = 1; break; }
-                        __nanosleep(128);
-                    }
-                }
-                named_sync(1, 128);
-                if (*s_abort) break;
-                if (cur.valid) {
-                    // selected slots come first; load the row's indices and logits at once
-                    const int32_t *ip = p.idx + row * topk;
-                    for (int kk = 0; kk < topk; ++kk) nsel += ip[kk] >= 0 ? 1 : 0;
-                    for (int kk = 0; kk < nsel; ++kk) lg[kk] = __ldcg(p.logits + hrow * topk + kk);
-                    for (int kk = 0; kk < nsel; ++kk) m = fmaxf(m, lg[kk]);
-                    float den = 0.f;
-                    for (int kk = 0; kk < nsel; ++kk) {
-                        lg[kk] = __expf(lg[kk] - m);
-                        den += lg[kk];
-                    }
-                    inv_den = nsel ? 1.f / den : 0.f;
-                    for (int kk = 0; kk < nsel; ++kk) lg[kk] *= inv_den;    // fusion weights
-                    if (p.w_out)
-                        for (int kk = 0; kk < topk; ++kk)
-                            p.w_out[hrow * topk + kk] = kk < nsel ? lg[kk] : 0.f;
-                }
-            }
             if (!wait_bar(&ofull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
-            // O chunk ch (32 columns) of this row -> partial slot or fused output
-            auto emit = [&](int ch, float (&o)[32]) {
-                if (!cur.tl.own) {
-                    // partial layout [entry][d/32][head][32] (fp16)
-                    __half *dst = p.part + (((row * topk + cur.k) * NCH + ch) * G + h) * 32;
+#pragma unroll 1
+            for (int ch = 0; ch < NCH; ch += 2) {
+                float o[2][32];
+                // two 32-column TMEM loads per wait
+                tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o[0]);
+                tc::tmem_ld32(tmem + C::O_COL + s * D + (ch + 1) * 32 + lane_off, o[1]);
+                tc::tmem_wait_ld();
+                if (!cur.valid) continue;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    // retrieved chunk: slot [entry][d/32][head][32]; own chunk: [t, h, d]
+                    __half *dst = cur.tl.own
+                        ? p.own + hrow * D + (ch + u) * 32
+                        : p.part + (((row * topk + cur.k) * NCH + ch + u) * G + h) * 32;
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                            pack_f16x2(o[8 * q + 0], o[8 * q + 1]), pack_f16x2(o[8 * q + 2], o[8 * q + 3]),
-                            pack_f16x2(o[8 * q + 4], o[8 * q + 5]), pack_f16x2(o[8 * q + 6], o[8 * q + 7]));
-                } else {
-                    // fusion: O += sum_k w_k * partial_k, four slots' loads in flight at a time
-                    for (int k0 = 0; k0 < nsel; k0 += 4) {
-                        uint4 u[4][4];
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            if (k0 + a < nsel) {
-                                const uint4 *src = reinterpret_cast<const uint4 *>(
-                                    p.part + (((row * topk + k0 + a) * NCH + ch) * G + h) * 32);
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) u[a][q] = __ldcg(src + q);
-                            }
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            if (k0 + a < nsel) {
-                                const float wk = lg[k0 + a];
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const __half2 *hh = reinterpret_cast<const __half2 *>(&u[a][q]);
-#pragma unroll
-                                    for (int z = 0; z < 4; ++z) {
-                                        const float2 v = __half22float2(hh[z]);
-                                        o[8 * q + 2 * z] = fmaf(wk, v.x, o[8 * q + 2 * z]);
-                                        o[8 * q + 2 * z + 1] = fmaf(wk, v.y, o[8 * q + 2 * z + 1]);
-                                    }
-                                }
-                            }
-                    }
-                    __nv_bfloat16 *dst = p.O + hrow * D + ch * 32;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                            pack_bf16x2(o[8 * q + 0], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
-                            pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
-                }
-            };
-            if (!cur.tl.own) {
-#pragma unroll 1
-                for (int ch = 0; ch < NCH; ch += 2) {
-                    float o0[32], o1[32];
-                    // two 32-column TMEM loads per wait
-                    tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o0);
-                    tc::tmem_ld32(tmem + C::O_COL + s * D + (ch + 1) * 32 + lane_off, o1);
-                    tc::tmem_wait_ld();
-                    if (!cur.valid) continue;
-                    emit(ch, o0);
-                    emit(ch + 1, o1);
-                }
-            } else {
-#pragma unroll 1
-                for (int ch = 0; ch < NCH; ++ch) {
-                    float o0[32];
-                    tc::tmem_ld32(tmem + C::O_COL + s * D + ch * 32 + lane_off, o0);
-                    tc::tmem_wait_ld();
-                    if (!cur.valid) continue;
-                    emit(ch, o0);
+                            pack_f16x2(o[u][8 * q + 0], o[u][8 * q + 1]), pack_f16x2(o[u][8 * q + 2], o[u][8 * q + 3]),
+                            pack_f16x2(o[u][8 * q + 4], o[u][8 * q + 5]), pack_f16x2(o[u][8 * q + 6], o[u][8 * q + 7]));
                 }
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&ofree[s]);
-            if (!cur.tl.own) ++pub_cnt;
         }
-        if (pub_cnt && !*s_abort) publish(p.done + pub_win, pub_cnt, 2, leader);
     }
 
     __syncthreads();
@@ -637,6 +511,69 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     tc::fence_after_sync();
     if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- fusion
+// One warp per (t, h) row: w = softmax over the selected chunks of the
+// logits, O = own + sum_k w_k * partial_k.  Lane l holds the D/32 consecutive
+// elements d = l*D/32 ..; in the partial layout these are chunk l/(32/NCH),
+// offset (l % (32/NCH)) * D/32 -- the same d.  Slot loads are unrolled so
+// several are in flight.
+template <int D, int G>
+__global__ void __launch_bounds__(256)
+fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
+            const float *__restrict__ logits, const int32_t *__restrict__ idx, int64_t rows, int H,
+            int Hkv, int topk, float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
+    constexpr int EPL = D / 32;                      // elements per lane (4 or 2)
+    constexpr int NCH = D / 32;                      // 32-wide chunks of d
+    constexpr int LPC = 32 / NCH;                    // lanes per chunk
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int64_t bt = row / H;
+    const int hh = (int)(row % H);
+    const int g = hh / G, h = hh % G;
+    const int64_t srow = bt * Hkv + g;               // selection row (t, g)
+    const int32_t ik = lane < topk ? idx[srow * topk + lane] : -1;
+    const int nsel = __popc(__ballot_sync(0xffffffffu, ik >= 0));   // valid slots come first
+    const float lg = lane < nsel ? logits[row * topk + lane] : -INFINITY;
+    float m = lg;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ex = lane < nsel ? __expf(lg - m) : 0.f;
+    float den = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float w = nsel ? ex / den : 0.f;
+    if (w_out && lane < topk) w_out[row * topk + lane] = w;
+
+    const int ch = lane / LPC, off = (lane % LPC) * EPL;
+    float acc[EPL];
+    {
+        const __half2 *s2 = reinterpret_cast<const __half2 *>(own + row * D + lane * EPL);
+#pragma unroll
+        for (int q = 0; q < EPL / 2; ++q) {
+            const float2 v = __half22float2(s2[q]);
+            acc[2 * q] = v.x;
+            acc[2 * q + 1] = v.y;
+        }
+    }
+    const __half *pbase = part + (((srow * topk) * NCH + ch) * G + h) * 32 + off;
+    const int64_t kstride = (int64_t)NCH * G * 32;   // halves between slots k and k+1
+#pragma unroll 8
+    for (int k = 0; k < nsel; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, w, k);
+        const __half2 *s2 = reinterpret_cast<const __half2 *>(pbase + k * kstride);
+#pragma unroll
+        for (int q = 0; q < EPL / 2; ++q) {
+            const float2 v = __half22float2(s2[q]);
+            acc[2 * q] = fmaf(wk, v.x, acc[2 * q]);
+            acc[2 * q + 1] = fmaf(wk, v.y, acc[2 * q + 1]);
+        }
+    }
+    __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(O + row * D + lane * EPL);
+#pragma unroll
+    for (int q = 0; q < EPL / 2; ++q) dst[q] = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
 }
 
 // ---------------------------------------------------------------- host side
@@ -692,12 +629,11 @@ struct TcLaunch {
     int B, H, Hkv, S, topk, own_chunk, lm_bf16;
     int64_t L, W, cap;
     float scale;
-    const int32_t *idx, *entries, *wntiles;
+    const int32_t *idx, *entries;
     const int4 *wtiles;
-    int32_t *done;
     const int64_t *seg_start;
     float *logits, *w_out;
-    __half *part;
+    __half *part, *own;
     void *O;
     unsigned *status;
     int num_sms;
@@ -719,10 +655,9 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     TcParams p;
-    p.Q = a.Q;
-    p.seg_start = a.seg_start; p.wtiles = a.wtiles; p.wntiles = a.wntiles; p.done = a.done;
-    p.entries = a.entries; p.idx = a.idx; p.lm = a.lm; p.logits = a.logits; p.w_out = a.w_out;
-    p.part = a.part; p.O = (__nv_bfloat16 *)a.O; p.status = a.status;
+    p.seg_start = a.seg_start; p.wtiles = a.wtiles;
+    p.entries = a.entries; p.lm = a.lm; p.logits = a.logits;
+    p.part = a.part; p.own = a.own; p.status = a.status;
     p.L = a.L; p.W = a.W; p.nwb = (a.L + a.W - 1) / a.W;
     p.NW = (int64_t)a.B * a.Hkv * p.nwb; p.cap = a.cap; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
@@ -731,6 +666,13 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     p.scale = a.scale;
     p.scale_log2e = a.scale * 1.4426950408889634f;
     kern<<<(unsigned)a.num_sms, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)a.B * a.L * a.H;
+    constexpr int kWarps = 8;
+    fuse_kernel<D, G><<<(unsigned)((rows + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
+        a.part, a.own, a.logits, a.idx, rows, a.H, a.Hkv, a.topk, a.w_out,
+        (__nv_bfloat16 *)a.O);
     return cudaGetLastError();
 }
 
