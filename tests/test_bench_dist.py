@@ -1,0 +1,80 @@
+"""bench.py's multi-GPU host logic on CPU: two gloo ranks check that the
+whole-job throughput is the work summed over ranks divided by the slowest
+rank's time, and that every rank draws an independent batch (weak scaling)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_prefill_inputs
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ws, r, local = bench.dist_env()
+        assert (ws, r, local) == (world, rank, rank)
+        # rank r processed (r+1) units in (r+1)*0.5 s
+        units, secs = bench.aggregate(dist, float(rank + 1), 0.5 * (rank + 1), "cpu")
+        wl = WORKLOADS["train_prefill_bf16"].with_(B=1, L=256)
+        x = make_prefill_inputs(wl.with_(seed=wl.seed + rank), "cpu")
+        q_sum = torch.tensor([float(x["Q"].float().sum())])
+        gathered = [torch.zeros(1) for _ in range(world)]
+        dist.all_gather(gathered, q_sum)
+        q.put((rank, units, secs, [float(g) for g in gathered]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_aggregation_and_independent_batches():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, units, secs, sums in res:
+        assert units == pytest.approx(3.0)        # 1 + 2 units over both ranks
+        assert secs == pytest.approx(1.0)         # max over ranks, not the sum
+        assert sums[0] != sums[1]                 # per-rank seeds give different batches
+
+
+def test_single_process_aggregation_is_identity():
+    assert bench.aggregate(None, 5.0, 2.0) == (5.0, 2.0)
+
+
+def test_flop_and_byte_counts_match_definitions():
+    wl = WORKLOADS["train_prefill_bf16"]
+    f = bench.prefill_flops(wl)
+    # hand count for one batch element, token by token
+    tot = 0
+    for t in range(wl.L):
+        nvis = t // wl.S
+        keff = min(wl.topk, nvis)
+        own = t - wl.S * nvis + 1
+        tot += (wl.Hkv * 2 * wl.d * nvis + wl.H * 2 * wl.d * keff + wl.H * 4 * wl.d * wl.S * keff
+                + wl.H * 4 * wl.d * own)
+    assert f["total"] == pytest.approx(wl.B * tot)
+    d5 = WORKLOADS["decode_32m_bf16"]
+    nc = d5.L // d5.S
+    assert bench.decode_bytes(d5) == d5.B * (d5.Hkv * nc * d5.d * 2 + d5.Hkv * 8 * 64 * d5.d * 2 * 2
+                                             + 2 * d5.H * d5.d * 2)
