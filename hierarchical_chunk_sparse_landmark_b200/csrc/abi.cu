@@ -20,8 +20,8 @@ cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool
                                void *O, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
                           const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
-                          int S, int topk, float scale, int splits, uint64_t *cand,
-                          unsigned *tickets, void *O, int32_t *idx_out, cudaStream_t st);
+                          int S, int topk, float scale, int splits, const DecodeScratch &ws,
+                          void *O, int32_t *idx_out, cudaStream_t st);
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
@@ -156,20 +156,30 @@ bool force_simt_path() {
     return v && strcmp(v, "simt") == 0;
 }
 
+// Decode workspace: status | tickets (the zeroed head) | sel | cand.
 struct DecodeLayout {
-    size_t tickets_off, cand_off, total;
+    size_t sel_off, cand_off, total;
     int splits;
+    DecodeScratch at(char *ws) const {
+        DecodeScratch s;
+        s.status = (unsigned *)ws;
+        s.tickets = (unsigned *)(ws + kStatusBytes);
+        s.sel = (int32_t *)(ws + sel_off);
+        s.cand = (uint64_t *)(ws + cand_off);
+        return s;
+    }
 };
 
 DecodeLayout decode_layout(int B, int Hkv, int64_t Lc, int S, int topk) {
     DecodeLayout p;
     const int64_t Nc = Lc / S;
+    const size_t pairs = (size_t)B * Hkv;
     p.splits = decode_splits(B, Hkv, Nc, num_sms());
-    size_t off = kStatusBytes;
-    p.tickets_off = off;
-    off = align_up(off + sizeof(unsigned) * (size_t)B * Hkv, 256);
+    size_t off = decode_zero_head(B, Hkv);
+    p.sel_off = off;
+    off = align_up(off + sizeof(int32_t) * pairs * topk, 256);
     p.cand_off = off;
-    off = align_up(off + sizeof(uint64_t) * (size_t)B * Hkv * p.splits * topk, 256);
+    off = align_up(off + sizeof(uint64_t) * pairs * p.splits * topk, 256);
     p.total = off;
     return p;
 }
@@ -352,10 +362,9 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
     char *ws = (char *)workspace;
     stage_mark(0, st);
     hsa_status_t r = from_cuda(launch_decode(q, Kc, Vc, dt == HSA_BF16, lm, lm_dt == HSA_BF16, B, H, Hkv,
-                                   Lc, d, S, topk, scale, lay.splits,
-                                   (uint64_t *)(ws + lay.cand_off),
-                                   (unsigned *)(ws + lay.tickets_off), O, idx_out, st));
-    t_launches = r == HSA_OK ? 1 : 0;
+                                   Lc, d, S, topk, scale, lay.splits, lay.at(ws), O,
+                                   idx_out, st));
+    t_launches = r == HSA_OK ? 2 : 0;
     stage_mark(1, st);
     return r;
 }

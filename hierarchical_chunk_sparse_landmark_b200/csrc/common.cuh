@@ -40,6 +40,46 @@ template <> struct Vec16<__nv_bfloat16> {
     }
 };
 
+// ---------------------------------------------------------------- packed fp32 pairs
+// Two fp32 values in one 64-bit register pair; ffma2 is an element-wise
+// a * b + c with one rounding per element, exactly like two fmaf calls.
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float sum_f2(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo + hi;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// acc += q2 . (one 16-byte vector of T), q2 = the matching fp32 pairs.
+template <typename T> struct Dot16;
+template <> struct Dot16<float> {
+    static constexpr int PAIRS = 2;
+    __device__ __forceinline__ static uint64_t fma(const uint4 &u, const uint64_t *q2, uint64_t acc) {
+        acc = ffma2(q2[0], pack_f2(__uint_as_float(u.x), __uint_as_float(u.y)), acc);
+        return ffma2(q2[1], pack_f2(__uint_as_float(u.z), __uint_as_float(u.w)), acc);
+    }
+};
+template <> struct Dot16<__nv_bfloat16> {
+    static constexpr int PAIRS = 4;
+    __device__ __forceinline__ static uint64_t pair(uint32_t w) {
+        return pack_f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    __device__ __forceinline__ static uint64_t fma(const uint4 &u, const uint64_t *q2, uint64_t acc) {
+        acc = ffma2(q2[0], pair(u.x), acc);
+        acc = ffma2(q2[1], pair(u.y), acc);
+        acc = ffma2(q2[2], pair(u.z), acc);
+        return ffma2(q2[3], pair(u.w), acc);
+    }
+};
+
 // Streaming 16-byte load that does not allocate in L1 (read-once data).
 __device__ __forceinline__ uint4 ld_stream16(const void *p) {
     uint4 r;
@@ -60,6 +100,12 @@ __device__ __forceinline__ uint32_t score_order_bits(float s) {
 }
 __device__ __forceinline__ uint64_t make_key(float s, int64_t idx) {
     return ((uint64_t)score_order_bits(s) << 32) | (uint64_t)(~(uint32_t)idx);
+}
+// Score of a key (inverse of score_order_bits); -inf for the empty key.
+__device__ __forceinline__ float key_score(uint64_t k) {
+    if (k == 0ull) return -INFINITY;
+    const uint32_t h = (uint32_t)(k >> 32);
+    return __uint_as_float((h & 0x80000000u) ? (h & 0x7fffffffu) : ~h);
 }
 __device__ __forceinline__ int32_t key_index(uint64_t k) {
     return k == 0ull ? -1 : (int32_t)(~(uint32_t)(k & 0xffffffffull));
@@ -86,6 +132,29 @@ struct WarpTopK {
     }
 };
 
+// Top-K of the keys a warp holds (M per lane, 0 = none; keys are distinct
+// unless 0): K rounds of a warp-wide maximum, the owner of each winner drops
+// it.  Returns in lane k < topk the k-th best key (0 when fewer exist).
+__device__ __forceinline__ uint64_t max_u64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+template <int M>
+__device__ __forceinline__ uint64_t warp_select_topk(uint64_t (&x)[M], int topk) {
+    const int lane = threadIdx.x & 31;
+    uint64_t out = 0ull;
+    for (int r = 0; r < topk; ++r) {
+        uint64_t best = x[0];
+#pragma unroll
+        for (int m = 1; m < M; ++m) best = max_u64(best, x[m]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) best = max_u64(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (best == 0ull) break;                  // no keys left (warp-uniform)
+        if (lane == r) out = best;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            if (x[m] == best) x[m] = 0ull;
+    }
+    return out;
+}
+
 // ---------------------------------------------------------------- status word
 // The first 256 bytes of every workspace.  word[0] = error flags set by kernels
 // (bit 0: a bounded wait gave up).
@@ -93,5 +162,19 @@ constexpr size_t kStatusBytes = 256;
 constexpr unsigned kFlagTimeout = 1u;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Decode scratch inside the caller's workspace.  The ticket array sits right
+// after the status word and must start at zero (the kernels leave it at
+// zero); everything else is rewritten by every call.
+struct DecodeScratch {
+    unsigned *status;     // status word
+    unsigned *tickets;    // [B*Hkv] scan blocks done
+    int32_t *sel;         // [B*Hkv*topk] selected chunks
+    uint64_t *cand;       // [B*Hkv*splits*topk] per-block candidate keys
+};
+// Bytes at the head of a decode workspace that must be zero before a call.
+__host__ __device__ constexpr size_t decode_zero_head(int64_t B, int64_t Hkv) {
+    return align_up(kStatusBytes + sizeof(unsigned) * (size_t)(B * Hkv), 256);
+}
 
 }  // namespace hsa

@@ -8,261 +8,469 @@
 // Length Generalization in Hierarchical Sparse Attention Models; fusion by
 // retrieval scores: HiLS Attention abstract.)
 //
-// The landmark scan is the HBM stream (the K/V cache itself is never read
-// except for the K selected chunks).  Grid = splits x (B*Hkv) blocks; each
-// block scans a contiguous range of landmark rows with 16-byte streaming loads
-// (a row is d elements = D/VEC lanes; a warp covers 32*16 contiguous bytes per
-// load), reduces each row's partial dot products with xor-shuffles and keeps a
-// warp-distributed top-K of 64-bit (score, ~index) keys.  Blocks publish their
-// K best keys, take a ticket, and the last block of each (b, g) merges all
-// candidates, resets the ticket and runs D3.  There is no inter-block wait.
+// The landmark scan is the HBM stream; the K/V cache is read only for the K
+// selected chunks.
+//
+// decode_scan_kernel: grid = splits x (B*Hkv), sized to one wave.  Each block
+// owns a contiguous range of landmark rows.  A producer warp streams the range
+// through a 4-stage shared-memory ring with 16 KB bulk async copies (full /
+// empty mbarriers, so consumers never wait on a block-wide barrier); eight
+// consumer warps score the rows: a quarter-warp holds one row, its dot product
+// with the scaled qbar uses packed fp32 FMAs and three xor-shuffles.  A float
+// threshold filters rows; only the rare candidates become 64-bit (score,
+// ~index) keys in a warp-distributed top-K.  Blocks publish their K best keys
+// and take a ticket; the last block of each (b, g) merges all candidates with
+// warp-parallel selection, writes the selection and resets the ticket.  No
+// block waits for another.
+//
+// decode_attend_kernel (launched as a programmatic dependent of the scan, so
+// its launch and its query loads overlap the scan's tail): one cluster of
+// min(K, 8) blocks per (b, g); see the kernel's comment.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+#include "tc.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace hsa {
 
-constexpr int kDecThreads = 256;
-constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kDecUnroll = 4;
+constexpr int kScanWarps = 8;                  // consumer warps
+constexpr int kScanThreads = (kScanWarps + 1) * 32;   // + one producer warp
+constexpr int kScanStages = 4;
+constexpr int kStageBytes = 16384;
+constexpr int kScanBlocksPerSm = 3;            // 64 KB ring + ~3 KB per block
+constexpr long long kScanWait = 4000000000LL;  // SM cycles (about 2 s)
 
 template <typename T, typename TL, int D>
-__global__ void __launch_bounds__(kDecThreads)
-decode_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T *__restrict__ Kc,
-              const T *__restrict__ Vc, int H, int Hkv, int64_t Lc, int S, int topk, float scale,
-              int splits, uint64_t *__restrict__ cand, unsigned *__restrict__ tickets,
-              T *__restrict__ O, int32_t *__restrict__ idx_out) {
-    constexpr int VEC = Vec16<TL>::N;
-    constexpr int LPR = D / VEC;          // lanes per landmark row
-    constexpr int RPW = 32 / LPR;         // rows per warp load
-    constexpr int VT = Vec16<T>::N;
-    constexpr int RS = D + VT;            // padded K/V row stride in shared memory
-    constexpr int R = D / 32;
+__global__ void __launch_bounds__(kScanThreads)
+decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, int Hkv, int64_t Nc,
+                   int topk, float scale, int splits, uint64_t *__restrict__ cand,
+                   unsigned *__restrict__ tickets, int32_t *__restrict__ sel_out,
+                   int32_t *__restrict__ idx_out, unsigned *__restrict__ status) {
+    constexpr int ROW_BYTES = D * (int)sizeof(TL);
+    constexpr int ROWS = kStageBytes / ROW_BYTES;           // landmark rows per stage
+    constexpr int VEC = Vec16<TL>::N;                        // elements per 16-byte vector
+    constexpr int LPR = 8;                                   // lanes per row (one quarter-warp)
+    constexpr int VPL = D / VEC / LPR;                       // 16-byte vectors per lane and row
+    constexpr int ITER = ROWS / (kScanWarps * 4);            // warp steps (4 rows each) per stage
+    static_assert(ROWS % (kScanWarps * 4) == 0, "stage must split evenly over warps");
+    static_assert(VPL >= 1, "row narrower than a quarter-warp");
 
+    extern __shared__ __align__(128) uint8_t ring[];         // [kScanStages][kStageBytes]
+    __shared__ uint64_t full[kScanStages], empty[kScanStages];
     __shared__ float qbar_s[D];
-    __shared__ uint64_t lists[kDecWarps][32];
-    __shared__ int is_last;
-    __shared__ int32_t sel_s[32];
-    __shared__ float wsel[16][32];
-    extern __shared__ float4 dyn4[];
+    __shared__ uint64_t lists[kScanWarps][32];
+    __shared__ int is_last, s_abort;
 
     const int split = blockIdx.x;
     const int64_t bg = blockIdx.y;
     const int64_t b = bg / Hkv;
     const int g = (int)(bg % Hkv);
     const int G = H / Hkv;
-    const int64_t Nc = Lc / S;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    for (int j = tid; j < D; j += kDecThreads) {
-        float a = 0.f;
-        for (int h = 0; h < G; ++h) a += to_f32(q[(b * H + g * G + h) * D + j]);
-        qbar_s[j] = a / (float)G;
-    }
-    __syncthreads();
-
-    // ---------------------------------------------------------------- D1: scan
-    const int col = (lane % LPR) * VEC;
-    const int sub = lane / LPR;
-    float qv[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) qv[e] = qbar_s[col + e];
     const int64_t r0 = (int64_t)split * Nc / splits;
     const int64_t r1 = (int64_t)(split + 1) * Nc / splits;
+    const int64_t nrows = r1 - r0;
+    const int64_t nst = (nrows + ROWS - 1) / ROWS;
     const TL *lm_bg = lm + bg * Nc * D;
+
+    if (tid == 0) {
+        for (int i = 0; i < kScanStages; ++i) {
+            tc::mbar_init(&full[i], 1);
+            tc::mbar_init(&empty[i], kScanWarps);
+        }
+        s_abort = 0;
+        tc::fence_barrier_init();
+    }
+    __syncthreads();
 
     WarpTopK tk;
     tk.init(topk);
     uint64_t thr = 0ull;
-    constexpr int STEP = kDecWarps * kDecUnroll * RPW;
-    for (int64_t base = r0; base < r1; base += STEP) {
-        uint4 raw[kDecUnroll];
-#pragma unroll
-        for (int u = 0; u < kDecUnroll; ++u) {
-            const int64_t row = base + (int64_t)(warp * kDecUnroll + u) * RPW + sub;
-            raw[u] = row < r1 ? ld_stream16(lm_bg + row * D + col) : make_uint4(0, 0, 0, 0);
+    if (warp == kScanWarps) {
+        // producer: one elected lane keeps kScanStages bulk copies in flight
+        if (lane == 0) {
+            int64_t issued = 0;
+            for (int64_t st = 0; st < nst; ++st) {
+                const int slot = (int)(st % kScanStages);
+                if (st >= kScanStages &&
+                    !tc::mbar_wait(&empty[slot], (uint32_t)(((st / kScanStages) - 1) & 1),
+                                   kScanWait)) {
+                    s_abort = 1;
+                    break;
+                }
+                const int64_t left = nrows - st * ROWS;
+                const uint32_t bytes = (uint32_t)((left < ROWS ? left : ROWS) * ROW_BYTES);
+                tc::mbar_expect_tx(&full[slot], bytes);
+                tc::bulk_load(ring + slot * kStageBytes, lm_bg + (r0 + st * ROWS) * D, bytes,
+                              &full[slot]);
+                issued = st + 1;
+            }
+            // the copies still in flight land before the block can exit
+            for (int64_t j = issued > kScanStages ? issued - kScanStages : 0; j < issued; ++j)
+                tc::mbar_wait(&full[j % kScanStages], (uint32_t)((j / kScanStages) & 1), kScanWait);
         }
-#pragma unroll
-        for (int u = 0; u < kDecUnroll; ++u) {
-            const int64_t row = base + (int64_t)(warp * kDecUnroll + u) * RPW + sub;
-            float f[VEC];
-            Vec16<TL>::unpack(raw[u], f);
+    } else {
+        // qbar (consumer warps only, while the first copies are in flight)
+        for (int j = tid; j < D; j += kScanWarps * 32) {
+            const T *qp = q + (b * H + (int64_t)g * G) * D + j;
             float a = 0.f;
+#pragma unroll 4
+            for (int h = 0; h < G; ++h) a += to_f32(qp[(int64_t)h * D]);
+            qbar_s[j] = a / (float)G;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kScanWarps * 32) : "memory");
+        // the 8 lanes of quarter-warp `sub` share one row; lane c holds the
+        // 16-byte vectors c, c + 8, ... of it and the matching scaled qbar pairs
+        const int c = lane & 7, sub = lane >> 3;
+        constexpr int PAIRS = Dot16<TL>::PAIRS;
+        uint64_t q2[VPL][PAIRS];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) a = fmaf(qv[e], f[e], a);
+        for (int j = 0; j < VPL; ++j)
 #pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            const uint64_t key = row < r1 ? make_key(scale * a, row) : 0ull;
+            for (int e = 0; e < PAIRS; ++e) {
+                const float *qp = qbar_s + (c + LPR * j) * VEC + 2 * e;
+                q2[j][e] = pack_f2(scale * qp[0], scale * qp[1]);
+            }
+        float tf = -INFINITY;          // score of the K-th best key so far
+        for (int64_t st = 0; st < nst; ++st) {
+            const int slot = (int)(st % kScanStages);
+            if (!tc::mbar_wait(&full[slot], (uint32_t)((st / kScanStages) & 1), kScanWait)) {
+                s_abort = 1;
+                break;
+            }
+            const int rows_here = (int)(nrows - st * ROWS < ROWS ? nrows - st * ROWS : ROWS);
+            const uint8_t *stage = ring + slot * kStageBytes;
 #pragma unroll
-            for (int s = 0; s < RPW; ++s) {
-                const uint64_t x = __shfl_sync(0xffffffffu, key, s * LPR);
-                if (x > thr) {
-                    tk.insert(x);
-                    thr = tk.threshold();
+            for (int it = 0; it < ITER; ++it) {
+                const int rr = (it * kScanWarps + warp) * 4 + sub;
+                const uint8_t *row = stage + rr * ROW_BYTES;
+                uint64_t acc = 0ull;
+#pragma unroll
+                for (int j = 0; j < VPL; ++j)
+                    acc = Dot16<TL>::fma(*reinterpret_cast<const uint4 *>(row + (c + LPR * j) * 16),
+                                         q2[j], acc);
+                float a = sum_f2(acc);
+                a += __shfl_xor_sync(0xffffffffu, a, 4);
+                a += __shfl_xor_sync(0xffffffffu, a, 2);
+                a += __shfl_xor_sync(0xffffffffu, a, 1);
+                // cheap float filter; ties and the exact order are settled on the keys
+                unsigned m = __ballot_sync(0xffffffffu, a >= tf && rr < rows_here) & 0x01010101u;
+                if (m) {
+                    const uint64_t key = make_key(a, r0 + st * ROWS + rr);
+                    while (m) {
+                        const int s = __ffs(m) - 1;
+                        m &= m - 1;
+                        const uint64_t x = __shfl_sync(0xffffffffu, key, s);
+                        if (x > thr) {
+                            tk.insert(x);
+                            thr = tk.threshold();
+                        }
+                    }
+                    tf = key_score(thr);
                 }
             }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[slot]);     // this warp is done with the slot
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // block merge of the warp lists
-    lists[warp][lane] = tk.v;
+    if (warp < kScanWarps) lists[warp][lane] = tk.v;
     __syncthreads();
     if (warp == 0) {
-        for (int w2 = 1; w2 < kDecWarps; ++w2) {
-            for (int k = 0; k < topk; ++k) {
-                const uint64_t x = lists[w2][k];
-                if (x > thr) {
-                    tk.insert(x);
-                    thr = tk.threshold();
-                }
-            }
-        }
-        if (lane < topk) cand[(bg * splits + split) * topk + lane] = tk.v;
+        uint64_t x[kScanWarps];
+#pragma unroll
+        for (int w2 = 0; w2 < kScanWarps; ++w2) x[w2] = lists[w2][lane];
+        const uint64_t best = warp_select_topk(x, topk);
+        if (lane < topk) cand[(bg * splits + split) * topk + lane] = best;
     }
+    if (s_abort && tid == 0) atomicOr(status, kFlagTimeout);
 
-    // ---------------------------------------------------------------- D2: last block merges
+    // last block of this (b, g) merges the candidates of every split
     __threadfence();
     __syncthreads();
     if (tid == 0) is_last = (atomicAdd(&tickets[bg], 1u) == (unsigned)(splits - 1));
     __syncthreads();
-    if (!is_last) return;
+    if (!is_last || warp >= kScanWarps) return;
     __threadfence();
-
-    tk.init(topk);
-    thr = 0ull;
+    // each consumer warp reduces its share of the candidates to a top-K, 256 at a time
     const int64_t ncand = (int64_t)splits * topk;
+    const int64_t per = (ncand + kScanWarps - 1) / kScanWarps;
+    const int64_t w0 = warp * per, w1 = w0 + per < ncand ? w0 + per : ncand;
     const uint64_t *cb = cand + bg * ncand;
-    for (int64_t c0 = (int64_t)warp * 32; c0 < ncand; c0 += kDecThreads) {
-        const uint64_t x = (c0 + lane < ncand)
-            ? (uint64_t)__ldcg(reinterpret_cast<const unsigned long long *>(cb + c0 + lane)) : 0ull;
-        for (int s = 0; s < 32; ++s) {
-            const uint64_t y = __shfl_sync(0xffffffffu, x, s);
-            if (y > thr) {
-                tk.insert(y);
-                thr = tk.threshold();
-            }
+    uint64_t mine = 0ull;
+    for (int64_t c0 = w0; c0 < w1; c0 += 8 * 32) {
+        uint64_t x[9];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int64_t i = c0 + m * 32 + lane;
+            x[m] = i < w1 ? (uint64_t)__ldcg(reinterpret_cast<const unsigned long long *>(cb + i))
+                          : 0ull;
         }
+        x[8] = mine;
+        mine = warp_select_topk(x, topk);
     }
-    __syncthreads();
-    lists[warp][lane] = tk.v;
-    __syncthreads();
+    lists[warp][lane] = mine;
+    asm volatile("bar.sync 1, %0;" ::"n"(kScanWarps * 32) : "memory");
     if (warp == 0) {
-        for (int w2 = 1; w2 < kDecWarps; ++w2) {
-            for (int k = 0; k < topk; ++k) {
-                const uint64_t x = lists[w2][k];
-                if (x > thr) {
-                    tk.insert(x);
-                    thr = tk.threshold();
-                }
-            }
-        }
+        uint64_t x[kScanWarps];
+#pragma unroll
+        for (int w2 = 0; w2 < kScanWarps; ++w2) x[w2] = lists[w2][lane];
+        const uint64_t best = warp_select_topk(x, topk);
         if (lane < topk) {
-            const int32_t i = key_index(tk.v);
-            sel_s[lane] = i;
+            const int32_t i = key_index(best);
+            sel_out[bg * topk + lane] = i;
             if (idx_out) idx_out[bg * topk + lane] = i;
         }
         if (lane == 0) tickets[bg] = 0u;        // ready for the next call
     }
-    __syncthreads();
+}
 
-    // ---------------------------------------------------------------- D3: attend + fuse
+// decode_attend_kernel: one thread-block cluster of C = min(K, 8) blocks per
+// (b, g); block c of the cluster takes the slots k = c, c + C, ...  For every
+// slot it stages the chunk's K and V, and for each head h computes the fusion
+// logit z = scale * q_h . l_k and the chunk output o (softmax inside the
+// chunk).  Across its slots a block keeps per head the running maximum m,
+// the sum Z of exp(z - m) and acc = sum of exp(z - m) * o, so that the
+// fusion softmax over the K slots is exact once the C partial states are
+// combined: O = sum_c exp(m_c - M) acc_c / sum_c exp(m_c - M) Z_c, M = max m_c.
+// The blocks combine through distributed shared memory, each writing its
+// share of O, in a fixed order (deterministic).
+constexpr int kAttThreads = 256;
+constexpr int kAttWarps = kAttThreads / 32;
+constexpr int kAttMaxCluster = 8;
+
+// R consecutive elements of a shared-memory row as fp32, one load instruction.
+template <typename T, int R>
+__device__ __forceinline__ void load_row_slice(const T *p, float (&v)[R]);
+template <>
+__device__ __forceinline__ void load_row_slice<__nv_bfloat16, 4>(const __nv_bfloat16 *p, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+template <>
+__device__ __forceinline__ void load_row_slice<__nv_bfloat16, 2>(const __nv_bfloat16 *p, float (&v)[2]) {
+    const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+    v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xffff0000u);
+}
+template <>
+__device__ __forceinline__ void load_row_slice<float, 4>(const float *p, float (&v)[4]) {
+    const float4 u = *reinterpret_cast<const float4 *>(p);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+}
+template <>
+__device__ __forceinline__ void load_row_slice<float, 2>(const float *p, float (&v)[2]) {
+    const float2 u = *reinterpret_cast<const float2 *>(p);
+    v[0] = u.x; v[1] = u.y;
+}
+
+template <typename T, int D>
+struct AttSmem {
+    static constexpr int VT = Vec16<T>::N;
+    static constexpr int RS = D + VT;                       // padded K/V row (elements)
+    // fp32 q [G][D], acc [G][D], m [16], Z [16], lrow [D], p [warps][64], then the
+    // K and V tiles; every region starts on a 16-byte boundary (G <= 16, D % 64 == 0)
+    static size_t bytes(int G) {
+        return sizeof(float) * (2 * (size_t)G * D + 2 * 16 + D + kAttWarps * 64) +
+               2 * sizeof(T) * 64 * RS;
+    }
+};
+
+template <typename T, typename TL, int D>
+__global__ void __launch_bounds__(kAttThreads)
+decode_attend_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T *__restrict__ Kc,
+                     const T *__restrict__ Vc, int H, int Hkv, int64_t Lc, int S, int topk,
+                     float scale, const int32_t *__restrict__ sel, T *__restrict__ O) {
+    constexpr int VT = AttSmem<T, D>::VT;
+    constexpr int RS = AttSmem<T, D>::RS;
+    constexpr int R = D / 32;
+    constexpr int VPR = D / VT;                              // 16-byte vectors per K/V row
+    constexpr int NV = 64 * VPR / kAttThreads;               // vectors per thread, K and V each
+    constexpr int LV = D * (int)sizeof(TL) / 16;             // 16-byte vectors per landmark row
+    static_assert(NV >= 1 && (64 * VPR) % kAttThreads == 0, "K/V tile must split over threads");
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ float4 dyn4[];
+    const int C = (int)cluster.num_blocks();
+    const int crank = (int)cluster.block_rank();
+    const int64_t bg = blockIdx.y;
+    const int64_t b = bg / Hkv;
+    const int g = (int)(bg % Hkv);
+    const int G = H / Hkv;
+    const int64_t Nc = Lc / S;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *qs = reinterpret_cast<float *>(dyn4);                  // [G][D]
-    T *ks = reinterpret_cast<T *>(qs + G * D);                    // [64][RS]
+    float *acc_s = qs + G * D;                                    // [G][D]
+    float *m_s = acc_s + G * D;                                   // [G], 16 reserved
+    float *z_s = m_s + 16;                                        // [G], 16 reserved
+    float *lrow = z_s + 16;                                       // [D]
+    float *ps = lrow + D;                                         // [warps][64]
+    T *ks = reinterpret_cast<T *>(ps + kAttWarps * 64);           // [64][RS]
     T *vs = ks + 64 * RS;
-    for (int e = tid; e < G * D; e += kDecThreads) qs[e] = to_f32(q[(b * H + g * G) * D + e]);
-    __syncthreads();
-    // fusion weights per head over the selection
-    for (int h = warp; h < G; h += kDecWarps) {
-        float s[32];
-        float mx = -INFINITY;
-        for (int k = 0; k < topk; ++k) {
-            const int32_t i = sel_s[k];
-            float a = 0.f;
-            if (i >= 0) {
-                const TL *lp = lm_bg + (int64_t)i * D;
-                for (int j = lane; j < D; j += 32) a = fmaf(qs[h * D + j], to_f32(lp[j]), a);
+
+    // the queries are an input: load them before waiting for the scan
+    {
+        const T *qg = q + (b * H + g * G) * (int64_t)D;
+        for (int e = tid; e < G * VPR; e += kAttThreads) {
+            float f[VT];
+            Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(qg + e * VT), f);
+#pragma unroll
+            for (int u = 0; u < VT; ++u) qs[e * VT + u] = f[u];
+        }
+        for (int e = tid; e < G * D; e += kAttThreads) acc_s[e] = 0.f;
+        for (int e = tid; e < G; e += kAttThreads) {
+            m_s[e] = -INFINITY;
+            z_s[e] = 0.f;
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the selection is written by the scan
+
+    for (int k = crank; k < topk; k += C) {
+        const int32_t ci = sel[bg * topk + k];
+        if (ci < 0) break;                     // padding only at the end of the selection
+        __syncthreads();                       // previous slot's tiles are no longer read
+        {
+            const int64_t first = (int64_t)ci * S;
+            const T *Kb = Kc + (bg * Lc + first) * D;
+            const T *Vb = Vc + (bg * Lc + first) * D;
+            uint4 kr[NV], vr[NV];
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int e = tid + u * kAttThreads;
+                kr[u] = ld_stream16(Kb + (int64_t)e * VT);
+                vr[u] = ld_stream16(Vb + (int64_t)e * VT);
             }
+            uint4 lr = make_uint4(0, 0, 0, 0);
+            const TL *lp = lm + (bg * Nc + ci) * D;
+            if (tid < LV)
+                lr = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(lp) + tid * 16);
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int e = tid + u * kAttThreads;
+                const int r = e / VPR, c = (e % VPR) * VT;
+                *reinterpret_cast<uint4 *>(ks + r * RS + c) = kr[u];
+                *reinterpret_cast<uint4 *>(vs + r * RS + c) = vr[u];
+            }
+            if (tid < LV) {
+                constexpr int LE = Vec16<TL>::N;
+                float f[LE];
+                Vec16<TL>::unpack(lr, f);
+#pragma unroll
+                for (int u = 0; u < LE; ++u) lrow[tid * LE + u] = f[u];
+            }
+        }
+        __syncthreads();
+        for (int h = warp; h < G; h += kAttWarps) {
+            const float *qh = qs + h * D;
+            // fusion logit scale * q_h . l_ci
+            float a = 0.f;
+#pragma unroll
+            for (int r = 0; r < R; ++r) a = fmaf(qh[lane + 32 * r], lrow[lane + 32 * r], a);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            s[k & 31] = i >= 0 ? scale * a : -INFINITY;
-            mx = fmaxf(mx, s[k & 31]);
-        }
-        float den = 0.f;
-        for (int k = 0; k < topk; ++k) {
-            s[k] = sel_s[k] >= 0 ? expf(s[k] - mx) : 0.f;
-            den += s[k];
-        }
-        if (lane == 0)
-            for (int k = 0; k < topk; ++k) wsel[h][k] = den > 0.f ? s[k] / den : 0.f;
-    }
-    float acc[2][R];
+            const float zl = scale * a;
+            // in-chunk scores: lane takes keys lane and lane + 32, two partial sums each
+            float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll 2
+            for (int c = 0; c < D / 2; c += VT) {
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[hh][r] = 0.f;
-    const T *Kbg = Kc + bg * Lc * D;
-    const T *Vbg = Vc + bg * Lc * D;
-    for (int k = 0; k < topk; ++k) {
-        const int32_t ci = sel_s[k];
-        if (ci < 0) continue;
-        __syncthreads();
-        const int64_t first = (int64_t)ci * S;
-        for (int e = tid; e < S * (D / VT); e += kDecThreads) {
-            const int r = e / (D / VT), c = (e % (D / VT)) * VT;
-            *reinterpret_cast<uint4 *>(ks + r * RS + c) = ld_stream16(Kbg + (first + r) * D + c);
-            *reinterpret_cast<uint4 *>(vs + r * RS + c) = ld_stream16(Vbg + (first + r) * D + c);
-        }
-        __syncthreads();
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int cc = c + hf * (D / 2);
+                        float f[VT];
+                        Vec16<T>::unpack(
+                            *reinterpret_cast<const uint4 *>(ks + (lane + 32 * u) * RS + cc), f);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = warp + hh * kDecWarps;
-            if (h >= G) break;
-            const float *qh = qs + h * D;
-            float lg[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int j = lane + 32 * u;
-                float a = 0.f;
-#pragma unroll 4
-                for (int c = 0; c < D; c += VT) {
-                    float f[VT];
-                    Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(ks + j * RS + c), f);
-#pragma unroll
-                    for (int e = 0; e < VT; ++e) a = fmaf(qh[c + e], f[e], a);
-                }
-                lg[u] = scale * a;
+                        for (int e = 0; e < VT; ++e) sc[u][hf] = fmaf(qh[cc + e], f[e], sc[u][hf]);
+                    }
             }
-            float mx = fmaxf(lg[0], lg[1]);
+            const float l0 = scale * (sc[0][0] + sc[0][1]), l1 = scale * (sc[1][0] + sc[1][1]);
+            float mx = fmaxf(l0, l1);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            float p0 = expf(lg[0] - mx), p1 = expf(lg[1] - mx);
+            const float p0 = expf(l0 - mx), p1 = expf(l1 - mx);
             float den = p0 + p1;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+            float *pw = ps + warp * 64;
+            pw[lane] = p0;
+            pw[lane + 32] = p1;
+            __syncwarp();
+            // P.V: lane owns the R consecutive elements R*lane .. R*lane + R - 1
             float o_r[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) o_r[r] = 0.f;
+#pragma unroll 8
             for (int j = 0; j < 64; ++j) {
-                const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
+                const float pj = pw[j];
+                float v[R];
+                load_row_slice<T, R>(vs + j * RS + R * lane, v);
 #pragma unroll
-                for (int r = 0; r < R; ++r)
-                    o_r[r] = fmaf(pj, to_f32(vs[j * RS + lane + 32 * r]), o_r[r]);
+                for (int r = 0; r < R; ++r) o_r[r] = fmaf(pj, v[r], o_r[r]);
             }
-            const float f = wsel[h][k] / den;
+            __syncwarp();
+            // fold (zl, o / den) into this block's running fusion state of head h
+            const float m_old = m_s[h];
+            const float m_new = fmaxf(m_old, zl);
+            const float c_old = expf(m_old - m_new);          // 0 while the state is empty
+            const float c_new = expf(zl - m_new);
+            const float f = c_new / den;
+            float *ah = acc_s + h * D + R * lane;
 #pragma unroll
-            for (int r = 0; r < R; ++r) acc[hh][r] = fmaf(f, o_r[r], acc[hh][r]);
+            for (int r = 0; r < R; ++r) ah[r] = ah[r] * c_old + o_r[r] * f;
+            __syncwarp();
+            if (lane == 0) {
+                z_s[h] = z_s[h] * c_old + c_new;
+                m_s[h] = m_new;
+            }
+            __syncwarp();
         }
     }
+
+    // combine the C block states of this (b, g); block c writes heads c, c + C, ...
+    // (all remote loads of a head are issued before any is used)
+    cluster.sync();
+    for (int h = crank + C * warp; h < G; h += C * kAttWarps) {
+        float mr[kAttMaxCluster], zr[kAttMaxCluster];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int h = warp + hh * kDecWarps;
-        if (h >= G) break;
-        T *op = O + (b * H + g * G + h) * (int64_t)D;
+        for (int r = 0; r < kAttMaxCluster; ++r) {
+            mr[r] = r < C ? cluster.map_shared_rank(m_s, r)[h] : -INFINITY;
+            zr[r] = r < C ? cluster.map_shared_rank(z_s, r)[h] : 0.f;
+        }
+        float ar[kAttMaxCluster][R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) op[lane + 32 * r] = from_f32<T>(acc[hh][r]);
+        for (int r = 0; r < kAttMaxCluster; ++r)
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+                ar[r][i] = r < C ? cluster.map_shared_rank(acc_s, r)[h * D + R * lane + i] : 0.f;
+        float M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kAttMaxCluster; ++r) M = fmaxf(M, mr[r]);
+        float Z = 0.f;
+        float o_r[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) o_r[i] = 0.f;
+#pragma unroll
+        for (int r = 0; r < kAttMaxCluster; ++r) {
+            const float cr = mr[r] > -INFINITY ? expf(mr[r] - M) : 0.f;   // 0: block had no slot
+            Z = fmaf(zr[r], cr, Z);
+#pragma unroll
+            for (int i = 0; i < R; ++i) o_r[i] = fmaf(ar[r][i], cr, o_r[i]);
+        }
+        const float inv = Z > 0.f ? 1.f / Z : 0.f;
+        T *op = O + (b * H + g * G + h) * (int64_t)D + R * lane;
+#pragma unroll
+        for (int i = 0; i < R; ++i) op[i] = from_f32<T>(o_r[i] * inv);
     }
+    cluster.sync();          // no block leaves while another still reads its state
 }
 
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms) {
     const int64_t pairs = (int64_t)B * Hkv;
-    int64_t s = (4LL * num_sms + pairs - 1) / pairs;
+    int64_t s = ((int64_t)kScanBlocksPerSm * num_sms + pairs - 1) / pairs;
     const int64_t max_s = (Nc + 255) / 256;          // at least 256 rows per split
     if (s > max_s) s = max_s;
     if (s < 1) s = 1;
@@ -270,35 +478,53 @@ int decode_splits(int B, int Hkv, int64_t Nc, int num_sms) {
     return (int)s;
 }
 
-size_t decode_dyn_smem(int G, int d, bool bf16) {
-    const int vt = bf16 ? 8 : 4;
-    const size_t el = bf16 ? 2 : 4;
-    return sizeof(float) * (size_t)G * d + 2 * el * 64 * (size_t)(d + vt);
-}
-
 template <typename T, typename TL, int D>
 static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc, const void *Vc,
                                    int B, int H, int Hkv, int64_t Lc, int S, int topk,
-                                   float scale, int splits, uint64_t *cand, unsigned *tickets,
-                                   void *O, int32_t *idx_out, cudaStream_t st) {
-    const size_t smem = decode_dyn_smem(H / Hkv, D, sizeof(T) == 2);
-    auto kern = decode_kernel<T, TL, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
+                                   float scale, int splits, const DecodeScratch &ws, void *O,
+                                   int32_t *idx_out, cudaStream_t st) {
+    const int64_t Nc = Lc / S;
     dim3 grid((unsigned)splits, (unsigned)(B * Hkv));
-    kern<<<grid, kDecThreads, smem, st>>>((const T *)q, (const TL *)lm, (const T *)Kc,
-                                          (const T *)Vc, H, Hkv, Lc, S, topk, scale, splits, cand,
-                                          tickets, (T *)O, idx_out);
-    return cudaGetLastError();
+    auto scan = decode_scan_kernel<T, TL, D>;
+    cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kScanStages * kStageBytes);
+    if (e != cudaSuccess) return e;
+    scan<<<grid, kScanThreads, kScanStages * kStageBytes, st>>>(
+        (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws.cand, ws.tickets,
+        ws.sel, idx_out, ws.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    const size_t smem = AttSmem<T, D>::bytes(H / Hkv);
+    auto kern = decode_attend_kernel<T, TL, D>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int C = topk < kAttMaxCluster ? topk : kAttMaxCluster;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C, (unsigned)(B * Hkv));
+    cfg.blockDim = dim3(kAttThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, (const T *)q, (const TL *)lm, (const T *)Kc,
+                              (const T *)Vc, H, Hkv, Lc, S, topk, scale, (const int32_t *)ws.sel,
+                              (T *)O);
 }
 
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
                           const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
-                          int S, int topk, float scale, int splits, uint64_t *cand,
-                          unsigned *tickets, void *O, int32_t *idx_out, cudaStream_t st) {
+                          int S, int topk, float scale, int splits, const DecodeScratch &ws,
+                          void *O, int32_t *idx_out, cudaStream_t st) {
 #define HSA_DEC(T, TL, DD) \
-    return launch_decode_t<T, TL, DD>(q, lm, Kc, Vc, B, H, Hkv, Lc, S, topk, scale, splits, cand, tickets, O, idx_out, st)
+    return launch_decode_t<T, TL, DD>(q, lm, Kc, Vc, B, H, Hkv, Lc, S, topk, scale, splits, ws, O, idx_out, st)
     using bf = __nv_bfloat16;
     if (bf16) {
         if (lm_bf16) { if (d == 128) HSA_DEC(bf, bf, 128); HSA_DEC(bf, bf, 64); }

@@ -110,7 +110,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
  * hsa_decode_workspace_size -- bytes of device workspace hsa_decode needs
  * (0 on invalid arguments; the size depends on the current device's SM
  * count).  It holds per-(sequence, group) tickets, the per-block candidate
- * lists and a status word.  A new workspace must be zero-filled once before
+ * lists, the selection and a status word.  A new workspace must be zero-filled once before
  * its first use; every completed call leaves the tickets at zero again.
  * Calls that share a workspace must be ordered (same stream).
  */
@@ -126,9 +126,12 @@ size_t hsa_decode_workspace_size(int B, int H, int Hkv, int64_t Lc, int d, int S
  *   lm       [B, Hkv, Lc/S, d]  lm_dt (bf16 or fp32)
  *   O        [B, H, d]          dt, written
  *   idx_out  [B, Hkv, topk] int32 or NULL
- * The landmark scan is split over many thread blocks; the last block of each
- * (sequence, KV group) merges the partial top-K lists, gathers the selected
- * chunks and writes O.  Cache offsets are 64-bit (Lc up to 2^31 - 1 tokens).
+ * Two kernels: the landmark scan is split over many thread blocks and the
+ * last block of each (sequence, KV group) merges their top-K lists into the
+ * selection; then a cluster of min(topk, 8) blocks per (sequence, group)
+ * gathers the selected chunks, attends inside them and fuses the results into
+ * O (launched as a programmatic dependent of the scan).  Cache offsets are
+ * 64-bit (Lc up to 2^31 - 1 tokens).
  */
 hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
                         const void *lm, hsa_dtype_t lm_dt,
