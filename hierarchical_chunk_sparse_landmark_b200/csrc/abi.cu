@@ -156,14 +156,16 @@ bool force_simt_path() {
     return v && strcmp(v, "simt") == 0;
 }
 
-// Decode workspace: status | tickets (the zeroed head) | sel | cand.
+// Decode workspace: status | tickets | unit counters (the zeroed head) | sel | cand.
 struct DecodeLayout {
     size_t sel_off, cand_off, total;
+    int64_t pairs;
     int splits;
     DecodeScratch at(char *ws) const {
         DecodeScratch s;
         s.status = (unsigned *)ws;
         s.tickets = (unsigned *)(ws + kStatusBytes);
+        s.next_unit = s.tickets + pairs;
         s.sel = (int32_t *)(ws + sel_off);
         s.cand = (uint64_t *)(ws + cand_off);
         return s;
@@ -174,6 +176,7 @@ DecodeLayout decode_layout(int B, int Hkv, int64_t Lc, int S, int topk) {
     DecodeLayout p;
     const int64_t Nc = Lc / S;
     const size_t pairs = (size_t)B * Hkv;
+    p.pairs = (int64_t)pairs;
     p.splits = decode_splits(B, Hkv, Nc, num_sms());
     size_t off = decode_zero_head(B, Hkv);
     p.sel_off = off;

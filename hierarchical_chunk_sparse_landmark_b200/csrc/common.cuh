@@ -155,6 +155,42 @@ __device__ __forceinline__ uint64_t warp_select_topk(uint64_t (&x)[M], int topk)
     return out;
 }
 
+// Sorted-list merging.  A warp register holds 32/KP lists (KP a power of two):
+// lanes s*KP .. s*KP + KP - 1 hold list s in descending order (0 = empty).
+// merge_lists returns, in the same layout, the KP best keys of the union of
+// list s of `a` and list s of `b`: the element-wise maximum of a and b reversed
+// is a bitonic sequence holding exactly those keys, and log2(KP) half-cleaner
+// steps sort it.
+__device__ __forceinline__ uint64_t merge_lists(uint64_t a, uint64_t b, int KP) {
+    const int lane = threadIdx.x & 31;
+    const int i = lane & (KP - 1);
+    const uint64_t br = __shfl_sync(0xffffffffu, b, lane - i + (KP - 1 - i));
+    uint64_t v = a > br ? a : br;
+    for (int j = KP >> 1; j > 0; j >>= 1) {
+        const uint64_t p = __shfl_xor_sync(0xffffffffu, v, j);
+        v = (i & j) ? (v < p ? v : p) : (v > p ? v : p);
+    }
+    return v;
+}
+// Merge the 32/KP lists of one register into one (returned in every segment).
+__device__ __forceinline__ uint64_t merge_segments(uint64_t v, int KP) {
+    for (int m = KP; m < 32; m <<= 1) v = merge_lists(v, __shfl_xor_sync(0xffffffffu, v, m), KP);
+    return v;
+}
+// Merge the lists of registers x[0 .. nr-1] (nr <= 8, warp-uniform) as a
+// tree: the merges of one level are independent, so their shuffles overlap.
+__device__ __forceinline__ uint64_t merge_regs8(uint64_t (&x)[8], int nr, int KP) {
+#pragma unroll
+    for (int w = 1; w < 8; w <<= 1)
+#pragma unroll
+        for (int i = 0; i + w < 8; i += 2 * w)
+            if (i + w < nr) x[i] = merge_lists(x[i], x[i + w], KP);
+    return x[0];
+}
+__host__ __device__ constexpr int pow2_at_least(int k) {
+    return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : k <= 8 ? 8 : k <= 16 ? 16 : 32;
+}
+
 // ---------------------------------------------------------------- status word
 // The first 256 bytes of every workspace.  word[0] = error flags set by kernels
 // (bit 0: a bounded wait gave up).
@@ -163,18 +199,20 @@ constexpr unsigned kFlagTimeout = 1u;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Decode scratch inside the caller's workspace.  The ticket array sits right
-// after the status word and must start at zero (the kernels leave it at
-// zero); everything else is rewritten by every call.
+// Decode scratch inside the caller's workspace.  The ticket and unit-counter
+// arrays sit right after the status word and must start at zero (the kernels
+// leave them at zero); everything else is rewritten by every call.
 struct DecodeScratch {
     unsigned *status;     // status word
     unsigned *tickets;    // [B*Hkv] scan blocks done
+    unsigned *next_unit;  // [B*Hkv] next landmark unit to hand out
     int32_t *sel;         // [B*Hkv*topk] selected chunks
     uint64_t *cand;       // [B*Hkv*splits*topk] per-block candidate keys
 };
-// Bytes at the head of a decode workspace that must be zero before a call.
+// Bytes at the head of a decode workspace that must be zero before a call
+// (status word, tickets, unit counters).
 __host__ __device__ constexpr size_t decode_zero_head(int64_t B, int64_t Hkv) {
-    return align_up(kStatusBytes + sizeof(unsigned) * (size_t)(B * Hkv), 256);
+    return align_up(kStatusBytes + 2 * sizeof(unsigned) * (size_t)(B * Hkv), 256);
 }
 
 }  // namespace hsa

@@ -42,14 +42,34 @@ constexpr int kStageBytes = 16384;
 constexpr int kScanBlocksPerSm = 3;            // 64 KB ring + ~3 KB per block
 constexpr long long kScanWait = 4000000000LL;  // SM cycles (about 2 s)
 
+// Top-K of `nlists` (<= 8 * 32 / KP) sorted lists of KP keys held in shared
+// memory (list l = lists[l][0 .. KP-1]); executed by one warp, lane k < KP
+// returns the k-th best.
+__device__ __forceinline__ uint64_t merge_smem_lists(const uint64_t (*lists)[32], int nlists,
+                                                     int KP) {
+    const int lane = threadIdx.x & 31;
+    const int per = 32 / KP, li = lane / KP, e = lane % KP;
+    const int nr = (nlists + per - 1) / per;
+    uint64_t x[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int l = r * per + li;
+        x[r] = (r < nr && l < nlists) ? lists[l][e] : 0ull;
+    }
+    return merge_segments(merge_regs8(x, nr, KP), KP);
+}
+
+// Grid: splits * B*Hkv blocks, 1-D, interleaved over (b, g) so that the blocks
+// of every (b, g) spread over all SMs.  Work is handed out in units of one
+// ring stage (ROWS landmark rows) from a per-(b, g) counter, so that blocks on
+// SMs that stream faster take more units.
 template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kScanThreads)
-decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, int Hkv, int64_t Nc,
-                   int topk, float scale, int splits, uint64_t *__restrict__ cand,
-                   unsigned *__restrict__ tickets, int32_t *__restrict__ sel_out,
-                   int32_t *__restrict__ idx_out, unsigned *__restrict__ status) {
+decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T *__restrict__ Kc,
+                   const T *__restrict__ Vc, int H, int Hkv, int64_t Nc, int S, int topk,
+                   float scale, int splits, DecodeScratch ws, int32_t *__restrict__ idx_out) {
     constexpr int ROW_BYTES = D * (int)sizeof(TL);
-    constexpr int ROWS = kStageBytes / ROW_BYTES;           // landmark rows per stage
+    constexpr int ROWS = kStageBytes / ROW_BYTES;           // landmark rows per stage (one unit)
     constexpr int VEC = Vec16<TL>::N;                        // elements per 16-byte vector
     constexpr int LPR = 8;                                   // lanes per row (one quarter-warp)
     constexpr int VPL = D / VEC / LPR;                       // 16-byte vectors per lane and row
@@ -59,21 +79,21 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
 
     extern __shared__ __align__(128) uint8_t ring[];         // [kScanStages][kStageBytes]
     __shared__ uint64_t full[kScanStages], empty[kScanStages];
+    __shared__ int64_t unit_of[kScanStages];                 // -1: no more units
     __shared__ float qbar_s[D];
     __shared__ uint64_t lists[kScanWarps][32];
     __shared__ int is_last, s_abort;
 
-    const int split = blockIdx.x;
-    const int64_t bg = blockIdx.y;
+    const int64_t pairs = (int64_t)gridDim.x / splits;
+    const int64_t bg = blockIdx.x % pairs;
+    const int split = (int)(blockIdx.x / pairs);
     const int64_t b = bg / Hkv;
     const int g = (int)(bg % Hkv);
     const int G = H / Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t r0 = (int64_t)split * Nc / splits;
-    const int64_t r1 = (int64_t)(split + 1) * Nc / splits;
-    const int64_t nrows = r1 - r0;
-    const int64_t nst = (nrows + ROWS - 1) / ROWS;
+    const int64_t nunits = (Nc + ROWS - 1) / ROWS;
     const TL *lm_bg = lm + bg * Nc * D;
+    const int KP = pow2_at_least(topk);
 
     if (tid == 0) {
         for (int i = 0; i < kScanStages; ++i) {
@@ -89,10 +109,13 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
     tk.init(topk);
     uint64_t thr = 0ull;
     if (warp == kScanWarps) {
-        // producer: one elected lane keeps kScanStages bulk copies in flight
+        // producer: one lane claims units (one claim ahead, so the atomic's
+        // latency overlaps the wait for a free slot) and keeps kScanStages
+        // bulk copies in flight; a unit of -1 tells the consumers to stop
         if (lane == 0) {
-            int64_t issued = 0;
-            for (int64_t st = 0; st < nst; ++st) {
+            int64_t u_next = (int64_t)atomicAdd(ws.next_unit + bg, 1u);
+            int64_t st = 0;
+            for (;; ++st) {
                 const int slot = (int)(st % kScanStages);
                 if (st >= kScanStages &&
                     !tc::mbar_wait(&empty[slot], (uint32_t)(((st / kScanStages) - 1) & 1),
@@ -100,15 +123,23 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
                     s_abort = 1;
                     break;
                 }
-                const int64_t left = nrows - st * ROWS;
+                const int64_t u = u_next;
+                if (u >= nunits) {
+                    unit_of[slot] = -1;
+                    tc::mbar_arrive(&full[slot]);
+                    ++st;
+                    break;
+                }
+                u_next = (int64_t)atomicAdd(ws.next_unit + bg, 1u);
+                const int64_t row0 = u * ROWS;
+                const int64_t left = Nc - row0;
                 const uint32_t bytes = (uint32_t)((left < ROWS ? left : ROWS) * ROW_BYTES);
+                unit_of[slot] = u;
                 tc::mbar_expect_tx(&full[slot], bytes);
-                tc::bulk_load(ring + slot * kStageBytes, lm_bg + (r0 + st * ROWS) * D, bytes,
-                              &full[slot]);
-                issued = st + 1;
+                tc::bulk_load(ring + slot * kStageBytes, lm_bg + row0 * D, bytes, &full[slot]);
             }
             // the copies still in flight land before the block can exit
-            for (int64_t j = issued > kScanStages ? issued - kScanStages : 0; j < issued; ++j)
+            for (int64_t j = st > kScanStages ? st - kScanStages : 0; j < st; ++j)
                 tc::mbar_wait(&full[j % kScanStages], (uint32_t)((j / kScanStages) & 1), kScanWait);
         }
     } else {
@@ -134,13 +165,16 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
                 q2[j][e] = pack_f2(scale * qp[0], scale * qp[1]);
             }
         float tf = -INFINITY;          // score of the K-th best key so far
-        for (int64_t st = 0; st < nst; ++st) {
+        for (int64_t st = 0;; ++st) {
             const int slot = (int)(st % kScanStages);
             if (!tc::mbar_wait(&full[slot], (uint32_t)((st / kScanStages) & 1), kScanWait)) {
                 s_abort = 1;
                 break;
             }
-            const int rows_here = (int)(nrows - st * ROWS < ROWS ? nrows - st * ROWS : ROWS);
+            const int64_t unit = unit_of[slot];
+            if (unit < 0) break;
+            const int64_t row0 = unit * ROWS;
+            const int rows_here = (int)(Nc - row0 < ROWS ? Nc - row0 : ROWS);
             const uint8_t *stage = ring + slot * kStageBytes;
 #pragma unroll
             for (int it = 0; it < ITER; ++it) {
@@ -158,7 +192,7 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
                 // cheap float filter; ties and the exact order are settled on the keys
                 unsigned m = __ballot_sync(0xffffffffu, a >= tf && rr < rows_here) & 0x01010101u;
                 if (m) {
-                    const uint64_t key = make_key(a, r0 + st * ROWS + rr);
+                    const uint64_t key = make_key(a, row0 + rr);
                     while (m) {
                         const int s = __ffs(m) - 1;
                         m &= m - 1;
@@ -180,51 +214,55 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
     if (warp < kScanWarps) lists[warp][lane] = tk.v;
     __syncthreads();
     if (warp == 0) {
-        uint64_t x[kScanWarps];
-#pragma unroll
-        for (int w2 = 0; w2 < kScanWarps; ++w2) x[w2] = lists[w2][lane];
-        const uint64_t best = warp_select_topk(x, topk);
-        if (lane < topk) cand[(bg * splits + split) * topk + lane] = best;
+        const uint64_t best = merge_smem_lists(lists, kScanWarps, KP);
+        if (lane < topk) ws.cand[(bg * splits + split) * topk + lane] = best;
+        __threadfence();                      // the candidates before the ticket
     }
-    if (s_abort && tid == 0) atomicOr(status, kFlagTimeout);
+    if (s_abort && tid == 0) atomicOr(ws.status, kFlagTimeout);
 
-    // last block of this (b, g) merges the candidates of every split
-    __threadfence();
+    // last block of this (b, g) merges the candidates of every block
     __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(&tickets[bg], 1u) == (unsigned)(splits - 1));
+    if (tid == 0) is_last = (atomicAdd(&ws.tickets[bg], 1u) == (unsigned)(splits - 1));
     __syncthreads();
     if (!is_last || warp >= kScanWarps) return;
     __threadfence();
-    // each consumer warp reduces its share of the candidates to a top-K, 256 at a time
-    const int64_t ncand = (int64_t)splits * topk;
-    const int64_t per = (ncand + kScanWarps - 1) / kScanWarps;
-    const int64_t w0 = warp * per, w1 = w0 + per < ncand ? w0 + per : ncand;
-    const uint64_t *cb = cand + bg * ncand;
-    uint64_t mine = 0ull;
-    for (int64_t c0 = w0; c0 < w1; c0 += 8 * 32) {
-        uint64_t x[9];
+    // each consumer warp merges groups of 32/KP block lists (warp w: groups
+    // w, w + 8, ...), eight groups per load batch, merged as a tree
+    const uint64_t *cb = ws.cand + bg * splits * topk;
+    const int per = 32 / KP, li = lane / KP, e = lane % KP;
+    const int64_t ngroups = (splits + per - 1) / per;
+    uint64_t acc = 0ull;
+    for (int64_t g0 = warp; g0 < ngroups; g0 += 8 * kScanWarps) {
+        uint64_t x[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int64_t i = c0 + m * 32 + lane;
-            x[m] = i < w1 ? (uint64_t)__ldcg(reinterpret_cast<const unsigned long long *>(cb + i))
-                          : 0ull;
+        for (int u = 0; u < 8; ++u) {
+            const int64_t gi = g0 + (int64_t)u * kScanWarps;
+            const int64_t l = gi * per + li;
+            x[u] = (gi < ngroups && l < splits && e < topk)
+                       ? (uint64_t)__ldcg(reinterpret_cast<const unsigned long long *>(cb + l * topk + e))
+                       : 0ull;
         }
-        x[8] = mine;
-        mine = warp_select_topk(x, topk);
+        acc = merge_lists(acc, merge_regs8(x, 8, KP), KP);
     }
-    lists[warp][lane] = mine;
+    lists[warp][lane] = merge_segments(acc, KP);
     asm volatile("bar.sync 1, %0;" ::"n"(kScanWarps * 32) : "memory");
     if (warp == 0) {
-        uint64_t x[kScanWarps];
-#pragma unroll
-        for (int w2 = 0; w2 < kScanWarps; ++w2) x[w2] = lists[w2][lane];
-        const uint64_t best = warp_select_topk(x, topk);
+        const uint64_t best = merge_smem_lists(lists, kScanWarps, KP);
         if (lane < topk) {
             const int32_t i = key_index(best);
-            sel_out[bg * topk + lane] = i;
+            ws.sel[bg * topk + lane] = i;
             if (idx_out) idx_out[bg * topk + lane] = i;
+            if (i >= 0) {                     // warm L2 with the chunks the attend kernel reads
+                const size_t off = ((size_t)bg * Nc * S + (size_t)i * S) * D;
+                const uint32_t bytes = (uint32_t)(S * D * sizeof(T));
+                tc::prefetch_l2(Kc + off, bytes);
+                tc::prefetch_l2(Vc + off, bytes);
+            }
         }
-        if (lane == 0) tickets[bg] = 0u;        // ready for the next call
+        if (lane == 0) {                      // ready for the next call
+            ws.tickets[bg] = 0u;
+            ws.next_unit[bg] = 0u;
+        }
     }
 }
 
@@ -468,13 +506,14 @@ decode_attend_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T
     cluster.sync();          // no block leaves while another still reads its state
 }
 
+// Blocks per (b, g): as many as fit in one wave (kScanBlocksPerSm per SM),
+// at least one, and no more than one per 256 landmark rows.
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms) {
     const int64_t pairs = (int64_t)B * Hkv;
-    int64_t s = ((int64_t)kScanBlocksPerSm * num_sms + pairs - 1) / pairs;
-    const int64_t max_s = (Nc + 255) / 256;          // at least 256 rows per split
+    int64_t s = (int64_t)kScanBlocksPerSm * num_sms / pairs;
+    const int64_t max_s = (Nc + 255) / 256;
     if (s > max_s) s = max_s;
     if (s < 1) s = 1;
-    if (s > 65535) s = 65535;
     return (int)s;
 }
 
@@ -484,14 +523,14 @@ static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc
                                    float scale, int splits, const DecodeScratch &ws, void *O,
                                    int32_t *idx_out, cudaStream_t st) {
     const int64_t Nc = Lc / S;
-    dim3 grid((unsigned)splits, (unsigned)(B * Hkv));
+    const unsigned grid = (unsigned)((int64_t)splits * B * Hkv);
     auto scan = decode_scan_kernel<T, TL, D>;
     cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kScanStages * kStageBytes);
     if (e != cudaSuccess) return e;
     scan<<<grid, kScanThreads, kScanStages * kStageBytes, st>>>(
-        (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws.cand, ws.tickets,
-        ws.sel, idx_out, ws.status);
+        (const T *)q, (const TL *)lm, (const T *)Kc, (const T *)Vc, H, Hkv, Nc, S, topk, scale,
+        splits, ws, idx_out);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 

@@ -8,12 +8,11 @@
 // cudaMalloc/cudaFree because they can synchronise the device.  Such a caller
 // cannot provide the workspace hsa_decode asks for.
 //
-// What it does instead: the decode scratch (per-(sequence, KV group) tickets,
-// candidate lists and the selection) lives in one
+// What it does instead: the decode scratch (per-(sequence, KV group) tickets
+// and work counters, candidate lists and the selection) lives in one
 // fixed-size array in device global memory that belongs to this library.
-// The array is declared at file
-// scope below, so every GPU that loads the library holds it until the process
-// exits.  Host code cannot use the array's name as a device address (on the
+// The array is declared at file scope below, so every GPU that loads the
+// library holds it until the process exits.  Host code cannot use the array's name as a device address (on the
 // host it names a stand-in), so the device address is looked up once per
 // device with cudaGetSymbolAddress and handed to the kernel.
 #include <mutex>
@@ -66,10 +65,10 @@ extern "C" hsa_status_t hsa_decode_noalloc(const void *q, const void *Kc, const 
     const hsa_status_t s = scratch_address(&scratch);
     if (s != HSA_OK) return s;
     {
-        // The status word and the ticket array (the head of the decode
-        // scratch) must start at zero; the rest is fully rewritten by every
-        // call.  The array keeps the previous call's contents, so the head is
-        // cleared here, on the caller's stream.
+        // The status word, the tickets and the work counters (the head of the
+        // decode scratch) must start at zero; the rest is fully rewritten by
+        // every call.  The array keeps the previous call's contents, so the
+        // head is cleared here, on the caller's stream.
         const size_t head = hsa::decode_zero_head(B, Hkv);
         const size_t clear = head < need ? head : need;
         if (cudaMemsetAsync(scratch, 0, clear, (cudaStream_t)stream) != cudaSuccess)
