@@ -26,15 +26,15 @@ int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
-                          int64_t *seg_start, cudaStream_t st);
+                          int64_t *seg_start, int4 *tiles, cudaStream_t st);
 struct TcLaunch {
     const void *Q, *K, *V, *lm;
     int B, H, Hkv, S, topk, own_chunk, lm_bf16;
     int64_t L, W, cap;
     float scale;
     const int32_t *idx, *entries;
-    const int4 *wtiles;
-    const int64_t *seg_start;
+    const int4 *tiles;                // one descriptor per queue position
+    const int64_t *qlen;              // number of tiles (device)
     float *logits, *w_out;
     __half *part, *own;
     void *O;
@@ -105,7 +105,7 @@ struct PrefillLayout {
     bool tc;
     int64_t W, NW, cap;
     size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
-        seg_off, part_off, own_off;
+        seg_off, tiles_off, part_off, own_off;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
@@ -121,7 +121,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     p.tc = tc_shape_ok(B, H, Hkv, L, d, topk);
     p.W = p.NW = p.cap = 0;
     p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
-    p.wntiles_off = p.done_off = p.seg_off = p.part_off = p.own_off = 0;
+    p.wntiles_off = p.done_off = p.seg_off = p.tiles_off = p.part_off = p.own_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
         p.W = tc_window(B, H, Hkv, L, d, topk, attend_tc_max_windows());
@@ -142,6 +142,8 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         off = align_up(off + sizeof(int32_t) * (size_t)p.NW, 256);
         p.seg_off = off;
         off = align_up(off + sizeof(int64_t) * (size_t)(2 * p.NW + 1), 256);
+        p.tiles_off = off;           // retrieved tiles + own-chunk tiles of every window
+        off = align_up(off + sizeof(int4) * (size_t)(p.NW * (p.cap + (p.W + ept - 1) / ept)), 256);
         p.part_off = off;
         off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
         p.own_off = off;
@@ -301,17 +303,17 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                           (int32_t *)(ws + lay.counts_off), (int32_t *)(ws + lay.cursor_off),
                           (int32_t *)(ws + lay.entries_off), (int4 *)(ws + lay.wtiles_off),
                           (int32_t *)(ws + lay.wntiles_off), (int32_t *)(ws + lay.done_off),
-                          (int64_t *)(ws + lay.seg_off), st);
+                          (int64_t *)(ws + lay.seg_off), (int4 *)(ws + lay.tiles_off), st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
-        t_launches += 4;
+        t_launches += 5;
         stage_mark(3, st);
         TcLaunch a;
         a.Q = Q; a.K = K; a.V = V; a.lm = lm_use; a.lm_bf16 = lm_bf16 ? 1 : 0;
         a.B = B; a.H = H; a.Hkv = Hkv; a.S = S; a.topk = topk; a.own_chunk = own_chunk;
         a.L = L; a.W = lay.W; a.cap = lay.cap; a.scale = scale;
         a.idx = idx; a.entries = (const int32_t *)(ws + lay.entries_off);
-        a.wtiles = (const int4 *)(ws + lay.wtiles_off);
-        a.seg_start = (const int64_t *)(ws + lay.seg_off);
+        a.tiles = (const int4 *)(ws + lay.tiles_off);
+        a.qlen = (const int64_t *)(ws + lay.seg_off) + 2 * lay.NW;
         a.logits = w_ws; a.w_out = w_out;
         a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;

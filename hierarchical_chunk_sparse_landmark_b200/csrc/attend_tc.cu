@@ -22,15 +22,20 @@
 //   w = softmax over the token's selected chunks of the logits,
 //   O = own_term + sum_k w_k * partial_k  (bf16 out).
 //
-// attend_tc_kernel: one persistent block per SM walks the tile queue with
-// four roles linked by mbarriers and double-buffered shared memory / TMEM:
-//   warp 0      producer  (tile metadata into a shared ring, landmark rows
-//                          into smem, TMA of the chunk's K and V)
-//   warp 10     Q gather  (one TMA box per entry: its G query-head rows)
-//   warp 1      MMA issuer (S of the next tile or P.V of the oldest pending
-//                          one, whichever is ready)
-//   warps 2-5   softmax   (thread = tile row = TMEM lane)
-//   warps 6-9   epilogue  (TMEM -> fp16 partial slots / own-chunk term)
+// attend_tc_kernel: one persistent block per SM walks the tile queue (a flat
+// list of tile descriptors) with these roles, linked by mbarriers, a ring of
+// three Q/K shared-memory slots, a ring of two V/P slots and double-buffered
+// TMEM accumulators:
+//   warp 0       producer  (tile metadata into a shared ring, landmark rows
+//                           into the K slot)
+//   warp 14      Q/K loads (one TMA box per entry: its G query-head rows; the
+//                           chunk's K)
+//   warp 15      V loads   (the chunk's V)
+//   warp 1       MMA issuer (S of the next tile or P.V of the oldest pending
+//                           one, whichever is ready)
+//   warps 2-5    softmax   (thread = tile row = TMEM lane)
+//   warps 6-13   epilogue  (two groups taking alternate tiles; TMEM -> fp16
+//                           partial slots / own-chunk term)
 // Tiles are independent, so no block waits on another.  Every wait is
 // bounded; on expiry the block sets the status flag in the workspace, lets
 // in-flight copies land, frees its TMEM and exits.
@@ -53,33 +58,42 @@ struct TcCfg {
     static constexpr int K_BYTES = KB * KBLK;
     static constexpr int V_BYTES = 64 * D * 2;
     static constexpr int P_BYTES = M * 64 * 2;   // probabilities, bf16
-    static constexpr int STAGE = Q_BYTES + K_BYTES + V_BYTES + P_BYTES;
-    static constexpr int SMEM = 1024 + 2 * STAGE + 256;
+    // Q and K are dead once S is computed, V and P only after P.V: they live
+    // in separate rings, three Q/K slots (loads run further ahead) and two V/P
+    // slots.  Every slot is a multiple of 1 KB (128-byte swizzle atoms).
+    static constexpr int NQK = 3, NVP = 2;
+    static constexpr int QK_STAGE = Q_BYTES + K_BYTES;
+    static constexpr int VP_STAGE = V_BYTES + P_BYTES;
+    static constexpr int BAR_OFF = NQK * QK_STAGE + NVP * VP_STAGE;
+    static constexpr int SMEM = 1024 + BAR_OFF + 256;
     // TMEM: S[2] at columns 0 / 128 (80 used), O[2] at 256 / 256 + D
     static constexpr uint32_t S_COL = 128;
     static constexpr uint32_t O_COL = 256;
     static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(QK_STAGE % 1024 == 0 && VP_STAGE % 1024 == 0, "slots must keep 1 KB alignment");
 };
 
 struct TcParams {
-    const int64_t *seg_start;     // [2 * NW + 1]
-    const int4 *wtiles;           // [NW * cap] retrieved-chunk tiles per window
+    const int4 *tiles;            // [qlen] tile descriptors in queue order
+    const int64_t *qlen;
     const int32_t *entries;
     const void *lm;               // [B, Hkv, Nc, D] bf16 or fp32
     float *logits;                // [B, L, H, topk] fusion logits
     __half *part;                 // [B*L*Hkv*topk entries][D/32][G][32] chunk outputs
     __half *own;                  // [B, L, H, D] own-chunk term
     unsigned *status;
-    int64_t L, W, nwb, NW, cap, Nc;
+    int64_t L, Nc;
     int H, Hkv, topk, S, add_own, lm_bf16;
     int q3d;                      // Q map is the 3-D (cols, rows, d-half) view
     float scale, scale_log2e;
 };
 
 constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
-constexpr int kThreads = 352;                       // 11 warps
-constexpr int kGatherWarp = 10;
-constexpr int kMaxWindows = 2048;                  // shared segment table size / 2
+constexpr int kThreads = 512;                       // 16 warps
+constexpr int kEpiWarp0 = 6;                        // epilogue groups: warps 6-9 and 10-13
+constexpr int kGatherWarp = 14;                     // Q and K loads
+constexpr int kVWarp = 15;                          // V loads
+constexpr int kOwnTileFlag = 1 << 30;               // in a descriptor's .w (bucket.cu)
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -102,37 +116,25 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
     return true;
 }
+// Parity to wait on before the u-th reuse of a ring slot (u >= 1): the
+// consumer's release of use u-1.
+__device__ __forceinline__ uint32_t reuse_parity(int64_t u) { return (uint32_t)((u + 1) & 1); }
 
 // A queue position decoded into one tile.
 struct Tile {
     int64_t bg, first, t0;   // first entry (retrieved) or first token (own)
     int chunk, n, own;
-    int64_t win;
 };
 
-__device__ __forceinline__ void decode_tile(const TcParams &p, const int64_t *seg, int nseg,
-                                            int64_t pos, int ept, Tile &tl) {
-    int lo = 0, hi = nseg;                  // seg[lo] <= pos < seg[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (seg[mid] <= pos) lo = mid; else hi = mid;
-    }
-    const int64_t j = pos - seg[lo];
-    if (lo == 0) { tl.own = 0; tl.win = 0; }
-    else if (lo == nseg - 1) { tl.own = 1; tl.win = p.NW - 1; }
-    else if (lo & 1) { tl.own = 0; tl.win = (lo + 1) / 2; }
-    else { tl.own = 1; tl.win = lo / 2 - 1; }
+__device__ __forceinline__ void decode_tile(const TcParams &p, int64_t pos, Tile &tl) {
+    const int4 d = p.tiles[pos];
+    tl.bg = d.x;
+    tl.own = (d.w & kOwnTileFlag) ? 1 : 0;
+    tl.n = d.w & (kOwnTileFlag - 1);
     if (!tl.own) {
-        const int4 d = p.wtiles[tl.win * p.cap + j];
-        tl.bg = d.x; tl.chunk = d.y; tl.first = d.z; tl.n = d.w; tl.t0 = 0;
+        tl.chunk = d.y; tl.first = d.z; tl.t0 = 0;
     } else {
-        tl.bg = tl.win / p.nwb;
-        const int64_t ts = (tl.win % p.nwb) * p.W;
-        const int64_t te = ts + p.W < p.L ? ts + p.W : p.L;
-        tl.t0 = ts + j * ept;
-        tl.n = (int)(te - tl.t0 < ept ? te - tl.t0 : ept);
-        tl.chunk = (int)(tl.t0 / p.S);
-        tl.first = 0;
+        tl.t0 = d.z; tl.chunk = (int)(tl.t0 / p.S); tl.first = 0;
     }
 }
 
@@ -141,7 +143,7 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int64_t *se
 // work lists).  code[e] = t * 32 + k of entry e (own tiles: t * 32).
 constexpr int kRing = 4;
 struct TileInfo {
-    int64_t bg, win;
+    int64_t bg;
     int chunk, n, own, pad;
     int32_t code[16];
 };
@@ -156,7 +158,7 @@ struct RowJob {
 
 __device__ __forceinline__ RowJob read_row(const TileInfo &ti, int e) {
     RowJob rj;
-    rj.tl.bg = ti.bg; rj.tl.win = ti.win; rj.tl.chunk = ti.chunk; rj.tl.n = ti.n;
+    rj.tl.bg = ti.bg; rj.tl.chunk = ti.chunk; rj.tl.n = ti.n;
     rj.tl.own = ti.own; rj.tl.first = 0; rj.tl.t0 = 0;
     rj.valid = e < ti.n;
     const int32_t code = rj.valid ? ti.code[e] : 0;
@@ -172,31 +174,36 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     using C = TcCfg<D, G>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    // stage s: [Q | K;l | V | P]
-    auto sQ = [&](int s) { return smem + s * C::STAGE; };
-    auto sK = [&](int s) { return smem + s * C::STAGE + C::Q_BYTES; };
-    auto sV = [&](int s) { return smem + s * C::STAGE + C::Q_BYTES + C::K_BYTES; };
-    auto sP = [&](int s) { return smem + s * C::STAGE + C::Q_BYTES + C::K_BYTES + C::V_BYTES; };
-    uint64_t *bars = (uint64_t *)(smem + 2 * C::STAGE);
-    uint64_t *full = bars, *empty = bars + 2, *sfull = bars + 4, *sfree = bars + 6;
-    uint64_t *pfull = bars + 8, *ofull = bars + 10, *ofree = bars + 12;
-    uint64_t *ifull = bars + 14, *ifree = bars + 14 + kRing;
-    uint32_t *s_tmem = (uint32_t *)(bars + 14 + 2 * kRing);
+    // Q/K slot q: [Q | K;l]; V/P slot v: [V | P]
+    auto sQ = [&](int q) { return smem + q * C::QK_STAGE; };
+    auto sK = [&](int q) { return smem + q * C::QK_STAGE + C::Q_BYTES; };
+    auto sV = [&](int v) { return smem + C::NQK * C::QK_STAGE + v * C::VP_STAGE; };
+    auto sP = [&](int v) { return smem + C::NQK * C::QK_STAGE + v * C::VP_STAGE + C::V_BYTES; };
+    uint64_t *bars = (uint64_t *)(smem + C::BAR_OFF);
+    uint64_t *qk_full = bars, *qk_empty = bars + 3;                    // [NQK]
+    uint64_t *v_full = bars + 6, *vp_empty = bars + 8;                 // [NVP]
+    uint64_t *sfull = bars + 10, *sfree = bars + 12, *pfull = bars + 14;
+    uint64_t *ofull = bars + 16, *ofree = bars + 18;
+    uint64_t *ifull = bars + 20, *ifree = bars + 20 + kRing;
+    uint32_t *s_tmem = (uint32_t *)(bars + 20 + 2 * kRing);
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
-    __shared__ int64_t seg[2 * kMaxWindows + 1];
     __shared__ TileInfo ring[kRing];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nseg = (int)(2 * p.NW);
-    for (int i = tid; i <= nseg; i += kThreads) seg[i] = p.seg_start[i];
     if (warp == 1) {
         tc::tmem_alloc(s_tmem, C::TMEM_COLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
+        for (int q = 0; q < C::NQK; ++q) {
+            tc::mbar_init(&qk_full[q], 2);     // Q/K loads + landmark rows
+            tc::mbar_init(&qk_empty[q], 1);    // S MMA done
+        }
+        for (int v = 0; v < C::NVP; ++v) {
+            tc::mbar_init(&v_full[v], 1);
+            tc::mbar_init(&vp_empty[v], 1);    // P.V MMA done
+        }
         for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(&full[s], 2);        // K/V producer + Q gather warp
-            tc::mbar_init(&empty[s], 1);
             tc::mbar_init(&sfull[s], 1);
             tc::mbar_init(&sfree[s], 128);
             tc::mbar_init(&pfull[s], 128);
@@ -205,7 +212,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         for (int i = 0; i < kRing; ++i) {
             tc::mbar_init(&ifull[i], 1);
-            tc::mbar_init(&ifree[i], 257);     // softmax + epilogue threads + gather warp
+            tc::mbar_init(&ifree[i], 258);     // softmax + one epilogue group + two loaders
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -214,17 +221,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    const int64_t qlen = seg[nseg];
+    const int64_t qlen = *p.qlen;
     const int64_t L = p.L;
     const int H = p.H, Hkv = p.Hkv, topk = p.topk, S = p.S;
-    constexpr int EPT = C::EPT;
     const int64_t my_tiles = qlen > blockIdx.x ? (qlen - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        // Software-pipelined two tiles deep: in iteration j the descriptor of
-        // tile j+2 and the entry codes / landmark row of tile j+1 are loaded
-        // while tile j is published and its copies are issued.
+        // Tile metadata and landmark rows.  Software-pipelined two tiles deep:
+        // in iteration j the descriptor of tile j+2 and the entry codes /
+        // landmark row of tile j+1 are loaded while tile j is published.
         auto load_rows = [&](const Tile &tl, int32_t &code, float (&x)[8]) {
             code = 0;
             if (lane < tl.n)
@@ -244,12 +250,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         Tile d0, d1;
         int32_t c0 = 0;
         float x0[8];
-        if (my_tiles > 0) decode_tile(p, seg, nseg, blockIdx.x, EPT, d0);
-        if (my_tiles > 1) decode_tile(p, seg, nseg, blockIdx.x + gridDim.x, EPT, d1);
+        if (my_tiles > 0) decode_tile(p, blockIdx.x, d0);
+        if (my_tiles > 1) decode_tile(p, blockIdx.x + gridDim.x, d1);
         if (my_tiles > 0) load_rows(d0, c0, x0);
         for (int64_t j = 0; j < my_tiles; ++j) {
             Tile d2;
-            if (j + 2 < my_tiles) decode_tile(p, seg, nseg, blockIdx.x + (j + 2) * gridDim.x, EPT, d2);
+            if (j + 2 < my_tiles) decode_tile(p, blockIdx.x + (j + 2) * gridDim.x, d2);
             int32_t c1 = 0;
             float x1[8];
             if (j + 1 < my_tiles) load_rows(d1, c1, x1);
@@ -257,31 +263,29 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             // publish the tile's metadata
             const int ri = (int)(j & (kRing - 1));
             int ok = 1;
-            if (lane == 0 && j >= kRing)
-                ok = wait_bar(&ifree[ri], (uint32_t)(((j / kRing) + 1) & 1), s_abort);
+            if (lane == 0 && j >= kRing) ok = wait_bar(&ifree[ri], reuse_parity(j / kRing), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             if (lane < 16) ring[ri].code[lane] = c0;
             if (lane == 0) {
-                ring[ri].bg = d0.bg; ring[ri].win = d0.win; ring[ri].chunk = d0.chunk;
+                ring[ri].bg = d0.bg; ring[ri].chunk = d0.chunk;
                 ring[ri].n = d0.n; ring[ri].own = d0.own;
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ifull[ri]);
 
-            // stage the tile's operands
-            const int s = (int)(j & 1);
-            if (lane == 0 && j >= 2) ok = wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort);
+            // landmark row of the chunk -> key rows 64 (bf16 high part), 65 (low part)
+            const int q = (int)(j % C::NQK);
+            if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             if (!d0.own && lane < D / 8) {
-                // landmark row of the chunk -> key rows 64 (bf16 high part), 65 (low part)
                 float hi[8], lo[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    hi[q] = __bfloat162float(__float2bfloat16_rn(x0[q]));
-                    lo[q] = x0[q] - hi[q];
+                for (int e = 0; e < 8; ++e) {
+                    hi[e] = __bfloat162float(__float2bfloat16_rn(x0[e]));
+                    lo[e] = x0[e] - hi[e];
                 }
                 const int kb = (lane * 8) / 64, c = ((lane * 8) % 64) / 8;
-                uint8_t *blk = sK(s) + kb * C::KBLK;
+                uint8_t *blk = sK(q) + kb * C::KBLK;
                 *reinterpret_cast<uint4 *>(blk + tc::sw128_offset(64, c)) =
                     make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
                                pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
@@ -291,52 +295,66 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tc::fence_proxy_async_smem();
             }
             __syncwarp();
-            if (lane == 0) {
-                // K and V of the chunk by TMA (the Q rows come from the gather warp)
-                tc::mbar_expect_tx(&full[s], (uint32_t)(2 * C::V_BYTES));
-                const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
-#pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb) {
-                    tc::tma_load_2d(sK(s) + kb * C::KBLK, &tmK, &full[s], kb * 64, krow);
-                    tc::tma_load_2d(sV(s) + kb * 8192, &tmV, &full[s], kb * 64, krow);
-                }
-            }
+            if (lane == 0) tc::mbar_arrive(&qk_full[q]);
             d0 = d1;
             d1 = d2;
             c0 = c1;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) x0[q] = x1[q];
+            for (int e = 0; e < 8; ++e) x0[e] = x1[e];
         }
-    } else if (warp == kGatherWarp) {
-        // ------------------------------------------------------------ Q gather
-        // One TMA box per entry: all G query-head rows of the entry (both
-        // 64-wide halves of d in one box when the 3-D view is available).
+    } else if (warp == kGatherWarp || warp == kVWarp) {
+        // ------------------------------------------------------------ loaders
+        // Q/K warp: one TMA box per entry (all G query-head rows, both halves
+        // of d when the 3-D view is available) plus the chunk's K.  V warp:
+        // the chunk's V, into the V/P ring.
+        const bool vw = warp == kVWarp;
         for (int64_t j = 0; j < my_tiles; ++j) {
             const int ri = (int)(j & (kRing - 1));
-            const int s = (int)(j & 1);
             int ok = 1;
-            if (lane == 0) {
-                ok = wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort);
-                if (ok && j >= 2) ok = wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort);
-            }
+            if (lane == 0) ok = wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const TileInfo &ti = ring[ri];
             const int n = ti.n;
-            const int64_t b = ti.bg / Hkv;
-            const int g = (int)(ti.bg % Hkv);
+            const int64_t bg = ti.bg;
+            const int chunk = ti.chunk;
             const int32_t code = lane < n ? ti.code[lane] : 0;
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ifree[ri]);
-            if (lane == 0) tc::mbar_expect_tx(&full[s], (uint32_t)(n * G * D * 2));
+            const int krow = (int)(bg * L + (int64_t)chunk * S);
+            if (vw) {
+                const int v = (int)(j % C::NVP);
+                if (lane == 0) {
+                    if (j >= C::NVP) ok = wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort);
+                    if (ok) {
+                        tc::mbar_expect_tx(&v_full[v], (uint32_t)C::V_BYTES);
+#pragma unroll
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tc::tma_load_2d(sV(v) + kb * 8192, &tmV, &v_full[v], kb * 64, krow);
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                continue;
+            }
+            const int q = (int)(j % C::NQK);
+            if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int64_t b = bg / Hkv;
+            const int g = (int)(bg % Hkv);
+            if (lane == 0) {
+                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(n * G * D * 2 + C::V_BYTES));
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tc::tma_load_2d(sK(q) + kb * C::KBLK, &tmK, &qk_full[q], kb * 64, krow);
+            }
             __syncwarp();
             if (lane < n) {
                 const int qrow = (int)((b * L + (int64_t)(code >> 5)) * H + (int64_t)g * G);
                 if (p.q3d) {
-                    tc::tma_load_3d(sQ(s) + lane * (C::KB * G * 128), &tmQ, &full[s], 0, qrow, 0);
+                    tc::tma_load_3d(sQ(q) + lane * (C::KB * G * 128), &tmQ, &qk_full[q], 0, qrow, 0);
                 } else {
 #pragma unroll
                     for (int kb = 0; kb < C::KB; ++kb)
-                        tc::tma_load_2d(sQ(s) + kb * (128 * 128) + lane * G * 128, &tmQ, &full[s],
+                        tc::tma_load_2d(sQ(q) + kb * (128 * 128) + lane * G * 128, &tmQ, &qk_full[q],
                                         kb * 64, qrow);
                 }
             }
@@ -347,43 +365,44 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, C::NS, false);
             constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
             auto issue_pv = [&](int64_t i) {
-                const int s = (int)(i & 1);
+                const int s = (int)(i & 1), v = (int)(i % C::NVP);
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP(s) + kk * 32), 16, 1024);
-                    const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sV(s) + kk * 2048), 8192, 1024);
+                    const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP(v) + kk * 32), 16, 1024);
+                    const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sV(v) + kk * 2048), 8192, 1024);
                     tc::mma_bf16(tmem + C::O_COL + s * D, ad, bd, IDESC_O, kk ? 1u : 0u);
                 }
                 tc::mma_commit(&ofull[s]);
-                tc::mma_commit(&empty[s]);
+                tc::mma_commit(&vp_empty[v]);
             };
-            // Issue S of the next tile or P.V of the oldest pending one, whichever
-            // is ready first (at most two tiles in flight, one per stage).
             auto issue_s = [&](int64_t j) {
-                const int s = (int)(j & 1);
+                const int s = (int)(j & 1), q = (int)(j % C::NQK);
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = p.q3d
-                            ? tc::sdesc_sw128(tc::smem_u32(sQ(s) + kb * (G * 128) + kk * 32), 16, C::KB * G * 128)
-                            : tc::sdesc_sw128(tc::smem_u32(sQ(s) + kb * 16384 + kk * 32), 16, 1024);
-                        const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sK(s) + kb * C::KBLK + kk * 32), 16, 1024);
+                            ? tc::sdesc_sw128(tc::smem_u32(sQ(q) + kb * (G * 128) + kk * 32), 16, C::KB * G * 128)
+                            : tc::sdesc_sw128(tc::smem_u32(sQ(q) + kb * 16384 + kk * 32), 16, 1024);
+                        const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sK(q) + kb * C::KBLK + kk * 32), 16, 1024);
                         tc::mma_bf16(tmem + s * C::S_COL, ad, bd, IDESC_S, (kb | kk) ? 1u : 0u);
                     }
                 tc::mma_commit(&sfull[s]);
+                tc::mma_commit(&qk_empty[q]);
             };
+            // S of tile j: its Q/K slot loaded and S slot j%2 read by the softmax
+            // of tile j-2.  P.V of tile i: P written, V loaded, O slot i%2 read
+            // by the epilogue of tile i-2.
             auto ready_s = [&](int64_t j) -> bool {
-                const int s = (int)(j & 1);
-                return tc::mbar_try_wait(&full[s], (uint32_t)((j >> 1) & 1)) &&
-                       (j < 2 || tc::mbar_try_wait(&sfree[s], (uint32_t)(((j >> 1) + 1) & 1)));
+                return tc::mbar_try_wait(&qk_full[j % C::NQK], (uint32_t)((j / C::NQK) & 1)) &&
+                       (j < 2 || tc::mbar_try_wait(&sfree[j & 1], reuse_parity(j >> 1)));
             };
             auto ready_pv = [&](int64_t i) -> bool {
-                const int s = (int)(i & 1);
-                return tc::mbar_try_wait(&pfull[s], (uint32_t)((i >> 1) & 1)) &&
-                       (i < 2 || tc::mbar_try_wait(&ofree[s], (uint32_t)(((i >> 1) + 1) & 1)));
+                return tc::mbar_try_wait(&pfull[i & 1], (uint32_t)((i >> 1) & 1)) &&
+                       tc::mbar_try_wait(&v_full[i % C::NVP], (uint32_t)((i / C::NVP) & 1)) &&
+                       (i < 2 || tc::mbar_try_wait(&ofree[i & 1], reuse_parity(i >> 1)));
             };
             int64_t ns = 0, npv = 0;
             long long t0 = clock64();
@@ -400,7 +419,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------ softmax
         const int q4 = warp & 3;                  // TMEM lane quarter
         const int r = q4 * 32 + lane;             // tile row
@@ -411,7 +430,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
             const RowJob cur = read_row(ring[ri], e);
             tc::mbar_arrive(&ifree[ri]);
-            const int s = (int)(j & 1);
+            const int s = (int)(j & 1), v = (int)(j % C::NVP);
             const int64_t b = cur.tl.bg / Hkv;
             const int g = (int)(cur.tl.bg % Hkv);
             if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
@@ -443,8 +462,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 l += s0[c] + s1[c];
             }
             const float f = cur.valid ? (cur.tl.own ? (float)p.add_own : 1.f) / l : 0.f;
-            if (j >= 2 && !wait_bar(&empty[s], (uint32_t)(((j >> 1) + 1) & 1), s_abort)) break;
-            uint8_t *prow = sP(s);
+            // P goes into V/P slot v, free once the P.V of tile j - NVP is done
+            if (j >= C::NVP && !wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort)) break;
+            uint8_t *prow = sP(v);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const float *src = c < 4 ? s0 + 8 * c : s1 + 8 * (c - 4);
@@ -457,14 +477,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&pfull[s]);
         }
-    } else {
+    } else if (warp < kGatherWarp) {
         // ------------------------------------------------------------ epilogue
+        // Two groups of four warps; group eg takes the tiles j = eg, eg+2, ...
+        // (TMEM O slot eg), so one tile's stores overlap the next one's.
+        const int eg = (warp - kEpiWarp0) >> 2;
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
         constexpr int NCH = D / 32;               // 32-column chunks of a row
-        for (int64_t j = 0; j < my_tiles; ++j) {
+        for (int64_t j = eg; j < my_tiles; j += 2) {
             const int ri = (int)(j & (kRing - 1));
             if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
             const RowJob cur = read_row(ring[ri], e);
@@ -491,10 +514,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         ? p.own + hrow * D + (ch + u) * 32
                         : p.part + (((row * topk + cur.k) * NCH + ch + u) * G + h) * 32;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                            pack_f16x2(o[u][8 * q + 0], o[u][8 * q + 1]), pack_f16x2(o[u][8 * q + 2], o[u][8 * q + 3]),
-                            pack_f16x2(o[u][8 * q + 4], o[u][8 * q + 5]), pack_f16x2(o[u][8 * q + 6], o[u][8 * q + 7]));
+                    for (int qq = 0; qq < 4; ++qq)
+                        reinterpret_cast<uint4 *>(dst)[qq] = make_uint4(
+                            pack_f16x2(o[u][8 * qq + 0], o[u][8 * qq + 1]), pack_f16x2(o[u][8 * qq + 2], o[u][8 * qq + 3]),
+                            pack_f16x2(o[u][8 * qq + 4], o[u][8 * qq + 5]), pack_f16x2(o[u][8 * qq + 6], o[u][8 * qq + 7]));
                 }
             }
             tc::fence_before_sync();
@@ -630,8 +653,8 @@ struct TcLaunch {
     int64_t L, W, cap;
     float scale;
     const int32_t *idx, *entries;
-    const int4 *wtiles;
-    const int64_t *seg_start;
+    const int4 *tiles;                // one descriptor per queue position
+    const int64_t *qlen;              // number of tiles (device)
     float *logits, *w_out;
     __half *part, *own;
     void *O;
@@ -655,11 +678,10 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     TcParams p;
-    p.seg_start = a.seg_start; p.wtiles = a.wtiles;
+    p.tiles = a.tiles; p.qlen = a.qlen;
     p.entries = a.entries; p.lm = a.lm; p.logits = a.logits;
     p.part = a.part; p.own = a.own; p.status = a.status;
-    p.L = a.L; p.W = a.W; p.nwb = (a.L + a.W - 1) / a.W;
-    p.NW = (int64_t)a.B * a.Hkv * p.nwb; p.cap = a.cap; p.Nc = a.L / a.S;
+    p.L = a.L; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
     p.lm_bf16 = a.lm_bf16;
     p.q3d = q3d ? 1 : 0;
@@ -676,7 +698,9 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-int64_t attend_tc_max_windows() { return kMaxWindows; }
+// The work lists hold no per-window state in shared memory any more; the
+// window count only sizes device arrays.
+int64_t attend_tc_max_windows() { return int64_t(1) << 20; }
 
 bool attend_tc_supported(bool bf16, int G, int d) {
     return bf16 && (G == 8 || G == 16) && (d == 64 || d == 128) && encode_fn() != nullptr;

@@ -14,13 +14,12 @@
 //   scan    -- bucket offsets, tile descriptors per window (one block per window)
 //   order   -- start of every segment of the work queue    (one block)
 //   scatter -- entry codes t*32+k into their bucket slots  (atomic cursors)
+//   flatten -- one descriptor per queue position           (one block per window)
 // The order of entries inside a bucket is not fixed, which does not change
 // any result: every tile row is computed independently of the other rows.
 //
-// Work queue (consumed by attend_tc.cu): segments
-//   C0, C1, O0, C2, O1, ..., C(n-1), O(n-2), O(n-1)
-// where Cn = retrieved-chunk tiles of window n and On = own-chunk/fusion tiles
-// of window n; On comes one window after Cn so that Cn has finished by then.
+// Work queue (consumed by attend_tc.cu): segments C0, O0, C1, O1, ... where
+// Cn = retrieved-chunk tiles of window n and On = own-chunk tiles of window n.
 #include "common.cuh"
 
 namespace hsa {
@@ -143,11 +142,7 @@ queue_order_kernel(const int32_t *__restrict__ wntiles, WinGeom wg, int64_t NW,
     const int64_t per = (nseg + kScanThreads - 1) / kScanThreads;
     const int64_t s0 = tid * per, s1 = (s0 + per < nseg) ? s0 + per : nseg;
     auto seg_len = [&](int64_t s) -> int64_t {
-        int64_t type_own, n;
-        if (s == 0) { type_own = 0; n = 0; }
-        else if (s == nseg - 1) { type_own = 1; n = NW - 1; }
-        else if (s & 1) { type_own = 0; n = (s + 1) / 2; }
-        else { type_own = 1; n = s / 2 - 1; }
+        const int64_t type_own = s & 1, n = s >> 1;
         if (!type_own) return wntiles[n];
         int64_t bg, ts, te;
         window_span(wg, n, bg, ts, te);
@@ -182,6 +177,29 @@ queue_order_kernel(const int32_t *__restrict__ wntiles, WinGeom wg, int64_t NW,
     if (nseg == 0 && tid == 0) seg_start[0] = 0;
 }
 
+// Flat tile list: tiles[q] = descriptor of queue position q, so the consumer
+// needs one load per tile instead of a search over segment starts.
+// {bg, chunk, first entry, n} for retrieved-chunk tiles; own-chunk tiles are
+// {bg, 0, first token, n | kOwnTileFlag} (the consumer derives the chunk).
+constexpr int kOwnTileFlag = 1 << 30;
+__global__ void __launch_bounds__(kBucketThreads)
+flatten_tiles_kernel(const int4 *__restrict__ wtiles, const int32_t *__restrict__ wntiles,
+                     const int64_t *__restrict__ seg_start, WinGeom wg,
+                     int4 *__restrict__ tiles) {
+    const int64_t n = blockIdx.x;
+    int64_t bg, ts, te;
+    window_span(wg, n, bg, ts, te);
+    const int64_t c0 = seg_start[2 * n], o0 = seg_start[2 * n + 1];
+    const int nc = wntiles[n];
+    for (int j = threadIdx.x; j < nc; j += blockDim.x) tiles[c0 + j] = wtiles[n * wg.cap + j];
+    const int64_t no = (te - ts + wg.ept - 1) / wg.ept;
+    for (int64_t j = threadIdx.x; j < no; j += blockDim.x) {
+        const int64_t t0 = ts + j * wg.ept;
+        const int64_t cnt = te - t0 < wg.ept ? te - t0 : wg.ept;
+        tiles[o0 + j] = make_int4((int)bg, 0, (int)t0, (int)cnt | kOwnTileFlag);
+    }
+}
+
 // entries[cursor[n, i]++] = t * 32 + k
 __global__ void __launch_bounds__(kBucketThreads)
 bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int32_t *__restrict__ cursor,
@@ -203,7 +221,7 @@ bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int32_t *__re
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
-                          int64_t *seg_start, cudaStream_t st) {
+                          int64_t *seg_start, int4 *tiles, cudaStream_t st) {
     WinGeom wg;
     wg.L = L; wg.Nc = Nc; wg.W = W; wg.nwb = (L + W - 1) / W;
     wg.Hkv = Hkv; wg.topk = topk; wg.ept = ept; wg.cap = cap;
@@ -222,6 +240,10 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bucket_scatter_kernel<<<grid, kBucketThreads, 0, st>>>(idx, wg, cursor, entries);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    flatten_tiles_kernel<<<(unsigned)NW, kBucketThreads, 0, st>>>(wtiles, wntiles, seg_start, wg,
+                                                                  tiles);
     return cudaGetLastError();
 }
 

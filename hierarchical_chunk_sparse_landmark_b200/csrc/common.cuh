@@ -172,6 +172,21 @@ __device__ __forceinline__ uint64_t merge_lists(uint64_t a, uint64_t b, int KP) 
     }
     return v;
 }
+// Sort every KP-lane segment of a register in descending order (bitonic
+// network; blocks of size k < KP alternate direction so that each pair forms
+// a bitonic sequence, the last stage sorts every segment descending).
+__device__ __forceinline__ uint64_t sort_segments_desc(uint64_t v, int KP) {
+    const int lane = threadIdx.x & 31;
+    for (int k = 2; k <= KP; k <<= 1)
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const uint64_t p = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool lower = (lane & j) == 0;
+            const bool desc = k == KP || (lane & k) == 0;
+            const uint64_t hi = v > p ? v : p, lo = v > p ? p : v;
+            v = (lower == desc) ? hi : lo;
+        }
+    return v;
+}
 // Merge the 32/KP lists of one register into one (returned in every segment).
 __device__ __forceinline__ uint64_t merge_segments(uint64_t v, int KP) {
     for (int m = KP; m < 32; m <<= 1) v = merge_lists(v, __shfl_xor_sync(0xffffffffu, v, m), KP);

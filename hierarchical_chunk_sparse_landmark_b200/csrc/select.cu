@@ -15,8 +15,8 @@
 // through shared memory 32 at a time.  Each thread scores one token against 8
 // chunks of a tile (fp32 FMA, float4 operands) into a shared score tile; then
 // each warp folds the tile into the sorted top-K lists of its 8 tokens, kept
-// warp-distributed (lane k holds a token's k-th best 64-bit key).  Only lanes
-// whose key beats the current K-th best take part in an insertion.
+// warp-distributed (lane k holds a token's k-th best 64-bit key), with
+// bitonic sorting and merging networks.
 #include "common.cuh"
 
 namespace hsa {
@@ -25,19 +25,6 @@ constexpr int kSelTokens = 64;   // tokens per block
 constexpr int kSelChunks = 32;   // landmark rows per shared-memory tile
 constexpr int kSelThreads = 256; // 8 warps, 8 tokens per warp
 constexpr int kSelTokPerWarp = kSelTokens / (kSelThreads / 32);
-
-// Insert x into a warp-distributed sorted list (lane k < topk holds entry k).
-// Executed by the whole warp with the same x; returns this lane's new entry.
-__device__ __forceinline__ uint64_t list_insert(uint64_t v, uint64_t x, int topk, int lane) {
-    const unsigned better = __ballot_sync(0xffffffffu, lane < topk && v > x);
-    const int pos = __popc(better);
-    const uint64_t up = __shfl_up_sync(0xffffffffu, v, 1);
-    if (lane < topk) {
-        if (lane == pos) v = x;
-        else if (lane > pos) v = up;
-    }
-    return v;
-}
 
 template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kSelThreads)
@@ -57,35 +44,79 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
     const int64_t t0 = (int64_t)tile * kSelTokens;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // qbar for the block's tokens (rows past L are zero).
-    for (int e = tid; e < kSelTokens * D; e += kSelThreads) {
-        const int r = e / D, j = e % D;
-        const int64_t t = t0 + r;
-        float acc = 0.f;
-        if (t < L) {
-            const T *qp = Q + ((b * L + t) * H + (int64_t)g * G) * D + j;
-            for (int h = 0; h < G; ++h) acc += to_f32(qp[(int64_t)h * D]);
-            acc = acc / (float)G;
+    // qbar for the block's tokens (rows past L are zero).  A thread owns one
+    // 16-byte vector (VT elements of d) of a token and sums it over the G
+    // heads; all of a thread's loads are independent, so many are in flight.
+    {
+        constexpr int VT = Vec16<T>::N;
+        constexpr int VPR = D / VT;                          // vectors per row
+        constexpr int PER = kSelTokens * VPR / kSelThreads;  // (token, vector) pairs per thread
+        static_assert(PER * kSelThreads == kSelTokens * VPR, "qbar pairs must split evenly");
+        float acc[PER][VT];
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+#pragma unroll
+            for (int v = 0; v < VT; ++v) acc[u][v] = 0.f;
+        for (int h = 0; h < G; ++h) {
+            uint4 raw[PER];
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = tid + u * kSelThreads, r = e / VPR, c = (e % VPR) * VT;
+                const int64_t t = t0 + r;
+                raw[u] = t < L ? ld_stream16(Q + ((b * L + t) * H + (int64_t)g * G + h) * D + c)
+                               : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                float f[VT];
+                Vec16<T>::unpack(raw[u], f);
+#pragma unroll
+                for (int v = 0; v < VT; ++v) acc[u][v] += f[v];
+            }
         }
-        qbar[r * (D + 4) + j] = acc;
+        const float inv = 1.f / (float)G;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * kSelThreads, r = e / VPR, c = (e % VPR) * VT;
+#pragma unroll
+            for (int v = 0; v < VT; ++v) qbar[r * (D + 4) + c + v] = acc[u][v] * inv;
+        }
     }
     const int64_t t_last = (t0 + kSelTokens - 1 < L ? t0 + kSelTokens - 1 : L - 1);
     const int64_t nvis_max = t_last / S;
 
     // scoring role: token tok_s, chunks sub + 4m of each tile
     const int tok_s = tid >> 2, sub = tid & 3;
-    // list role: this warp's tokens
-    uint64_t v[kSelTokPerWarp], thr[kSelTokPerWarp];
+    // list role: this warp's tokens, each a sorted list of KP keys replicated
+    // in every KP-lane segment of v[u] (lane k < topk holds the k-th best)
+    const int KP = pow2_at_least(topk);
+    uint64_t v[kSelTokPerWarp];
 #pragma unroll
-    for (int u = 0; u < kSelTokPerWarp; ++u) { v[u] = 0ull; thr[u] = 0ull; }
+    for (int u = 0; u < kSelTokPerWarp; ++u) v[u] = 0ull;
 
     const TL *lm_bg = lm + ((int64_t)b * Hkv + g) * Nc * D;
     for (int64_t c0 = 0; c0 < nvis_max; c0 += kSelChunks) {
         __syncthreads();
-        for (int e = tid; e < kSelChunks * D; e += kSelThreads) {
-            const int r = e / D, j = e % D;
-            const int64_t i = c0 + r;
-            lmt[r * (D + 4) + j] = i < nvis_max ? to_f32(lm_bg[i * D + j]) : 0.f;
+        {
+            // landmark rows c0 .. c0+31 as fp32, 16-byte loads all in flight
+            constexpr int VL = Vec16<TL>::N;
+            constexpr int LPT = kSelChunks * (D / VL) / kSelThreads;   // vectors per thread
+            uint4 raw[LPT];
+#pragma unroll
+            for (int u = 0; u < LPT; ++u) {
+                const int e = tid + u * kSelThreads, r = e / (D / VL), c = (e % (D / VL)) * VL;
+                const int64_t i = c0 + r;
+                raw[u] = i < nvis_max ? *reinterpret_cast<const uint4 *>(lm_bg + i * D + c)
+                                      : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < LPT; ++u) {
+                const int e = tid + u * kSelThreads, r = e / (D / VL), c = (e % (D / VL)) * VL;
+                float f[VL];
+                Vec16<TL>::unpack(raw[u], f);
+#pragma unroll
+                for (int v = 0; v < VL; ++v) lmt[r * (D + 4) + c + v] = f[v];
+            }
         }
         __syncthreads();
         {
@@ -110,6 +141,9 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
             for (int m = 0; m < 8; ++m) sc[tok_s * 33 + sub + 4 * m] = scale * acc[m];
         }
         __syncthreads();
+        // fold the tile into each token's top-KP list: bitonic-sort the 32
+        // keys into KP-long runs, merge the runs, merge into the running list
+        // (the warp's 8 tokens are independent chains of shuffles)
 #pragma unroll
         for (int u = 0; u < kSelTokPerWarp; ++u) {
             const int tok = warp * kSelTokPerWarp + u;
@@ -117,16 +151,7 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
             const int64_t nvis = t < L ? t / S : 0;
             const int64_t i = c0 + lane;
             const uint64_t key = i < nvis ? make_key(sc[tok * 33 + lane], i) : 0ull;
-            unsigned m = __ballot_sync(0xffffffffu, key > thr[u]);
-            while (m) {
-                const int s = __ffs(m) - 1;
-                m &= m - 1;
-                const uint64_t x = __shfl_sync(0xffffffffu, key, s);
-                if (x > thr[u]) {
-                    v[u] = list_insert(v[u], x, topk, lane);
-                    thr[u] = __shfl_sync(0xffffffffu, v[u], topk - 1);
-                }
-            }
+            v[u] = merge_lists(v[u], merge_segments(sort_segments_desc(key, KP), KP), KP);
         }
     }
 
@@ -134,8 +159,6 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
     // logits the warp is split into KP slots (KP = topk rounded up to a power
     // of two) of PARTS = 32/KP lanes; the lanes of slot k split d and reduce
     // with PARTS-wide shuffles, so all slots of a head are computed at once.
-    int KP = 1;
-    while (KP < topk) KP <<= 1;
     const int PARTS = 32 / KP;
     const int slot = lane / PARTS, part = lane % PARTS;
     const int span = D / PARTS;                       // d elements per lane
