@@ -35,7 +35,7 @@ struct TcLaunch {
     const int32_t *idx, *entries;
     const int4 *tiles;                // one descriptor per queue position
     const int64_t *qlen;              // number of tiles (device)
-    float *logits, *w_out;
+    float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
     __half *part, *own;
     void *O;
     unsigned *status;
@@ -105,7 +105,7 @@ struct PrefillLayout {
     bool tc;
     int64_t W, NW, cap;
     size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
-        seg_off, tiles_off, part_off, own_off;
+        seg_off, tiles_off, zf_off, ownf_off, part_off, own_off;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
@@ -122,6 +122,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     p.W = p.NW = p.cap = 0;
     p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
     p.wntiles_off = p.done_off = p.seg_off = p.tiles_off = p.part_off = p.own_off = 0;
+    p.zf_off = p.ownf_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
         p.W = tc_window(B, H, Hkv, L, d, topk, attend_tc_max_windows());
@@ -144,6 +145,10 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         off = align_up(off + sizeof(int64_t) * (size_t)(2 * p.NW + 1), 256);
         p.tiles_off = off;           // retrieved tiles + own-chunk tiles of every window
         off = align_up(off + sizeof(int4) * (size_t)(p.NW * (p.cap + (p.W + ept - 1) / ept)), 256);
+        p.zf_off = off;
+        off = align_up(off + 2 * sizeof(float) * (size_t)B * L * H * topk, 256);
+        p.ownf_off = off;
+        off = align_up(off + sizeof(float) * (size_t)B * L * H, 256);
         p.part_off = off;
         off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
         p.own_off = off;
@@ -287,9 +292,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
     const bool use_tc = bf16 && lay.tc && !force_simt_path() &&
                         attend_tc_supported(bf16, H / Hkv, d);
     // The tensor-core path computes the fusion logits inside its S tiles and
-    // the weights in its fusion epilogue; the workspace weight region then
-    // holds the logits.
-    float *w_ws = (float *)(ws + lay.w_off);
+    // the weights in fuse_kernel, so the selection skips them there.
     cudaError_t e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
                                   use_tc ? nullptr : w, st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
@@ -314,7 +317,8 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.idx = idx; a.entries = (const int32_t *)(ws + lay.entries_off);
         a.tiles = (const int4 *)(ws + lay.tiles_off);
         a.qlen = (const int64_t *)(ws + lay.seg_off) + 2 * lay.NW;
-        a.logits = w_ws; a.w_out = w_out;
+        a.zf = (float *)(ws + lay.zf_off); a.own_f = (float *)(ws + lay.ownf_off);
+        a.w_out = w_out;
         a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;
         a.num_sms = num_sms();

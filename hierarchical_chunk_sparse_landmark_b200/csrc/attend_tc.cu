@@ -12,25 +12,27 @@
 // fusion logit scale * q_h . l_chunk:
 //
 //   S = Q_rows . [K_chunk ; l_hi ; l_lo]^T  M=128, N=80, K=d  (tcgen05 -> TMEM)
-//   P = exp(S*scale - rowmax) / rowsum      per row in registers, bf16 -> smem
-//   O = P . V_chunk                         M=128, N=d, K=64  (tcgen05 -> TMEM)
-//   partial[t, g, k] = O (fp16), logit[t, h, k] = scale * (S[:,64] + S[:,65])
+//   P = 2^-6 exp(S*scale - rowmax)          per row in registers, bf16 -> TMEM
+//   O = P . V_chunk                         M=128, N=d, K=64  (tcgen05, A from TMEM)
+//   partial[t, g, k] = O (fp16); per (t, h, k): the fusion logit
+//   scale * (S[:,64] + S[:,65]) and f = 1 / sum of the row's P
 //
 // Own tiles: 128/G consecutive tokens of a chunk against that chunk with the
-// causal mask (keys c*S .. t); their output (the own-chunk term) goes to an
-// fp16 array.  fuse_kernel then completes the method, one warp per (t, h):
+// causal mask (keys c*S .. t); their output (the own-chunk term, same scaling,
+// f = own_chunk / row sum) goes to an fp16 array.  fuse_kernel then completes
+// the method, one warp per (t, h):
 //   w = softmax over the token's selected chunks of the logits,
-//   O = own_term + sum_k w_k * partial_k  (bf16 out).
+//   O = f_own * own + sum_k w_k * f_k * partial_k  (bf16 out).
 //
 // attend_tc_kernel: one persistent block per SM walks the tile queue (a flat
 // list of tile descriptors) with these roles, linked by mbarriers, a ring of
-// three Q/K shared-memory slots, a ring of two V/P slots and double-buffered
-// TMEM accumulators:
-//   warp 0       producer  (tile metadata into a shared ring, landmark rows
-//                           into the K slot)
+// three Q/K shared-memory slots, a ring of two V slots and double-buffered
+// TMEM accumulators (S, P and O):
+//   warps 0, 15  producers (even / odd tiles: tile metadata into a shared
+//                           ring, landmark rows into the K slot, TMA of the
+//                           chunk's V)
 //   warp 14      Q/K loads (one TMA box per entry: its G query-head rows; the
 //                           chunk's K)
-//   warp 15      V loads   (the chunk's V)
 //   warp 1       MMA issuer (S of the next tile or P.V of the oldest pending
 //                           one, whichever is ready)
 //   warps 2-5    softmax   (thread = tile row = TMEM lane)
@@ -57,17 +59,19 @@ struct TcCfg {
     static constexpr int KBLK = NS * 128;        // one 64-wide d block of [K; l]
     static constexpr int K_BYTES = KB * KBLK;
     static constexpr int V_BYTES = 64 * D * 2;
-    static constexpr int P_BYTES = M * 64 * 2;   // probabilities, bf16
-    // Q and K are dead once S is computed, V and P only after P.V: they live
-    // in separate rings, three Q/K slots (loads run further ahead) and two V/P
-    // slots.  Every slot is a multiple of 1 KB (128-byte swizzle atoms).
-    static constexpr int NQK = 3, NVP = 2;
+    static constexpr int K_TMA_BYTES = 64 * D * 2;   // the 64 key rows (rows 64+ are written in smem)
+    // Q and K are dead once S is computed, V only after P.V: they live in
+    // separate rings of three slots each, so loads run up to three tiles ahead.  Every slot is a multiple of 1 KB (128-byte swizzle atoms).
+    static constexpr int NQK = 3, NVP = 3;
     static constexpr int QK_STAGE = Q_BYTES + K_BYTES;
-    static constexpr int VP_STAGE = V_BYTES + P_BYTES;
+    static constexpr int VP_STAGE = V_BYTES;
     static constexpr int BAR_OFF = NQK * QK_STAGE + NVP * VP_STAGE;
-    static constexpr int SMEM = 1024 + BAR_OFF + 256;
-    // TMEM: S[2] at columns 0 / 128 (80 used), O[2] at 256 / 256 + D
+    static constexpr int BAR_BYTES = 512;        // mbarriers + TMEM address + abort flag
+    static constexpr int SMEM = 1024 + BAR_OFF + BAR_BYTES;
+    // TMEM: S[2] at columns 0 / 128 (80 used); P[2] (bf16 pairs, 32 columns)
+    // right after each S at 80 / 208; O[2] at 256 / 256 + D
     static constexpr uint32_t S_COL = 128;
+    static constexpr uint32_t P_OFF = 80;
     static constexpr uint32_t O_COL = 256;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(QK_STAGE % 1024 == 0 && VP_STAGE % 1024 == 0, "slots must keep 1 KB alignment");
@@ -78,7 +82,8 @@ struct TcParams {
     const int64_t *qlen;
     const int32_t *entries;
     const void *lm;               // [B, Hkv, Nc, D] bf16 or fp32
-    float *logits;                // [B, L, H, topk] fusion logits
+    float *zf;                    // [B, L, H, topk] x (fusion logit, 1 / chunk row sum)
+    float *own_f;                 // [B, L, H] add_own / own-chunk row sum
     __half *part;                 // [B*L*Hkv*topk entries][D/32][G][32] chunk outputs
     __half *own;                  // [B, L, H, D] own-chunk term
     unsigned *status;
@@ -92,7 +97,7 @@ constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
 constexpr int kThreads = 512;                       // 16 warps
 constexpr int kEpiWarp0 = 6;                        // epilogue groups: warps 6-9 and 10-13
 constexpr int kGatherWarp = 14;                     // Q and K loads
-constexpr int kVWarp = 15;                          // V loads
+constexpr int kProducer2 = 15;                      // second producer (odd tiles)
 constexpr int kOwnTileFlag = 1 << 30;               // in a descriptor's .w (bucket.cu)
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -126,8 +131,7 @@ struct Tile {
     int chunk, n, own;
 };
 
-__device__ __forceinline__ void decode_tile(const TcParams &p, int64_t pos, Tile &tl) {
-    const int4 d = p.tiles[pos];
+__device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Tile &tl) {
     tl.bg = d.x;
     tl.own = (d.w & kOwnTileFlag) ? 1 : 0;
     tl.n = d.w & (kOwnTileFlag - 1);
@@ -146,6 +150,16 @@ struct TileInfo {
     int64_t bg;
     int chunk, n, own, pad;
     int32_t code[16];
+};
+
+// The producer's prefetch ring: descriptor, entry codes and raw landmark row
+// (up to d fp32 values) of the next tiles.
+constexpr int kMeta = 8;
+template <int D>
+struct alignas(16) TileMetaT {
+    int4 desc;
+    int32_t code[16];
+    uint8_t lrow[D * 4];
 };
 
 // Per-row view of a tile for the softmax and epilogue threads.
@@ -174,20 +188,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     using C = TcCfg<D, G>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    // Q/K slot q: [Q | K;l]; V/P slot v: [V | P]
+    // Q/K slot q: [Q | K;l]; V slot v
     auto sQ = [&](int q) { return smem + q * C::QK_STAGE; };
     auto sK = [&](int q) { return smem + q * C::QK_STAGE + C::Q_BYTES; };
     auto sV = [&](int v) { return smem + C::NQK * C::QK_STAGE + v * C::VP_STAGE; };
-    auto sP = [&](int v) { return smem + C::NQK * C::QK_STAGE + v * C::VP_STAGE + C::V_BYTES; };
     uint64_t *bars = (uint64_t *)(smem + C::BAR_OFF);
     uint64_t *qk_full = bars, *qk_empty = bars + 3;                    // [NQK]
-    uint64_t *v_full = bars + 6, *vp_empty = bars + 8;                 // [NVP]
-    uint64_t *sfull = bars + 10, *sfree = bars + 12, *pfull = bars + 14;
-    uint64_t *ofull = bars + 16, *ofree = bars + 18;
-    uint64_t *ifull = bars + 20, *ifree = bars + 20 + kRing;
-    uint32_t *s_tmem = (uint32_t *)(bars + 20 + 2 * kRing);
+    uint64_t *v_full = bars + 6, *vp_empty = bars + 9;                 // [NVP]
+    uint64_t *sfull = bars + 12, *sfree = bars + 14, *pfull = bars + 16;
+    uint64_t *ofull = bars + 18, *ofree = bars + 20, *pempty = bars + 22;
+    uint64_t *ifull = bars + 24, *ifree = bars + 24 + kRing;
+    uint32_t *s_tmem = (uint32_t *)(bars + 24 + 2 * kRing);
+    static_assert((24 + 2 * kRing) * 8 + 8 <= C::BAR_BYTES, "barrier block overflows its reserve");
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
     __shared__ TileInfo ring[kRing];
+    using TileMeta = TileMetaT<D>;
+    __shared__ TileMeta meta[kMeta];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (warp == 1) {
@@ -209,10 +225,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::mbar_init(&pfull[s], 128);
             tc::mbar_init(&ofull[s], 1);
             tc::mbar_init(&ofree[s], 128);
+            tc::mbar_init(&pempty[s], 1);      // P.V done: TMEM P slot free
         }
         for (int i = 0; i < kRing; ++i) {
             tc::mbar_init(&ifull[i], 1);
-            tc::mbar_init(&ifree[i], 258);     // softmax + one epilogue group + two loaders
+            tc::mbar_init(&ifree[i], 257);     // softmax + one epilogue group + Q/K loader
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -226,39 +243,52 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int H = p.H, Hkv = p.Hkv, topk = p.topk, S = p.S;
     const int64_t my_tiles = qlen > blockIdx.x ? (qlen - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        // Tile metadata and landmark rows.  Software-pipelined two tiles deep:
-        // in iteration j the descriptor of tile j+2 and the entry codes /
-        // landmark row of tile j+1 are loaded while tile j is published.
-        auto load_rows = [&](const Tile &tl, int32_t &code, float (&x)[8]) {
-            code = 0;
-            if (lane < tl.n)
-                code = tl.own ? (int32_t)((tl.t0 + lane) * 32) : p.entries[tl.first + lane];
-            if (!tl.own && lane < D / 8) {
-                const int64_t li = (tl.bg * p.Nc + tl.chunk) * D + lane * 8;
-                if (p.lm_bf16) {
-                    Vec16<__nv_bfloat16>::unpack(
-                        *reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.lm + li), x);
-                } else {
-                    const uint4 *src = reinterpret_cast<const uint4 *>((const float *)p.lm + li);
-                    Vec16<float>::unpack(src[0], x);
-                    Vec16<float>::unpack(src[1], x + 4);
+    if (warp == 0 || warp == kProducer2) {
+        // ------------------------------------------------------------ producers
+        // Tile metadata and landmark rows; producer pid takes the tiles
+        // j = 2u + pid.  Its descriptors are fetched two of its tiles ahead and
+        // entry codes / landmark rows one tile ahead with cp.async into its
+        // half of a shared ring, so it never waits on a fresh global load.
+        // Virtual iterations u = -2, -1 only fill the ring; every iteration
+        // commits exactly two copy groups, so "at most 2 pending" means: this
+        // tile's rows and the descriptor of the next one have landed.
+        const int pid = warp == 0 ? 0 : 1;
+        const int64_t my_u = (my_tiles - pid + 1) / 2;
+        auto slot_of = [&](int64_t u) -> TileMeta & { return meta[pid * (kMeta / 2) + (u & (kMeta / 2 - 1))]; };
+        auto issue_desc = [&](int64_t u) {
+            if (lane == 0 && u >= 0 && u < my_u)
+                tc::cp_async16(&slot_of(u).desc, p.tiles + blockIdx.x + (2 * u + pid) * gridDim.x);
+            tc::cp_async_commit();
+        };
+        auto issue_rows = [&](int64_t u) {
+            if (u >= 0 && u < my_u) {
+                TileMeta &mt = slot_of(u);
+                Tile tl;
+                decode_tile(p, mt.desc, tl);
+                if (!tl.own) {
+                    if (lane < tl.n) tc::cp_async4(&mt.code[lane], p.entries + tl.first + lane);
+                    constexpr int LB = D * 4 / 16;                 // 16-byte pieces of an fp32 row
+                    const int pieces = p.lm_bf16 ? LB / 2 : LB;
+                    const uint8_t *src = (const uint8_t *)p.lm +
+                        (size_t)(tl.bg * p.Nc + tl.chunk) * D * (p.lm_bf16 ? 2 : 4);
+                    if (lane < pieces) tc::cp_async16(mt.lrow + lane * 16, src + lane * 16);
                 }
             }
+            tc::cp_async_commit();
         };
-        Tile d0, d1;
-        int32_t c0 = 0;
-        float x0[8];
-        if (my_tiles > 0) decode_tile(p, blockIdx.x, d0);
-        if (my_tiles > 1) decode_tile(p, blockIdx.x + gridDim.x, d1);
-        if (my_tiles > 0) load_rows(d0, c0, x0);
-        for (int64_t j = 0; j < my_tiles; ++j) {
-            Tile d2;
-            if (j + 2 < my_tiles) decode_tile(p, blockIdx.x + (j + 2) * gridDim.x, d2);
-            int32_t c1 = 0;
-            float x1[8];
-            if (j + 1 < my_tiles) load_rows(d1, c1, x1);
+        for (int64_t u = -2; u < my_u; ++u) {
+            issue_desc(u + 2);
+            tc::cp_async_wait<2>();
+            __syncwarp();
+            issue_rows(u + 1);
+            if (u < 0) continue;
+            tc::cp_async_wait<2>();
+            __syncwarp();
+            const int64_t j = 2 * u + pid;
+            TileMeta &mt = slot_of(u);
+            Tile d0;
+            decode_tile(p, mt.desc, d0);
+            const int32_t c0 = lane < d0.n ? (d0.own ? (int32_t)((d0.t0 + lane) * 32) : mt.code[lane]) : 0;
 
             // publish the tile's metadata
             const int ri = (int)(j & (kRing - 1));
@@ -278,6 +308,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             if (!d0.own && lane < D / 8) {
+                float x0[8];
+                if (p.lm_bf16) {
+                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(mt.lrow + lane * 16), x0);
+                } else {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(mt.lrow + lane * 32);
+                    Vec16<float>::unpack(src[0], x0);
+                    Vec16<float>::unpack(src[1], x0 + 4);
+                }
                 float hi[8], lo[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -296,18 +334,27 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&qk_full[q]);
-            d0 = d1;
-            d1 = d2;
-            c0 = c1;
+
+            // V of the chunk into V slot j % 3, free once the P.V of tile j - 3
+            // is done
+            const int v = (int)(j % C::NVP);
+            if (lane == 0) {
+                if (j >= C::NVP) ok = wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort);
+                if (ok) {
+                    tc::mbar_expect_tx(&v_full[v], (uint32_t)C::V_BYTES);
+                    const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x0[e] = x1[e];
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tc::tma_load_2d(sV(v) + kb * 8192, &tmV, &v_full[v], kb * 64, krow);
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         }
-    } else if (warp == kGatherWarp || warp == kVWarp) {
-        // ------------------------------------------------------------ loaders
-        // Q/K warp: one TMA box per entry (all G query-head rows, both halves
-        // of d when the 3-D view is available) plus the chunk's K.  V warp:
-        // the chunk's V, into the V/P ring.
-        const bool vw = warp == kVWarp;
+        tc::cp_async_wait<0>();
+    } else if (warp == kGatherWarp) {
+        // ------------------------------------------------------------ Q/K loads
+        // One TMA box per entry (all G query-head rows, both halves of d when
+        // the 3-D view is available) plus the chunk's K.
         for (int64_t j = 0; j < my_tiles; ++j) {
             const int ri = (int)(j & (kRing - 1));
             int ok = 1;
@@ -321,27 +368,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ifree[ri]);
             const int krow = (int)(bg * L + (int64_t)chunk * S);
-            if (vw) {
-                const int v = (int)(j % C::NVP);
-                if (lane == 0) {
-                    if (j >= C::NVP) ok = wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort);
-                    if (ok) {
-                        tc::mbar_expect_tx(&v_full[v], (uint32_t)C::V_BYTES);
-#pragma unroll
-                        for (int kb = 0; kb < C::KB; ++kb)
-                            tc::tma_load_2d(sV(v) + kb * 8192, &tmV, &v_full[v], kb * 64, krow);
-                    }
-                }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-                continue;
-            }
             const int q = (int)(j % C::NQK);
             if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const int64_t b = bg / Hkv;
             const int g = (int)(bg % Hkv);
             if (lane == 0) {
-                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(n * G * D * 2 + C::V_BYTES));
+                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(n * G * D * 2 + C::K_TMA_BYTES));
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
                     tc::tma_load_2d(sK(q) + kb * C::KBLK, &tmK, &qk_full[q], kb * 64, krow);
@@ -369,12 +402,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP(v) + kk * 32), 16, 1024);
+                    // A = P from TMEM: 16 keys = 8 packed columns per step
+                    const uint32_t pa = tmem + s * C::S_COL + C::P_OFF + kk * 8;
                     const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sV(v) + kk * 2048), 8192, 1024);
-                    tc::mma_bf16(tmem + C::O_COL + s * D, ad, bd, IDESC_O, kk ? 1u : 0u);
+                    tc::mma_bf16_ts(tmem + C::O_COL + s * D, pa, bd, IDESC_O, kk ? 1u : 0u);
                 }
                 tc::mma_commit(&ofull[s]);
                 tc::mma_commit(&vp_empty[v]);
+                tc::mma_commit(&pempty[s]);
             };
             auto issue_s = [&](int64_t j) {
                 const int s = (int)(j & 1), q = (int)(j % C::NQK);
@@ -430,7 +465,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
             const RowJob cur = read_row(ring[ri], e);
             tc::mbar_arrive(&ifree[ri]);
-            const int s = (int)(j & 1), v = (int)(j % C::NVP);
+            const int s = (int)(j & 1);
             const int64_t b = cur.tl.bg / Hkv;
             const int g = (int)(cur.tl.bg % Hkv);
             if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
@@ -443,38 +478,57 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&sfree[s]);
-            if (cur.valid && !cur.tl.own)
-                p.logits[((b * L + cur.t) * H + (int64_t)g * G + h) * topk + cur.k] =
-                    p.scale * (l_hi + l_lo);
-            const int nk = (cur.tl.own && cur.valid) ? (int)(cur.t - (int64_t)cur.tl.chunk * S) + 1 : 64;
-            float mx = -INFINITY;
+            // own-chunk rows see keys c*S .. t only: mask the rest to -inf
+            if (cur.tl.own) {
+                const int nk = cur.valid ? (int)(cur.t - (int64_t)cur.tl.chunk * S) + 1 : 64;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                if (c < nk) mx = fmaxf(mx, s0[c]);
-                if (c + 32 < nk) mx = fmaxf(mx, s1[c]);
+                for (int c = 0; c < 32; ++c) {
+                    if (c >= nk) s0[c] = -INFINITY;
+                    if (c + 32 >= nk) s1[c] = -INFINITY;
+                }
             }
-            const float ms = mx * p.scale_log2e;
-            float l = 0.f;
+            float m4[4] = {s0[0], s0[1], s1[0], s1[1]};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                s0[c] = c < nk ? tc::ex2_approx(fmaf(s0[c], p.scale_log2e, -ms)) : 0.f;
-                s1[c] = c + 32 < nk ? tc::ex2_approx(fmaf(s1[c], p.scale_log2e, -ms)) : 0.f;
-                l += s0[c] + s1[c];
+            for (int c = 2; c < 32; c += 2) {
+                m4[0] = tc::max3(m4[0], s0[c], s0[c + 1]);
+                m4[1] = tc::max3(m4[1], s1[c], s1[c + 1]);
             }
-            const float f = cur.valid ? (cur.tl.own ? (float)p.add_own : 1.f) / l : 0.f;
-            // P goes into V/P slot v, free once the P.V of tile j - NVP is done
-            if (j >= C::NVP && !wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort)) break;
-            uint8_t *prow = sP(v);
+            const float mx = fmaxf(fmaxf(m4[0], m4[2]), fmaxf(m4[1], m4[3]));
+            // P = 2^-6 exp(S*scale - rowmax), unnormalised: the 2^-6 (an
+            // exponent shift) keeps the chunk output P.V within max |V| for
+            // its fp16 store; 1/rowsum is applied by fuse_kernel
+            const float ms = fmaf(mx, p.scale_log2e, 6.f);
+            const uint64_t c2 = pack_f2(p.scale_log2e, p.scale_log2e), m2 = pack_f2(-ms, -ms);
+            uint64_t l2 = 0ull;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float *src = c < 4 ? s0 + 8 * c : s1 + 8 * (c - 4);
-                const uint4 u = make_uint4(pack_bf16x2(src[0] * f, src[1] * f),
-                                           pack_bf16x2(src[2] * f, src[3] * f),
-                                           pack_bf16x2(src[4] * f, src[5] * f),
-                                           pack_bf16x2(src[6] * f, src[7] * f));
-                *reinterpret_cast<uint4 *>(prow + tc::sw128_offset(r, c)) = u;
+            for (int c = 0; c < 32; c += 2) {
+                float a0, a1, b0, b1;
+                unpack_f2(ffma2(pack_f2(s0[c], s0[c + 1]), c2, m2), a0, a1);
+                unpack_f2(ffma2(pack_f2(s1[c], s1[c + 1]), c2, m2), b0, b1);
+                s0[c] = tc::ex2_approx(a0); s0[c + 1] = tc::ex2_approx(a1);
+                s1[c] = tc::ex2_approx(b0); s1[c + 1] = tc::ex2_approx(b1);
+                l2 = add_f2(l2, add_f2(pack_f2(s0[c], s0[c + 1]), pack_f2(s1[c], s1[c + 1])));
             }
-            tc::fence_proxy_async_smem();
+            if (cur.valid) {
+                const float f = (cur.tl.own ? (float)p.add_own : 1.f) / sum_f2(l2);
+                if (cur.tl.own)
+                    p.own_f[(b * L + cur.t) * H + (int64_t)g * G + h] = f;
+                else
+                    reinterpret_cast<float2 *>(p.zf)[((b * L + cur.t) * H + (int64_t)g * G + h) * topk + cur.k] =
+                        make_float2(p.scale * (l_hi + l_lo), f);
+            }
+            // P goes into TMEM next to S slot s (this thread's lane, keys packed
+            // in pairs), free once the P.V of tile j - 2 is done
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                pk[c] = pack_bf16x2(s0[2 * c], s0[2 * c + 1]);
+                pk[16 + c] = pack_bf16x2(s1[2 * c], s1[2 * c + 1]);
+            }
+            if (j >= 2 && !wait_bar(&pempty[s], reuse_parity(j >> 1), s_abort)) break;
+            tc::tmem_st32(tmem + s * C::S_COL + C::P_OFF + lane_off, pk);
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
             tc::mbar_arrive(&pfull[s]);
         }
     } else if (warp < kGatherWarp) {
@@ -538,15 +592,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 // ---------------------------------------------------------------- fusion
 // One warp per (t, h) row: w = softmax over the selected chunks of the
-// logits, O = own + sum_k w_k * partial_k.  Lane l holds the D/32 consecutive
-// elements d = l*D/32 ..; in the partial layout these are chunk l/(32/NCH),
-// offset (l % (32/NCH)) * D/32 -- the same d.  Slot loads are unrolled so
-// several are in flight.
+// logits, O = f_own * own + sum_k w_k * f_k * partial_k, f = the reciprocal
+// row sums of the unnormalised chunk outputs.  Lane l holds the D/32
+// consecutive elements d = l*D/32 ..; in the partial layout these are chunk
+// l/(32/NCH), offset (l % (32/NCH)) * D/32 -- the same d.  Slot loads are
+// unrolled so several are in flight.
 template <int D, int G>
 __global__ void __launch_bounds__(256)
 fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
-            const float *__restrict__ logits, const int32_t *__restrict__ idx, int64_t rows, int H,
-            int Hkv, int topk, float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
+            const float2 *__restrict__ zf, const float *__restrict__ own_f,
+            const int32_t *__restrict__ idx, int64_t rows, int H, int Hkv, int topk,
+            float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
     constexpr int EPL = D / 32;                      // elements per lane (4 or 2)
     constexpr int NCH = D / 32;                      // 32-wide chunks of d
     constexpr int LPC = 32 / NCH;                    // lanes per chunk
@@ -559,33 +615,35 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
     const int64_t srow = bt * Hkv + g;               // selection row (t, g)
     const int32_t ik = lane < topk ? idx[srow * topk + lane] : -1;
     const int nsel = __popc(__ballot_sync(0xffffffffu, ik >= 0));   // valid slots come first
-    const float lg = lane < nsel ? logits[row * topk + lane] : -INFINITY;
-    float m = lg;
+    const float2 z = lane < nsel ? zf[row * topk + lane] : make_float2(-INFINITY, 0.f);
+    float m = z.x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float ex = lane < nsel ? __expf(lg - m) : 0.f;
+    const float ex = lane < nsel ? __expf(z.x - m) : 0.f;
     float den = ex;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float w = nsel ? ex / den : 0.f;
     if (w_out && lane < topk) w_out[row * topk + lane] = w;
+    const float wf = w * z.y;                        // weight of the unnormalised slot output
 
     const int ch = lane / LPC, off = (lane % LPC) * EPL;
     float acc[EPL];
     {
+        const float fo = own_f[row];
         const __half2 *s2 = reinterpret_cast<const __half2 *>(own + row * D + lane * EPL);
 #pragma unroll
         for (int q = 0; q < EPL / 2; ++q) {
             const float2 v = __half22float2(s2[q]);
-            acc[2 * q] = v.x;
-            acc[2 * q + 1] = v.y;
+            acc[2 * q] = fo * v.x;
+            acc[2 * q + 1] = fo * v.y;
         }
     }
     const __half *pbase = part + (((srow * topk) * NCH + ch) * G + h) * 32 + off;
     const int64_t kstride = (int64_t)NCH * G * 32;   // halves between slots k and k+1
 #pragma unroll 8
     for (int k = 0; k < nsel; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, w, k);
+        const float wk = __shfl_sync(0xffffffffu, wf, k);
         const __half2 *s2 = reinterpret_cast<const __half2 *>(pbase + k * kstride);
 #pragma unroll
         for (int q = 0; q < EPL / 2; ++q) {
@@ -655,7 +713,7 @@ struct TcLaunch {
     const int32_t *idx, *entries;
     const int4 *tiles;                // one descriptor per queue position
     const int64_t *qlen;              // number of tiles (device)
-    float *logits, *w_out;
+    float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
     __half *part, *own;
     void *O;
     unsigned *status;
@@ -679,7 +737,7 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     TcParams p;
     p.tiles = a.tiles; p.qlen = a.qlen;
-    p.entries = a.entries; p.lm = a.lm; p.logits = a.logits;
+    p.entries = a.entries; p.lm = a.lm; p.zf = a.zf; p.own_f = a.own_f;
     p.part = a.part; p.own = a.own; p.status = a.status;
     p.L = a.L; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
@@ -693,7 +751,7 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     const int64_t rows = (int64_t)a.B * a.L * a.H;
     constexpr int kWarps = 8;
     fuse_kernel<D, G><<<(unsigned)((rows + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
-        a.part, a.own, a.logits, a.idx, rows, a.H, a.Hkv, a.topk, a.w_out,
+        a.part, a.own, (const float2 *)a.zf, a.own_f, a.idx, rows, a.H, a.Hkv, a.topk, a.w_out,
         (__nv_bfloat16 *)a.O);
     return cudaGetLastError();
 }
