@@ -20,7 +20,7 @@
 // Own tiles: 128/G consecutive tokens of a chunk against that chunk with the
 // causal mask (keys c*S .. t); their output (the own-chunk term, same scaling,
 // f = own_chunk / row sum) goes to an fp16 array.  fuse_kernel then completes
-// the method, one warp per (t, h):
+// the method, one warp per (t, g):
 //   w = softmax over the token's selected chunks of the logits,
 //   O = f_own * own + sum_k w_k * f_k * partial_k  (bf16 out).
 //
@@ -591,70 +591,102 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 // ---------------------------------------------------------------- fusion
-// One warp per (t, h) row: w = softmax over the selected chunks of the
-// logits, O = f_own * own + sum_k w_k * f_k * partial_k, f = the reciprocal
-// row sums of the unnormalised chunk outputs.  Lane l holds the D/32
-// consecutive elements d = l*D/32 ..; in the partial layout these are chunk
-// l/(32/NCH), offset (l % (32/NCH)) * D/32 -- the same d.  Slot loads are
-// unrolled so several are in flight.
+// One warp per (t, g): w = softmax over the token's selected chunks of the
+// logits (per head), O = f_own * own + sum_k w_k * f_k * partial_k, f = the
+// reciprocal row sums of the unnormalised chunk outputs.  A slot's partials
+// of the whole group are one contiguous block [d/32][G][32] fp16 (G*d*2
+// bytes), read with 16-byte loads: lane l takes pieces p = l + 32 i, i.e.
+// columns 8*(p%4) .. +8 of chunk p/(4G) of head (p/4) % G -- head l/4 (+8 i for
+// G = 16).  Four slots' loads are in flight at a time.
 template <int D, int G>
 __global__ void __launch_bounds__(256)
 fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
             const float2 *__restrict__ zf, const float *__restrict__ own_f,
-            const int32_t *__restrict__ idx, int64_t rows, int H, int Hkv, int topk,
+            const int32_t *__restrict__ idx, int64_t groups, int H, int Hkv, int topk,
             float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
-    constexpr int EPL = D / 32;                      // elements per lane (4 or 2)
-    constexpr int NCH = D / 32;                      // 32-wide chunks of d
-    constexpr int LPC = 32 / NCH;                    // lanes per chunk
+    constexpr int NP = G * D / 256;                  // 16-byte pieces per lane and slot
+    constexpr int HPL = G / 8;                       // heads per lane
+    static_assert(NP >= 1 && (NP % HPL) == 0, "pieces must cover the heads evenly");
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const int64_t bt = row / H;
-    const int hh = (int)(row % H);
-    const int g = hh / G, h = hh % G;
-    const int64_t srow = bt * Hkv + g;               // selection row (t, g)
-    const int32_t ik = lane < topk ? idx[srow * topk + lane] : -1;
-    const int nsel = __popc(__ballot_sync(0xffffffffu, ik >= 0));   // valid slots come first
-    const float2 z = lane < nsel ? zf[row * topk + lane] : make_float2(-INFINITY, 0.f);
-    float m = z.x;
+    const int64_t srow = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (srow >= groups) return;                      // srow = (b*L + t)*Hkv + g
+    const int64_t bt = srow / Hkv;
+    const int g = (int)(srow % Hkv);
+    const int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && idx[srow * topk + lane] >= 0));
+    // per-head fusion weights of this lane's heads (softmax over the valid slots)
+    float m[HPL], inv[HPL];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float ex = lane < nsel ? __expf(z.x - m) : 0.f;
-    float den = ex;
+    for (int j = 0; j < HPL; ++j) {
+        const int h = (lane >> 2) + 8 * j;
+        const float2 *zh = zf + ((bt * H + (int64_t)g * G + h) * topk);
+        float mm = -INFINITY;
+        for (int k = 0; k < nsel; ++k) mm = fmaxf(mm, zh[k].x);
+        float den = 0.f;
+        for (int k = 0; k < nsel; ++k) den += __expf(zh[k].x - mm);
+        m[j] = mm;
+        inv[j] = nsel ? 1.f / den : 0.f;
+        if (w_out && (lane & 3) == 0)
+            for (int k = 0; k < topk; ++k)
+                w_out[(bt * H + (int64_t)g * G + h) * topk + k] =
+                    k < nsel ? __expf(zh[k].x - mm) * inv[j] : 0.f;
+    }
+    // own term
+    float acc[NP][8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    const float w = nsel ? ex / den : 0.f;
-    if (w_out && lane < topk) w_out[row * topk + lane] = w;
-    const float wf = w * z.y;                        // weight of the unnormalised slot output
-
-    const int ch = lane / LPC, off = (lane % LPC) * EPL;
-    float acc[EPL];
-    {
-        const float fo = own_f[row];
-        const __half2 *s2 = reinterpret_cast<const __half2 *>(own + row * D + lane * EPL);
+    for (int i = 0; i < NP; ++i) {
+        const int pc = lane + 32 * i;
+        const int ch = pc / (4 * G), h = (pc >> 2) % G, q = pc & 3;
+        const int64_t hrow = bt * H + (int64_t)g * G + h;
+        const float fo = own_f[hrow];
+        const uint4 u = *reinterpret_cast<const uint4 *>(own + hrow * D + ch * 32 + q * 8);
+        const __half2 *h2 = reinterpret_cast<const __half2 *>(&u);
 #pragma unroll
-        for (int q = 0; q < EPL / 2; ++q) {
-            const float2 v = __half22float2(s2[q]);
-            acc[2 * q] = fo * v.x;
-            acc[2 * q + 1] = fo * v.y;
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h2[e]);
+            acc[i][2 * e] = fo * f.x;
+            acc[i][2 * e + 1] = fo * f.y;
         }
     }
-    const __half *pbase = part + (((srow * topk) * NCH + ch) * G + h) * 32 + off;
-    const int64_t kstride = (int64_t)NCH * G * 32;   // halves between slots k and k+1
-#pragma unroll 8
-    for (int k = 0; k < nsel; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, wf, k);
-        const __half2 *s2 = reinterpret_cast<const __half2 *>(pbase + k * kstride);
+    // retrieved slots, four at a time
+    const uint4 *pb = reinterpret_cast<const uint4 *>(part + srow * topk * (int64_t)(G * D));
+    for (int k0 = 0; k0 < nsel; k0 += 4) {
+        uint4 raw[4][NP];
+        float wk[4][HPL];
 #pragma unroll
-        for (int q = 0; q < EPL / 2; ++q) {
-            const float2 v = __half22float2(s2[q]);
-            acc[2 * q] = fmaf(wk, v.x, acc[2 * q]);
-            acc[2 * q + 1] = fmaf(wk, v.y, acc[2 * q + 1]);
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u < nsel ? k0 + u : k0;
+#pragma unroll
+            for (int i = 0; i < NP; ++i) raw[u][i] = pb[(int64_t)k * (G * D / 8) + lane + 32 * i];
+#pragma unroll
+            for (int j = 0; j < HPL; ++j) {
+                const int h = (lane >> 2) + 8 * j;
+                const float2 z = zf[(bt * H + (int64_t)g * G + h) * topk + k];
+                wk[u][j] = k0 + u < nsel ? __expf(z.x - m[j]) * inv[j] * z.y : 0.f;
+            }
         }
-    }
-    __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(O + row * D + lane * EPL);
 #pragma unroll
-    for (int q = 0; q < EPL / 2; ++q) dst[q] = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                const float w = wk[u][i % HPL];
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[u][i]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(h2[e]);
+                    acc[i][2 * e] = fmaf(w, f.x, acc[i][2 * e]);
+                    acc[i][2 * e + 1] = fmaf(w, f.y, acc[i][2 * e + 1]);
+                }
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+        const int pc = lane + 32 * i;
+        const int ch = pc / (4 * G), h = (pc >> 2) % G, q = pc & 3;
+        const int64_t hrow = bt * H + (int64_t)g * G + h;
+        *reinterpret_cast<uint4 *>(O + hrow * D + ch * 32 + q * 8) =
+            make_uint4(pack_bf16x2(acc[i][0], acc[i][1]), pack_bf16x2(acc[i][2], acc[i][3]),
+                       pack_bf16x2(acc[i][4], acc[i][5]), pack_bf16x2(acc[i][6], acc[i][7]));
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -748,10 +780,10 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     kern<<<(unsigned)a.num_sms, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t rows = (int64_t)a.B * a.L * a.H;
+    const int64_t groups = (int64_t)a.B * a.L * a.Hkv;
     constexpr int kWarps = 8;
-    fuse_kernel<D, G><<<(unsigned)((rows + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
-        a.part, a.own, (const float2 *)a.zf, a.own_f, a.idx, rows, a.H, a.Hkv, a.topk, a.w_out,
+    fuse_kernel<D, G><<<(unsigned)((groups + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
+        a.part, a.own, (const float2 *)a.zf, a.own_f, a.idx, groups, a.H, a.Hkv, a.topk, a.w_out,
         (__nv_bfloat16 *)a.O);
     return cudaGetLastError();
 }
