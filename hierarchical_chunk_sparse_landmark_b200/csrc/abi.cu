@@ -43,7 +43,7 @@ struct TcLaunch {
 };
 bool attend_tc_supported(bool bf16, int G, int d);
 int64_t attend_tc_max_windows();
-cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st);
+cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st, cudaEvent_t mid);
 }  // namespace hsa
 
 using namespace hsa;
@@ -205,6 +205,9 @@ thread_local int t_launches = 0;      // kernels launched by this thread's last 
 inline void stage_mark(int i, cudaStream_t st) {
     if (i < t_n_stage_events && t_stage_events[i]) cudaEventRecord(t_stage_events[i], st);
 }
+inline cudaEvent_t stage_event(int i) {
+    return i < t_n_stage_events ? t_stage_events[i] : nullptr;
+}
 
 }  // namespace
 
@@ -322,15 +325,16 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;
         a.num_sms = num_sms();
-        e = launch_attend_tc(a, d, st);
+        e = launch_attend_tc(a, d, st, stage_event(4));
         t_launches += e == cudaSuccess ? 2 : 0;
     } else {
         stage_mark(3, st);
         e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale,
                                O, st);
         t_launches += e == cudaSuccess ? 1 : 0;
+        stage_mark(4, st);            // the SIMT kernel fuses in place
     }
-    stage_mark(4, st);
+    stage_mark(5, st);
     return from_cuda(e);
 }
 

@@ -753,7 +753,7 @@ struct TcLaunch {
 };
 
 template <int D, int G>
-static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
+static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEvent_t mid) {
     using C = TcCfg<D, G>;
     CUtensorMap mq, mk, mv;
     // the single-box entry layout has a uniform 8-row atom stride only when an
@@ -780,6 +780,7 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st) {
     kern<<<(unsigned)a.num_sms, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (mid && (e = cudaEventRecord(mid, st)) != cudaSuccess) return e;
     const int64_t groups = (int64_t)a.B * a.L * a.Hkv;
     constexpr int kWarps = 8;
     fuse_kernel<D, G><<<(unsigned)((groups + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
@@ -796,10 +797,12 @@ bool attend_tc_supported(bool bf16, int G, int d) {
     return bf16 && (G == 8 || G == 16) && (d == 64 || d == 128) && encode_fn() != nullptr;
 }
 
-cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st) {
+// `mid` (may be null) is recorded between the attention and fusion kernels.
+cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st, cudaEvent_t mid) {
     const int G = a.H / a.Hkv;
-    if (d == 128) return G == 8 ? launch_attend_tc_t<128, 8>(a, st) : launch_attend_tc_t<128, 16>(a, st);
-    return G == 8 ? launch_attend_tc_t<64, 8>(a, st) : launch_attend_tc_t<64, 16>(a, st);
+    if (d == 128)
+        return G == 8 ? launch_attend_tc_t<128, 8>(a, st, mid) : launch_attend_tc_t<128, 16>(a, st, mid);
+    return G == 8 ? launch_attend_tc_t<64, 8>(a, st, mid) : launch_attend_tc_t<64, 16>(a, st, mid);
 }
 
 }  // namespace hsa

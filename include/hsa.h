@@ -189,8 +189,9 @@ hsa_status_t hsa_check(void *workspace, void *stream);
  * record events[i] (cudaEvent_t values passed as void*) on their stream at
  * stage boundary i, for i < n:
  *   hsa_prefill: 0 start, 1 after the landmark kernel (DHSA mode), 2 after
- *                selection, 3 after the work-list build, 4 after attention
- *                (end of the call);
+ *                selection, 3 after the work-list build, 4 after the
+ *                attention kernel, 5 after the fusion kernel (end of the
+ *                call; 4 and 5 coincide on the path that fuses in place);
  *   hsa_decode:  0 start, 1 end.
  * Boundaries a call does not reach are not recorded.  n must be 0..8.  The
  * events belong to the caller.  No effect on results.
