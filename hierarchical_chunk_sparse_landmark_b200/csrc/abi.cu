@@ -23,6 +23,10 @@ cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf
                           int S, int topk, float scale, int splits, const DecodeScratch &ws,
                           void *O, int32_t *idx_out, cudaStream_t st);
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
+bool select_tc_supported();
+cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, void *split, int B,
+                             int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
+                             int32_t *idx, unsigned *status, cudaStream_t st);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
@@ -105,7 +109,7 @@ struct PrefillLayout {
     bool tc;
     int64_t W, NW, cap;
     size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
-        seg_off, tiles_off, zf_off, ownf_off, part_off, own_off;
+        seg_off, tiles_off, zf_off, ownf_off, part_off, own_off, lmsplit_off;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
@@ -122,7 +126,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     p.W = p.NW = p.cap = 0;
     p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
     p.wntiles_off = p.done_off = p.seg_off = p.tiles_off = p.part_off = p.own_off = 0;
-    p.zf_off = p.ownf_off = 0;
+    p.zf_off = p.ownf_off = p.lmsplit_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
         p.W = tc_window(B, H, Hkv, L, d, topk, attend_tc_max_windows());
@@ -153,6 +157,8 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
         p.own_off = off;
         off = align_up(off + sizeof(__half) * (size_t)B * L * H * d, 256);
+        p.lmsplit_off = off;         // fp32 landmarks as two bf16 parts (tensor-core selection)
+        off = align_up(off + 2 * sizeof(__half) * (size_t)B * Hkv * Nc * d, 256);
     }
     p.total = off;
     return p;
@@ -160,6 +166,11 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
 
 bool force_simt_path() {
     const char *v = getenv("HSA_PREFILL_PATH");
+    return v && strcmp(v, "simt") == 0;
+}
+// Selection on CUDA cores even where the tensor-core selection applies (A/B checks).
+bool force_simt_select() {
+    const char *v = getenv("HSA_SELECT_PATH");
     return v && strcmp(v, "simt") == 0;
 }
 
@@ -296,10 +307,17 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                         attend_tc_supported(bf16, H / Hkv, d);
     // The tensor-core path computes the fusion logits inside its S tiles and
     // the weights in fuse_kernel, so the selection skips them there.
-    cudaError_t e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
-                                  use_tc ? nullptr : w, st);
+    cudaError_t e;
+    const bool tc_select = use_tc && L >= S && (H / Hkv) % 8 == 0 && select_tc_supported() &&
+                           !force_simt_select();
+    if (tc_select)
+        e = launch_select_tc(Q, lm_use, lm_bf16, ws + lay.lmsplit_off, B, H, Hkv, L, d, S, topk,
+                             scale, idx, (unsigned *)ws, st);
+    else
+        e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
+                          use_tc ? nullptr : w, st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
-    t_launches += 1;
+    t_launches += (tc_select && !lm_bf16) ? 2 : 1;     // fp32 landmarks: split + select
     stage_mark(2, st);
     if (use_tc) {
         const int64_t Nc = L / S;

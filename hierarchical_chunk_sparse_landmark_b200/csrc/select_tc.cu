@@ -1,0 +1,400 @@
+// select_tc.cu -- prefill chunk selection with the group scores on the
+// 5th-generation tensor cores.
+//
+// For each (b, t, g): qbar = mean of the G heads' queries, sbar_i = scale *
+// qbar . l_i over the visible chunks i < floor(t/S), and the top-K chunks by
+// (score desc, index asc).  (Per-token top-K retrieval over chunk landmarks:
+// Understanding and Improving Length Generalization in Hierarchical Sparse
+// Attention Models, "Methodology in Plain English".)
+//
+// Per (b, g) the scores are the dense product [L x d] . [d x Nc] (block-causal:
+// only chunks before a token's own chunk count), so they run as tcgen05 MMA
+// tiles: M = 128 tokens, N = 128 chunks, K = d, fp32 accumulate in TMEM.
+// bf16 operands keep fp32 accuracy by splitting: qbar = q0 + q1 + q2 (three
+// bf16 parts, exact for an fp32 value) against bf16 landmarks, or, for fp32
+// landmarks l = l0 + l1, qbar = q0 + q1 and the products q0.l0 + q1.l0 + q0.l1
+// (the q1.l1 term is below 2^-16 of the score and dropped).  The parts are
+// chained as one accumulation per tile.
+//
+// select_tc_kernel: one block per (128-token block, b*Hkv + g), heavy blocks
+// first.  All warps first build the qbar parts in shared memory (128-byte
+// swizzled, K-major); then
+//   warp 0      producer  (TMA of landmark tiles, two stages)
+//   warp 1      MMA issuer (one score tile per landmark tile, two TMEM buffers)
+//   warps 2-5   top-K     (thread = token = TMEM lane: causal mask, a sorted
+//                          register list of 64-bit keys, insertion only past
+//                          the current K-th key)
+// Every wait is bounded; on expiry the block sets the status flag, lets its
+// copies and MMAs land, frees its TMEM and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace hsa {
+
+template <int D, bool LM32>
+struct SelCfg {
+    static constexpr int M = 128;                 // tokens per block
+    static constexpr int N = 128;                 // chunks per tile
+    static constexpr int KB = D / 64;             // 64-element blocks of d
+    static constexpr int QP = LM32 ? 2 : 3;       // qbar parts
+    static constexpr int LP = LM32 ? 2 : 1;       // landmark parts
+    static constexpr int A_PART = M * D * 2;
+    static constexpr int B_PART = N * D * 2;
+    static constexpr int STAGES = 2;
+    static constexpr int B_STAGE = LP * B_PART;
+    static constexpr int BAR_OFF = QP * A_PART + STAGES * B_STAGE;
+    static constexpr int SMEM = 1024 + BAR_OFF + 256;
+    static constexpr uint32_t TMEM_COLS = 2 * N;
+};
+
+constexpr int kSelTcThreads = 192;                  // 6 warps
+constexpr long long kSelWait = 4000000000LL;        // SM cycles (about 2 s)
+
+struct SelTcParams {
+    const void *Q;                  // [B, L, H, D] bf16
+    int32_t *idx;                   // [B, L, Hkv, topk]
+    unsigned *status;
+    int64_t L, Nc;
+    int H, Hkv, S, topk;
+    float scale;
+};
+
+__device__ __forceinline__ bool sel_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!tc::mbar_try_wait(bar, parity)) {
+        if (*abort || clock64() - t0 > kSelWait) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+template <int D, bool LM32, int KP>
+__global__ void __launch_bounds__(kSelTcThreads, 1)
+select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant__ CUtensorMap tmL1,
+                 const SelTcParams p) {
+    using C = SelCfg<D, LM32>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;                                        // [QP][KB][M x 128 B]
+    auto sB = [&](int s) { return smem + C::QP * C::A_PART + s * C::B_STAGE; };   // [LP][KB][N x 128 B]
+    uint64_t *bars = (uint64_t *)(smem + C::BAR_OFF);
+    uint64_t *full = bars, *empty = bars + 2, *tfull = bars + 4, *tfree = bars + 6;
+    uint32_t *s_tmem = (uint32_t *)(bars + 8);
+    volatile int *s_abort = (volatile int *)(s_tmem + 1);
+
+    const int ntb = (int)((p.L + C::M - 1) / C::M);
+    const int tb = ntb - 1 - (int)blockIdx.x;                  // heavy blocks first
+    const int64_t bg = blockIdx.y;
+    const int64_t b = bg / p.Hkv;
+    const int g = (int)(bg % p.Hkv);
+    const int G = p.H / p.Hkv;
+    const int64_t L = p.L;
+    const int64_t t0 = (int64_t)tb * C::M;
+    const int64_t t_last = t0 + C::M - 1 < L ? t0 + C::M - 1 : L - 1;
+    const int64_t nvis_max = t_last / p.S;                     // visible to the block's last token
+    const int ntiles = (int)((nvis_max + C::N - 1) / C::N);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 1) {
+        tc::tmem_alloc(s_tmem, C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+            tc::mbar_init(&tfull[s], 1);
+            tc::mbar_init(&tfree[s], 128);
+        }
+        *s_abort = 0;
+        tc::fence_barrier_init();
+    }
+    // qbar = (1/G) sum_h q_h, split into bf16 parts, 128-byte swizzled K-major.
+    // A thread owns (token, 16-byte vector) pairs and keeps two pairs' loads of
+    // eight heads in flight (G is a multiple of 8 on this path).
+    {
+        constexpr int VPR = D / 8;                            // 16-byte vectors per row
+        constexpr int NPAIR = C::M * VPR;
+        const float inv_g = 1.f / (float)G;
+        for (int e0 = tid; e0 < NPAIR; e0 += 2 * kSelTcThreads) {
+            float acc[2][8];
+            const __nv_bfloat16 *qp[2];
+            bool live[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * kSelTcThreads;
+                const int r = e / VPR, c = e % VPR;
+                const int64_t t = t0 + r;
+                live[u] = e < NPAIR && t < L;
+                qp[u] = (const __nv_bfloat16 *)p.Q + ((b * L + (live[u] ? t : 0)) * p.H + (int64_t)g * G) * D + c * 8;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+            }
+            for (int h0 = 0; h0 < G; h0 += 8) {
+                uint4 raw[2][8];
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int h = 0; h < 8; ++h)
+                        raw[u][h] = live[u] ? ld_stream16(qp[u] + (int64_t)(h0 + h) * D) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        float f[8];
+                        Vec16<__nv_bfloat16>::unpack(raw[u][h], f);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[u][i] += f[i];
+                    }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * kSelTcThreads;
+                if (e >= NPAIR) continue;
+                const int r = e / VPR, c = e % VPR;
+                const uint32_t off = (uint32_t)((c / 8) * (C::M * 128)) + tc::sw128_offset(r, c % 8);
+                float x[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = acc[u][i] * inv_g;
+#pragma unroll
+                for (int part = 0; part < C::QP; ++part) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t lo = bf16_bits_rn(x[2 * i]), hi = bf16_bits_rn(x[2 * i + 1]);
+                        w[i] = lo | (hi << 16);
+                        x[2 * i] -= __uint_as_float(lo << 16);
+                        x[2 * i + 1] -= __uint_as_float(hi << 16);
+                    }
+                    *reinterpret_cast<uint4 *>(sA + part * C::A_PART + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        tc::fence_proxy_async_smem();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            for (int n = 0; n < ntiles; ++n) {
+                const int s = n & 1;
+                if (n >= 2 && !sel_wait(&empty[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
+                tc::mbar_expect_tx(&full[s], (uint32_t)C::B_STAGE);
+                const int row0 = (int)(bg * p.Nc + (int64_t)n * C::N);
+#pragma unroll
+                for (int lp = 0; lp < C::LP; ++lp)
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tc::tma_load_2d(sB(s) + lp * C::B_PART + kb * (C::N * 128), lp ? &tmL1 : &tmL0,
+                                        &full[s], kb * 64, row0);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = tc::idesc_bf16_f32(128, C::N, false);
+            // (qbar part, landmark part) of every product term
+            constexpr int NPROD = 3;
+            const int pa[NPROD] = {0, 1, LM32 ? 0 : 2};
+            const int pl[NPROD] = {0, 0, LM32 ? 1 : 0};
+            for (int n = 0; n < ntiles; ++n) {
+                const int s = n & 1;
+                if (!sel_wait(&full[s], (uint32_t)((n >> 1) & 1), s_abort)) break;
+                if (n >= 2 && !sel_wait(&tfree[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
+                tc::fence_after_sync();
+                uint32_t acc = 0;
+#pragma unroll
+                for (int pr = 0; pr < NPROD; ++pr)
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = tc::sdesc_sw128(
+                                tc::smem_u32(sA + pa[pr] * C::A_PART + kb * (C::M * 128) + kk * 32), 16, 1024);
+                            const uint64_t bd = tc::sdesc_sw128(
+                                tc::smem_u32(sB(s) + pl[pr] * C::B_PART + kb * (C::N * 128) + kk * 32), 16, 1024);
+                            tc::mma_bf16(tmem + s * C::N, ad, bd, IDESC, acc);
+                            acc = 1;
+                        }
+                tc::mma_commit(&tfull[s]);
+                tc::mma_commit(&empty[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ top-K
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int64_t t = t0 + r;
+        const int64_t nvis = t < L ? t / p.S : 0;
+        uint64_t v[KP];
+#pragma unroll
+        for (int i = 0; i < KP; ++i) v[i] = 0ull;
+        float tf = -INFINITY;                                  // score of v[KP-1]
+        for (int n = 0; n < ntiles; ++n) {
+            const int s = n & 1;
+            if (!sel_wait(&tfull[s], (uint32_t)((n >> 1) & 1), s_abort)) break;
+            tc::fence_after_sync();
+#pragma unroll 1
+            for (int cb = 0; cb < C::N / 32; ++cb) {
+                float sc[32];
+                tc::tmem_ld32(tmem + s * C::N + cb * 32 + lane_off, sc);
+                tc::tmem_wait_ld();
+                const int64_t c0 = (int64_t)n * C::N + cb * 32;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float sv = p.scale * sc[c];
+                    if (c0 + c < nvis && sv >= tf) {
+                        uint64_t x = make_key(sv, c0 + c);
+                        if (x > v[KP - 1]) {
+#pragma unroll
+                            for (int i = 0; i < KP; ++i) {
+                                const uint64_t hi = v[i] > x ? v[i] : x;
+                                x = v[i] > x ? x : v[i];
+                                v[i] = hi;
+                            }
+                            tf = key_score(v[KP - 1]);
+                        }
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&tfree[s]);
+        }
+        if (t < L) {
+            int32_t *dst = p.idx + ((b * L + t) * p.Hkv + g) * p.topk;
+#pragma unroll
+            for (int k = 0; k < KP; ++k)
+                if (k < p.topk) dst[k] = key_index(v[k]);
+        }
+    }
+
+    __syncthreads();
+    if (*s_abort) {
+        if (tid == 0) atomicOr(p.status, kFlagTimeout);
+        const long long t1 = clock64();
+        while (clock64() - t1 < 20000000) { }
+    }
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// fp32 landmarks -> two bf16 parts l0 = rn(x), l1 = rn(x - l0).
+__global__ void __launch_bounds__(256)
+split_landmarks_kernel(const float4 *__restrict__ lm, uint2 *__restrict__ l0, uint2 *__restrict__ l1,
+                       int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 x = lm[i];
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[4], r[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            h[e] = bf16_bits_rn(xs[e]);
+            r[e] = bf16_bits_rn(xs[e] - __uint_as_float(h[e] << 16));
+        }
+        l0[i] = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+        l1[i] = make_uint2(r[0] | (r[1] << 16), r[2] | (r[3] << 16));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*SelEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static SelEncodeFn sel_encode_fn() {
+    static SelEncodeFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = (SelEncodeFn)ptr;
+    }
+    return fn;
+}
+
+// bf16 landmark rows [rows, D]: boxes of 64 columns x 128 rows, 128-byte swizzle;
+// rows past the end read as zero.
+static bool sel_make_map(CUtensorMap *m, const void *base, uint64_t rows, int D) {
+    SelEncodeFn enc = sel_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64u, 128u};
+    const cuuint32_t es[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int D, bool LM32, int KP>
+static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l0, const void *l1,
+                                      cudaStream_t st) {
+    using C = SelCfg<D, LM32>;
+    const uint64_t rows = (uint64_t)B * p.Hkv * p.Nc;
+    CUtensorMap m0, m1;
+    if (!sel_make_map(&m0, l0, rows, D)) return cudaErrorInvalidValue;
+    if (LM32) {
+        if (!sel_make_map(&m1, l1, rows, D)) return cudaErrorInvalidValue;
+    } else {
+        m1 = m0;
+    }
+    auto kern = select_tc_kernel<D, LM32, KP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((p.L + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
+    kern<<<grid, kSelTcThreads, C::SMEM, st>>>(m0, m1, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool LM32>
+static cudaError_t launch_select_tc_k(const SelTcParams &p, int B, const void *l0, const void *l1,
+                                      cudaStream_t st) {
+    if (p.topk <= 8) return launch_select_tc_t<D, LM32, 8>(p, B, l0, l1, st);
+    if (p.topk <= 16) return launch_select_tc_t<D, LM32, 16>(p, B, l0, l1, st);
+    return launch_select_tc_t<D, LM32, 32>(p, B, l0, l1, st);
+}
+
+bool select_tc_supported() { return sel_encode_fn() != nullptr; }
+
+// Q bf16; landmarks bf16 (lm_bf16) or fp32 (split into `split` = 2 bf16 arrays
+// of B*Hkv*Nc*d elements first).  Nc = L / S >= 1; G = H / Hkv a multiple of 8.
+cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, void *split, int B,
+                             int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
+                             int32_t *idx, unsigned *status, cudaStream_t st) {
+    SelTcParams p;
+    p.Q = Q; p.idx = idx; p.status = status;
+    p.L = L; p.Nc = L / S; p.H = H; p.Hkv = Hkv; p.S = S; p.topk = topk; p.scale = scale;
+    const int64_t n = (int64_t)B * Hkv * p.Nc * d;
+    if (lm_bf16) {
+        return d == 128 ? launch_select_tc_k<128, false>(p, B, lm, nullptr, st)
+                        : launch_select_tc_k<64, false>(p, B, lm, nullptr, st);
+    }
+    __nv_bfloat16 *l0 = (__nv_bfloat16 *)split, *l1 = l0 + n;
+    const int64_t n4 = n / 4;
+    const unsigned blocks = (unsigned)((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
+    split_landmarks_kernel<<<blocks, 256, 0, st>>>((const float4 *)lm, (uint2 *)l0, (uint2 *)l1, n4);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return d == 128 ? launch_select_tc_k<128, true>(p, B, l0, l1, st)
+                    : launch_select_tc_k<64, true>(p, B, l0, l1, st);
+}
+
+}  // namespace hsa
