@@ -303,46 +303,72 @@ def run_ours(args, dist, rank, world):
 
 
 def e2e_prefill(args, wl, x, ws, dev, dist):
-    """Same metric through the public API with host buffers: pinned host ->
-    device copies of Q/K/V/landmarks, the call, and the device -> host copy of O,
-    all inside the timed region (CUDA events on the stream)."""
+    """Same metric through the public API with host buffers, as a serving loop
+    runs it: every step copies its Q/K/V/landmarks from pinned host memory to
+    the device, calls hsa_prefill and copies O back to pinned host memory.
+    Two buffer slots and three streams (host->device, compute, device->host)
+    let the copies of one step overlap the neighbouring steps; events keep a
+    slot's buffers until the step that last used them is done.  The timed
+    region runs from the first input copy to the last output copy."""
     import torch
 
     import hierarchical_chunk_sparse_landmark_b200 as hsa
     hQ, hK, hV = (x[k].cpu().pin_memory() for k in ("Q", "K", "V"))
     hlm = x["lm"].cpu().pin_memory() if x["lm"] is not None else None
-    dQ, dK, dV = torch.empty_like(x["Q"]), torch.empty_like(x["K"]), torch.empty_like(x["V"])
-    dlm = torch.empty_like(x["lm"]) if hlm is not None else None
-    hO = torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory()
-    dO = torch.empty_like(x["Q"])
-    steps = max(3, args.steps // 4)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
-
-    def one():
-        dQ.copy_(hQ, non_blocking=True)
-        dK.copy_(hK, non_blocking=True)
-        dV.copy_(hV, non_blocking=True)
-        if dlm is not None:
-            dlm.copy_(hlm, non_blocking=True)
-        hsa.prefill(dQ, dK, dV, dlm, S=wl.S, topk=wl.topk, own_chunk=wl.own_chunk, out=dO, ws=ws)
-        hO.copy_(dO, non_blocking=True)
-
+    slots = []
     for _ in range(2):
-        one()
+        slots.append({
+            "Q": torch.empty_like(x["Q"]), "K": torch.empty_like(x["K"]),
+            "V": torch.empty_like(x["V"]),
+            "lm": torch.empty_like(x["lm"]) if hlm is not None else None,
+            "O": torch.empty_like(x["Q"]),
+            "hO": torch.empty(x["Q"].shape, dtype=x["Q"].dtype).pin_memory(),
+            "in": torch.cuda.Event(), "comp": torch.cuda.Event(), "out": torch.cuda.Event()})
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    steps = max(4, args.steps // 2)
+
+    def issue(i):
+        sl = slots[i % 2]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(sl["comp"])          # step i-2 no longer reads the inputs
+            sl["Q"].copy_(hQ, non_blocking=True)
+            sl["K"].copy_(hK, non_blocking=True)
+            sl["V"].copy_(hV, non_blocking=True)
+            if hlm is not None:
+                sl["lm"].copy_(hlm, non_blocking=True)
+            sl["in"].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(sl["in"])
+            if i >= 2:
+                s_comp.wait_event(sl["out"])         # step i-2's O has been copied out
+            hsa.prefill(sl["Q"], sl["K"], sl["V"], sl["lm"], S=wl.S, topk=wl.topk,
+                        own_chunk=wl.own_chunk, out=sl["O"], ws=ws)
+            sl["comp"].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(sl["comp"])
+            sl["hO"].copy_(sl["O"], non_blocking=True)
+            sl["out"].record(s_out)
+
+    for i in range(2):
+        issue(i)
     torch.cuda.synchronize()
-    for a, b in ev:
-        a.record()
-        one()
-        b.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for i in range(steps):
+        issue(i)
+    s_out.wait_event(slots[(steps - 1) % 2]["out"])
+    t1.record(s_out)
     torch.cuda.synchronize()
-    secs = sum(a.elapsed_time(b) for a, b in ev) / 1e3
+    hsa.check(ws)
+    secs = t0.elapsed_time(t1) / 1e3
     flops = prefill_flops(wl)["total"]
     units, tmax = aggregate(dist, flops * steps / 1e12, secs, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV) + ((hlm,) if hlm is not None else ()))
     return {"value": round(units / tmax, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": hO.numel() * hO.element_size(), "steps": steps,
-            "ms_per_step": round(tmax * 1e3 / steps, 4)}
+            "d2h_bytes_per_step": slots[0]["hO"].numel() * slots[0]["hO"].element_size(),
+            "steps": steps, "ms_per_step": round(tmax * 1e3 / steps, 4),
+            "pipeline": "2 buffer slots; host->device, compute and device->host on separate streams"}
 
 
 def bench_decode(args, dev, peaks, rank, dist):
