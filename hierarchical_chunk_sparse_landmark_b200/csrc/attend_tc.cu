@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const TcParams p) {
     using C = TcCfg<D, G>;
+    grid_dep_wait();                      // the work lists are written by the previous kernels
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     // Q/K slot q: [Q | K;l]; V slot v
@@ -607,6 +608,7 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
     constexpr int NP = G * D / 256;                  // 16-byte pieces per lane and slot
     constexpr int HPL = G / 8;                       // heads per lane
     static_assert(NP >= 1 && (NP % HPL) == 0, "pieces must cover the heads evenly");
+    grid_dep_wait();                                 // the chunk outputs come from attend_tc_kernel
     const int lane = threadIdx.x & 31;
     const int64_t srow = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (srow >= groups) return;                      // srow = (b*L + t)*Hkv + g
@@ -777,16 +779,17 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     p.q3d = q3d ? 1 : 0;
     p.scale = a.scale;
     p.scale_log2e = a.scale * 1.4426950408889634f;
-    kern<<<(unsigned)a.num_sms, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3((unsigned)a.num_sms), dim3(kThreads), (size_t)C::SMEM, st, mq, mk, mv, p);
     if (e != cudaSuccess) return e;
+    // with a timing event between the two kernels the fusion kernel is launched
+    // plainly (an event between them ends the programmatic overlap anyway)
     if (mid && (e = cudaEventRecord(mid, st)) != cudaSuccess) return e;
     const int64_t groups = (int64_t)a.B * a.L * a.Hkv;
     constexpr int kWarps = 8;
-    fuse_kernel<D, G><<<(unsigned)((groups + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
-        a.part, a.own, (const float2 *)a.zf, a.own_f, a.idx, groups, a.H, a.Hkv, a.topk, a.w_out,
-        (__nv_bfloat16 *)a.O);
-    return cudaGetLastError();
+    const dim3 fgrid((unsigned)((groups + kWarps - 1) / kWarps));
+    return launch_pdl(fuse_kernel<D, G>, fgrid, dim3(32 * kWarps), 0, st, a.part, a.own,
+                      (const float2 *)a.zf, (const float *)a.own_f, (const int32_t *)a.idx, groups,
+                      a.H, a.Hkv, a.topk, a.w_out, (__nv_bfloat16 *)a.O);
 }
 
 // The work lists hold no per-window state in shared memory any more; the

@@ -44,6 +44,7 @@ __device__ __forceinline__ void window_span(const WinGeom &w, int64_t n, int64_t
 __global__ void __launch_bounds__(kBucketThreads)
 bucket_count_kernel(const int32_t *__restrict__ idx, WinGeom wg, int use_smem,
                     int32_t *__restrict__ counts) {
+    grid_dep_wait();
     extern __shared__ int32_t hist[];
     const int g = blockIdx.y, b = blockIdx.z;
     const int64_t bg = (int64_t)b * wg.Hkv + g;
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(kScanThreads)
 bucket_scan_kernel(const int32_t *__restrict__ counts, WinGeom wg, int32_t *__restrict__ cursor,
                    int4 *__restrict__ wtiles, int32_t *__restrict__ wntiles,
                    int32_t *__restrict__ done) {
+    grid_dep_wait();
     __shared__ int64_t warp_e[32], warp_t[32];
     const int64_t n = blockIdx.x;
     int64_t bg, t_start, t_end;
@@ -136,6 +138,7 @@ bucket_scan_kernel(const int32_t *__restrict__ counts, WinGeom wg, int32_t *__re
 __global__ void __launch_bounds__(kScanThreads)
 queue_order_kernel(const int32_t *__restrict__ wntiles, WinGeom wg, int64_t NW,
                    int64_t *__restrict__ seg_start) {
+    grid_dep_wait();
     __shared__ int64_t warp_s[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t nseg = 2 * NW;
@@ -186,6 +189,7 @@ __global__ void __launch_bounds__(kBucketThreads)
 flatten_tiles_kernel(const int4 *__restrict__ wtiles, const int32_t *__restrict__ wntiles,
                      const int64_t *__restrict__ seg_start, WinGeom wg,
                      int4 *__restrict__ tiles) {
+    grid_dep_wait();
     const int64_t n = blockIdx.x;
     int64_t bg, ts, te;
     window_span(wg, n, bg, ts, te);
@@ -204,6 +208,7 @@ flatten_tiles_kernel(const int4 *__restrict__ wtiles, const int32_t *__restrict_
 __global__ void __launch_bounds__(kBucketThreads)
 bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int32_t *__restrict__ cursor,
                       int32_t *__restrict__ entries) {
+    grid_dep_wait();
     const int g = blockIdx.y, b = blockIdx.z;
     const int64_t bg = (int64_t)b * wg.Hkv + g;
     const int64_t t = (int64_t)blockIdx.x * kBucketThreads + threadIdx.x;
@@ -229,22 +234,19 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
     dim3 grid((unsigned)((L + kBucketThreads - 1) / kBucketThreads), (unsigned)Hkv, (unsigned)B);
     const int use_smem = Nc <= 8192 ? 1 : 0;
     const size_t smem = use_smem ? sizeof(int32_t) * (size_t)(Nc > 0 ? Nc : 1) : 0;
+    // the count pass follows the counts memset (not a kernel): plain launch
     bucket_count_kernel<<<grid, kBucketThreads, smem, st>>>(idx, wg, use_smem, counts);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bucket_scan_kernel<<<(unsigned)NW, kScanThreads, 0, st>>>(counts, wg, cursor, wtiles, wntiles,
-                                                            done);
-    e = cudaGetLastError();
+    e = launch_pdl(bucket_scan_kernel, dim3((unsigned)NW), dim3(kScanThreads), 0, st, counts, wg,
+                   cursor, wtiles, wntiles, done);
     if (e != cudaSuccess) return e;
-    queue_order_kernel<<<1, kScanThreads, 0, st>>>(wntiles, wg, NW, seg_start);
-    e = cudaGetLastError();
+    e = launch_pdl(queue_order_kernel, dim3(1), dim3(kScanThreads), 0, st, wntiles, wg, NW, seg_start);
     if (e != cudaSuccess) return e;
-    bucket_scatter_kernel<<<grid, kBucketThreads, 0, st>>>(idx, wg, cursor, entries);
-    e = cudaGetLastError();
+    e = launch_pdl(bucket_scatter_kernel, grid, dim3(kBucketThreads), 0, st, idx, wg, cursor, entries);
     if (e != cudaSuccess) return e;
-    flatten_tiles_kernel<<<(unsigned)NW, kBucketThreads, 0, st>>>(wtiles, wntiles, seg_start, wg,
-                                                                  tiles);
-    return cudaGetLastError();
+    return launch_pdl(flatten_tiles_kernel, dim3((unsigned)NW), dim3(kBucketThreads), 0, st,
+                      wtiles, wntiles, seg_start, wg, tiles);
 }
 
 }  // namespace hsa

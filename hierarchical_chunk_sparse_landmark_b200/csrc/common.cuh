@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace hsa {
 
 // ---------------------------------------------------------------- element access
@@ -212,6 +214,30 @@ __device__ __forceinline__ uint64_t merge_regs8(uint64_t (&x)[8], int nr, int KP
 }
 __host__ __device__ constexpr int pow2_at_least(int k) {
     return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : k <= 8 ? 8 : k <= 16 ? 16 : 32;
+}
+
+// ---------------------------------------------------------------- launch chaining
+// Kernels of one call run in stream order.  A kernel launched with
+// launch_pdl may be scheduled while its predecessor drains (programmatic
+// dependent launch); it must call grid_dep_wait() before touching anything
+// the predecessor writes (the wait returns once that grid has completed and
+// its writes are visible; without a programmatic predecessor it returns at once).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------- status word

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kSelTcThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant__ CUtensorMap tmL1,
                  const SelTcParams p) {
     using C = SelCfg<D, LM32>;
+    grid_dep_wait();                      // landmarks may come from the previous kernels
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sA = smem;                                        // [QP][KB][M x 128 B]
@@ -296,6 +297,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
 __global__ void __launch_bounds__(256)
 split_landmarks_kernel(const float4 *__restrict__ lm, uint2 *__restrict__ l0, uint2 *__restrict__ l1,
                        int64_t n4) {
+    grid_dep_wait();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float4 x = lm[i];
@@ -360,8 +362,7 @@ static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((p.L + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
-    kern<<<grid, kSelTcThreads, C::SMEM, st>>>(m0, m1, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(kSelTcThreads), (size_t)C::SMEM, st, m0, m1, p);
 }
 
 template <int D, bool LM32>
@@ -390,8 +391,8 @@ cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, void *
     __nv_bfloat16 *l0 = (__nv_bfloat16 *)split, *l1 = l0 + n;
     const int64_t n4 = n / 4;
     const unsigned blocks = (unsigned)((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
-    split_landmarks_kernel<<<blocks, 256, 0, st>>>((const float4 *)lm, (uint2 *)l0, (uint2 *)l1, n4);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(split_landmarks_kernel, dim3(blocks), dim3(256), 0, st,
+                               (const float4 *)lm, (uint2 *)l0, (uint2 *)l1, n4);
     if (e != cudaSuccess) return e;
     return d == 128 ? launch_select_tc_k<128, true>(p, B, l0, l1, st)
                     : launch_select_tc_k<64, true>(p, B, l0, l1, st);
