@@ -204,23 +204,49 @@ flatten_tiles_kernel(const int4 *__restrict__ wtiles, const int32_t *__restrict_
     }
 }
 
-// entries[cursor[n, i]++] = t * 32 + k
+// entries[cursor[n, i]++] = t * 32 + k.  A block's 256 tokens lie in one window
+// (W is a multiple of 256).  With the chunk histogram in shared memory, each
+// entry takes its rank within the block by a shared atomic, the block reserves
+// each chunk's range with one global atomic, and the entries are written
+// at base + rank.
 __global__ void __launch_bounds__(kBucketThreads)
-bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int32_t *__restrict__ cursor,
-                      int32_t *__restrict__ entries) {
+bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int use_smem,
+                      int32_t *__restrict__ cursor, int32_t *__restrict__ entries) {
     grid_dep_wait();
+    extern __shared__ int32_t hist[];             // [Nc] counts, then range bases
     const int g = blockIdx.y, b = blockIdx.z;
-    const int64_t bg = (int64_t)b * wg.Hkv + g;
     const int64_t t = (int64_t)blockIdx.x * kBucketThreads + threadIdx.x;
-    if (t >= wg.L) return;
-    const int64_t n = bg * wg.nwb + t / wg.W;
-    const int32_t *ip = idx + (((int64_t)b * wg.L + t) * wg.Hkv + g) * wg.topk;
-    for (int k = 0; k < wg.topk; ++k) {
-        const int32_t i = ip[k];
-        if (i < 0) break;
-        const int32_t p = atomicAdd(&cursor[n * wg.Nc + i], 1);
-        entries[p] = (int32_t)(t * 32 + k);
+    const int64_t bg = (int64_t)b * wg.Hkv + g;
+    const int64_t n = bg * wg.nwb + ((int64_t)blockIdx.x * kBucketThreads) / wg.W;
+    const int32_t *ip = idx + (((int64_t)b * wg.L + (t < wg.L ? t : 0)) * wg.Hkv + g) * wg.topk;
+    if (!use_smem) {
+        if (t >= wg.L) return;
+        for (int k = 0; k < wg.topk; ++k) {
+            const int32_t i = ip[k];
+            if (i < 0) break;                       // padding only at the end
+            const int32_t pos = atomicAdd(&cursor[n * wg.Nc + i], 1);
+            entries[pos] = (int32_t)(t * 32 + k);
+        }
+        return;
     }
+    for (int64_t i = threadIdx.x; i < wg.Nc; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    int32_t chunk[32], rank[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        chunk[k] = -1;
+        if (k < wg.topk && t < wg.L) chunk[k] = ip[k];
+        rank[k] = chunk[k] >= 0 ? atomicAdd(&hist[chunk[k]], 1) : 0;
+    }
+    __syncthreads();
+    for (int64_t i = threadIdx.x; i < wg.Nc; i += blockDim.x) {
+        const int32_t c = hist[i];
+        hist[i] = c ? atomicAdd(&cursor[n * wg.Nc + i], c) : 0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+        if (chunk[k] >= 0) entries[hist[chunk[k]] + rank[k]] = (int32_t)(t * 32 + k);
 }
 
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
@@ -243,7 +269,8 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
     if (e != cudaSuccess) return e;
     e = launch_pdl(queue_order_kernel, dim3(1), dim3(kScanThreads), 0, st, wntiles, wg, NW, seg_start);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(bucket_scatter_kernel, grid, dim3(kBucketThreads), 0, st, idx, wg, cursor, entries);
+    e = launch_pdl(bucket_scatter_kernel, grid, dim3(kBucketThreads), smem, st, idx, wg, use_smem,
+                   cursor, entries);
     if (e != cudaSuccess) return e;
     return launch_pdl(flatten_tiles_kernel, dim3((unsigned)NW), dim3(kBucketThreads), 0, st,
                       wtiles, wntiles, seg_start, wg, tiles);
