@@ -24,6 +24,8 @@
 //   warps 2-5   top-K     (thread = token = TMEM lane: causal mask, a sorted
 //                          register list of 64-bit keys, insertion only past
 //                          the current K-th key)
+// (warps 6-11 only help build qbar; the first two landmark tiles are requested
+// before that, so their loads overlap it.)
 // Every wait is bounded; on expiry the block sets the status flag, lets its
 // copies and MMAs land, frees its TMEM and exits.
 #include <cuda.h>
@@ -49,7 +51,7 @@ struct SelCfg {
     static constexpr uint32_t TMEM_COLS = 2 * N;
 };
 
-constexpr int kSelTcThreads = 192;                  // 6 warps
+constexpr int kSelTcThreads = 384;                  // 12 warps (6-11 only help build qbar)
 constexpr long long kSelWait = 4000000000LL;        // SM cycles (about 2 s)
 
 struct SelTcParams {
@@ -119,6 +121,20 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         *s_abort = 0;
         tc::fence_barrier_init();
     }
+    // the first landmark tiles do not depend on qbar: start their loads now
+    auto issue_tile = [&](int n) {
+        const int s = n & 1;
+        tc::mbar_expect_tx(&full[s], (uint32_t)C::B_STAGE);
+        const int row0 = (int)(bg * p.Nc + (int64_t)n * C::N);
+#pragma unroll
+        for (int lp = 0; lp < C::LP; ++lp)
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+                tc::tma_load_2d(sB(s) + lp * C::B_PART + kb * (C::N * 128), lp ? &tmL1 : &tmL0,
+                                &full[s], kb * 64, row0);
+    };
+    if (tid == 0)
+        for (int n = 0; n < ntiles && n < C::STAGES; ++n) issue_tile(n);
     // qbar = (1/G) sum_h q_h, split into bf16 parts, 128-byte swizzled K-major.
     // A thread owns (token, 16-byte vector) pairs and keeps two pairs' loads of
     // eight heads in flight (G is a multiple of 8 on this path).
@@ -190,17 +206,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            for (int n = 0; n < ntiles; ++n) {
+            for (int n = C::STAGES; n < ntiles; ++n) {
                 const int s = n & 1;
-                if (n >= 2 && !sel_wait(&empty[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
-                tc::mbar_expect_tx(&full[s], (uint32_t)C::B_STAGE);
-                const int row0 = (int)(bg * p.Nc + (int64_t)n * C::N);
-#pragma unroll
-                for (int lp = 0; lp < C::LP; ++lp)
-#pragma unroll
-                    for (int kb = 0; kb < C::KB; ++kb)
-                        tc::tma_load_2d(sB(s) + lp * C::B_PART + kb * (C::N * 128), lp ? &tmL1 : &tmL0,
-                                        &full[s], kb * 64, row0);
+                if (!sel_wait(&empty[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
+                issue_tile(n);
             }
         }
     } else if (warp == 1) {
@@ -234,7 +243,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
                 tc::mma_commit(&empty[s]);
             }
         }
-    } else {
+    } else if (warp < 6) {
         // ------------------------------------------------------------ top-K
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
