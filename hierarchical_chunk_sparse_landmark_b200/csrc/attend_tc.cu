@@ -30,9 +30,8 @@
 // TMEM accumulators (S, P and O):
 //   warps 0, 15  producers (even / odd tiles: tile metadata into a shared
 //                           ring, landmark rows into the K slot, TMA of the
-//                           chunk's V)
-//   warp 14      Q/K loads (one TMA box per entry: its G query-head rows; the
-//                           chunk's K)
+//                           Q rows -- one box per entry, its G query-head rows
+//                           -- and of the chunk's K and V)
 //   warp 1       MMA issuer (S of the next tile or P.V of the oldest pending
 //                           one, whichever is ready)
 //   warps 2-5    softmax   (thread = tile row = TMEM lane)
@@ -96,7 +95,7 @@ struct TcParams {
 constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
 constexpr int kThreads = 512;                       // 16 warps
 constexpr int kEpiWarp0 = 6;                        // epilogue groups: warps 6-9 and 10-13
-constexpr int kGatherWarp = 14;                     // Q and K loads
+constexpr int kEpiEnd = 14;                         // epilogue warps end here; warp 14 has no role
 constexpr int kProducer2 = 15;                      // second producer (odd tiles)
 constexpr int kOwnTileFlag = 1 << 30;               // in a descriptor's .w (bucket.cu)
 
@@ -213,7 +212,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     if (tid == 0) {
         for (int q = 0; q < C::NQK; ++q) {
-            tc::mbar_init(&qk_full[q], 2);     // Q/K loads + landmark rows
+            tc::mbar_init(&qk_full[q], 1);     // producer: landmark rows written, Q/K loads expected
             tc::mbar_init(&qk_empty[q], 1);    // S MMA done
         }
         for (int v = 0; v < C::NVP; ++v) {
@@ -230,7 +229,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         for (int i = 0; i < kRing; ++i) {
             tc::mbar_init(&ifull[i], 1);
-            tc::mbar_init(&ifree[i], 257);     // softmax + one epilogue group + Q/K loader
+            tc::mbar_init(&ifree[i], 256);     // softmax + one epilogue group
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -334,55 +333,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tc::fence_proxy_async_smem();
             }
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&qk_full[q]);
-
-            // V of the chunk into V slot j % 3, free once the P.V of tile j - 3
-            // is done
-            const int v = (int)(j % C::NVP);
+            // Q rows (one TMA box per entry: all G query-head rows, both halves of d
+            // when the 3-D view is available) and the chunk's K
+            const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
             if (lane == 0) {
-                if (j >= C::NVP) ok = wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort);
-                if (ok) {
-                    tc::mbar_expect_tx(&v_full[v], (uint32_t)C::V_BYTES);
-                    const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
-#pragma unroll
-                    for (int kb = 0; kb < C::KB; ++kb)
-                        tc::tma_load_2d(sV(v) + kb * 8192, &tmV, &v_full[v], kb * 64, krow);
-                }
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        }
-        tc::cp_async_wait<0>();
-    } else if (warp == kGatherWarp) {
-        // ------------------------------------------------------------ Q/K loads
-        // One TMA box per entry (all G query-head rows, both halves of d when
-        // the 3-D view is available) plus the chunk's K.
-        for (int64_t j = 0; j < my_tiles; ++j) {
-            const int ri = (int)(j & (kRing - 1));
-            int ok = 1;
-            if (lane == 0) ok = wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const TileInfo &ti = ring[ri];
-            const int n = ti.n;
-            const int64_t bg = ti.bg;
-            const int chunk = ti.chunk;
-            const int32_t code = lane < n ? ti.code[lane] : 0;
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&ifree[ri]);
-            const int krow = (int)(bg * L + (int64_t)chunk * S);
-            const int q = (int)(j % C::NQK);
-            if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const int64_t b = bg / Hkv;
-            const int g = (int)(bg % Hkv);
-            if (lane == 0) {
-                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(n * G * D * 2 + C::K_TMA_BYTES));
+                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(d0.n * G * D * 2 + C::K_TMA_BYTES));
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
                     tc::tma_load_2d(sK(q) + kb * C::KBLK, &tmK, &qk_full[q], kb * 64, krow);
             }
             __syncwarp();
-            if (lane < n) {
-                const int qrow = (int)((b * L + (int64_t)(code >> 5)) * H + (int64_t)g * G);
+            if (lane < d0.n) {
+                const int64_t bq = d0.bg / Hkv;
+                const int gq = (int)(d0.bg % Hkv);
+                const int qrow = (int)((bq * L + (int64_t)(c0 >> 5)) * H + (int64_t)gq * G);
                 if (p.q3d) {
                     tc::tma_load_3d(sQ(q) + lane * (C::KB * G * 128), &tmQ, &qk_full[q], 0, qrow, 0);
                 } else {
@@ -392,7 +356,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                         kb * 64, qrow);
                 }
             }
+
+            // V of the chunk into V slot j % 3, free once the P.V of tile j - 3
+            // is done
+            const int v = (int)(j % C::NVP);
+            if (lane == 0) {
+                if (j >= C::NVP) ok = wait_bar(&vp_empty[v], reuse_parity(j / C::NVP), s_abort);
+                if (ok) {
+                    tc::mbar_expect_tx(&v_full[v], (uint32_t)C::V_BYTES);
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tc::tma_load_2d(sV(v) + kb * 8192, &tmV, &v_full[v], kb * 64, krow);
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         }
+        tc::cp_async_wait<0>();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -532,7 +511,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::fence_before_sync();
             tc::mbar_arrive(&pfull[s]);
         }
-    } else if (warp < kGatherWarp) {
+    } else if (warp < kEpiEnd) {
         // ------------------------------------------------------------ epilogue
         // Two groups of four warps; group eg takes the tiles j = eg, eg+2, ...
         // (TMEM O slot eg), so one tile's stores overlap the next one's.
