@@ -21,7 +21,9 @@
 // ~index) keys in a warp-distributed top-K.  Blocks publish their K best keys
 // and take a ticket; the last block of each (b, g) merges all candidates with
 // warp-parallel selection, writes the selection and resets the ticket.  No
-// block waits for another.
+// block waits for another.  (Prefetching the selected K/V chunks into L2 from
+// that block was tried: it lengthened the scan's tail by more than it saved
+// the attend kernel.)
 //
 // decode_attend_kernel (launched as a programmatic dependent of the scan, so
 // its launch and its query loads overlap the scan's tail): one cluster of
@@ -65,9 +67,8 @@ __device__ __forceinline__ uint64_t merge_smem_lists(const uint64_t (*lists)[32]
 // SMs that stream faster take more units.
 template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kScanThreads)
-decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T *__restrict__ Kc,
-                   const T *__restrict__ Vc, int H, int Hkv, int64_t Nc, int S, int topk,
-                   float scale, int splits, DecodeScratch ws, int32_t *__restrict__ idx_out) {
+decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, int Hkv, int64_t Nc,
+                   int topk, float scale, int splits, DecodeScratch ws, int32_t *__restrict__ idx_out) {
     constexpr int ROW_BYTES = D * (int)sizeof(TL);
     constexpr int ROWS = kStageBytes / ROW_BYTES;           // landmark rows per stage (one unit)
     constexpr int VEC = Vec16<TL>::N;                        // elements per 16-byte vector
@@ -252,12 +253,6 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T *
             const int32_t i = key_index(best);
             ws.sel[bg * topk + lane] = i;
             if (idx_out) idx_out[bg * topk + lane] = i;
-            if (i >= 0) {                     // warm L2 with the chunks the attend kernel reads
-                const size_t off = ((size_t)bg * Nc * S + (size_t)i * S) * D;
-                const uint32_t bytes = (uint32_t)(S * D * sizeof(T));
-                tc::prefetch_l2(Kc + off, bytes);
-                tc::prefetch_l2(Vc + off, bytes);
-            }
         }
         if (lane == 0) {                      // ready for the next call
             ws.tickets[bg] = 0u;
@@ -529,8 +524,7 @@ static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc
                                          kScanStages * kStageBytes);
     if (e != cudaSuccess) return e;
     scan<<<grid, kScanThreads, kScanStages * kStageBytes, st>>>(
-        (const T *)q, (const TL *)lm, (const T *)Kc, (const T *)Vc, H, Hkv, Nc, S, topk, scale,
-        splits, ws, idx_out);
+        (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws, idx_out);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
