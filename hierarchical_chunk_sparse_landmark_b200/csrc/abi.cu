@@ -1,6 +1,6 @@
 // abi.cu -- the extern "C" entry points of libhsa (declared in include/hsa.h):
 // argument validation, workspace layout and kernel dispatch.
-#include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -40,7 +40,7 @@ struct TcLaunch {
     const int4 *tiles;                // one descriptor per queue position
     const int64_t *qlen;              // number of tiles (device)
     float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
-    __half *part, *own;
+    __nv_bfloat16 *part, *own;
     void *O;
     unsigned *status;
     int num_sms;
@@ -154,11 +154,11 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         p.ownf_off = off;
         off = align_up(off + sizeof(float) * (size_t)B * L * H, 256);
         p.part_off = off;
-        off = align_up(off + sizeof(__half) * (size_t)B * L * H * topk * d, 256);
+        off = align_up(off + sizeof(__nv_bfloat16) * (size_t)B * L * H * topk * d, 256);
         p.own_off = off;
-        off = align_up(off + sizeof(__half) * (size_t)B * L * H * d, 256);
+        off = align_up(off + sizeof(__nv_bfloat16) * (size_t)B * L * H * d, 256);
         p.lmsplit_off = off;         // fp32 landmarks as two bf16 parts (tensor-core selection)
-        off = align_up(off + 2 * sizeof(__half) * (size_t)B * Hkv * Nc * d, 256);
+        off = align_up(off + 2 * sizeof(__nv_bfloat16) * (size_t)B * Hkv * Nc * d, 256);
     }
     p.total = off;
     return p;
@@ -340,7 +340,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.qlen = (const int64_t *)(ws + lay.seg_off) + 2 * lay.NW;
         a.zf = (float *)(ws + lay.zf_off); a.own_f = (float *)(ws + lay.ownf_off);
         a.w_out = w_out;
-        a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
+        a.part = (__nv_bfloat16 *)(ws + lay.part_off); a.own = (__nv_bfloat16 *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;
         a.num_sms = num_sms();
         e = launch_attend_tc(a, d, st, stage_event(4));

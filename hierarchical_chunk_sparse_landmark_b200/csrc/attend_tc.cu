@@ -12,14 +12,14 @@
 // fusion logit scale * q_h . l_chunk:
 //
 //   S = Q_rows . [K_chunk ; l_hi ; l_lo]^T  M=128, N=80, K=d  (tcgen05 -> TMEM)
-//   P = 2^-6 exp(S*scale - rowmax)          per row in registers, bf16 -> TMEM
+//   P = exp(S*scale - rowmax)               per row in registers, bf16 -> TMEM
 //   O = P . V_chunk                         M=128, N=d, K=64  (tcgen05, A from TMEM)
-//   partial[t, g, k] = O (fp16); per (t, h, k): the fusion logit
+//   partial[t, g, k] = O (bf16); per (t, h, k): the fusion logit
 //   scale * (S[:,64] + S[:,65]) and f = 1 / sum of the row's P
 //
 // Own tiles: 128/G consecutive tokens of a chunk against that chunk with the
 // causal mask (keys c*S .. t); their output (the own-chunk term, same scaling,
-// f = own_chunk / row sum) goes to an fp16 array.  fuse_kernel then completes
+// f = own_chunk / row sum) goes to a bf16 array.  fuse_kernel then completes
 // the method, one warp per (t, g):
 //   w = softmax over the token's selected chunks of the logits,
 //   O = f_own * own + sum_k w_k * f_k * partial_k  (bf16 out).
@@ -35,13 +35,13 @@
 //   warp 1       MMA issuer (S of the next tile or P.V of the oldest pending
 //                           one, whichever is ready)
 //   warps 2-5    softmax   (thread = tile row = TMEM lane)
-//   warps 6-13   epilogue  (two groups taking alternate tiles; TMEM -> fp16
+//   warps 6-13   epilogue  (two groups taking alternate tiles; TMEM -> bf16
 //                           partial slots / own-chunk term)
 // Tiles are independent, so no block waits on another.  Every wait is
 // bounded; on expiry the block sets the status flag in the workspace, lets
 // in-flight copies land, frees its TMEM and exits.
 #include <cuda.h>
-#include <cuda_fp16.h>
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -83,8 +83,8 @@ struct TcParams {
     const void *lm;               // [B, Hkv, Nc, D] bf16 or fp32
     float *zf;                    // [B, L, H, topk] x (fusion logit, 1 / chunk row sum)
     float *own_f;                 // [B, L, H] add_own / own-chunk row sum
-    __half *part;                 // [B*L*Hkv*topk entries][D/32][G][32] chunk outputs
-    __half *own;                  // [B, L, H, D] own-chunk term
+    __nv_bfloat16 *part;          // [B*L*Hkv*topk entries][D/8][G][8] chunk outputs
+    __nv_bfloat16 *own;           // [B*L*Hkv rows (t, g)][D/8][G][8] own-chunk term
     unsigned *status;
     int64_t L, Nc;
     int H, Hkv, topk, S, add_own, lm_bf16;
@@ -103,9 +103,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&v);
 }
-__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
-    __half2 v = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&v);
+// Two floats to a bf16 pair on the integer pipe: add half an ulp of bf16 to
+// the fp32 bit pattern and keep the high halves (one byte permute).  Rounds to
+// nearest with ties away from zero (round-to-nearest-even differs only on
+// exact ties).  The conversion instruction shares the transcendental pipe
+// with ex2, which the softmax keeps busy; the integer pipe is mostly idle.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float a, float b) {
+    return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+}
+// 2^x of two packed floats (x <= 0) on the FMA pipe, so that part of the
+// softmax's exponentials leave the MUFU unit: Cody-Waite style reduction
+// x = n + f with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to an
+// integer) and |f| <= 1/2, a cubic for 2^f, and n added to the exponent
+// field.  The cubic's coefficients are a least-squares fit of 2^f on
+// [-1/2, 1/2] in relative error (iteratively reweighted towards the minimax
+// fit); its relative error is below 7.5e-5, under the 2^-9 of the bf16 P it
+// feeds.  x is clamped at -126 so the exponent field stays >= 0: inputs below
+// that (and -inf, the causal mask) give a value below 2^-125 instead of 0.
+constexpr int kPolyPairs = 0;   // of the 16 column pairs of each 32-column half
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    float a, b;
+    unpack_f2(x2, a, b);
+    const uint64_t x = pack_f2(fmaxf(a, -126.f), fmaxf(b, -126.f));
+    const uint64_t j = add_f2(x, pack_f2(12582912.f, 12582912.f));          // low bits: round(x)
+    const uint64_t n = add_f2(j, pack_f2(-12582912.f, -12582912.f));
+    const uint64_t f = ffma2(n, pack_f2(-1.f, -1.f), x);                     // x - n
+    uint64_t y = ffma2(pack_f2(0.0551716685f, 0.0551716685f), f, pack_f2(0.242611140f, 0.242611140f));
+    y = ffma2(y, f, pack_f2(0.693260968f, 0.693260968f));
+    y = ffma2(y, f, pack_f2(0.999928057f, 0.999928057f));
+    float y0, y1, j0, j1;
+    unpack_f2(y, y0, y1);
+    unpack_f2(j, j0, j1);
+    return pack_f2(__uint_as_float(__float_as_uint(y0) + (__float_as_uint(j0) << 23)),
+                   __uint_as_float(__float_as_uint(y1) + (__float_as_uint(j1) << 23)));
+}
+
+// bf16 pair -> two floats (exact: the bf16 bits are the high half of fp32)
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
 // Bounded mbarrier wait that also gives up when another role aborted.
@@ -137,7 +172,7 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Ti
     if (!tl.own) {
         tl.chunk = d.y; tl.first = d.z; tl.t0 = 0;
     } else {
-        tl.t0 = d.z; tl.chunk = (int)(tl.t0 / p.S); tl.first = 0;
+        tl.t0 = d.z; tl.chunk = (int)(tl.t0 >> 6); tl.first = 0;     // S = 64 on this path
     }
 }
 
@@ -147,7 +182,7 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Ti
 constexpr int kRing = 4;
 struct TileInfo {
     int64_t bg;
-    int chunk, n, own, pad;
+    int chunk, n, own, b, g, pad;  // bg = b * Hkv + g, split once by the producer
     int32_t code[16];
 };
 
@@ -165,7 +200,7 @@ struct alignas(16) TileMetaT {
 struct RowJob {
     Tile tl;
     int64_t t;
-    int k;
+    int k, b, g;
     bool valid;
 };
 
@@ -173,6 +208,7 @@ __device__ __forceinline__ RowJob read_row(const TileInfo &ti, int e) {
     RowJob rj;
     rj.tl.bg = ti.bg; rj.tl.chunk = ti.chunk; rj.tl.n = ti.n;
     rj.tl.own = ti.own; rj.tl.first = 0; rj.tl.t0 = 0;
+    rj.b = ti.b; rj.g = ti.g;
     rj.valid = e < ti.n;
     const int32_t code = rj.valid ? ti.code[e] : 0;
     rj.t = code >> 5;
@@ -289,6 +325,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             Tile d0;
             decode_tile(p, mt.desc, d0);
             const int32_t c0 = lane < d0.n ? (d0.own ? (int32_t)((d0.t0 + lane) * 32) : mt.code[lane]) : 0;
+            const int bq = (int)d0.bg / Hkv;            // bg < 2^31 (checked on the host)
+            const int gq = (int)d0.bg - bq * Hkv;
 
             // publish the tile's metadata
             const int ri = (int)(j & (kRing - 1));
@@ -299,6 +337,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (lane == 0) {
                 ring[ri].bg = d0.bg; ring[ri].chunk = d0.chunk;
                 ring[ri].n = d0.n; ring[ri].own = d0.own;
+                ring[ri].b = bq; ring[ri].g = gq;
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ifull[ri]);
@@ -344,8 +383,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             __syncwarp();
             if (lane < d0.n) {
-                const int64_t bq = d0.bg / Hkv;
-                const int gq = (int)(d0.bg % Hkv);
                 const int qrow = (int)((bq * L + (int64_t)(c0 >> 5)) * H + (int64_t)gq * G);
                 if (p.q3d) {
                     tc::tma_load_3d(sQ(q) + lane * (C::KB * G * 128), &tmQ, &qk_full[q], 0, qrow, 0);
@@ -446,8 +483,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const RowJob cur = read_row(ring[ri], e);
             tc::mbar_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
-            const int64_t b = cur.tl.bg / Hkv;
-            const int g = (int)(cur.tl.bg % Hkv);
+            const int64_t b = cur.b;
+            const int g = cur.g;
             if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
             float s0[32], s1[32], l_hi, l_lo;
@@ -474,23 +511,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 m4[1] = tc::max3(m4[1], s1[c], s1[c + 1]);
             }
             const float mx = fmaxf(fmaxf(m4[0], m4[2]), fmaxf(m4[1], m4[3]));
-            // P = 2^-6 exp(S*scale - rowmax), unnormalised: the 2^-6 (an
-            // exponent shift) keeps the chunk output P.V within max |V| for
-            // its fp16 store; 1/rowsum is applied by fuse_kernel
-            const float ms = fmaf(mx, p.scale_log2e, 6.f);
+            // P = exp(S*scale - rowmax), unnormalised (1/rowsum is applied by
+            // fuse_kernel; P.V stays within 64 max |V|, far inside bf16 range)
+            const float ms = mx * p.scale_log2e;
             const uint64_t c2 = pack_f2(p.scale_log2e, p.scale_log2e), m2 = pack_f2(-ms, -ms);
             uint64_t l2 = 0ull;
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
                 float a0, a1, b0, b1;
-                unpack_f2(ffma2(pack_f2(s0[c], s0[c + 1]), c2, m2), a0, a1);
-                unpack_f2(ffma2(pack_f2(s1[c], s1[c + 1]), c2, m2), b0, b1);
-                s0[c] = tc::ex2_approx(a0); s0[c + 1] = tc::ex2_approx(a1);
-                s1[c] = tc::ex2_approx(b0); s1[c + 1] = tc::ex2_approx(b1);
+                const uint64_t xa = ffma2(pack_f2(s0[c], s0[c + 1]), c2, m2);
+                const uint64_t xb = ffma2(pack_f2(s1[c], s1[c + 1]), c2, m2);
+                if (c / 2 < kPolyPairs) {
+                    unpack_f2(exp2_poly2(xa), s0[c], s0[c + 1]);
+                } else {
+                    unpack_f2(xa, a0, a1);
+                    s0[c] = tc::ex2_approx(a0); s0[c + 1] = tc::ex2_approx(a1);
+                }
+                if (c / 2 < kPolyPairs) {
+                    unpack_f2(exp2_poly2(xb), s1[c], s1[c + 1]);
+                } else {
+                    unpack_f2(xb, b0, b1);
+                    s1[c] = tc::ex2_approx(b0); s1[c + 1] = tc::ex2_approx(b1);
+                }
                 l2 = add_f2(l2, add_f2(pack_f2(s0[c], s0[c + 1]), pack_f2(s1[c], s1[c + 1])));
             }
             if (cur.valid) {
-                const float f = (cur.tl.own ? (float)p.add_own : 1.f) / sum_f2(l2);
+                const float f = __fdividef(cur.tl.own ? (float)p.add_own : 1.f, sum_f2(l2));
                 if (cur.tl.own)
                     p.own_f[(b * L + cur.t) * H + (int64_t)g * G + h] = f;
                 else
@@ -502,8 +548,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             uint32_t pk[32];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                pk[c] = pack_bf16x2(s0[2 * c], s0[2 * c + 1]);
-                pk[16 + c] = pack_bf16x2(s1[2 * c], s1[2 * c + 1]);
+                pk[c] = pack_bf16x2_int(s0[2 * c], s0[2 * c + 1]);
+                pk[16 + c] = pack_bf16x2_int(s1[2 * c], s1[2 * c + 1]);
             }
             if (j >= 2 && !wait_bar(&pempty[s], reuse_parity(j >> 1), s_abort)) break;
             tc::tmem_st32(tmem + s * C::S_COL + C::P_OFF + lane_off, pk);
@@ -527,10 +573,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const RowJob cur = read_row(ring[ri], e);
             tc::mbar_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
-            const int64_t b = cur.tl.bg / Hkv;
-            const int g = (int)(cur.tl.bg % Hkv);
-            const int64_t row = (b * L + cur.t) * Hkv + g;       // (t, g) selection row
-            const int64_t hrow = (b * L + cur.t) * H + (int64_t)g * G + h;
+            const int64_t b = cur.b;
+            const int g = cur.g;
+            // one contiguous G*D block per (t, g, k) (own term: per (t, g)), 16-byte
+            // pieces ordered [d/8][head]: the G heads' pieces of a column group
+            // are adjacent, so every store instruction writes whole lines
+            const int64_t row = (b * L + cur.t) * Hkv + g;
+            uint4 *blk = reinterpret_cast<uint4 *>(cur.tl.own ? p.own + row * (G * D)
+                                                              : p.part + (row * topk + cur.k) * (G * D));
             if (!wait_bar(&ofull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
 #pragma unroll 1
@@ -543,15 +593,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 if (!cur.valid) continue;
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    // retrieved chunk: slot [entry][d/32][head][32]; own chunk: [t, h, d]
-                    __half *dst = cur.tl.own
-                        ? p.own + hrow * D + (ch + u) * 32
-                        : p.part + (((row * topk + cur.k) * NCH + ch + u) * G + h) * 32;
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq)
-                        reinterpret_cast<uint4 *>(dst)[qq] = make_uint4(
-                            pack_f16x2(o[u][8 * qq + 0], o[u][8 * qq + 1]), pack_f16x2(o[u][8 * qq + 2], o[u][8 * qq + 3]),
-                            pack_f16x2(o[u][8 * qq + 4], o[u][8 * qq + 5]), pack_f16x2(o[u][8 * qq + 6], o[u][8 * qq + 7]));
+                        blk[((ch + u) * 4 + qq) * G + h] = make_uint4(
+                            pack_bf16x2_int(o[u][8 * qq + 0], o[u][8 * qq + 1]),
+                            pack_bf16x2_int(o[u][8 * qq + 2], o[u][8 * qq + 3]),
+                            pack_bf16x2_int(o[u][8 * qq + 4], o[u][8 * qq + 5]),
+                            pack_bf16x2_int(o[u][8 * qq + 6], o[u][8 * qq + 7]));
                 }
             }
             tc::fence_before_sync();
@@ -574,56 +622,49 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // One warp per (t, g): w = softmax over the token's selected chunks of the
 // logits (per head), O = f_own * own + sum_k w_k * f_k * partial_k, f = the
 // reciprocal row sums of the unnormalised chunk outputs.  A slot's partials
-// of the whole group are one contiguous block [d/32][G][32] fp16 (G*d*2
-// bytes), read with 16-byte loads: lane l takes pieces p = l + 32 i, i.e.
-// columns 8*(p%4) .. +8 of chunk p/(4G) of head (p/4) % G -- head l/4 (+8 i for
-// G = 16).  Four slots' loads are in flight at a time.
+// of the whole group are one contiguous block of 16-byte pieces ordered
+// [d/8][G] (G*d*2 bytes; the own term has the same layout), read with
+// coalesced 16-byte loads: lane l takes pieces l + 32 i, all of head l % G
+// (G divides 32), columns 8 * ((l + 32 i) / G) .. +8.  Four slots' loads are
+// in flight at a time.
 template <int D, int G>
 __global__ void __launch_bounds__(256)
-fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
+fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restrict__ own,
             const float2 *__restrict__ zf, const float *__restrict__ own_f,
             const int32_t *__restrict__ idx, int64_t groups, int H, int Hkv, int topk,
             float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
     constexpr int NP = G * D / 256;                  // 16-byte pieces per lane and slot
-    constexpr int HPL = G / 8;                       // heads per lane
-    static_assert(NP >= 1 && (NP % HPL) == 0, "pieces must cover the heads evenly");
+    static_assert(NP >= 1 && 32 % G == 0, "a lane's pieces must all belong to one head");
     grid_dep_wait();                                 // the chunk outputs come from attend_tc_kernel
     const int lane = threadIdx.x & 31;
     const int64_t srow = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (srow >= groups) return;                      // srow = (b*L + t)*Hkv + g
     const int64_t bt = srow / Hkv;
     const int g = (int)(srow % Hkv);
+    const int h = lane % G;
+    const int64_t hrow = bt * H + (int64_t)g * G + h;
     const int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && idx[srow * topk + lane] >= 0));
-    // per-head fusion weights of this lane's heads (softmax over the valid slots)
-    float m[HPL], inv[HPL];
-#pragma unroll
-    for (int j = 0; j < HPL; ++j) {
-        const int h = (lane >> 2) + 8 * j;
-        const float2 *zh = zf + ((bt * H + (int64_t)g * G + h) * topk);
-        float mm = -INFINITY;
-        for (int k = 0; k < nsel; ++k) mm = fmaxf(mm, zh[k].x);
-        float den = 0.f;
-        for (int k = 0; k < nsel; ++k) den += __expf(zh[k].x - mm);
-        m[j] = mm;
-        inv[j] = nsel ? 1.f / den : 0.f;
-        if (w_out && (lane & 3) == 0)
-            for (int k = 0; k < topk; ++k)
-                w_out[(bt * H + (int64_t)g * G + h) * topk + k] =
-                    k < nsel ? __expf(zh[k].x - mm) * inv[j] : 0.f;
-    }
+    // fusion weights of this lane's head (softmax over the valid slots)
+    const float2 *zh = zf + hrow * topk;
+    float m = -INFINITY;
+    for (int k = 0; k < nsel; ++k) m = fmaxf(m, zh[k].x);
+    float den = 0.f;
+    for (int k = 0; k < nsel; ++k) den += __expf(zh[k].x - m);
+    const float inv = nsel ? 1.f / den : 0.f;
+    if (w_out && lane < G)
+        for (int k = 0; k < topk; ++k)
+            w_out[hrow * topk + k] = k < nsel ? __expf(zh[k].x - m) * inv : 0.f;
     // own term
     float acc[NP][8];
+    const uint4 *ob = reinterpret_cast<const uint4 *>(own + srow * (int64_t)(G * D));
+    const float fo = own_f[hrow];
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
-        const int pc = lane + 32 * i;
-        const int ch = pc / (4 * G), h = (pc >> 2) % G, q = pc & 3;
-        const int64_t hrow = bt * H + (int64_t)g * G + h;
-        const float fo = own_f[hrow];
-        const uint4 u = *reinterpret_cast<const uint4 *>(own + hrow * D + ch * 32 + q * 8);
-        const __half2 *h2 = reinterpret_cast<const __half2 *>(&u);
+        const uint4 u = ob[lane + 32 * i];
+        const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&u);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h2[e]);
+            const float2 f = unpack_bf16x2(w2[e]);
             acc[i][2 * e] = fo * f.x;
             acc[i][2 * e + 1] = fo * f.y;
         }
@@ -632,39 +673,32 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
     const uint4 *pb = reinterpret_cast<const uint4 *>(part + srow * topk * (int64_t)(G * D));
     for (int k0 = 0; k0 < nsel; k0 += 4) {
         uint4 raw[4][NP];
-        float wk[4][HPL];
+        float wk[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int k = k0 + u < nsel ? k0 + u : k0;
 #pragma unroll
             for (int i = 0; i < NP; ++i) raw[u][i] = pb[(int64_t)k * (G * D / 8) + lane + 32 * i];
-#pragma unroll
-            for (int j = 0; j < HPL; ++j) {
-                const int h = (lane >> 2) + 8 * j;
-                const float2 z = zf[(bt * H + (int64_t)g * G + h) * topk + k];
-                wk[u][j] = k0 + u < nsel ? __expf(z.x - m[j]) * inv[j] * z.y : 0.f;
-            }
+            const float2 z = zh[k];
+            wk[u] = k0 + u < nsel ? __expf(z.x - m) * inv * z.y : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int i = 0; i < NP; ++i) {
-                const float w = wk[u][i % HPL];
-                const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[u][i]);
+                const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&raw[u][i]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 f = __half22float2(h2[e]);
-                    acc[i][2 * e] = fmaf(w, f.x, acc[i][2 * e]);
-                    acc[i][2 * e + 1] = fmaf(w, f.y, acc[i][2 * e + 1]);
+                    const float2 f = unpack_bf16x2(w2[e]);
+                    acc[i][2 * e] = fmaf(wk[u], f.x, acc[i][2 * e]);
+                    acc[i][2 * e + 1] = fmaf(wk[u], f.y, acc[i][2 * e + 1]);
                 }
             }
     }
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
-        const int pc = lane + 32 * i;
-        const int ch = pc / (4 * G), h = (pc >> 2) % G, q = pc & 3;
-        const int64_t hrow = bt * H + (int64_t)g * G + h;
-        *reinterpret_cast<uint4 *>(O + hrow * D + ch * 32 + q * 8) =
+        const int c8 = (lane + 32 * i) / G;
+        *reinterpret_cast<uint4 *>(O + hrow * D + c8 * 8) =
             make_uint4(pack_bf16x2(acc[i][0], acc[i][1]), pack_bf16x2(acc[i][2], acc[i][3]),
                        pack_bf16x2(acc[i][4], acc[i][5]), pack_bf16x2(acc[i][6], acc[i][7]));
     }
@@ -727,7 +761,7 @@ struct TcLaunch {
     const int4 *tiles;                // one descriptor per queue position
     const int64_t *qlen;              // number of tiles (device)
     float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
-    __half *part, *own;
+    __nv_bfloat16 *part, *own;
     void *O;
     unsigned *status;
     int num_sms;
