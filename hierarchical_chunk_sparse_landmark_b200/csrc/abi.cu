@@ -24,7 +24,8 @@ cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf
                           void *O, int32_t *idx_out, cudaStream_t st);
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
 bool select_tc_supported();
-cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, void *split, int B,
+cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaStream_t st);
+cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
                              int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
                              int32_t *idx, unsigned *status, cudaStream_t st);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
@@ -157,7 +158,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         off = align_up(off + sizeof(__nv_bfloat16) * (size_t)B * L * H * topk * d, 256);
         p.own_off = off;
         off = align_up(off + sizeof(__nv_bfloat16) * (size_t)B * L * H * d, 256);
-        p.lmsplit_off = off;         // fp32 landmarks as two bf16 parts (tensor-core selection)
+        p.lmsplit_off = off;         // fp32 landmarks as two bf16 planes (tensor-core path)
         off = align_up(off + 2 * sizeof(__nv_bfloat16) * (size_t)B * Hkv * Nc * d, 256);
     }
     p.total = off;
@@ -308,16 +309,24 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
     // The tensor-core path computes the fusion logits inside its S tiles and
     // the weights in fuse_kernel, so the selection skips them there.
     cudaError_t e;
+    // fp32 landmarks on the tensor-core path: split once into bf16 high / low
+    // planes, which the selection and the attention tiles both read
+    void *lm_split = ws + lay.lmsplit_off;
+    if (use_tc && !lm_bf16 && L >= S) {
+        e = launch_split_landmarks(lm_use, lm_split, (int64_t)B * Hkv * (L / S) * d, st);
+        if (e != cudaSuccess) return HSA_ERR_CUDA;
+        t_launches += 1;
+    }
     const bool tc_select = use_tc && L >= S && (H / Hkv) % 8 == 0 && select_tc_supported() &&
                            !force_simt_select();
     if (tc_select)
-        e = launch_select_tc(Q, lm_use, lm_bf16, ws + lay.lmsplit_off, B, H, Hkv, L, d, S, topk,
-                             scale, idx, (unsigned *)ws, st);
+        e = launch_select_tc(Q, lm_use, lm_bf16, lm_split, B, H, Hkv, L, d, S, topk, scale, idx,
+                             (unsigned *)ws, st);
     else
         e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
                           use_tc ? nullptr : w, st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
-    t_launches += (tc_select && !lm_bf16) ? 2 : 1;     // fp32 landmarks: split + select
+    t_launches += 1;
     stage_mark(2, st);
     if (use_tc) {
         const int64_t Nc = L / S;
@@ -332,7 +341,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         t_launches += 5;
         stage_mark(3, st);
         TcLaunch a;
-        a.Q = Q; a.K = K; a.V = V; a.lm = lm_use; a.lm_bf16 = lm_bf16 ? 1 : 0;
+        a.Q = Q; a.K = K; a.V = V; a.lm = lm_bf16 ? lm_use : lm_split; a.lm_bf16 = lm_bf16 ? 1 : 0;
         a.B = B; a.H = H; a.Hkv = Hkv; a.S = S; a.topk = topk; a.own_chunk = own_chunk;
         a.L = L; a.W = lay.W; a.cap = lay.cap; a.scale = scale;
         a.idx = idx; a.entries = (const int32_t *)(ws + lay.entries_off);

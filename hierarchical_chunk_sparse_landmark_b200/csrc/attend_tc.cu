@@ -32,8 +32,8 @@
 //                           ring, landmark rows into the K slot, TMA of the
 //                           Q rows -- one box per entry, its G query-head rows
 //                           -- and of the chunk's K and V)
-//   warp 1       MMA issuer (S of the next tile or P.V of the oldest pending
-//                           one, whichever is ready)
+//   warp 1       MMA issuer for S
+//   warp 14      MMA issuer for P.V
 //   warps 2-5    softmax   (thread = tile row = TMEM lane)
 //   warps 6-13   epilogue  (two groups taking alternate tiles; TMEM -> bf16
 //                           partial slots / own-chunk term)
@@ -80,14 +80,14 @@ struct TcParams {
     const int4 *tiles;            // [qlen] tile descriptors in queue order
     const int64_t *qlen;
     const int32_t *entries;
-    const void *lm;               // [B, Hkv, Nc, D] bf16 or fp32
     float *zf;                    // [B, L, H, topk] x (fusion logit, 1 / chunk row sum)
     float *own_f;                 // [B, L, H] add_own / own-chunk row sum
     __nv_bfloat16 *part;          // [B*L*Hkv*topk entries][D/8][G][8] chunk outputs
     __nv_bfloat16 *own;           // [B*L*Hkv rows (t, g)][D/8][G][8] own-chunk term
     unsigned *status;
     int64_t L, Nc;
-    int H, Hkv, topk, S, add_own, lm_bf16;
+    int H, Hkv, topk, S, add_own;
+    int lm_rows;                  // landmark rows per chunk: 1 (bf16) or 2 (bf16 high, low of fp32)
     int q3d;                      // Q map is the 3-D (cols, rows, d-half) view
     float scale, scale_log2e;
 };
@@ -95,7 +95,8 @@ struct TcParams {
 constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
 constexpr int kThreads = 512;                       // 16 warps
 constexpr int kEpiWarp0 = 6;                        // epilogue groups: warps 6-9 and 10-13
-constexpr int kEpiEnd = 14;                         // epilogue warps end here; warp 14 has no role
+constexpr int kEpiEnd = 14;                         // epilogue warps end here
+constexpr int kPvWarp = 14;                         // issues the P.V products
 constexpr int kProducer2 = 15;                      // second producer (odd tiles)
 constexpr int kOwnTileFlag = 1 << 30;               // in a descriptor's .w (bucket.cu)
 
@@ -155,6 +156,21 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
     return true;
 }
+// Warp-level forms: every lane waits (a wait by one lane and a broadcast was
+// slower) and the warp votes on the outcome, so a break on abort is
+// warp-uniform; one arrive stands for all 32 lanes, each of which fenced its
+// own prior tcgen05 work before the warp sync.
+// Barriers that warps release count warps, not threads: a per-thread arrive
+// is one shared-memory atomic each, and 640 of them per tile queued up
+// behind every other barrier operation of the block.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, abort)) != 0;
+}
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) tc::mbar_arrive(bar);
+}
+
 // Parity to wait on before the u-th reuse of a ring slot (u >= 1): the
 // consumer's release of use u-1.
 __device__ __forceinline__ uint32_t reuse_parity(int64_t u) { return (uint32_t)((u + 1) & 1); }
@@ -186,16 +202,6 @@ struct TileInfo {
     int32_t code[16];
 };
 
-// The producer's prefetch ring: descriptor, entry codes and raw landmark row
-// (up to d fp32 values) of the next tiles.
-constexpr int kMeta = 8;
-template <int D>
-struct alignas(16) TileMetaT {
-    int4 desc;
-    int32_t code[16];
-    uint8_t lrow[D * 4];
-};
-
 // Per-row view of a tile for the softmax and epilogue threads.
 struct RowJob {
     Tile tl;
@@ -219,7 +225,8 @@ __device__ __forceinline__ RowJob read_row(const TileInfo &ti, int e) {
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const TcParams p) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmL,
+                 const TcParams p) {
     using C = TcCfg<D, G>;
     grid_dep_wait();                      // the work lists are written by the previous kernels
     extern __shared__ uint8_t smem_raw[];
@@ -238,10 +245,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     static_assert((24 + 2 * kRing) * 8 + 8 <= C::BAR_BYTES, "barrier block overflows its reserve");
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
     __shared__ TileInfo ring[kRing];
-    using TileMeta = TileMetaT<D>;
-    __shared__ TileMeta meta[kMeta];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // key rows 64..79 of every K block: the landmark rows land in 64 (and 65)
+    // by TMA; the rest stay zero (row 65 too when landmarks are bf16)
+    for (int i = tid; i < C::NQK * C::KB * 16 * 8; i += kThreads) {
+        const int q = i / (C::KB * 128), kb = (i / 128) % C::KB, o = i % 128;
+        reinterpret_cast<uint4 *>(sK(q) + kb * C::KBLK + 64 * 128)[o] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    tc::fence_proxy_async_smem();
     if (warp == 1) {
         tc::tmem_alloc(s_tmem, C::TMEM_COLS);
         tc::tmem_relinquish();
@@ -257,15 +269,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&sfull[s], 1);
-            tc::mbar_init(&sfree[s], 128);
-            tc::mbar_init(&pfull[s], 128);
+            tc::mbar_init(&sfree[s], 4);       // one arrive per softmax warp
+            tc::mbar_init(&pfull[s], 4);
             tc::mbar_init(&ofull[s], 1);
-            tc::mbar_init(&ofree[s], 128);
+            tc::mbar_init(&ofree[s], 4);       // one arrive per epilogue warp
             tc::mbar_init(&pempty[s], 1);      // P.V done: TMEM P slot free
         }
         for (int i = 0; i < kRing; ++i) {
             tc::mbar_init(&ifull[i], 1);
-            tc::mbar_init(&ifree[i], 256);     // softmax + one epilogue group
+            tc::mbar_init(&ifree[i], 8);       // softmax warps + one epilogue group's warps
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -281,50 +293,28 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     if (warp == 0 || warp == kProducer2) {
         // ------------------------------------------------------------ producers
-        // Tile metadata and landmark rows; producer pid takes the tiles
-        // j = 2u + pid.  Its descriptors are fetched two of its tiles ahead and
-        // entry codes / landmark rows one tile ahead with cp.async into its
-        // half of a shared ring, so it never waits on a fresh global load.
-        // Virtual iterations u = -2, -1 only fill the ring; every iteration
-        // commits exactly two copy groups, so "at most 2 pending" means: this
-        // tile's rows and the descriptor of the next one have landed.
+        // Producer pid takes the tiles j = 2u + pid.  The descriptor of tile
+        // u + 2 and the entry codes of tile u + 1 are loaded into registers one
+        // iteration ahead, so their latency hides behind the current tile.
         const int pid = warp == 0 ? 0 : 1;
         const int64_t my_u = (my_tiles - pid + 1) / 2;
-        auto slot_of = [&](int64_t u) -> TileMeta & { return meta[pid * (kMeta / 2) + (u & (kMeta / 2 - 1))]; };
-        auto issue_desc = [&](int64_t u) {
-            if (lane == 0 && u >= 0 && u < my_u)
-                tc::cp_async16(&slot_of(u).desc, p.tiles + blockIdx.x + (2 * u + pid) * gridDim.x);
-            tc::cp_async_commit();
+        auto load_desc = [&](int64_t u) -> int4 {
+            return u < my_u ? __ldg(p.tiles + blockIdx.x + (2 * u + pid) * gridDim.x) : make_int4(0, 0, 0, 0);
         };
-        auto issue_rows = [&](int64_t u) {
-            if (u >= 0 && u < my_u) {
-                TileMeta &mt = slot_of(u);
-                Tile tl;
-                decode_tile(p, mt.desc, tl);
-                if (!tl.own) {
-                    if (lane < tl.n) tc::cp_async4(&mt.code[lane], p.entries + tl.first + lane);
-                    constexpr int LB = D * 4 / 16;                 // 16-byte pieces of an fp32 row
-                    const int pieces = p.lm_bf16 ? LB / 2 : LB;
-                    const uint8_t *src = (const uint8_t *)p.lm +
-                        (size_t)(tl.bg * p.Nc + tl.chunk) * D * (p.lm_bf16 ? 2 : 4);
-                    if (lane < pieces) tc::cp_async16(mt.lrow + lane * 16, src + lane * 16);
-                }
-            }
-            tc::cp_async_commit();
+        auto load_code = [&](const int4 &d) -> int32_t {
+            Tile tl;
+            decode_tile(p, d, tl);
+            return (!tl.own && lane < tl.n) ? __ldg(p.entries + tl.first + lane) : 0;
         };
-        for (int64_t u = -2; u < my_u; ++u) {
-            issue_desc(u + 2);
-            tc::cp_async_wait<2>();
-            __syncwarp();
-            issue_rows(u + 1);
-            if (u < 0) continue;
-            tc::cp_async_wait<2>();
-            __syncwarp();
+        int4 d_cur = load_desc(0), d_nxt = load_desc(1);
+        int32_t code_cur = load_code(d_cur);
+        for (int64_t u = 0; u < my_u; ++u) {
+            const int4 d_n2 = load_desc(u + 2);
+            const int32_t code_nxt = load_code(d_nxt);
             const int64_t j = 2 * u + pid;
-            TileMeta &mt = slot_of(u);
             Tile d0;
-            decode_tile(p, mt.desc, d0);
-            const int32_t c0 = lane < d0.n ? (d0.own ? (int32_t)((d0.t0 + lane) * 32) : mt.code[lane]) : 0;
+            decode_tile(p, d_cur, d0);
+            const int32_t c0 = lane < d0.n ? (d0.own ? (int32_t)((d0.t0 + lane) * 32) : code_cur) : 0;
             const int bq = (int)d0.bg / Hkv;            // bg < 2^31 (checked on the host)
             const int gq = (int)d0.bg - bq * Hkv;
 
@@ -342,44 +332,30 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ifull[ri]);
 
-            // landmark row of the chunk -> key rows 64 (bf16 high part), 65 (low part)
+            // Q/K slot j % 3, free once the S of tile j - 3 is done: the chunk's
+            // K rows, its landmark (bf16 high / low parts as key rows 64, 65)
+            // and one Q box per entry (all G query-head rows, both halves of d
+            // when the 3-D view is available), all on one transaction count
             const int q = (int)(j % C::NQK);
             if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (!d0.own && lane < D / 8) {
-                float x0[8];
-                if (p.lm_bf16) {
-                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(mt.lrow + lane * 16), x0);
-                } else {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(mt.lrow + lane * 32);
-                    Vec16<float>::unpack(src[0], x0);
-                    Vec16<float>::unpack(src[1], x0 + 4);
-                }
-                float hi[8], lo[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    hi[e] = __bfloat162float(__float2bfloat16_rn(x0[e]));
-                    lo[e] = x0[e] - hi[e];
-                }
-                const int kb = (lane * 8) / 64, c = ((lane * 8) % 64) / 8;
-                uint8_t *blk = sK(q) + kb * C::KBLK;
-                *reinterpret_cast<uint4 *>(blk + tc::sw128_offset(64, c)) =
-                    make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
-                               pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
-                *reinterpret_cast<uint4 *>(blk + tc::sw128_offset(65, c)) =
-                    make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
-                               pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
-                tc::fence_proxy_async_smem();
-            }
-            __syncwarp();
-            // Q rows (one TMA box per entry: all G query-head rows, both halves of d
-            // when the 3-D view is available) and the chunk's K
             const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
             if (lane == 0) {
-                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(d0.n * G * D * 2 + C::K_TMA_BYTES));
+                const uint32_t lbytes = d0.own ? 0u : (uint32_t)(C::KB * 128 * p.lm_rows);
+                tc::mbar_expect_tx(&qk_full[q], (uint32_t)(d0.n * G * D * 2 + C::K_TMA_BYTES) + lbytes);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
                     tc::tma_load_2d(sK(q) + kb * C::KBLK, &tmK, &qk_full[q], kb * 64, krow);
+                if (!d0.own) {
+                    const int lrow = (int)(d0.bg * p.Nc + d0.chunk);
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb) {
+                        if (p.lm_rows == 2)
+                            tc::tma_load_3d(sK(q) + kb * C::KBLK + 64 * 128, &tmL, &qk_full[q], kb * 64, lrow, 0);
+                        else
+                            tc::tma_load_2d(sK(q) + kb * C::KBLK + 64 * 128, &tmL, &qk_full[q], kb * 64, lrow);
+                    }
+                }
             }
             __syncwarp();
             if (lane < d0.n) {
@@ -407,10 +383,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            d_cur = d_nxt; d_nxt = d_n2; code_cur = code_nxt;
         }
-        tc::cp_async_wait<0>();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == kPvWarp) {
+        // ------------------------------------------------------------ MMA issuers
+        // Two threads issue tcgen05.mma: warp 1 the S products, warp 14 the
+        // P.V products, each waiting only on its own inputs, so one stream's
+        // barrier checks (each an mbarrier round trip of ~100+ cycles) never
+        // delay the other.  The streams touch disjoint TMEM columns (S at
+        // s*128 .. +80, P at s*128 + 80 .. +112, O at 256 + s*D) and commit to
+        // their own barriers; a commit tracks only its own thread's MMAs.
         if (lane == 0) {
             constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, C::NS, false);
             constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
@@ -444,30 +426,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tc::mma_commit(&sfull[s]);
                 tc::mma_commit(&qk_empty[q]);
             };
-            // S of tile j: its Q/K slot loaded and S slot j%2 read by the softmax
-            // of tile j-2.  P.V of tile i: P written, V loaded, O slot i%2 read
-            // by the epilogue of tile i-2.
-            auto ready_s = [&](int64_t j) -> bool {
-                return tc::mbar_try_wait(&qk_full[j % C::NQK], (uint32_t)((j / C::NQK) & 1)) &&
-                       (j < 2 || tc::mbar_try_wait(&sfree[j & 1], reuse_parity(j >> 1)));
-            };
-            auto ready_pv = [&](int64_t i) -> bool {
-                return tc::mbar_try_wait(&pfull[i & 1], (uint32_t)((i >> 1) & 1)) &&
-                       tc::mbar_try_wait(&v_full[i % C::NVP], (uint32_t)((i / C::NVP) & 1)) &&
-                       (i < 2 || tc::mbar_try_wait(&ofree[i & 1], reuse_parity(i >> 1)));
-            };
-            int64_t ns = 0, npv = 0;
-            long long t0 = clock64();
-            while (npv < my_tiles) {
-                if (ns < my_tiles && ns - npv < 2 && ready_s(ns)) {
-                    issue_s(ns++);
-                    t0 = clock64();
-                } else if (npv < ns && ready_pv(npv)) {
-                    issue_pv(npv++);
-                    t0 = clock64();
-                } else if (*s_abort || clock64() - t0 > kWaitBudget) {
-                    *s_abort = 1;
-                    break;
+            if (warp == 1) {
+                // S of tile j: its Q/K slot loaded, S slot j%2 read by the
+                // softmax of tile j-2
+                for (int64_t j = 0; j < my_tiles; ++j) {
+                    if (!wait_bar(&qk_full[j % C::NQK], (uint32_t)((j / C::NQK) & 1), s_abort)) break;
+                    if (j >= 2 && !wait_bar(&sfree[j & 1], reuse_parity(j >> 1), s_abort)) break;
+                    issue_s(j);
+                }
+            } else {
+                // P.V of tile i: P written, V loaded, O slot i%2 read by the
+                // epilogue of tile i-2
+                for (int64_t i = 0; i < my_tiles; ++i) {
+                    if (!wait_bar(&pfull[i & 1], (uint32_t)((i >> 1) & 1), s_abort)) break;
+                    if (!wait_bar(&v_full[i % C::NVP], (uint32_t)((i / C::NVP) & 1), s_abort)) break;
+                    if (i >= 2 && !wait_bar(&ofree[i & 1], reuse_parity(i >> 1), s_abort)) break;
+                    issue_pv(i);
                 }
             }
         }
@@ -479,13 +453,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int e = r / G, h = r % G;
         for (int64_t j = 0; j < my_tiles; ++j) {
             const int ri = (int)(j & (kRing - 1));
-            if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
+            if (!warp_wait(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
             const RowJob cur = read_row(ring[ri], e);
-            tc::mbar_arrive(&ifree[ri]);
+            warp_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
             const int64_t b = cur.b;
             const int g = cur.g;
-            if (!wait_bar(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
+            if (!warp_wait(&sfull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
             float s0[32], s1[32], l_hi, l_lo;
             const uint32_t ta = tmem + s * C::S_COL + lane_off;
@@ -494,7 +468,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::tmem_ld2(ta + 64, l_hi, l_lo);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
-            tc::mbar_arrive(&sfree[s]);
+            warp_arrive(&sfree[s]);
             // own-chunk rows see keys c*S .. t only: mask the rest to -inf
             if (cur.tl.own) {
                 const int nk = cur.valid ? (int)(cur.t - (int64_t)cur.tl.chunk * S) + 1 : 64;
@@ -551,11 +525,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 pk[c] = pack_bf16x2_int(s0[2 * c], s0[2 * c + 1]);
                 pk[16 + c] = pack_bf16x2_int(s1[2 * c], s1[2 * c + 1]);
             }
-            if (j >= 2 && !wait_bar(&pempty[s], reuse_parity(j >> 1), s_abort)) break;
+            if (j >= 2 && !warp_wait(&pempty[s], reuse_parity(j >> 1), s_abort)) break;
             tc::tmem_st32(tmem + s * C::S_COL + C::P_OFF + lane_off, pk);
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            tc::mbar_arrive(&pfull[s]);
+            warp_arrive(&pfull[s]);
         }
     } else if (warp < kEpiEnd) {
         // ------------------------------------------------------------ epilogue
@@ -569,9 +543,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         constexpr int NCH = D / 32;               // 32-column chunks of a row
         for (int64_t j = eg; j < my_tiles; j += 2) {
             const int ri = (int)(j & (kRing - 1));
-            if (!wait_bar(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
+            if (!warp_wait(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
             const RowJob cur = read_row(ring[ri], e);
-            tc::mbar_arrive(&ifree[ri]);
+            warp_arrive(&ifree[ri]);
             const int s = (int)(j & 1);
             const int64_t b = cur.b;
             const int g = cur.g;
@@ -581,7 +555,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const int64_t row = (b * L + cur.t) * Hkv + g;
             uint4 *blk = reinterpret_cast<uint4 *>(cur.tl.own ? p.own + row * (G * D)
                                                               : p.part + (row * topk + cur.k) * (G * D));
-            if (!wait_bar(&ofull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
+            if (!warp_wait(&ofull[s], (uint32_t)((j >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
 #pragma unroll 1
             for (int ch = 0; ch < NCH; ch += 2) {
@@ -603,7 +577,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
             }
             tc::fence_before_sync();
-            tc::mbar_arrive(&ofree[s]);
+            warp_arrive(&ofree[s]);
         }
     }
 
@@ -736,6 +710,21 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
            CUDA_SUCCESS;
 }
 
+// 3-D bf16 view of two planes [2][rows, D]: one box (64, 1, 2) brings a row's
+// 64-column block from both planes as two consecutive 128B-swizzled rows.
+static bool make_map_planes(CUtensorMap *m, const void *base, uint64_t rows, int D) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, 2u};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+    const cuuint32_t box[3] = {64u, 1u, 2u};
+    const cuuint32_t es[3] = {1u, 1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // 3-D bf16 view of [rows, D] (D = 128) as (64 columns, rows, 2 halves of d),
 // strides 2*D and 128 bytes: one box (64, G, 2) brings all of an entry's G
 // rows, both halves, as two 128B-swizzled [G x 128 B] blocks.
@@ -753,7 +742,10 @@ static bool make_map_q3d(CUtensorMap *m, const void *base, uint64_t rows, int D,
 }
 
 struct TcLaunch {
-    const void *Q, *K, *V, *lm;
+    const void *Q, *K, *V;
+    // landmarks as bf16 rows: [B*Hkv*Nc, D] (lm_bf16) or the two planes
+    // [2][B*Hkv*Nc, D] of an fp32 landmark's bf16 high and low parts
+    const void *lm;
     int B, H, Hkv, S, topk, own_chunk, lm_bf16;
     int64_t L, W, cap;
     float scale;
@@ -770,7 +762,7 @@ struct TcLaunch {
 template <int D, int G>
 static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEvent_t mid) {
     using C = TcCfg<D, G>;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, ml;
     // the single-box entry layout has a uniform 8-row atom stride only when an
     // entry is exactly one atom (G = 8) and d has two halves
     bool q3d = (G == 8 && D == 128) &&
@@ -779,20 +771,24 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     if (!make_map(&mk, a.K, (uint64_t)a.B * a.Hkv * a.L, D, 64) ||
         !make_map(&mv, a.V, (uint64_t)a.B * a.Hkv * a.L, D, 64))
         return cudaErrorInvalidValue;
+    const uint64_t lrows = (uint64_t)a.B * a.Hkv * (a.L / a.S);
+    if (lrows == 0) ml = mk;                       // no chunk tiles: the map is never used
+    else if (!(a.lm_bf16 ? make_map(&ml, a.lm, lrows, D, 1) : make_map_planes(&ml, a.lm, lrows, D)))
+        return cudaErrorInvalidValue;
     auto kern = attend_tc_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     TcParams p;
     p.tiles = a.tiles; p.qlen = a.qlen;
-    p.entries = a.entries; p.lm = a.lm; p.zf = a.zf; p.own_f = a.own_f;
+    p.entries = a.entries; p.zf = a.zf; p.own_f = a.own_f;
     p.part = a.part; p.own = a.own; p.status = a.status;
     p.L = a.L; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
-    p.lm_bf16 = a.lm_bf16;
+    p.lm_rows = a.lm_bf16 ? 1 : 2;
     p.q3d = q3d ? 1 : 0;
     p.scale = a.scale;
     p.scale_log2e = a.scale * 1.4426950408889634f;
-    e = launch_pdl(kern, dim3((unsigned)a.num_sms), dim3(kThreads), (size_t)C::SMEM, st, mq, mk, mv, p);
+    e = launch_pdl(kern, dim3((unsigned)a.num_sms), dim3(kThreads), (size_t)C::SMEM, st, mq, mk, mv, ml, p);
     if (e != cudaSuccess) return e;
     // with a timing event between the two kernels the fusion kernel is launched
     // plainly (an event between them ends the programmatic overlap anyway)

@@ -384,25 +384,30 @@ static cudaError_t launch_select_tc_k(const SelTcParams &p, int B, const void *l
 
 bool select_tc_supported() { return sel_encode_fn() != nullptr; }
 
-// Q bf16; landmarks bf16 (lm_bf16) or fp32 (split into `split` = 2 bf16 arrays
-// of B*Hkv*Nc*d elements first).  Nc = L / S >= 1; G = H / Hkv a multiple of 8.
-cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, void *split, int B,
+// fp32 landmarks [n] -> two bf16 planes: split = [hi (n) | lo (n)].
+cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaStream_t st) {
+    __nv_bfloat16 *l0 = (__nv_bfloat16 *)split, *l1 = l0 + n;
+    const int64_t n4 = n / 4;
+    const unsigned blocks = (unsigned)((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
+    return launch_pdl(split_landmarks_kernel, dim3(blocks), dim3(256), 0, st,
+                      (const float4 *)lm, (uint2 *)l0, (uint2 *)l1, n4);
+}
+
+// Q bf16; landmarks bf16 (lm_bf16), else the two bf16 planes `split` of fp32
+// landmarks (launch_split_landmarks, B*Hkv*Nc*d elements each).  Nc = L / S
+// >= 1; G = H / Hkv a multiple of 8.
+cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
                              int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
                              int32_t *idx, unsigned *status, cudaStream_t st) {
     SelTcParams p;
     p.Q = Q; p.idx = idx; p.status = status;
     p.L = L; p.Nc = L / S; p.H = H; p.Hkv = Hkv; p.S = S; p.topk = topk; p.scale = scale;
-    const int64_t n = (int64_t)B * Hkv * p.Nc * d;
     if (lm_bf16) {
         return d == 128 ? launch_select_tc_k<128, false>(p, B, lm, nullptr, st)
                         : launch_select_tc_k<64, false>(p, B, lm, nullptr, st);
     }
-    __nv_bfloat16 *l0 = (__nv_bfloat16 *)split, *l1 = l0 + n;
-    const int64_t n4 = n / 4;
-    const unsigned blocks = (unsigned)((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
-    cudaError_t e = launch_pdl(split_landmarks_kernel, dim3(blocks), dim3(256), 0, st,
-                               (const float4 *)lm, (uint2 *)l0, (uint2 *)l1, n4);
-    if (e != cudaSuccess) return e;
+    const int64_t n = (int64_t)B * Hkv * p.Nc * d;
+    const __nv_bfloat16 *l0 = (const __nv_bfloat16 *)split, *l1 = l0 + n;
     return d == 128 ? launch_select_tc_k<128, true>(p, B, l0, l1, st)
                     : launch_select_tc_k<64, true>(p, B, l0, l1, st);
 }
