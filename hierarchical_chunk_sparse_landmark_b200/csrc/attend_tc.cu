@@ -599,16 +599,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // of the whole group are one contiguous block of 16-byte pieces ordered
 // [d/8][G] (G*d*2 bytes; the own term has the same layout), read with
 // coalesced 16-byte loads: lane l takes pieces l + 32 i, all of head l % G
-// (G divides 32), columns 8 * ((l + 32 i) / G) .. +8.  Four slots' loads are
-// in flight at a time.
-template <int D, int G>
-__global__ void __launch_bounds__(256)
+// (G divides 32), columns 8 * ((l + 32 i) / G) .. +8.  The own term's and
+// the first slots' loads go out before the selection count is known.
+// Two blocks per SM where a lane's pieces allow (G*d <= 1024), else one: the
+// loads in flight per warp, not the warp count, keep HBM busy.
+template <int D, int G, int KP>
+__global__ void __launch_bounds__(256, (G * D / 256) <= 4 ? 2 : 1)
 fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restrict__ own,
             const float2 *__restrict__ zf, const float *__restrict__ own_f,
             const int32_t *__restrict__ idx, int64_t groups, int H, int Hkv, int topk,
             float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
     constexpr int NP = G * D / 256;                  // 16-byte pieces per lane and slot
+    constexpr int SLOT = G * D / 8;                  // 16-byte pieces per slot
     static_assert(NP >= 1 && 32 % G == 0, "a lane's pieces must all belong to one head");
+    constexpr int SG = NP <= 4 ? 4 : 2;              // slots whose loads are in flight together
+    static_assert(KP % SG == 0 && KP <= 32, "slots are taken SG at a time");
     grid_dep_wait();                                 // the chunk outputs come from attend_tc_kernel
     const int lane = threadIdx.x & 31;
     const int64_t srow = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
@@ -617,25 +622,39 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
     const int g = (int)(srow % Hkv);
     const int h = lane % G;
     const int64_t hrow = bt * H + (int64_t)g * G + h;
+    const uint4 *pb = reinterpret_cast<const uint4 *>(part + srow * topk * (int64_t)(G * D));
+    const uint4 *ob = reinterpret_cast<const uint4 *>(own + srow * (int64_t)(G * D));
+    // The loads that do not depend on the selection go out first: the own term
+    // and the first SG slots (a slot past the valid ones is zeroed below).
+    uint4 rown[NP], raw[SG][NP];
+#pragma unroll
+    for (int i = 0; i < NP; ++i) rown[i] = ob[lane + 32 * i];
+#pragma unroll
+    for (int u = 0; u < SG; ++u)
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+            raw[u][i] = u < topk ? pb[(int64_t)u * SLOT + lane + 32 * i] : make_uint4(0u, 0u, 0u, 0u);
     const int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && idx[srow * topk + lane] >= 0));
-    // fusion weights of this lane's head (softmax over the valid slots)
+    // fusion weights of this lane's head: softmax of the logits over the valid slots
     const float2 *zh = zf + hrow * topk;
+    float zx[KP];
+#pragma unroll
+    for (int k = 0; k < KP; ++k) zx[k] = k < nsel ? zh[k].x : -INFINITY;
     float m = -INFINITY;
-    for (int k = 0; k < nsel; ++k) m = fmaxf(m, zh[k].x);
+#pragma unroll
+    for (int k = 0; k < KP; ++k) m = fmaxf(m, zx[k]);
     float den = 0.f;
-    for (int k = 0; k < nsel; ++k) den += __expf(zh[k].x - m);
+#pragma unroll
+    for (int k = 0; k < KP; ++k) den += k < nsel ? __expf(zx[k] - m) : 0.f;
     const float inv = nsel ? 1.f / den : 0.f;
     if (w_out && lane < G)
         for (int k = 0; k < topk; ++k)
             w_out[hrow * topk + k] = k < nsel ? __expf(zh[k].x - m) * inv : 0.f;
-    // own term
     float acc[NP][8];
-    const uint4 *ob = reinterpret_cast<const uint4 *>(own + srow * (int64_t)(G * D));
     const float fo = own_f[hrow];
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
-        const uint4 u = ob[lane + 32 * i];
-        const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&u);
+        const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&rown[i]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = unpack_bf16x2(w2[e]);
@@ -643,31 +662,33 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
             acc[i][2 * e + 1] = fo * f.y;
         }
     }
-    // retrieved slots, four at a time
-    const uint4 *pb = reinterpret_cast<const uint4 *>(part + srow * topk * (int64_t)(G * D));
-    for (int k0 = 0; k0 < nsel; k0 += 4) {
-        uint4 raw[4][NP];
-        float wk[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u < nsel ? k0 + u : k0;
+    for (int k0 = 0; k0 < KP; k0 += SG) {
+        if (k0 >= nsel) break;
+        if (k0 > 0) {
 #pragma unroll
-            for (int i = 0; i < NP; ++i) raw[u][i] = pb[(int64_t)k * (G * D / 8) + lane + 32 * i];
-            const float2 z = zh[k];
-            wk[u] = k0 + u < nsel ? __expf(z.x - m) * inv * z.y : 0.f;
+            for (int u = 0; u < SG; ++u)
+#pragma unroll
+                for (int i = 0; i < NP; ++i)
+                    raw[u][i] = k0 + u < nsel ? pb[(int64_t)(k0 + u) * SLOT + lane + 32 * i]
+                                              : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < SG; ++u) {
+            const bool valid = k0 + u < nsel;
+            const float wk = valid ? __expf(zx[k0 + u] - m) * inv * zh[k0 + u].y : 0.f;
 #pragma unroll
             for (int i = 0; i < NP; ++i) {
-                const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&raw[u][i]);
+                const uint4 rv = valid ? raw[u][i] : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&rv);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 f = unpack_bf16x2(w2[e]);
-                    acc[i][2 * e] = fmaf(wk[u], f.x, acc[i][2 * e]);
-                    acc[i][2 * e + 1] = fmaf(wk[u], f.y, acc[i][2 * e + 1]);
+                    acc[i][2 * e] = fmaf(wk, f.x, acc[i][2 * e]);
+                    acc[i][2 * e + 1] = fmaf(wk, f.y, acc[i][2 * e + 1]);
                 }
             }
+        }
     }
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
@@ -796,7 +817,8 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     const int64_t groups = (int64_t)a.B * a.L * a.Hkv;
     constexpr int kWarps = 8;
     const dim3 fgrid((unsigned)((groups + kWarps - 1) / kWarps));
-    return launch_pdl(fuse_kernel<D, G>, fgrid, dim3(32 * kWarps), 0, st, a.part, a.own,
+    auto fk = a.topk <= 8 ? fuse_kernel<D, G, 8> : a.topk <= 16 ? fuse_kernel<D, G, 16> : fuse_kernel<D, G, 32>;
+    return launch_pdl(fk, fgrid, dim3(32 * kWarps), 0, st, a.part, a.own,
                       (const float2 *)a.zf, (const float *)a.own_f, (const int32_t *)a.idx, groups,
                       a.H, a.Hkv, a.topk, a.w_out, (__nv_bfloat16 *)a.O);
 }
