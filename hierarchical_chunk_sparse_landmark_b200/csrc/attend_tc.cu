@@ -26,17 +26,17 @@
 //
 // attend_tc_kernel: one persistent block per SM walks the tile queue (a flat
 // list of tile descriptors) with these roles, linked by mbarriers, a ring of
-// three Q/K shared-memory slots, a ring of two V slots and double-buffered
-// TMEM accumulators (S, P and O):
-//   warps 0, 15  producers (even / odd tiles: tile metadata into a shared
-//                           ring, landmark rows into the K slot, TMA of the
-//                           Q rows -- one box per entry, its G query-head rows
-//                           -- and of the chunk's K and V)
+// three Q/K shared-memory slots, a ring of three V slots and double-buffered
+// TMEM accumulators (S, P and O); each role reads the descriptors (and its
+// row's entry code) itself, one to two tiles ahead, into registers:
+//   warps 0, 15  producers (even / odd tiles: TMA of the chunk's K, its
+//                           landmark rows into key rows 64/65, the Q rows --
+//                           one box per entry, its G query-head rows -- and V)
 //   warp 1       MMA issuer for S
 //   warp 14      MMA issuer for P.V
-//   warps 2-5    softmax   (thread = tile row = TMEM lane)
-//   warps 6-13   epilogue  (two groups taking alternate tiles; TMEM -> bf16
-//                           partial slots / own-chunk term)
+//   warps 2-9    softmax   (two groups taking alternate tiles; thread = tile
+//                           row = TMEM lane)
+//   warps 10-13  epilogue  (TMEM -> bf16 partial slots / own-chunk term)
 // Tiles are independent, so no block waits on another.  Every wait is
 // bounded; on expiry the block sets the status flag in the workspace, lets
 // in-flight copies land, frees its TMEM and exits.
@@ -94,7 +94,7 @@ struct TcParams {
 
 constexpr long long kWaitBudget = 4000000000LL;    // SM cycles (about 2 s)
 constexpr int kThreads = 512;                       // 16 warps
-constexpr int kEpiWarp0 = 6;                        // epilogue groups: warps 6-9 and 10-13
+constexpr int kEpiWarp0 = 10;                       // softmax groups: warps 2-5, 6-9; epilogue 10-13
 constexpr int kEpiEnd = 14;                         // epilogue warps end here
 constexpr int kPvWarp = 14;                         // issues the P.V products
 constexpr int kProducer2 = 15;                      // second producer (odd tiles)
@@ -192,16 +192,6 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Ti
     }
 }
 
-// Tile metadata the producer publishes to the softmax and epilogue roles
-// through a small shared-memory ring (so only the producer walks the global
-// work lists).  code[e] = t * 32 + k of entry e (own tiles: t * 32).
-constexpr int kRing = 4;
-struct TileInfo {
-    int64_t bg;
-    int chunk, n, own, b, g, pad;  // bg = b * Hkv + g, split once by the producer
-    int32_t code[16];
-};
-
 // Per-row view of a tile for the softmax and epilogue threads.
 struct RowJob {
     Tile tl;
@@ -210,15 +200,42 @@ struct RowJob {
     bool valid;
 };
 
-__device__ __forceinline__ RowJob read_row(const TileInfo &ti, int e) {
+// Every role walks its own tiles j0, j0 + step, ... and reads their metadata
+// itself: the descriptor two of its tiles ahead and this thread's entry code
+// (row e) one tile ahead go into registers, so no role waits on a fresh load
+// or on another role's hand-over.
+struct TileFeed {
+    int4 d1, d2;       // descriptors of the current and the next tile
+    int32_t c1;        // this row's entry code in the current tile
+};
+__device__ __forceinline__ int4 load_desc(const TcParams &p, int64_t j, int64_t my_tiles) {
+    return j < my_tiles ? __ldg(p.tiles + blockIdx.x + j * gridDim.x) : make_int4(0, 0, 0, 0);
+}
+__device__ __forceinline__ int32_t load_code(const TcParams &p, const int4 &d, int e) {
+    Tile tl;
+    decode_tile(p, d, tl);
+    if (e >= tl.n) return 0;
+    return tl.own ? (int32_t)((tl.t0 + e) * 32) : __ldg(p.entries + tl.first + e);
+}
+__device__ __forceinline__ void feed_init(TileFeed &f, const TcParams &p, int64_t j0, int64_t step,
+                                          int64_t my_tiles, int e) {
+    f.d1 = load_desc(p, j0, my_tiles);
+    f.d2 = load_desc(p, j0 + step, my_tiles);
+    f.c1 = load_code(p, f.d1, e);
+}
+// The row job of the current tile; advances the feed to the next one.
+__device__ __forceinline__ RowJob feed_next(TileFeed &f, const TcParams &p, int64_t j, int64_t step,
+                                            int64_t my_tiles, int e) {
+    const int4 d3 = load_desc(p, j + 2 * step, my_tiles);
+    const int32_t c2 = load_code(p, f.d2, e);
     RowJob rj;
-    rj.tl.bg = ti.bg; rj.tl.chunk = ti.chunk; rj.tl.n = ti.n;
-    rj.tl.own = ti.own; rj.tl.first = 0; rj.tl.t0 = 0;
-    rj.b = ti.b; rj.g = ti.g;
-    rj.valid = e < ti.n;
-    const int32_t code = rj.valid ? ti.code[e] : 0;
-    rj.t = code >> 5;
-    rj.k = code & 31;
+    decode_tile(p, f.d1, rj.tl);
+    rj.valid = e < rj.tl.n;
+    rj.t = f.c1 >> 5;
+    rj.k = f.c1 & 31;
+    rj.b = (int)rj.tl.bg / p.Hkv;                  // bg < 2^31 (checked on the host)
+    rj.g = (int)rj.tl.bg - rj.b * p.Hkv;
+    f.d1 = f.d2; f.d2 = d3; f.c1 = c2;
     return rj;
 }
 
@@ -240,11 +257,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     uint64_t *v_full = bars + 6, *vp_empty = bars + 9;                 // [NVP]
     uint64_t *sfull = bars + 12, *sfree = bars + 14, *pfull = bars + 16;
     uint64_t *ofull = bars + 18, *ofree = bars + 20, *pempty = bars + 22;
-    uint64_t *ifull = bars + 24, *ifree = bars + 24 + kRing;
-    uint32_t *s_tmem = (uint32_t *)(bars + 24 + 2 * kRing);
-    static_assert((24 + 2 * kRing) * 8 + 8 <= C::BAR_BYTES, "barrier block overflows its reserve");
+    uint32_t *s_tmem = (uint32_t *)(bars + 24);
+    static_assert(24 * 8 + 8 <= C::BAR_BYTES, "barrier block overflows its reserve");
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
-    __shared__ TileInfo ring[kRing];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // key rows 64..79 of every K block: the landmark rows land in 64 (and 65)
@@ -274,10 +289,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::mbar_init(&ofull[s], 1);
             tc::mbar_init(&ofree[s], 4);       // one arrive per epilogue warp
             tc::mbar_init(&pempty[s], 1);      // P.V done: TMEM P slot free
-        }
-        for (int i = 0; i < kRing; ++i) {
-            tc::mbar_init(&ifull[i], 1);
-            tc::mbar_init(&ifree[i], 8);       // softmax warps + one epilogue group's warps
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -318,20 +329,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const int bq = (int)d0.bg / Hkv;            // bg < 2^31 (checked on the host)
             const int gq = (int)d0.bg - bq * Hkv;
 
-            // publish the tile's metadata
-            const int ri = (int)(j & (kRing - 1));
             int ok = 1;
-            if (lane == 0 && j >= kRing) ok = wait_bar(&ifree[ri], reuse_parity(j / kRing), s_abort);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (lane < 16) ring[ri].code[lane] = c0;
-            if (lane == 0) {
-                ring[ri].bg = d0.bg; ring[ri].chunk = d0.chunk;
-                ring[ri].n = d0.n; ring[ri].own = d0.own;
-                ring[ri].b = bq; ring[ri].g = gq;
-            }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&ifull[ri]);
-
             // Q/K slot j % 3, free once the S of tile j - 3 is done: the chunk's
             // K rows, its landmark (bf16 high / low parts as key rows 64, 65)
             // and one Q box per entry (all G query-head rows, both halves of d
@@ -451,11 +449,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int r = q4 * 32 + lane;             // tile row
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
-        for (int64_t j = 0; j < my_tiles; ++j) {
-            const int ri = (int)(j & (kRing - 1));
-            if (!warp_wait(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
-            const RowJob cur = read_row(ring[ri], e);
-            warp_arrive(&ifree[ri]);
+        const int sg = (warp - 2) >> 2;
+        TileFeed feed;
+        feed_init(feed, p, sg, 2, my_tiles, e);
+        for (int64_t j = sg; j < my_tiles; j += 2) {
+            const RowJob cur = feed_next(feed, p, j, 2, my_tiles, e);
             const int s = (int)(j & 1);
             const int64_t b = cur.b;
             const int g = cur.g;
@@ -533,19 +531,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
     } else if (warp < kEpiEnd) {
         // ------------------------------------------------------------ epilogue
-        // Two groups of four warps; group eg takes the tiles j = eg, eg+2, ...
-        // (TMEM O slot eg), so one tile's stores overlap the next one's.
-        const int eg = (warp - kEpiWarp0) >> 2;
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
         constexpr int NCH = D / 32;               // 32-column chunks of a row
-        for (int64_t j = eg; j < my_tiles; j += 2) {
-            const int ri = (int)(j & (kRing - 1));
-            if (!warp_wait(&ifull[ri], (uint32_t)((j / kRing) & 1), s_abort)) break;
-            const RowJob cur = read_row(ring[ri], e);
-            warp_arrive(&ifree[ri]);
+        TileFeed feed;
+        feed_init(feed, p, 0, 1, my_tiles, e);
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            const RowJob cur = feed_next(feed, p, j, 1, my_tiles, e);
             const int s = (int)(j & 1);
             const int64_t b = cur.b;
             const int g = cur.g;
