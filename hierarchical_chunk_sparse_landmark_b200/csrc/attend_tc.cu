@@ -610,8 +610,13 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
     static_assert(KP % SG == 0 && KP <= 32, "slots are taken SG at a time");
     grid_dep_wait();                                 // the chunk outputs come from attend_tc_kernel
     const int lane = threadIdx.x & 31;
-    const int64_t srow = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    if (srow >= groups) return;                      // srow = (b*L + t)*Hkv + g
+    // Rows in reverse: attend_tc_kernel writes the chunk outputs window by
+    // window, so when it ends L2 still holds the last windows' outputs; those
+    // are read first.  Every consumed 128-byte line is then discarded from L2
+    // (the data is dead), so dirty lines still there are never written back.
+    const int64_t lin = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (lin >= groups) return;
+    const int64_t srow = groups - 1 - lin;           // srow = (b*L + t)*Hkv + g
     const int64_t bt = srow / Hkv;
     const int g = (int)(srow % Hkv);
     const int h = lane % G;
@@ -646,6 +651,7 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
             w_out[hrow * topk + k] = k < nsel ? __expf(zh[k].x - m) * inv : 0.f;
     float acc[NP][8];
     const float fo = own_f[hrow];
+    constexpr int LINES = G * D * 2 / 128;           // 128-byte lines of one slot
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
         const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&rown[i]);
@@ -656,6 +662,8 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
             acc[i][2 * e + 1] = fo * f.y;
         }
     }
+    __syncwarp();
+    for (int l = lane; l < LINES; l += 32) tc::discard_l2(reinterpret_cast<const uint8_t *>(ob) + l * 128);
 #pragma unroll
     for (int k0 = 0; k0 < KP; k0 += SG) {
         if (k0 >= nsel) break;
@@ -683,6 +691,10 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
                 }
             }
         }
+        __syncwarp();
+        const int nv = nsel - k0 < SG ? nsel - k0 : SG;  // slots of this group that were read
+        for (int l = lane; l < nv * LINES; l += 32)
+            tc::discard_l2(reinterpret_cast<const uint8_t *>(pb + (int64_t)k0 * SLOT) + l * 128);
     }
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
