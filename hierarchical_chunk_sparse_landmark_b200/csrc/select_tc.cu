@@ -258,8 +258,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             const int s = n & 1;
             if (!sel_wait(&tfull[s], (uint32_t)((n >> 1) & 1), s_abort)) break;
             tc::fence_after_sync();
+            // 32-column blocks past the block's last visible chunk hold nothing
+            const int64_t vis = nvis_max - (int64_t)n * C::N;
+            const int ncb = vis >= C::N ? C::N / 32 : (int)((vis + 31) / 32);
 #pragma unroll 1
-            for (int cb = 0; cb < C::N / 32; ++cb) {
+            for (int cb = 0; cb < ncb; ++cb) {
                 float sc[32];
                 tc::tmem_ld32(tmem + s * C::N + cb * 32 + lane_off, sc);
                 tc::tmem_wait_ld();
