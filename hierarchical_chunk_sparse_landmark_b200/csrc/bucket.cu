@@ -6,15 +6,17 @@
 // chunk they selected: a tile is one chunk's K/V and up to 128/G entries (G
 // query-head rows each) that chose it, so each chunk's K/V is read once per
 // tile instead of once per query.  Grouping is done per token window (W
-// consecutive tokens of one (b, g)): the per-entry partial outputs of a window
-// are written and then fused while they are still in L2.
+// consecutive tokens of one (b, g); one window spans the whole sequence unless
+// the window count would exceed the work lists' limit).
 //
 // Passes over the selection (all windows at once):
 //   count   -- entries per (window, chunk)                 (shared-memory histogram)
 //   scan    -- bucket offsets, tile descriptors per window (one block per window)
-//   order   -- start of every segment of the work queue    (one block)
-//   scatter -- entry codes t*32+k into their bucket slots  (atomic cursors)
-//   flatten -- one descriptor per queue position           (one block per window)
+//   fill    -- one launch, two kinds of blocks:
+//              scatter: entry codes t*32+k into their bucket slots (atomic cursors)
+//              flatten: one descriptor per queue position, each window's block
+//                       taking its segment starts from the tile counts of the
+//                       windows before it
 // The order of entries inside a bucket is not fixed, which does not change
 // any result: every tile row is computed independently of the other rows.
 //
@@ -134,90 +136,20 @@ bucket_scan_kernel(const int32_t *__restrict__ counts, WinGeom wg, int32_t *__re
     }
 }
 
-// One block: seg_start[s] for the 2*NW queue segments (see the file comment).
-__global__ void __launch_bounds__(kScanThreads)
-queue_order_kernel(const int32_t *__restrict__ wntiles, WinGeom wg, int64_t NW,
-                   int64_t *__restrict__ seg_start) {
-    grid_dep_wait();
-    __shared__ int64_t warp_s[32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t nseg = 2 * NW;
-    const int64_t per = (nseg + kScanThreads - 1) / kScanThreads;
-    const int64_t s0 = tid * per, s1 = (s0 + per < nseg) ? s0 + per : nseg;
-    auto seg_len = [&](int64_t s) -> int64_t {
-        const int64_t type_own = s & 1, n = s >> 1;
-        if (!type_own) return wntiles[n];
-        int64_t bg, ts, te;
-        window_span(wg, n, bg, ts, te);
-        return (te - ts + wg.ept - 1) / wg.ept;
-    };
-    int64_t sum = 0;
-    for (int64_t s = s0; s < s1; ++s) sum += seg_len(s);
-    int64_t inc = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int64_t a = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += a;
-    }
-    if (lane == 31) warp_s[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        int64_t a = warp_s[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int64_t x = __shfl_up_sync(0xffffffffu, a, o);
-            if (lane >= o) a += x;
-        }
-        warp_s[lane] = a;
-    }
-    __syncthreads();
-    int64_t off = inc - sum + (warp ? warp_s[warp - 1] : 0);
-    for (int64_t s = s0; s < s1; ++s) {
-        seg_start[s] = off;
-        off += seg_len(s);
-    }
-    if (s1 == nseg && s0 < s1) seg_start[nseg] = off;
-    if (nseg == 0 && tid == 0) seg_start[0] = 0;
-}
-
-// Flat tile list: tiles[q] = descriptor of queue position q, so the consumer
-// needs one load per tile instead of a search over segment starts.
-// {bg, chunk, first entry, n} for retrieved-chunk tiles; own-chunk tiles are
-// {bg, 0, first token, n | kOwnTileFlag} (the consumer derives the chunk).
-constexpr int kOwnTileFlag = 1 << 30;
-__global__ void __launch_bounds__(kBucketThreads)
-flatten_tiles_kernel(const int4 *__restrict__ wtiles, const int32_t *__restrict__ wntiles,
-                     const int64_t *__restrict__ seg_start, WinGeom wg,
-                     int4 *__restrict__ tiles) {
-    grid_dep_wait();
-    const int64_t n = blockIdx.x;
-    int64_t bg, ts, te;
-    window_span(wg, n, bg, ts, te);
-    const int64_t c0 = seg_start[2 * n], o0 = seg_start[2 * n + 1];
-    const int nc = wntiles[n];
-    for (int j = threadIdx.x; j < nc; j += blockDim.x) tiles[c0 + j] = wtiles[n * wg.cap + j];
-    const int64_t no = (te - ts + wg.ept - 1) / wg.ept;
-    for (int64_t j = threadIdx.x; j < no; j += blockDim.x) {
-        const int64_t t0 = ts + j * wg.ept;
-        const int64_t cnt = te - t0 < wg.ept ? te - t0 : wg.ept;
-        tiles[o0 + j] = make_int4((int)bg, 0, (int)t0, (int)cnt | kOwnTileFlag);
-    }
-}
-
 // entries[cursor[n, i]++] = t * 32 + k.  A block's 256 tokens lie in one window
 // (W is a multiple of 256).  With the chunk histogram in shared memory, each
 // entry takes its rank within the block by a shared atomic, the block reserves
 // each chunk's range with one global atomic, and the entries are written
 // at base + rank.
-__global__ void __launch_bounds__(kBucketThreads)
-bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int use_smem,
-                      int32_t *__restrict__ cursor, int32_t *__restrict__ entries) {
-    grid_dep_wait();
-    extern __shared__ int32_t hist[];             // [Nc] counts, then range bases
-    const int g = blockIdx.y, b = blockIdx.z;
-    const int64_t t = (int64_t)blockIdx.x * kBucketThreads + threadIdx.x;
-    const int64_t bg = (int64_t)b * wg.Hkv + g;
-    const int64_t n = bg * wg.nwb + ((int64_t)blockIdx.x * kBucketThreads) / wg.W;
+__device__ __forceinline__ void bucket_scatter(const int32_t *__restrict__ idx, const WinGeom &wg,
+                                               int use_smem, int64_t blk, int32_t *__restrict__ cursor,
+                                               int32_t *__restrict__ entries, int32_t *hist) {
+    // blk enumerates (token block, g, b) with the token block fastest
+    const int64_t ntb = (wg.L + kBucketThreads - 1) / kBucketThreads;
+    const int64_t tb = blk % ntb, bg = blk / ntb;
+    const int g = (int)(bg % wg.Hkv), b = (int)(bg / wg.Hkv);
+    const int64_t t = tb * kBucketThreads + threadIdx.x;
+    const int64_t n = bg * wg.nwb + (tb * kBucketThreads) / wg.W;
     const int32_t *ip = idx + (((int64_t)b * wg.L + (t < wg.L ? t : 0)) * wg.Hkv + g) * wg.topk;
     if (!use_smem) {
         if (t >= wg.L) return;
@@ -249,6 +181,63 @@ bucket_scatter_kernel(const int32_t *__restrict__ idx, WinGeom wg, int use_smem,
         if (chunk[k] >= 0) entries[hist[chunk[k]] + rank[k]] = (int32_t)(t * 32 + k);
 }
 
+// Flat tile list: tiles[q] = descriptor of queue position q, so the consumer
+// needs one load per tile instead of a search over segment starts.
+// {bg, chunk, first entry, n} for retrieved-chunk tiles; own-chunk tiles are
+// {bg, 0, first token, n | kOwnTileFlag} (the consumer derives the chunk).
+// Window n's segments start after the tiles of windows 0 .. n-1 (queue order
+// C0 O0 C1 O1 ...); the last window also writes the queue length.
+constexpr int kOwnTileFlag = 1 << 30;
+__device__ __forceinline__ int64_t own_tiles(const WinGeom &wg, int64_t n) {
+    int64_t bg, ts, te;
+    window_span(wg, n, bg, ts, te);
+    return (te - ts + wg.ept - 1) / wg.ept;
+}
+__device__ __forceinline__ void bucket_flatten(const int4 *__restrict__ wtiles,
+                                               const int32_t *__restrict__ wntiles, const WinGeom &wg,
+                                               int64_t n, int64_t NW, int64_t *__restrict__ seg_start,
+                                               int4 *__restrict__ tiles, int64_t *red) {
+    int64_t part = 0;
+    for (int64_t m = threadIdx.x; m < n; m += blockDim.x) part += wntiles[m] + own_tiles(wg, m);
+    for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
+    __syncthreads();
+    int64_t c0 = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) c0 += red[w];
+    const int nc = wntiles[n];
+    const int64_t o0 = c0 + nc, no = own_tiles(wg, n);
+    if (threadIdx.x == 0) {
+        seg_start[2 * n] = c0;
+        seg_start[2 * n + 1] = o0;
+        if (n == NW - 1) seg_start[2 * NW] = o0 + no;
+    }
+    int64_t bg, ts, te;
+    window_span(wg, n, bg, ts, te);
+    for (int j = threadIdx.x; j < nc; j += blockDim.x) tiles[c0 + j] = wtiles[n * wg.cap + j];
+    for (int64_t j = threadIdx.x; j < no; j += blockDim.x) {
+        const int64_t t0 = ts + j * wg.ept;
+        const int64_t cnt = te - t0 < wg.ept ? te - t0 : wg.ept;
+        tiles[o0 + j] = make_int4((int)bg, 0, (int)t0, (int)cnt | kOwnTileFlag);
+    }
+}
+
+// Blocks [0, nscatter) scatter entries, blocks [nscatter, nscatter + NW) flatten
+// one window each; both read only what bucket_scan_kernel wrote.
+__global__ void __launch_bounds__(kBucketThreads)
+bucket_fill_kernel(const int32_t *__restrict__ idx, WinGeom wg, int use_smem, int64_t nscatter,
+                   int64_t NW, int32_t *__restrict__ cursor, int32_t *__restrict__ entries,
+                   const int4 *__restrict__ wtiles, const int32_t *__restrict__ wntiles,
+                   int64_t *__restrict__ seg_start, int4 *__restrict__ tiles) {
+    grid_dep_wait();
+    extern __shared__ int32_t hist[];             // [Nc] counts, then range bases
+    __shared__ int64_t red[kBucketThreads / 32];
+    const int64_t blk = blockIdx.x;
+    if (blk < nscatter)
+        bucket_scatter(idx, wg, use_smem, blk, cursor, entries, hist);
+    else
+        bucket_flatten(wtiles, wntiles, wg, blk - nscatter, NW, seg_start, tiles, red);
+}
+
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
@@ -267,13 +256,11 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
     e = launch_pdl(bucket_scan_kernel, dim3((unsigned)NW), dim3(kScanThreads), 0, st, counts, wg,
                    cursor, wtiles, wntiles, done);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(queue_order_kernel, dim3(1), dim3(kScanThreads), 0, st, wntiles, wg, NW, seg_start);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(bucket_scatter_kernel, grid, dim3(kBucketThreads), smem, st, idx, wg, use_smem,
-                   cursor, entries);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(flatten_tiles_kernel, dim3((unsigned)NW), dim3(kBucketThreads), 0, st,
-                      wtiles, wntiles, seg_start, wg, tiles);
+    const int64_t nscatter = (int64_t)grid.x * grid.y * grid.z;
+    if (NW == 0 && nscatter == 0) return cudaSuccess;
+    return launch_pdl(bucket_fill_kernel, dim3((unsigned)(nscatter + NW)), dim3(kBucketThreads), smem, st,
+                      idx, wg, use_smem, nscatter, NW, cursor, entries, (const int4 *)wtiles,
+                      (const int32_t *)wntiles, seg_start, tiles);
 }
 
 }  // namespace hsa
