@@ -112,33 +112,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 __device__ __forceinline__ uint32_t pack_bf16x2_int(float a, float b) {
     return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
 }
-// 2^x of two packed floats (x <= 0) on the FMA pipe, so that part of the
-// softmax's exponentials leave the MUFU unit: Cody-Waite style reduction
-// x = n + f with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to an
-// integer) and |f| <= 1/2, a cubic for 2^f, and n added to the exponent
-// field.  The cubic's coefficients are a least-squares fit of 2^f on
-// [-1/2, 1/2] in relative error (iteratively reweighted towards the minimax
-// fit); its relative error is below 7.5e-5, under the 2^-9 of the bf16 P it
-// feeds.  x is clamped at -126 so the exponent field stays >= 0: inputs below
-// that (and -inf, the causal mask) give a value below 2^-125 instead of 0.
-constexpr int kPolyPairs = 0;   // of the 16 column pairs of each 32-column half
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-    float a, b;
-    unpack_f2(x2, a, b);
-    const uint64_t x = pack_f2(fmaxf(a, -126.f), fmaxf(b, -126.f));
-    const uint64_t j = add_f2(x, pack_f2(12582912.f, 12582912.f));          // low bits: round(x)
-    const uint64_t n = add_f2(j, pack_f2(-12582912.f, -12582912.f));
-    const uint64_t f = ffma2(n, pack_f2(-1.f, -1.f), x);                     // x - n
-    uint64_t y = ffma2(pack_f2(0.0551716685f, 0.0551716685f), f, pack_f2(0.242611140f, 0.242611140f));
-    y = ffma2(y, f, pack_f2(0.693260968f, 0.693260968f));
-    y = ffma2(y, f, pack_f2(0.999928057f, 0.999928057f));
-    float y0, y1, j0, j1;
-    unpack_f2(y, y0, y1);
-    unpack_f2(j, j0, j1);
-    return pack_f2(__uint_as_float(__float_as_uint(y0) + (__float_as_uint(j0) << 23)),
-                   __uint_as_float(__float_as_uint(y1) + (__float_as_uint(j1) << 23)));
-}
-
 // bf16 pair -> two floats (exact: the bf16 bits are the high half of fp32)
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
@@ -491,20 +464,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
                 float a0, a1, b0, b1;
-                const uint64_t xa = ffma2(pack_f2(s0[c], s0[c + 1]), c2, m2);
-                const uint64_t xb = ffma2(pack_f2(s1[c], s1[c + 1]), c2, m2);
-                if (c / 2 < kPolyPairs) {
-                    unpack_f2(exp2_poly2(xa), s0[c], s0[c + 1]);
-                } else {
-                    unpack_f2(xa, a0, a1);
-                    s0[c] = tc::ex2_approx(a0); s0[c + 1] = tc::ex2_approx(a1);
-                }
-                if (c / 2 < kPolyPairs) {
-                    unpack_f2(exp2_poly2(xb), s1[c], s1[c + 1]);
-                } else {
-                    unpack_f2(xb, b0, b1);
-                    s1[c] = tc::ex2_approx(b0); s1[c + 1] = tc::ex2_approx(b1);
-                }
+                unpack_f2(ffma2(pack_f2(s0[c], s0[c + 1]), c2, m2), a0, a1);
+                unpack_f2(ffma2(pack_f2(s1[c], s1[c + 1]), c2, m2), b0, b1);
+                s0[c] = tc::ex2_approx(a0); s0[c + 1] = tc::ex2_approx(a1);
+                s1[c] = tc::ex2_approx(b0); s1[c + 1] = tc::ex2_approx(b1);
                 l2 = add_f2(l2, add_f2(pack_f2(s0[c], s0[c + 1]), pack_f2(s1[c], s1[c + 1])));
             }
             if (cur.valid) {
