@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include "attend_tc.h"
 #include "common.cuh"
 #include "hsa.h"
 
@@ -32,23 +33,6 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
                           int64_t *seg_start, int4 *tiles, cudaStream_t st);
-struct TcLaunch {
-    const void *Q, *K, *V, *lm;
-    int B, H, Hkv, S, topk, own_chunk, lm_bf16;
-    int64_t L, W, cap;
-    float scale;
-    const int32_t *idx, *entries;
-    const int4 *tiles;                // one descriptor per queue position
-    const int64_t *qlen;              // number of tiles (device)
-    float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
-    __nv_bfloat16 *part, *own;
-    void *O;
-    unsigned *status;
-    int num_sms;
-};
-bool attend_tc_supported(bool bf16, int G, int d);
-int64_t attend_tc_max_windows();
-cudaError_t launch_attend_tc(const TcLaunch &a, int d, cudaStream_t st, cudaEvent_t mid);
 }  // namespace hsa
 
 using namespace hsa;

@@ -43,6 +43,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "attend_tc.h"
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -730,24 +731,6 @@ static bool make_map_q3d(CUtensorMap *m, const void *base, uint64_t rows, int D,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
-
-struct TcLaunch {
-    const void *Q, *K, *V;
-    // landmarks as bf16 rows: [B*Hkv*Nc, D] (lm_bf16) or the two planes
-    // [2][B*Hkv*Nc, D] of an fp32 landmark's bf16 high and low parts
-    const void *lm;
-    int B, H, Hkv, S, topk, own_chunk, lm_bf16;
-    int64_t L, W, cap;
-    float scale;
-    const int32_t *idx, *entries;
-    const int4 *tiles;                // one descriptor per queue position
-    const int64_t *qlen;              // number of tiles (device)
-    float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
-    __nv_bfloat16 *part, *own;
-    void *O;
-    unsigned *status;
-    int num_sms;
-};
 
 template <int D, int G>
 static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEvent_t mid) {
