@@ -279,6 +279,12 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
     const void *lm_use = lm;
     bool lm_bf16 = lm_dt == HSA_BF16;
     stage_mark(0, st);
+    const bool use_tc = bf16 && lay.tc && !force_simt_path() &&
+                        attend_tc_supported(bf16, H / Hkv, d);
+    // the bucket counts are zeroed first, so that every kernel of the chain
+    // can follow its predecessor as a programmatic dependent
+    if (use_tc && cudaMemsetAsync(ws + lay.counts_off, 0, lay.counts_bytes, st) != cudaSuccess)
+        return HSA_ERR_CUDA;
     if (!lm) {
         float *lm_ws = (float *)(ws + lay.lm_off);
         cudaError_t e = launch_landmarks(K, bf16, lm_ws, B, Hkv, L, d, st);
@@ -288,8 +294,6 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         lm_bf16 = false;
     }
     stage_mark(1, st);
-    const bool use_tc = bf16 && lay.tc && !force_simt_path() &&
-                        attend_tc_supported(bf16, H / Hkv, d);
     // The tensor-core path computes the fusion logits inside its S tiles and
     // the weights in fuse_kernel, so the selection skips them there.
     cudaError_t e;
@@ -314,15 +318,13 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
     stage_mark(2, st);
     if (use_tc) {
         const int64_t Nc = L / S;
-        if (cudaMemsetAsync(ws + lay.counts_off, 0, lay.counts_bytes, st) != cudaSuccess)
-            return HSA_ERR_CUDA;
         e = launch_bucket(idx, B, Hkv, L, topk, Nc, 128 / (H / Hkv), lay.W, lay.cap,
                           (int32_t *)(ws + lay.counts_off), (int32_t *)(ws + lay.cursor_off),
                           (int32_t *)(ws + lay.entries_off), (int4 *)(ws + lay.wtiles_off),
                           (int32_t *)(ws + lay.wntiles_off), (int32_t *)(ws + lay.done_off),
                           (int64_t *)(ws + lay.seg_off), (int4 *)(ws + lay.tiles_off), st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
-        t_launches += 5;
+        t_launches += 3;                  // count, scan, fill (scatter + flatten)
         stage_mark(3, st);
         TcLaunch a;
         a.Q = Q; a.K = K; a.V = V; a.lm = lm_bf16 ? lm_use : lm_split; a.lm_bf16 = lm_bf16 ? 1 : 0;

@@ -249,9 +249,10 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
     dim3 grid((unsigned)((L + kBucketThreads - 1) / kBucketThreads), (unsigned)Hkv, (unsigned)B);
     const int use_smem = Nc <= 8192 ? 1 : 0;
     const size_t smem = use_smem ? sizeof(int32_t) * (size_t)(Nc > 0 ? Nc : 1) : 0;
-    // the count pass follows the counts memset (not a kernel): plain launch
-    bucket_count_kernel<<<grid, kBucketThreads, smem, st>>>(idx, wg, use_smem, counts);
-    cudaError_t e = cudaGetLastError();
+    // the counts were zeroed before the selection: the count pass follows the
+    // selection kernel as a programmatic dependent
+    cudaError_t e = launch_pdl(bucket_count_kernel, grid, dim3(kBucketThreads), smem, st, idx, wg,
+                               use_smem, counts);
     if (e != cudaSuccess) return e;
     e = launch_pdl(bucket_scan_kernel, dim3((unsigned)NW), dim3(kScanThreads), 0, st, counts, wg,
                    cursor, wtiles, wntiles, done);
