@@ -335,7 +335,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.qlen = (const int64_t *)(ws + lay.seg_off) + 2 * lay.NW;
         a.zf = (float *)(ws + lay.zf_off); a.own_f = (float *)(ws + lay.ownf_off);
         a.w_out = w_out;
-        a.part = (__nv_bfloat16 *)(ws + lay.part_off); a.own = (__nv_bfloat16 *)(ws + lay.own_off);
+        a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;
         a.num_sms = num_sms();
         e = launch_attend_tc(a, d, st, stage_event(4));

@@ -12,14 +12,14 @@
 // fusion logit scale * q_h . l_chunk:
 //
 //   S = Q_rows . [K_chunk ; l_hi ; l_lo]^T  M=128, N=80, K=d  (tcgen05 -> TMEM)
-//   P = exp(S*scale - rowmax)               per row in registers, bf16 -> TMEM
+//   P = 2^-6 exp(S*scale - rowmax)          per row in registers, bf16 -> TMEM
 //   O = P . V_chunk                         M=128, N=d, K=64  (tcgen05, A from TMEM)
-//   partial[t, g, k] = O (bf16); per (t, h, k): the fusion logit
+//   partial[t, g, k] = O (fp16); per (t, h, k): the fusion logit
 //   scale * (S[:,64] + S[:,65]) and f = 1 / sum of the row's P
 //
 // Own tiles: 128/G consecutive tokens of a chunk against that chunk with the
 // causal mask (keys c*S .. t); their output (the own-chunk term, same scaling,
-// f = own_chunk / row sum) goes to a bf16 array.  fuse_kernel then completes
+// f = own_chunk / row sum) goes to an fp16 array.  fuse_kernel then completes
 // the method, one warp per (t, g):
 //   w = softmax over the token's selected chunks of the logits,
 //   O = f_own * own + sum_k w_k * f_k * partial_k  (bf16 out).
@@ -36,12 +36,13 @@
 //   warp 14      MMA issuer for P.V
 //   warps 2-9    softmax   (two groups taking alternate tiles; thread = tile
 //                           row = TMEM lane)
-//   warps 10-13  epilogue  (TMEM -> bf16 partial slots / own-chunk term)
+//   warps 10-13  epilogue  (TMEM -> fp16 partial slots / own-chunk term)
 // Tiles are independent, so no block waits on another.  Every wait is
 // bounded; on expiry the block sets the status flag in the workspace, lets
 // in-flight copies land, frees its TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "attend_tc.h"
 #include "common.cuh"
@@ -83,8 +84,8 @@ struct TcParams {
     const int32_t *entries;
     float *zf;                    // [B, L, H, topk] x (fusion logit, 1 / chunk row sum)
     float *own_f;                 // [B, L, H] add_own / own-chunk row sum
-    __nv_bfloat16 *part;          // [B*L*Hkv*topk entries][D/8][G][8] chunk outputs
-    __nv_bfloat16 *own;           // [B*L*Hkv rows (t, g)][D/8][G][8] own-chunk term
+    __half *part;                 // [B*L*Hkv*topk entries][D/8][G][8] chunk outputs
+    __half *own;                  // [B*L*Hkv rows (t, g)][D/8][G][8] own-chunk term
     unsigned *status;
     int64_t L, Nc;
     int H, Hkv, topk, S, add_own;
@@ -108,14 +109,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // Two floats to a bf16 pair on the integer pipe: add half an ulp of bf16 to
 // the fp32 bit pattern and keep the high halves (one byte permute).  Rounds to
 // nearest with ties away from zero (round-to-nearest-even differs only on
-// exact ties).  The conversion instruction shares the transcendental pipe
-// with ex2, which the softmax keeps busy; the integer pipe is mostly idle.
+// exact ties); used for P, whose pairs the P.V MMA reads from TMEM.
 __device__ __forceinline__ uint32_t pack_bf16x2_int(float a, float b) {
     return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
 }
-// bf16 pair -> two floats (exact: the bf16 bits are the high half of fp32)
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+// Chunk outputs are fp16 (11-bit significand): with bf16 the rounding of a
+// partial and of the final O together could exceed the 2e-2 bf16 output
+// tolerance where |O| approaches 4.
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&u));
 }
 
 // Bounded mbarrier wait that also gives up when another role aborted.
@@ -458,8 +464,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             const float mx = fmaxf(fmaxf(m4[0], m4[2]), fmaxf(m4[1], m4[3]));
             // P = exp(S*scale - rowmax), unnormalised (1/rowsum is applied by
-            // fuse_kernel; P.V stays within 64 max |V|, far inside bf16 range)
-            const float ms = mx * p.scale_log2e;
+            // fuse_kernel; the 2^-6, an exponent shift, keeps P.V within
+            // max |V| for its fp16 store)
+            const float ms = fmaf(mx, p.scale_log2e, 6.f);
             const uint64_t c2 = pack_f2(p.scale_log2e, p.scale_log2e), m2 = pack_f2(-ms, -ms);
             uint64_t l2 = 0ull;
 #pragma unroll
@@ -528,10 +535,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq)
                         blk[((ch + u) * 4 + qq) * G + h] = make_uint4(
-                            pack_bf16x2_int(o[u][8 * qq + 0], o[u][8 * qq + 1]),
-                            pack_bf16x2_int(o[u][8 * qq + 2], o[u][8 * qq + 3]),
-                            pack_bf16x2_int(o[u][8 * qq + 4], o[u][8 * qq + 5]),
-                            pack_bf16x2_int(o[u][8 * qq + 6], o[u][8 * qq + 7]));
+                            pack_f16x2(o[u][8 * qq + 0], o[u][8 * qq + 1]),
+                            pack_f16x2(o[u][8 * qq + 2], o[u][8 * qq + 3]),
+                            pack_f16x2(o[u][8 * qq + 4], o[u][8 * qq + 5]),
+                            pack_f16x2(o[u][8 * qq + 6], o[u][8 * qq + 7]));
                 }
             }
             tc::fence_before_sync();
@@ -563,7 +570,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // loads in flight per warp, not the warp count, keep HBM busy.
 template <int D, int G, int KP>
 __global__ void __launch_bounds__(256, (G * D / 256) <= 4 ? 2 : 1)
-fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restrict__ own,
+fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
             const float2 *__restrict__ zf, const float *__restrict__ own_f,
             const int32_t *__restrict__ idx, int64_t groups, int H, int Hkv, int topk,
             float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
@@ -621,7 +628,7 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
         const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&rown[i]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(w2[e]);
+            const float2 f = unpack_f16x2(w2[e]);
             acc[i][2 * e] = fo * f.x;
             acc[i][2 * e + 1] = fo * f.y;
         }
@@ -649,7 +656,7 @@ fuse_kernel(const __nv_bfloat16 *__restrict__ part, const __nv_bfloat16 *__restr
                 const uint32_t *w2 = reinterpret_cast<const uint32_t *>(&rv);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 f = unpack_bf16x2(w2[e]);
+                    const float2 f = unpack_f16x2(w2[e]);
                     acc[i][2 * e] = fmaf(wk, f.x, acc[i][2 * e]);
                     acc[i][2 * e + 1] = fmaf(wk, f.y, acc[i][2 * e + 1]);
                 }

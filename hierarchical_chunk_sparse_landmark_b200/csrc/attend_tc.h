@@ -2,6 +2,7 @@
 // attention (attend_tc.cu), shared with the C-ABI dispatch (abi.cu).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,7 +20,7 @@ struct TcLaunch {
     const int4 *tiles;                // one descriptor per queue position
     const int64_t *qlen;              // number of tiles (device)
     float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
-    __nv_bfloat16 *part, *own;
+    __half *part, *own;              // fp16 chunk outputs / own-chunk term
     void *O;
     unsigned *status;
     int num_sms;

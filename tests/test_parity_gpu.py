@@ -106,6 +106,17 @@ def test_prefill_landmark_modes(oracle_lib, lm_kind):
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
 
 
+@pytest.mark.parametrize("seed", [5, 11, 23])
+def test_prefill_large_outputs(oracle_lib, seed):
+    # Few visible chunks and doubled landmarks concentrate the attention, so |O|
+    # approaches max |V| and the rounding of the chunk outputs matters most.
+    wl = Workload("concentrated", "prefill", "bf16", B=1, L=64 * 6 + 9, H=16, Hkv=2, d=128,
+                  S=64, topk=4, landmarks="input_x2", seed=seed)
+    x = make_prefill_inputs(wl, DEV)
+    rep, _ = prefill_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+
+
 def test_prefill_explicit_scale(oracle_lib):
     wl = small("f32", B=1, L=300, H=4, Hkv=1, d=64)
     x = make_prefill_inputs(wl, DEV)
