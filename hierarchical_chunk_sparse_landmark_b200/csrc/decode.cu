@@ -95,6 +95,7 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
     const int64_t nunits = (Nc + ROWS - 1) / ROWS;
     const TL *lm_bg = lm + bg * Nc * D;
     const int KP = pow2_at_least(topk);
+    grid_dep_wait();            // inputs and workspace may come from the previous kernel
 
     if (tid == 0) {
         for (int i = 0; i < kScanStages; ++i) {
@@ -523,9 +524,10 @@ static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc
     cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kScanStages * kStageBytes);
     if (e != cudaSuccess) return e;
-    scan<<<grid, kScanThreads, kScanStages * kStageBytes, st>>>(
-        (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws, idx_out);
-    e = cudaGetLastError();
+    // a programmatic dependent of whatever precedes it on the stream (it waits
+    // for that before reading anything), so its launch overlaps the tail
+    e = launch_pdl(scan, dim3(grid), dim3(kScanThreads), (size_t)(kScanStages * kStageBytes), st,
+                   (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws, idx_out);
     if (e != cudaSuccess) return e;
 
     const size_t smem = AttSmem<T, D>::bytes(H / Hkv);
