@@ -26,9 +26,14 @@
 //                          the current K-th key)
 // (warps 6-11 only help build qbar; the first two landmark tiles are requested
 // before that, so their loads overlap it.)
+// select_tc_half_kernel takes the case where every chunk fits one score tile
+// (Nc <= 128): qbar built per 64-column block of d into one buffer, two blocks
+// per SM (see the comment above it).
 // Every wait is bounded; on expiry the block sets the status flag, lets its
 // copies and MMAs land, frees its TMEM and exits.
 #include <cuda.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -305,6 +310,229 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
+// ---------------------------------------------------------------- one score tile
+// When every chunk fits one N-tile (Nc <= 128, i.e. L <= 8192 at S = 64), the
+// block builds qbar one 64-column block of d at a time into the same buffer:
+// the score MMAs of block kb run while nothing else waits on them, and the
+// next block is written once they are done (`half` barrier).  With one
+// landmark stage and one TMEM score slot the block needs about 80 KB (bf16
+// landmarks) or 96 KB (fp32 landmarks) of shared memory and 256 threads of at
+// most 128 registers, so two blocks share an SM: one block's loads of the
+// query rows overlap the other's MMAs and top-K, and a 4 x 4096-token batch
+// runs in a single wave.
+template <int D, bool LM32>
+struct SelHalfCfg {
+    static constexpr int M = 128, N = 128, KB = D / 64;
+    static constexpr int QP = LM32 ? 2 : 3;
+    static constexpr int LP = LM32 ? 2 : 1;
+    static constexpr int A_PART = M * 128;            // one 64-column block of qbar
+    static constexpr int B_PART = N * D * 2;
+    static constexpr int BAR_OFF = QP * A_PART + LP * B_PART;
+    static constexpr int SMEM = 1024 + BAR_OFF + 256;
+    static constexpr uint32_t TMEM_COLS = N;
+};
+constexpr int kSelHalfThreads = 256;                // 8 warps: all build qbar; 2-5 also top-K
+
+template <int D, bool LM32, int KP>
+__global__ void __launch_bounds__(kSelHalfThreads, 2)
+select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant__ CUtensorMap tmL1,
+                      const SelTcParams p) {
+    using C = SelHalfCfg<D, LM32>;
+    grid_dep_wait();                      // landmarks may come from the previous kernels
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;                                        // [QP][M x 128 B]
+    uint8_t *sB = smem + C::QP * C::A_PART;                    // [LP][KB][N x 128 B]
+    uint64_t *bars = (uint64_t *)(smem + C::BAR_OFF);
+    uint64_t *full = bars, *half = bars + 1, *tfull = bars + 2;
+    uint32_t *s_tmem = (uint32_t *)(bars + 3);
+    volatile int *s_abort = (volatile int *)(s_tmem + 1);
+
+    const int ntb = (int)((p.L + C::M - 1) / C::M);
+    const int tb = ntb - 1 - (int)blockIdx.x;                  // heavy blocks first
+    const int64_t bg = blockIdx.y;
+    const int64_t b = bg / p.Hkv;
+    const int g = (int)(bg % p.Hkv);
+    const int G = p.H / p.Hkv;
+    const int64_t L = p.L;
+    const int64_t t0 = (int64_t)tb * C::M;
+    const int64_t t_last = t0 + C::M - 1 < L ? t0 + C::M - 1 : L - 1;
+    const int64_t nvis_max = t_last / p.S;                     // visible to the block's last token
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 1) {
+        tc::tmem_alloc(s_tmem, C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(full, 1);
+        tc::mbar_init(half, 1);
+        tc::mbar_init(tfull, 1);
+        *s_abort = 0;
+        tc::fence_barrier_init();
+        // the landmark tile does not depend on qbar: start its loads now
+        tc::mbar_expect_tx(full, (uint32_t)(C::LP * C::B_PART));
+        const int row0 = (int)(bg * p.Nc);
+#pragma unroll
+        for (int lp = 0; lp < C::LP; ++lp)
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+                tc::tma_load_2d(sB + lp * C::B_PART + kb * (C::N * 128), lp ? &tmL1 : &tmL0, full,
+                                kb * 64, row0);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+    const float inv_g = 1.f / (float)G;
+    bool ok = true;
+    for (int kb = 0; kb < C::KB; ++kb) {
+        if (kb > 0) {
+            // the MMAs of block kb-1 are done reading the buffer
+            ok = sel_wait(half, (uint32_t)((kb - 1) & 1), s_abort);
+            if (!__syncthreads_and(ok)) break;
+        }
+        // qbar columns kb*64 .. +64: a thread owns (token, 16-byte vector)
+        // pairs and keeps two pairs' loads of eight heads in flight
+        constexpr int NPAIR = C::M * 8;
+        for (int e0 = tid; e0 < NPAIR; e0 += 2 * kSelHalfThreads) {
+            float acc[2][8];
+            const __nv_bfloat16 *qp[2];
+            bool live[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * kSelHalfThreads;
+                const int r = e / 8, c = e % 8;
+                const int64_t t = t0 + r;
+                live[u] = e < NPAIR && t < L;
+                qp[u] = (const __nv_bfloat16 *)p.Q + ((b * L + (live[u] ? t : 0)) * p.H + (int64_t)g * G) * D +
+                        kb * 64 + c * 8;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+            }
+            for (int h0 = 0; h0 < G; h0 += 8) {
+                uint4 raw[2][8];
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int h = 0; h < 8; ++h)
+                        raw[u][h] = live[u] ? ld_stream16(qp[u] + (int64_t)(h0 + h) * D) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        float f[8];
+                        Vec16<__nv_bfloat16>::unpack(raw[u][h], f);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[u][i] += f[i];
+                    }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * kSelHalfThreads;
+                if (e >= NPAIR) continue;
+                const int r = e / 8, c = e % 8;
+                const uint32_t off = tc::sw128_offset(r, c);
+                float x[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = acc[u][i] * inv_g;
+#pragma unroll
+                for (int part = 0; part < C::QP; ++part) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t lo = bf16_bits_rn(x[2 * i]), hi = bf16_bits_rn(x[2 * i + 1]);
+                        w[i] = lo | (hi << 16);
+                        x[2 * i] -= __uint_as_float(lo << 16);
+                        x[2 * i + 1] -= __uint_as_float(hi << 16);
+                    }
+                    *reinterpret_cast<uint4 *>(sA + part * C::A_PART + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (warp == 1 && lane == 0) {
+            // the score products of this block of d (see SelCfg's split)
+            constexpr uint32_t IDESC = tc::idesc_bf16_f32(128, C::N, false);
+            constexpr int NPROD = 3;
+            const int pa[NPROD] = {0, 1, LM32 ? 0 : 2};
+            const int pl[NPROD] = {0, 0, LM32 ? 1 : 0};
+            bool go = kb > 0 || sel_wait(full, 0u, s_abort);
+            if (go) {
+                tc::fence_after_sync();
+#pragma unroll
+                for (int pr = 0; pr < NPROD; ++pr)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sA + pa[pr] * C::A_PART + kk * 32), 16, 1024);
+                        const uint64_t bd = tc::sdesc_sw128(
+                            tc::smem_u32(sB + pl[pr] * C::B_PART + kb * (C::N * 128) + kk * 32), 16, 1024);
+                        tc::mma_bf16(tmem, ad, bd, IDESC, (kb | pr | kk) ? 1u : 0u);
+                    }
+                tc::mma_commit(kb + 1 < C::KB ? half : tfull);
+            }
+        }
+    }
+    if (warp >= 2 && warp < 6) {
+        // ------------------------------------------------------------ top-K
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int64_t t = t0 + r;
+        const int64_t nvis = t < L ? t / p.S : 0;
+        uint64_t v[KP];
+#pragma unroll
+        for (int i = 0; i < KP; ++i) v[i] = 0ull;
+        float tf = -INFINITY;                                  // score of v[KP-1]
+        if (ok && sel_wait(tfull, 0u, s_abort)) {
+            tc::fence_after_sync();
+            // 32-column blocks past the block's last visible chunk hold nothing
+            const int ncb = nvis_max >= C::N ? C::N / 32 : (int)((nvis_max + 31) / 32);
+#pragma unroll 1
+            for (int cb = 0; cb < ncb; ++cb) {
+                float sc[32];
+                tc::tmem_ld32(tmem + cb * 32 + lane_off, sc);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float sv = p.scale * sc[c];
+                    if (cb * 32 + c < nvis && sv >= tf) {
+                        uint64_t x = make_key(sv, cb * 32 + c);
+                        if (x > v[KP - 1]) {
+#pragma unroll
+                            for (int i = 0; i < KP; ++i) {
+                                const uint64_t hi = v[i] > x ? v[i] : x;
+                                x = v[i] > x ? x : v[i];
+                                v[i] = hi;
+                            }
+                            tf = key_score(v[KP - 1]);
+                        }
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            if (t < L) {
+                int32_t *dst = p.idx + ((b * L + t) * p.Hkv + g) * p.topk;
+#pragma unroll
+                for (int k = 0; k < KP; ++k)
+                    if (k < p.topk) dst[k] = key_index(v[k]);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (*s_abort) {
+        if (tid == 0) atomicOr(p.status, kFlagTimeout);
+        const long long t1 = clock64();
+        while (clock64() - t1 < 20000000) { }
+    }
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
 // fp32 landmarks -> two bf16 parts l0 = rn(x), l1 = rn(x - l0).
 __global__ void __launch_bounds__(256)
 split_landmarks_kernel(const float4 *__restrict__ lm, uint2 *__restrict__ l0, uint2 *__restrict__ l1,
@@ -358,6 +586,13 @@ static bool sel_make_map(CUtensorMap *m, const void *base, uint64_t rows, int D)
            CUDA_SUCCESS;
 }
 
+// HSA_SELECT_TILES=multi keeps the multi-tile kernel for every length (tests
+// run both kernels on the same shapes).
+static bool force_multi_tile() {
+    const char *v = getenv("HSA_SELECT_TILES");
+    return v && strcmp(v, "multi") == 0;
+}
+
 template <int D, bool LM32, int KP>
 static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l0, const void *l1,
                                       cudaStream_t st) {
@@ -370,10 +605,18 @@ static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l
     } else {
         m1 = m0;
     }
+    dim3 grid((unsigned)((p.L + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
+    if (p.Nc <= SelHalfCfg<D, LM32>::N && !force_multi_tile()) {
+        // every chunk fits one score tile: qbar built per 64-column block, two blocks per SM
+        using H = SelHalfCfg<D, LM32>;
+        auto kern = select_tc_half_kernel<D, LM32, KP>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, H::SMEM);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, grid, dim3(kSelHalfThreads), (size_t)H::SMEM, st, m0, m1, p);
+    }
     auto kern = select_tc_kernel<D, LM32, KP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((p.L + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
     return launch_pdl(kern, grid, dim3(kSelTcThreads), (size_t)C::SMEM, st, m0, m1, p);
 }
 

@@ -117,6 +117,21 @@ def test_prefill_large_outputs(oracle_lib, seed):
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
 
 
+@pytest.mark.parametrize("tiles", ["one", "multi"])
+@pytest.mark.parametrize("lm_kind", ["bf16", "f32"])
+def test_prefill_selection_kernels(oracle_lib, monkeypatch, tiles, lm_kind):
+    # Up to 128 chunks the tensor-core selection builds qbar per 64-column
+    # block (two blocks per SM); HSA_SELECT_TILES=multi keeps the multi-tile
+    # kernel, so both kernels see the same shapes here.
+    if tiles == "multi":
+        monkeypatch.setenv("HSA_SELECT_TILES", "multi")
+    wl = small("bf16", B=2, L=64 * 33 + 17, topk=8, seed=41)
+    x = make_prefill_inputs(wl, DEV)
+    lm = x["lm"].float() if lm_kind == "f32" else None
+    rep, _ = prefill_parity(oracle_lib, wl, x, lm_override=lm)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+
+
 def test_prefill_explicit_scale(oracle_lib):
     wl = small("f32", B=1, L=300, H=4, Hkv=1, d=64)
     x = make_prefill_inputs(wl, DEV)
