@@ -227,10 +227,10 @@ def decode_noalloc(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.
 
 def set_stage_events(events) -> None:
     """Timing hook: record these torch.cuda.Event objects at the stage
-    boundaries of this thread's next calls (see hsa_set_stage_events); pass
-    an empty list to stop."""
-    arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event)
-                                                    for e in events])
+    boundaries of this thread's next calls (see hsa_set_stage_events); None
+    skips a boundary; pass an empty list to stop."""
+    arr = (ctypes.c_void_p * max(1, len(events)))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     _check(lib().hsa_set_stage_events(arr, len(events)), "hsa_set_stage_events")
 
 

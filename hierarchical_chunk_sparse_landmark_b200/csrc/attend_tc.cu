@@ -172,6 +172,12 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Ti
     }
 }
 
+// 16-byte store with an L2 cache policy (createpolicy) attached.
+__device__ __forceinline__ void st_policy(uint4 *p, uint64_t pol, uint4 v) {
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;"
+                 ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol) : "memory");
+}
+
 // Per-row view of a tile for the softmax and epilogue threads.
 struct RowJob {
     Tile tl;
@@ -507,6 +513,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int e = r / G, h = r % G;
         constexpr int NCH = D / 32;               // 32-column chunks of a row
+        // chunk outputs are evicted from L2 first: the Q / K / V rows the
+        // other tiles re-read stay (measured: 4 us of 160 on the train shape)
+        uint64_t pol;
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
         TileFeed feed;
         feed_init(feed, p, 0, 1, my_tiles, e);
         for (int64_t j = 0; j < my_tiles; ++j) {
@@ -534,11 +544,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 for (int u = 0; u < 2; ++u) {
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq)
-                        blk[((ch + u) * 4 + qq) * G + h] = make_uint4(
+                        st_policy(&blk[((ch + u) * 4 + qq) * G + h], pol, make_uint4(
                             pack_f16x2(o[u][8 * qq + 0], o[u][8 * qq + 1]),
                             pack_f16x2(o[u][8 * qq + 2], o[u][8 * qq + 3]),
                             pack_f16x2(o[u][8 * qq + 4], o[u][8 * qq + 5]),
-                            pack_f16x2(o[u][8 * qq + 6], o[u][8 * qq + 7]));
+                            pack_f16x2(o[u][8 * qq + 6], o[u][8 * qq + 7])));
                 }
             }
             tc::fence_before_sync();
