@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-decode] [--no-e2e] [--no-cpu-baseline]
+                    [--decode-workload NAME]
 
 One step = one full hsa_prefill call (landmarks when DHSA, selection, work
 list, in-chunk attention, fusion, own-chunk term) over one batch of the
@@ -312,7 +313,8 @@ def run_ours(args, dist, rank, world):
     del x, out
     torch.cuda.empty_cache()
     if args.decode:
-        res["decode_32m"] = bench_decode(args, dev, peaks, rank, dist)
+        key = "decode_32m" if args.decode_workload == "decode_32m_bf16" else "decode_" + args.decode_workload
+        res[key] = bench_decode(args, dev, peaks, rank, dist)
     if rank == 0 and world == 1 and args.cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(args, wl)
     return res
@@ -392,14 +394,15 @@ def bench_decode(args, dev, peaks, rank, dist):
 
     import hierarchical_chunk_sparse_landmark_b200 as hsa
     from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_decode_inputs
-    wl = WORKLOADS["decode_32m_bf16"].with_(seed=rank)
+    wl = WORKLOADS[args.decode_workload].with_(seed=rank)
     x = make_decode_inputs(wl, dev)
     out = torch.empty_like(x["q"])
     ws = hsa.workspace(hsa.decode_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S, wl.topk),
                        dev)
-    # The landmark stream alone (B*Hkv*Nc*d bf16 = 256 MiB) is larger than the
-    # 126 MB L2, so calls run back to back without a flush: nothing a call
-    # reads can still be in L2 from the previous one in any useful amount.
+    # The landmark stream alone (B*Hkv*Nc*d bf16 = 256 MiB for both decode
+    # workloads) is larger than the 126 MB L2, so calls run back to back without
+    # a flush: nothing a call reads can still be in L2 from the previous one in
+    # any useful amount.
     steps = max(5, args.steps)
     for _ in range(3):
         hsa.decode(x["q"], x["K"], x["V"], x["lm"], topk=wl.topk, out=out, ws=ws)
@@ -518,6 +521,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--decode-workload", default="decode_32m_bf16",
+                    help="decode workload of the decode line (decode_32m_bf16, batched_decode_bf16)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
