@@ -84,8 +84,8 @@ struct TcParams {
     const int32_t *entries;
     float *zf;                    // [B, L, H, topk] x (fusion logit, 1 / chunk row sum)
     float *own_f;                 // [B, L, H] add_own / own-chunk row sum
-    __half *part;                 // [B*L*Hkv*topk entries][D/8][G][8] chunk outputs
-    __half *own;                  // [B*L*Hkv rows (t, g)][D/8][G][8] own-chunk term
+    __half *part;                 // [B*L*Hkv*topk entries][D/16][G][16] chunk outputs
+    __half *own;                  // [B*L*Hkv rows (t, g)][D/16][G][16] own-chunk term
     unsigned *status;
     int64_t L, Nc;
     int H, Hkv, topk, S, add_own;
@@ -170,12 +170,6 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Ti
     } else {
         tl.t0 = d.z; tl.chunk = (int)(tl.t0 >> 6); tl.first = 0;     // S = 64 on this path
     }
-}
-
-// 16-byte store with an L2 cache policy (createpolicy) attached.
-__device__ __forceinline__ void st_policy(uint4 *p, uint64_t pol, uint4 v) {
-    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;"
-                 ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol) : "memory");
 }
 
 // Per-row view of a tile for the softmax and epilogue threads.
@@ -524,9 +518,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const int s = (int)(j & 1);
             const int64_t b = cur.b;
             const int g = cur.g;
-            // one contiguous G*D block per (t, g, k) (own term: per (t, g)), 16-byte
-            // pieces ordered [d/8][head]: the G heads' pieces of a column group
-            // are adjacent, so every store instruction writes whole lines
+            // one contiguous G*D block per (t, g, k) (own term: per (t, g)), 32-byte
+            // pieces ordered [d/16][head]: the G heads' pieces of a column group
+            // are adjacent, so every 256-bit store instruction writes whole lines
             const int64_t row = (b * L + cur.t) * Hkv + g;
             uint4 *blk = reinterpret_cast<uint4 *>(cur.tl.own ? p.own + row * (G * D)
                                                               : p.part + (row * topk + cur.k) * (G * D));
@@ -543,12 +537,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq)
-                        st_policy(&blk[((ch + u) * 4 + qq) * G + h], pol, make_uint4(
-                            pack_f16x2(o[u][8 * qq + 0], o[u][8 * qq + 1]),
-                            pack_f16x2(o[u][8 * qq + 2], o[u][8 * qq + 3]),
-                            pack_f16x2(o[u][8 * qq + 4], o[u][8 * qq + 5]),
-                            pack_f16x2(o[u][8 * qq + 6], o[u][8 * qq + 7])));
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t w8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) w8[i] = pack_f16x2(o[u][16 * hh + 2 * i], o[u][16 * hh + 2 * i + 1]);
+                        uint32_t *dst = reinterpret_cast<uint32_t *>(blk) + ((((ch + u) * 2 + hh) * G + h) * 8);
+                        asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;"
+                                     :: "l"(dst), "r"(w8[0]), "r"(w8[1]), "r"(w8[2]), "r"(w8[3]), "r"(w8[4]),
+                                        "r"(w8[5]), "r"(w8[6]), "r"(w8[7]), "l"(pol) : "memory");
+                    }
                 }
             }
             tc::fence_before_sync();
@@ -571,10 +568,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // One warp per (t, g): w = softmax over the token's selected chunks of the
 // logits (per head), O = f_own * own + sum_k w_k * f_k * partial_k, f = the
 // reciprocal row sums of the unnormalised chunk outputs.  A slot's partials
-// of the whole group are one contiguous block of 16-byte pieces ordered
-// [d/8][G] (G*d*2 bytes; the own term has the same layout), read with
-// coalesced 16-byte loads: lane l takes pieces l + 32 i, all of head l % G
-// (G divides 32), columns 8 * ((l + 32 i) / G) .. +8.  The own term's and
+// of the whole group are one contiguous block of 32-byte pieces ordered
+// [d/16][G] (G*d*2 bytes; the own term has the same layout), read with
+// coalesced 16-byte loads: lane l takes 16-byte pieces l + 32 i (halves of the
+// 32-byte pieces), all of head (l / 2) % G (G divides 16), columns
+// 16 * ((l + 32 i) / 2G) + 8 * (l % 2) .. +8.  The own term's and
 // the first slots' loads go out before the selection count is known.
 // Two blocks per SM where a lane's pieces allow (G*d <= 1024), else one: the
 // loads in flight per warp, not the warp count, keep HBM busy.
@@ -600,7 +598,7 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
     const int64_t srow = groups - 1 - lin;           // srow = (b*L + t)*Hkv + g
     const int64_t bt = srow / Hkv;
     const int g = (int)(srow % Hkv);
-    const int h = lane % G;
+    const int h = (lane >> 1) % G;
     const int64_t hrow = bt * H + (int64_t)g * G + h;
     const uint4 *pb = reinterpret_cast<const uint4 *>(part + srow * topk * (int64_t)(G * D));
     const uint4 *ob = reinterpret_cast<const uint4 *>(own + srow * (int64_t)(G * D));
@@ -627,7 +625,7 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
 #pragma unroll
     for (int k = 0; k < KP; ++k) den += k < nsel ? __expf(zx[k] - m) : 0.f;
     const float inv = nsel ? 1.f / den : 0.f;
-    if (w_out && lane < G)
+    if (w_out && lane < 2 * G && (lane & 1) == 0)
         for (int k = 0; k < topk; ++k)
             w_out[hrow * topk + k] = k < nsel ? __expf(zh[k].x - m) * inv : 0.f;
     float acc[NP][8];
@@ -679,7 +677,8 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
     }
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
-        const int c8 = (lane + 32 * i) / G;
+        const int pc = lane + 32 * i;
+        const int c8 = (pc >> 1) / G * 2 + (pc & 1);
         *reinterpret_cast<uint4 *>(O + hrow * D + c8 * 8) =
             make_uint4(pack_bf16x2(acc[i][0], acc[i][1]), pack_bf16x2(acc[i][2], acc[i][3]),
                        pack_bf16x2(acc[i][4], acc[i][5]), pack_bf16x2(acc[i][6], acc[i][7]));
