@@ -52,7 +52,8 @@ struct SelCfg {
     static constexpr int STAGES = 2;
     static constexpr int B_STAGE = LP * B_PART;
     static constexpr int BAR_OFF = QP * A_PART + STAGES * B_STAGE;
-    static constexpr int SMEM = 1024 + BAR_OFF + 256;
+    static constexpr int STAGE_OFF = BAR_OFF + 256;      // top-K score rows [32][128] fp32
+    static constexpr int SMEM = 1024 + STAGE_OFF + 32 * 128 * 4;
     static constexpr uint32_t TMEM_COLS = 2 * N;
 };
 
@@ -82,6 +83,45 @@ __device__ __forceinline__ bool sel_wait(uint64_t *bar, uint32_t parity, volatil
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// One 32-column block of a token's scores (chunks c0 .. c0+31, visible below
+// nvis) into its sorted list v of KP 64-bit keys (score bits, ~index).  The
+// lane first marks its candidates (score >= its current K-th score), then
+// takes them one per loop trip from its own 32-float row of `stage` (shared
+// memory, column-major so the rows of a warp's lanes share no bank): the warp
+// runs as many trips as its busiest lane needs, instead of the insertion at
+// every column where any lane has a candidate.  Candidates are taken in column
+// order and the keys order (score, then lower index) totally, so the result
+// does not depend on the order.
+template <int KP>
+__device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, int64_t nvis, float scale,
+                                           uint64_t (&v)[KP], float &tf, float *stage, int r) {
+    uint32_t mask = 0;
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+        if (c0 + c < nvis && scale * sc[c] >= tf) mask |= 1u << c;
+    if (mask) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) stage[c * 128 + r] = sc[c];
+    }
+    while (mask) {
+        const int c = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const float sv = scale * stage[c * 128 + r];
+        if (sv >= tf) {
+            uint64_t x = make_key(sv, c0 + c);
+            if (x > v[KP - 1]) {
+#pragma unroll
+                for (int i = 0; i < KP; ++i) {
+                    const uint64_t hi = v[i] > x ? v[i] : x;
+                    x = v[i] > x ? x : v[i];
+                    v[i] = hi;
+                }
+                tf = key_score(v[KP - 1]);
+            }
+        }
+    }
 }
 
 template <int D, bool LM32, int KP>
@@ -271,23 +311,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
                 float sc[32];
                 tc::tmem_ld32(tmem + s * C::N + cb * 32 + lane_off, sc);
                 tc::tmem_wait_ld();
-                const int64_t c0 = (int64_t)n * C::N + cb * 32;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float sv = p.scale * sc[c];
-                    if (c0 + c < nvis && sv >= tf) {
-                        uint64_t x = make_key(sv, c0 + c);
-                        if (x > v[KP - 1]) {
-#pragma unroll
-                            for (int i = 0; i < KP; ++i) {
-                                const uint64_t hi = v[i] > x ? v[i] : x;
-                                x = v[i] > x ? x : v[i];
-                                v[i] = hi;
-                            }
-                            tf = key_score(v[KP - 1]);
-                        }
-                    }
-                }
+                topk_block<KP>(sc, (int64_t)n * C::N + cb * 32, nvis, p.scale, v, tf,
+                               (float *)(smem + C::STAGE_OFF), r);
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&tfree[s]);
@@ -330,6 +355,9 @@ struct SelHalfCfg {
     static constexpr int BAR_OFF = QP * A_PART + LP * B_PART;
     static constexpr int SMEM = 1024 + BAR_OFF + 256;
     static constexpr uint32_t TMEM_COLS = N;
+    // the top-K score rows ([32][128] fp32) reuse the qbar buffer: the top-K
+    // starts once the last score MMA, its last reader, has completed
+    static_assert(QP * A_PART >= 32 * 128 * 4, "top-K rows must fit the qbar buffer");
 };
 constexpr int kSelHalfThreads = 256;                // 8 warps: all build qbar; 2-5 also top-K
 
@@ -496,22 +524,7 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
                 float sc[32];
                 tc::tmem_ld32(tmem + cb * 32 + lane_off, sc);
                 tc::tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float sv = p.scale * sc[c];
-                    if (cb * 32 + c < nvis && sv >= tf) {
-                        uint64_t x = make_key(sv, cb * 32 + c);
-                        if (x > v[KP - 1]) {
-#pragma unroll
-                            for (int i = 0; i < KP; ++i) {
-                                const uint64_t hi = v[i] > x ? v[i] : x;
-                                x = v[i] > x ? x : v[i];
-                                v[i] = hi;
-                            }
-                            tf = key_score(v[KP - 1]);
-                        }
-                    }
-                }
+                topk_block<KP>(sc, (int64_t)cb * 32, nvis, p.scale, v, tf, (float *)sA, r);
             }
             tc::fence_before_sync();
             if (t < L) {
