@@ -79,11 +79,22 @@ bool tc_shape_ok(int B, int H, int Hkv, int64_t L, int d, int topk) {
     return true;
 }
 
-// Token window of the work lists: one window per (b, g) -- the tiles carry no
-// dependencies, so larger windows only make the chunk buckets fuller.
+// Token window of the work lists.  A window's tiles re-read each of its
+// tokens' query rows once per selected chunk, spread over the window's whole
+// run, so the window's query rows (W * G * d * 2 bytes) should stay in L2:
+// windows of at most ~16 MB of them (8192 tokens at G = 8, d = 128), else one
+// window per (b, g) -- bigger windows fill the chunk buckets better (on the
+// L = 131072 prefill: 8192-token windows 3.01 ms, 16384 3.06, 32768 3.18,
+// one window 3.55).  The
+// window is a multiple of 256 tokens (the work-list blocks' size);
+// HSA_TC_WINDOW overrides it for experiments.
 int64_t tc_window(int B, int H, int Hkv, int64_t L, int d, int topk, int64_t max_windows) {
-    (void)H; (void)d; (void)topk;
+    (void)topk;
     int64_t W = (L + 255) / 256 * 256;
+    const int64_t q_bytes_per_token = (int64_t)(H / Hkv) * d * 2;
+    int64_t cap = (int64_t(16) << 20) / q_bytes_per_token / 256 * 256;
+    if (const char *v = getenv("HSA_TC_WINDOW")) cap = atoll(v) / 256 * 256;
+    if (cap >= 256 && W > cap) W = cap;
     while ((int64_t)B * Hkv * ((L + W - 1) / W) > max_windows) W *= 2;
     return W;
 }
