@@ -132,6 +132,18 @@ def test_prefill_selection_kernels(oracle_lib, monkeypatch, tiles, lm_kind):
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
 
 
+@pytest.mark.parametrize("H,Hkv", [(8, 1), (16, 1)])
+def test_prefill_several_windows(oracle_lib, monkeypatch, H, Hkv):
+    # Long sequences split the work lists into token windows (a window's query
+    # rows should stay in L2); 512-token windows force that path on a small
+    # shape: several windows per (b, g), ragged last one.
+    monkeypatch.setenv("HSA_TC_WINDOW", "512")
+    wl = small("bf16", B=2, L=64 * 37 + 29, H=H, Hkv=Hkv, topk=8, seed=77)
+    x = make_prefill_inputs(wl, DEV)
+    rep, _ = prefill_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+
+
 def test_prefill_explicit_scale(oracle_lib):
     wl = small("f32", B=1, L=300, H=4, Hkv=1, d=64)
     x = make_prefill_inputs(wl, DEV)
