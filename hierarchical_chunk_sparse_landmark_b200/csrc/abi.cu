@@ -76,6 +76,7 @@ bool tc_shape_ok(int B, int H, int Hkv, int64_t L, int d, int topk) {
     if (L >= (int64_t(1) << 26)) return false;                      // entry code t*32+k
     if ((int64_t)B * L * H >= INT32_MAX) return false;              // TMA row of Q
     if ((int64_t)B * Hkv * L * topk >= INT32_MAX) return false;     // entry index
+    if ((int64_t)B * Hkv * Hkv >= (int64_t(1) << 32)) return false; // (b, g) split by a multiply
     return true;
 }
 

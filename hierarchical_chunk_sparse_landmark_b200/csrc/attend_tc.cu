@@ -89,6 +89,7 @@ struct TcParams {
     unsigned *status;
     int64_t L, Nc;
     int H, Hkv, topk, S, add_own;
+    uint64_t hkv_mul;             // floor(2^32 / Hkv) + 1: bg / Hkv = (bg * hkv_mul) >> 32
     int lm_rows;                  // landmark rows per chunk: 1 (bf16) or 2 (bf16 high, low of fp32)
     int q3d;                      // Q map is the 3-D (cols, rows, d-half) view
     float scale, scale_log2e;
@@ -155,6 +156,13 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar) {
 // consumer's release of use u-1.
 __device__ __forceinline__ uint32_t reuse_parity(int64_t u) { return (uint32_t)((u + 1) & 1); }
 
+// bg / Hkv by a multiply-high instead of a runtime divide (a long dependent
+// sequence in every role's per-tile decode): exact while bg * Hkv < 2^32,
+// which the host checks.
+__device__ __forceinline__ int div_hkv(const TcParams &p, int64_t bg) {
+    return (int)(((uint64_t)bg * p.hkv_mul) >> 32);
+}
+
 // A queue position decoded into one tile.
 struct Tile {
     int64_t bg, first, t0;   // first entry (retrieved) or first token (own)
@@ -213,7 +221,7 @@ __device__ __forceinline__ RowJob feed_next(TileFeed &f, const TcParams &p, int6
     rj.valid = e < rj.tl.n;
     rj.t = f.c1 >> 5;
     rj.k = f.c1 & 31;
-    rj.b = (int)rj.tl.bg / p.Hkv;                  // bg < 2^31 (checked on the host)
+    rj.b = div_hkv(p, rj.tl.bg);
     rj.g = (int)rj.tl.bg - rj.b * p.Hkv;
     f.d1 = f.d2; f.d2 = d3; f.c1 = c2;
     return rj;
@@ -306,7 +314,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             Tile d0;
             decode_tile(p, d_cur, d0);
             const int32_t c0 = lane < d0.n ? (d0.own ? (int32_t)((d0.t0 + lane) * 32) : code_cur) : 0;
-            const int bq = (int)d0.bg / Hkv;            // bg < 2^31 (checked on the host)
+            const int bq = div_hkv(p, d0.bg);
             const int gq = (int)d0.bg - bq * Hkv;
 
             int ok = 1;
@@ -374,33 +382,41 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (lane == 0) {
             constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, C::NS, false);
             constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
+            // Descriptors are built once for slot 0; a slot or a K step moves
+            // only the start-address field (bytes / 16; every operand sits below
+            // 256 KB, so the 14-bit field never carries), so an MMA costs the
+            // issuing thread one add per operand.
+            const uint64_t ad0 = p.q3d ? tc::sdesc_sw128(tc::smem_u32(sQ(0)), 16, C::KB * G * 128)
+                                       : tc::sdesc_sw128(tc::smem_u32(sQ(0)), 16, 1024);
+            const uint32_t a_kb = p.q3d ? (uint32_t)(G * 128 / 16) : (uint32_t)(16384 / 16);
+            const uint64_t bd0 = tc::sdesc_sw128(tc::smem_u32(sK(0)), 16, 1024);
+            const uint64_t vd0 = tc::sdesc_sw128(tc::smem_u32(sV(0)), 8192, 1024);
             auto issue_pv = [&](int64_t i) {
                 const int s = (int)(i & 1), v = (int)(i % C::NVP);
+                const uint64_t vd = vd0 + (uint64_t)(v * (C::VP_STAGE / 16));
+                const uint32_t pa = tmem + s * C::S_COL + C::P_OFF, od = tmem + C::O_COL + s * D;
                 tc::fence_after_sync();
+                // A = P from TMEM: 16 keys = 8 packed columns per step
+                tc::mma_bf16_ts(od, pa, vd, IDESC_O, 0u);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    // A = P from TMEM: 16 keys = 8 packed columns per step
-                    const uint32_t pa = tmem + s * C::S_COL + C::P_OFF + kk * 8;
-                    const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sV(v) + kk * 2048), 8192, 1024);
-                    tc::mma_bf16_ts(tmem + C::O_COL + s * D, pa, bd, IDESC_O, kk ? 1u : 0u);
-                }
+                for (int kk = 1; kk < 4; ++kk)
+                    tc::mma_bf16_ts(od, pa + kk * 8, vd + (uint64_t)(kk * 2048 / 16), IDESC_O, 1u);
                 tc::mma_commit(&ofull[s]);
                 tc::mma_commit(&vp_empty[v]);
                 tc::mma_commit(&pempty[s]);
             };
             auto issue_s = [&](int64_t j) {
                 const int s = (int)(j & 1), q = (int)(j % C::NQK);
+                const uint64_t ad = ad0 + (uint64_t)(q * (C::QK_STAGE / 16));
+                const uint64_t bd = bd0 + (uint64_t)(q * (C::QK_STAGE / 16));
+                const uint32_t sd = tmem + s * C::S_COL;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = p.q3d
-                            ? tc::sdesc_sw128(tc::smem_u32(sQ(q) + kb * (G * 128) + kk * 32), 16, C::KB * G * 128)
-                            : tc::sdesc_sw128(tc::smem_u32(sQ(q) + kb * 16384 + kk * 32), 16, 1024);
-                        const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(sK(q) + kb * C::KBLK + kk * 32), 16, 1024);
-                        tc::mma_bf16(tmem + s * C::S_COL, ad, bd, IDESC_S, (kb | kk) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(sd, ad + (uint64_t)(kb * a_kb + kk * 2),
+                                     bd + (uint64_t)(kb * (C::KBLK / 16) + kk * 2), IDESC_S, (kb | kk) ? 1u : 0u);
                 tc::mma_commit(&sfull[s]);
                 tc::mma_commit(&qk_empty[q]);
             };
@@ -773,6 +789,7 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     p.part = a.part; p.own = a.own; p.status = a.status;
     p.L = a.L; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
+    p.hkv_mul = (uint64_t)(0x100000000ull / (uint64_t)a.Hkv) + 1ull;
     p.lm_rows = a.lm_bf16 ? 1 : 2;
     p.q3d = q3d ? 1 : 0;
     p.scale = a.scale;
