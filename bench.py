@@ -166,16 +166,37 @@ def kernel_source_hash(files) -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str, src_files) -> float | None:
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
-    the current source of that kernel (else None)."""
+def measured_traffic(kernel: str, src_files, key: str = "dram_bytes_per_launch") -> float | None:
+    """Per-launch DRAM bytes (`key`: read + write, or the write part alone)
+    from the committed ncu summary, if it was taken on the current source of
+    that kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(kernel)
     if not d or d.get("source_hash") != kernel_source_hash(src_files):
         return None
-    return d.get("dram_bytes_per_launch")
+    return d.get(key)
+
+
+def hbm_write_gbs(dev, gib: int = 1, reps: int = 5) -> float:
+    """Write-only HBM bandwidth of this GPU: a 1 GiB fill (8x L2), CUDA events.
+    A kernel whose DRAM traffic is mostly writes is bound by this, not by the
+    read + write copy bandwidth of the peaks file."""
+    import torch
+    buf = torch.empty(gib << 30, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        buf.fill_(1)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        buf.fill_(1)
+    b.record()
+    torch.cuda.synchronize()
+    gbs = reps * buf.numel() / (a.elapsed_time(b) / 1e3) / 1e9
+    del buf
+    torch.cuda.empty_cache()
+    return gbs
 
 
 # ----------------------------------------------------------------------------- dist
@@ -279,12 +300,25 @@ def run_ours(args, dist, rank, world):
     attn_files = ["hierarchical_chunk_sparse_landmark_b200/csrc/" +
                   ("attend_tc.cu" if tc_path else "attend_simt.cu")]
     kname = "attend_tc_kernel" if tc_path else "attend_simt_kernel"
+    kfile = attn_files[0].rsplit("/", 1)[1][:-3]
     roofline = {"kernel": kname, "bound": "tensor", "achieved": round(attn_tf, 3),
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 5),
-                "traffic": measured_traffic(attn_files[0].rsplit("/", 1)[1][:-3], attn_files),
+                "traffic": measured_traffic(kfile, attn_files),
                 "peak_source": peaks["source"] + " bf16 burst",
                 "algorithmic_flops_per_launch": flops["attention_kernel"],
                 "ms_per_launch": round(attn_s * 1e3, 4)}
+    # What the kernel actually runs into: the DRAM write-back of its chunk
+    # outputs (design traffic, not algorithmic), against the write-only HBM
+    # bandwidth measured here.
+    wbytes = measured_traffic(kfile, attn_files, "dram_write_bytes_per_launch")
+    if tc_path and wbytes:
+        wpeak = hbm_write_gbs(dev)
+        wach = wbytes / attn_s / 1e9
+        roofline["dram_write"] = {"bytes_per_launch": wbytes, "achieved": round(wach, 1),
+                                  "peak": round(wpeak, 1), "unit": "GB/s",
+                                  "frac": round(wach / wpeak, 4),
+                                  "peak_source": "write-only HBM bandwidth measured in this run "
+                                                 "(1 GiB fill)"}
 
     res = {
         "metric": "HSA prefill TFLOP/s (train-shape workload) + 32M-ctx decode tokens/s",
