@@ -21,10 +21,11 @@
 // swizzled, K-major); then
 //   warp 0      producer  (TMA of landmark tiles, two stages)
 //   warp 1      MMA issuer (one score tile per landmark tile, two TMEM buffers)
-//   warps 2-5   top-K     (thread = token = TMEM lane: causal mask, a sorted
+//   warps 2-9   top-K     (thread = token = TMEM lane: causal mask, a sorted
 //                          register list of 64-bit keys, insertion only past
-//                          the current K-th key)
-// (warps 6-11 only help build qbar; the first two landmark tiles are requested
+//                          the current K-th key; two groups of four warps over
+//                          alternate 32-column blocks, lists merged at the end)
+// (warps 10-11 only help build qbar; the first two landmark tiles are requested
 // before that, so their loads overlap it.)
 // select_tc_half_kernel takes the case where every chunk fits one score tile
 // (Nc <= 128): qbar built per 64-column block of d into one buffer, two blocks
@@ -52,8 +53,9 @@ struct SelCfg {
     static constexpr int STAGES = 2;
     static constexpr int B_STAGE = LP * B_PART;
     static constexpr int BAR_OFF = QP * A_PART + STAGES * B_STAGE;
-    static constexpr int STAGE_OFF = BAR_OFF + 256;      // top-K score rows [32][128] fp32
-    static constexpr int SMEM = 1024 + STAGE_OFF + 32 * 128 * 4;
+    static constexpr int STAGE_OFF = BAR_OFF + 256;      // top-K score rows [2 groups][32][128] fp32
+    static constexpr int SMEM = 1024 + STAGE_OFF + 2 * 32 * 128 * 4;
+    static_assert(STAGES * B_STAGE >= 32 * 128 * 8, "top-K lists must fit the landmark stages");
     static constexpr uint32_t TMEM_COLS = 2 * N;
 };
 
@@ -124,6 +126,27 @@ __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, in
     }
 }
 
+// The top-K runs in two groups of four warps (thread = token = TMEM lane),
+// each over alternate 32-column blocks of the scores into its own sorted list;
+// group 1 leaves its list in shared memory (`lists`, [KP][128] keys) and group
+// 0 folds it into its own.  Keys are distinct (they hold the chunk index), so
+// the result is the K largest keys of the token whatever the split.
+template <int KP>
+__device__ __forceinline__ void merge_keys(uint64_t (&v)[KP], const uint64_t *lists, int r) {
+#pragma unroll
+    for (int j = 0; j < KP; ++j) {
+        uint64_t x = lists[j * 128 + r];
+        if (x > v[KP - 1]) {
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                const uint64_t hi = v[i] > x ? v[i] : x;
+                x = v[i] > x ? x : v[i];
+                v[i] = hi;
+            }
+        }
+    }
+}
+
 template <int D, bool LM32, int KP>
 __global__ void __launch_bounds__(kSelTcThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant__ CUtensorMap tmL1,
@@ -161,7 +184,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             tc::mbar_init(&full[s], 1);
             tc::mbar_init(&empty[s], 1);
             tc::mbar_init(&tfull[s], 1);
-            tc::mbar_init(&tfree[s], 128);
+            tc::mbar_init(&tfree[s], 256);     // one arrive per top-K thread
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -263,35 +286,40 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             constexpr uint32_t IDESC = tc::idesc_bf16_f32(128, C::N, false);
             // (qbar part, landmark part) of every product term
             constexpr int NPROD = 3;
-            const int pa[NPROD] = {0, 1, LM32 ? 0 : 2};
-            const int pl[NPROD] = {0, 0, LM32 ? 1 : 0};
+            constexpr int pa[NPROD] = {0, 1, LM32 ? 0 : 2};
+            constexpr int pl[NPROD] = {0, 0, LM32 ? 1 : 0};
+            // descriptors built once; an operand offset moves only the start-
+            // address field (bytes / 16, shared memory below 256 KB: no carry)
+            const uint64_t ad0 = tc::sdesc_sw128(tc::smem_u32(sA), 16, 1024);
+            const uint64_t bd0 = tc::sdesc_sw128(tc::smem_u32(sB(0)), 16, 1024);
             for (int n = 0; n < ntiles; ++n) {
                 const int s = n & 1;
                 if (!sel_wait(&full[s], (uint32_t)((n >> 1) & 1), s_abort)) break;
                 if (n >= 2 && !sel_wait(&tfree[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
                 tc::fence_after_sync();
-                uint32_t acc = 0;
+                const uint64_t bds = bd0 + (uint64_t)(s * (C::B_STAGE / 16));
+                const uint32_t dt = tmem + s * C::N;
 #pragma unroll
                 for (int pr = 0; pr < NPROD; ++pr)
 #pragma unroll
                     for (int kb = 0; kb < C::KB; ++kb)
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = tc::sdesc_sw128(
-                                tc::smem_u32(sA + pa[pr] * C::A_PART + kb * (C::M * 128) + kk * 32), 16, 1024);
-                            const uint64_t bd = tc::sdesc_sw128(
-                                tc::smem_u32(sB(s) + pl[pr] * C::B_PART + kb * (C::N * 128) + kk * 32), 16, 1024);
-                            tc::mma_bf16(tmem + s * C::N, ad, bd, IDESC, acc);
-                            acc = 1;
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_bf16(dt, ad0 + (uint64_t)((pa[pr] * C::A_PART + kb * (C::M * 128) + kk * 32) / 16),
+                                         bds + (uint64_t)((pl[pr] * C::B_PART + kb * (C::N * 128) + kk * 32) / 16),
+                                         IDESC, (pr | kb | kk) ? 1u : 0u);
                 tc::mma_commit(&tfull[s]);
                 tc::mma_commit(&empty[s]);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ------------------------------------------------------------ top-K
+        // group 0 (warps 2-5) takes the 32-column blocks 0 and 2 of every
+        // score tile, group 1 (warps 6-9) blocks 1 and 3 (see merge_keys)
         const int q4 = warp & 3;
+        const int hg = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;
+        float *stage = (float *)(smem + C::STAGE_OFF) + hg * (32 * 128);
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int64_t t = t0 + r;
         const int64_t nvis = t < L ? t / p.S : 0;
@@ -307,17 +335,24 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             const int64_t vis = nvis_max - (int64_t)n * C::N;
             const int ncb = vis >= C::N ? C::N / 32 : (int)((vis + 31) / 32);
 #pragma unroll 1
-            for (int cb = 0; cb < ncb; ++cb) {
+            for (int cb = hg; cb < ncb; cb += 2) {
                 float sc[32];
                 tc::tmem_ld32(tmem + s * C::N + cb * 32 + lane_off, sc);
                 tc::tmem_wait_ld();
-                topk_block<KP>(sc, (int64_t)n * C::N + cb * 32, nvis, p.scale, v, tf,
-                               (float *)(smem + C::STAGE_OFF), r);
+                topk_block<KP>(sc, (int64_t)n * C::N + cb * 32, nvis, p.scale, v, tf, stage, r);
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&tfree[s]);
         }
-        if (t < L) {
+        // the landmark stages are dead once the last tile's scores are in TMEM
+        uint64_t *lists = reinterpret_cast<uint64_t *>(sB(0));
+        if (hg == 1) {
+#pragma unroll
+            for (int k = 0; k < KP; ++k) lists[k * 128 + r] = v[k];
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");     // the two top-K groups
+        if (hg == 0 && t < L) {
+            merge_keys<KP>(v, lists, r);
             int32_t *dst = p.idx + ((b * L + t) * p.Hkv + g) * p.topk;
 #pragma unroll
             for (int k = 0; k < KP; ++k)

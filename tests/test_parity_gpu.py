@@ -132,6 +132,36 @@ def test_prefill_selection_kernels(oracle_lib, monkeypatch, tiles, lm_kind):
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
 
 
+@pytest.mark.parametrize("topk", [3, 17, 32])
+@pytest.mark.parametrize("tiles", ["one", "multi"])
+def test_prefill_tc_selection_topk(oracle_lib, monkeypatch, topk, tiles):
+    # The tensor-core selection (G = 8) at each compiled list length (8, 16 and
+    # 32 keys) in both kernels (the multi-tile kernel splits the top-K between
+    # two warp groups over alternate 32-chunk column blocks and merges their
+    # lists per token).
+    if tiles == "multi":
+        monkeypatch.setenv("HSA_SELECT_TILES", "multi")
+    wl = small("bf16", B=1, L=64 * 40 + 5, H=16, Hkv=2, topk=topk, seed=100 + topk)
+    x = make_prefill_inputs(wl, DEV)
+    rep, _ = prefill_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+
+
+@pytest.mark.parametrize("topk", [8, 32])
+def test_prefill_tc_selection_many_tiles(oracle_lib, topk):
+    # 300 chunks: three score tiles of 128 chunks, the last one ragged (two of
+    # its four 32-column blocks), so both top-K groups see full, partial and
+    # empty blocks.  Sampled rows: random ones, the first tokens of chunks next
+    # to the tile edges, and the tail.
+    wl = small("bf16", B=1, L=64 * 300 + 5, H=16, Hkv=2, topk=topk, seed=200 + topk)
+    x = make_prefill_inputs(wl, DEV)
+    rng = np.random.default_rng(topk)
+    edges = np.concatenate([np.arange(c * 64 - 2, c * 64 + 3) for c in (1, 2, 33, 128, 129, 256, 257, 299)])
+    rows = np.unique(np.concatenate([rng.integers(0, wl.L, 400), edges, np.arange(wl.L - 70, wl.L)]))
+    rep, _ = prefill_parity(oracle_lib, wl, x, rows=rows)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+
+
 @pytest.mark.parametrize("H,Hkv", [(8, 1), (16, 1)])
 def test_prefill_several_windows(oracle_lib, monkeypatch, H, Hkv):
     # Long sequences split the work lists into token windows (a window's query
