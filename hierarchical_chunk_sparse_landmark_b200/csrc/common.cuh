@@ -142,29 +142,6 @@ struct WarpTopK {
     }
 };
 
-// Top-K of the keys a warp holds (M per lane, 0 = none; keys are distinct
-// unless 0): K rounds of a warp-wide maximum, the owner of each winner drops
-// it.  Returns in lane k < topk the k-th best key (0 when fewer exist).
-__device__ __forceinline__ uint64_t max_u64(uint64_t a, uint64_t b) { return a > b ? a : b; }
-template <int M>
-__device__ __forceinline__ uint64_t warp_select_topk(uint64_t (&x)[M], int topk) {
-    const int lane = threadIdx.x & 31;
-    uint64_t out = 0ull;
-    for (int r = 0; r < topk; ++r) {
-        uint64_t best = x[0];
-#pragma unroll
-        for (int m = 1; m < M; ++m) best = max_u64(best, x[m]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) best = max_u64(best, __shfl_xor_sync(0xffffffffu, best, o));
-        if (best == 0ull) break;                  // no keys left (warp-uniform)
-        if (lane == r) out = best;
-#pragma unroll
-        for (int m = 0; m < M; ++m)
-            if (x[m] == best) x[m] = 0ull;
-    }
-    return out;
-}
-
 // Sorted-list merging.  A warp register holds 32/KP lists (KP a power of two):
 // lanes s*KP .. s*KP + KP - 1 hold list s in descending order (0 = empty).
 // merge_lists returns, in the same layout, the KP best keys of the union of
