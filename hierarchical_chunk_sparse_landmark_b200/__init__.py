@@ -7,7 +7,9 @@ binding (PyTorch supplies device memory and streams) plus the seeded synthetic
 workloads used by the tests and the benchmark.
 """
 from ._binding import (HSAError, check, last_call_launches, decode, decode_workspace_size, landmarks, lib, prefill,
-                       prefill_workspace_size, set_stage_events, status_string, workspace)
+                       prefill_workspace_size, selftest_wait_expiry, set_stage_events, status_string,
+                       workspace)
 
 __all__ = ["HSAError", "check", "last_call_launches", "decode", "decode_workspace_size", "landmarks", "lib", "prefill",
-           "prefill_workspace_size", "set_stage_events", "status_string", "workspace"]
+           "prefill_workspace_size", "selftest_wait_expiry", "set_stage_events", "status_string",
+           "workspace"]

@@ -23,7 +23,7 @@ HSA_F32, HSA_BF16 = 0, 1
 EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_decode_workspace_size", "hsa_decode", "hsa_check", "hsa_status_string",
             "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches",
-            "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch")
+            "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry")
 
 
 class HSAError(RuntimeError):
@@ -49,6 +49,7 @@ def _declare(lib):
     lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
                                vp, vp, vp, sz, vp]
     lib.hsa_check.argtypes = [vp, vp]
+    lib.hsa_selftest_wait_expiry.argtypes = [vp, sz, i64, vp]
     lib.hsa_decode_noalloc.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
                                        i32, f32, vp, vp, vp]
     lib.hsa_decode_noalloc_max_scratch.argtypes = []
@@ -57,7 +58,8 @@ def _declare(lib):
     lib.hsa_status_string.argtypes = [i32]
     lib.hsa_status_string.restype = ctypes.c_char_p
     for n in ("hsa_landmarks", "hsa_prefill", "hsa_decode", "hsa_check", "hsa_version",
-              "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc"):
+              "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
+              "hsa_selftest_wait_expiry"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -237,6 +239,15 @@ def set_stage_events(events) -> None:
 def last_call_launches() -> int:
     """Kernels launched by this thread's most recent library call."""
     return int(lib().hsa_last_call_launches())
+
+
+def selftest_wait_expiry(ws, budget_cycles: int = 2_000_000):
+    """Run the library's bounded-wait failure path once: a device wait that
+    nothing completes gives up after `budget_cycles` and flags the status word
+    of `ws`; the following check(ws) raises HSAError with status HSA_ERR_TIMEOUT."""
+    _dev(ws, "ws")
+    _check(lib().hsa_selftest_wait_expiry(_ptr(ws), ws.numel() * ws.element_size(), int(budget_cycles),
+                                          _stream(ws.device)), "hsa_selftest_wait_expiry")
 
 
 def check(ws=None, device=None):

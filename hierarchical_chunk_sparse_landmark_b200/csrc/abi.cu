@@ -33,6 +33,7 @@ cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int top
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
                           int64_t *seg_start, int4 *tiles, cudaStream_t st);
+cudaError_t launch_selftest_wait(unsigned *status, long long budget, cudaStream_t st);
 }  // namespace hsa
 
 using namespace hsa;
@@ -405,6 +406,14 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
     t_launches = r == HSA_OK ? 2 : 0;
     stage_mark(1, st);
     return r;
+}
+
+hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t budget_cycles,
+                                      void *stream) {
+    if (!workspace || ws_bytes < 16 || ((uintptr_t)workspace & 15) != 0) return HSA_ERR_INVALID_ARG;
+    if (budget_cycles < 1 || budget_cycles > 4000000000LL) return HSA_ERR_INVALID_ARG;
+    return hsa::launch_selftest_wait((unsigned *)workspace, (long long)budget_cycles,
+                                     (cudaStream_t)stream) == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
 }
 
 hsa_status_t hsa_check(void *workspace, void *stream) {

@@ -175,6 +175,22 @@ hsa_status_t hsa_decode_noalloc(const void *q, const void *Kc, const void *Vc, h
 size_t hsa_decode_noalloc_max_scratch(void);
 
 /*
+ * hsa_selftest_wait_expiry -- exercises the failure path of the kernels'
+ * bounded waits (see hsa_check): launches one block whose mbarrier wait can
+ * never complete, because nothing arrives on it; after `budget_cycles` SM
+ * cycles the block gives up, sets the timeout flag in the status word at the
+ * head of `workspace` and exits, as every kernel of the library does when one
+ * of its waits runs out.  A following hsa_check(workspace, stream) returns
+ * HSA_ERR_TIMEOUT and clears the flag; the CUDA context stays usable.
+ *   workspace     any workspace of this library (>= 16 bytes), zero-filled
+ *   budget_cycles 1 .. 4e9 (2e6 is about 1 ms)
+ * Returns HSA_ERR_INVALID_ARG for a bad argument, HSA_ERR_CUDA if the launch
+ * fails, else HSA_OK (the expiry itself is reported by hsa_check).
+ */
+hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t budget_cycles,
+                                      void *stream);
+
+/*
  * hsa_check -- synchronises `stream`, then reads the status word at the head
  * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
  * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up (and clears

@@ -131,3 +131,12 @@ def test_product_path_has_no_cpu_tensors_path():
     import torch
     with pytest.raises(ValueError):
         hsa.prefill(torch.zeros(1, 64, 2, 64), torch.zeros(1, 1, 64, 64), torch.zeros(1, 1, 64, 64))
+
+
+def test_selftest_rejects_before_launch():
+    lib = B.lib()
+    assert lib.hsa_selftest_wait_expiry(None, 4096, 1000, None) == B.HSA_ERR_INVALID_ARG
+    assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 8, 1000, None) == B.HSA_ERR_INVALID_ARG
+    assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A + 4), 4096, 1000, None) == B.HSA_ERR_INVALID_ARG
+    assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 4096, 0, None) == B.HSA_ERR_INVALID_ARG
+    assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 4096, 5_000_000_000, None) == B.HSA_ERR_INVALID_ARG

@@ -174,6 +174,24 @@ def test_prefill_several_windows(oracle_lib, monkeypatch, H, Hkv):
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
 
 
+def test_bounded_wait_expiry_is_reported_and_context_survives(oracle_lib):
+    # The failure path of every bounded device wait, made to run out on
+    # purpose (a wait that nothing completes, ~1 ms): the status word is
+    # flagged, hsa.check reports the timeout once, and the same context then
+    # runs the prefill path with parity.
+    from hierarchical_chunk_sparse_landmark_b200 import _binding as B
+    ws = torch.zeros(4096, dtype=torch.uint8, device=DEV)
+    hsa.selftest_wait_expiry(ws, budget_cycles=2_000_000)
+    with pytest.raises(hsa.HSAError) as e:
+        hsa.check(ws)
+    assert e.value.status == B.HSA_ERR_TIMEOUT
+    hsa.check(ws)                       # the flag was cleared
+    wl = small("bf16", B=1, L=64 * 12 + 7, H=16, Hkv=2, topk=4, seed=9)
+    x = make_prefill_inputs(wl, DEV)
+    rep, _ = prefill_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary()
+
+
 def test_prefill_explicit_scale(oracle_lib):
     wl = small("f32", B=1, L=300, H=4, Hkv=1, d=64)
     x = make_prefill_inputs(wl, DEV)
