@@ -78,6 +78,14 @@ def decode_bytes(wl, lm_elem_bytes=2) -> float:
     return float(wl.B * per_seq)
 
 
+def landmark_bytes(wl) -> float:
+    """HBM bytes the DHSA landmark pass must move: the keys of every complete
+    chunk read once and each chunk's fp32 landmark written."""
+    el = 2 if wl.dtype == "bf16" else 4
+    Nc = wl.L // wl.S
+    return float(wl.B * wl.Hkv * Nc * (wl.S * wl.d * el + wl.d * 4))
+
+
 # ----------------------------------------------------------------------------- environment
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -342,6 +350,18 @@ def run_ours(args, dist, rank, world):
         "roofline": roofline, "clocks": clocks, "gpu_launches": launches,
     }
 
+    if wl.landmarks == "dhsa":
+        # the landmark stage of the breakdown steps: the work-list counts
+        # memset (a few KB) and the landmark kernel, L2 flushed before each step
+        lm_s = statistics.mean(lm_ms) / 1e3
+        nb = landmark_bytes(wl)
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        res["landmarks_roofline"] = {"kernel": "landmarks_kernel", "bound": "hbm",
+                                     "achieved": round(nb / lm_s / 1e9, 1), "peak": hbm,
+                                     "unit": "GB/s", "frac": round(nb / lm_s / 1e9 / hbm, 4),
+                                     "algorithmic_bytes_per_launch": nb,
+                                     "ms_per_launch": round(lm_s * 1e3, 4),
+                                     "peak_source": peaks["source"] + " copy bandwidth"}
     if args.e2e:
         res["e2e"] = e2e_prefill(args, wl, x, ws, dev, dist)
     del x, out

@@ -78,3 +78,18 @@ def test_flop_and_byte_counts_match_definitions():
     nc = d5.L // d5.S
     assert bench.decode_bytes(d5) == d5.B * (d5.Hkv * nc * d5.d * 2 + d5.Hkv * 8 * 64 * d5.d * 2 * 2
                                              + 2 * d5.H * d5.d * 2)
+
+
+def test_work_counts_of_the_long_and_decode_workloads():
+    # the published per-step counts of the long prefill and the two decode
+    # workloads (algorithmic work only, dense work avoided not counted)
+    lp = WORKLOADS["long_prefill_bf16"]
+    f = bench.prefill_flops(lp)
+    assert f["selection"] == pytest.approx(6.87e10, rel=2e-3)
+    assert f["fusion"] == pytest.approx(4.29e9, rel=2e-3)
+    assert f["in_chunk"] == pytest.approx(5.485e11, rel=2e-3)
+    assert f["own_chunk"] == pytest.approx(3.49e10, rel=2e-3)
+    # DHSA landmark pass: 1 x 2 x 131072 x 128 bf16 keys read, 2048 fp32 landmarks per head written
+    assert bench.landmark_bytes(lp) == 2 * (131072 * 128 * 2 + 2048 * 128 * 4)
+    assert bench.decode_bytes(WORKLOADS["decode_32m_bf16"]) == 268_967_936
+    assert bench.decode_bytes(WORKLOADS["batched_decode_bf16"]) == 285_474_816
