@@ -93,3 +93,16 @@ def test_work_counts_of_the_long_and_decode_workloads():
     assert bench.landmark_bytes(lp) == 2 * (131072 * 128 * 2 + 2048 * 128 * 4)
     assert bench.decode_bytes(WORKLOADS["decode_32m_bf16"]) == 268_967_936
     assert bench.decode_bytes(WORKLOADS["batched_decode_bf16"]) == 285_474_816
+
+
+def test_traffic_record_is_tied_to_its_workload():
+    # the committed ncu DRAM figure of the attention kernel was taken on one
+    # workload; other workloads must not report it
+    files = ["hierarchical_chunk_sparse_landmark_b200/csrc/attend_tc.cu"]
+    t = bench.measured_traffic("attend_tc", files, workload="train_prefill_bf16")
+    if t is None:
+        pytest.skip("traffic record predates the current attend_tc.cu")
+    assert t > 0
+    assert bench.measured_traffic("attend_tc", files, workload="long_prefill_bf16") is None
+    assert bench.measured_traffic("attend_tc", files, "dram_write_bytes_per_launch",
+                                  workload="long_prefill_bf16") is None
