@@ -140,3 +140,23 @@ def test_selftest_rejects_before_launch():
     assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A + 4), 4096, 1000, None) == B.HSA_ERR_INVALID_ARG
     assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 4096, 0, None) == B.HSA_ERR_INVALID_ARG
     assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 4096, 5_000_000_000, None) == B.HSA_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c_and_the_example_links(tmp_path):
+    # include/hsa.h is a C header: a C99 program that drives prefill and decode
+    # through it (tests/c_abi_example.c) compiles with warnings as errors and
+    # links against libhsa.so and the CUDA runtime.  Running it needs a B200.
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    cuda_inc = "/usr/local/cuda/include"
+    if cc is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime_api.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    pkg = os.path.dirname(B.LIB_PATH)
+    exe = tmp_path / "c_abi_example"
+    cmd = [cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+           "-I", cuda_inc, os.path.join(ROOT, "tests", "c_abi_example.c"), "-L", pkg, "-lhsa",
+           "-L", "/usr/local/cuda/lib64", "-lcudart", "-lm", "-o", str(exe)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert exe.exists()
