@@ -11,9 +11,11 @@ over ranks / max-over-ranks device time (weak scaling: every rank runs its own
 independent batch, seeded by rank; no collective on the data path).  The same
 JSON line carries the 32M-context decode figure (tokens/s and HBM roofline),
 the roofline of the dominant kernel timed live with CUDA events on the
-launching stream, an end-to-end figure through host buffers, the SM clocks
-sampled during the timed region and the fp64 CPU oracle timed on a bounded
-sample of the same workload.
+launching stream (FLOP/s against the bf16 peak, and its chunk-output DRAM
+writes against the write-only HBM bandwidth measured in the run), the
+landmark kernel's HBM roofline for DHSA workloads, an end-to-end figure
+through host buffers, the SM clocks sampled during the timed region and the
+fp64 CPU oracle timed on a bounded sample of the same workload.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference for this
 method) on the host cores, each step a bounded sample of the workload.
