@@ -379,3 +379,96 @@ def test_decode_fewer_chunks_than_topk(oracle_lib):
     assert (dec["idx"][0, 0, 3:] == -1).all()
     assert np.isinf(dec["gap"][0, 0])
     np.testing.assert_allclose(dec["w"].sum(-1), 1.0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- forced selection
+def _hand_inputs(g):
+    L, H, d = g["L"], g["H"], g["d"]
+    Q = np.broadcast_to(np.array(g["Q_per_position"]), (1, L, H, d)).copy()
+    return Q, np.array(g["K"])[None, None], np.array(g["V"])[None, None], np.array(g["lm"])[None, None]
+
+
+def test_forced_selection_hand_rows(oracle_lib):
+    """Rows recomputed on a given selection (the entry point the GPU parity
+    tests use on near-tie rows), worked by hand on the 6-token example:
+    a reordered set keeps O and reorders w; pads and chunks that are not
+    visible from the row (its own chunk or later ones) are dropped."""
+    base = json.load(open(os.path.join(GOLDEN, "hand_example.json")))
+    g = json.load(open(os.path.join(GOLDEN, "forced_and_gap.json")))["forced"]
+    Q, K, V, lm = _hand_inputs(base)
+    rows = np.array(g["rows"], dtype=np.int64)
+    forced = np.array(g["forced_idx"], dtype=np.int32)[:, None, :]
+    r = oracle_lib.prefill(Q, K, V, lm, base["S"], base["topk"], base["own_chunk"],
+                           base["scale"], rows=rows, forced_idx=forced)
+    np.testing.assert_array_equal(r["idx"][:, 0, :], np.array(g["expected_idx"]))
+    np.testing.assert_allclose(r["O"], np.array(g["expected_O"]), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(r["w"], np.array(g["expected_w"]), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("own_chunk", [0, 1])
+def test_forced_selection_equal_to_own_is_bit_identical(oracle_lib, own_chunk):
+    """Forcing the oracle's own selection reproduces its outputs bit for bit."""
+    B, L, H, Hkv, d, S, topk = 2, 200, 4, 2, 8, 16, 3
+    Q, K, V, lm = rand_case(17, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk, own_chunk)
+    f = oracle_lib.prefill(Q, K, V, lm, S, topk, own_chunk, forced_idx=r["idx"])
+    np.testing.assert_array_equal(f["idx"], r["idx"])
+    np.testing.assert_array_equal(f["O"], r["O"])
+    np.testing.assert_array_equal(f["w"], r["w"])
+    np.testing.assert_array_equal(f["sbar"], r["sbar"])
+    assert np.isnan(f["gap"]).all()
+
+
+def test_forced_selection_swapped_chunk_matches_bruteforce(oracle_lib):
+    """One selected chunk swapped for an unselected visible one: O equals the
+    fusion, written out separately here, of attention over the forced chunks."""
+    B, L, H, Hkv, d, S, topk = 1, 160, 2, 1, 4, 16, 3
+    Q, K, V, lm = rand_case(18, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill(Q, K, V, lm, S, topk, own_chunk=0)
+    rows = np.arange(8 * S, L)
+    forced = r["idx"][rows].copy()
+    for n, t in enumerate(rows):
+        unsel = [c for c in range(t // S) if c not in forced[n, 0]]
+        forced[n, 0, 1] = unsel[n % len(unsel)]
+    f = oracle_lib.prefill(Q, K, V, lm, S, topk, own_chunk=0, rows=rows, forced_idx=forced)
+    scale = 1 / math.sqrt(d)
+    for n, t in enumerate(rows):
+        for h in range(H):
+            sel = forced[n, 0]
+            logit = lm[0, 0, sel] @ Q[0, t, h] * scale
+            wgt = np.exp(logit - logit.max())
+            wgt /= wgt.sum()
+            o = sum(wgt[j] * sdpa_full(Q[0, t, h][None], K[0, 0, i * S:(i + 1) * S],
+                                       V[0, 0, i * S:(i + 1) * S], scale)[0]
+                    for j, i in enumerate(sel))
+            np.testing.assert_allclose(f["O"][n, h], o, atol=1e-12)
+            np.testing.assert_allclose(f["w"][n, h], wgt, atol=1e-14)
+
+
+# --------------------------------------------------------------------------- near-tie gap
+@pytest.mark.parametrize("topk", [1, 2, 3])
+def test_prefill_gap_hand_scores(oracle_lib, topk):
+    """gap = K-th minus (K+1)-th group score, +inf when at most K chunks are
+    visible, on scores set by hand (tests/golden/forced_and_gap.json)."""
+    g = json.load(open(os.path.join(GOLDEN, "forced_and_gap.json")))["gap"]
+    S, L = g["S"], g["L"]
+    s = np.array(g["scores"])
+    lm = np.zeros((1, 1, len(s), 2))
+    lm[0, 0, :, 0] = s
+    Q = np.zeros((1, L, 1, 2))
+    Q[..., 0] = 1.0
+    K = np.zeros((1, 1, L, 2))
+    r = oracle_lib.prefill(Q, K, K, lm, S, topk, scale=1.0)
+    want = np.array([np.inf if v == "inf" else v for v in g["expected_gap"][str(topk)]])
+    np.testing.assert_array_equal(r["gap"][:, 0], want)
+
+
+def test_decode_gap_hand_scores(oracle_lib):
+    g = json.load(open(os.path.join(GOLDEN, "forced_and_gap.json")))["gap"]
+    s = np.array(g["scores"])
+    lm = np.zeros((1, 1, len(s), 2))
+    lm[0, 0, :, 0] = s
+    q = np.array([[[1.0, 0.0]]])
+    for k, v in g["decode"]["expected_gap"].items():
+        r = oracle_lib.decode_select(q, lm, int(k), scale=1.0)
+        assert r["gap"][0, 0] == (np.inf if v == "inf" else v), (k, r["gap"])

@@ -39,6 +39,17 @@ MUTANTS = {
                                 "const int64_t first = sel[kk] * S + (sel[kk] > 0 ? -1 : 1);\n"),
     "fusion_weight_from_group_query": ("wk[kk] = scale * dot(q_h, lm_bg", "wk[kk] = scale * dot(qbar, lm_bg"),
     "decode_weights_unnormalised": ("softmax_inplace(wk, nsel);", ";"),
+    # near-tie gap: the next pair down the ranking (off by one)
+    "gap_off_by_one": ("gap_val = nvis > topk ? cand[topk - 1].score - cand[topk].score : INFINITY;",
+                       "gap_val = nvis > topk + 1 ? cand[topk].score - cand[topk + 1].score : INFINITY;"),
+    "decode_gap_off_by_one": ("gap[bg] = Nc > topk ? cand[topk - 1].score - cand[topk].score : INFINITY;",
+                              "gap[bg] = Nc > topk + 1 ? cand[topk].score - cand[topk + 1].score : INFINITY;"),
+    # forced selection: chunks not visible from the row are kept
+    "forced_visibility_filter_dropped": ("if (f[kk] >= 0 && f[kk] < nvis) sel[nsel++] = f[kk];",
+                                         "if (f[kk] >= 0 && f[kk] < Nc) sel[nsel++] = f[kk];"),
+    # forced selection: slots taken in reverse order
+    "forced_slots_reversed": ("const int32_t *f = forced_idx + (r * Hkv + g) * topk;",
+                              "int32_t f[64]; for (int kk = 0; kk < topk; ++kk) f[kk] = forced_idx[(r * Hkv + g) * topk + topk - 1 - kk];"),
 }
 
 
