@@ -6,10 +6,12 @@ The computation runs in hand-written CUDA kernels behind a C ABI
 binding (PyTorch supplies device memory and streams) plus the seeded synthetic
 workloads used by the tests and the benchmark.
 """
-from ._binding import (HSAError, check, last_call_launches, decode, decode_workspace_size, landmarks, lib, prefill,
-                       prefill_workspace_size, selftest_wait_expiry, set_stage_events, status_string,
-                       workspace)
+from ._binding import (HSAError, check, decode, decode_noalloc, decode_workspace_size,
+                       landmarks, last_call_kernels, last_call_launches, lib, path_overrides,
+                       prefill, prefill_workspace_size, selftest_wait_expiry, set_stage_events,
+                       status_string, workspace)
 
-__all__ = ["HSAError", "check", "last_call_launches", "decode", "decode_workspace_size", "landmarks", "lib", "prefill",
+__all__ = ["HSAError", "check", "decode", "decode_noalloc", "decode_workspace_size", "landmarks",
+           "last_call_kernels", "last_call_launches", "lib", "path_overrides", "prefill",
            "prefill_workspace_size", "selftest_wait_expiry", "set_stage_events", "status_string",
            "workspace"]

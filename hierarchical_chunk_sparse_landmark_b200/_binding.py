@@ -20,10 +20,17 @@ HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED = 0, 1, 2
 HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT = 3, 4, 5
 HSA_F32, HSA_BF16 = 0, 1
 
+# kernel families of a call (hsa_last_call_kernels) and path overrides
+K_LANDMARKS, K_SPLIT_LANDMARKS, K_SELECT_TC_ONE_TILE, K_SELECT_TC_MULTI_TILE = 1, 2, 4, 8
+K_SELECT_SIMT, K_WORK_LISTS, K_ATTEND_TC, K_FUSE, K_ATTEND_SIMT = 16, 32, 64, 128, 256
+K_DECODE_SCAN, K_DECODE_ATTEND = 512, 1024
+PATH_SIMT_PREFILL, PATH_SIMT_SELECT, PATH_MULTI_TILE_SELECT = 1, 2, 4
+
 EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_decode_workspace_size", "hsa_decode", "hsa_check", "hsa_status_string",
             "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches",
-            "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry")
+            "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry",
+            "hsa_last_call_kernels", "hsa_set_path_overrides")
 
 
 class HSAError(RuntimeError):
@@ -55,11 +62,14 @@ def _declare(lib):
     lib.hsa_decode_noalloc_max_scratch.argtypes = []
     lib.hsa_decode_noalloc_max_scratch.restype = sz
     lib.hsa_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
+    lib.hsa_last_call_kernels.argtypes = []
+    lib.hsa_last_call_kernels.restype = ctypes.c_uint
+    lib.hsa_set_path_overrides.argtypes = [i32, i64]
     lib.hsa_status_string.argtypes = [i32]
     lib.hsa_status_string.restype = ctypes.c_char_p
     for n in ("hsa_landmarks", "hsa_prefill", "hsa_decode", "hsa_check", "hsa_version",
               "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
-              "hsa_selftest_wait_expiry"):
+              "hsa_selftest_wait_expiry", "hsa_set_path_overrides"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -220,9 +230,10 @@ def decode_noalloc(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.
         out = torch.empty_like(q)
     if idx_out is True:
         idx_out = torch.empty(B, Hkv, topk, dtype=torch.int32, device=q.device)
-    st = lib().hsa_decode_noalloc(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm),
-                                  _dtype_code(lm), B, H, Hkv, Lc, d, S, topk, float(scale),
-                                  _ptr(out), _ptr(_opt(idx_out)), _stream(q.device))
+    with torch.cuda.device(q.device):      # the array is looked up on the current device
+        st = lib().hsa_decode_noalloc(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm),
+                                      _dtype_code(lm), B, H, Hkv, Lc, d, S, topk, float(scale),
+                                      _ptr(out), _ptr(_opt(idx_out)), _stream(q.device))
     _check(st, "hsa_decode_noalloc")
     return out, _opt(idx_out)
 
@@ -241,10 +252,40 @@ def last_call_launches() -> int:
     return int(lib().hsa_last_call_launches())
 
 
-def selftest_wait_expiry(ws, budget_cycles: int = 2_000_000):
+def last_call_kernels() -> int:
+    """Kernel families (K_* bits) of this thread's most recent library call."""
+    return int(lib().hsa_last_call_kernels())
+
+
+class path_overrides:
+    """Context manager: this thread's prefill calls take the paths named by
+    ``flags`` (PATH_* bits) and token windows of ``window_tokens`` (0 = the
+    library's choice); see hsa_set_path_overrides.  Restores the defaults."""
+
+    def __init__(self, flags: int = 0, window_tokens: int = 0):
+        self.flags, self.window = int(flags), int(window_tokens)
+
+    def __enter__(self):
+        _check(lib().hsa_set_path_overrides(self.flags, self.window), "hsa_set_path_overrides")
+        return self
+
+    def __exit__(self, *exc):
+        lib().hsa_set_path_overrides(0, 0)
+        return False
+
+
+def selftest_wait_expiry(ws, budget_cycles: int = 2_000_000, device=None):
     """Run the library's bounded-wait failure path once: a device wait that
     nothing completes gives up after `budget_cycles` and flags the status word
-    of `ws`; the following check(ws) raises HSAError with status HSA_ERR_TIMEOUT."""
+    of `ws`; the following check(ws) raises HSAError with status HSA_ERR_TIMEOUT.
+    ``ws=None`` aims at the status word of decode_noalloc's fixed array on
+    ``device`` (reported by check(None, device))."""
+    if ws is None:
+        dev = torch.device(device if device is not None else "cuda")
+        with torch.cuda.device(dev):
+            _check(lib().hsa_selftest_wait_expiry(None, 0, int(budget_cycles), _stream(dev)),
+                   "hsa_selftest_wait_expiry")
+        return
     _dev(ws, "ws")
     _check(lib().hsa_selftest_wait_expiry(_ptr(ws), ws.numel() * ws.element_size(), int(budget_cycles),
                                           _stream(ws.device)), "hsa_selftest_wait_expiry")

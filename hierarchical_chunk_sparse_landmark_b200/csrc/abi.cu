@@ -28,12 +28,16 @@ bool select_tc_supported();
 cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaStream_t st);
 cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
                              int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
-                             int32_t *idx, unsigned *status, cudaStream_t st);
+                             int32_t *idx, unsigned *status, bool force_multi_tile, bool *multi,
+                             cudaStream_t st);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
                           int64_t *seg_start, int4 *tiles, cudaStream_t st);
 cudaError_t launch_selftest_wait(unsigned *status, long long budget, cudaStream_t st);
+// Status word of hsa_decode_noalloc's fixed array on the stream's device
+// (decode_noalloc.cu); nullptr when the array is unused there and !mark.
+hsa_status_t noalloc_status_word(cudaStream_t stream, bool mark, void **out);
 }  // namespace hsa
 
 using namespace hsa;
@@ -44,6 +48,12 @@ constexpr int kChunk = 64;
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 bool dtype_ok(hsa_dtype_t t) { return t == HSA_F32 || t == HSA_BF16; }
+
+// Per-thread path overrides (hsa_set_path_overrides) and the kernels of the
+// thread's last call (hsa_last_call_kernels).
+thread_local int t_path_flags = 0;
+thread_local int64_t t_window_tokens = 0;
+thread_local unsigned t_kernels = 0;
 
 // Shape checks shared by every call.  INVALID_ARG for impossible requests,
 // UNSUPPORTED for valid ones this build does not implement.
@@ -89,13 +99,13 @@ bool tc_shape_ok(int B, int H, int Hkv, int64_t L, int d, int topk) {
 // L = 131072 prefill: 8192-token windows 3.01 ms, 16384 3.06, 32768 3.18,
 // one window 3.55).  The
 // window is a multiple of 256 tokens (the work-list blocks' size);
-// HSA_TC_WINDOW overrides it for experiments.
+// hsa_set_path_overrides can set it (tests force several windows on small shapes).
 int64_t tc_window(int B, int H, int Hkv, int64_t L, int d, int topk, int64_t max_windows) {
     (void)topk;
     int64_t W = (L + 255) / 256 * 256;
     const int64_t q_bytes_per_token = (int64_t)(H / Hkv) * d * 2;
     int64_t cap = (int64_t(16) << 20) / q_bytes_per_token / 256 * 256;
-    if (const char *v = getenv("HSA_TC_WINDOW")) cap = atoll(v) / 256 * 256;
+    if (t_window_tokens > 0) cap = t_window_tokens / 256 * 256;
     if (cap >= 256 && W > cap) W = cap;
     while ((int64_t)B * Hkv * ((L + W - 1) / W) > max_windows) W *= 2;
     return W;
@@ -162,15 +172,10 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     return p;
 }
 
-bool force_simt_path() {
-    const char *v = getenv("HSA_PREFILL_PATH");
-    return v && strcmp(v, "simt") == 0;
-}
+bool force_simt_path() { return (t_path_flags & HSA_PATH_SIMT_PREFILL) != 0; }
 // Selection on CUDA cores even where the tensor-core selection applies (A/B checks).
-bool force_simt_select() {
-    const char *v = getenv("HSA_SELECT_PATH");
-    return v && strcmp(v, "simt") == 0;
-}
+bool force_simt_select() { return (t_path_flags & HSA_PATH_SIMT_SELECT) != 0; }
+bool force_multi_tile_select() { return (t_path_flags & HSA_PATH_MULTI_TILE_SELECT) != 0; }
 
 // Decode workspace: status | tickets | unit counters (the zeroed head) | sel | cand.
 struct DecodeLayout {
@@ -226,6 +231,17 @@ int hsa_version(void) { return 100; }
 
 int hsa_last_call_launches(void) { return t_launches; }
 
+unsigned hsa_last_call_kernels(void) { return t_kernels; }
+
+hsa_status_t hsa_set_path_overrides(int flags, int64_t window_tokens) {
+    const int known = HSA_PATH_SIMT_PREFILL | HSA_PATH_SIMT_SELECT | HSA_PATH_MULTI_TILE_SELECT;
+    if ((flags & ~known) != 0 || window_tokens < 0 || (window_tokens > 0 && window_tokens < 256))
+        return HSA_ERR_INVALID_ARG;
+    t_path_flags = flags;
+    t_window_tokens = window_tokens;
+    return HSA_OK;
+}
+
 hsa_status_t hsa_set_stage_events(void *const *events, int n) {
     if (n < 0 || n > kMaxStageEvents || (n > 0 && !events)) return HSA_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) t_stage_events[i] = (cudaEvent_t)events[i];
@@ -251,9 +267,11 @@ hsa_status_t hsa_landmarks(const void *K, hsa_dtype_t k_dt, float *lm_out, int B
     if (s != HSA_OK) return s;
     if (!dtype_ok(k_dt)) return HSA_ERR_UNSUPPORTED;
     t_launches = 0;
+    t_kernels = 0;
     if (L / S == 0) return HSA_OK;
     if (!K || !lm_out || !aligned16(K) || !aligned16(lm_out)) return HSA_ERR_INVALID_ARG;
     t_launches = 1;
+    t_kernels = HSA_K_LANDMARKS;
     return from_cuda(launch_landmarks(K, k_dt == HSA_BF16, lm_out, B, Hkv, L, d,
                                       (cudaStream_t)stream));
 }
@@ -274,6 +292,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
     if (own_chunk != 0 && own_chunk != 1) return HSA_ERR_INVALID_ARG;
     if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
     t_launches = 0;
+    t_kernels = 0;
     if (L == 0) return HSA_OK;
     const void *ptrs[] = {Q, K, V, O, workspace};
     for (const void *p : ptrs)
@@ -303,6 +322,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         cudaError_t e = launch_landmarks(K, bf16, lm_ws, B, Hkv, L, d, st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
         t_launches += L / S > 0 ? 1 : 0;
+        t_kernels |= L / S > 0 ? (unsigned)HSA_K_LANDMARKS : 0u;
         lm_use = lm_ws;
         lm_bf16 = false;
     }
@@ -317,17 +337,21 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         e = launch_split_landmarks(lm_use, lm_split, (int64_t)B * Hkv * (L / S) * d, st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
         t_launches += 1;
+        t_kernels |= HSA_K_SPLIT_LANDMARKS;
     }
     const bool tc_select = use_tc && L >= S && (H / Hkv) % 8 == 0 && select_tc_supported() &&
                            !force_simt_select();
+    bool multi = false;
     if (tc_select)
         e = launch_select_tc(Q, lm_use, lm_bf16, lm_split, B, H, Hkv, L, d, S, topk, scale, idx,
-                             (unsigned *)ws, st);
+                             (unsigned *)ws, force_multi_tile_select(), &multi, st);
     else
         e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
                           use_tc ? nullptr : w, st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
     t_launches += 1;
+    t_kernels |= !tc_select ? HSA_K_SELECT_SIMT
+                            : multi ? HSA_K_SELECT_TC_MULTI_TILE : HSA_K_SELECT_TC_ONE_TILE;
     stage_mark(2, st);
     if (use_tc) {
         const int64_t Nc = L / S;
@@ -338,6 +362,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                           (int64_t *)(ws + lay.seg_off), (int4 *)(ws + lay.tiles_off), st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
         t_launches += 3;                  // count, scan, fill (scatter + flatten)
+        t_kernels |= HSA_K_WORK_LISTS;
         stage_mark(3, st);
         TcLaunch a;
         a.Q = Q; a.K = K; a.V = V; a.lm = lm_bf16 ? lm_use : lm_split; a.lm_bf16 = lm_bf16 ? 1 : 0;
@@ -353,11 +378,13 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.num_sms = num_sms();
         e = launch_attend_tc(a, d, st, stage_event(4));
         t_launches += e == cudaSuccess ? 2 : 0;
+        t_kernels |= e == cudaSuccess ? (unsigned)(HSA_K_ATTEND_TC | HSA_K_FUSE) : 0u;
     } else {
         stage_mark(3, st);
         e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale,
                                O, st);
         t_launches += e == cudaSuccess ? 1 : 0;
+        t_kernels |= e == cudaSuccess ? (unsigned)HSA_K_ATTEND_SIMT : 0u;
         stage_mark(4, st);            // the SIMT kernel fuses in place
     }
     stage_mark(5, st);
@@ -380,6 +407,7 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
     if (Lc % S != 0) return HSA_ERR_INVALID_ARG;
     if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
     t_launches = 0;
+    t_kernels = 0;
     if (!q || !O || !workspace || !aligned16(q) || !aligned16(O) || !aligned16(workspace))
         return HSA_ERR_INVALID_ARG;
     if (idx_out && !aligned16(idx_out)) return HSA_ERR_INVALID_ARG;
@@ -404,14 +432,21 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
                                    Lc, d, S, topk, scale, lay.splits, lay.at(ws), O,
                                    idx_out, st));
     t_launches = r == HSA_OK ? 2 : 0;
+    t_kernels = r == HSA_OK ? (unsigned)(HSA_K_DECODE_SCAN | HSA_K_DECODE_ATTEND) : 0u;
     stage_mark(1, st);
     return r;
 }
 
 hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t budget_cycles,
                                       void *stream) {
-    if (!workspace || ws_bytes < 16 || ((uintptr_t)workspace & 15) != 0) return HSA_ERR_INVALID_ARG;
     if (budget_cycles < 1 || budget_cycles > 4000000000LL) return HSA_ERR_INVALID_ARG;
+    if (!workspace) {
+        // aimed at the status word of hsa_decode_noalloc's array on the stream's device
+        const hsa_status_t s = noalloc_status_word((cudaStream_t)stream, true, &workspace);
+        if (s != HSA_OK) return s;
+        ws_bytes = kStatusBytes;
+    }
+    if (ws_bytes < 16 || ((uintptr_t)workspace & 15) != 0) return HSA_ERR_INVALID_ARG;
     return hsa::launch_selftest_wait((unsigned *)workspace, (long long)budget_cycles,
                                      (cudaStream_t)stream) == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
 }
@@ -419,7 +454,13 @@ hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t 
 hsa_status_t hsa_check(void *workspace, void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
-    if (!workspace) return HSA_OK;
+    if (!workspace) {
+        // Calls without a workspace (hsa_decode_noalloc) flag the status word
+        // at the head of the library's array on the stream's device.
+        if (noalloc_status_word((cudaStream_t)stream, false, &workspace) != HSA_OK)
+            return HSA_ERR_CUDA;
+        if (!workspace) return HSA_OK;
+    }
     unsigned flags = 0;
     if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
         return HSA_ERR_CUDA;

@@ -634,16 +634,9 @@ static bool sel_make_map(CUtensorMap *m, const void *base, uint64_t rows, int D)
            CUDA_SUCCESS;
 }
 
-// HSA_SELECT_TILES=multi keeps the multi-tile kernel for every length (tests
-// run both kernels on the same shapes).
-static bool force_multi_tile() {
-    const char *v = getenv("HSA_SELECT_TILES");
-    return v && strcmp(v, "multi") == 0;
-}
-
 template <int D, bool LM32, int KP>
 static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l0, const void *l1,
-                                      cudaStream_t st) {
+                                      bool force_multi_tile, bool *multi, cudaStream_t st) {
     using C = SelCfg<D, LM32>;
     const uint64_t rows = (uint64_t)B * p.Hkv * p.Nc;
     CUtensorMap m0, m1;
@@ -654,7 +647,8 @@ static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l
         m1 = m0;
     }
     dim3 grid((unsigned)((p.L + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
-    if (p.Nc <= SelHalfCfg<D, LM32>::N && !force_multi_tile()) {
+    *multi = !(p.Nc <= SelHalfCfg<D, LM32>::N && !force_multi_tile);
+    if (!*multi) {
         // every chunk fits one score tile: qbar built per 64-column block, two blocks per SM
         using H = SelHalfCfg<D, LM32>;
         auto kern = select_tc_half_kernel<D, LM32, KP>;
@@ -670,10 +664,10 @@ static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l
 
 template <int D, bool LM32>
 static cudaError_t launch_select_tc_k(const SelTcParams &p, int B, const void *l0, const void *l1,
-                                      cudaStream_t st) {
-    if (p.topk <= 8) return launch_select_tc_t<D, LM32, 8>(p, B, l0, l1, st);
-    if (p.topk <= 16) return launch_select_tc_t<D, LM32, 16>(p, B, l0, l1, st);
-    return launch_select_tc_t<D, LM32, 32>(p, B, l0, l1, st);
+                                      bool fm, bool *multi, cudaStream_t st) {
+    if (p.topk <= 8) return launch_select_tc_t<D, LM32, 8>(p, B, l0, l1, fm, multi, st);
+    if (p.topk <= 16) return launch_select_tc_t<D, LM32, 16>(p, B, l0, l1, fm, multi, st);
+    return launch_select_tc_t<D, LM32, 32>(p, B, l0, l1, fm, multi, st);
 }
 
 bool select_tc_supported() { return sel_encode_fn() != nullptr; }
@@ -689,21 +683,24 @@ cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaS
 
 // Q bf16; landmarks bf16 (lm_bf16), else the two bf16 planes `split` of fp32
 // landmarks (launch_split_landmarks, B*Hkv*Nc*d elements each).  Nc = L / S
-// >= 1; G = H / Hkv a multiple of 8.
+// >= 1; G = H / Hkv a multiple of 8.  Up to 128 chunks the one-tile kernel
+// runs unless `force_multi_tile`; `*multi` tells which kernel was launched.
 cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
                              int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
-                             int32_t *idx, unsigned *status, cudaStream_t st) {
+                             int32_t *idx, unsigned *status, bool force_multi_tile, bool *multi,
+                             cudaStream_t st) {
     SelTcParams p;
     p.Q = Q; p.idx = idx; p.status = status;
     p.L = L; p.Nc = L / S; p.H = H; p.Hkv = Hkv; p.S = S; p.topk = topk; p.scale = scale;
+    const bool fm = force_multi_tile;
     if (lm_bf16) {
-        return d == 128 ? launch_select_tc_k<128, false>(p, B, lm, nullptr, st)
-                        : launch_select_tc_k<64, false>(p, B, lm, nullptr, st);
+        return d == 128 ? launch_select_tc_k<128, false>(p, B, lm, nullptr, fm, multi, st)
+                        : launch_select_tc_k<64, false>(p, B, lm, nullptr, fm, multi, st);
     }
     const int64_t n = (int64_t)B * Hkv * p.Nc * d;
     const __nv_bfloat16 *l0 = (const __nv_bfloat16 *)split, *l1 = l0 + n;
-    return d == 128 ? launch_select_tc_k<128, true>(p, B, l0, l1, st)
-                    : launch_select_tc_k<64, true>(p, B, l0, l1, st);
+    return d == 128 ? launch_select_tc_k<128, true>(p, B, l0, l1, fm, multi, st)
+                    : launch_select_tc_k<64, true>(p, B, l0, l1, fm, multi, st);
 }
 
 }  // namespace hsa

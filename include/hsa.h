@@ -60,6 +60,28 @@ typedef enum {
 
 typedef enum { HSA_F32 = 0, HSA_BF16 = 1 } hsa_dtype_t;
 
+/* Kernel families a call launched (hsa_last_call_kernels). */
+enum {
+    HSA_K_LANDMARKS = 1u << 0,            /* DHSA landmarks (hsa_landmarks, or prefill with lm = NULL) */
+    HSA_K_SPLIT_LANDMARKS = 1u << 1,      /* fp32 landmarks split into bf16 high/low planes */
+    HSA_K_SELECT_TC_ONE_TILE = 1u << 2,   /* tensor-core selection, all chunks in one score tile */
+    HSA_K_SELECT_TC_MULTI_TILE = 1u << 3, /* tensor-core selection over several score tiles */
+    HSA_K_SELECT_SIMT = 1u << 4,          /* selection on CUDA cores */
+    HSA_K_WORK_LISTS = 1u << 5,           /* chunk buckets and tile lists */
+    HSA_K_ATTEND_TC = 1u << 6,            /* tensor-core in-chunk attention */
+    HSA_K_FUSE = 1u << 7,                 /* fusion of the chunk outputs */
+    HSA_K_ATTEND_SIMT = 1u << 8,          /* in-chunk attention + fusion on CUDA cores */
+    HSA_K_DECODE_SCAN = 1u << 9,          /* decode landmark scan + top-K */
+    HSA_K_DECODE_ATTEND = 1u << 10        /* decode attend + fusion */
+};
+
+/* Path overrides (hsa_set_path_overrides). */
+enum {
+    HSA_PATH_SIMT_PREFILL = 1,            /* prefill on CUDA cores even where tensor cores apply */
+    HSA_PATH_SIMT_SELECT = 2,             /* selection on CUDA cores even where tensor cores apply */
+    HSA_PATH_MULTI_TILE_SELECT = 4        /* the multi-tile tensor-core selection at any length */
+};
+
 /*
  * hsa_landmarks -- DHSA landmarks: l[b,g,i] = sqrt(S) * mean of the S keys of
  * chunk i (Dynamic Hierarchical Sparse Attention review, "What carries the
@@ -155,16 +177,21 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
  *  - Sizes whose scratch (hsa_decode_workspace_size) exceeds that array are
  *    rejected with HSA_ERR_WORKSPACE before anything is launched; invalid
  *    arguments return the same status hsa_decode would.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture on the device.
+ *  - Every call looks up the array's device address on the stream's device
+ *    (cudaGetSymbolAddress, with that device current); the first call on a
+ *    device loads the array, so make it before any stream capture on that
+ *    device.  The stream's device must be the current device, as for
+ *    hsa_decode.
  *  - Every call on a device shares the one array, and the array keeps the
  *    previous call's contents.  Each call clears the part that must start at
- *    zero with cudaMemsetAsync on `stream`.  Calls that can overlap on the
- *    GPU (different streams, or several host threads without ordering) race
- *    on the array and give wrong results: order them on one stream.
+ *    zero (tickets and work counters) with cudaMemsetAsync on `stream`.
+ *    Calls that can overlap on the GPU (different streams, or several host
+ *    threads without ordering) race on the array and give wrong results:
+ *    order them on one stream.
+ *  - The array starts with a status word.  A call whose device-side bounded
+ *    wait runs out sets its timeout flag there; the flag survives later calls
+ *    until hsa_check(NULL, stream) returns HSA_ERR_TIMEOUT and clears it.
  *  - No cudaMalloc, cudaFree or other allocating routine is called.
- * hsa_check(NULL, stream) reports errors of a call.
  */
 hsa_status_t hsa_decode_noalloc(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
                                 const void *lm, hsa_dtype_t lm_dt,
@@ -182,7 +209,10 @@ size_t hsa_decode_noalloc_max_scratch(void);
  * head of `workspace` and exits, as every kernel of the library does when one
  * of its waits runs out.  A following hsa_check(workspace, stream) returns
  * HSA_ERR_TIMEOUT and clears the flag; the CUDA context stays usable.
- *   workspace     any workspace of this library (>= 16 bytes), zero-filled
+ *   workspace     any workspace of this library (>= 16 bytes), zero-filled;
+ *                 NULL aims at the status word of hsa_decode_noalloc's array
+ *                 on the stream's device (then hsa_check(NULL, stream)
+ *                 reports the flag)
  *   budget_cycles 1 .. 4e9 (2e6 is about 1 ms)
  * Returns HSA_ERR_INVALID_ARG for a bad argument, HSA_ERR_CUDA if the launch
  * fails, else HSA_OK (the expiry itself is reported by hsa_check).
@@ -195,7 +225,10 @@ hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t 
  * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
  * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up (and clears
  * the word), HSA_ERR_CUDA if the stream reports an error, HSA_OK otherwise.
- * `workspace` may be NULL to check the stream only.
+ * With workspace = NULL it reads the status word of hsa_decode_noalloc's
+ * array on the stream's device (if this process has used that array there),
+ * which collects the flags of every hsa_decode_noalloc call since the last
+ * check.
  */
 hsa_status_t hsa_check(void *workspace, void *stream);
 
@@ -219,6 +252,26 @@ hsa_status_t hsa_set_stage_events(void *const *events, int n);
  * recent hsa_prefill / hsa_decode / hsa_landmarks call launched.
  */
 int hsa_last_call_launches(void);
+
+/*
+ * hsa_last_call_kernels -- the kernel families (HSA_K_* bits) that the calling
+ * thread's most recent hsa_prefill / hsa_decode / hsa_landmarks call launched:
+ * which path the dispatch took for those sizes and dtypes.
+ */
+unsigned hsa_last_call_kernels(void);
+
+/*
+ * hsa_set_path_overrides -- testing and measurement hook.  Until called again,
+ * hsa_prefill and hsa_prefill_workspace_size calls made by the CALLING THREAD
+ * take the paths named by `flags` (HSA_PATH_* bits; 0 = the library's own
+ * choice) and, if window_tokens > 0, split the tensor-core work lists into
+ * token windows of that many tokens (rounded down to a multiple of 256; 0 =
+ * the library's own choice).  Results are the same on every path up to the
+ * rounding of each; a workspace must be sized under the same overrides as
+ * the call that uses it.  Returns HSA_ERR_INVALID_ARG for unknown flags or a
+ * window of 1..255 tokens.  The library reads no environment variables.
+ */
+hsa_status_t hsa_set_path_overrides(int flags, int64_t window_tokens);
 
 /* hsa_status_string -- static, NUL-terminated description of a status. */
 const char *hsa_status_string(hsa_status_t status);

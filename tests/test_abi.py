@@ -133,9 +133,36 @@ def test_product_path_has_no_cpu_tensors_path():
         hsa.prefill(torch.zeros(1, 64, 2, 64), torch.zeros(1, 1, 64, 64), torch.zeros(1, 1, 64, 64))
 
 
+def test_path_overrides_validate_their_arguments():
+    lib = B.lib()
+    assert lib.hsa_set_path_overrides(8, 0) == B.HSA_ERR_INVALID_ARG        # unknown flag
+    assert lib.hsa_set_path_overrides(0, 100) == B.HSA_ERR_INVALID_ARG      # window < 256
+    assert lib.hsa_set_path_overrides(0, -1) == B.HSA_ERR_INVALID_ARG
+    assert lib.hsa_set_path_overrides(7, 512) == B.HSA_OK
+    assert lib.hsa_set_path_overrides(0, 0) == B.HSA_OK
+
+
+def test_window_override_changes_the_workspace_layout():
+    # the work lists of 512-token windows need more tile slots than one window
+    # per sequence; the override applies to this thread's size queries too
+    base = hsa.prefill_workspace_size(2, 16, 2, 64 * 37 + 29, 128, 64, 8)
+    with hsa.path_overrides(0, 512):
+        small = hsa.prefill_workspace_size(2, 16, 2, 64 * 37 + 29, 128, 64, 8)
+    assert small != base and hsa.prefill_workspace_size(2, 16, 2, 64 * 37 + 29, 128, 64, 8) == base
+
+
+def test_library_reads_no_environment_variables():
+    import re
+    csrc = os.path.join(ROOT, "hierarchical_chunk_sparse_landmark_b200", "csrc")
+    for f in os.listdir(csrc):
+        src = open(os.path.join(csrc, f)).read()
+        assert not re.search(r"\bgetenv\s*\(", src), f
+
+
 def test_selftest_rejects_before_launch():
     lib = B.lib()
-    assert lib.hsa_selftest_wait_expiry(None, 4096, 1000, None) == B.HSA_ERR_INVALID_ARG
+    # NULL aims at hsa_decode_noalloc's array; a bad budget is still rejected first
+    assert lib.hsa_selftest_wait_expiry(None, 0, 0, None) == B.HSA_ERR_INVALID_ARG
     assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 8, 1000, None) == B.HSA_ERR_INVALID_ARG
     assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A + 4), 4096, 1000, None) == B.HSA_ERR_INVALID_ARG
     assert lib.hsa_selftest_wait_expiry(ctypes.c_void_p(A), 4096, 0, None) == B.HSA_ERR_INVALID_ARG

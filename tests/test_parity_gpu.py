@@ -13,6 +13,7 @@ import pytest
 import torch
 
 import hierarchical_chunk_sparse_landmark_b200 as hsa
+from hierarchical_chunk_sparse_landmark_b200 import _binding as B
 from hierarchical_chunk_sparse_landmark_b200.workloads import (WORKLOADS, Workload,
                                                                make_decode_inputs,
                                                                make_prefill_inputs)
@@ -29,13 +30,33 @@ def _np(t):
         else t.detach().cpu().numpy().astype(np.float64)
 
 
-def prefill_parity(oracle_lib, wl: Workload, x: dict, rows=None, lm_override=None, scale=0.0,
-                   report=None):
-    """Run hsa.prefill on x and compare rows (flattened b*L+t; default all)."""
-    lm = x["lm"] if lm_override is None else lm_override
+TC_PATH = B.K_WORK_LISTS | B.K_ATTEND_TC | B.K_FUSE
+
+
+def expect_tc_path(kernels: int, tc: bool):
+    """The dispatch took the tensor-core chain (tc) or the CUDA-core path."""
+    if tc:
+        assert kernels & TC_PATH == TC_PATH and not kernels & B.K_ATTEND_SIMT, hex(kernels)
+    else:
+        assert kernels & B.K_ATTEND_SIMT and not kernels & B.K_ATTEND_TC, hex(kernels)
+
+
+_WORKLOAD_LM = object()
+
+
+def prefill_parity(oracle_lib, wl: Workload, x: dict, rows=None, lm_override=_WORKLOAD_LM,
+                   scale=0.0, report=None):
+    """Run hsa.prefill on x and compare rows (flattened b*L+t; default all).
+    The call gets its own zero-filled workspace, whose status word is checked;
+    the kernel families it launched are returned in ``report.kernels``."""
+    lm = x["lm"] if lm_override is _WORKLOAD_LM else lm_override     # None: DHSA landmarks
+    B_, L_, H_, d_ = x["Q"].shape
+    ws = torch.zeros(max(256, hsa.prefill_workspace_size(B_, H_, wl.Hkv, L_, d_, wl.S, wl.topk)),
+                     dtype=torch.uint8, device=DEV)
     O, idx, w = hsa.prefill(x["Q"], x["K"], x["V"], lm, S=wl.S, topk=wl.topk,
-                            own_chunk=wl.own_chunk, scale=scale, idx_out=True, w_out=True)
-    hsa.check()
+                            own_chunk=wl.own_chunk, scale=scale, idx_out=True, w_out=True, ws=ws)
+    kernels = hsa.last_call_kernels()
+    hsa.check(ws)
     B, L, H, d = x["Q"].shape
     Hkv = wl.Hkv
     if rows is None:
@@ -51,6 +72,7 @@ def prefill_parity(oracle_lib, wl: Workload, x: dict, rows=None, lm_override=Non
     got_w = w.reshape(B * L, H, wl.topk)[rt].cpu().numpy().astype(np.float64)
     got_O = _np(O.reshape(B * L, H, d)[rt])
     rep = report or ParityReport()
+    rep.kernels = kernels
     rep.rows += len(rows)
     differs = compare_selection(ref["idx"], ref["sbar"], ref["gap"], got_idx, rep)
     ref_O = ref["O"]
@@ -84,26 +106,35 @@ def test_prefill_small_all_rows(oracle_lib, dtype, d, H, Hkv):
     x = make_prefill_inputs(wl, DEV)
     rep, _ = prefill_parity(oracle_lib, wl, x)
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    expect_tc_path(rep.kernels, dtype == "bf16" and H // Hkv in (8, 16))
 
 
 @pytest.mark.parametrize("topk", [1, 2, 8, 17, 32])
 @pytest.mark.parametrize("own", [0, 1])
-def test_prefill_topk_and_own_chunk(oracle_lib, topk, own):
-    wl = small("bf16", B=1, L=64 * 40 + 5, topk=topk, own=own, seed=topk)
+@pytest.mark.parametrize("H,Hkv,d", [(8, 2, 128), (16, 2, 128), (16, 1, 64)])
+def test_prefill_topk_and_own_chunk(oracle_lib, topk, own, H, Hkv, d):
+    # G = 4 takes the CUDA-core path, G = 8 and 16 the tensor-core chain
+    # (own_chunk = 0 there still computes the own tiles, with weight 0)
+    wl = small("bf16", B=1, L=64 * 40 + 5, H=H, Hkv=Hkv, d=d, topk=topk, own=own, seed=topk)
     x = make_prefill_inputs(wl, DEV)
     rep, (O, idx, w) = prefill_parity(oracle_lib, wl, x)
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    expect_tc_path(rep.kernels, H // Hkv in (8, 16))
     if not own:   # no visible chunk and no own term: exactly zero
         assert torch.all(O[:, :64] == 0)
 
 
 @pytest.mark.parametrize("lm_kind", ["dhsa", "f32"])
-def test_prefill_landmark_modes(oracle_lib, lm_kind):
-    wl = small("bf16", B=2, L=64 * 9 + 31, lm="dhsa" if lm_kind == "dhsa" else "input")
+@pytest.mark.parametrize("H,Hkv", [(8, 2), (16, 2)])
+def test_prefill_landmark_modes(oracle_lib, lm_kind, H, Hkv):
+    wl = small("bf16", B=2, L=64 * 9 + 31, H=H, Hkv=Hkv,
+               lm="dhsa" if lm_kind == "dhsa" else "input")
     x = make_prefill_inputs(wl, DEV)
     lm = None if lm_kind == "dhsa" else x["lm"].float()
     rep, _ = prefill_parity(oracle_lib, wl, x, lm_override=lm)
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    expect_tc_path(rep.kernels, H // Hkv == 8)
+    assert bool(rep.kernels & B.K_LANDMARKS) == (lm_kind == "dhsa")
 
 
 @pytest.mark.parametrize("seed", [5, 11, 23])
@@ -118,33 +149,60 @@ def test_prefill_large_outputs(oracle_lib, seed):
 
 
 @pytest.mark.parametrize("tiles", ["one", "multi"])
-@pytest.mark.parametrize("lm_kind", ["bf16", "f32"])
-def test_prefill_selection_kernels(oracle_lib, monkeypatch, tiles, lm_kind):
-    # Up to 128 chunks the tensor-core selection builds qbar per 64-column
-    # block (two blocks per SM); HSA_SELECT_TILES=multi keeps the multi-tile
-    # kernel, so both kernels see the same shapes here.
-    if tiles == "multi":
-        monkeypatch.setenv("HSA_SELECT_TILES", "multi")
-    wl = small("bf16", B=2, L=64 * 33 + 17, topk=8, seed=41)
+@pytest.mark.parametrize("lm_kind", ["bf16", "f32", "dhsa"])
+@pytest.mark.parametrize("H,Hkv", [(16, 2), (16, 1)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_tc_selection_branches(oracle_lib, tiles, lm_kind, H, Hkv, d):
+    # Every tensor-core selection kernel the dispatch can launch, element by
+    # element: one score tile (up to 128 chunks; qbar built per 64-column
+    # block, two blocks per SM) and the multi-tile kernel (forced here on the
+    # same shape), each with bf16 landmarks (3 qbar parts), fp32 landmarks
+    # split into two bf16 planes (2 x 2 parts) and the DHSA landmarks computed
+    # on the device (fp32, same split), at d = 64 and 128 and G = 8 and 16.
+    wl = small("bf16", B=2, L=64 * 33 + 17, H=H, Hkv=Hkv, d=d, topk=8, seed=41 + d + H // Hkv)
     x = make_prefill_inputs(wl, DEV)
-    lm = x["lm"].float() if lm_kind == "f32" else None
-    rep, _ = prefill_parity(oracle_lib, wl, x, lm_override=lm)
+    lm = {"bf16": x["lm"], "f32": x["lm"].float() * 1.25, "dhsa": None}[lm_kind]
+    flags = B.PATH_MULTI_TILE_SELECT if tiles == "multi" else 0
+    with hsa.path_overrides(flags):
+        rep, _ = prefill_parity(oracle_lib, wl, x, lm_override=lm)
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    expect_tc_path(rep.kernels, True)
+    want = B.K_SELECT_TC_MULTI_TILE if tiles == "multi" else B.K_SELECT_TC_ONE_TILE
+    assert rep.kernels & want, hex(rep.kernels)
+    assert bool(rep.kernels & B.K_SPLIT_LANDMARKS) == (lm_kind != "bf16")
 
 
-@pytest.mark.parametrize("topk", [3, 17, 32])
+@pytest.mark.parametrize("lm_kind", ["bf16", "f32", "dhsa"])
+@pytest.mark.parametrize("H,Hkv,d", [(16, 2, 128), (16, 1, 64)])
+def test_prefill_tc_selection_above_one_tile(oracle_lib, lm_kind, H, Hkv, d):
+    # 150 chunks: the multi-tile kernel is the dispatch's own choice; every
+    # landmark mode, sampled rows including the chunks next to the tile edge.
+    wl = small("bf16", B=1, L=64 * 150 + 7, H=H, Hkv=Hkv, d=d, topk=8, seed=300 + d)
+    x = make_prefill_inputs(wl, DEV)
+    lm = {"bf16": x["lm"], "f32": x["lm"].float(), "dhsa": None}[lm_kind]
+    rng = np.random.default_rng(d)
+    edges = np.concatenate([np.arange(c * 64 - 2, c * 64 + 3) for c in (1, 127, 128, 129, 149)])
+    rows = np.unique(np.concatenate([rng.integers(0, wl.L, 500), edges, np.arange(wl.L - 70, wl.L)]))
+    rep, _ = prefill_parity(oracle_lib, wl, x, rows=rows, lm_override=lm)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    assert rep.kernels & B.K_SELECT_TC_MULTI_TILE, hex(rep.kernels)
+    expect_tc_path(rep.kernels, True)
+
+
+@pytest.mark.parametrize("topk", [1, 3, 17, 32])
 @pytest.mark.parametrize("tiles", ["one", "multi"])
-def test_prefill_tc_selection_topk(oracle_lib, monkeypatch, topk, tiles):
+def test_prefill_tc_selection_topk(oracle_lib, topk, tiles):
     # The tensor-core selection (G = 8) at each compiled list length (8, 16 and
     # 32 keys) in both kernels (the multi-tile kernel splits the top-K between
     # two warp groups over alternate 32-chunk column blocks and merges their
     # lists per token).
-    if tiles == "multi":
-        monkeypatch.setenv("HSA_SELECT_TILES", "multi")
     wl = small("bf16", B=1, L=64 * 40 + 5, H=16, Hkv=2, topk=topk, seed=100 + topk)
     x = make_prefill_inputs(wl, DEV)
-    rep, _ = prefill_parity(oracle_lib, wl, x)
+    with hsa.path_overrides(B.PATH_MULTI_TILE_SELECT if tiles == "multi" else 0):
+        rep, _ = prefill_parity(oracle_lib, wl, x)
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    want = B.K_SELECT_TC_MULTI_TILE if tiles == "multi" else B.K_SELECT_TC_ONE_TILE
+    assert rep.kernels & want, hex(rep.kernels)
 
 
 @pytest.mark.parametrize("topk", [8, 32])
@@ -163,15 +221,31 @@ def test_prefill_tc_selection_many_tiles(oracle_lib, topk):
 
 
 @pytest.mark.parametrize("H,Hkv", [(8, 1), (16, 1)])
-def test_prefill_several_windows(oracle_lib, monkeypatch, H, Hkv):
+def test_prefill_several_windows(oracle_lib, H, Hkv):
     # Long sequences split the work lists into token windows (a window's query
     # rows should stay in L2); 512-token windows force that path on a small
     # shape: several windows per (b, g), ragged last one.
-    monkeypatch.setenv("HSA_TC_WINDOW", "512")
     wl = small("bf16", B=2, L=64 * 37 + 29, H=H, Hkv=Hkv, topk=8, seed=77)
     x = make_prefill_inputs(wl, DEV)
-    rep, _ = prefill_parity(oracle_lib, wl, x)
+    with hsa.path_overrides(0, 512):
+        rep, _ = prefill_parity(oracle_lib, wl, x)
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+    expect_tc_path(rep.kernels, True)
+
+
+def test_prefill_simt_overrides_match_oracle(oracle_lib):
+    # The CUDA-core prefill and the CUDA-core selection, forced on a shape the
+    # tensor cores would take: both still match the oracle.
+    wl = small("bf16", B=1, L=64 * 20 + 3, H=16, Hkv=2, topk=8, seed=51)
+    x = make_prefill_inputs(wl, DEV)
+    with hsa.path_overrides(B.PATH_SIMT_PREFILL):
+        rep, _ = prefill_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary()
+    expect_tc_path(rep.kernels, False)
+    with hsa.path_overrides(B.PATH_SIMT_SELECT):
+        rep, _ = prefill_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary()
+    assert rep.kernels & B.K_SELECT_SIMT and rep.kernels & B.K_ATTEND_TC, hex(rep.kernels)
 
 
 def test_bounded_wait_expiry_is_reported_and_context_survives(oracle_lib):
@@ -179,7 +253,6 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(oracle_lib):
     # purpose (a wait that nothing completes, ~1 ms): the status word is
     # flagged, hsa.check reports the timeout once, and the same context then
     # runs the prefill path with parity.
-    from hierarchical_chunk_sparse_landmark_b200 import _binding as B
     ws = torch.zeros(4096, dtype=torch.uint8, device=DEV)
     hsa.selftest_wait_expiry(ws, budget_cycles=2_000_000)
     with pytest.raises(hsa.HSAError) as e:
