@@ -2,21 +2,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-decode] [--no-e2e] [--no-cpu-baseline]
-                    [--decode-workload NAME]
+                    [--no-extra] [--decode-workload NAME]
 
-One step = one full hsa_prefill call (landmarks when DHSA, selection, work
-list, in-chunk attention, fusion, own-chunk term) over one batch of the
-workload, inputs resident in HBM.  ``value`` is algorithmic TFLOP/s summed
-over ranks / max-over-ranks device time (weak scaling: every rank runs its own
-independent batch, seeded by rank; no collective on the data path).  The same
-JSON line carries the 32M-context decode figure (tokens/s and HBM roofline),
-the roofline of the dominant kernel timed live with CUDA events on the
-launching stream (FLOP/s against the bf16 peak, and its chunk-output DRAM
-writes against the write-only HBM bandwidth measured in the run), the
-landmark kernel's HBM roofline for DHSA workloads, an end-to-end figure
-through host buffers, the SM clocks sampled during the timed region and the
-fp64 CPU oracle timed on a bounded sample of the same workload.
+One step = one full hsa_prefill call (DHSA landmarks, selection, work lists,
+in-chunk attention, fusion, own-chunk term) over one batch of the workload,
+inputs resident in HBM.  The main line is the largest single-GPU prefill
+workload (L = 131072, DHSA landmarks computed on the device, planted needle
+chunks).  ``value`` is algorithmic TFLOP/s summed over ranks / max-over-ranks
+device time (weak scaling: every rank runs its own independent batch, seeded
+by rank; no collective on the data path).
 
+The same JSON line carries: the roofline of the dominant kernel timed live
+with CUDA events on the launching stream; the landmark kernel's HBM roofline;
+an end-to-end figure through host buffers; the SM clocks sampled during the
+timed region; the fp64 CPU oracle timed on a bounded sample of the same
+workload, whose rows double as a parity sample of the GPU's outputs (near-ties
+counted); the train-shape bf16 and the fp32 prefill workloads, each with its
+roofline (tensor-core bf16 peak, resp. the FP32 CUDA-core peak); and the
+32M-context and batched decode lines (tokens/s, HBM roofline, parity of every
+sequence against the oracle).
+
+``--gpus N`` without a launcher starts N ranks itself (one process per GPU).
 ``--impl reference`` times the fp64 CPU oracle (the only reference for this
 method) on the host cores, each step a bounded sample of the workload.
 """
@@ -192,26 +198,6 @@ def measured_traffic(kernel: str, src_files, key: str = "dram_bytes_per_launch",
     return d.get(key)
 
 
-def hbm_write_gbs(dev, gib: int = 1, reps: int = 5) -> float:
-    """Write-only HBM bandwidth of this GPU: a 1 GiB fill (8x L2), CUDA events.
-    A kernel whose DRAM traffic is mostly writes is bound by this, not by the
-    read + write copy bandwidth of the peaks file."""
-    import torch
-    buf = torch.empty(gib << 30, dtype=torch.uint8, device=dev)
-    for _ in range(2):
-        buf.fill_(1)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(reps):
-        buf.fill_(1)
-    b.record()
-    torch.cuda.synchronize()
-    gbs = reps * buf.numel() / (a.elapsed_time(b) / 1e3) / 1e9
-    del buf
-    torch.cuda.empty_cache()
-    return gbs
-
-
 # ----------------------------------------------------------------------------- dist
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -235,38 +221,48 @@ def aggregate(dist, value_units: float, seconds: float, device=None):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_ours(args, dist, rank, world):
+METRIC = "HSA prefill TFLOP/s + 32M-ctx decode tokens/s (% of B200 roofline)"
+ATTN_SRC = "hierarchical_chunk_sparse_landmark_b200/csrc/"
+
+
+def fp32_simt_peak_tflops(peaks) -> float:
+    """FP32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x the
+    maximum SM clock (1965 MHz on these GPUs) = 74.4 TFLOP/s."""
+    return SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+
+
+def bench_prefill(args, name, dev, peaks, rank, dist, steps, warmup, keep_inputs=False):
+    """Time hsa_prefill on one workload: `steps` timed calls after `warmup`,
+    L2 flushed between calls (outside the events).  Returns the line's figures
+    (and the device inputs and one call's outputs when keep_inputs)."""
     import torch
 
     import hierarchical_chunk_sparse_landmark_b200 as hsa
-    from hierarchical_chunk_sparse_landmark_b200.workloads import (WORKLOADS,
-                                                                   make_decode_inputs,
-                                                                   make_prefill_inputs)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    peaks = load_peaks()
-    wl = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_prefill_inputs
+    wl = WORKLOADS[name].with_(seed=WORKLOADS[name].seed + rank)
     x = make_prefill_inputs(wl, dev)
     flops = prefill_flops(wl)
     out = torch.empty_like(x["Q"])
     ws = hsa.workspace(hsa.prefill_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S,
                                                   wl.topk), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    # timed steps record only the events the roofline needs (step start, both
-    # sides of the attention kernel, step end): an event between two kernels
+    # timed steps record only the events the roofline needs (call start, both
+    # sides of the attention kernel, call end): an event between two kernels
     # ends their programmatic launch overlap.  The stage breakdown comes from a
-    # few extra steps with an event at every stage boundary.
-    timed_ev = [make_events(4) for _ in range(args.steps)]
-    n_brk = min(3, args.steps)
+    # few extra calls with an event at every stage boundary.
+    timed_ev = [make_events(4) for _ in range(steps)]
+    n_brk = min(3, steps)
     stage_ev = [make_events(6) for _ in range(n_brk)]
 
     def step():
         hsa.prefill(x["Q"], x["K"], x["V"], x["lm"], S=wl.S, topk=wl.topk,
                     own_chunk=wl.own_chunk, out=out, ws=ws)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
         flush.fill_(1)
     hsa.check(ws)
+    kernels = hsa.last_call_kernels()
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -277,7 +273,7 @@ def run_ours(args, dist, rank, world):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(uuid) as clk:
-        for i in range(args.steps):
+        for i in range(steps):
             e = timed_ev[i]
             hsa.set_stage_events([e[0], None, None, e[1], e[2], e[3]])
             step()
@@ -298,74 +294,110 @@ def run_ours(args, dist, rank, world):
     step_ms = [e[0].elapsed_time(e[3]) for e in timed_ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in timed_ev]
     fuse_ms = [e[2].elapsed_time(e[3]) for e in timed_ev]
-    sel_ms = [e[1].elapsed_time(e[2]) for e in stage_ev]
-    lm_ms = [e[0].elapsed_time(e[1]) for e in stage_ev]
-    bkt_ms = [e[2].elapsed_time(e[3]) for e in stage_ev]
     total_s = sum(step_ms) / 1e3
-    units, tmax = aggregate(dist, flops["total"] * args.steps / 1e12, total_s, dev)
-    value = units / tmax
-    clocks = clk.summary()
-
+    units, tmax = aggregate(dist, flops["total"] * steps / 1e12, total_s, dev)
+    tc_path = bool(kernels & 64)                     # HSA_K_ATTEND_TC
     attn_s = statistics.mean(attn_ms) / 1e3
-    attn_tf = flops["attention_kernel"] / attn_s / 1e12
-    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    tc_path = wl.dtype == "bf16" and wl.G in (8, 16) and wl.d in (64, 128)
-    attn_files = ["hierarchical_chunk_sparse_landmark_b200/csrc/" +
-                  ("attend_tc.cu" if tc_path else "attend_simt.cu")]
-    kname = "attend_tc_kernel" if tc_path else "attend_simt_kernel"
-    kfile = attn_files[0].rsplit("/", 1)[1][:-3]
-    roofline = {"kernel": kname, "bound": "tensor", "achieved": round(attn_tf, 3),
-                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 5),
-                "traffic": measured_traffic(kfile, attn_files, workload=wl.name),
-                "peak_source": peaks["source"] + " bf16 burst",
-                "algorithmic_flops_per_launch": flops["attention_kernel"],
-                "ms_per_launch": round(attn_s * 1e3, 4)}
-    # What the kernel actually runs into: the DRAM write-back of its chunk
-    # outputs (design traffic, not algorithmic), against the write-only HBM
-    # bandwidth measured here.
-    wbytes = measured_traffic(kfile, attn_files, "dram_write_bytes_per_launch", workload=wl.name)
-    if tc_path and wbytes:
-        wpeak = hbm_write_gbs(dev)
-        wach = wbytes / attn_s / 1e9
-        roofline["dram_write"] = {"bytes_per_launch": wbytes, "achieved": round(wach, 1),
-                                  "peak": round(wpeak, 1), "unit": "GB/s",
-                                  "frac": round(wach / wpeak, 4),
-                                  "peak_source": "write-only HBM bandwidth measured in this run "
-                                                 "(1 GiB fill)"}
+    kfile = "attend_tc" if tc_path else "attend_simt"
+    files = [ATTN_SRC + kfile + ".cu"]
+    if tc_path:
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        kflops = flops["attention_kernel"]
+        roofline = {"kernel": "attend_tc_kernel", "bound": "tensor",
+                    "peak_source": peaks["source"] + " bf16 burst"}
+        stage = {"landmarks": round(statistics.mean(e[0].elapsed_time(e[1]) for e in stage_ev), 4),
+                 "selection": round(statistics.mean(e[1].elapsed_time(e[2]) for e in stage_ev), 4),
+                 "work_list": round(statistics.mean(e[2].elapsed_time(e[3]) for e in stage_ev), 4),
+                 "attention": round(statistics.mean(attn_ms), 4),
+                 "fusion": round(statistics.mean(fuse_ms), 4),
+                 "note": "attention and fusion from the timed calls; landmarks, selection and "
+                         "work lists from %d extra calls with an event at every stage "
+                         "boundary" % n_brk}
+    else:
+        # fp32 path: selection and attention+fusion on CUDA cores; the
+        # attention kernel fuses in place, so the whole call is the unit
+        peak = fp32_simt_peak_tflops(peaks)
+        kflops = flops["total"]
+        attn_s = statistics.mean(step_ms) / 1e3
+        roofline = {"kernel": "select_kernel + attend_simt_kernel (whole call)", "bound": "alu",
+                    "peak_source": "FP32 CUDA-core peak: 148 SMs x 128 lanes x 2 flop x "
+                                   "%.0f MHz" % peaks.get("sm_max_mhz", 1965.0)}
+        stage = None
+    ach = kflops / attn_s / 1e12
+    roofline.update({"achieved": round(ach, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(ach / peak, 5),
+                     "traffic": measured_traffic(kfile, files, workload=wl.name),
+                     "algorithmic_flops_per_launch": kflops,
+                     "ms_per_launch": round(attn_s * 1e3, 4)})
+    res = {"workload": wl.name, "value": round(units / tmax, 4), "unit": "TFLOP/s",
+           "ms_per_step": round(tmax * 1e3 / steps, 4), "steps": steps,
+           "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "Hkv": wl.Hkv,
+                      "d": wl.d, "S": wl.S, "topk": wl.topk, "own_chunk": wl.own_chunk,
+                      "landmarks": wl.landmarks, "dtype": wl.dtype},
+           "roofline": roofline, "clocks": clk.summary(), "gpu_launches": launches,
+           "flops_per_step": flops}
+    if stage is not None:
+        res["stage_ms"] = stage
+    extra = None
+    if keep_inputs:
+        O, idx, _ = hsa.prefill(x["Q"], x["K"], x["V"], x["lm"], S=wl.S, topk=wl.topk,
+                                own_chunk=wl.own_chunk, idx_out=True, ws=ws)
+        hsa.check(ws)
+        extra = {"wl": wl, "x": x, "O": O, "idx": idx, "ws": ws}
+    else:
+        del x, out
+    del flush
+    torch.cuda.empty_cache()
+    return res, extra
 
+
+def run_ours(args, dist, rank, world):
+    import torch
+
+    import hierarchical_chunk_sparse_landmark_b200 as hsa
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    main, keep = bench_prefill(args, args.workload, dev, peaks, rank, dist, args.steps,
+                               args.warmup, keep_inputs=True)
+    wl, x = keep["wl"], keep["x"]
     res = {
-        "metric": "HSA prefill TFLOP/s (train-shape workload) + 32M-ctx decode tokens/s",
-        "value": round(value, 4), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(tmax * 1e3 / args.steps, 4),
+        "metric": METRIC,
+        "value": main["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (seeded N(0,1), per-rank seed)",
-        "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "Hkv": wl.Hkv,
-                   "d": wl.d, "S": wl.S, "topk": wl.topk, "own_chunk": wl.own_chunk,
-                   "landmarks": wl.landmarks, "parallelism": f"independent batches x{world}",
-                   "l2": "flushed between timed steps (256 MiB write)"},
-        "stage_ms": {"landmarks": round(statistics.mean(lm_ms), 4),
-                     "selection": round(statistics.mean(sel_ms), 4),
-                     "work_list": round(statistics.mean(bkt_ms), 4),
-                     "attention": round(statistics.mean(attn_ms), 4),
-                     "fusion": round(statistics.mean(fuse_ms), 4),
-                     "note": "attention and fusion from the timed steps; landmarks, selection "
-                             "and work lists from %d extra steps with an event at every stage "
-                             "boundary" % n_brk},
-        "flops_per_step": flops,
-        "roofline": roofline, "clocks": clocks, "gpu_launches": launches,
+        "config": dict(main["config"], parallelism=f"independent batches x{world}",
+                       l2="flushed between timed steps (256 MiB write)"),
+        "stage_ms": main.get("stage_ms"),
+        "flops_per_step": main["flops_per_step"],
+        "roofline": main["roofline"], "clocks": main["clocks"], "gpu_launches": main["gpu_launches"],
     }
-
     if wl.landmarks == "dhsa":
         res["landmarks_roofline"] = landmark_roofline(hsa, wl, x, peaks, dev)
     if args.e2e:
-        res["e2e"] = e2e_prefill(args, wl, x, ws, dev, dist)
-    del x, out
-    torch.cuda.empty_cache()
-    if args.decode:
-        key = "decode_32m" if args.decode_workload == "decode_32m_bf16" else "decode_" + args.decode_workload
-        res[key] = bench_decode(args, dev, peaks, rank, dist)
+        res["e2e"] = e2e_prefill(args, wl, x, keep["ws"], dev, dist)
     if rank == 0 and world == 1 and args.cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(args, wl)
+        cb, par = cpu_baseline_and_parity(args, keep)
+        res["cpu_baseline"] = cb
+        res["parity"] = par
+    del keep, x
+    torch.cuda.empty_cache()
+    if args.extra:
+        for name, key in (("train_prefill_bf16", "train_prefill"),
+                          ("tiny_prefill_f32", "tiny_prefill_f32")):
+            if name != args.workload:
+                r, _ = bench_prefill(args, name, dev, peaks, rank, dist, max(5, args.steps // 2), 3)
+                r.pop("flops_per_step", None)
+                res[key] = r
+    if args.decode:
+        names = [args.decode_workload]
+        if args.extra and "batched_decode_bf16" not in names:
+            names.append("batched_decode_bf16")
+        for name in names:
+            key = "decode_32m" if name == "decode_32m_bf16" else \
+                "decode_batched" if name == "batched_decode_bf16" else "decode_" + name
+            res[key] = bench_decode(args, name, dev, peaks, rank, dist,
+                                    parity=(rank == 0 and world == 1 and args.cpu_baseline))
     return res
 
 
@@ -427,6 +459,10 @@ def e2e_prefill(args, wl, x, ws, dev, dist):
             "in": torch.cuda.Event(), "comp": torch.cuda.Event(), "out": torch.cuda.Event()})
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     steps = max(4, args.steps // 2)
+    # one workspace per compute stream (the binding caches them per stream)
+    with torch.cuda.stream(s_comp):
+        ws = hsa.workspace(hsa.prefill_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S,
+                                                      wl.topk), dev)
 
     def issue(i):
         sl = slots[i % 2]
@@ -466,18 +502,20 @@ def e2e_prefill(args, wl, x, ws, dev, dist):
     flops = prefill_flops(wl)["total"]
     units, tmax = aggregate(dist, flops * steps / 1e12, secs, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV) + ((hlm,) if hlm is not None else ()))
+    del slots
+    torch.cuda.empty_cache()
     return {"value": round(units / tmax, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": slots[0]["hO"].numel() * slots[0]["hO"].element_size(),
+            "d2h_bytes_per_step": int(x["Q"].numel() * x["Q"].element_size()),
             "steps": steps, "ms_per_step": round(tmax * 1e3 / steps, 4),
             "pipeline": "2 buffer slots; host->device, compute and device->host on separate streams"}
 
 
-def bench_decode(args, dev, peaks, rank, dist):
+def bench_decode(args, name, dev, peaks, rank, dist, parity=False):
     import torch
 
     import hierarchical_chunk_sparse_landmark_b200 as hsa
     from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_decode_inputs
-    wl = WORKLOADS[args.decode_workload].with_(seed=rank)
+    wl = WORKLOADS[name].with_(seed=rank)
     x = make_decode_inputs(wl, dev)
     out = torch.empty_like(x["q"])
     ws = hsa.workspace(hsa.decode_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S, wl.topk),
@@ -505,16 +543,23 @@ def bench_decode(args, dev, peaks, rank, dist):
     per = secs / steps
     gbs = nbytes / per / 1e9
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    del x
+    files = [ATTN_SRC + "decode.cu"]
+    traffic = measured_traffic("decode", files, workload=wl.name)
+    res = {"workload": wl.name, "value": round(toks / tmax, 2), "unit": "tokens/s",
+           "ms_per_step": round(per * 1e3, 4), "steps": steps,
+           "roofline": {"kernel": "decode_scan_kernel + decode_attend_kernel (whole call)",
+                        "bound": "hbm", "achieved": round(gbs, 1),
+                        "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                        "traffic": traffic, "algorithmic_bytes_per_launch": nbytes,
+                        "peak_source": peaks["source"] + " copy bandwidth"},
+           "l2": "no flush: inputs (256 MiB of landmarks) larger than L2, calls back to back"}
+    if parity:
+        O, idx = hsa.decode(x["q"], x["K"], x["V"], x["lm"], topk=wl.topk, idx_out=True, ws=ws)
+        hsa.check(ws)
+        res["parity"] = decode_parity_sample(wl, x, O, idx)
+    del x, out
     torch.cuda.empty_cache()
-    return {"workload": wl.name, "value": round(toks / tmax, 2), "unit": "tokens/s",
-            "ms_per_step": round(per * 1e3, 4), "steps": steps,
-            "roofline": {"kernel": "decode_scan_kernel + decode_attend_kernel (whole call)",
-                         "bound": "hbm", "achieved": round(gbs, 1),
-                         "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-                         "traffic": None, "algorithmic_bytes_per_launch": nbytes,
-                         "peak_source": peaks["source"] + " copy bandwidth"},
-            "l2": "no flush: inputs (256 MiB of landmarks) larger than L2, calls back to back"}
+    return res
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -533,35 +578,105 @@ def sample_flops(wl, rows) -> float:
                   + H * 4 * d * own).sum())
 
 
+def _host_f64(t):
+    import torch
+    return None if t is None else t.detach().to("cpu").to(torch.float64).numpy()
+
+
 def cpu_baseline(args, wl, budget_s: float = 12.0, x_host=None):
     """Time the fp64 oracle, as it stands, on the host cores over a bounded
-    sample of rows of the same workload; throughput in the same unit."""
+    sample of rows of the same workload; throughput in the same unit.
+    ``x_host`` may hold the inputs (numpy float64 K, V, lm and a torch Q on any
+    device, of which only the sampled rows are copied).  Returns the figure
+    and the oracle's results for the first sample (rows, outputs)."""
     import torch
 
     import oracle
     from hierarchical_chunk_sparse_landmark_b200.workloads import make_prefill_inputs
     orc = oracle.Oracle()
-    x = x_host if x_host is not None else make_prefill_inputs(wl, "cpu")
-    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
-    K, V, lm = f64(x["K"]), f64(x["V"]), f64(x["lm"])
-    Qall = x["Q"].reshape(wl.B * wl.L, wl.H, wl.d)
+    if x_host is None:
+        x = make_prefill_inputs(wl, "cpu")
+        x_host = {"K": _host_f64(x["K"]), "V": _host_f64(x["V"]), "lm": _host_f64(x["lm"]),
+                  "Q": x["Q"]}
+    K, V, lm = x_host["K"], x_host["V"], x_host["lm"]
+    Qall = x_host["Q"].reshape(wl.B * wl.L, wl.H, wl.d)
     n = 256
     total_f, total_s, total_rows, it = 0.0, 0.0, 0, 0
+    first = None
     while total_s < budget_s:
         rows = oracle_sample_rows(wl, n, seed=it)
         it += 1
-        Qr = f64(Qall[torch.as_tensor(rows)])
+        Qr = _host_f64(Qall[torch.as_tensor(rows, device=Qall.device)])
         t0 = time.perf_counter()
-        orc.prefill(None, K, V, lm, wl.S, wl.topk, wl.own_chunk, rows=rows, Q_rows=Qr)
+        r = orc.prefill(None, K, V, lm, wl.S, wl.topk, wl.own_chunk, rows=rows, Q_rows=Qr)
         dt = time.perf_counter() - t0
+        if first is None:
+            first = (rows, Qr, r)
         total_f += sample_flops(wl, rows)
         total_s += dt
         total_rows += len(rows)
         n = min(4 * n, 8192)
-    return {"value": round(total_f / total_s / 1e12, 6), "unit": "TFLOP/s",
+    info = {"value": round(total_f / total_s / 1e12, 6), "unit": "TFLOP/s",
             "cores": orc.num_threads(), "kind": "oracle",
             "sample": f"{total_rows} random rows (all heads) of {wl.name}, fp64 C/OpenMP oracle",
             "seconds": round(total_s, 2)}
+    return info, first
+
+
+def cpu_baseline_and_parity(args, keep):
+    """The oracle timed on the host cores (cpu_baseline) on the very inputs the
+    GPU read, copied back; the rows of its first sample then double as a
+    parity sample of the GPU call made outside the timed region: selection
+    compared set by set (near-ties counted, their outputs recomputed on the
+    GPU's selection), O within the workload dtype's tolerance."""
+    import torch
+
+    import oracle
+    from oracle.parity import ATOL, ParityReport, compare_outputs, compare_selection
+    wl, x = keep["wl"], keep["x"]
+    xh = {"K": _host_f64(x["K"]), "V": _host_f64(x["V"]), "lm": _host_f64(x["lm"]), "Q": x["Q"]}
+    info, (rows, Qr, ref) = cpu_baseline(args, wl, x_host=xh)
+    rt = torch.as_tensor(rows, device=keep["O"].device)
+    got_idx = keep["idx"].reshape(wl.B * wl.L, wl.Hkv, wl.topk)[rt].cpu().numpy()
+    got_O = _host_f64(keep["O"].reshape(wl.B * wl.L, wl.H, wl.d)[rt])
+    rep = ParityReport(rows=len(rows))
+    differs = compare_selection(ref["idx"], ref["sbar"], ref["gap"], ref["smag"], got_idx, rep)
+    ref_O = ref["O"]
+    if differs.any():
+        sel = np.where(differs.any(axis=1))[0]
+        forced = oracle.Oracle().prefill(None, xh["K"], xh["V"], xh["lm"], wl.S, wl.topk,
+                                         wl.own_chunk, rows=rows[sel], Q_rows=Qr[sel],
+                                         forced_idx=got_idx[sel])
+        ref_O = ref_O.copy()
+        ref_O[sel] = forced["O"]
+    compare_outputs(ref_O, got_O, ATOL[wl.dtype], rep)
+    par = {"workload": wl.name, "rows": int(len(rows)), "groups": int(len(rows) * wl.Hkv),
+           "near_ties": rep.near_ties, "set_mismatch": rep.set_mismatch,
+           "order_mismatch": rep.order_mismatch, "max_abs_err": float(f"{rep.max_abs_err:.4g}"),
+           "atol": ATOL[wl.dtype], "ok": rep.ok,
+           "how": "first sample of the cpu_baseline rows, GPU call outside the timed region"}
+    return info, par
+
+
+def decode_parity_sample(wl, x, O, idx):
+    """Every sequence of a decode workload against the oracle (the oracle
+    scans all landmarks and attends over the chunks it selects)."""
+    import oracle
+    from oracle import gather_chunks
+    from oracle.parity import ATOL, ParityReport, compare_outputs, compare_selection
+    orc = oracle.Oracle()
+    q, lm = _host_f64(x["q"]), _host_f64(x["lm"])
+    sel = orc.decode_select(q, lm, wl.topk)
+    got = idx.cpu().numpy()
+    rep = ParityReport(rows=wl.B)
+    differs = compare_selection(sel["idx"], sel["sbar"], sel["gap"], sel["smag"], got, rep)
+    use = np.where(differs[:, :, None], got, sel["idx"])
+    ref = orc.decode_attend(q, lm, gather_chunks(x["K"], use, wl.S), gather_chunks(x["V"], use, wl.S),
+                            use, wl.S)
+    compare_outputs(ref["O"], _host_f64(O), ATOL[wl.dtype], rep)
+    return {"sequences": wl.B, "groups": wl.B * wl.Hkv, "near_ties": rep.near_ties,
+            "set_mismatch": rep.set_mismatch, "order_mismatch": rep.order_mismatch,
+            "max_abs_err": float(f"{rep.max_abs_err:.4g}"), "atol": ATOL[wl.dtype], "ok": rep.ok}
 
 
 def run_reference(args, rank, world):
@@ -571,45 +686,91 @@ def run_reference(args, rank, world):
         return None
     wl = WORKLOADS[args.workload]
     x = make_prefill_inputs(wl, "cpu")
+    xh = {"K": _host_f64(x["K"]), "V": _host_f64(x["V"]), "lm": _host_f64(x["lm"]), "Q": x["Q"]}
     per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(args, wl, budget_s=per_step_budget / 4, x_host=x)
+        cpu_baseline(args, wl, budget_s=per_step_budget / 4, x_host=xh)
     vals, secs = [], 0.0
     info = None
     for _ in range(args.steps):
-        info = cpu_baseline(args, wl, budget_s=per_step_budget, x_host=x)
+        info, _ = cpu_baseline(args, wl, budget_s=per_step_budget, x_host=xh)
         vals.append(info["value"])
         secs += info["seconds"]
     value = statistics.mean(vals)
-    return {"impl": "reference", "metric": "HSA prefill TFLOP/s (train-shape workload) "
-            "+ 32M-ctx decode tokens/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup,
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(secs * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "Hkv": wl.Hkv,
-                       "d": wl.d, "S": wl.S, "topk": wl.topk},
+                       "d": wl.d, "S": wl.S, "topk": wl.topk, "own_chunk": wl.own_chunk,
+                       "landmarks": wl.landmarks, "dtype": wl.dtype,
+                       "parallelism": f"independent batches x{world}",
+                       "l2": "not applicable (host)"},
             "cpu_baseline": {"kind": "oracle", "cores": info["cores"], "sample": info["sample"],
                              "value": value, "unit": "TFLOP/s"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------- launch
+def free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def launch_ranks(n: int, cmd: list, env: dict | None = None, timeout_s: float = 3600.0) -> int:
+    """Start `cmd` as n ranks of one job on this node (RANK, LOCAL_RANK,
+    WORLD_SIZE, MASTER_ADDR=127.0.0.1 and a free MASTER_PORT in each rank's
+    environment), the way torchrun does; rank 0's output is passed through,
+    the others' stdout is dropped.  Returns the worst exit code."""
+    base = dict(os.environ if env is None else env)
+    base.update(WORLD_SIZE=str(n), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(free_port()))
+    procs = []
+    for r in range(n):
+        e = dict(base, RANK=str(r), LOCAL_RANK=str(r))
+        procs.append(subprocess.Popen(cmd, env=e, stdout=None if r == 0 else subprocess.DEVNULL))
+    deadline = time.time() + timeout_s
+    rcs = []
+    for p in procs:
+        try:
+            rcs.append(p.wait(timeout=max(1.0, deadline - time.time())))
+        except subprocess.TimeoutExpired:
+            p.kill()
+            rcs.append(124)
+    return max((abs(rc) for rc in rcs), default=0)
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="train_prefill_bf16")
+    ap.add_argument("--workload", default="long_prefill_bf16",
+                    help="prefill workload of the main line (long_prefill_bf16, the largest "
+                         "single-GPU prefill; train_prefill_bf16; tiny_prefill_f32)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-extra", dest="extra", action="store_false",
+                    help="leave out the lines of the other workloads (train-shape and fp32 "
+                         "prefill, batched decode)")
     ap.add_argument("--decode-workload", default="decode_32m_bf16",
                     help="decode workload of the decode line (decode_32m_bf16, batched_decode_bf16)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU, started here when no launcher did it
+        return launch_ranks(args.gpus, [sys.executable, os.path.abspath(__file__), *argv])
     world, rank, local = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)

@@ -107,7 +107,7 @@ WORKLOADS = {
 }
 
 # The workload the prefill throughput figure is quoted on.
-PRIMARY_WORKLOAD = "train_prefill_bf16"
+PRIMARY_WORKLOAD = "long_prefill_bf16"
 
 
 def storage_dtype(wl: Workload) -> torch.dtype:

@@ -43,9 +43,9 @@ def _bind(lib):
     i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
     lib.hsa_oracle_landmarks.argtypes = [dp, i32, i32, i64, i32, i32, dp]
     lib.hsa_oracle_prefill.argtypes = [dp, i64p, i64, dp, dp, dp, i32, i32, i32, i64, i32, i32,
-                                       i32, i32, dbl, i32p, dp, i32p, dp, dp, dp]
+                                       i32, i32, dbl, i32p, dp, i32p, dp, dp, dp, dp]
     lib.hsa_oracle_decode_select.argtypes = [dp, dp, i32, i32, i32, i64, i32, i32, dbl, i32p,
-                                             dp, dp]
+                                             dp, dp, dp]
     lib.hsa_oracle_decode_attend.argtypes = [dp, dp, dp, dp, i32p, i32, i32, i32, i64, i32,
                                              i32, i32, dbl, dp, dp]
     for name in ("hsa_oracle_landmarks", "hsa_oracle_prefill", "hsa_oracle_decode_select",
@@ -110,7 +110,9 @@ class Oracle:
         Q [B,L,H,d] (or pass ``Q_rows`` [n,H,d] with ``rows``), K/V [B,Hkv,L,d],
         lm [B,Hkv,L//S,d] or None (DHSA landmarks from K).  ``rows`` are
         flattened positions b*L+t (default: every position).
-        Returns dict O [n,H,d], idx [n,Hkv,K], w [n,H,K], sbar [n,Hkv,K], gap [n,Hkv].
+        Returns dict O [n,H,d], idx [n,Hkv,K], w [n,H,K], sbar [n,Hkv,K], gap [n,Hkv],
+        smag [n,Hkv,K+1] (magnitudes of the selected scores' terms, then of the
+        (K+1)-th candidate's).
         """
         k, v = _f64(K), _f64(V)
         B, Hkv, L, d = k.shape
@@ -133,6 +135,7 @@ class Oracle:
         w = np.zeros((n, H, topk), dtype=np.float64)
         sbar = np.zeros((n, Hkv, topk), dtype=np.float64)
         gap = np.zeros((n, Hkv), dtype=np.float64)
+        smag = np.zeros((n, Hkv, topk + 1), dtype=np.float64)
         fi = None
         if forced_idx is not None:
             fi = np.ascontiguousarray(forced_idx, dtype=np.int32)
@@ -142,23 +145,24 @@ class Oracle:
             _dp(lmf), B, H, Hkv, L, d, S, topk, int(own_chunk), float(scale),
             None if fi is None else fi.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
             _dp(O), idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(w), _dp(sbar),
-            _dp(gap))
+            _dp(gap), _dp(smag))
         _check(rc, "prefill")
-        return {"O": O, "idx": idx, "w": w, "sbar": sbar, "gap": gap, "rows": rows}
+        return {"O": O, "idx": idx, "w": w, "sbar": sbar, "gap": gap, "smag": smag, "rows": rows}
 
     def decode_select(self, q, lm, topk: int, scale: float = 0.0):
-        """q [B,H,d], lm [B,Hkv,Nc,d] -> dict idx [B,Hkv,K], sbar, gap."""
+        """q [B,H,d], lm [B,Hkv,Nc,d] -> dict idx [B,Hkv,K], sbar, gap, smag."""
         qf, lmf = _f64(q), _f64(lm)
         B, H, d = qf.shape
         _, Hkv, Nc, _ = lmf.shape
         idx = np.zeros((B, Hkv, topk), dtype=np.int32)
         sbar = np.zeros((B, Hkv, topk), dtype=np.float64)
         gap = np.zeros((B, Hkv), dtype=np.float64)
+        smag = np.zeros((B, Hkv, topk + 1), dtype=np.float64)
         rc = self.lib.hsa_oracle_decode_select(
             _dp(qf), _dp(lmf), B, H, Hkv, Nc, d, topk, float(scale),
-            idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(sbar), _dp(gap))
+            idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(sbar), _dp(gap), _dp(smag))
         _check(rc, "decode_select")
-        return {"idx": idx, "sbar": sbar, "gap": gap}
+        return {"idx": idx, "sbar": sbar, "gap": gap, "smag": smag}
 
     def decode_attend(self, q, lm, Kg, Vg, idx, S: int, scale: float = 0.0):
         """Attention + fusion over gathered chunks Kg/Vg [B,Hkv,K,S,d] named by idx."""

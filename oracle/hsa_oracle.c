@@ -80,6 +80,17 @@ static double dot(const double *x, const double *y, int n)
     return acc;
 }
 
+/* Magnitude of the terms of the dot product x . y: sum_j |x_j * y_j|.  A
+ * score computed in finite precision carries rounding errors relative to this
+ * sum, not to the (possibly cancelled) value of the score itself; the near-tie
+ * rule of the parity checks measures score gaps against it. */
+static double abs_dot(const double *x, const double *y, int n)
+{
+    double acc = 0.0;
+    for (int j = 0; j < n; ++j) acc += fabs(x[j] * y[j]);
+    return acc;
+}
+
 /*
  * Ordinary softmax attention of one query over n consecutive key/value rows
  * (HiLS: attention "independently with each retrieved chunk").
@@ -165,12 +176,18 @@ int hsa_oracle_landmarks(const double *k, int B, int Hkv, int64_t L, int d, int 
  *   gap        [n_rows, Hkv]        score(K-th) - score(K+1-th) of the group
  *                                   ranking, +inf when at most K chunks are
  *                                   visible, NaN with forced_idx
+ *   smag       [n_rows, Hkv, topk+1] magnitude scale * sum_j |qbar_j l_ij| of
+ *                                   the group score of each selected chunk in
+ *                                   rank order (0 padded), and in the last
+ *                                   slot that of the (K+1)-th ranked chunk
+ *                                   (0 when there is none or with forced_idx)
  */
 int hsa_oracle_prefill(const double *q, const int64_t *rows, int64_t n_rows,
                        const double *k, const double *v, const double *lm,
                        int B, int H, int Hkv, int64_t L, int d, int S, int topk,
                        int own_chunk, double scale, const int32_t *forced_idx,
-                       double *O, int32_t *idx, double *w, double *sbar, double *gap)
+                       double *O, int32_t *idx, double *w, double *sbar, double *gap,
+                       double *smag)
 {
     if (!q || !rows || !k || !v || !O) return ORACLE_BAD_ARG;
     if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || L < 1 || d < 1 || S < 1 || topk < 1)
@@ -250,6 +267,13 @@ int hsa_oracle_prefill(const double *q, const int64_t *rows, int64_t n_rows,
                     sbar[(r * Hkv + g) * topk + kk] =
                         kk < nsel ? scale * dot(qbar, lm_bg + sel[kk] * d, d) : 0.0;
             if (gap) gap[r * Hkv + g] = gap_val;
+            if (smag) {
+                double *m = smag + (r * Hkv + g) * (topk + 1);
+                for (int kk = 0; kk < topk; ++kk)
+                    m[kk] = kk < nsel ? scale * abs_dot(qbar, lm_bg + sel[kk] * d, d) : 0.0;
+                m[topk] = (!forced_idx && nvis > topk)
+                              ? scale * abs_dot(qbar, lm_bg + cand[topk].index * d, d) : 0.0;
+            }
 
             for (int h = 0; h < G; ++h) {
                 const int hh = g * G + h;
@@ -295,10 +319,12 @@ int hsa_oracle_prefill(const double *q, const int64_t *rows, int64_t n_rows,
  *   idx  [B, Hkv, topk]  (-1 padded when Nc < topk)
  *   sbar [B, Hkv, topk]  group scores of the selected chunks (may be NULL)
  *   gap  [B, Hkv]        score(K-th) - score(K+1-th), +inf if Nc <= K (may be NULL)
+ *   smag [B, Hkv, topk+1] magnitudes scale * sum_j |qbar_j l_ij| of the selected
+ *                        chunks' scores and, last, of the (K+1)-th (may be NULL)
  */
 int hsa_oracle_decode_select(const double *q, const double *lm, int B, int H, int Hkv,
                              int64_t Nc, int d, int topk, double scale,
-                             int32_t *idx, double *sbar, double *gap)
+                             int32_t *idx, double *sbar, double *gap, double *smag)
 {
     if (!q || !lm || !idx) return ORACLE_BAD_ARG;
     if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || Nc < 0 || d < 1 || topk < 1)
@@ -330,6 +356,11 @@ int hsa_oracle_decode_select(const double *q, const double *lm, int B, int H, in
             if (sbar) sbar[bg * topk + kk] = kk < nsel ? cand[kk].score : 0.0;
         }
         if (gap) gap[bg] = Nc > topk ? cand[topk - 1].score - cand[topk].score : INFINITY;
+        if (smag) {
+            double *m = smag + bg * (topk + 1);
+            for (int kk = 0; kk <= topk; ++kk)
+                m[kk] = kk < Nc ? scale * abs_dot(qbar, lm_bg + cand[kk].index * d, d) : 0.0;
+        }
         free(qbar);
         free(cand);
     }

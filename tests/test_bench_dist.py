@@ -106,3 +106,29 @@ def test_traffic_record_is_tied_to_its_workload():
     assert bench.measured_traffic("attend_tc", files, workload="long_prefill_bf16") is None
     assert bench.measured_traffic("attend_tc", files, "dram_write_bytes_per_launch",
                                   workload="long_prefill_bf16") is None
+
+
+def test_launch_ranks_starts_a_whole_job(capfd):
+    # bench.launch_ranks (what `bench.py --gpus N` does without torchrun) on a
+    # CPU stand-in for the device step: two ranks join one gloo group, the
+    # line reports n_gpus = 2 and the work summed over both ranks.
+    import json
+    import sys
+    standin = os.path.join(os.path.dirname(__file__), "_bench_rank_standin.py")
+    rc = bench.launch_ranks(2, [sys.executable, standin], timeout_s=120)
+    assert rc == 0
+    out = capfd.readouterr().out.strip().splitlines()
+    line = json.loads(out[-1])
+    assert line["n_gpus"] == 2 and line["units"] == pytest.approx(3.0)
+    assert line["seconds"] >= 0.1                   # the slower rank's time
+    assert line["value"] == pytest.approx(line["units"] / line["seconds"])
+
+
+def test_bench_main_self_launches_without_a_launcher(monkeypatch):
+    calls = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench, "launch_ranks", lambda n, cmd, **kw: calls.append((n, cmd)) or 0)
+    assert bench.main(["--gpus", "4", "--steps", "3", "--warmup", "3"]) == 0
+    n, cmd = calls[0]
+    assert n == 4 and cmd[1].endswith("bench.py") and cmd[2:] == ["--gpus", "4", "--steps", "3",
+                                                                  "--warmup", "3"]

@@ -472,3 +472,27 @@ def test_decode_gap_hand_scores(oracle_lib):
     for k, v in g["decode"]["expected_gap"].items():
         r = oracle_lib.decode_select(q, lm, int(k), scale=1.0)
         assert r["gap"][0, 0] == (np.inf if v == "inf" else v), (k, r["gap"])
+
+
+def test_score_term_magnitudes_hand_case(oracle_lib):
+    """smag: scale * sum_j |qbar_j l_ij| of each selected chunk in rank order,
+    then of the (K+1)-th ranked chunk.  Hand case with one cancelling score:
+    qbar = (1, 1); l0 = (2, -2) scores 0 from terms of magnitude 4;
+    l1 = (1, 0.5) scores 1.5 (magnitude 1.5); l2 = (0.25, 0.25) scores 0.5."""
+    S, d = 2, 2
+    lm = np.array([[[[2.0, -2.0], [1.0, 0.5], [0.25, 0.25]]]])
+    L = 8                                          # row t = 6, 7 sees all three chunks
+    Q = np.ones((1, L, 1, d))
+    K = np.zeros((1, 1, L, d))
+    r1 = oracle_lib.prefill(Q, K, K, lm, S, 1, scale=1.0, rows=np.array([7]))
+    np.testing.assert_array_equal(r1["idx"][0, 0], [1])
+    np.testing.assert_array_equal(r1["smag"][0, 0], [1.5, 0.5])
+    assert r1["gap"][0, 0] == 1.0
+    r2 = oracle_lib.prefill(Q, K, K, lm, S, 2, scale=1.0, rows=np.array([7]))
+    np.testing.assert_array_equal(r2["idx"][0, 0], [1, 2])
+    np.testing.assert_array_equal(r2["smag"][0, 0], [1.5, 0.5, 4.0])
+    assert r2["gap"][0, 0] == 0.5
+    r3 = oracle_lib.prefill(Q, K, K, lm, S, 3, scale=0.5, rows=np.array([7]))
+    np.testing.assert_array_equal(r3["smag"][0, 0], [0.75, 0.25, 2.0, 0.0])   # no 4th chunk
+    dec = oracle_lib.decode_select(np.ones((1, 1, d)), lm, 2, scale=1.0)
+    np.testing.assert_array_equal(dec["smag"][0, 0], [1.5, 0.5, 4.0])

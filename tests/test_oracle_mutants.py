@@ -44,6 +44,9 @@ MUTANTS = {
                        "gap_val = nvis > topk + 1 ? cand[topk].score - cand[topk + 1].score : INFINITY;"),
     "decode_gap_off_by_one": ("gap[bg] = Nc > topk ? cand[topk - 1].score - cand[topk].score : INFINITY;",
                               "gap[bg] = Nc > topk + 1 ? cand[topk].score - cand[topk + 1].score : INFINITY;"),
+    # near-tie scale: the magnitude of a score's terms taken as |score|
+    "score_magnitude_without_abs": ("for (int j = 0; j < n; ++j) acc += fabs(x[j] * y[j]);",
+                                    "for (int j = 0; j < n; ++j) acc += x[j] * y[j];"),
     # forced selection: chunks not visible from the row are kept
     "forced_visibility_filter_dropped": ("if (f[kk] >= 0 && f[kk] < nvis) sel[nsel++] = f[kk];",
                                          "if (f[kk] >= 0 && f[kk] < Nc) sel[nsel++] = f[kk];"),

@@ -74,7 +74,7 @@ def prefill_parity(oracle_lib, wl: Workload, x: dict, rows=None, lm_override=_WO
     rep = report or ParityReport()
     rep.kernels = kernels
     rep.rows += len(rows)
-    differs = compare_selection(ref["idx"], ref["sbar"], ref["gap"], got_idx, rep)
+    differs = compare_selection(ref["idx"], ref["sbar"], ref["gap"], ref["smag"], got_idx, rep)
     ref_O = ref["O"]
     if differs.any():   # near-ties: recompute those rows on the device's selection
         sel = np.where(differs.any(axis=1))[0]
@@ -312,7 +312,7 @@ def decode_parity(oracle_lib, wl: Workload, x: dict, report=None):
     got_idx = idx.cpu().numpy()
     rep = report or ParityReport()
     rep.rows += q.shape[0]
-    differs = compare_selection(sel["idx"], sel["sbar"], sel["gap"], got_idx, rep)
+    differs = compare_selection(sel["idx"], sel["sbar"], sel["gap"], sel["smag"], got_idx, rep)
     use = np.where(differs[:, :, None], got_idx, sel["idx"])
     Kg, Vg = gather_chunks(x["K"], use, wl.S), gather_chunks(x["V"], use, wl.S)
     ref = oracle_lib.decode_attend(q, lm, Kg, Vg, use, wl.S)

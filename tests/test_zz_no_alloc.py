@@ -50,7 +50,7 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls(oracle_lib):
         # and within the bf16 tolerance of the fp64 oracle
         rep = ParityReport(rows=wl.B)
         got = idx.cpu().numpy()
-        differs = compare_selection(sel["idx"], sel["sbar"], sel["gap"], got, rep)
+        differs = compare_selection(sel["idx"], sel["sbar"], sel["gap"], sel["smag"], got, rep)
         use = np.where(differs[:, :, None], got, sel["idx"])
         ref = oracle_lib.decode_attend(q, lm, gather_chunks(x["K"], use, wl.S),
                                        gather_chunks(x["V"], use, wl.S), use, wl.S)
