@@ -519,7 +519,7 @@ def bench_decode(args, name, dev, peaks, rank, dist, parity=False):
     x = make_decode_inputs(wl, dev)
     out = torch.empty_like(x["q"])
     ws = hsa.workspace(hsa.decode_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S, wl.topk),
-                       dev)
+                       dev, ("decode", wl.B * wl.Hkv))
     # The landmark stream alone (B*Hkv*Nc*d bf16 = 256 MiB for both decode
     # workloads) is larger than the 126 MB L2, so calls run back to back without
     # a flush: nothing a call reads can still be in L2 from the previous one in

@@ -125,14 +125,21 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-# Workspaces are cached per (device, stream): calls on one stream are ordered,
-# so reusing the buffer there is safe.
+# Workspaces are cached per (device, stream, kind): calls on one stream are
+# ordered, so reusing the buffer there is safe.  A prefill and a decode never
+# share one (each relies on its own regions being left as its previous call
+# left them), and decode workspaces are also keyed by B*Hkv: their
+# per-(sequence, group) counters must start at zero, which a completed call
+# guarantees only for the counters it used.
 _ws_cache: dict = {}
 
 
-def workspace(nbytes: int, device) -> torch.Tensor:
+def workspace(nbytes: int, device, kind: str = "prefill") -> torch.Tensor:
+    """A zero-filled (on creation) device workspace of at least `nbytes`,
+    cached per (device, current stream, kind); kind is "prefill" or
+    ("decode", B*Hkv)."""
     device = torch.device(device)
-    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream, kind)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < nbytes:
         ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
@@ -206,7 +213,7 @@ def decode(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.0, out=N
         idx_out = torch.empty(B, Hkv, topk, dtype=torch.int32, device=dev)
     nbytes = decode_workspace_size(B, H, Hkv, Lc, d, S, topk)
     if ws is None:
-        ws = workspace(nbytes, dev)
+        ws = workspace(nbytes, dev, ("decode", B * Hkv))
     st = lib().hsa_decode(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm), _dtype_code(lm),
                           B, H, Hkv, Lc, d, S, topk, float(scale), _ptr(out),
                           _ptr(_opt(idx_out)), _ptr(ws), ws.numel() * ws.element_size(),

@@ -131,10 +131,15 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
 /*
  * hsa_decode_workspace_size -- bytes of device workspace hsa_decode needs
  * (0 on invalid arguments; the size depends on the current device's SM
- * count).  It holds per-(sequence, group) tickets, the per-block candidate
- * lists, the selection and a status word.  A new workspace must be zero-filled once before
- * its first use; every completed call leaves the tickets at zero again.
- * Calls that share a workspace must be ordered (same stream).
+ * count).  It holds a status word, per-(sequence, group) tickets and work
+ * counters (right after the status word), the selection and the per-block
+ * candidate lists.  The tickets and counters must be zero when a call starts:
+ * zero-fill a workspace before its first use and whenever the previous call
+ * on it had another B*Hkv or it held anything else in between (a completed
+ * call leaves at zero only the tickets and counters it used; the selection
+ * and candidates of a call with fewer (sequence, group) pairs lie where a
+ * larger call's counters go).  Calls that share a workspace must be ordered
+ * (same stream).
  */
 size_t hsa_decode_workspace_size(int B, int H, int Hkv, int64_t Lc, int d, int S, int topk);
 
