@@ -6,12 +6,16 @@ The computation runs in hand-written CUDA kernels behind a C ABI
 binding (PyTorch supplies device memory and streams) plus the seeded synthetic
 workloads used by the tests and the benchmark.
 """
-from ._binding import (HSAError, check, decode, decode_noalloc, decode_workspace_size,
+from ._binding import (HSAError, check, decode, decode_context_parallel, decode_cp_attend,
+                       decode_cp_candidates, decode_cp_combine, decode_cp_merge, decode_noalloc,
+                       decode_workspace_size,
                        landmarks, last_call_kernels, last_call_launches, lib, path_overrides,
                        prefill, prefill_workspace_size, selftest_wait_expiry, set_stage_events,
                        status_string, workspace)
 
-__all__ = ["HSAError", "check", "decode", "decode_noalloc", "decode_workspace_size", "landmarks",
+__all__ = ["HSAError", "check", "decode", "decode_context_parallel", "decode_cp_attend",
+           "decode_cp_candidates", "decode_cp_combine", "decode_cp_merge", "decode_noalloc",
+           "decode_workspace_size", "landmarks",
            "last_call_kernels", "last_call_launches", "lib", "path_overrides", "prefill",
            "prefill_workspace_size", "selftest_wait_expiry", "set_stage_events", "status_string",
            "workspace"]

@@ -23,14 +23,15 @@ HSA_F32, HSA_BF16 = 0, 1
 # kernel families of a call (hsa_last_call_kernels) and path overrides
 K_LANDMARKS, K_SPLIT_LANDMARKS, K_SELECT_TC_ONE_TILE, K_SELECT_TC_MULTI_TILE = 1, 2, 4, 8
 K_SELECT_SIMT, K_WORK_LISTS, K_ATTEND_TC, K_FUSE, K_ATTEND_SIMT = 16, 32, 64, 128, 256
-K_DECODE_SCAN, K_DECODE_ATTEND = 512, 1024
+K_DECODE_SCAN, K_DECODE_ATTEND, K_DECODE_CP_MERGE, K_DECODE_CP_COMBINE = 512, 1024, 2048, 4096
 PATH_SIMT_PREFILL, PATH_SIMT_SELECT, PATH_MULTI_TILE_SELECT = 1, 2, 4
 
 EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_decode_workspace_size", "hsa_decode", "hsa_check", "hsa_status_string",
             "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches",
             "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry",
-            "hsa_last_call_kernels", "hsa_set_path_overrides")
+            "hsa_last_call_kernels", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
+            "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine")
 
 
 class HSAError(RuntimeError):
@@ -65,11 +66,18 @@ def _declare(lib):
     lib.hsa_last_call_kernels.argtypes = []
     lib.hsa_last_call_kernels.restype = ctypes.c_uint
     lib.hsa_set_path_overrides.argtypes = [i32, i64]
+    lib.hsa_decode_cp_candidates.argtypes = [vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32,
+                                             f32, i64, vp, vp, vp, sz, vp]
+    lib.hsa_decode_cp_merge.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp]
+    lib.hsa_decode_cp_attend.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
+                                         i32, f32, i64, vp, vp, vp, vp, vp]
+    lib.hsa_decode_cp_combine.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     lib.hsa_status_string.argtypes = [i32]
     lib.hsa_status_string.restype = ctypes.c_char_p
     for n in ("hsa_landmarks", "hsa_prefill", "hsa_decode", "hsa_check", "hsa_version",
               "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
-              "hsa_selftest_wait_expiry", "hsa_set_path_overrides"):
+              "hsa_selftest_wait_expiry", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
+              "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -243,6 +251,101 @@ def decode_noalloc(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.
                                       _ptr(out), _ptr(_opt(idx_out)), _stream(q.device))
     _check(st, "hsa_decode_noalloc")
     return out, _opt(idx_out)
+
+
+# ----------------------------------------------------------------------------- context parallel
+def decode_cp_candidates(q, lm, chunk_offset: int, *, S: int = 64, topk: int = 8,
+                         scale: float = 0.0, ws=None):
+    """Step 1 of a context-parallel decode on one shard: lm [B,Hkv,n,d] holds
+    chunks chunk_offset .. chunk_offset+n-1 of the whole cache.  Returns the
+    shard's top-K candidates (scores [B,Hkv,topk] fp32, global chunk indices
+    [B,Hkv,topk] int32, -1 where the shard has fewer chunks)."""
+    _dev(q, "q")
+    _dev(lm, "lm")
+    B, H, d = q.shape
+    _, Hkv, n, _ = lm.shape
+    dev = q.device
+    score = torch.empty(B, Hkv, topk, dtype=torch.float32, device=dev)
+    cidx = torch.empty(B, Hkv, topk, dtype=torch.int32, device=dev)
+    Lc = n * S
+    if ws is None:
+        ws = workspace(max(256, decode_workspace_size(B, H, Hkv, Lc, d, S, topk)), dev,
+                       ("decode", B * Hkv))
+    _check(lib().hsa_decode_cp_candidates(_ptr(q), _dtype_code(q), _ptr(lm), _dtype_code(lm), B, H,
+                                          Hkv, Lc, d, S, topk, float(scale), int(chunk_offset),
+                                          _ptr(score), _ptr(cidx), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(dev)),
+           "hsa_decode_cp_candidates")
+    return score, cidx
+
+
+def decode_cp_merge(scores, cidx):
+    """Step 2: the global top-K from the gathered candidates of R shards
+    (scores [R,B,Hkv,topk] fp32, cidx [R,B,Hkv,topk] int32) -> idx [B,Hkv,topk]."""
+    _dev(scores, "scores")
+    _dev(cidx, "cidx")
+    R, B, Hkv, topk = scores.shape
+    idx = torch.empty(B, Hkv, topk, dtype=torch.int32, device=scores.device)
+    _check(lib().hsa_decode_cp_merge(_ptr(scores), _ptr(cidx), R, B, Hkv, topk, _ptr(idx),
+                                     _stream(scores.device)), "hsa_decode_cp_merge")
+    return idx
+
+
+def decode_cp_attend(q, K, V, lm, chunk_offset: int, idx, *, S: int = 64, scale: float = 0.0):
+    """Step 3: the shard's per-head fusion state over the selected chunks it
+    holds (K/V [B,Hkv,n*S,d], lm [B,Hkv,n,d]) -> m, Z [B,H], acc [B,H,d] fp32."""
+    for nm, t in (("q", q), ("K", K), ("V", V), ("lm", lm), ("idx", idx)):
+        _dev(t, nm)
+    B, H, d = q.shape
+    _, Hkv, Lc, _ = K.shape
+    topk = idx.shape[-1]
+    dev = q.device
+    m = torch.empty(B, H, dtype=torch.float32, device=dev)
+    Z = torch.empty(B, H, dtype=torch.float32, device=dev)
+    acc = torch.empty(B, H, d, dtype=torch.float32, device=dev)
+    _check(lib().hsa_decode_cp_attend(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm),
+                                      _dtype_code(lm), B, H, Hkv, Lc, d, S, topk, float(scale),
+                                      int(chunk_offset), _ptr(idx), _ptr(m), _ptr(Z), _ptr(acc),
+                                      _stream(dev)), "hsa_decode_cp_attend")
+    return m, Z, acc
+
+
+def decode_cp_combine(m, Z, acc, dtype=torch.bfloat16):
+    """Step 4: O [B,H,d] from the gathered states of R shards (m, Z [R,B,H],
+    acc [R,B,H,d])."""
+    for nm, t in (("m", m), ("Z", Z), ("acc", acc)):
+        _dev(t, nm)
+    R, B, H, d = acc.shape
+    O = torch.empty(B, H, d, dtype=dtype, device=acc.device)
+    _check(lib().hsa_decode_cp_combine(_ptr(m), _ptr(Z), _ptr(acc), R, B, H, d, _dtype_code(O),
+                                       _ptr(O), _stream(acc.device)), "hsa_decode_cp_combine")
+    return O
+
+
+def decode_context_parallel(q, K, V, lm, chunk_offset: int, *, S: int = 64, topk: int = 8,
+                            scale: float = 0.0, group=None):
+    """One rank's part of a decode whose cache is cut along the sequence into
+    contiguous chunk ranges, one per rank of `group` (torch.distributed; NCCL
+    on GPUs): this rank holds K/V [B,Hkv,n*S,d] and lm [B,Hkv,n,d], chunks
+    chunk_offset .. chunk_offset+n-1; q [B,H,d] is the same on every rank.
+    The two exchanges are all-gathers over the group (candidates, then fusion
+    states); every rank returns the same (O, idx).  Without a process group
+    (or with one rank) the shard is the whole cache."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group) if (group is not None or dist.is_initialized()) else 1
+
+    def gather(t):
+        if world == 1:
+            return t.unsqueeze(0)
+        out = torch.empty((world,) + tuple(t.shape), dtype=t.dtype, device=t.device)
+        dist.all_gather_into_tensor(out, t.contiguous(), group=group)
+        return out
+
+    score, cidx = decode_cp_candidates(q, lm, chunk_offset, S=S, topk=topk, scale=scale)
+    idx = decode_cp_merge(gather(score), gather(cidx))
+    m, Z, acc = decode_cp_attend(q, K, V, lm, chunk_offset, idx, S=S, scale=scale)
+    O = decode_cp_combine(gather(m), gather(Z), gather(acc), dtype=q.dtype)
+    return O, idx
 
 
 def set_stage_events(events) -> None:

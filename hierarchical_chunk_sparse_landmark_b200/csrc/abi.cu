@@ -22,7 +22,12 @@ cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
                           const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
                           int S, int topk, float scale, int splits, const DecodeScratch &ws,
-                          void *O, int32_t *idx_out, cudaStream_t st);
+                          void *O, int32_t *idx_out, const DecodeShard &sh, int stages,
+                          const int32_t *sel, cudaStream_t st);
+cudaError_t launch_decode_cp_merge(const float *score, const int32_t *cidx, int R, int B, int Hkv,
+                                   int topk, int32_t *idx, cudaStream_t st);
+cudaError_t launch_decode_cp_combine(const float *m, const float *Z, const float *acc, int R,
+                                     int B, int H, int d, bool bf16, void *O, cudaStream_t st);
 int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
 bool select_tc_supported();
 cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaStream_t st);
@@ -428,12 +433,113 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
     if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
     char *ws = (char *)workspace;
     stage_mark(0, st);
+    const DecodeShard whole = {0, nullptr, nullptr, nullptr, nullptr, nullptr};
     hsa_status_t r = from_cuda(launch_decode(q, Kc, Vc, dt == HSA_BF16, lm, lm_dt == HSA_BF16, B, H, Hkv,
                                    Lc, d, S, topk, scale, lay.splits, lay.at(ws), O,
-                                   idx_out, st));
+                                   idx_out, whole, 0, nullptr, st));
     t_launches = r == HSA_OK ? 2 : 0;
     t_kernels = r == HSA_OK ? (unsigned)(HSA_K_DECODE_SCAN | HSA_K_DECODE_ATTEND) : 0u;
     stage_mark(1, st);
+    return r;
+}
+
+hsa_status_t hsa_decode_cp_candidates(const void *q, hsa_dtype_t dt, const void *lm,
+                                      hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t Lc, int d,
+                                      int S, int topk, float scale, int64_t chunk_offset,
+                                      float *cand_score, int32_t *cand_idx, void *workspace,
+                                      size_t ws_bytes, void *stream) {
+    hsa_status_t s = check_shape(B, H, Hkv, Lc, d, S, topk);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
+    if (Lc % S != 0 || chunk_offset < 0 || chunk_offset + Lc / S > (int64_t)INT32_MAX)
+        return HSA_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    t_kernels = 0;
+    const void *ptrs[] = {q, cand_score, cand_idx, workspace};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t nc = (size_t)B * Hkv * topk;
+    if (Lc == 0) {   // an empty shard has no candidates
+        if (cudaMemsetAsync(cand_idx, 0xff, sizeof(int32_t) * nc, st) != cudaSuccess)
+            return HSA_ERR_CUDA;
+        return cudaMemsetAsync(cand_score, 0, sizeof(float) * nc, st) == cudaSuccess
+                   ? HSA_OK : HSA_ERR_CUDA;
+    }
+    if (!lm || !aligned16(lm)) return HSA_ERR_INVALID_ARG;
+    const DecodeLayout lay = decode_layout(B, Hkv, Lc, S, topk);
+    if (ws_bytes < lay.total) return HSA_ERR_WORKSPACE;
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    const DecodeShard sh = {chunk_offset, cand_score, cand_idx, nullptr, nullptr, nullptr};
+    const hsa_status_t r = from_cuda(launch_decode(q, nullptr, nullptr, dt == HSA_BF16, lm,
+                                                   lm_dt == HSA_BF16, B, H, Hkv, Lc, d, S, topk,
+                                                   scale, lay.splits, lay.at((char *)workspace),
+                                                   nullptr, nullptr, sh, 1, nullptr, st));
+    t_launches = r == HSA_OK ? 1 : 0;
+    t_kernels = r == HSA_OK ? (unsigned)HSA_K_DECODE_SCAN : 0u;
+    return r;
+}
+
+hsa_status_t hsa_decode_cp_merge(const float *cand_score, const int32_t *cand_idx, int R, int B,
+                                 int Hkv, int topk, int32_t *idx, void *stream) {
+    if (R < 1 || B < 1 || Hkv < 1 || topk < 1) return HSA_ERR_INVALID_ARG;
+    if (topk > 32) return HSA_ERR_UNSUPPORTED;
+    if (!cand_score || !cand_idx || !idx) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    t_kernels = 0;
+    const hsa_status_t r = from_cuda(launch_decode_cp_merge(cand_score, cand_idx, R, B, Hkv, topk,
+                                                            idx, (cudaStream_t)stream));
+    t_launches = r == HSA_OK ? 1 : 0;
+    t_kernels = r == HSA_OK ? (unsigned)HSA_K_DECODE_CP_MERGE : 0u;
+    return r;
+}
+
+hsa_status_t hsa_decode_cp_attend(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                                  const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                                  int64_t Lc, int d, int S, int topk, float scale,
+                                  int64_t chunk_offset, const int32_t *idx, float *m, float *Z,
+                                  float *acc, void *stream) {
+    hsa_status_t s = check_shape(B, H, Hkv, Lc, d, S, topk);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
+    if (Lc % S != 0 || chunk_offset < 0 || chunk_offset + Lc / S > (int64_t)INT32_MAX)
+        return HSA_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    t_kernels = 0;
+    const void *ptrs[] = {q, idx, m, Z, acc};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    if (Lc > 0) {
+        const void *cache[] = {Kc, Vc, lm};
+        for (const void *p : cache)
+            if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    }
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    const DecodeShard sh = {chunk_offset, nullptr, nullptr, m, Z, acc};
+    DecodeScratch none = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    const hsa_status_t r = from_cuda(launch_decode(q, Kc, Vc, dt == HSA_BF16, lm,
+                                                   lm_dt == HSA_BF16, B, H, Hkv, Lc, d, S, topk,
+                                                   scale, 1, none, nullptr, nullptr, sh, 2, idx,
+                                                   (cudaStream_t)stream));
+    t_launches = r == HSA_OK ? 1 : 0;
+    t_kernels = r == HSA_OK ? (unsigned)HSA_K_DECODE_ATTEND : 0u;
+    return r;
+}
+
+hsa_status_t hsa_decode_cp_combine(const float *m, const float *Z, const float *acc, int R, int B,
+                                   int H, int d, hsa_dtype_t dt, void *O, void *stream) {
+    if (R < 1 || B < 1 || H < 1 || d < 1) return HSA_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return HSA_ERR_UNSUPPORTED;
+    if (!m || !Z || !acc || !O || !aligned16(O)) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    t_kernels = 0;
+    const hsa_status_t r = from_cuda(launch_decode_cp_combine(m, Z, acc, R, B, H, d,
+                                                              dt == HSA_BF16, O,
+                                                              (cudaStream_t)stream));
+    t_launches = r == HSA_OK ? 1 : 0;
+    t_kernels = r == HSA_OK ? (unsigned)HSA_K_DECODE_CP_COMBINE : 0u;
     return r;
 }
 

@@ -235,6 +235,15 @@ struct DecodeScratch {
     int32_t *sel;         // [B*Hkv*topk] selected chunks
     uint64_t *cand;       // [B*Hkv*splits*topk] per-block candidate keys
 };
+// A decode over one shard of a cache cut into contiguous chunk ranges
+// (context parallel); all zero / null for a whole cache.
+struct DecodeShard {
+    int64_t c0;            // global index of the shard's first chunk
+    float *cand_score;     // [B*Hkv*topk] or null: the shard's top-K scores (scan)
+    int32_t *cand_idx;     // [B*Hkv*topk] or null: their global chunk indices (-1: none)
+    float *m, *Z, *acc;    // [B*H], [B*H], [B*H*d] or null: fusion state instead of O (attend)
+};
+
 // Bytes at the head of a decode workspace that must be zero before a call
 // (status word, tickets, unit counters).
 __host__ __device__ constexpr size_t decode_zero_head(int64_t B, int64_t Hkv) {

@@ -28,6 +28,17 @@
 // decode_attend_kernel (launched as a programmatic dependent of the scan, so
 // its launch and its query loads overlap the scan's tail): one cluster of
 // min(K, 8) blocks per (b, g); see the kernel's comment.
+//
+// Context-parallel decode (a cache cut into contiguous chunk ranges, one per
+// GPU) runs the same two kernels on each shard with a DecodeShard: the scan
+// keys carry global chunk indices and its merge also writes the shard's top-K
+// (score, index) candidates; after the candidates of all shards are gathered,
+// decode_cp_merge_kernel takes the global top-K in the same total order; the
+// attend kernel then folds only the selected chunks the shard holds and writes
+// its per-head fusion state (m, Z, acc) instead of O; after the states are
+// gathered, decode_cp_combine_kernel combines them in shard order.  A global
+// top-K chunk is within its own shard's top K, so the result equals the
+// single-GPU decode.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -68,7 +79,8 @@ __device__ __forceinline__ uint64_t merge_smem_lists(const uint64_t (*lists)[32]
 template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kScanThreads)
 decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, int Hkv, int64_t Nc,
-                   int topk, float scale, int splits, DecodeScratch ws, int32_t *__restrict__ idx_out) {
+                   int topk, float scale, int splits, DecodeScratch ws, int32_t *__restrict__ idx_out,
+                   DecodeShard sh) {
     constexpr int ROW_BYTES = D * (int)sizeof(TL);
     constexpr int ROWS = kStageBytes / ROW_BYTES;           // landmark rows per stage (one unit)
     constexpr int VEC = Vec16<TL>::N;                        // elements per 16-byte vector
@@ -194,7 +206,7 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
                 // cheap float filter; ties and the exact order are settled on the keys
                 unsigned m = __ballot_sync(0xffffffffu, a >= tf && rr < rows_here) & 0x01010101u;
                 if (m) {
-                    const uint64_t key = make_key(a, row0 + rr);
+                    const uint64_t key = make_key(a, sh.c0 + row0 + rr);
                     while (m) {
                         const int s = __ffs(m) - 1;
                         m &= m - 1;
@@ -254,6 +266,10 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
             const int32_t i = key_index(best);
             ws.sel[bg * topk + lane] = i;
             if (idx_out) idx_out[bg * topk + lane] = i;
+            if (sh.cand_idx) {                // the shard's candidates for the exchange
+                sh.cand_idx[bg * topk + lane] = i;
+                sh.cand_score[bg * topk + lane] = key_score(best);
+            }
         }
         if (lane == 0) {                      // ready for the next call
             ws.tickets[bg] = 0u;
@@ -317,7 +333,8 @@ template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kAttThreads)
 decode_attend_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T *__restrict__ Kc,
                      const T *__restrict__ Vc, int H, int Hkv, int64_t Lc, int S, int topk,
-                     float scale, const int32_t *__restrict__ sel, T *__restrict__ O) {
+                     float scale, const int32_t *__restrict__ sel, T *__restrict__ O,
+                     DecodeShard sh) {
     constexpr int VT = AttSmem<T, D>::VT;
     constexpr int RS = AttSmem<T, D>::RS;
     constexpr int R = D / 32;
@@ -362,8 +379,10 @@ decode_attend_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T
     asm volatile("griddepcontrol.wait;" ::: "memory");   // the selection is written by the scan
 
     for (int k = crank; k < topk; k += C) {
-        const int32_t ci = sel[bg * topk + k];
-        if (ci < 0) break;                     // padding only at the end of the selection
+        const int32_t cg_ = sel[bg * topk + k];
+        if (cg_ < 0) break;                    // padding only at the end of the selection
+        const int64_t ci = (int64_t)cg_ - sh.c0;        // index within this cache (shard)
+        if (ci < 0 || ci >= Nc) continue;      // another shard's chunk (block-uniform)
         __syncthreads();                       // previous slot's tiles are no longer read
         {
             const int64_t first = (int64_t)ci * S;
@@ -494,8 +513,19 @@ decode_attend_kernel(const T *__restrict__ q, const TL *__restrict__ lm, const T
 #pragma unroll
             for (int i = 0; i < R; ++i) o_r[i] = fmaf(ar[r][i], cr, o_r[i]);
         }
+        const int64_t bh = b * H + g * G + h;
+        if (sh.acc) {                          // this shard's fusion state instead of O
+            float *ap = sh.acc + bh * D + R * lane;
+#pragma unroll
+            for (int i = 0; i < R; ++i) ap[i] = o_r[i];
+            if (lane == 0) {
+                sh.m[bh] = M;
+                sh.Z[bh] = Z;
+            }
+            continue;
+        }
         const float inv = Z > 0.f ? 1.f / Z : 0.f;
-        T *op = O + (b * H + g * G + h) * (int64_t)D + R * lane;
+        T *op = O + bh * (int64_t)D + R * lane;
 #pragma unroll
         for (int i = 0; i < R; ++i) op[i] = from_f32<T>(o_r[i] * inv);
     }
@@ -513,22 +543,98 @@ int decode_splits(int B, int Hkv, int64_t Nc, int num_sms) {
     return (int)s;
 }
 
+// ---------------------------------------------------------------- context parallel
+// Global top-K over R shards' candidates (gathered [R][B*Hkv][topk] scores and
+// global indices, -1 for none), one warp per (b, g): every candidate above the
+// current K-th key enters a warp-distributed sorted list; keys order (score,
+// then lower index) totally, so the visiting order does not matter.
+__global__ void __launch_bounds__(32)
+decode_cp_merge_kernel(const float *__restrict__ score, const int32_t *__restrict__ cidx, int R,
+                       int64_t pairs, int topk, int32_t *__restrict__ idx) {
+    const int64_t bg = blockIdx.x;
+    const int lane = threadIdx.x;
+    WarpTopK tk;
+    tk.init(topk);
+    uint64_t thr = 0ull;
+    const int64_t n = (int64_t)R * topk;
+    for (int64_t i0 = 0; i0 < n; i0 += 32) {
+        const int64_t i = i0 + lane;
+        uint64_t key = 0ull;
+        if (i < n) {
+            const int64_t r = i / topk, k = i % topk;
+            const int64_t at = (r * pairs + bg) * topk + k;
+            const int32_t ci = cidx[at];
+            if (ci >= 0) key = make_key(score[at], ci);
+        }
+        unsigned m = __ballot_sync(0xffffffffu, key > thr);
+        while (m) {
+            const int s = __ffs(m) - 1;
+            m &= m - 1;
+            const uint64_t x = __shfl_sync(0xffffffffu, key, s);
+            if (x > thr) {
+                tk.insert(x);
+                thr = tk.threshold();
+            }
+        }
+    }
+    if (lane < topk) idx[bg * topk + lane] = key_index(tk.v);
+}
+
+// O from R shards' fusion states (gathered [R][B*H] m, Z and [R][B*H][D] acc),
+// combined in shard order: O = sum_r e^{m_r - M} acc_r / sum_r e^{m_r - M} Z_r,
+// M = max_r m_r; a shard that held no selected chunk has m = -inf.  One warp
+// per (b, h).
+template <typename T>
+__global__ void __launch_bounds__(256)
+decode_cp_combine_kernel(const float *__restrict__ m, const float *__restrict__ Z,
+                         const float *__restrict__ acc, int R, int64_t rows, int D,
+                         T *__restrict__ O) {
+    const int64_t bh = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (bh >= rows) return;
+    float M = -INFINITY;
+    for (int r = 0; r < R; ++r) M = fmaxf(M, m[(int64_t)r * rows + bh]);
+    float z = 0.f;
+    for (int r = 0; r < R; ++r) {
+        const float mr = m[(int64_t)r * rows + bh];
+        z += mr > -INFINITY ? expf(mr - M) * Z[(int64_t)r * rows + bh] : 0.f;
+    }
+    const float inv = z > 0.f ? 1.f / z : 0.f;
+    for (int c = lane; c < D; c += 32) {
+        float a = 0.f;
+        for (int r = 0; r < R; ++r) {
+            const float mr = m[(int64_t)r * rows + bh];
+            if (mr > -INFINITY) a = fmaf(expf(mr - M), acc[((int64_t)r * rows + bh) * D + c], a);
+        }
+        O[bh * D + c] = from_f32<T>(a * inv);
+    }
+}
+
+// What a decode launch runs: both kernels (a whole cache), the scan only
+// (a shard's candidates) or the attend kernel only (a shard's state).
+enum DecodeStages { kDecodeBoth = 0, kDecodeScanOnly = 1, kDecodeAttendOnly = 2 };
+
 template <typename T, typename TL, int D>
 static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc, const void *Vc,
                                    int B, int H, int Hkv, int64_t Lc, int S, int topk,
                                    float scale, int splits, const DecodeScratch &ws, void *O,
-                                   int32_t *idx_out, cudaStream_t st) {
+                                   int32_t *idx_out, const DecodeShard &sh, int stages,
+                                   const int32_t *sel, cudaStream_t st) {
     const int64_t Nc = Lc / S;
     const unsigned grid = (unsigned)((int64_t)splits * B * Hkv);
-    auto scan = decode_scan_kernel<T, TL, D>;
-    cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kScanStages * kStageBytes);
-    if (e != cudaSuccess) return e;
-    // a programmatic dependent of whatever precedes it on the stream (it waits
-    // for that before reading anything), so its launch overlaps the tail
-    e = launch_pdl(scan, dim3(grid), dim3(kScanThreads), (size_t)(kScanStages * kStageBytes), st,
-                   (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws, idx_out);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (stages != kDecodeAttendOnly) {
+        auto scan = decode_scan_kernel<T, TL, D>;
+        e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kScanStages * kStageBytes);
+        if (e != cudaSuccess) return e;
+        // a programmatic dependent of whatever precedes it on the stream (it waits
+        // for that before reading anything), so its launch overlaps the tail
+        e = launch_pdl(scan, dim3(grid), dim3(kScanThreads), (size_t)(kScanStages * kStageBytes),
+                       st, (const T *)q, (const TL *)lm, H, Hkv, Nc, topk, scale, splits, ws,
+                       idx_out, sh);
+        if (e != cudaSuccess || stages == kDecodeScanOnly) return e;
+    }
 
     const size_t smem = AttSmem<T, D>::bytes(H / Hkv);
     auto kern = decode_attend_kernel<T, TL, D>;
@@ -550,16 +656,18 @@ static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, (const T *)q, (const TL *)lm, (const T *)Kc,
-                              (const T *)Vc, H, Hkv, Lc, S, topk, scale, (const int32_t *)ws.sel,
-                              (T *)O);
+                              (const T *)Vc, H, Hkv, Lc, S, topk, scale,
+                              sel ? sel : (const int32_t *)ws.sel, (T *)O, sh);
 }
 
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
                           const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
                           int S, int topk, float scale, int splits, const DecodeScratch &ws,
-                          void *O, int32_t *idx_out, cudaStream_t st) {
+                          void *O, int32_t *idx_out, const DecodeShard &sh, int stages,
+                          const int32_t *sel, cudaStream_t st) {
 #define HSA_DEC(T, TL, DD) \
-    return launch_decode_t<T, TL, DD>(q, lm, Kc, Vc, B, H, Hkv, Lc, S, topk, scale, splits, ws, O, idx_out, st)
+    return launch_decode_t<T, TL, DD>(q, lm, Kc, Vc, B, H, Hkv, Lc, S, topk, scale, splits, ws, O, \
+                                      idx_out, sh, stages, sel, st)
     using bf = __nv_bfloat16;
     if (bf16) {
         if (lm_bf16) { if (d == 128) HSA_DEC(bf, bf, 128); HSA_DEC(bf, bf, 64); }
@@ -570,6 +678,25 @@ cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf
     if (d == 128) HSA_DEC(float, float, 128);
     HSA_DEC(float, float, 64);
 #undef HSA_DEC
+}
+
+cudaError_t launch_decode_cp_merge(const float *score, const int32_t *cidx, int R, int B, int Hkv,
+                                   int topk, int32_t *idx, cudaStream_t st) {
+    const int64_t pairs = (int64_t)B * Hkv;
+    decode_cp_merge_kernel<<<(unsigned)pairs, 32, 0, st>>>(score, cidx, R, pairs, topk, idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_cp_combine(const float *m, const float *Z, const float *acc, int R,
+                                     int B, int H, int d, bool bf16, void *O, cudaStream_t st) {
+    const int64_t rows = (int64_t)B * H;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (bf16)
+        decode_cp_combine_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(m, Z, acc, R, rows, d,
+                                                                       (__nv_bfloat16 *)O);
+    else
+        decode_cp_combine_kernel<float><<<blocks, 256, 0, st>>>(m, Z, acc, R, rows, d, (float *)O);
+    return cudaGetLastError();
 }
 
 }  // namespace hsa

@@ -87,22 +87,30 @@ __device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-// One 32-column block of a token's scores (chunks c0 .. c0+31, visible below
-// nvis) into its sorted list v of KP 64-bit keys (score bits, ~index).  The
-// lane first marks its candidates (score >= its current K-th score), then
-// takes them one per loop trip from its own 32-float row of `stage` (shared
-// memory, column-major so the rows of a warp's lanes share no bank): the warp
-// runs as many trips as its busiest lane needs, instead of the insertion at
-// every column where any lane has a candidate.  Candidates are taken in column
-// order and the keys order (score, then lower index) totally, so the result
-// does not depend on the order.
+// One 32-column block of a token's scores (chunks c0 .. c0+31, of which the
+// first `lim` are visible) into its sorted list v of KP 64-bit keys (score
+// bits, ~index).  The lane first marks its candidates -- unscaled scores at or
+// above its current K-th score divided by the scale, a bound loosened by 1e-6
+// so that no column whose scaled score reaches it is missed; the exact test
+// follows -- then takes them one per loop trip from its own 32-float row of
+// `stage` (shared memory, column-major so the rows of a warp's lanes share no
+// bank): the warp runs as many trips as its busiest lane needs, instead of
+// the insertion at every column where any lane has a candidate.  Candidates
+// are taken in column order and the keys order (score, then lower index)
+// totally, so the result does not depend on the order.
+__device__ __forceinline__ int visible_in_block(int64_t nvis, int64_t c0) {
+    const int64_t n = nvis - c0;
+    return n <= 0 ? 0 : n >= 32 ? 32 : (int)n;
+}
 template <int KP>
-__device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, int64_t nvis, float scale,
+__device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, int lim, float scale,
                                            uint64_t (&v)[KP], float &tf, float *stage, int r) {
+    const float tq = tf / scale;                                // scale > 0
+    const float tr = tq - fabsf(tq) * 1e-6f;                    // -inf stays -inf
     uint32_t mask = 0;
 #pragma unroll
-    for (int c = 0; c < 32; ++c)
-        if (c0 + c < nvis && scale * sc[c] >= tf) mask |= 1u << c;
+    for (int c = 0; c < 32; ++c) mask |= (sc[c] >= tr ? 1u : 0u) << c;
+    mask &= lim >= 32 ? 0xffffffffu : (1u << lim) - 1u;
     if (mask) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) stage[c * 128 + r] = sc[c];
@@ -184,7 +192,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             tc::mbar_init(&full[s], 1);
             tc::mbar_init(&empty[s], 1);
             tc::mbar_init(&tfull[s], 1);
-            tc::mbar_init(&tfree[s], 256);     // one arrive per top-K thread
+            tc::mbar_init(&tfree[s], 8);       // one arrive per top-K warp
         }
         *s_abort = 0;
         tc::fence_barrier_init();
@@ -329,20 +337,30 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         float tf = -INFINITY;                                  // score of v[KP-1]
         for (int n = 0; n < ntiles; ++n) {
             const int s = n & 1;
-            if (!sel_wait(&tfull[s], (uint32_t)((n >> 1) & 1), s_abort)) break;
+            // warp-uniform outcome: the TMEM loads below are .sync.aligned
+            if (!__all_sync(0xffffffffu, sel_wait(&tfull[s], (uint32_t)((n >> 1) & 1), s_abort)))
+                break;
             tc::fence_after_sync();
             // 32-column blocks past the block's last visible chunk hold nothing
             const int64_t vis = nvis_max - (int64_t)n * C::N;
             const int ncb = vis >= C::N ? C::N / 32 : (int)((vis + 31) / 32);
-#pragma unroll 1
-            for (int cb = hg; cb < ncb; cb += 2) {
-                float sc[32];
-                tc::tmem_ld32(tmem + s * C::N + cb * 32 + lane_off, sc);
+            // this group's two 32-column blocks (cb = hg, hg + 2): both loads
+            // are issued before one wait
+            if (hg < ncb) {
+                float sc0[32], sc1[32];
+                const bool two = hg + 2 < ncb;
+                tc::tmem_ld32(tmem + s * C::N + hg * 32 + lane_off, sc0);
+                if (two) tc::tmem_ld32(tmem + s * C::N + (hg + 2) * 32 + lane_off, sc1);
                 tc::tmem_wait_ld();
-                topk_block<KP>(sc, (int64_t)n * C::N + cb * 32, nvis, p.scale, v, tf, stage, r);
+                const int64_t c0 = (int64_t)n * C::N + hg * 32;
+                topk_block<KP>(sc0, c0, visible_in_block(nvis, c0), p.scale, v, tf, stage, r);
+                if (two)
+                    topk_block<KP>(sc1, c0 + 64, visible_in_block(nvis, c0 + 64), p.scale, v, tf,
+                                   stage, r);
             }
             tc::fence_before_sync();
-            tc::mbar_arrive(&tfree[s]);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tfree[s]);
         }
         // the landmark stages are dead once the last tile's scores are in TMEM
         uint64_t *lists = reinterpret_cast<uint64_t *>(sB(0));
@@ -550,16 +568,27 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
 #pragma unroll
         for (int i = 0; i < KP; ++i) v[i] = 0ull;
         float tf = -INFINITY;                                  // score of v[KP-1]
-        if (ok && sel_wait(tfull, 0u, s_abort)) {
+        // warp-uniform outcome: the TMEM loads below are .sync.aligned
+        if (__all_sync(0xffffffffu, ok && sel_wait(tfull, 0u, s_abort))) {
             tc::fence_after_sync();
             // 32-column blocks past the block's last visible chunk hold nothing
             const int ncb = nvis_max >= C::N ? C::N / 32 : (int)((nvis_max + 31) / 32);
+            // two blocks' loads per wait where the registers allow (two blocks of
+            // 32 scores next to a 16-key list stay within the 128 registers a
+            // thread has at two blocks per SM)
+            constexpr int STEP = KP <= 8 ? 2 : 1;
 #pragma unroll 1
-            for (int cb = 0; cb < ncb; ++cb) {
-                float sc[32];
-                tc::tmem_ld32(tmem + cb * 32 + lane_off, sc);
+            for (int cb = 0; cb < ncb; cb += STEP) {
+                float sc0[32], sc1[32];
+                const bool two = STEP == 2 && cb + 1 < ncb;
+                tc::tmem_ld32(tmem + cb * 32 + lane_off, sc0);
+                if (two) tc::tmem_ld32(tmem + (cb + 1) * 32 + lane_off, sc1);
                 tc::tmem_wait_ld();
-                topk_block<KP>(sc, (int64_t)cb * 32, nvis, p.scale, v, tf, (float *)sA, r);
+                const int64_t c0 = (int64_t)cb * 32;
+                topk_block<KP>(sc0, c0, visible_in_block(nvis, c0), p.scale, v, tf, (float *)sA, r);
+                if (two)
+                    topk_block<KP>(sc1, c0 + 32, visible_in_block(nvis, c0 + 32), p.scale, v, tf,
+                                   (float *)sA, r);
             }
             tc::fence_before_sync();
             if (t < L) {

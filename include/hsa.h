@@ -72,7 +72,9 @@ enum {
     HSA_K_FUSE = 1u << 7,                 /* fusion of the chunk outputs */
     HSA_K_ATTEND_SIMT = 1u << 8,          /* in-chunk attention + fusion on CUDA cores */
     HSA_K_DECODE_SCAN = 1u << 9,          /* decode landmark scan + top-K */
-    HSA_K_DECODE_ATTEND = 1u << 10        /* decode attend + fusion */
+    HSA_K_DECODE_ATTEND = 1u << 10,       /* decode attend + fusion (or a shard's fusion state) */
+    HSA_K_DECODE_CP_MERGE = 1u << 11,     /* global top-K over the shards' candidates */
+    HSA_K_DECODE_CP_COMBINE = 1u << 12    /* O from the shards' fusion states */
 };
 
 /* Path overrides (hsa_set_path_overrides). */
@@ -205,6 +207,55 @@ hsa_status_t hsa_decode_noalloc(const void *q, const void *Kc, const void *Vc, h
 
 /* hsa_decode_noalloc_max_scratch -- size in bytes of hsa_decode_noalloc's array. */
 size_t hsa_decode_noalloc_max_scratch(void);
+
+/*
+ * Context-parallel decode: hsa_decode for a KV cache cut along the sequence
+ * into R contiguous chunk ranges (shards), one per GPU, for contexts larger
+ * than one GPU's memory (the HSA summary reports retrieval up to 32M tokens,
+ * "Main Findings").  The method is unchanged; only where its steps run moves.
+ * Each rank calls, in order:
+ *   1. hsa_decode_cp_candidates on its shard: the shard's top-K chunks by the
+ *      group score, as (score, global chunk index) candidates;
+ *   2. an all-gather of the candidates over the R ranks (the caller's
+ *      collective, e.g. NCCL), then hsa_decode_cp_merge: the global top-K in
+ *      the single-GPU order (larger score first, lower index on ties).  A
+ *      chunk of the global top-K is within its own shard's top K, so the
+ *      selection equals hsa_decode's;
+ *   3. hsa_decode_cp_attend on its shard: attention inside the selected
+ *      chunks it holds, folded into a per-head fusion state m (largest fusion
+ *      logit), Z (sum of exp(z - m)), acc (sum of exp(z - m) * chunk output);
+ *   4. an all-gather of the states, then hsa_decode_cp_combine: O, the
+ *      fusion softmax over the selection written as a sum over shards.
+ * Every rank gets the same idx and O.  Shard r holds chunks
+ * [chunk_offset, chunk_offset + Lc/S) of the whole cache, Lc its own length
+ * (a multiple of S, may be 0); q is the same on every rank.
+ */
+/* Step 1.  lm [B, Hkv, Lc/S, d]; cand_score [B, Hkv, topk] fp32 and cand_idx
+ * [B, Hkv, topk] int32 (global chunk indices, best first; -1 and score 0 where
+ * the shard has fewer than topk chunks).  workspace as for hsa_decode with the
+ * shard's sizes (hsa_decode_workspace_size(B, H, Hkv, Lc, d, S, topk)). */
+hsa_status_t hsa_decode_cp_candidates(const void *q, hsa_dtype_t dt, const void *lm,
+                                      hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t Lc, int d,
+                                      int S, int topk, float scale, int64_t chunk_offset,
+                                      float *cand_score, int32_t *cand_idx, void *workspace,
+                                      size_t ws_bytes, void *stream);
+/* Step 2.  cand_score / cand_idx [R, B, Hkv, topk] (the gathered step-1
+ * outputs, in rank order) -> idx [B, Hkv, topk] (-1 padded). */
+hsa_status_t hsa_decode_cp_merge(const float *cand_score, const int32_t *cand_idx, int R, int B,
+                                 int Hkv, int topk, int32_t *idx, void *stream);
+/* Step 3.  Kc, Vc [B, Hkv, Lc, d], lm [B, Hkv, Lc/S, d] (the shard's), idx
+ * [B, Hkv, topk] from step 2 -> m, Z [B, H] and acc [B, H, d] fp32 (m = -inf,
+ * Z = 0, acc = 0 for heads whose group has no selected chunk on this shard). */
+hsa_status_t hsa_decode_cp_attend(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                                  const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                                  int64_t Lc, int d, int S, int topk, float scale,
+                                  int64_t chunk_offset, const int32_t *idx, float *m, float *Z,
+                                  float *acc, void *stream);
+/* Step 4.  m, Z [R, B, H], acc [R, B, H, d] (gathered, rank order) ->
+ * O [B, H, d] in dt: O = sum_r e^{m_r - M} acc_r / sum_r e^{m_r - M} Z_r,
+ * M = max_r m_r (O = 0 where no shard held a selected chunk). */
+hsa_status_t hsa_decode_cp_combine(const float *m, const float *Z, const float *acc, int R, int B,
+                                   int H, int d, hsa_dtype_t dt, void *O, void *stream);
 
 /*
  * hsa_selftest_wait_expiry -- exercises the failure path of the kernels'
