@@ -48,8 +48,11 @@ def _bind(lib):
                                              dp, dp, dp]
     lib.hsa_oracle_decode_attend.argtypes = [dp, dp, dp, dp, i32p, i32, i32, i32, i64, i32,
                                              i32, i32, dbl, dp, dp]
+    lib.hsa_oracle_prefill_variant.argtypes = [dp, i64p, i64, dp, dp, dp, i32, i32, i32, i64, i32,
+                                               i32, i32, i32, dbl, i32, i32, i32, dp, i32p, dp]
     for name in ("hsa_oracle_landmarks", "hsa_oracle_prefill", "hsa_oracle_decode_select",
-                 "hsa_oracle_decode_attend", "hsa_oracle_num_threads"):
+                 "hsa_oracle_decode_attend", "hsa_oracle_num_threads",
+                 "hsa_oracle_prefill_variant"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -148,6 +151,33 @@ class Oracle:
             _dp(gap), _dp(smag))
         _check(rc, "prefill")
         return {"O": O, "idx": idx, "w": w, "sbar": sbar, "gap": gap, "smag": smag, "rows": rows}
+
+    def prefill_variant(self, Q, K, V, lm, S: int, topk: int, own_chunk: int = 1,
+                        scale: float = 0.0, interval: int = 1, pool_mean: int = 0,
+                        union_softmax: int = 0, rows=None):
+        """Retrieval variants (see hsa_oracle_prefill_variant): one selection
+        per `interval` tokens (first token's or mean group query), HiLS fusion
+        or one softmax over the union of the selected keys.  Q [B,L,H,d] (all
+        tokens), K/V [B,Hkv,L,d], lm [B,Hkv,L//S,d] or None (DHSA).
+        Returns dict O [n,H,d], idx [n,Hkv,K], w [n,H,K]."""
+        qf, k, v = _f64(Q), _f64(K), _f64(V)
+        B, L, H, d = qf.shape
+        Hkv = k.shape[1]
+        if rows is None:
+            rows = np.arange(B * L, dtype=np.int64)
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rows.shape[0]
+        lmf = None if lm is None else _f64(lm)
+        O = np.zeros((n, H, d), dtype=np.float64)
+        idx = np.zeros((n, Hkv, topk), dtype=np.int32)
+        w = np.zeros((n, H, topk), dtype=np.float64)
+        rc = self.lib.hsa_oracle_prefill_variant(
+            _dp(qf), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _dp(k), _dp(v),
+            _dp(lmf), B, H, Hkv, L, d, S, topk, int(own_chunk), float(scale), int(interval),
+            int(pool_mean), int(union_softmax), _dp(O),
+            idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(w))
+        _check(rc, "prefill_variant")
+        return {"O": O, "idx": idx, "w": w, "rows": rows}
 
     def decode_select(self, q, lm, topk: int, scale: float = 0.0):
         """q [B,H,d], lm [B,Hkv,Nc,d] -> dict idx [B,Hkv,K], sbar, gap, smag."""

@@ -312,6 +312,171 @@ int hsa_oracle_prefill(const double *q, const int64_t *rows, int64_t n_rows,
 }
 
 /*
+ * Prefill forward of the retrieval variants, for a list of query rows.
+ *
+ * Retrieval interval (HSA summary, "Main Findings": per-token retrieval
+ * against per-8-token retrieval).  Tokens are cut into blocks of `interval`
+ * consecutive tokens starting at 0 (interval divides S, so a block never
+ * straddles a chunk boundary and all its tokens see the same chunks).  One
+ * selection serves every token of a block; its group query is
+ *   pool_mean = 0: the group query of the block's first token (it is known
+ *                  when the block starts: the causal reading);
+ *   pool_mean = 1: the mean over the block's tokens of their group queries
+ *                  (the DHSA chunk-level query: sqrt(|C|) times the mean of
+ *                  the chunk's queries, "What carries the argument", when
+ *                  interval = S; the positive factor sqrt(|C|) does not change
+ *                  the ranking and is left out).
+ * The visible chunks are those before the block's chunk.  interval = 1 is
+ * the per-token retrieval of hsa_oracle_prefill.
+ *
+ * Fusion:
+ *   union_softmax = 0: softmax inside each selected chunk, outputs fused by
+ *                      the softmax over the selection of the head's landmark
+ *                      scores (HiLS Attention abstract), own chunk added;
+ *   union_softmax = 1: one softmax over the keys of all selected chunks and,
+ *                      with own_chunk, the causal own-chunk keys (Dynamic
+ *                      Hierarchical Sparse Attention review, "What carries the
+ *                      argument": attention under the selected-chunk mask).
+ *
+ *   Q    [B, L, H, d]  all queries (pooling reads the block's other tokens)
+ *   rows [n_rows]      flattened positions b*L + t to compute
+ * Outputs O [n_rows, H, d], idx [n_rows, Hkv, topk] (may be NULL),
+ * w [n_rows, H, topk] (may be NULL; the fusion weights of the HiLS form,
+ * zero with union_softmax).
+ */
+int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_rows,
+                               const double *k, const double *v, const double *lm,
+                               int B, int H, int Hkv, int64_t L, int d, int S, int topk,
+                               int own_chunk, double scale, int interval, int pool_mean,
+                               int union_softmax, double *O, int32_t *idx, double *w)
+{
+    if (!Q || !rows || !k || !v || !O) return ORACLE_BAD_ARG;
+    if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || L < 1 || d < 1 || S < 1 || topk < 1)
+        return ORACLE_BAD_ARG;
+    if (interval < 1 || S % interval != 0) return ORACLE_BAD_ARG;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * L) return ORACLE_BAD_ARG;
+    const int G = H / Hkv;
+    const int64_t Nc = L / S;
+    if (scale == 0.0) scale = 1.0 / sqrt((double)d);
+
+    double *lm_dhsa = NULL;
+    if (!lm) {
+        lm_dhsa = (double *)malloc(sizeof(double) * (size_t)B * Hkv * (Nc > 0 ? Nc : 1) * d);
+        if (!lm_dhsa) return ORACLE_NO_MEMORY;
+        hsa_oracle_landmarks(k, B, Hkv, L, d, S, lm_dhsa);
+        lm = lm_dhsa;
+    }
+    int status = ORACLE_OK;
+    const int64_t maxkeys = (int64_t)topk * S + S;
+
+#pragma omp parallel
+    {
+        candidate_t *cand = (candidate_t *)malloc(sizeof(candidate_t) * (size_t)(Nc > 0 ? Nc : 1));
+        double *qbar = (double *)malloc(sizeof(double) * d);
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(maxkeys > topk ? maxkeys : topk));
+        double *o_part = (double *)malloc(sizeof(double) * d);
+        double *o_row = (double *)malloc(sizeof(double) * d);
+        double *wk = (double *)malloc(sizeof(double) * topk);
+        int64_t *sel = (int64_t *)malloc(sizeof(int64_t) * topk);
+        int64_t *keyrow = (int64_t *)malloc(sizeof(int64_t) * (size_t)maxkeys);
+        if (!cand || !qbar || !logit || !o_part || !o_row || !wk || !sel || !keyrow) {
+#pragma omp atomic write
+            status = ORACLE_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t rg = 0; rg < n_rows * Hkv; ++rg) {
+            if (status != ORACLE_OK) continue;
+            const int64_t r = rg / Hkv;
+            const int g = (int)(rg % Hkv);
+            const int64_t b = rows[r] / L;
+            const int64_t t = rows[r] % L;
+            const int64_t t0 = (t / interval) * interval;      /* the block's first token */
+            const int64_t t1 = t0 + interval < L ? t0 + interval : L;
+            const int64_t c = t / S;                            /* own chunk (= t0's) */
+            const int64_t nvis = c;
+            const double *lm_bg = lm + ((b * Hkv + g) * Nc) * d;
+            const double *k_bg = k + ((b * Hkv + g) * L) * d;
+            const double *v_bg = v + ((b * Hkv + g) * L) * d;
+
+            /* the block's group query: first token's, or the mean over its tokens */
+            const int64_t u1 = pool_mean ? t1 : t0 + 1;
+            for (int j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int64_t u = t0; u < u1; ++u)
+                    for (int h = 0; h < G; ++h) acc += Q[((b * L + u) * H + g * G + h) * d + j];
+                qbar[j] = acc / ((double)G * (double)(u1 - t0));
+            }
+            for (int64_t i = 0; i < nvis; ++i) {
+                cand[i].score = scale * dot(qbar, lm_bg + i * d, d);
+                cand[i].index = i;
+            }
+            qsort(cand, (size_t)nvis, sizeof(candidate_t), candidate_order);
+            const int64_t nsel = nvis < topk ? nvis : topk;
+            for (int64_t kk = 0; kk < nsel; ++kk) sel[kk] = cand[kk].index;
+            if (idx)
+                for (int kk = 0; kk < topk; ++kk)
+                    idx[(r * Hkv + g) * topk + kk] = kk < nsel ? (int32_t)sel[kk] : -1;
+
+            for (int h = 0; h < G; ++h) {
+                const int hh = g * G + h;
+                const double *q_h = Q + ((b * L + t) * H + hh) * d;
+                for (int j = 0; j < d; ++j) o_row[j] = 0.0;
+                for (int kk = 0; kk < topk; ++kk) wk[kk] = 0.0;
+                if (!union_softmax) {
+                    /* HiLS form: each token's own landmark scores weight the chunks */
+                    for (int64_t kk = 0; kk < nsel; ++kk)
+                        wk[kk] = scale * dot(q_h, lm_bg + sel[kk] * d, d);
+                    softmax_inplace(wk, (int)nsel);
+                    for (int64_t kk = 0; kk < nsel; ++kk) {
+                        const int64_t first = sel[kk] * S;
+                        chunk_attention(q_h, k_bg + first * d, v_bg + first * d, S, d, scale,
+                                        logit, o_part);
+                        for (int j = 0; j < d; ++j) o_row[j] += wk[kk] * o_part[j];
+                    }
+                    if (own_chunk) {
+                        const int64_t first = c * S;
+                        chunk_attention(q_h, k_bg + first * d, v_bg + first * d, t - first + 1,
+                                        d, scale, logit, o_part);
+                        for (int j = 0; j < d; ++j) o_row[j] += o_part[j];
+                    }
+                } else {
+                    /* DHSA form: one softmax over the union of the selected keys */
+                    int64_t nk = 0;
+                    for (int64_t kk = 0; kk < nsel; ++kk)
+                        for (int64_t jj = 0; jj < S; ++jj) keyrow[nk++] = sel[kk] * S + jj;
+                    if (own_chunk)
+                        for (int64_t jj = c * S; jj <= t; ++jj) keyrow[nk++] = jj;
+                    if (nk > 0) {
+                        double m = -INFINITY;
+                        for (int64_t e = 0; e < nk; ++e) {
+                            logit[e] = scale * dot(q_h, k_bg + keyrow[e] * d, d);
+                            if (logit[e] > m) m = logit[e];
+                        }
+                        double den = 0.0;
+                        for (int64_t e = 0; e < nk; ++e) {
+                            logit[e] = exp(logit[e] - m);
+                            den += logit[e];
+                        }
+                        for (int64_t e = 0; e < nk; ++e) {
+                            const double p = logit[e] / den;
+                            for (int j = 0; j < d; ++j) o_row[j] += p * v_bg[keyrow[e] * d + j];
+                        }
+                    }
+                }
+                memcpy(O + (r * H + hh) * d, o_row, sizeof(double) * d);
+                if (w)
+                    for (int kk = 0; kk < topk; ++kk) w[(r * H + hh) * topk + kk] = wk[kk];
+            }
+        }
+        free(cand); free(qbar); free(logit); free(o_part); free(o_row); free(wk); free(sel);
+        free(keyrow);
+    }
+    free(lm_dhsa);
+    return status;
+}
+
+/*
  * Decode, step 1: selection for one new query per sequence at position Lc
  * (R12: all Nc = Lc/S chunks visible).
  *   q    [B, H, d]

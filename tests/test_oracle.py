@@ -496,3 +496,78 @@ def test_score_term_magnitudes_hand_case(oracle_lib):
     np.testing.assert_array_equal(r3["smag"][0, 0], [0.75, 0.25, 2.0, 0.0])   # no 4th chunk
     dec = oracle_lib.decode_select(np.ones((1, 1, d)), lm, 2, scale=1.0)
     np.testing.assert_array_equal(dec["smag"][0, 0], [1.5, 0.5, 4.0])
+
+
+# --------------------------------------------------------------------------- retrieval variants
+def test_variant_interval_one_is_the_per_token_oracle(oracle_lib):
+    """Retrieval every token with the HiLS fusion is hsa_oracle_prefill."""
+    Q, K, V, lm = rand_case(30, 2, 70, 4, 2, 8, 8)
+    for own in (0, 1):
+        a = oracle_lib.prefill(Q, K, V, lm, 8, 3, own)
+        for pool in (0, 1):
+            b = oracle_lib.prefill_variant(Q, K, V, lm, 8, 3, own, pool_mean=pool)
+            np.testing.assert_array_equal(a["idx"], b["idx"])
+            np.testing.assert_allclose(a["O"], b["O"], atol=1e-13, rtol=0)
+            np.testing.assert_allclose(a["w"], b["w"], atol=1e-14, rtol=0)
+
+
+@pytest.mark.parametrize("interval", [2, 4, 8])
+def test_variant_first_token_retrieval_reuses_the_block_start_selection(oracle_lib, interval):
+    """One selection per block of `interval` tokens, decided by the block's
+    first token: token t uses the per-token selection of its block start, and
+    its output is the per-token oracle's output on that forced selection."""
+    B, L, H, Hkv, d, S, topk = 1, 8 * 13 + 5, 4, 2, 8, 8, 3
+    Q, K, V, lm = rand_case(31, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill_variant(Q, K, V, lm, S, topk, 1, interval=interval)
+    starts = (np.arange(L) // interval) * interval
+    per_tok = oracle_lib.prefill(Q, K, V, lm, S, topk, 1)
+    np.testing.assert_array_equal(r["idx"], per_tok["idx"][starts])
+    forced = oracle_lib.prefill(Q, K, V, lm, S, topk, 1, forced_idx=per_tok["idx"][starts])
+    np.testing.assert_allclose(r["O"], forced["O"], atol=1e-13, rtol=0)
+    np.testing.assert_allclose(r["w"], forced["w"], atol=1e-14, rtol=0)
+
+
+@pytest.mark.parametrize("interval", [4, 8])
+def test_variant_mean_pooled_selection_is_the_top_k_of_the_block_mean(oracle_lib, interval):
+    """Mean pooling (the DHSA chunk-level query at interval = S): the block's
+    selection is the top-K, lower index on ties, of the landmark scores of the
+    mean over its tokens and the group's heads, computed here with numpy."""
+    B, L, H, Hkv, d, S, topk = 2, 8 * 11 + 3, 4, 2, 8, 8, 3
+    Q, K, V, lm = rand_case(32, B, L, H, Hkv, d, S)
+    r = oracle_lib.prefill_variant(Q, K, V, lm, S, topk, 1, interval=interval, pool_mean=1)
+    G = H // Hkv
+    for b in range(B):
+        for t in range(L):
+            t0 = (t // interval) * interval
+            t1 = min(t0 + interval, L)
+            for g in range(Hkv):
+                qm = Q[b, t0:t1, g * G:(g + 1) * G].mean(axis=(0, 1))
+                nvis = t // S
+                s = lm[b, g, :nvis] @ qm
+                want = np.lexsort((np.arange(nvis), -s))[:topk]
+                got = r["idx"][b * L + t, g]
+                np.testing.assert_array_equal(got[:len(want)], want)
+                assert (got[len(want):] == -1).all()
+
+
+def test_variant_union_softmax_matches_the_numpy_restatement(oracle_lib):
+    """One softmax over the union of the selected keys (and the own chunk)
+    equals oracle/variants.py's numpy restatement, which is pinned to SDPA."""
+    from oracle import variants
+    Q, K, V, lm = rand_case(33, 2, 53, 4, 2, 8, 8)
+    for own in (0, 1):
+        r = oracle_lib.prefill_variant(Q, K, V, lm, 8, 2, own, union_softmax=1)
+        ref = variants.flat_union_prefill(Q, K, V, lm, 8, 2, own)
+        np.testing.assert_array_equal(r["idx"].reshape(ref["idx"].shape), ref["idx"])
+        np.testing.assert_allclose(r["O"].reshape(ref["O"].shape), ref["O"], atol=1e-12, rtol=0)
+        assert (r["w"] == 0).all()
+
+
+def test_variant_union_softmax_of_every_chunk_is_causal_attention(oracle_lib):
+    """All visible chunks selected plus the own chunk: plain causal attention
+    (PyTorch SDPA in float64)."""
+    Q, K, V, lm = rand_case(34, 1, 48, 4, 2, 8, 8)
+    for interval in (1, 8):
+        r = oracle_lib.prefill_variant(Q, K, V, lm, 8, 6, 1, union_softmax=1, interval=interval)
+        ref = sdpa_causal(Q, K, V, 2)
+        np.testing.assert_allclose(r["O"].reshape(ref.shape), ref, atol=1e-12, rtol=0)

@@ -47,6 +47,17 @@ MUTANTS = {
     # near-tie scale: the magnitude of a score's terms taken as |score|
     "score_magnitude_without_abs": ("for (int j = 0; j < n; ++j) acc += fabs(x[j] * y[j]);",
                                     "for (int j = 0; j < n; ++j) acc += x[j] * y[j];"),
+    # retrieval variants: each token decides for itself instead of its block start
+    "variant_block_start_ignored": ("const int64_t t0 = (t / interval) * interval;",
+                                    "const int64_t t0 = t;"),
+    # retrieval variants: the union softmax leaves out the own chunk, or its last key
+    "variant_union_drops_own_chunk": ("if (own_chunk)\n                        for (int64_t jj = c * S; jj <= t; ++jj)",
+                                      "if (0)\n                        for (int64_t jj = c * S; jj <= t; ++jj)"),
+    "variant_union_own_excludes_self": ("for (int64_t jj = c * S; jj <= t; ++jj) keyrow[nk++] = jj;",
+                                        "for (int64_t jj = c * S; jj < t; ++jj) keyrow[nk++] = jj;"),
+    # retrieval variants: mean pooling over the block's first token only
+    "variant_mean_pool_first_only": ("const int64_t u1 = pool_mean ? t1 : t0 + 1;",
+                                     "const int64_t u1 = t0 + 1;"),
     # forced selection: chunks not visible from the row are kept
     "forced_visibility_filter_dropped": ("if (f[kk] >= 0 && f[kk] < nvis) sel[nsel++] = f[kk];",
                                          "if (f[kk] >= 0 && f[kk] < Nc) sel[nsel++] = f[kk];"),
