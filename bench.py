@@ -76,6 +76,17 @@ def prefill_flops(wl) -> dict:
             "attention_kernel": chunk + ownf + fuse}
 
 
+def chunk_output_bytes(wl) -> float:
+    """Bytes of fp16 chunk outputs the tensor-core attention writes (and the
+    fusion reads back): one G*d block per selected (token, group, chunk) and
+    one own-chunk block per (token, group).  Design traffic of the chunk-
+    bucketed schedule, not algorithmic work: with random selections a token's
+    chunks are processed on different SMs, so each chunk output crosses from
+    an SM to L2 once."""
+    _, keff, _ = prefill_token_counts(wl)
+    return float(wl.B * wl.Hkv * (keff + 1).sum() * wl.G * wl.d * 2)
+
+
 def decode_bytes(wl, lm_elem_bytes=2) -> float:
     """Algorithmic HBM bytes of one decode step: every visible landmark, the K
     and V of the selected chunks, q and O.  The full cache is never read."""
@@ -329,6 +340,13 @@ def bench_prefill(args, name, dev, peaks, rank, dist, steps, warmup, keep_inputs
                      "traffic": measured_traffic(kfile, files, workload=wl.name),
                      "algorithmic_flops_per_launch": kflops,
                      "ms_per_launch": round(attn_s * 1e3, 4)})
+    if tc_path:
+        # what the kernel actually streams: its chunk outputs, SM -> L2 -> HBM
+        cob = chunk_output_bytes(wl)
+        roofline["chunk_outputs"] = {"bytes_per_launch": cob,
+                                     "achieved_GBps": round(cob / attn_s / 1e9, 1),
+                                     "note": "fp16 chunk outputs written by the attention kernel "
+                                             "and read back by the fusion kernel"}
     res = {"workload": wl.name, "value": round(units / tmax, 4), "unit": "TFLOP/s",
            "ms_per_step": round(tmax * 1e3 / steps, 4), "steps": steps,
            "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "Hkv": wl.Hkv,

@@ -31,7 +31,14 @@ EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_version", "hsa_set_stage_events", "hsa_last_call_launches",
             "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry",
             "hsa_last_call_kernels", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
-            "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine")
+            "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
+            "hsa_prefill_variant")
+
+
+class Variant(ctypes.Structure):
+    """hsa_variant_t: retrieval interval, pooling of the block's queries, fusion form."""
+    _fields_ = [("retrieval_interval", ctypes.c_int), ("pool_mean", ctypes.c_int),
+                ("union_softmax", ctypes.c_int)]
 
 
 class HSAError(RuntimeError):
@@ -52,6 +59,9 @@ def _declare(lib):
     lib.hsa_prefill_workspace_size.restype = sz
     lib.hsa_prefill.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, i32,
                                 f32, vp, vp, vp, vp, sz, vp]
+    lib.hsa_prefill_variant.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
+                                        i32, i32, f32, ctypes.POINTER(Variant), vp, vp, vp, vp,
+                                        sz, vp]
     lib.hsa_decode_workspace_size.argtypes = [i32, i32, i32, i64, i32, i32, i32]
     lib.hsa_decode_workspace_size.restype = sz
     lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
@@ -77,7 +87,8 @@ def _declare(lib):
     for n in ("hsa_landmarks", "hsa_prefill", "hsa_decode", "hsa_check", "hsa_version",
               "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
               "hsa_selftest_wait_expiry", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
-              "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine"):
+              "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
+              "hsa_prefill_variant"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -171,9 +182,14 @@ def prefill_workspace_size(B, H, Hkv, L, d, S, topk) -> int:
 
 
 def prefill(Q, K, V, lm=None, *, S: int = 64, topk: int = 8, own_chunk: int = 1,
-            scale: float = 0.0, out=None, idx_out=None, w_out=None, ws=None):
+            scale: float = 0.0, out=None, idx_out=None, w_out=None, ws=None,
+            retrieval_interval: int = 1, pool_mean: bool = False, union_softmax: bool = False):
     """Hierarchical chunk-sparse prefill.  Returns (O, idx, w); idx/w are None
-    unless buffers are given or ``idx_out=True`` / ``w_out=True``."""
+    unless buffers are given or ``idx_out=True`` / ``w_out=True``.  The
+    keyword arguments after ``ws`` select a retrieval variant (hsa_variant_t):
+    one selection per ``retrieval_interval`` tokens from the block's first
+    token (or the mean of its queries with ``pool_mean``), and one softmax
+    over the union of the selected keys with ``union_softmax``."""
     for n, t in (("Q", Q), ("K", K), ("V", V)):
         _dev(t, n)
     B, L, H, d = Q.shape
@@ -194,11 +210,12 @@ def prefill(Q, K, V, lm=None, *, S: int = 64, topk: int = 8, own_chunk: int = 1,
     nbytes = prefill_workspace_size(B, H, Hkv, L, d, S, topk)
     if ws is None:
         ws = workspace(nbytes, dev)
-    st = lib().hsa_prefill(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(lm),
-                           _dtype_code(lm) if lm is not None else HSA_F32, B, H, Hkv, L, d, S,
-                           topk, int(own_chunk), float(scale), _ptr(out),
-                           _ptr(_opt(idx_out)), _ptr(_opt(w_out)), _ptr(ws),
-                           ws.numel() * ws.element_size(), _stream(dev))
+    var = Variant(int(retrieval_interval), int(bool(pool_mean)), int(bool(union_softmax)))
+    st = lib().hsa_prefill_variant(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(lm),
+                                   _dtype_code(lm) if lm is not None else HSA_F32, B, H, Hkv, L,
+                                   d, S, topk, int(own_chunk), float(scale), ctypes.byref(var),
+                                   _ptr(out), _ptr(_opt(idx_out)), _ptr(_opt(w_out)), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(dev))
     _check(st, "hsa_prefill")
     return out, _opt(idx_out), _opt(w_out)
 

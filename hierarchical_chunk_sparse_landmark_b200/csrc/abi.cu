@@ -13,12 +13,12 @@ namespace hsa {
 cudaError_t launch_landmarks(const void *K, bool bf16, float *lm, int B, int Hkv, int64_t L,
                              int d, cudaStream_t st);
 cudaError_t launch_select(const void *Q, bool q_bf16, const void *lm, bool lm_bf16, int B, int H,
-                          int Hkv, int64_t L, int d, int S, int topk, float scale, int32_t *idx,
-                          float *w, cudaStream_t st);
+                          int Hkv, int64_t L, int d, int S, int topk, float scale, int R,
+                          int pool_mean, int32_t *idx, float *w, cudaStream_t st);
 cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool bf16,
                                const int32_t *idx, const float *w, int B, int H, int Hkv,
                                int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                               void *O, cudaStream_t st);
+                               int union_softmax, void *O, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
                           const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
                           int S, int topk, float scale, int splits, const DecodeScratch &ws,
@@ -33,8 +33,8 @@ bool select_tc_supported();
 cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaStream_t st);
 cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
                              int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
-                             int32_t *idx, unsigned *status, bool force_multi_tile, bool *multi,
-                             cudaStream_t st);
+                             int R, int pool_mean, int32_t *idx, unsigned *status,
+                             bool force_multi_tile, bool *multi, cudaStream_t st);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
                           int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
@@ -122,7 +122,7 @@ struct PrefillLayout {
     bool tc;
     int64_t W, NW, cap;
     size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
-        seg_off, tiles_off, zf_off, ownf_off, part_off, own_off, lmsplit_off;
+        seg_off, tiles_off, zf_off, ownf_off, ownm_off, part_off, own_off, lmsplit_off;
 };
 
 PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
@@ -139,7 +139,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     p.W = p.NW = p.cap = 0;
     p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
     p.wntiles_off = p.done_off = p.seg_off = p.tiles_off = p.part_off = p.own_off = 0;
-    p.zf_off = p.ownf_off = p.lmsplit_off = 0;
+    p.zf_off = p.ownf_off = p.ownm_off = p.lmsplit_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
         p.W = tc_window(B, H, Hkv, L, d, topk, attend_tc_max_windows());
@@ -165,6 +165,8 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         p.zf_off = off;
         off = align_up(off + 2 * sizeof(float) * (size_t)B * L * H * topk, 256);
         p.ownf_off = off;
+        off = align_up(off + sizeof(float) * (size_t)B * L * H, 256);
+        p.ownm_off = off;            // own-chunk row maxima (union-softmax fusion)
         off = align_up(off + sizeof(float) * (size_t)B * L * H, 256);
         p.part_off = off;
         off = align_up(off + sizeof(__nv_bfloat16) * (size_t)B * L * H * topk * d, 256);
@@ -291,8 +293,23 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                          int d, int S, int topk, int own_chunk, float scale, void *O,
                          int32_t *idx_out, float *w_out, void *workspace, size_t ws_bytes,
                          void *stream) {
+    return hsa_prefill_variant(Q, K, V, dt, lm, lm_dt, B, H, Hkv, L, d, S, topk, own_chunk, scale,
+                               nullptr, O, idx_out, w_out, workspace, ws_bytes, stream);
+}
+
+hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                 const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                                 int64_t L, int d, int S, int topk, int own_chunk, float scale,
+                                 const hsa_variant_t *variant, void *O, int32_t *idx_out,
+                                 float *w_out, void *workspace, size_t ws_bytes, void *stream) {
     hsa_status_t s = check_shape(B, H, Hkv, L, d, S, topk);
     if (s != HSA_OK) return s;
+    const int R = variant ? variant->retrieval_interval : 1;
+    const int pool_mean = variant ? variant->pool_mean : 0;
+    const int union_softmax = variant ? variant->union_softmax : 0;
+    if (R < 1 || S % R != 0 || (pool_mean != 0 && pool_mean != 1) ||
+        (union_softmax != 0 && union_softmax != 1))
+        return HSA_ERR_INVALID_ARG;
     if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
     if (own_chunk != 0 && own_chunk != 1) return HSA_ERR_INVALID_ARG;
     if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
@@ -348,11 +365,12 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                            !force_simt_select();
     bool multi = false;
     if (tc_select)
-        e = launch_select_tc(Q, lm_use, lm_bf16, lm_split, B, H, Hkv, L, d, S, topk, scale, idx,
-                             (unsigned *)ws, force_multi_tile_select(), &multi, st);
-    else
-        e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, idx,
-                          use_tc ? nullptr : w, st);
+        e = launch_select_tc(Q, lm_use, lm_bf16, lm_split, B, H, Hkv, L, d, S, topk, scale, R,
+                             pool_mean, idx, (unsigned *)ws, force_multi_tile_select(), &multi, st);
+    else   // the CUDA-core attention takes the fusion weights from the selection
+        e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, R, pool_mean,
+                          idx, use_tc ? nullptr : (union_softmax ? (float *)(ws + lay.w_off) : w),
+                          st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
     t_launches += 1;
     t_kernels |= !tc_select ? HSA_K_SELECT_SIMT
@@ -377,6 +395,7 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         a.tiles = (const int4 *)(ws + lay.tiles_off);
         a.qlen = (const int64_t *)(ws + lay.seg_off) + 2 * lay.NW;
         a.zf = (float *)(ws + lay.zf_off); a.own_f = (float *)(ws + lay.ownf_off);
+        a.own_m = (float *)(ws + lay.ownm_off); a.union_softmax = union_softmax;
         a.w_out = w_out;
         a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;
@@ -386,8 +405,11 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
         t_kernels |= e == cudaSuccess ? (unsigned)(HSA_K_ATTEND_TC | HSA_K_FUSE) : 0u;
     } else {
         stage_mark(3, st);
-        e = launch_attend_simt(Q, K, V, bf16, idx, w, B, H, Hkv, L, d, S, topk, own_chunk, scale,
-                               O, st);
+        e = launch_attend_simt(Q, K, V, bf16, idx, union_softmax ? (float *)(ws + lay.w_off) : w,
+                               B, H, Hkv, L, d, S, topk, own_chunk, scale, union_softmax, O, st);
+        // the union softmax has no per-chunk fusion weights: w_out reads 0
+        if (e == cudaSuccess && union_softmax && w_out)
+            e = cudaMemsetAsync(w_out, 0, sizeof(float) * (size_t)B * L * H * topk, st);
         t_launches += e == cudaSuccess ? 1 : 0;
         t_kernels |= e == cudaSuccess ? (unsigned)HSA_K_ATTEND_SIMT : 0u;
         stage_mark(4, st);            // the SIMT kernel fuses in place

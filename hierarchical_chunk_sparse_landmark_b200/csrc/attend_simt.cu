@@ -12,6 +12,11 @@
 // the head dimension, accumulating w_k * o_k in registers.  This is the fp32
 // path (fp32 accumulate end to end) and the reference layout for the
 // tensor-core path.
+//
+// Union-softmax variant (one softmax over the keys of all selected chunks and
+// the own chunk; Dynamic Hierarchical Sparse Attention review): the chunk
+// results are folded with a running maximum instead of the fusion weights,
+// acc = sum_k e^{m_k - M} P_k V_k, den = sum_k e^{m_k - M} sum P_k, O = acc / den.
 #include "common.cuh"
 
 namespace hsa {
@@ -20,7 +25,8 @@ template <typename T, int D>
 __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K,
                                    const T *__restrict__ V, const int32_t *__restrict__ idx,
                                    const float *__restrict__ w, int H, int Hkv, int64_t L, int S,
-                                   int topk, int own_chunk, float scale, T *__restrict__ O) {
+                                   int topk, int own_chunk, float scale, int union_softmax,
+                                   T *__restrict__ O) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int PAD = VEC;                     // 16 bytes of padding per row
     constexpr int RS = D + PAD;                  // row stride (elements)
@@ -44,6 +50,7 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    float run_m = -INFINITY, run_den = 0.f;      // union softmax: running max and sum
 
     const int64_t c_t = t / S;
     const T *Kbg = K + ((int64_t)b * Hkv + g) * L * D;
@@ -60,7 +67,7 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
             if (ci < 0) continue;                    // uniform across the block
             first = (int64_t)ci * S;
             nkeys = S;
-            wt = w[(row * H + h) * topk + it];
+            wt = union_softmax ? 1.f : w[(row * H + h) * topk + it];
         } else {
             first = c_t * S;
             nkeys = (int)(t - first + 1);
@@ -112,9 +119,24 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
 #pragma unroll
             for (int r = 0; r < R; ++r) o_r[r] = fmaf(pj, to_f32(vs[j * RS + lane + 32 * r]), o_r[r]);
         }
-        const float f = wt / den;
+        if (!union_softmax) {
+            const float f = wt / den;
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[r] = fmaf(f, o_r[r], acc[r]);
+            for (int r = 0; r < R; ++r) acc[r] = fmaf(f, o_r[r], acc[r]);
+        } else {
+            const float m_new = fmaxf(run_m, mx);
+            const float c_old = run_m > -INFINITY ? expf(run_m - m_new) : 0.f;
+            const float c_new = expf(mx - m_new);
+            run_den = run_den * c_old + den * c_new;
+#pragma unroll
+            for (int r = 0; r < R; ++r) acc[r] = acc[r] * c_old + o_r[r] * c_new;
+            run_m = m_new;
+        }
+    }
+    if (union_softmax) {
+        const float inv = run_den > 0.f ? 1.f / run_den : 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] *= inv;
     }
     T *op = O + (row * H + h) * (int64_t)D;
 #pragma unroll
@@ -125,7 +147,7 @@ template <typename T, int D>
 static cudaError_t launch_attend_simt_t(const void *Q, const void *K, const void *V,
                                         const int32_t *idx, const float *w, int B, int H,
                                         int Hkv, int64_t L, int S, int topk, int own_chunk,
-                                        float scale, void *O, cudaStream_t st) {
+                                        float scale, int union_softmax, void *O, cudaStream_t st) {
     constexpr int VEC = Vec16<T>::N;
     const int G = H / Hkv;
     const size_t smem = sizeof(float) * G * D + 2 * sizeof(T) * 64 * (D + VEC);
@@ -135,19 +157,19 @@ static cudaError_t launch_attend_simt_t(const void *Q, const void *K, const void
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)L, (unsigned)Hkv, (unsigned)B);
     kern<<<grid, 32 * G, smem, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, w, H, Hkv,
-                                     L, S, topk, own_chunk, scale, (T *)O);
+                                     L, S, topk, own_chunk, scale, union_softmax, (T *)O);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool bf16,
                                const int32_t *idx, const float *w, int B, int H, int Hkv,
                                int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                               void *O, cudaStream_t st) {
+                               int union_softmax, void *O, cudaStream_t st) {
     if (bf16)
-        return d == 128 ? launch_attend_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st)
-                        : launch_attend_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st);
-    return d == 128 ? launch_attend_simt_t<float, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st)
-                    : launch_attend_simt_t<float, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, O, st);
+        return d == 128 ? launch_attend_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st)
+                        : launch_attend_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st);
+    return d == 128 ? launch_attend_simt_t<float, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st)
+                    : launch_attend_simt_t<float, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st);
 }
 
 }  // namespace hsa

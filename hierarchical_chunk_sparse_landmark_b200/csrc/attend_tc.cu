@@ -23,6 +23,13 @@
 // the method, one warp per (t, g):
 //   w = softmax over the token's selected chunks of the logits,
 //   O = f_own * own + sum_k w_k * f_k * partial_k  (bf16 out).
+// Union-softmax variant (one softmax over the keys of all selected chunks and
+// the own chunk; Dynamic Hierarchical Sparse Attention review): the tiles
+// store each row's scaled maximum x = scale * max(S) and row sum r instead of
+// (fusion logit, 1 / r), and the fusion is
+//   O = sum_k e^{x_k - M} partial_k / sum_k e^{x_k - M} r_k,  M = max_k x_k
+// over the selected chunks and the own chunk (when attended); both sums carry
+// the same 2^-6, so it cancels.
 //
 // attend_tc_kernel: one persistent block per SM walks the tile queue (a flat
 // list of tile descriptors) with these roles, linked by mbarriers, a ring of
@@ -83,7 +90,8 @@ struct TcParams {
     const int64_t *qlen;
     const int32_t *entries;
     float *zf;                    // [B, L, H, topk] x (fusion logit, 1 / chunk row sum)
-    float *own_f;                 // [B, L, H] add_own / own-chunk row sum
+    float *own_f;                 // [B, L, H] add_own / own-chunk row sum (union: add_own * row sum)
+    float *own_m;                 // [B, L, H] own-chunk scale * row max (union softmax only)
     __half *part;                 // [B*L*Hkv*topk entries][D/16][G][16] chunk outputs
     __half *own;                  // [B*L*Hkv rows (t, g)][D/16][G][16] own-chunk term
     unsigned *status;
@@ -92,6 +100,7 @@ struct TcParams {
     uint64_t hkv_mul;             // floor(2^32 / Hkv) + 1: bg / Hkv = (bg * hkv_mul) >> 32
     int lm_rows;                  // landmark rows per chunk: 1 (bf16) or 2 (bf16 high, low of fp32)
     int q3d;                      // Q map is the 3-D (cols, rows, d-half) view
+    int union_softmax;            // what the rows store for the fusion (see the file comment)
     float scale, scale_log2e;
 };
 
@@ -495,12 +504,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 l2 = add_f2(l2, add_f2(pack_f2(s0[c], s0[c + 1]), pack_f2(s1[c], s1[c + 1])));
             }
             if (cur.valid) {
-                const float f = __fdividef(cur.tl.own ? (float)p.add_own : 1.f, sum_f2(l2));
-                if (cur.tl.own)
-                    p.own_f[(b * L + cur.t) * H + (int64_t)g * G + h] = f;
-                else
-                    reinterpret_cast<float2 *>(p.zf)[((b * L + cur.t) * H + (int64_t)g * G + h) * topk + cur.k] =
-                        make_float2(p.scale * (l_hi + l_lo), f);
+                const int64_t hrow = (b * L + cur.t) * H + (int64_t)g * G + h;
+                const float rs = sum_f2(l2);
+                if (!p.union_softmax) {
+                    const float f = __fdividef(cur.tl.own ? (float)p.add_own : 1.f, rs);
+                    if (cur.tl.own)
+                        p.own_f[hrow] = f;
+                    else
+                        reinterpret_cast<float2 *>(p.zf)[hrow * topk + cur.k] =
+                            make_float2(p.scale * (l_hi + l_lo), f);
+                } else if (cur.tl.own) {
+                    p.own_f[hrow] = (float)p.add_own * rs;
+                    p.own_m[hrow] = p.scale * mx;
+                } else {
+                    reinterpret_cast<float2 *>(p.zf)[hrow * topk + cur.k] = make_float2(p.scale * mx, rs);
+                }
             }
             // P goes into TMEM next to S slot s (this thread's lane, keys packed
             // in pairs), free once the P.V of tile j - 2 is done
@@ -596,6 +614,7 @@ template <int D, int G, int KP>
 __global__ void __launch_bounds__(256, (G * D / 256) <= 4 ? 2 : 1)
 fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
             const float2 *__restrict__ zf, const float *__restrict__ own_f,
+            const float *__restrict__ own_m, int union_softmax,
             const int32_t *__restrict__ idx, int64_t groups, int H, int Hkv, int topk,
             float *__restrict__ w_out, __nv_bfloat16 *__restrict__ O) {
     constexpr int NP = G * D / 256;                  // 16-byte pieces per lane and slot
@@ -630,22 +649,27 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
             raw[u][i] = u < topk ? pb[(int64_t)u * SLOT + lane + 32 * i] : make_uint4(0u, 0u, 0u, 0u);
     const int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && idx[srow * topk + lane] >= 0));
     // fusion weights of this lane's head: softmax of the logits over the valid slots
+    // (union softmax: e^{x_k - M} over the slots and the own term, normalised by
+    // the matching sum of row sums)
     const float2 *zh = zf + hrow * topk;
     float zx[KP];
 #pragma unroll
     for (int k = 0; k < KP; ++k) zx[k] = k < nsel ? zh[k].x : -INFINITY;
-    float m = -INFINITY;
+    const float fown = own_f[hrow];
+    const float xown = union_softmax && fown > 0.f ? own_m[hrow] : -INFINITY;
+    float m = xown;
 #pragma unroll
     for (int k = 0; k < KP; ++k) m = fmaxf(m, zx[k]);
-    float den = 0.f;
+    float den = union_softmax && fown > 0.f ? __expf(xown - m) * fown : 0.f;
 #pragma unroll
-    for (int k = 0; k < KP; ++k) den += k < nsel ? __expf(zx[k] - m) : 0.f;
-    const float inv = nsel ? 1.f / den : 0.f;
+    for (int k = 0; k < KP; ++k)
+        den += k < nsel ? __expf(zx[k] - m) * (union_softmax ? zh[k].y : 1.f) : 0.f;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
     if (w_out && lane < 2 * G && (lane & 1) == 0)
         for (int k = 0; k < topk; ++k)
-            w_out[hrow * topk + k] = k < nsel ? __expf(zh[k].x - m) * inv : 0.f;
+            w_out[hrow * topk + k] = (k < nsel && !union_softmax) ? __expf(zh[k].x - m) * inv : 0.f;
     float acc[NP][8];
-    const float fo = own_f[hrow];
+    const float fo = union_softmax ? (fown > 0.f ? __expf(xown - m) * inv : 0.f) : fown;
     constexpr int LINES = G * D * 2 / 128;           // 128-byte lines of one slot
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
@@ -673,7 +697,9 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
 #pragma unroll
         for (int u = 0; u < SG; ++u) {
             const bool valid = k0 + u < nsel;
-            const float wk = valid ? __expf(zx[k0 + u] - m) * inv * zh[k0 + u].y : 0.f;
+            const float wk = !valid ? 0.f
+                             : union_softmax ? __expf(zx[k0 + u] - m) * inv
+                                             : __expf(zx[k0 + u] - m) * inv * zh[k0 + u].y;
 #pragma unroll
             for (int i = 0; i < NP; ++i) {
                 const uint4 rv = valid ? raw[u][i] : make_uint4(0u, 0u, 0u, 0u);
@@ -785,7 +811,8 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     if (e != cudaSuccess) return e;
     TcParams p;
     p.tiles = a.tiles; p.qlen = a.qlen;
-    p.entries = a.entries; p.zf = a.zf; p.own_f = a.own_f;
+    p.entries = a.entries; p.zf = a.zf; p.own_f = a.own_f; p.own_m = a.own_m;
+    p.union_softmax = a.union_softmax;
     p.part = a.part; p.own = a.own; p.status = a.status;
     p.L = a.L; p.Nc = a.L / a.S;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
@@ -804,7 +831,8 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     const dim3 fgrid((unsigned)((groups + kWarps - 1) / kWarps));
     auto fk = a.topk <= 8 ? fuse_kernel<D, G, 8> : a.topk <= 16 ? fuse_kernel<D, G, 16> : fuse_kernel<D, G, 32>;
     return launch_pdl(fk, fgrid, dim3(32 * kWarps), 0, st, a.part, a.own,
-                      (const float2 *)a.zf, (const float *)a.own_f, (const int32_t *)a.idx, groups,
+                      (const float2 *)a.zf, (const float *)a.own_f, (const float *)a.own_m,
+                      a.union_softmax, (const int32_t *)a.idx, groups,
                       a.H, a.Hkv, a.topk, a.w_out, (__nv_bfloat16 *)a.O);
 }
 

@@ -20,6 +20,8 @@ struct TcLaunch {
     const int4 *tiles;                // one descriptor per queue position
     const int64_t *qlen;              // number of tiles (device)
     float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
+    float *own_m;                     // [B, L, H]: own-chunk row max (union softmax)
+    int union_softmax;                // 1: one softmax over the union of the selected keys
     __half *part, *own;              // fp16 chunk outputs / own-chunk term
     void *O;
     unsigned *status;

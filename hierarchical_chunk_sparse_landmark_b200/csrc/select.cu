@@ -10,7 +10,12 @@
 // Length Generalization in Hierarchical Sparse Attention Models, "Methodology
 // in Plain English"; fusion by retrieval scores: HiLS Attention abstract.)
 //
-// One block owns 64 consecutive tokens of one (b, g).  Their qbar rows stay
+// With a retrieval interval R > 1 (one selection per R consecutive tokens,
+// R divides S) the block's 64 rows are selection rows: row u serves tokens
+// u*R .. u*R+R-1 and its group query is token u*R's (pool_mean = 0) or the
+// mean over those tokens (pool_mean = 1); the fusion weights stay per token.
+//
+// One block owns 64 consecutive (selection) rows of one (b, g).  Their qbar rows stay
 // in shared memory while the landmark rows of the visible chunks stream
 // through shared memory 32 at a time.  Each thread scores one token against 8
 // chunks of a tile (fp32 FMA, float4 operands) into a shared score tile; then
@@ -29,19 +34,20 @@ constexpr int kSelTokPerWarp = kSelTokens / (kSelThreads / 32);
 template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv, int64_t L,
-              int S, int topk, float scale, int32_t *__restrict__ idx_out,
+              int S, int topk, float scale, int R, int pool_mean, int32_t *__restrict__ idx_out,
               float *__restrict__ w_out) {
     extern __shared__ float4 smem4[];
     float *qbar = reinterpret_cast<float *>(smem4);                 // [64][D+4]
     float *lmt = qbar + kSelTokens * (D + 4);                        // [32][D+4]
     float *sc = lmt + kSelChunks * (D + 4);                          // [64][33]
 
-    const int n_tiles = (int)((L + kSelTokens - 1) / kSelTokens);
+    const int64_t Lsel = (L + R - 1) / R;                           // selection rows
+    const int n_tiles = (int)((Lsel + kSelTokens - 1) / kSelTokens);
     const int tile = n_tiles - 1 - (int)blockIdx.x;                 // heavy tiles first
     const int g = blockIdx.y, b = blockIdx.z;
     const int G = H / Hkv;
     const int64_t Nc = L / S;
-    const int64_t t0 = (int64_t)tile * kSelTokens;
+    const int64_t t0 = (int64_t)tile * kSelTokens;                  // first selection row
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // qbar for the block's tokens (rows past L are zero).  A thread owns one
@@ -57,14 +63,19 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
         for (int u = 0; u < PER; ++u)
 #pragma unroll
             for (int v = 0; v < VT; ++v) acc[u][v] = 0.f;
-        for (int h = 0; h < G; ++h) {
+        // (token, head) pairs of a row: the G heads of its first token, or of
+        // each of its tokens (pool_mean); rows and tokens past the end add 0
+        const int npairs = pool_mean ? G * R : G;
+        for (int h = 0; h < npairs; ++h) {
+            const int tok = h / G, hd = h % G;
             uint4 raw[PER];
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int e = tid + u * kSelThreads, r = e / VPR, c = (e % VPR) * VT;
-                const int64_t t = t0 + r;
-                raw[u] = t < L ? ld_stream16(Q + ((b * L + t) * H + (int64_t)g * G + h) * D + c)
-                               : make_uint4(0, 0, 0, 0);
+                const int64_t t = (t0 + r) * R + tok;
+                raw[u] = (t0 + r < Lsel && t < L)
+                             ? ld_stream16(Q + ((b * L + t) * H + (int64_t)g * G + hd) * D + c)
+                             : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
@@ -74,16 +85,18 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
                 for (int v = 0; v < VT; ++v) acc[u][v] += f[v];
             }
         }
-        const float inv = 1.f / (float)G;
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int e = tid + u * kSelThreads, r = e / VPR, c = (e % VPR) * VT;
+            const int64_t left = L - (t0 + r) * R;
+            const int n = pool_mean ? G * (int)(left < R ? (left > 0 ? left : 1) : R) : G;
+            const float inv = 1.f / (float)n;
 #pragma unroll
             for (int v = 0; v < VT; ++v) qbar[r * (D + 4) + c + v] = acc[u][v] * inv;
         }
     }
-    const int64_t t_last = (t0 + kSelTokens - 1 < L ? t0 + kSelTokens - 1 : L - 1);
-    const int64_t nvis_max = t_last / S;
+    const int64_t t_last = (t0 + kSelTokens - 1 < Lsel ? t0 + kSelTokens - 1 : Lsel - 1);
+    const int64_t nvis_max = t_last * R / S;
 
     // scoring role: token tok_s, chunks sub + 4m of each tile
     const int tok_s = tid >> 2, sub = tid & 3;
@@ -147,8 +160,8 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
 #pragma unroll
         for (int u = 0; u < kSelTokPerWarp; ++u) {
             const int tok = warp * kSelTokPerWarp + u;
-            const int64_t t = t0 + tok;
-            const int64_t nvis = t < L ? t / S : 0;
+            const int64_t t = t0 + tok;                              // selection row
+            const int64_t nvis = t < Lsel ? t * R / S : 0;
             const int64_t i = c0 + lane;
             const uint64_t key = i < nvis ? make_key(sc[tok * 33 + lane], i) : 0ull;
             v[u] = merge_lists(v[u], merge_segments(sort_segments_desc(key, KP), KP), KP);
@@ -164,14 +177,19 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
     const int span = D / PARTS;                       // d elements per lane
 #pragma unroll 1
     for (int u = 0; u < kSelTokPerWarp; ++u) {
-        const int64_t t = t0 + warp * kSelTokPerWarp + u;
-        if (t >= L) continue;
+        const int64_t row = t0 + warp * kSelTokPerWarp + u;
+        if (row >= Lsel) continue;
         const int32_t sel = lane < topk ? key_index(v[u]) : -1;
-        if (lane < topk && idx_out) idx_out[((b * L + t) * Hkv + g) * topk + lane] = sel;
-        if (w_out == nullptr) continue;     // weights computed downstream (tensor-core path)
         const int32_t my_sel = __shfl_sync(0xffffffffu, sel, slot < 32 ? slot : 0);
         const bool active = slot < topk && my_sel >= 0;
         const TL *lp = lm_bg + (int64_t)(my_sel > 0 ? my_sel : 0) * D + part * span;
+        // the row's selection serves its R tokens; the weights are per token
+#pragma unroll 1
+        for (int j = 0; j < R; ++j) {
+        const int64_t t = row * R + j;
+        if (t >= L) break;
+        if (lane < topk && idx_out) idx_out[((b * L + t) * Hkv + g) * topk + lane] = sel;
+        if (w_out == nullptr) continue;     // weights computed downstream (tensor-core path)
 #pragma unroll 1
         for (int h = 0; h < G; ++h) {
             const int hh = g * G + h;
@@ -193,42 +211,44 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
             if (part == 0 && slot < topk)
                 w_out[((b * L + t) * H + hh) * topk + slot] = (active && den > 0.f) ? e / den : 0.f;
         }
+        }
     }
 }
 
 template <typename T, typename TL, int D>
 static cudaError_t launch_select_t(const void *Q, const void *lm, int B, int H, int Hkv,
-                                   int64_t L, int S, int topk, float scale, int32_t *idx,
-                                   float *w, cudaStream_t st) {
+                                   int64_t L, int S, int topk, float scale, int R, int pool_mean,
+                                   int32_t *idx, float *w, cudaStream_t st) {
     const size_t smem =
         sizeof(float) * ((kSelTokens + kSelChunks) * (D + 4) + kSelTokens * 33);
     auto kern = select_kernel<T, TL, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((L + kSelTokens - 1) / kSelTokens), (unsigned)Hkv, (unsigned)B);
+    const int64_t Lsel = (L + R - 1) / R;
+    dim3 grid((unsigned)((Lsel + kSelTokens - 1) / kSelTokens), (unsigned)Hkv, (unsigned)B);
     kern<<<grid, kSelThreads, smem, st>>>((const T *)Q, (const TL *)lm, H, Hkv, L, S, topk,
-                                          scale, idx, w);
+                                          scale, R, pool_mean, idx, w);
     return cudaGetLastError();
 }
 
 template <typename T, typename TL>
 static cudaError_t launch_select_l(const void *Q, const void *lm, int B, int H, int Hkv,
-                                   int64_t L, int d, int S, int topk, float scale, int32_t *idx,
-                                   float *w, cudaStream_t st) {
-    return d == 128 ? launch_select_t<T, TL, 128>(Q, lm, B, H, Hkv, L, S, topk, scale, idx, w, st)
-                    : launch_select_t<T, TL, 64>(Q, lm, B, H, Hkv, L, S, topk, scale, idx, w, st);
+                                   int64_t L, int d, int S, int topk, float scale, int R,
+                                   int pool_mean, int32_t *idx, float *w, cudaStream_t st) {
+    return d == 128 ? launch_select_t<T, TL, 128>(Q, lm, B, H, Hkv, L, S, topk, scale, R, pool_mean, idx, w, st)
+                    : launch_select_t<T, TL, 64>(Q, lm, B, H, Hkv, L, S, topk, scale, R, pool_mean, idx, w, st);
 }
 
 cudaError_t launch_select(const void *Q, bool q_bf16, const void *lm, bool lm_bf16, int B, int H,
-                          int Hkv, int64_t L, int d, int S, int topk, float scale, int32_t *idx,
-                          float *w, cudaStream_t st) {
+                          int Hkv, int64_t L, int d, int S, int topk, float scale, int R,
+                          int pool_mean, int32_t *idx, float *w, cudaStream_t st) {
     using bf = __nv_bfloat16;
     if (q_bf16)
-        return lm_bf16 ? launch_select_l<bf, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st)
-                       : launch_select_l<bf, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st);
-    return lm_bf16 ? launch_select_l<float, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st)
-                   : launch_select_l<float, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, idx, w, st);
+        return lm_bf16 ? launch_select_l<bf, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st)
+                       : launch_select_l<bf, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st);
+    return lm_bf16 ? launch_select_l<float, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st)
+                   : launch_select_l<float, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st);
 }
 
 }  // namespace hsa

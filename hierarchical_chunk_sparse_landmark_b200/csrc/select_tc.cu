@@ -44,7 +44,8 @@ namespace hsa {
 template <int D, bool LM32>
 struct SelCfg {
     static constexpr int M = 128;                 // tokens per block
-    static constexpr int N = 128;                 // chunks per tile
+    static constexpr int N = 128;                 // chunks per score tile (four stages of
+                                                  // 64 chunks were tried: slower)
     static constexpr int KB = D / 64;             // 64-element blocks of d
     static constexpr int QP = LM32 ? 2 : 3;       // qbar parts
     static constexpr int LP = LM32 ? 2 : 1;       // landmark parts
@@ -69,7 +70,22 @@ struct SelTcParams {
     int64_t L, Nc;
     int H, Hkv, S, topk;
     float scale;
+    // one selection per R consecutive tokens (R divides S): selection row u
+    // serves tokens u*R .. u*R+R-1; its group query is token u*R's
+    // (pool_mean = 0) or the mean over the row's tokens (pool_mean = 1)
+    int64_t Lsel;                   // selection rows, ceil(L / R)
+    int R, pool_mean;
 };
+
+// Number of (token, head) query rows summed into the group query of
+// selection row u: the G heads of token u*R, or of every token of the row
+// (pool_mean).  Eight consecutive pairs share a token (G is a multiple of 8
+// on the tensor-core path).
+__device__ __forceinline__ int qbar_pairs(const SelTcParams &p, int G, int64_t u) {
+    if (!p.pool_mean) return G;
+    const int64_t left = p.L - u * p.R;
+    return G * (int)(left < p.R ? left : p.R);
+}
 
 __device__ __forceinline__ bool sel_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (tc::mbar_try_wait(bar, parity)) return true;
@@ -85,6 +101,21 @@ __device__ __forceinline__ bool sel_wait(uint64_t *bar, uint32_t parity, volatil
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// Insert key x (distinct from every key held) into the sorted list v of KP
+// keys, dropping the smallest.  The KP comparisons are independent of each
+// other and every slot takes its new value from its own and its upper
+// neighbour's comparison, so the insertion is a few dependent steps, not a
+// chain through the whole list.
+template <int KP>
+__device__ __forceinline__ void insert_key(uint64_t (&v)[KP], uint64_t x) {
+    bool gt[KP];
+#pragma unroll
+    for (int i = 0; i < KP; ++i) gt[i] = v[i] > x;
+#pragma unroll
+    for (int i = KP - 1; i > 0; --i) v[i] = gt[i] ? v[i] : (gt[i - 1] ? x : v[i - 1]);
+    v[0] = gt[0] ? v[0] : x;
 }
 
 // One 32-column block of a token's scores (chunks c0 .. c0+31, of which the
@@ -106,7 +137,23 @@ template <int KP>
 __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, int lim, float scale,
                                            uint64_t (&v)[KP], float &tf, float *stage, int r) {
     const float tq = tf / scale;                                // scale > 0
-    const float tr = tq - fabsf(tq) * 1e-6f;                    // -inf stays -inf
+    float tr = tq - fabsf(tq) * 1e-6f;                          // -inf stays -inf
+    if (tf == -INFINITY && lim == 32 && KP < 32) {
+        // empty list, full block: the smallest of the maxima of KP groups of
+        // 32/KP columns is a lower bound on the KP-th largest of the 32 (each
+        // group holds a score at or above it), so only scores at or above it
+        // can enter; this keeps the first block from inserting every column
+        constexpr int GS = 32 / (KP < 32 ? KP : 16);
+        float bound = INFINITY;
+#pragma unroll
+        for (int g0 = 0; g0 < 32; g0 += GS) {
+            float m = sc[g0];
+#pragma unroll
+            for (int c = 1; c < GS; ++c) m = fmaxf(m, sc[g0 + c]);
+            bound = fminf(bound, m);
+        }
+        tr = bound;
+    }
     uint32_t mask = 0;
 #pragma unroll
     for (int c = 0; c < 32; ++c) mask |= (sc[c] >= tr ? 1u : 0u) << c;
@@ -120,14 +167,9 @@ __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, in
         mask &= mask - 1;
         const float sv = scale * stage[c * 128 + r];
         if (sv >= tf) {
-            uint64_t x = make_key(sv, c0 + c);
+            const uint64_t x = make_key(sv, c0 + c);
             if (x > v[KP - 1]) {
-#pragma unroll
-                for (int i = 0; i < KP; ++i) {
-                    const uint64_t hi = v[i] > x ? v[i] : x;
-                    x = v[i] > x ? x : v[i];
-                    v[i] = hi;
-                }
+                insert_key<KP>(v, x);
                 tf = key_score(v[KP - 1]);
             }
         }
@@ -143,15 +185,8 @@ template <int KP>
 __device__ __forceinline__ void merge_keys(uint64_t (&v)[KP], const uint64_t *lists, int r) {
 #pragma unroll
     for (int j = 0; j < KP; ++j) {
-        uint64_t x = lists[j * 128 + r];
-        if (x > v[KP - 1]) {
-#pragma unroll
-            for (int i = 0; i < KP; ++i) {
-                const uint64_t hi = v[i] > x ? v[i] : x;
-                x = v[i] > x ? x : v[i];
-                v[i] = hi;
-            }
-        }
+        const uint64_t x = lists[j * 128 + r];
+        if (x > v[KP - 1]) insert_key<KP>(v, x);
     }
 }
 
@@ -166,20 +201,23 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     uint8_t *sA = smem;                                        // [QP][KB][M x 128 B]
     auto sB = [&](int s) { return smem + C::QP * C::A_PART + s * C::B_STAGE; };   // [LP][KB][N x 128 B]
     uint64_t *bars = (uint64_t *)(smem + C::BAR_OFF);
-    uint64_t *full = bars, *empty = bars + 2, *tfull = bars + 4, *tfree = bars + 6;
-    uint32_t *s_tmem = (uint32_t *)(bars + 8);
+    uint64_t *full = bars, *empty = bars + C::STAGES;                  // [STAGES]
+    uint64_t *tfull = bars + 2 * C::STAGES, *tfree = tfull + 2;        // [2] TMEM slots
+    uint32_t *s_tmem = (uint32_t *)(tfree + 2);
+    static_assert((2 * C::STAGES + 4) * 8 + 8 <= 256, "barrier block overflows its reserve");
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
 
-    const int ntb = (int)((p.L + C::M - 1) / C::M);
+    const int ntb = (int)((p.Lsel + C::M - 1) / C::M);
     const int tb = ntb - 1 - (int)blockIdx.x;                  // heavy blocks first
     const int64_t bg = blockIdx.y;
     const int64_t b = bg / p.Hkv;
     const int g = (int)(bg % p.Hkv);
     const int G = p.H / p.Hkv;
-    const int64_t L = p.L;
-    const int64_t t0 = (int64_t)tb * C::M;
-    const int64_t t_last = t0 + C::M - 1 < L ? t0 + C::M - 1 : L - 1;
-    const int64_t nvis_max = t_last / p.S;                     // visible to the block's last token
+    const int64_t L = p.L, Lsel = p.Lsel;
+    const int R = p.R;
+    const int64_t t0 = (int64_t)tb * C::M;                     // first selection row
+    const int64_t t_last = t0 + C::M - 1 < Lsel ? t0 + C::M - 1 : Lsel - 1;
+    const int64_t nvis_max = t_last * R / p.S;                 // visible to the block's last row
     const int ntiles = (int)((nvis_max + C::N - 1) / C::N);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -188,9 +226,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
             tc::mbar_init(&full[s], 1);
             tc::mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&tfull[s], 1);
             tc::mbar_init(&tfree[s], 8);       // one arrive per top-K warp
         }
@@ -199,7 +239,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     }
     // the first landmark tiles do not depend on qbar: start their loads now
     auto issue_tile = [&](int n) {
-        const int s = n & 1;
+        const int s = n % C::STAGES;
         tc::mbar_expect_tx(&full[s], (uint32_t)C::B_STAGE);
         const int row0 = (int)(bg * p.Nc + (int64_t)n * C::N);
 #pragma unroll
@@ -217,28 +257,32 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     {
         constexpr int VPR = D / 8;                            // 16-byte vectors per row
         constexpr int NPAIR = C::M * VPR;
-        const float inv_g = 1.f / (float)G;
         for (int e0 = tid; e0 < NPAIR; e0 += 2 * kSelTcThreads) {
-            float acc[2][8];
+            float acc[2][8], inv[2];
             const __nv_bfloat16 *qp[2];
-            bool live[2];
+            int npairs[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int e = e0 + u * kSelTcThreads;
                 const int r = e / VPR, c = e % VPR;
                 const int64_t t = t0 + r;
-                live[u] = e < NPAIR && t < L;
-                qp[u] = (const __nv_bfloat16 *)p.Q + ((b * L + (live[u] ? t : 0)) * p.H + (int64_t)g * G) * D + c * 8;
+                const bool live = e < NPAIR && t < Lsel;
+                npairs[u] = live ? qbar_pairs(p, G, t) : 0;
+                inv[u] = live ? 1.f / (float)npairs[u] : 0.f;
+                qp[u] = (const __nv_bfloat16 *)p.Q + ((b * L + (live ? t * R : 0)) * p.H + (int64_t)g * G) * D + c * 8;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
             }
-            for (int h0 = 0; h0 < G; h0 += 8) {
+            const int nmax = npairs[0] > npairs[1] ? npairs[0] : npairs[1];
+            for (int h0 = 0; h0 < nmax; h0 += 8) {
+                // pairs h0 .. h0+7: token h0 / G of the row, heads h0 % G ..
+                const int64_t off = (int64_t)(h0 / G) * p.H * D + (int64_t)(h0 % G) * D;
                 uint4 raw[2][8];
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int h = 0; h < 8; ++h)
-                        raw[u][h] = live[u] ? ld_stream16(qp[u] + (int64_t)(h0 + h) * D) : make_uint4(0, 0, 0, 0);
+                        raw[u][h] = h0 < npairs[u] ? ld_stream16(qp[u] + off + (int64_t)h * D) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -257,7 +301,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
                 const uint32_t off = (uint32_t)((c / 8) * (C::M * 128)) + tc::sw128_offset(r, c % 8);
                 float x[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[i] = acc[u][i] * inv_g;
+                for (int i = 0; i < 8; ++i) x[i] = acc[u][i] * inv[u];
 #pragma unroll
                 for (int part = 0; part < C::QP; ++part) {
                     uint32_t w[4];
@@ -283,8 +327,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             for (int n = C::STAGES; n < ntiles; ++n) {
-                const int s = n & 1;
-                if (!sel_wait(&empty[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
+                const int s = n % C::STAGES;
+                if (!sel_wait(&empty[s], (uint32_t)(((n / C::STAGES) + 1) & 1), s_abort)) break;
                 issue_tile(n);
             }
         }
@@ -301,12 +345,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             const uint64_t ad0 = tc::sdesc_sw128(tc::smem_u32(sA), 16, 1024);
             const uint64_t bd0 = tc::sdesc_sw128(tc::smem_u32(sB(0)), 16, 1024);
             for (int n = 0; n < ntiles; ++n) {
-                const int s = n & 1;
-                if (!sel_wait(&full[s], (uint32_t)((n >> 1) & 1), s_abort)) break;
-                if (n >= 2 && !sel_wait(&tfree[s], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
+                const int s = n % C::STAGES, ts = n & 1;          // landmark stage, TMEM slot
+                if (!sel_wait(&full[s], (uint32_t)((n / C::STAGES) & 1), s_abort)) break;
+                if (n >= 2 && !sel_wait(&tfree[ts], (uint32_t)(((n >> 1) + 1) & 1), s_abort)) break;
                 tc::fence_after_sync();
                 const uint64_t bds = bd0 + (uint64_t)(s * (C::B_STAGE / 16));
-                const uint32_t dt = tmem + s * C::N;
+                const uint32_t dt = tmem + ts * C::N;
 #pragma unroll
                 for (int pr = 0; pr < NPROD; ++pr)
 #pragma unroll
@@ -316,7 +360,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
                             tc::mma_bf16(dt, ad0 + (uint64_t)((pa[pr] * C::A_PART + kb * (C::M * 128) + kk * 32) / 16),
                                          bds + (uint64_t)((pl[pr] * C::B_PART + kb * (C::N * 128) + kk * 32) / 16),
                                          IDESC, (pr | kb | kk) ? 1u : 0u);
-                tc::mma_commit(&tfull[s]);
+                tc::mma_commit(&tfull[ts]);
                 tc::mma_commit(&empty[s]);
             }
         }
@@ -329,8 +373,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         const int r = q4 * 32 + lane;
         float *stage = (float *)(smem + C::STAGE_OFF) + hg * (32 * 128);
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const int64_t t = t0 + r;
-        const int64_t nvis = t < L ? t / p.S : 0;
+        const int64_t t = t0 + r;                              // selection row
+        const int64_t nvis = t < Lsel ? t * R / p.S : 0;
         uint64_t v[KP];
 #pragma unroll
         for (int i = 0; i < KP; ++i) v[i] = 0ull;
@@ -369,12 +413,15 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
             for (int k = 0; k < KP; ++k) lists[k * 128 + r] = v[k];
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");     // the two top-K groups
-        if (hg == 0 && t < L) {
+        if (hg == 0 && t < Lsel) {
             merge_keys<KP>(v, lists, r);
-            int32_t *dst = p.idx + ((b * L + t) * p.Hkv + g) * p.topk;
+            // the row's selection serves its R tokens
+            for (int j = 0; j < R && t * R + j < L; ++j) {
+                int32_t *dst = p.idx + ((b * L + t * R + j) * p.Hkv + g) * p.topk;
 #pragma unroll
-            for (int k = 0; k < KP; ++k)
-                if (k < p.topk) dst[k] = key_index(v[k]);
+                for (int k = 0; k < KP; ++k)
+                    if (k < p.topk) dst[k] = key_index(v[k]);
+            }
         }
     }
 
@@ -429,16 +476,17 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
     uint32_t *s_tmem = (uint32_t *)(bars + 3);
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
 
-    const int ntb = (int)((p.L + C::M - 1) / C::M);
+    const int ntb = (int)((p.Lsel + C::M - 1) / C::M);
     const int tb = ntb - 1 - (int)blockIdx.x;                  // heavy blocks first
     const int64_t bg = blockIdx.y;
     const int64_t b = bg / p.Hkv;
     const int g = (int)(bg % p.Hkv);
     const int G = p.H / p.Hkv;
-    const int64_t L = p.L;
-    const int64_t t0 = (int64_t)tb * C::M;
-    const int64_t t_last = t0 + C::M - 1 < L ? t0 + C::M - 1 : L - 1;
-    const int64_t nvis_max = t_last / p.S;                     // visible to the block's last token
+    const int64_t L = p.L, Lsel = p.Lsel;
+    const int R = p.R;
+    const int64_t t0 = (int64_t)tb * C::M;                     // first selection row
+    const int64_t t_last = t0 + C::M - 1 < Lsel ? t0 + C::M - 1 : Lsel - 1;
+    const int64_t nvis_max = t_last * R / p.S;                 // visible to the block's last row
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 1) {
@@ -465,7 +513,6 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    const float inv_g = 1.f / (float)G;
     bool ok = true;
     for (int kb = 0; kb < C::KB; ++kb) {
         if (kb > 0) {
@@ -477,27 +524,31 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
         // pairs and keeps two pairs' loads of eight heads in flight
         constexpr int NPAIR = C::M * 8;
         for (int e0 = tid; e0 < NPAIR; e0 += 2 * kSelHalfThreads) {
-            float acc[2][8];
+            float acc[2][8], inv[2];
             const __nv_bfloat16 *qp[2];
-            bool live[2];
+            int npairs[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int e = e0 + u * kSelHalfThreads;
                 const int r = e / 8, c = e % 8;
                 const int64_t t = t0 + r;
-                live[u] = e < NPAIR && t < L;
-                qp[u] = (const __nv_bfloat16 *)p.Q + ((b * L + (live[u] ? t : 0)) * p.H + (int64_t)g * G) * D +
+                const bool live = e < NPAIR && t < Lsel;
+                npairs[u] = live ? qbar_pairs(p, G, t) : 0;
+                inv[u] = live ? 1.f / (float)npairs[u] : 0.f;
+                qp[u] = (const __nv_bfloat16 *)p.Q + ((b * L + (live ? t * R : 0)) * p.H + (int64_t)g * G) * D +
                         kb * 64 + c * 8;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
             }
-            for (int h0 = 0; h0 < G; h0 += 8) {
+            const int nmax = npairs[0] > npairs[1] ? npairs[0] : npairs[1];
+            for (int h0 = 0; h0 < nmax; h0 += 8) {
+                const int64_t off = (int64_t)(h0 / G) * p.H * D + (int64_t)(h0 % G) * D;
                 uint4 raw[2][8];
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int h = 0; h < 8; ++h)
-                        raw[u][h] = live[u] ? ld_stream16(qp[u] + (int64_t)(h0 + h) * D) : make_uint4(0, 0, 0, 0);
+                        raw[u][h] = h0 < npairs[u] ? ld_stream16(qp[u] + off + (int64_t)h * D) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -516,7 +567,7 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
                 const uint32_t off = tc::sw128_offset(r, c);
                 float x[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[i] = acc[u][i] * inv_g;
+                for (int i = 0; i < 8; ++i) x[i] = acc[u][i] * inv[u];
 #pragma unroll
                 for (int part = 0; part < C::QP; ++part) {
                     uint32_t w[4];
@@ -562,8 +613,8 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const int64_t t = t0 + r;
-        const int64_t nvis = t < L ? t / p.S : 0;
+        const int64_t t = t0 + r;                              // selection row
+        const int64_t nvis = t < Lsel ? t * R / p.S : 0;
         uint64_t v[KP];
 #pragma unroll
         for (int i = 0; i < KP; ++i) v[i] = 0ull;
@@ -591,8 +642,8 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
                                    (float *)sA, r);
             }
             tc::fence_before_sync();
-            if (t < L) {
-                int32_t *dst = p.idx + ((b * L + t) * p.Hkv + g) * p.topk;
+            for (int j = 0; j < R && t < Lsel && t * R + j < L; ++j) {
+                int32_t *dst = p.idx + ((b * L + t * R + j) * p.Hkv + g) * p.topk;
 #pragma unroll
                 for (int k = 0; k < KP; ++k)
                     if (k < p.topk) dst[k] = key_index(v[k]);
@@ -648,14 +699,14 @@ static SelEncodeFn sel_encode_fn() {
     return fn;
 }
 
-// bf16 landmark rows [rows, D]: boxes of 64 columns x 128 rows, 128-byte swizzle;
-// rows past the end read as zero.
-static bool sel_make_map(CUtensorMap *m, const void *base, uint64_t rows, int D) {
+// bf16 landmark rows [rows, D]: boxes of 64 columns x box_rows rows (one
+// score tile's chunks), 128-byte swizzle; rows past the end read as zero.
+static bool sel_make_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows) {
     SelEncodeFn enc = sel_encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64u, 128u};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
     const cuuint32_t es[2] = {1u, 1u};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -668,15 +719,16 @@ static cudaError_t launch_select_tc_t(const SelTcParams &p, int B, const void *l
                                       bool force_multi_tile, bool *multi, cudaStream_t st) {
     using C = SelCfg<D, LM32>;
     const uint64_t rows = (uint64_t)B * p.Hkv * p.Nc;
+    dim3 grid((unsigned)((p.Lsel + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
+    *multi = !(p.Nc <= SelHalfCfg<D, LM32>::N && !force_multi_tile);
+    const int box_rows = *multi ? C::N : SelHalfCfg<D, LM32>::N;
     CUtensorMap m0, m1;
-    if (!sel_make_map(&m0, l0, rows, D)) return cudaErrorInvalidValue;
+    if (!sel_make_map(&m0, l0, rows, D, box_rows)) return cudaErrorInvalidValue;
     if (LM32) {
-        if (!sel_make_map(&m1, l1, rows, D)) return cudaErrorInvalidValue;
+        if (!sel_make_map(&m1, l1, rows, D, box_rows)) return cudaErrorInvalidValue;
     } else {
         m1 = m0;
     }
-    dim3 grid((unsigned)((p.L + C::M - 1) / C::M), (unsigned)(B * p.Hkv));
-    *multi = !(p.Nc <= SelHalfCfg<D, LM32>::N && !force_multi_tile);
     if (!*multi) {
         // every chunk fits one score tile: qbar built per 64-column block, two blocks per SM
         using H = SelHalfCfg<D, LM32>;
@@ -716,11 +768,12 @@ cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaS
 // runs unless `force_multi_tile`; `*multi` tells which kernel was launched.
 cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
                              int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
-                             int32_t *idx, unsigned *status, bool force_multi_tile, bool *multi,
-                             cudaStream_t st) {
+                             int R, int pool_mean, int32_t *idx, unsigned *status,
+                             bool force_multi_tile, bool *multi, cudaStream_t st) {
     SelTcParams p;
     p.Q = Q; p.idx = idx; p.status = status;
     p.L = L; p.Nc = L / S; p.H = H; p.Hkv = Hkv; p.S = S; p.topk = topk; p.scale = scale;
+    p.R = R; p.pool_mean = pool_mean; p.Lsel = (L + R - 1) / R;
     const bool fm = force_multi_tile;
     if (lm_bf16) {
         return d == 128 ? launch_select_tc_k<128, false>(p, B, lm, nullptr, fm, multi, st)

@@ -131,6 +131,48 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Retrieval variants of the prefill (hsa_prefill_variant).  Zero-filled it is
+ * hsa_prefill's method except retrieval_interval, which must then be 1.
+ *  retrieval_interval  R >= 1 dividing S: one selection per block of R
+ *                      consecutive tokens (blocks start at token 0), shared by
+ *                      the block's tokens; 1 = per-token retrieval.  The HSA
+ *                      summary ("Main Findings") compares per-token with
+ *                      per-8-token retrieval (R = 8).
+ *  pool_mean           0: the block's selection is that of its first token
+ *                      (its group query, its visible chunks -- the block never
+ *                      straddles a chunk, so all its tokens see the same ones);
+ *                      1: the group query is the mean over the block's tokens
+ *                      (with R = S, the DHSA chunk-level query: sqrt(|C|) times
+ *                      the mean of the chunk's queries, "What carries the
+ *                      argument"; the positive factor does not change the
+ *                      ranking).  The fusion weights stay per token.
+ *  union_softmax       0: softmax inside each selected chunk, outputs fused by
+ *                      the softmax of the token's landmark scores (HiLS);
+ *                      1: one softmax over the keys of all selected chunks and,
+ *                      with own_chunk, of the own chunk's keys c_t*S .. t (the
+ *                      DHSA form of attention under the selected-chunk mask);
+ *                      w_out is then all zero.
+ */
+typedef struct {
+    int retrieval_interval;
+    int pool_mean;
+    int union_softmax;
+} hsa_variant_t;
+
+/*
+ * hsa_prefill_variant -- hsa_prefill with a retrieval variant (NULL: the
+ * per-token HiLS method of hsa_prefill, which calls this).  Same arguments,
+ * layouts, workspace (hsa_prefill_workspace_size) and statuses; an invalid
+ * variant returns HSA_ERR_INVALID_ARG.
+ */
+hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                 const void *lm, hsa_dtype_t lm_dt,
+                                 int B, int H, int Hkv, int64_t L, int d, int S, int topk,
+                                 int own_chunk, float scale, const hsa_variant_t *variant,
+                                 void *O, int32_t *idx_out, float *w_out,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * hsa_decode_workspace_size -- bytes of device workspace hsa_decode needs
  * (0 on invalid arguments; the size depends on the current device's SM
  * count).  It holds a status word, per-(sequence, group) tickets and work

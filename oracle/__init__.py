@@ -49,7 +49,8 @@ def _bind(lib):
     lib.hsa_oracle_decode_attend.argtypes = [dp, dp, dp, dp, i32p, i32, i32, i32, i64, i32,
                                              i32, i32, dbl, dp, dp]
     lib.hsa_oracle_prefill_variant.argtypes = [dp, i64p, i64, dp, dp, dp, i32, i32, i32, i64, i32,
-                                               i32, i32, i32, dbl, i32, i32, i32, dp, i32p, dp]
+                                               i32, i32, i32, dbl, i32, i32, i32, dp, i32p, dp,
+                                               dp, dp, dp]
     for name in ("hsa_oracle_landmarks", "hsa_oracle_prefill", "hsa_oracle_decode_select",
                  "hsa_oracle_decode_attend", "hsa_oracle_num_threads",
                  "hsa_oracle_prefill_variant"):
@@ -159,7 +160,8 @@ class Oracle:
         per `interval` tokens (first token's or mean group query), HiLS fusion
         or one softmax over the union of the selected keys.  Q [B,L,H,d] (all
         tokens), K/V [B,Hkv,L,d], lm [B,Hkv,L//S,d] or None (DHSA).
-        Returns dict O [n,H,d], idx [n,Hkv,K], w [n,H,K]."""
+        Returns dict O [n,H,d], idx [n,Hkv,K], w [n,H,K], sbar [n,Hkv,K],
+        gap [n,Hkv], smag [n,Hkv,K+1] (of the block's selection, as for prefill)."""
         qf, k, v = _f64(Q), _f64(K), _f64(V)
         B, L, H, d = qf.shape
         Hkv = k.shape[1]
@@ -171,13 +173,17 @@ class Oracle:
         O = np.zeros((n, H, d), dtype=np.float64)
         idx = np.zeros((n, Hkv, topk), dtype=np.int32)
         w = np.zeros((n, H, topk), dtype=np.float64)
+        sbar = np.zeros((n, Hkv, topk), dtype=np.float64)
+        gap = np.zeros((n, Hkv), dtype=np.float64)
+        smag = np.zeros((n, Hkv, topk + 1), dtype=np.float64)
         rc = self.lib.hsa_oracle_prefill_variant(
             _dp(qf), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _dp(k), _dp(v),
             _dp(lmf), B, H, Hkv, L, d, S, topk, int(own_chunk), float(scale), int(interval),
             int(pool_mean), int(union_softmax), _dp(O),
-            idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(w))
+            idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(w), _dp(sbar), _dp(gap),
+            _dp(smag))
         _check(rc, "prefill_variant")
-        return {"O": O, "idx": idx, "w": w, "rows": rows}
+        return {"O": O, "idx": idx, "w": w, "sbar": sbar, "gap": gap, "smag": smag, "rows": rows}
 
     def decode_select(self, q, lm, topk: int, scale: float = 0.0):
         """q [B,H,d], lm [B,Hkv,Nc,d] -> dict idx [B,Hkv,K], sbar, gap, smag."""

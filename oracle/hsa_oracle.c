@@ -342,13 +342,16 @@ int hsa_oracle_prefill(const double *q, const int64_t *rows, int64_t n_rows,
  *   rows [n_rows]      flattened positions b*L + t to compute
  * Outputs O [n_rows, H, d], idx [n_rows, Hkv, topk] (may be NULL),
  * w [n_rows, H, topk] (may be NULL; the fusion weights of the HiLS form,
- * zero with union_softmax).
+ * zero with union_softmax), and, as for hsa_oracle_prefill, the block
+ * selection's group scores sbar [n_rows, Hkv, topk], gap [n_rows, Hkv] and
+ * score-term magnitudes smag [n_rows, Hkv, topk+1] (all may be NULL).
  */
 int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_rows,
                                const double *k, const double *v, const double *lm,
                                int B, int H, int Hkv, int64_t L, int d, int S, int topk,
                                int own_chunk, double scale, int interval, int pool_mean,
-                               int union_softmax, double *O, int32_t *idx, double *w)
+                               int union_softmax, double *O, int32_t *idx, double *w,
+                               double *sbar, double *gap, double *smag)
 {
     if (!Q || !rows || !k || !v || !O) return ORACLE_BAD_ARG;
     if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || L < 1 || d < 1 || S < 1 || topk < 1)
@@ -417,6 +420,17 @@ int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_r
             if (idx)
                 for (int kk = 0; kk < topk; ++kk)
                     idx[(r * Hkv + g) * topk + kk] = kk < nsel ? (int32_t)sel[kk] : -1;
+            if (sbar)
+                for (int kk = 0; kk < topk; ++kk)
+                    sbar[(r * Hkv + g) * topk + kk] = kk < nsel ? cand[kk].score : 0.0;
+            if (gap)
+                gap[r * Hkv + g] = nvis > topk ? cand[topk - 1].score - cand[topk].score : INFINITY;
+            if (smag) {
+                double *m = smag + (r * Hkv + g) * (topk + 1);
+                for (int kk = 0; kk < topk; ++kk)
+                    m[kk] = kk < nsel ? scale * abs_dot(qbar, lm_bg + sel[kk] * d, d) : 0.0;
+                m[topk] = nvis > topk ? scale * abs_dot(qbar, lm_bg + cand[topk].index * d, d) : 0.0;
+            }
 
             for (int h = 0; h < G; ++h) {
                 const int hh = g * G + h;

@@ -571,3 +571,17 @@ def test_variant_union_softmax_of_every_chunk_is_causal_attention(oracle_lib):
         r = oracle_lib.prefill_variant(Q, K, V, lm, 8, 6, 1, union_softmax=1, interval=interval)
         ref = sdpa_causal(Q, K, V, 2)
         np.testing.assert_allclose(r["O"].reshape(ref.shape), ref, atol=1e-12, rtol=0)
+
+
+def test_variant_gap_and_magnitudes_are_those_of_the_block_selection(oracle_lib):
+    """The near-tie gap and score-term magnitudes of a block's selection are
+    those of the per-token oracle at the block's first token (first-token
+    pooling), for every token of the block."""
+    Q, K, V, lm = rand_case(35, 1, 8 * 9 + 5, 4, 2, 8, 8)
+    L = Q.shape[1]
+    r = oracle_lib.prefill_variant(Q, K, V, lm, 8, 3, 1, interval=4)
+    starts = (np.arange(L) // 4) * 4
+    ref = oracle_lib.prefill(Q, K, V, lm, 8, 3, 1, rows=starts)
+    np.testing.assert_array_equal(r["sbar"], ref["sbar"])
+    np.testing.assert_array_equal(r["gap"], ref["gap"])
+    np.testing.assert_array_equal(r["smag"], ref["smag"])
