@@ -49,8 +49,8 @@ def _bind(lib):
     lib.hsa_oracle_decode_attend.argtypes = [dp, dp, dp, dp, i32p, i32, i32, i32, i64, i32,
                                              i32, i32, dbl, dp, dp]
     lib.hsa_oracle_prefill_variant.argtypes = [dp, i64p, i64, dp, dp, dp, i32, i32, i32, i64, i32,
-                                               i32, i32, i32, dbl, i32, i32, i32, dp, i32p, dp,
-                                               dp, dp, dp]
+                                               i32, i32, i32, dbl, i32, i32, i32, i64p, i64, dp,
+                                               i32p, dp, dp, dp, dp]
     for name in ("hsa_oracle_landmarks", "hsa_oracle_prefill", "hsa_oracle_decode_select",
                  "hsa_oracle_decode_attend", "hsa_oracle_num_threads",
                  "hsa_oracle_prefill_variant"):
@@ -155,11 +155,13 @@ class Oracle:
 
     def prefill_variant(self, Q, K, V, lm, S: int, topk: int, own_chunk: int = 1,
                         scale: float = 0.0, interval: int = 1, pool_mean: int = 0,
-                        union_softmax: int = 0, rows=None):
+                        union_softmax: int = 0, rows=None, bounds=None):
         """Retrieval variants (see hsa_oracle_prefill_variant): one selection
         per `interval` tokens (first token's or mean group query), HiLS fusion
         or one softmax over the union of the selected keys.  Q [B,L,H,d] (all
-        tokens), K/V [B,Hkv,L,d], lm [B,Hkv,L//S,d] or None (DHSA).
+        tokens), K/V [B,Hkv,L,d], lm [B,Hkv,L//S,d] or None (DHSA).  ``bounds``
+        (n+1 increasing token offsets from 0 to L): variable-length chunks, lm
+        then [B,Hkv,n,d] or None (sqrt(|C|) * mean of each chunk's keys).
         Returns dict O [n,H,d], idx [n,Hkv,K], w [n,H,K], sbar [n,Hkv,K],
         gap [n,Hkv], smag [n,Hkv,K+1] (of the block's selection, as for prefill)."""
         qf, k, v = _f64(Q), _f64(K), _f64(V)
@@ -176,10 +178,13 @@ class Oracle:
         sbar = np.zeros((n, Hkv, topk), dtype=np.float64)
         gap = np.zeros((n, Hkv), dtype=np.float64)
         smag = np.zeros((n, Hkv, topk + 1), dtype=np.float64)
+        bnd = None if bounds is None else np.ascontiguousarray(bounds, dtype=np.int64)
         rc = self.lib.hsa_oracle_prefill_variant(
             _dp(qf), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _dp(k), _dp(v),
             _dp(lmf), B, H, Hkv, L, d, S, topk, int(own_chunk), float(scale), int(interval),
-            int(pool_mean), int(union_softmax), _dp(O),
+            int(pool_mean), int(union_softmax),
+            None if bnd is None else bnd.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+            0 if bnd is None else len(bnd) - 1, _dp(O),
             idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _dp(w), _dp(sbar), _dp(gap),
             _dp(smag))
         _check(rc, "prefill_variant")

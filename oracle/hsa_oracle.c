@@ -338,6 +338,15 @@ int hsa_oracle_prefill(const double *q, const int64_t *rows, int64_t n_rows,
  *                      Hierarchical Sparse Attention review, "What carries the
  *                      argument": attention under the selected-chunk mask).
  *
+ * Variable-length chunks (Dynamic Hierarchical Sparse Attention review, "What
+ * carries the argument": chunks of varying size, represented by sqrt(|C|)
+ * times the mean of their keys): with bounds = {0 = c_0 < c_1 < ... < c_n = L}
+ * chunk i holds tokens c_i .. c_{i+1} - 1, its landmark (lm == NULL) is
+ * sqrt(|C_i|) * mean of its keys, the visible chunks of token t are those
+ * before the chunk holding t, and the own chunk starts at that chunk's first
+ * token.  bounds == NULL: chunks of S tokens (the last may be partial and has
+ * no landmark).  interval must be 1 with bounds.
+ *
  *   Q    [B, L, H, d]  all queries (pooling reads the block's other tokens)
  *   rows [n_rows]      flattened positions b*L + t to compute
  * Outputs O [n_rows, H, d], idx [n_rows, Hkv, topk] (may be NULL),
@@ -350,7 +359,8 @@ int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_r
                                const double *k, const double *v, const double *lm,
                                int B, int H, int Hkv, int64_t L, int d, int S, int topk,
                                int own_chunk, double scale, int interval, int pool_mean,
-                               int union_softmax, double *O, int32_t *idx, double *w,
+                               int union_softmax, const int64_t *bounds, int64_t n_chunks,
+                               double *O, int32_t *idx, double *w,
                                double *sbar, double *gap, double *smag)
 {
     if (!Q || !rows || !k || !v || !O) return ORACLE_BAD_ARG;
@@ -359,19 +369,44 @@ int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_r
     if (interval < 1 || S % interval != 0) return ORACLE_BAD_ARG;
     for (int64_t r = 0; r < n_rows; ++r)
         if (rows[r] < 0 || rows[r] >= (int64_t)B * L) return ORACLE_BAD_ARG;
+    int64_t maxlen = S;                    /* longest chunk */
+    if (bounds) {
+        if (interval != 1 || n_chunks < 1 || bounds[0] != 0 || bounds[n_chunks] != L)
+            return ORACLE_BAD_ARG;
+        maxlen = 0;
+        for (int64_t i = 0; i < n_chunks; ++i) {
+            if (bounds[i + 1] <= bounds[i]) return ORACLE_BAD_ARG;
+            if (bounds[i + 1] - bounds[i] > maxlen) maxlen = bounds[i + 1] - bounds[i];
+        }
+    }
     const int G = H / Hkv;
-    const int64_t Nc = L / S;
+    /* chunks with a landmark: every varlen chunk, the complete ones of fixed S */
+    const int64_t Nc = bounds ? n_chunks : L / S;
     if (scale == 0.0) scale = 1.0 / sqrt((double)d);
 
     double *lm_dhsa = NULL;
     if (!lm) {
         lm_dhsa = (double *)malloc(sizeof(double) * (size_t)B * Hkv * (Nc > 0 ? Nc : 1) * d);
         if (!lm_dhsa) return ORACLE_NO_MEMORY;
-        hsa_oracle_landmarks(k, B, Hkv, L, d, S, lm_dhsa);
+        if (!bounds) {
+            hsa_oracle_landmarks(k, B, Hkv, L, d, S, lm_dhsa);
+        } else {
+            /* sqrt(|C_i|) * mean of chunk i's keys */
+            for (int64_t bg = 0; bg < (int64_t)B * Hkv; ++bg)
+                for (int64_t i = 0; i < Nc; ++i) {
+                    const int64_t n = bounds[i + 1] - bounds[i];
+                    for (int j = 0; j < d; ++j) {
+                        double sum = 0.0;
+                        for (int64_t r = bounds[i]; r < bounds[i + 1]; ++r)
+                            sum += k[(bg * L + r) * d + j];
+                        lm_dhsa[(bg * Nc + i) * d + j] = sqrt((double)n) * (sum / (double)n);
+                    }
+                }
+        }
         lm = lm_dhsa;
     }
     int status = ORACLE_OK;
-    const int64_t maxkeys = (int64_t)topk * S + S;
+    const int64_t maxkeys = (int64_t)topk * maxlen + maxlen;
 
 #pragma omp parallel
     {
@@ -396,8 +431,14 @@ int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_r
             const int64_t t = rows[r] % L;
             const int64_t t0 = (t / interval) * interval;      /* the block's first token */
             const int64_t t1 = t0 + interval < L ? t0 + interval : L;
-            const int64_t c = t / S;                            /* own chunk (= t0's) */
+            /* own chunk (t0's): the chunk holding t; chunks before it are visible */
+            int64_t c = t / S;
+            if (bounds) {
+                c = 0;
+                while (bounds[c + 1] <= t) ++c;
+            }
             const int64_t nvis = c;
+            const int64_t own_first = bounds ? bounds[c] : c * S;
             const double *lm_bg = lm + ((b * Hkv + g) * Nc) * d;
             const double *k_bg = k + ((b * Hkv + g) * L) * d;
             const double *v_bg = v + ((b * Hkv + g) * L) * d;
@@ -443,24 +484,27 @@ int hsa_oracle_prefill_variant(const double *Q, const int64_t *rows, int64_t n_r
                         wk[kk] = scale * dot(q_h, lm_bg + sel[kk] * d, d);
                     softmax_inplace(wk, (int)nsel);
                     for (int64_t kk = 0; kk < nsel; ++kk) {
-                        const int64_t first = sel[kk] * S;
-                        chunk_attention(q_h, k_bg + first * d, v_bg + first * d, S, d, scale,
+                        const int64_t first = bounds ? bounds[sel[kk]] : sel[kk] * S;
+                        const int64_t len = bounds ? bounds[sel[kk] + 1] - first : S;
+                        chunk_attention(q_h, k_bg + first * d, v_bg + first * d, len, d, scale,
                                         logit, o_part);
                         for (int j = 0; j < d; ++j) o_row[j] += wk[kk] * o_part[j];
                     }
                     if (own_chunk) {
-                        const int64_t first = c * S;
-                        chunk_attention(q_h, k_bg + first * d, v_bg + first * d, t - first + 1,
-                                        d, scale, logit, o_part);
+                        chunk_attention(q_h, k_bg + own_first * d, v_bg + own_first * d,
+                                        t - own_first + 1, d, scale, logit, o_part);
                         for (int j = 0; j < d; ++j) o_row[j] += o_part[j];
                     }
                 } else {
                     /* DHSA form: one softmax over the union of the selected keys */
                     int64_t nk = 0;
-                    for (int64_t kk = 0; kk < nsel; ++kk)
-                        for (int64_t jj = 0; jj < S; ++jj) keyrow[nk++] = sel[kk] * S + jj;
+                    for (int64_t kk = 0; kk < nsel; ++kk) {
+                        const int64_t first = bounds ? bounds[sel[kk]] : sel[kk] * S;
+                        const int64_t len = bounds ? bounds[sel[kk] + 1] - first : S;
+                        for (int64_t jj = 0; jj < len; ++jj) keyrow[nk++] = first + jj;
+                    }
                     if (own_chunk)
-                        for (int64_t jj = c * S; jj <= t; ++jj) keyrow[nk++] = jj;
+                        for (int64_t jj = own_first; jj <= t; ++jj) keyrow[nk++] = jj;
                     if (nk > 0) {
                         double m = -INFINITY;
                         for (int64_t e = 0; e < nk; ++e) {

@@ -585,3 +585,52 @@ def test_variant_gap_and_magnitudes_are_those_of_the_block_selection(oracle_lib)
     np.testing.assert_array_equal(r["sbar"], ref["sbar"])
     np.testing.assert_array_equal(r["gap"], ref["gap"])
     np.testing.assert_array_equal(r["smag"], ref["smag"])
+
+
+# --------------------------------------------------------------------------- variable-length chunks
+@pytest.mark.parametrize("own", [0, 1])
+@pytest.mark.parametrize("given_lm", [False, True])
+def test_varlen_chunks_match_the_numpy_restatement(oracle_lib, own, given_lm):
+    """Variable-length chunks in the C oracle equal oracle/varlen.py (pinned
+    to the fixed-chunk oracle, to causal attention and to the landmark closed
+    form), for DHSA landmarks sqrt(|C|) * mean and for given landmarks."""
+    from oracle import varlen
+    rng = np.random.default_rng(40 + own + 2 * given_lm)
+    B, L, H, Hkv, d = 2, 71, 4, 2, 8
+    Q = rng.standard_normal((B, L, H, d))
+    K = rng.standard_normal((B, Hkv, L, d))
+    V = rng.standard_normal((B, Hkv, L, d))
+    bounds = [0, 5, 13, 14, 30, 37, 50, 64, 71]
+    n = len(bounds) - 1
+    lm = rng.standard_normal((B, Hkv, n, d)) if given_lm else None
+    for union in (0, 1):
+        r = oracle_lib.prefill_variant(Q, K, V, lm, 16, 3, own, bounds=bounds, union_softmax=union)
+        if union:
+            continue
+        ref = varlen.varlen_prefill(Q, K, V, bounds, 3, own, lm=lm)
+        np.testing.assert_array_equal(r["idx"], ref["idx"].reshape(B * L, Hkv, 3))
+        np.testing.assert_allclose(r["O"], ref["O"].reshape(B * L, H, d), atol=1e-12, rtol=0)
+
+
+def test_varlen_union_softmax_of_every_chunk_is_causal_attention(oracle_lib):
+    """Variable chunks, every visible chunk selected and the own chunk: one
+    softmax over all keys up to t, i.e. causal attention (float64 SDPA)."""
+    Q, K, V, _ = rand_case(41, 1, 40, 4, 2, 8, 8)
+    bounds = [0, 3, 11, 12, 25, 33, 40]
+    r = oracle_lib.prefill_variant(Q, K, V, None, 8, 6, 1, bounds=bounds, union_softmax=1)
+    ref = sdpa_causal(Q, K, V, 2)
+    np.testing.assert_allclose(r["O"].reshape(ref.shape), ref, atol=1e-12, rtol=0)
+
+
+def test_varlen_uniform_bounds_equal_fixed_chunks(oracle_lib):
+    """Boundaries every S tokens (the last chunk partial and, unlike the fixed
+    form, holding a landmark of its own): selection over the complete chunks
+    is unchanged only where the partial chunk is not visible, i.e. everywhere
+    when L is a multiple of S; then the outputs equal the fixed-chunk oracle."""
+    Q, K, V, lm = rand_case(42, 2, 64, 4, 2, 8, 8)
+    bounds = list(range(0, 65, 8))
+    for own in (0, 1):
+        r = oracle_lib.prefill_variant(Q, K, V, lm, 8, 3, own, bounds=bounds)
+        ref = oracle_lib.prefill(Q, K, V, lm, 8, 3, own)
+        np.testing.assert_array_equal(r["idx"], ref["idx"])
+        np.testing.assert_allclose(r["O"], ref["O"], atol=1e-13, rtol=0)

@@ -58,6 +58,11 @@ MUTANTS = {
     # retrieval variants: mean pooling over the block's first token only
     "variant_mean_pool_first_only": ("const int64_t u1 = pool_mean ? t1 : t0 + 1;",
                                      "const int64_t u1 = t0 + 1;"),
+    # variable-length chunks: own chunk starting at a multiple of S, landmark without sqrt(|C|)
+    "varlen_own_chunk_fixed_start": ("const int64_t own_first = bounds ? bounds[c] : c * S;",
+                                     "const int64_t own_first = c * S;"),
+    "varlen_landmark_without_sqrt": ("lm_dhsa[(bg * Nc + i) * d + j] = sqrt((double)n) * (sum / (double)n);",
+                                     "lm_dhsa[(bg * Nc + i) * d + j] = sum / (double)n;"),
     # forced selection: chunks not visible from the row are kept
     "forced_visibility_filter_dropped": ("if (f[kk] >= 0 && f[kk] < nvis) sel[nsel++] = f[kk];",
                                          "if (f[kk] >= 0 && f[kk] < Nc) sel[nsel++] = f[kk];"),
