@@ -32,7 +32,7 @@ EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry",
             "hsa_last_call_kernels", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
             "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
-            "hsa_prefill_variant")
+            "hsa_prefill_variant", "hsa_prefill_varlen_workspace_size", "hsa_prefill_varlen")
 
 
 class Variant(ctypes.Structure):
@@ -62,6 +62,10 @@ def _declare(lib):
     lib.hsa_prefill_variant.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
                                         i32, i32, f32, ctypes.POINTER(Variant), vp, vp, vp, vp,
                                         sz, vp]
+    lib.hsa_prefill_varlen_workspace_size.argtypes = [i32, i32, i32, i64, i32, i64, i32]
+    lib.hsa_prefill_varlen_workspace_size.restype = sz
+    lib.hsa_prefill_varlen.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, vp,
+                                       i64, i32, i32, f32, i32, vp, vp, vp, vp, sz, vp]
     lib.hsa_decode_workspace_size.argtypes = [i32, i32, i32, i64, i32, i32, i32]
     lib.hsa_decode_workspace_size.restype = sz
     lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
@@ -88,7 +92,7 @@ def _declare(lib):
               "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
               "hsa_selftest_wait_expiry", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
               "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
-              "hsa_prefill_variant"):
+              "hsa_prefill_variant", "hsa_prefill_varlen"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -217,6 +221,54 @@ def prefill(Q, K, V, lm=None, *, S: int = 64, topk: int = 8, own_chunk: int = 1,
                                    _ptr(out), _ptr(_opt(idx_out)), _ptr(_opt(w_out)), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(dev))
     _check(st, "hsa_prefill")
+    return out, _opt(idx_out), _opt(w_out)
+
+
+def prefill_varlen_workspace_size(B, H, Hkv, L, d, n_chunks, topk) -> int:
+    return int(lib().hsa_prefill_varlen_workspace_size(B, H, Hkv, L, d, n_chunks, topk))
+
+
+def prefill_varlen(Q, K, V, bounds, lm=None, *, topk: int = 8, own_chunk: int = 1,
+                   scale: float = 0.0, union_softmax: bool = False, out=None, idx_out=None,
+                   w_out=None, ws=None):
+    """Prefill over variable-length chunks (hsa_prefill_varlen): ``bounds``
+    holds the n+1 chunk boundaries 0 = b_0 < ... < b_n = L (a sequence, or an
+    int32 tensor on Q's device), each chunk at most 64 tokens.  ``lm`` is
+    [B, Hkv, n, d] or None (sqrt(|C|) * mean of each chunk's keys).  Returns
+    (O, idx, w) as prefill does.  Wrong boundaries are found on the device:
+    check(ws) then raises HSA_ERR_INVALID_ARG."""
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _dev(t, n)
+    B, L, H, d = Q.shape
+    Hkv = K.shape[1]
+    if K.shape != (B, Hkv, L, d) or V.shape != K.shape:
+        raise ValueError("K and V must be [B, Hkv, L, d] matching Q [B, L, H, d]")
+    dev = Q.device
+    if not isinstance(bounds, torch.Tensor):
+        bounds = torch.tensor(list(bounds), dtype=torch.int32, device=dev)
+    _dev(bounds, "bounds")
+    if bounds.dtype != torch.int32 or bounds.dim() != 1 or bounds.numel() < 2:
+        raise ValueError("bounds must be a 1-D int32 tensor of n_chunks + 1 offsets")
+    n_chunks = bounds.numel() - 1
+    if lm is not None:
+        _dev(lm, "lm")
+        if lm.shape != (B, Hkv, n_chunks, d):
+            raise ValueError(f"lm must be [B, Hkv, n_chunks, d] = {(B, Hkv, n_chunks, d)}")
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx_out is True:
+        idx_out = torch.empty(B, L, Hkv, topk, dtype=torch.int32, device=dev)
+    if w_out is True:
+        w_out = torch.empty(B, L, H, topk, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(prefill_varlen_workspace_size(B, H, Hkv, L, d, n_chunks, topk), dev)
+    st = lib().hsa_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(lm),
+                                  _dtype_code(lm) if lm is not None else HSA_F32, B, H, Hkv, L,
+                                  d, _ptr(bounds), n_chunks, topk, int(own_chunk), float(scale),
+                                  int(bool(union_softmax)), _ptr(out), _ptr(_opt(idx_out)),
+                                  _ptr(_opt(w_out)), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(dev))
+    _check(st, "hsa_prefill_varlen")
     return out, _opt(idx_out), _opt(w_out)
 
 

@@ -13,12 +13,18 @@ namespace hsa {
 cudaError_t launch_landmarks(const void *K, bool bf16, float *lm, int B, int Hkv, int64_t L,
                              int d, cudaStream_t st);
 cudaError_t launch_select(const void *Q, bool q_bf16, const void *lm, bool lm_bf16, int B, int H,
-                          int Hkv, int64_t L, int d, int S, int topk, float scale, int R,
-                          int pool_mean, int32_t *idx, float *w, cudaStream_t st);
+                          int Hkv, int64_t L, int d, int S, int64_t Nc, const int32_t *bounds,
+                          const int32_t *tok_chunk, int topk, float scale, int R, int pool_mean,
+                          int32_t *idx, float *w, cudaStream_t st);
 cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool bf16,
                                const int32_t *idx, const float *w, int B, int H, int Hkv,
                                int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                               int union_softmax, void *O, cudaStream_t st);
+                               int union_softmax, const int32_t *bounds, const int32_t *tok_chunk,
+                               void *O, cudaStream_t st);
+cudaError_t launch_varlen_setup(const int32_t *bounds, int64_t n, int64_t L, int32_t *bs,
+                                int32_t *tok_chunk, unsigned *status, cudaStream_t st);
+cudaError_t launch_landmarks_varlen(const void *K, bool bf16, float *lm, int B, int Hkv, int64_t L,
+                                    int d, const int32_t *bounds, int64_t n, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
                           const void *lm, bool lm_bf16, int B, int H, int Hkv, int64_t Lc, int d,
                           int S, int topk, float scale, int splits, const DecodeScratch &ws,
@@ -32,13 +38,15 @@ int decode_splits(int B, int Hkv, int64_t Nc, int num_sms);
 bool select_tc_supported();
 cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaStream_t st);
 cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
-                             int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
-                             int R, int pool_mean, int32_t *idx, unsigned *status,
+                             int H, int Hkv, int64_t L, int d, int S, int64_t Nc, int topk,
+                             float scale, int R, int pool_mean, const int32_t *bounds,
+                             const int32_t *tok_chunk, int32_t *idx, unsigned *status,
                              bool force_multi_tile, bool *multi, cudaStream_t st);
 cudaError_t launch_bucket(const int32_t *idx, int B, int Hkv, int64_t L, int topk, int64_t Nc,
-                          int ept, int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
+                          int S, const int32_t *bounds, const int32_t *tok_chunk, int ept,
+                          int64_t W, int64_t cap, int32_t *counts, int32_t *cursor,
                           int32_t *entries, int4 *wtiles, int32_t *wntiles, int32_t *done,
-                          int64_t *seg_start, int4 *tiles, cudaStream_t st);
+                          int32_t *wown, int64_t *seg_start, int4 *tiles, cudaStream_t st);
 cudaError_t launch_selftest_wait(unsigned *status, long long budget, cudaStream_t st);
 // Status word of hsa_decode_noalloc's fixed array on the stream's device
 // (decode_noalloc.cu); nullptr when the array is unused there and !mark.
@@ -117,17 +125,18 @@ int64_t tc_window(int B, int H, int Hkv, int64_t L, int d, int topk, int64_t max
 }
 
 struct PrefillLayout {
-    size_t idx_off, w_off, lm_off, total;
+    size_t idx_off, w_off, lm_off, tokc_off, bnds_off, total;
     // tensor-core path (present when tc_shape_ok)
     bool tc;
     int64_t W, NW, cap;
     size_t counts_off, counts_bytes, cursor_off, entries_off, wtiles_off, wntiles_off, done_off,
-        seg_off, tiles_off, zf_off, ownf_off, ownm_off, part_off, own_off, lmsplit_off;
+        wown_off, seg_off, tiles_off, zf_off, ownf_off, ownm_off, part_off, own_off, lmsplit_off;
 };
 
-PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
+// Nc: chunks with a landmark (L / S, or the number of variable-length chunks).
+PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, int64_t Nc,
+                             bool varlen) {
     PrefillLayout p;
-    const int64_t Nc = L / S;
     size_t off = kStatusBytes;
     p.idx_off = off;
     off = align_up(off + sizeof(int32_t) * (size_t)B * L * Hkv * topk, 256);
@@ -135,10 +144,14 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     off = align_up(off + sizeof(float) * (size_t)B * L * H * topk, 256);
     p.lm_off = off;
     off = align_up(off + sizeof(float) * (size_t)B * Hkv * Nc * d, 256);
+    p.tokc_off = off;                // chunk of every token (variable-length chunks)
+    if (varlen) off = align_up(off + sizeof(int32_t) * (size_t)L, 256);
+    p.bnds_off = off;                // checked boundaries + verdict (variable-length chunks)
+    if (varlen) off = align_up(off + sizeof(int32_t) * (size_t)(Nc + 2), 256);
     p.tc = tc_shape_ok(B, H, Hkv, L, d, topk);
     p.W = p.NW = p.cap = 0;
     p.counts_off = p.counts_bytes = p.cursor_off = p.entries_off = p.wtiles_off = 0;
-    p.wntiles_off = p.done_off = p.seg_off = p.tiles_off = p.part_off = p.own_off = 0;
+    p.wntiles_off = p.done_off = p.wown_off = p.seg_off = p.tiles_off = p.part_off = p.own_off = 0;
     p.zf_off = p.ownf_off = p.ownm_off = p.lmsplit_off = 0;
     if (p.tc) {
         const int ept = 128 / (H / Hkv);
@@ -158,10 +171,15 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
         off = align_up(off + sizeof(int32_t) * (size_t)p.NW, 256);
         p.done_off = off;
         off = align_up(off + sizeof(int32_t) * (size_t)p.NW, 256);
+        p.wown_off = off;            // own-chunk tiles per window
+        off = align_up(off + sizeof(int32_t) * (size_t)p.NW, 256);
         p.seg_off = off;
         off = align_up(off + sizeof(int64_t) * (size_t)(2 * p.NW + 1), 256);
         p.tiles_off = off;           // retrieved tiles + own-chunk tiles of every window
-        off = align_up(off + sizeof(int4) * (size_t)(p.NW * (p.cap + (p.W + ept - 1) / ept)), 256);
+        // own-chunk tiles: a window's tokens in groups of ept, cut at chunk
+        // starts as well with variable-length chunks (at most one per token)
+        const int64_t own_cap = varlen ? p.W : (p.W + ept - 1) / ept;
+        off = align_up(off + sizeof(int4) * (size_t)(p.NW * (p.cap + own_cap)), 256);
         p.zf_off = off;
         off = align_up(off + 2 * sizeof(float) * (size_t)B * L * H * topk, 256);
         p.ownf_off = off;
@@ -285,7 +303,14 @@ hsa_status_t hsa_landmarks(const void *K, hsa_dtype_t k_dt, float *lm_out, int B
 
 size_t hsa_prefill_workspace_size(int B, int H, int Hkv, int64_t L, int d, int S, int topk) {
     if (check_shape(B, H, Hkv, L, d, S, topk) != HSA_OK) return 0;
-    return prefill_layout(B, H, Hkv, L, d, S, topk).total;
+    return prefill_layout(B, H, Hkv, L, d, S, topk, L / S, false).total;
+}
+
+size_t hsa_prefill_varlen_workspace_size(int B, int H, int Hkv, int64_t L, int d, int64_t n_chunks,
+                                         int topk) {
+    if (check_shape(B, H, Hkv, L, d, kChunk, topk) != HSA_OK) return 0;
+    if (n_chunks < 1 || n_chunks > L || n_chunks * (int64_t)kMaxVarChunk < L) return 0;
+    return prefill_layout(B, H, Hkv, L, d, kChunk, topk, n_chunks, true).total;
 }
 
 hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
@@ -297,11 +322,18 @@ hsa_status_t hsa_prefill(const void *Q, const void *K, const void *V, hsa_dtype_
                                nullptr, O, idx_out, w_out, workspace, ws_bytes, stream);
 }
 
-hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
-                                 const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
-                                 int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                                 const hsa_variant_t *variant, void *O, int32_t *idx_out,
-                                 float *w_out, void *workspace, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The prefill behind every entry point: chunks of S tokens (bounds == null)
+// or n_chunks variable-length chunks (bounds on the device).
+hsa_status_t prefill_impl(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                          const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t L,
+                          int d, int S, int topk, int own_chunk, float scale,
+                          const hsa_variant_t *variant, const int32_t *bounds, int64_t n_chunks,
+                          void *O, int32_t *idx_out, float *w_out, void *workspace,
+                          size_t ws_bytes, void *stream) {
     hsa_status_t s = check_shape(B, H, Hkv, L, d, S, topk);
     if (s != HSA_OK) return s;
     const int R = variant ? variant->retrieval_interval : 1;
@@ -321,12 +353,15 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
         if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
     if ((lm && !aligned16(lm)) || (idx_out && !aligned16(idx_out)) || (w_out && !aligned16(w_out)))
         return HSA_ERR_INVALID_ARG;
-    const PrefillLayout lay = prefill_layout(B, H, Hkv, L, d, S, topk);
+    const bool varlen = bounds != nullptr;
+    const int64_t Nc = varlen ? n_chunks : L / S;
+    const PrefillLayout lay = prefill_layout(B, H, Hkv, L, d, S, topk, Nc, varlen);
     if (ws_bytes < lay.total) return HSA_ERR_WORKSPACE;
     if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
 
     cudaStream_t st = (cudaStream_t)stream;
     char *ws = (char *)workspace;
+    int32_t *tok_chunk = varlen ? (int32_t *)(ws + lay.tokc_off) : nullptr;
     int32_t *idx = idx_out ? idx_out : (int32_t *)(ws + lay.idx_off);
     float *w = w_out ? w_out : (float *)(ws + lay.w_off);
     const bool bf16 = dt == HSA_BF16;
@@ -339,12 +374,23 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
     // can follow its predecessor as a programmatic dependent
     if (use_tc && cudaMemsetAsync(ws + lay.counts_off, 0, lay.counts_bytes, st) != cudaSuccess)
         return HSA_ERR_CUDA;
+    if (varlen) {   // checked boundaries and the chunk of every token; every later
+                    // kernel reads those (wrong boundaries flag the status word)
+        int32_t *bs = (int32_t *)(ws + lay.bnds_off);
+        if (launch_varlen_setup(bounds, n_chunks, L, bs, tok_chunk, (unsigned *)ws, st) !=
+            cudaSuccess)
+            return HSA_ERR_CUDA;
+        t_launches += 2;
+        bounds = bs;
+    }
     if (!lm) {
         float *lm_ws = (float *)(ws + lay.lm_off);
-        cudaError_t e = launch_landmarks(K, bf16, lm_ws, B, Hkv, L, d, st);
+        cudaError_t e = varlen ? launch_landmarks_varlen(K, bf16, lm_ws, B, Hkv, L, d, bounds,
+                                                         n_chunks, st)
+                               : launch_landmarks(K, bf16, lm_ws, B, Hkv, L, d, st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
-        t_launches += L / S > 0 ? 1 : 0;
-        t_kernels |= L / S > 0 ? (unsigned)HSA_K_LANDMARKS : 0u;
+        t_launches += Nc > 0 ? 1 : 0;
+        t_kernels |= Nc > 0 ? (unsigned)HSA_K_LANDMARKS : 0u;
         lm_use = lm_ws;
         lm_bf16 = false;
     }
@@ -355,33 +401,34 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
     // fp32 landmarks on the tensor-core path: split once into bf16 high / low
     // planes, which the selection and the attention tiles both read
     void *lm_split = ws + lay.lmsplit_off;
-    if (use_tc && !lm_bf16 && L >= S) {
-        e = launch_split_landmarks(lm_use, lm_split, (int64_t)B * Hkv * (L / S) * d, st);
+    if (use_tc && !lm_bf16 && Nc > 0) {
+        e = launch_split_landmarks(lm_use, lm_split, (int64_t)B * Hkv * Nc * d, st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
         t_launches += 1;
         t_kernels |= HSA_K_SPLIT_LANDMARKS;
     }
-    const bool tc_select = use_tc && L >= S && (H / Hkv) % 8 == 0 && select_tc_supported() &&
+    const bool tc_select = use_tc && Nc > 0 && (H / Hkv) % 8 == 0 && select_tc_supported() &&
                            !force_simt_select();
     bool multi = false;
     if (tc_select)
-        e = launch_select_tc(Q, lm_use, lm_bf16, lm_split, B, H, Hkv, L, d, S, topk, scale, R,
-                             pool_mean, idx, (unsigned *)ws, force_multi_tile_select(), &multi, st);
+        e = launch_select_tc(Q, lm_use, lm_bf16, lm_split, B, H, Hkv, L, d, S, Nc, topk, scale, R,
+                             pool_mean, bounds, tok_chunk, idx, (unsigned *)ws,
+                             force_multi_tile_select(), &multi, st);
     else   // the CUDA-core attention takes the fusion weights from the selection
-        e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, topk, scale, R, pool_mean,
-                          idx, use_tc ? nullptr : (union_softmax ? (float *)(ws + lay.w_off) : w),
-                          st);
+        e = launch_select(Q, bf16, lm_use, lm_bf16, B, H, Hkv, L, d, S, Nc, bounds, tok_chunk,
+                          topk, scale, R, pool_mean, idx,
+                          use_tc ? nullptr : (union_softmax ? (float *)(ws + lay.w_off) : w), st);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
     t_launches += 1;
     t_kernels |= !tc_select ? HSA_K_SELECT_SIMT
                             : multi ? HSA_K_SELECT_TC_MULTI_TILE : HSA_K_SELECT_TC_ONE_TILE;
     stage_mark(2, st);
     if (use_tc) {
-        const int64_t Nc = L / S;
-        e = launch_bucket(idx, B, Hkv, L, topk, Nc, 128 / (H / Hkv), lay.W, lay.cap,
-                          (int32_t *)(ws + lay.counts_off), (int32_t *)(ws + lay.cursor_off),
-                          (int32_t *)(ws + lay.entries_off), (int4 *)(ws + lay.wtiles_off),
-                          (int32_t *)(ws + lay.wntiles_off), (int32_t *)(ws + lay.done_off),
+        e = launch_bucket(idx, B, Hkv, L, topk, Nc, S, bounds, tok_chunk, 128 / (H / Hkv), lay.W,
+                          lay.cap, (int32_t *)(ws + lay.counts_off),
+                          (int32_t *)(ws + lay.cursor_off), (int32_t *)(ws + lay.entries_off),
+                          (int4 *)(ws + lay.wtiles_off), (int32_t *)(ws + lay.wntiles_off),
+                          (int32_t *)(ws + lay.done_off), (int32_t *)(ws + lay.wown_off),
                           (int64_t *)(ws + lay.seg_off), (int4 *)(ws + lay.tiles_off), st);
         if (e != cudaSuccess) return HSA_ERR_CUDA;
         t_launches += 3;                  // count, scan, fill (scatter + flatten)
@@ -396,6 +443,7 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
         a.qlen = (const int64_t *)(ws + lay.seg_off) + 2 * lay.NW;
         a.zf = (float *)(ws + lay.zf_off); a.own_f = (float *)(ws + lay.ownf_off);
         a.own_m = (float *)(ws + lay.ownm_off); a.union_softmax = union_softmax;
+        a.Nc = Nc; a.bounds = bounds; a.tok_chunk = tok_chunk;
         a.w_out = w_out;
         a.part = (__half *)(ws + lay.part_off); a.own = (__half *)(ws + lay.own_off);
         a.O = O; a.status = (unsigned *)ws;
@@ -406,7 +454,8 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
     } else {
         stage_mark(3, st);
         e = launch_attend_simt(Q, K, V, bf16, idx, union_softmax ? (float *)(ws + lay.w_off) : w,
-                               B, H, Hkv, L, d, S, topk, own_chunk, scale, union_softmax, O, st);
+                               B, H, Hkv, L, d, S, topk, own_chunk, scale, union_softmax, bounds,
+                               tok_chunk, O, st);
         // the union softmax has no per-chunk fusion weights: w_out reads 0
         if (e == cudaSuccess && union_softmax && w_out)
             e = cudaMemsetAsync(w_out, 0, sizeof(float) * (size_t)B * L * H * topk, st);
@@ -416,6 +465,33 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
     }
     stage_mark(5, st);
     return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                 const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                                 int64_t L, int d, int S, int topk, int own_chunk, float scale,
+                                 const hsa_variant_t *variant, void *O, int32_t *idx_out,
+                                 float *w_out, void *workspace, size_t ws_bytes, void *stream) {
+    return prefill_impl(Q, K, V, dt, lm, lm_dt, B, H, Hkv, L, d, S, topk, own_chunk, scale,
+                        variant, nullptr, 0, O, idx_out, w_out, workspace, ws_bytes, stream);
+}
+
+hsa_status_t hsa_prefill_varlen(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                                int64_t L, int d, const int32_t *bounds, int64_t n_chunks,
+                                int topk, int own_chunk, float scale, int union_softmax,
+                                void *O, int32_t *idx_out, float *w_out, void *workspace,
+                                size_t ws_bytes, void *stream) {
+    if (n_chunks < 1 || n_chunks > L || n_chunks * (int64_t)kMaxVarChunk < L)
+        return L == 0 ? HSA_OK : HSA_ERR_INVALID_ARG;
+    if (!bounds || !aligned16(bounds)) return HSA_ERR_INVALID_ARG;
+    const hsa_variant_t v = {1, 0, union_softmax};
+    return prefill_impl(Q, K, V, dt, lm, lm_dt, B, H, Hkv, L, d, kChunk, topk, own_chunk, scale,
+                        &v, bounds, n_chunks, O, idx_out, w_out, workspace, ws_bytes, stream);
 }
 
 size_t hsa_decode_workspace_size(int B, int H, int Hkv, int64_t Lc, int d, int S, int topk) {
@@ -592,10 +668,10 @@ hsa_status_t hsa_check(void *workspace, void *stream) {
     unsigned flags = 0;
     if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
         return HSA_ERR_CUDA;
-    if (flags & kFlagTimeout) {
+    if (flags & (kFlagTimeout | kFlagBadBounds)) {
         const unsigned zero = 0;
         cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice);
-        return HSA_ERR_TIMEOUT;
+        return (flags & kFlagTimeout) ? HSA_ERR_TIMEOUT : HSA_ERR_INVALID_ARG;
     }
     return HSA_OK;
 }

@@ -26,7 +26,7 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
                                    const T *__restrict__ V, const int32_t *__restrict__ idx,
                                    const float *__restrict__ w, int H, int Hkv, int64_t L, int S,
                                    int topk, int own_chunk, float scale, int union_softmax,
-                                   T *__restrict__ O) {
+                                   Chunks ch, T *__restrict__ O) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int PAD = VEC;                     // 16 bytes of padding per row
     constexpr int RS = D + PAD;                  // row stride (elements)
@@ -52,7 +52,7 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
     float run_m = -INFINITY, run_den = 0.f;      // union softmax: running max and sum
 
-    const int64_t c_t = t / S;
+    const int64_t c_t = chunk_of(ch, t);
     const T *Kbg = K + ((int64_t)b * Hkv + g) * L * D;
     const T *Vbg = V + ((int64_t)b * Hkv + g) * L * D;
     const int32_t *ip = idx + (row * Hkv + g) * topk;
@@ -65,11 +65,11 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
         if (it < topk) {
             const int32_t ci = ip[it];
             if (ci < 0) continue;                    // uniform across the block
-            first = (int64_t)ci * S;
-            nkeys = S;
+            first = chunk_first(ch, ci);
+            nkeys = chunk_len(ch, ci);
             wt = union_softmax ? 1.f : w[(row * H + h) * topk + it];
         } else {
-            first = c_t * S;
+            first = chunk_first(ch, c_t);
             nkeys = (int)(t - first + 1);
             wt = 1.f;
         }
@@ -77,10 +77,11 @@ __global__ void attend_simt_kernel(const T *__restrict__ Q, const T *__restrict_
         const int vec_per_row = D / VEC;
         for (int e = threadIdx.x; e < nkeys * vec_per_row; e += nthr) {
             const int r = e / vec_per_row, c = (e % vec_per_row) * VEC;
+            const bool in = first + r < L;             // clamped boundaries stay in the cache
             *reinterpret_cast<uint4 *>(ks + r * RS + c) =
-                *reinterpret_cast<const uint4 *>(Kbg + (first + r) * D + c);
+                in ? *reinterpret_cast<const uint4 *>(Kbg + (first + r) * D + c) : make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4 *>(vs + r * RS + c) =
-                *reinterpret_cast<const uint4 *>(Vbg + (first + r) * D + c);
+                in ? *reinterpret_cast<const uint4 *>(Vbg + (first + r) * D + c) : make_uint4(0, 0, 0, 0);
         }
         __syncthreads();
         // logits for keys lane and lane+32
@@ -147,7 +148,8 @@ template <typename T, int D>
 static cudaError_t launch_attend_simt_t(const void *Q, const void *K, const void *V,
                                         const int32_t *idx, const float *w, int B, int H,
                                         int Hkv, int64_t L, int S, int topk, int own_chunk,
-                                        float scale, int union_softmax, void *O, cudaStream_t st) {
+                                        float scale, int union_softmax, Chunks ch, void *O,
+                                        cudaStream_t st) {
     constexpr int VEC = Vec16<T>::N;
     const int G = H / Hkv;
     const size_t smem = sizeof(float) * G * D + 2 * sizeof(T) * 64 * (D + VEC);
@@ -157,19 +159,21 @@ static cudaError_t launch_attend_simt_t(const void *Q, const void *K, const void
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)L, (unsigned)Hkv, (unsigned)B);
     kern<<<grid, 32 * G, smem, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, w, H, Hkv,
-                                     L, S, topk, own_chunk, scale, union_softmax, (T *)O);
+                                     L, S, topk, own_chunk, scale, union_softmax, ch, (T *)O);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool bf16,
                                const int32_t *idx, const float *w, int B, int H, int Hkv,
                                int64_t L, int d, int S, int topk, int own_chunk, float scale,
-                               int union_softmax, void *O, cudaStream_t st) {
+                               int union_softmax, const int32_t *bounds, const int32_t *tok_chunk,
+                               void *O, cudaStream_t st) {
+    const Chunks ch = {bounds, tok_chunk, L, S};
     if (bf16)
-        return d == 128 ? launch_attend_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st)
-                        : launch_attend_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st);
-    return d == 128 ? launch_attend_simt_t<float, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st)
-                    : launch_attend_simt_t<float, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, O, st);
+        return d == 128 ? launch_attend_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, ch, O, st)
+                        : launch_attend_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, ch, O, st);
+    return d == 128 ? launch_attend_simt_t<float, 128>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, ch, O, st)
+                    : launch_attend_simt_t<float, 64>(Q, K, V, idx, w, B, H, Hkv, L, S, topk, own_chunk, scale, union_softmax, ch, O, st);
 }
 
 }  // namespace hsa

@@ -101,6 +101,7 @@ struct TcParams {
     int lm_rows;                  // landmark rows per chunk: 1 (bf16) or 2 (bf16 high, low of fp32)
     int q3d;                      // Q map is the 3-D (cols, rows, d-half) view
     int union_softmax;            // what the rows store for the fusion (see the file comment)
+    Chunks ch;                    // chunks of S tokens or variable-length ones (<= 64 tokens)
     float scale, scale_log2e;
 };
 
@@ -182,10 +183,11 @@ __device__ __forceinline__ void decode_tile(const TcParams &p, const int4 &d, Ti
     tl.bg = d.x;
     tl.own = (d.w & kOwnTileFlag) ? 1 : 0;
     tl.n = d.w & (kOwnTileFlag - 1);
+    tl.chunk = d.y;                      // the tile's chunk (own tiles: the tokens' chunk)
     if (!tl.own) {
-        tl.chunk = d.y; tl.first = d.z; tl.t0 = 0;
+        tl.first = d.z; tl.t0 = 0;
     } else {
-        tl.t0 = d.z; tl.chunk = (int)(tl.t0 >> 6); tl.first = 0;     // S = 64 on this path
+        tl.t0 = d.z; tl.first = 0;
     }
 }
 
@@ -296,7 +298,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tmem = *s_tmem;
     const int64_t qlen = *p.qlen;
     const int64_t L = p.L;
-    const int H = p.H, Hkv = p.Hkv, topk = p.topk, S = p.S;
+    const int H = p.H, Hkv = p.Hkv, topk = p.topk;
     const int64_t my_tiles = qlen > blockIdx.x ? (qlen - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
     if (warp == 0 || warp == kProducer2) {
@@ -334,7 +336,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const int q = (int)(j % C::NQK);
             if (lane == 0 && j >= C::NQK) ok = wait_bar(&qk_empty[q], reuse_parity(j / C::NQK), s_abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const int krow = (int)(d0.bg * L + (int64_t)d0.chunk * S);
+            const int krow = (int)(d0.bg * L + chunk_first(p.ch, d0.chunk));
             if (lane == 0) {
                 const uint32_t lbytes = d0.own ? 0u : (uint32_t)(C::KB * 128 * p.lm_rows);
                 tc::mbar_expect_tx(&qk_full[q], (uint32_t)(d0.n * G * D * 2 + C::K_TMA_BYTES) + lbytes);
@@ -472,9 +474,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             warp_arrive(&sfree[s]);
-            // own-chunk rows see keys c*S .. t only: mask the rest to -inf
-            if (cur.tl.own) {
-                const int nk = cur.valid ? (int)(cur.t - (int64_t)cur.tl.chunk * S) + 1 : 64;
+            // own-chunk rows see the keys of their chunk up to t only, and a
+            // variable-length chunk has fewer than 64 keys (the rows past it
+            // belong to the next chunk): mask the rest to -inf
+            int nk = 64;
+            if (cur.tl.own)
+                nk = cur.valid ? (int)(cur.t - chunk_first(p.ch, cur.tl.chunk)) + 1 : 64;
+            else if (p.ch.bounds)
+                nk = chunk_len(p.ch, cur.tl.chunk);
+            if (nk < 64) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     if (c >= nk) s0[c] = -INFINITY;
@@ -802,7 +810,7 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     if (!make_map(&mk, a.K, (uint64_t)a.B * a.Hkv * a.L, D, 64) ||
         !make_map(&mv, a.V, (uint64_t)a.B * a.Hkv * a.L, D, 64))
         return cudaErrorInvalidValue;
-    const uint64_t lrows = (uint64_t)a.B * a.Hkv * (a.L / a.S);
+    const uint64_t lrows = (uint64_t)a.B * a.Hkv * a.Nc;
     if (lrows == 0) ml = mk;                       // no chunk tiles: the map is never used
     else if (!(a.lm_bf16 ? make_map(&ml, a.lm, lrows, D, 1) : make_map_planes(&ml, a.lm, lrows, D)))
         return cudaErrorInvalidValue;
@@ -813,8 +821,9 @@ static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEv
     p.tiles = a.tiles; p.qlen = a.qlen;
     p.entries = a.entries; p.zf = a.zf; p.own_f = a.own_f; p.own_m = a.own_m;
     p.union_softmax = a.union_softmax;
+    p.ch.bounds = a.bounds; p.ch.tok_chunk = a.tok_chunk; p.ch.L = a.L; p.ch.S = a.S;
     p.part = a.part; p.own = a.own; p.status = a.status;
-    p.L = a.L; p.Nc = a.L / a.S;
+    p.L = a.L; p.Nc = a.Nc;
     p.H = a.H; p.Hkv = a.Hkv; p.topk = a.topk; p.S = a.S; p.add_own = a.own_chunk;
     p.hkv_mul = (uint64_t)(0x100000000ull / (uint64_t)a.Hkv) + 1ull;
     p.lm_rows = a.lm_bf16 ? 1 : 2;

@@ -22,6 +22,8 @@ struct TcLaunch {
     float *zf, *own_f, *w_out;        // zf: [B, L, H, topk] float2; own_f: [B, L, H]
     float *own_m;                     // [B, L, H]: own-chunk row max (union softmax)
     int union_softmax;                // 1: one softmax over the union of the selected keys
+    int64_t Nc;                       // chunks with a landmark
+    const int32_t *bounds, *tok_chunk;  // variable-length chunks (null: chunks of S tokens)
     __half *part, *own;              // fp16 chunk outputs / own-chunk term
     void *O;
     unsigned *status;

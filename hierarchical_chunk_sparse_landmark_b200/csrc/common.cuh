@@ -217,11 +217,41 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// ---------------------------------------------------------------- chunk geometry
+// Chunks of S tokens, or variable-length chunks given by their boundaries
+// (chunk c holds tokens bounds[c] .. bounds[c+1] - 1, at most 64 of them;
+// tok_chunk[t] = the chunk holding token t).  The helpers clamp what they
+// return to [0, L] and lengths to [0, 64], so that kernels stay inside their
+// buffers whatever the boundaries hold (wrong boundaries are reported through
+// the status word by varlen_setup_kernel).
+struct Chunks {
+    const int32_t *bounds;      // [n+1] or null: chunks of S tokens
+    const int32_t *tok_chunk;   // [L]   or null
+    int64_t L;
+    int S;
+};
+constexpr int kMaxVarChunk = 64;
+__device__ __forceinline__ int64_t chunk_first(const Chunks &c, int64_t i) {
+    if (!c.bounds) return i * c.S;
+    const int64_t f = c.bounds[i];
+    return f < 0 ? 0 : f > c.L ? c.L : f;
+}
+__device__ __forceinline__ int chunk_len(const Chunks &c, int64_t i) {
+    if (!c.bounds) return c.S;
+    const int64_t n = (int64_t)c.bounds[i + 1] - c.bounds[i];
+    return n < 0 ? 0 : n > kMaxVarChunk ? kMaxVarChunk : (int)n;
+}
+// Chunk holding token t: the chunks before it are the visible ones.
+__device__ __forceinline__ int64_t chunk_of(const Chunks &c, int64_t t) {
+    return c.tok_chunk ? (int64_t)c.tok_chunk[t] : t / c.S;
+}
+
 // ---------------------------------------------------------------- status word
 // The first 256 bytes of every workspace.  word[0] = error flags set by kernels
 // (bit 0: a bounded wait gave up).
 constexpr size_t kStatusBytes = 256;
 constexpr unsigned kFlagTimeout = 1u;
+constexpr unsigned kFlagBadBounds = 2u;     // variable-length chunk boundaries invalid
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -81,4 +81,108 @@ cudaError_t launch_landmarks(const void *K, bool bf16, float *lm, int B, int Hkv
                     : launch_landmarks_t<float, 64>(K, lm, B, Hkv, L, st);
 }
 
+// ---------------------------------------------------------------- variable-length chunks
+// Checks the boundaries (0 = b_0 < b_1 < ... < b_n = L, no chunk longer than
+// 64 tokens) in one block and stores the verdict in bs[n + 1].  Wrong
+// boundaries also set kFlagBadBounds in the status word (hsa_check reports
+// them).
+__global__ void __launch_bounds__(1024)
+varlen_check_kernel(const int32_t *__restrict__ bounds, int64_t n, int64_t L,
+                    int32_t *__restrict__ bs, unsigned *__restrict__ status) {
+    bool bad = false;
+    for (int64_t c = threadIdx.x; c < n; c += blockDim.x) {
+        const int64_t lo = bounds[c], hi = bounds[c + 1];
+        bad |= hi <= lo || hi - lo > kMaxVarChunk || lo < 0 || hi > L;
+        bad |= c == 0 && lo != 0;
+        bad |= c == n - 1 && hi != L;
+    }
+    bad = __syncthreads_or(bad);
+    if (threadIdx.x == 0) {
+        bs[n + 1] = bad ? 1 : 0;
+        if (bad) atomicOr(status, kFlagBadBounds);
+    }
+}
+
+// The boundaries every later kernel reads, bs[0..n], and tok_chunk[t] = the
+// chunk holding token t.  bs is a copy of the caller's boundaries when they
+// passed the check and an even split of the L tokens into n chunks otherwise
+// (each 1..64 tokens, as n <= L <= 64 n), so that no kernel of a call with
+// wrong boundaries reads or writes outside its buffers.  One thread per chunk.
+__global__ void __launch_bounds__(256)
+varlen_setup_kernel(const int32_t *__restrict__ bounds, int64_t n, int64_t L,
+                    int32_t *__restrict__ bs, int32_t *__restrict__ tok_chunk) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= n) return;
+    const bool bad = bs[n + 1] != 0;
+    const int64_t lo = bad ? c * L / n : bounds[c];
+    const int64_t hi = bad ? (c + 1) * L / n : bounds[c + 1];
+    bs[c] = (int32_t)lo;
+    if (c == n - 1) bs[n] = (int32_t)hi;
+    for (int64_t t = lo; t < hi; ++t) tok_chunk[t] = (int32_t)c;
+}
+
+// sqrt(|C|) * mean of the keys of each variable-length chunk = sum / sqrt(|C|):
+// one warp per (b, g, chunk), lanes over 16-byte column slices.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+landmarks_varlen_kernel(const T *__restrict__ K, float *__restrict__ lm, int64_t total,
+                        Chunks ch, int64_t n) {
+    constexpr int VEC = Vec16<T>::N;
+    constexpr int LPR = D / VEC;                              // lanes per row slice
+    const int lane = threadIdx.x & 31;
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (w >= total) return;
+    const int64_t bg = w / n, i = w % n;
+    const int64_t first = chunk_first(ch, i);
+    const int len = chunk_len(ch, i);
+    const int rows_per_step = 32 / LPR;                       // rows a warp reads at once
+    const int col = (lane % LPR) * VEC, r0 = lane / LPR;
+    float acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    for (int r = r0; r < len; r += rows_per_step) {
+        if (first + r >= ch.L) break;
+        float f[VEC];
+        Vec16<T>::unpack(ld_stream16(K + (bg * ch.L + first + r) * D + col), f);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+    }
+    // fold the rows_per_step partial rows (lanes with equal column slices)
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (lane < LPR) {
+        const float f = len > 0 ? rsqrtf((float)len) : 0.f;
+        float *dst = lm + w * D + col;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) dst[e] = acc[e] * f;
+    }
+}
+
+cudaError_t launch_varlen_setup(const int32_t *bounds, int64_t n, int64_t L, int32_t *bs,
+                                int32_t *tok_chunk, unsigned *status, cudaStream_t st) {
+    varlen_check_kernel<<<1, 1024, 0, st>>>(bounds, n, L, bs, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    varlen_setup_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(bounds, n, L, bs, tok_chunk);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_landmarks_varlen(const void *K, bool bf16, float *lm, int B, int Hkv, int64_t L,
+                                    int d, const int32_t *bounds, int64_t n, cudaStream_t st) {
+    const int64_t total = (int64_t)B * Hkv * n;
+    if (total == 0) return cudaSuccess;
+    Chunks ch = {bounds, nullptr, L, 64};
+    const unsigned grid = (unsigned)((total + 7) / 8);
+    if (bf16) {
+        if (d == 128) landmarks_varlen_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)K, lm, total, ch, n);
+        else landmarks_varlen_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)K, lm, total, ch, n);
+    } else {
+        if (d == 128) landmarks_varlen_kernel<float, 128><<<grid, 256, 0, st>>>((const float *)K, lm, total, ch, n);
+        else landmarks_varlen_kernel<float, 64><<<grid, 256, 0, st>>>((const float *)K, lm, total, ch, n);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace hsa

@@ -34,8 +34,8 @@ constexpr int kSelTokPerWarp = kSelTokens / (kSelThreads / 32);
 template <typename T, typename TL, int D>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv, int64_t L,
-              int S, int topk, float scale, int R, int pool_mean, int32_t *__restrict__ idx_out,
-              float *__restrict__ w_out) {
+              int S, int64_t Nc, Chunks ch, int topk, float scale, int R, int pool_mean,
+              int32_t *__restrict__ idx_out, float *__restrict__ w_out) {
     extern __shared__ float4 smem4[];
     float *qbar = reinterpret_cast<float *>(smem4);                 // [64][D+4]
     float *lmt = qbar + kSelTokens * (D + 4);                        // [32][D+4]
@@ -46,7 +46,6 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
     const int tile = n_tiles - 1 - (int)blockIdx.x;                 // heavy tiles first
     const int g = blockIdx.y, b = blockIdx.z;
     const int G = H / Hkv;
-    const int64_t Nc = L / S;
     const int64_t t0 = (int64_t)tile * kSelTokens;                  // first selection row
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -96,7 +95,7 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
         }
     }
     const int64_t t_last = (t0 + kSelTokens - 1 < Lsel ? t0 + kSelTokens - 1 : Lsel - 1);
-    const int64_t nvis_max = t_last * R / S;
+    const int64_t nvis_max = chunk_of(ch, t_last * R);
 
     // scoring role: token tok_s, chunks sub + 4m of each tile
     const int tok_s = tid >> 2, sub = tid & 3;
@@ -161,7 +160,7 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
         for (int u = 0; u < kSelTokPerWarp; ++u) {
             const int tok = warp * kSelTokPerWarp + u;
             const int64_t t = t0 + tok;                              // selection row
-            const int64_t nvis = t < Lsel ? t * R / S : 0;
+            const int64_t nvis = t < Lsel ? chunk_of(ch, t * R) : 0;
             const int64_t i = c0 + lane;
             const uint64_t key = i < nvis ? make_key(sc[tok * 33 + lane], i) : 0ull;
             v[u] = merge_lists(v[u], merge_segments(sort_segments_desc(key, KP), KP), KP);
@@ -217,8 +216,8 @@ select_kernel(const T *__restrict__ Q, const TL *__restrict__ lm, int H, int Hkv
 
 template <typename T, typename TL, int D>
 static cudaError_t launch_select_t(const void *Q, const void *lm, int B, int H, int Hkv,
-                                   int64_t L, int S, int topk, float scale, int R, int pool_mean,
-                                   int32_t *idx, float *w, cudaStream_t st) {
+                                   int64_t L, int S, int64_t Nc, Chunks ch, int topk, float scale,
+                                   int R, int pool_mean, int32_t *idx, float *w, cudaStream_t st) {
     const size_t smem =
         sizeof(float) * ((kSelTokens + kSelChunks) * (D + 4) + kSelTokens * 33);
     auto kern = select_kernel<T, TL, D>;
@@ -227,28 +226,33 @@ static cudaError_t launch_select_t(const void *Q, const void *lm, int B, int H, 
     if (e != cudaSuccess) return e;
     const int64_t Lsel = (L + R - 1) / R;
     dim3 grid((unsigned)((Lsel + kSelTokens - 1) / kSelTokens), (unsigned)Hkv, (unsigned)B);
-    kern<<<grid, kSelThreads, smem, st>>>((const T *)Q, (const TL *)lm, H, Hkv, L, S, topk,
-                                          scale, R, pool_mean, idx, w);
+    kern<<<grid, kSelThreads, smem, st>>>((const T *)Q, (const TL *)lm, H, Hkv, L, S, Nc, ch,
+                                          topk, scale, R, pool_mean, idx, w);
     return cudaGetLastError();
 }
 
 template <typename T, typename TL>
 static cudaError_t launch_select_l(const void *Q, const void *lm, int B, int H, int Hkv,
-                                   int64_t L, int d, int S, int topk, float scale, int R,
-                                   int pool_mean, int32_t *idx, float *w, cudaStream_t st) {
-    return d == 128 ? launch_select_t<T, TL, 128>(Q, lm, B, H, Hkv, L, S, topk, scale, R, pool_mean, idx, w, st)
-                    : launch_select_t<T, TL, 64>(Q, lm, B, H, Hkv, L, S, topk, scale, R, pool_mean, idx, w, st);
+                                   int64_t L, int d, int S, int64_t Nc, Chunks ch, int topk,
+                                   float scale, int R, int pool_mean, int32_t *idx, float *w,
+                                   cudaStream_t st) {
+    return d == 128 ? launch_select_t<T, TL, 128>(Q, lm, B, H, Hkv, L, S, Nc, ch, topk, scale, R, pool_mean, idx, w, st)
+                    : launch_select_t<T, TL, 64>(Q, lm, B, H, Hkv, L, S, Nc, ch, topk, scale, R, pool_mean, idx, w, st);
 }
 
+// Nc: chunks with a landmark (L / S, or the number of variable-length chunks
+// given by bounds / tok_chunk, both null for chunks of S tokens).
 cudaError_t launch_select(const void *Q, bool q_bf16, const void *lm, bool lm_bf16, int B, int H,
-                          int Hkv, int64_t L, int d, int S, int topk, float scale, int R,
-                          int pool_mean, int32_t *idx, float *w, cudaStream_t st) {
+                          int Hkv, int64_t L, int d, int S, int64_t Nc, const int32_t *bounds,
+                          const int32_t *tok_chunk, int topk, float scale, int R, int pool_mean,
+                          int32_t *idx, float *w, cudaStream_t st) {
     using bf = __nv_bfloat16;
+    const Chunks ch = {bounds, tok_chunk, L, S};
     if (q_bf16)
-        return lm_bf16 ? launch_select_l<bf, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st)
-                       : launch_select_l<bf, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st);
-    return lm_bf16 ? launch_select_l<float, bf>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st)
-                   : launch_select_l<float, float>(Q, lm, B, H, Hkv, L, d, S, topk, scale, R, pool_mean, idx, w, st);
+        return lm_bf16 ? launch_select_l<bf, bf>(Q, lm, B, H, Hkv, L, d, S, Nc, ch, topk, scale, R, pool_mean, idx, w, st)
+                       : launch_select_l<bf, float>(Q, lm, B, H, Hkv, L, d, S, Nc, ch, topk, scale, R, pool_mean, idx, w, st);
+    return lm_bf16 ? launch_select_l<float, bf>(Q, lm, B, H, Hkv, L, d, S, Nc, ch, topk, scale, R, pool_mean, idx, w, st)
+                   : launch_select_l<float, float>(Q, lm, B, H, Hkv, L, d, S, Nc, ch, topk, scale, R, pool_mean, idx, w, st);
 }
 
 }  // namespace hsa

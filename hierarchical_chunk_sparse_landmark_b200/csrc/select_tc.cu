@@ -75,6 +75,7 @@ struct SelTcParams {
     // (pool_mean = 0) or the mean over the row's tokens (pool_mean = 1)
     int64_t Lsel;                   // selection rows, ceil(L / R)
     int R, pool_mean;
+    Chunks ch;                      // chunks of S tokens or variable-length ones (R = 1)
 };
 
 // Number of (token, head) query rows summed into the group query of
@@ -217,7 +218,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     const int R = p.R;
     const int64_t t0 = (int64_t)tb * C::M;                     // first selection row
     const int64_t t_last = t0 + C::M - 1 < Lsel ? t0 + C::M - 1 : Lsel - 1;
-    const int64_t nvis_max = t_last * R / p.S;                 // visible to the block's last row
+    const int64_t nvis_max = chunk_of(p.ch, t_last * R);       // visible to the block's last row
     const int ntiles = (int)((nvis_max + C::N - 1) / C::N);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -374,7 +375,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         float *stage = (float *)(smem + C::STAGE_OFF) + hg * (32 * 128);
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int64_t t = t0 + r;                              // selection row
-        const int64_t nvis = t < Lsel ? t * R / p.S : 0;
+        const int64_t nvis = t < Lsel ? chunk_of(p.ch, t * R) : 0;
         uint64_t v[KP];
 #pragma unroll
         for (int i = 0; i < KP; ++i) v[i] = 0ull;
@@ -486,7 +487,7 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
     const int R = p.R;
     const int64_t t0 = (int64_t)tb * C::M;                     // first selection row
     const int64_t t_last = t0 + C::M - 1 < Lsel ? t0 + C::M - 1 : Lsel - 1;
-    const int64_t nvis_max = t_last * R / p.S;                 // visible to the block's last row
+    const int64_t nvis_max = chunk_of(p.ch, t_last * R);       // visible to the block's last row
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 1) {
@@ -614,7 +615,7 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int64_t t = t0 + r;                              // selection row
-        const int64_t nvis = t < Lsel ? t * R / p.S : 0;
+        const int64_t nvis = t < Lsel ? chunk_of(p.ch, t * R) : 0;
         uint64_t v[KP];
 #pragma unroll
         for (int i = 0; i < KP; ++i) v[i] = 0ull;
@@ -767,13 +768,15 @@ cudaError_t launch_split_landmarks(const void *lm, void *split, int64_t n, cudaS
 // >= 1; G = H / Hkv a multiple of 8.  Up to 128 chunks the one-tile kernel
 // runs unless `force_multi_tile`; `*multi` tells which kernel was launched.
 cudaError_t launch_select_tc(const void *Q, const void *lm, bool lm_bf16, const void *split, int B,
-                             int H, int Hkv, int64_t L, int d, int S, int topk, float scale,
-                             int R, int pool_mean, int32_t *idx, unsigned *status,
+                             int H, int Hkv, int64_t L, int d, int S, int64_t Nc, int topk,
+                             float scale, int R, int pool_mean, const int32_t *bounds,
+                             const int32_t *tok_chunk, int32_t *idx, unsigned *status,
                              bool force_multi_tile, bool *multi, cudaStream_t st) {
     SelTcParams p;
     p.Q = Q; p.idx = idx; p.status = status;
-    p.L = L; p.Nc = L / S; p.H = H; p.Hkv = Hkv; p.S = S; p.topk = topk; p.scale = scale;
+    p.L = L; p.Nc = Nc; p.H = H; p.Hkv = Hkv; p.S = S; p.topk = topk; p.scale = scale;
     p.R = R; p.pool_mean = pool_mean; p.Lsel = (L + R - 1) / R;
+    p.ch.bounds = bounds; p.ch.tok_chunk = tok_chunk; p.ch.L = L; p.ch.S = S;
     const bool fm = force_multi_tile;
     if (lm_bf16) {
         return d == 128 ? launch_select_tc_k<128, false>(p, B, lm, nullptr, fm, multi, st)

@@ -29,6 +29,9 @@ Value recipes
   sequence, uniform in [0, Nc).  The landmark row l[b, g, i*] is replaced by
   8*sqrt(d) * qbar / |qbar|^2, qbar being the mean of the group's query heads,
   so that the needle's group score is 8 (before bf16 rounding of the row).
+* Variable-length chunks (``make_varlen_bounds``): chunk lengths drawn uniform
+  in [lo, hi] from a seeded CPU generator until they cover L tokens, the last
+  chunk cut to what is left; landmarks for them (when given) ~ 2 * N(0, 1).
 """
 from __future__ import annotations
 
@@ -44,6 +47,7 @@ __all__ = [
     "PRIMARY_WORKLOAD",
     "make_prefill_inputs",
     "make_decode_inputs",
+    "make_varlen_bounds",
     "storage_dtype",
 ]
 
@@ -215,3 +219,16 @@ def make_decode_inputs(wl: Workload, device="cpu") -> dict:
             out["lm"][b, :, int(depth[b]), :] = row[b].to(dt)
         out["needle_chunk"] = depth.tolist()
     return out
+
+
+def make_varlen_bounds(L: int, seed: int, lo: int = 1, hi: int = 64) -> list:
+    """Chunk boundaries 0 = b_0 < ... < b_n = L with lengths uniform in [lo, hi]
+    (the last one cut to the tokens left)."""
+    assert 1 <= lo <= hi
+    g = torch.Generator()
+    g.manual_seed(seed)
+    bounds = [0]
+    while bounds[-1] < L:
+        n = int(torch.randint(lo, hi + 1, (1,), generator=g))
+        bounds.append(min(L, bounds[-1] + n))
+    return bounds

@@ -173,6 +173,38 @@ hsa_status_t hsa_prefill_variant(const void *Q, const void *K, const void *V, hs
                                  void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Variable-length chunks (Dynamic Hierarchical Sparse Attention review, "What
+ * carries the argument": chunks of varying size, each represented by
+ * sqrt(|C|) times the mean of its keys, which keeps the landmark scores of
+ * chunks of different sizes comparable).  The chunks are given by their
+ * boundaries, shared by the batch:
+ *   bounds   [n_chunks + 1] int32, DEVICE, 0 = b_0 < b_1 < ... < b_n = L;
+ *            chunk c holds tokens b_c .. b_{c+1} - 1, at most 64 of them
+ * Everything else is hsa_prefill's method with chunk c in place of the
+ * fixed chunks: token t selects among the chunks before the chunk holding t,
+ * attends inside each selected chunk (all its keys) and, with own_chunk,
+ * causally over its own chunk from that chunk's first token.  With lm = NULL
+ * the landmarks are sqrt(|C|) * mean of each chunk's keys; an lm given is
+ * [B, Hkv, n_chunks, d].  union_softmax as in hsa_variant_t.  Every chunk has
+ * a landmark (the last one too, unlike the fixed-size form's partial tail).
+ * The boundaries are checked on the device: wrong ones make hsa_check return
+ * HSA_ERR_INVALID_ARG, and the call then computes as if the boundaries were
+ * the even split b_c = floor(c * L / n_chunks) (so no kernel reads or writes
+ * outside its buffers).  On the host: HSA_ERR_INVALID_ARG unless
+ * 1 <= n_chunks <= L <= 64 * n_chunks (L = 0 returns HSA_OK) and bounds is a
+ * 16-byte aligned device pointer.  Two more kernels than hsa_prefill (the
+ * check and the token-to-chunk table).
+ */
+size_t hsa_prefill_varlen_workspace_size(int B, int H, int Hkv, int64_t L, int d, int64_t n_chunks,
+                                         int topk);
+hsa_status_t hsa_prefill_varlen(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                                int64_t L, int d, const int32_t *bounds, int64_t n_chunks,
+                                int topk, int own_chunk, float scale, int union_softmax,
+                                void *O, int32_t *idx_out, float *w_out, void *workspace,
+                                size_t ws_bytes, void *stream);
+
+/*
  * hsa_decode_workspace_size -- bytes of device workspace hsa_decode needs
  * (0 on invalid arguments; the size depends on the current device's SM
  * count).  It holds a status word, per-(sequence, group) tickets and work
@@ -321,8 +353,10 @@ hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t 
 /*
  * hsa_check -- synchronises `stream`, then reads the status word at the head
  * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
- * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up (and clears
- * the word), HSA_ERR_CUDA if the stream reports an error, HSA_OK otherwise.
+ * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up,
+ * HSA_ERR_INVALID_ARG if hsa_prefill_varlen found its chunk boundaries wrong
+ * (either clears the word), HSA_ERR_CUDA if the stream reports an error,
+ * HSA_OK otherwise.
  * With workspace = NULL it reads the status word of hsa_decode_noalloc's
  * array on the stream's device (if this process has used that array there),
  * which collects the flags of every hsa_decode_noalloc call since the last

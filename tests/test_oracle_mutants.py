@@ -51,10 +51,10 @@ MUTANTS = {
     "variant_block_start_ignored": ("const int64_t t0 = (t / interval) * interval;",
                                     "const int64_t t0 = t;"),
     # retrieval variants: the union softmax leaves out the own chunk, or its last key
-    "variant_union_drops_own_chunk": ("if (own_chunk)\n                        for (int64_t jj = c * S; jj <= t; ++jj)",
-                                      "if (0)\n                        for (int64_t jj = c * S; jj <= t; ++jj)"),
-    "variant_union_own_excludes_self": ("for (int64_t jj = c * S; jj <= t; ++jj) keyrow[nk++] = jj;",
-                                        "for (int64_t jj = c * S; jj < t; ++jj) keyrow[nk++] = jj;"),
+    "variant_union_drops_own_chunk": ("if (own_chunk)\n                        for (int64_t jj = own_first; jj <= t; ++jj)",
+                                      "if (0)\n                        for (int64_t jj = own_first; jj <= t; ++jj)"),
+    "variant_union_own_excludes_self": ("for (int64_t jj = own_first; jj <= t; ++jj) keyrow[nk++] = jj;",
+                                        "for (int64_t jj = own_first; jj < t; ++jj) keyrow[nk++] = jj;"),
     # retrieval variants: mean pooling over the block's first token only
     "variant_mean_pool_first_only": ("const int64_t u1 = pool_mean ? t1 : t0 + 1;",
                                      "const int64_t u1 = t0 + 1;"),
