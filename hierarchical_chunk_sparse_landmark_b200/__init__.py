@@ -10,7 +10,8 @@ from ._binding import (HSAError, check, decode, decode_context_parallel, decode_
                        decode_cp_candidates, decode_cp_combine, decode_cp_merge, decode_noalloc,
                        decode_workspace_size,
                        landmarks, last_call_kernels, last_call_launches, lib, path_overrides,
-                       prefill, prefill_varlen, prefill_varlen_workspace_size,
+                       prefill, prefill_backward, prefill_backward_workspace_size,
+                       prefill_varlen, prefill_varlen_workspace_size,
                        prefill_workspace_size, selftest_wait_expiry, set_stage_events,
                        status_string, workspace)
 
@@ -18,5 +19,5 @@ __all__ = ["HSAError", "check", "decode", "decode_context_parallel", "decode_cp_
            "decode_cp_candidates", "decode_cp_combine", "decode_cp_merge", "decode_noalloc",
            "decode_workspace_size", "landmarks",
            "last_call_kernels", "last_call_launches", "lib", "path_overrides", "prefill",
-           "prefill_varlen", "prefill_varlen_workspace_size", "prefill_workspace_size", "selftest_wait_expiry", "set_stage_events", "status_string",
+           "prefill_backward", "prefill_backward_workspace_size", "prefill_varlen", "prefill_varlen_workspace_size", "prefill_workspace_size", "selftest_wait_expiry", "set_stage_events", "status_string",
            "workspace"]

@@ -24,6 +24,7 @@ HSA_F32, HSA_BF16 = 0, 1
 K_LANDMARKS, K_SPLIT_LANDMARKS, K_SELECT_TC_ONE_TILE, K_SELECT_TC_MULTI_TILE = 1, 2, 4, 8
 K_SELECT_SIMT, K_WORK_LISTS, K_ATTEND_TC, K_FUSE, K_ATTEND_SIMT = 16, 32, 64, 128, 256
 K_DECODE_SCAN, K_DECODE_ATTEND, K_DECODE_CP_MERGE, K_DECODE_CP_COMBINE = 512, 1024, 2048, 4096
+K_BACKWARD = 8192
 PATH_SIMT_PREFILL, PATH_SIMT_SELECT, PATH_MULTI_TILE_SELECT = 1, 2, 4
 
 EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
@@ -32,7 +33,8 @@ EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_decode_noalloc", "hsa_decode_noalloc_max_scratch", "hsa_selftest_wait_expiry",
             "hsa_last_call_kernels", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
             "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
-            "hsa_prefill_variant", "hsa_prefill_varlen_workspace_size", "hsa_prefill_varlen")
+            "hsa_prefill_variant", "hsa_prefill_varlen_workspace_size", "hsa_prefill_varlen",
+            "hsa_prefill_backward_workspace_size", "hsa_prefill_backward")
 
 
 class Variant(ctypes.Structure):
@@ -66,6 +68,10 @@ def _declare(lib):
     lib.hsa_prefill_varlen_workspace_size.restype = sz
     lib.hsa_prefill_varlen.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, vp,
                                        i64, i32, i32, f32, i32, vp, vp, vp, vp, sz, vp]
+    lib.hsa_prefill_backward_workspace_size.argtypes = [i32, i32, i32, i64, i32, i32, i32, i32]
+    lib.hsa_prefill_backward_workspace_size.restype = sz
+    lib.hsa_prefill_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, i32, i32, i32, i64,
+                                         i32, i32, i32, i32, f32, vp, vp, vp, vp, vp, sz, vp]
     lib.hsa_decode_workspace_size.argtypes = [i32, i32, i32, i64, i32, i32, i32]
     lib.hsa_decode_workspace_size.restype = sz
     lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
@@ -92,7 +98,7 @@ def _declare(lib):
               "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
               "hsa_selftest_wait_expiry", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
               "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
-              "hsa_prefill_variant", "hsa_prefill_varlen"):
+              "hsa_prefill_variant", "hsa_prefill_varlen", "hsa_prefill_backward"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -270,6 +276,49 @@ def prefill_varlen(Q, K, V, bounds, lm=None, *, topk: int = 8, own_chunk: int = 
                                   _stream(dev))
     _check(st, "hsa_prefill_varlen")
     return out, _opt(idx_out), _opt(w_out)
+
+
+def prefill_backward_workspace_size(B, H, Hkv, L, d, S, topk, dhsa: bool) -> int:
+    return int(lib().hsa_prefill_backward_workspace_size(B, H, Hkv, L, d, S, topk, int(dhsa)))
+
+
+def prefill_backward(Q, K, V, idx, dO, lm=None, *, S: int = 64, own_chunk: int = 1,
+                     scale: float = 0.0, dQ=None, dK=None, dV=None, dlm=None, ws=None):
+    """Gradients of sum(dO * O) for the prefill with the selection ``idx``
+    [B, L, Hkv, topk] (int32, the forward's) held fixed (hsa_prefill_backward).
+    Returns fp32 (dQ [B,L,H,d], dK, dV [B,Hkv,L,d], dlm [B,Hkv,L//S,d] or None
+    with DHSA landmarks, whose gradient is folded into dK)."""
+    for n, t in (("Q", Q), ("K", K), ("V", V), ("idx", idx), ("dO", dO)):
+        _dev(t, n)
+    B, L, H, d = Q.shape
+    Hkv = K.shape[1]
+    if K.shape != (B, Hkv, L, d) or V.shape != K.shape or dO.shape != Q.shape:
+        raise ValueError("K, V must be [B, Hkv, L, d] and dO like Q [B, L, H, d]")
+    if idx.dtype != torch.int32 or idx.dim() != 4 or idx.shape[:3] != (B, L, Hkv):
+        raise ValueError("idx must be int32 [B, L, Hkv, topk]")
+    topk = idx.shape[3]
+    dev = Q.device
+    if lm is not None:
+        _dev(lm, "lm")
+        if lm.shape != (B, Hkv, L // S, d):
+            raise ValueError(f"lm must be [B, Hkv, L//S, d] = {(B, Hkv, L // S, d)}")
+        if dlm is None:
+            dlm = torch.empty(B, Hkv, L // S, d, dtype=torch.float32, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dQ = torch.empty(B, L, H, d, **f32) if dQ is None else dQ
+    dK = torch.empty(B, Hkv, L, d, **f32) if dK is None else dK
+    dV = torch.empty(B, Hkv, L, d, **f32) if dV is None else dV
+    nbytes = prefill_backward_workspace_size(B, H, Hkv, L, d, S, topk, lm is None)
+    if ws is None:
+        ws = workspace(nbytes, dev, "backward")
+    st = lib().hsa_prefill_backward(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(lm),
+                                    _dtype_code(lm) if lm is not None else HSA_F32, _ptr(idx),
+                                    _ptr(dO), B, H, Hkv, L, d, S, topk, int(own_chunk),
+                                    float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                    _ptr(dlm if lm is not None else None), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(dev))
+    _check(st, "hsa_prefill_backward")
+    return dQ, dK, dV, (dlm if lm is not None else None)
 
 
 def decode_workspace_size(B, H, Hkv, Lc, d, S, topk) -> int:

@@ -655,6 +655,67 @@ hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t 
                                      (cudaStream_t)stream) == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
 }
 
+size_t hsa_prefill_backward_workspace_size(int B, int H, int Hkv, int64_t L, int d, int S,
+                                           int topk, int dhsa) {
+    if (check_shape(B, H, Hkv, L, d, S, topk) != HSA_OK) return 0;
+    if (L >= ((int64_t)1 << 26) || (int64_t)B * Hkv * L * topk >= (int64_t)INT32_MAX) return 0;
+    return bwd_layout(B, H, Hkv, L, d, S, topk, dhsa != 0).total;
+}
+
+hsa_status_t hsa_prefill_backward(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                  const void *lm, hsa_dtype_t lm_dt, const int32_t *idx,
+                                  const void *dO, int B, int H, int Hkv, int64_t L, int d, int S,
+                                  int topk, int own_chunk, float scale, float *dQ, float *dK,
+                                  float *dV, float *dlm, void *workspace, size_t ws_bytes,
+                                  void *stream) {
+    hsa_status_t s = check_shape(B, H, Hkv, L, d, S, topk);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
+    if (own_chunk != 0 && own_chunk != 1) return HSA_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || scale == INFINITY) return HSA_ERR_INVALID_ARG;
+    // entry codes t*32 + slot and entry offsets are 32-bit
+    if (L >= ((int64_t)1 << 26) || (int64_t)B * Hkv * L * topk >= (int64_t)INT32_MAX)
+        return HSA_ERR_UNSUPPORTED;
+    t_launches = 0;
+    t_kernels = 0;
+    if (L == 0) return HSA_OK;
+    const void *ptrs[] = {Q, K, V, dO, idx, dQ, dK, dV, workspace};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    const bool dhsa = lm == nullptr;
+    if (!dhsa && (!aligned16(lm) || !dlm || !aligned16(dlm))) return HSA_ERR_INVALID_ARG;
+    const BwdLayout lay = bwd_layout(B, H, Hkv, L, d, S, topk, dhsa);
+    if (ws_bytes < lay.total) return HSA_ERR_WORKSPACE;
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    cudaStream_t st = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    BwdArgs a;
+    a.Q = Q; a.K = K; a.V = V; a.dO = dO; a.lm = lm;
+    a.lm_bf16 = lm_dt == HSA_BF16; a.bf16 = dt == HSA_BF16; a.dhsa = dhsa;
+    a.idx = idx; a.B = B; a.H = H; a.Hkv = Hkv; a.d = d; a.S = S; a.topk = topk;
+    a.own_chunk = own_chunk; a.L = L; a.scale = scale;
+    a.dQ = dQ; a.dK = dK; a.dV = dV; a.dlm = dhsa ? nullptr : dlm; a.ws = workspace;
+    stage_mark(0, st);
+    if (dhsa) {   // the landmarks the forward used: sqrt(S) * mean of each chunk's keys
+        float *lm_ws = (float *)(ws + lay.lm_off);
+        if (lay.Nc > 0) {
+            if (launch_landmarks(K, a.bf16, lm_ws, B, Hkv, L, d, st) != cudaSuccess)
+                return HSA_ERR_CUDA;
+            t_launches += 1;
+            t_kernels |= HSA_K_LANDMARKS;
+        }
+        a.lm = lm_ws;
+        a.lm_bf16 = 0;
+    }
+    const cudaError_t e = launch_backward(a, lay, st);
+    if (e == cudaSuccess) {
+        t_launches += lay.Nc > 0 ? 6 : 4;     // row, [hist], scan, [scatter], key, reduce
+        t_kernels |= HSA_K_BACKWARD;
+    }
+    stage_mark(1, st);
+    return from_cuda(e);
+}
+
 hsa_status_t hsa_check(void *workspace, void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return HSA_ERR_CUDA;
@@ -668,7 +729,7 @@ hsa_status_t hsa_check(void *workspace, void *stream) {
     unsigned flags = 0;
     if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
         return HSA_ERR_CUDA;
-    if (flags & (kFlagTimeout | kFlagBadBounds)) {
+    if (flags & (kFlagTimeout | kFlagBadBounds | kFlagBadIdx)) {
         const unsigned zero = 0;
         cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice);
         return (flags & kFlagTimeout) ? HSA_ERR_TIMEOUT : HSA_ERR_INVALID_ARG;

@@ -252,6 +252,7 @@ __device__ __forceinline__ int64_t chunk_of(const Chunks &c, int64_t t) {
 constexpr size_t kStatusBytes = 256;
 constexpr unsigned kFlagTimeout = 1u;
 constexpr unsigned kFlagBadBounds = 2u;     // variable-length chunk boundaries invalid
+constexpr unsigned kFlagBadIdx = 4u;        // backward: a selection entry names no visible chunk
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -279,5 +280,24 @@ struct DecodeShard {
 __host__ __device__ constexpr size_t decode_zero_head(int64_t B, int64_t Hkv) {
     return align_up(kStatusBytes + 2 * sizeof(unsigned) * (size_t)(B * Hkv), 256);
 }
+
+// Prefill backward (backward.cu): workspace layout and arguments.
+struct BwdLayout {
+    int64_t BG, Nc, NcAll, TB, NTB, E, max_seg;
+    size_t lm_off, coef_off, cnt_off, cnt_bytes, entries_off, segs_off, nseg_off, cseg_off,
+        part_off, total;
+};
+BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, bool dhsa);
+struct BwdArgs {
+    const void *Q, *K, *V, *dO, *lm;
+    int lm_bf16, bf16, dhsa;
+    const int32_t *idx;
+    int B, H, Hkv, d, S, topk, own_chunk;
+    int64_t L;
+    float scale;
+    float *dQ, *dK, *dV, *dlm;
+    void *ws;
+};
+cudaError_t launch_backward(const BwdArgs &a, const BwdLayout &p, cudaStream_t st);
 
 }  // namespace hsa

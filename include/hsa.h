@@ -74,7 +74,8 @@ enum {
     HSA_K_DECODE_SCAN = 1u << 9,          /* decode landmark scan + top-K */
     HSA_K_DECODE_ATTEND = 1u << 10,       /* decode attend + fusion (or a shard's fusion state) */
     HSA_K_DECODE_CP_MERGE = 1u << 11,     /* global top-K over the shards' candidates */
-    HSA_K_DECODE_CP_COMBINE = 1u << 12    /* O from the shards' fusion states */
+    HSA_K_DECODE_CP_COMBINE = 1u << 12,   /* O from the shards' fusion states */
+    HSA_K_BACKWARD = 1u << 13             /* prefill gradients (hsa_prefill_backward) */
 };
 
 /* Path overrides (hsa_set_path_overrides). */
@@ -203,6 +204,51 @@ hsa_status_t hsa_prefill_varlen(const void *Q, const void *K, const void *V, hsa
                                 int topk, int own_chunk, float scale, int union_softmax,
                                 void *O, int32_t *idx_out, float *w_out, void *workspace,
                                 size_t ws_bytes, void *stream);
+
+/*
+ * Prefill backward (HiLS Attention abstract: the retrieval scores are trained
+ * end to end by the language-model loss; HSA "Methodology in Plain English"
+ * for the forward it differentiates).  Gradients of sum(dO * O) for the
+ * hsa_prefill forward, with the selection held fixed (a hard top-K has no
+ * gradient): `idx` is the forward's selection.  Per query row (t, h) of group
+ * g with selected chunks i_1 .. i_K, w = softmax_k(scale q.l_{i_k}) and
+ * p_k = softmax_j(scale q.k_j) over chunk i_k (own chunk: weight 1, keys
+ * c_t*S .. t):
+ *   u_kj = dO.v_j, dw_k = p_k.u_k, dz_k = w_k (dw_k - sum_k' w_k' dw_k'),
+ *   da_kj = w_k p_kj (u_kj - dw_k);
+ *   dQ[t,h]   = scale (sum_kj da_kj k_j + sum_k dz_k l_{i_k})
+ *   dK[j]    += scale da_kj q,  dV[j] += w_k p_kj dO,  dlm[i_k] += scale dz_k q
+ * and with DHSA landmarks (lm = NULL, l = sqrt(S) * mean of the chunk's keys,
+ * as hsa_prefill computes them) dlm / sqrt(S) is added to every key of the
+ * chunk instead of being returned.
+ *   Q, dO    [B, L, H, d]       dt (bf16 or fp32)
+ *   K, V     [B, Hkv, L, d]     dt
+ *   lm       [B, Hkv, L/S, d]   lm_dt, or NULL (DHSA)
+ *   idx      [B, L, Hkv, topk]  int32, the forward's selection (-1: empty
+ *                               slot; an entry naming a chunk that is not
+ *                               before the token's own chunk is skipped and
+ *                               reported by hsa_check as HSA_ERR_INVALID_ARG)
+ *   dQ       [B, L, H, d]       fp32, written
+ *   dK, dV   [B, Hkv, L, d]     fp32, written (every row)
+ *   dlm      [B, Hkv, L/S, d]   fp32, written; required when lm is given,
+ *                               ignored (may be NULL) in DHSA mode
+ * Gradients accumulate in fp32 in a fixed order: the results are
+ * bit-reproducible run to run.  CUDA cores throughout: a row pass (dQ and the
+ * fusion coefficients), a stable sort of the selection by chunk, a per-chunk
+ * key pass (dK, dV, dlm partials over segments of at most 1024 query rows)
+ * and an ordered reduction.  Supports L < 2^26 and B*Hkv*L*topk < 2^31
+ * (else HSA_ERR_UNSUPPORTED); workspace from
+ * hsa_prefill_backward_workspace_size (dhsa = 1 when lm will be NULL), no
+ * zero-fill needed.  All buffers 16-byte aligned.
+ */
+size_t hsa_prefill_backward_workspace_size(int B, int H, int Hkv, int64_t L, int d, int S,
+                                           int topk, int dhsa);
+hsa_status_t hsa_prefill_backward(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
+                                  const void *lm, hsa_dtype_t lm_dt, const int32_t *idx,
+                                  const void *dO, int B, int H, int Hkv, int64_t L, int d, int S,
+                                  int topk, int own_chunk, float scale, float *dQ, float *dK,
+                                  float *dV, float *dlm, void *workspace, size_t ws_bytes,
+                                  void *stream);
 
 /*
  * hsa_decode_workspace_size -- bytes of device workspace hsa_decode needs
@@ -355,6 +401,7 @@ hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t 
  * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
  * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up,
  * HSA_ERR_INVALID_ARG if hsa_prefill_varlen found its chunk boundaries wrong
+ * or hsa_prefill_backward a selection entry that names no visible chunk
  * (either clears the word), HSA_ERR_CUDA if the stream reports an error,
  * HSA_OK otherwise.
  * With workspace = NULL it reads the status word of hsa_decode_noalloc's
@@ -373,7 +420,7 @@ hsa_status_t hsa_check(void *workspace, void *stream);
  *                selection, 3 after the work-list build, 4 after the
  *                attention kernel, 5 after the fusion kernel (end of the
  *                call; 4 and 5 coincide on the path that fuses in place);
- *   hsa_decode:  0 start, 1 end.
+ *   hsa_decode, hsa_prefill_backward:  0 start, 1 end.
  * Boundaries a call does not reach are not recorded.  n must be 0..8.  The
  * events belong to the caller.  No effect on results.
  */
@@ -381,14 +428,16 @@ hsa_status_t hsa_set_stage_events(void *const *events, int n);
 
 /*
  * hsa_last_call_launches -- number of kernels the calling thread's most
- * recent hsa_prefill / hsa_decode / hsa_landmarks call launched.
+ * recent hsa_prefill* / hsa_decode* / hsa_landmarks / hsa_prefill_backward
+ * call launched.
  */
 int hsa_last_call_launches(void);
 
 /*
  * hsa_last_call_kernels -- the kernel families (HSA_K_* bits) that the calling
- * thread's most recent hsa_prefill / hsa_decode / hsa_landmarks call launched:
- * which path the dispatch took for those sizes and dtypes.
+ * thread's most recent hsa_prefill* / hsa_decode* / hsa_landmarks /
+ * hsa_prefill_backward call launched: which path the dispatch took for those
+ * sizes and dtypes.
  */
 unsigned hsa_last_call_kernels(void);
 
