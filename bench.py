@@ -76,6 +76,20 @@ def prefill_flops(wl) -> dict:
             "attention_kernel": chunk + ownf + fuse}
 
 
+def backward_flops(wl) -> float:
+    """Algorithmic FLOPs of one prefill backward (selection held fixed): per
+    (token, head, selected chunk) the five 64 x d products of attention's
+    backward -- scores recomputed, dO.V^T, dV, dQ, dK (2.5x the forward's two)
+    -- plus the fusion logit, its dq and dl terms (3 x 2d); the own chunk the
+    same five products over its causal keys."""
+    _, keff, own = prefill_token_counts(wl)
+    d, H, S, B = wl.d, wl.H, wl.S, wl.B
+    chunk = B * float((H * 10 * d * S * keff).sum())
+    fuse = B * float((H * 6 * d * keff).sum())
+    ownf = B * float((H * 10 * d * own).sum())
+    return chunk + fuse + ownf
+
+
 def chunk_output_bytes(wl) -> float:
     """Bytes of fp16 chunk outputs the tensor-core attention writes (and the
     fusion reads back): one G*d block per selected (token, group, chunk) and
@@ -369,6 +383,79 @@ def bench_prefill(args, name, dev, peaks, rank, dist, steps, warmup, keep_inputs
     return res, extra
 
 
+def bench_backward(args, name, dev, peaks, rank, dist, steps, warmup):
+    """Time hsa_prefill_backward on one workload (the forward's selection held
+    fixed, computed once outside the timed region; L2 flushed between calls).
+    CUDA cores end to end, so the roofline is the FP32 CUDA-core peak."""
+    import torch
+
+    import hierarchical_chunk_sparse_landmark_b200 as hsa
+    from hierarchical_chunk_sparse_landmark_b200.workloads import WORKLOADS, make_prefill_inputs
+    wl = WORKLOADS[name].with_(seed=WORKLOADS[name].seed + rank)
+    x = make_prefill_inputs(wl, dev)
+    _, idx, _ = hsa.prefill(x["Q"], x["K"], x["V"], x["lm"], S=wl.S, topk=wl.topk,
+                            own_chunk=wl.own_chunk, idx_out=True)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed + 11)
+    dO = torch.randn(x["Q"].shape, generator=g, device=dev).to(x["Q"].dtype)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dQ = torch.empty(x["Q"].shape, **f32)
+    dK = torch.empty(x["K"].shape, **f32)
+    dV = torch.empty(x["V"].shape, **f32)
+    dlm = None if x["lm"] is None else torch.empty(x["lm"].shape, **f32)
+    ws = hsa.workspace(hsa.prefill_backward_workspace_size(wl.B, wl.H, wl.Hkv, wl.L, wl.d, wl.S,
+                                                           wl.topk, x["lm"] is None), dev,
+                       "backward")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [make_events(2) for _ in range(steps)]
+
+    def step():
+        hsa.prefill_backward(x["Q"], x["K"], x["V"], idx, dO, x["lm"], S=wl.S,
+                             own_chunk=wl.own_chunk, dQ=dQ, dK=dK, dV=dV, dlm=dlm, ws=ws)
+
+    for _ in range(warmup):
+        step()
+        flush.fill_(1)
+    hsa.check(ws)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    launches = 0
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as clk:
+        for i in range(steps):
+            hsa.set_stage_events(ev[i])
+            step()
+            launches += hsa.last_call_launches()
+            hsa.set_stage_events([])
+            flush.fill_(1)
+        torch.cuda.synchronize()
+    hsa.check(ws)
+    ms = [e[0].elapsed_time(e[1]) for e in ev]
+    flops = backward_flops(wl)
+    units, tmax = aggregate(dist, flops * steps / 1e12, sum(ms) / 1e3, dev)
+    peak = fp32_simt_peak_tflops(peaks)
+    ach = flops / (statistics.mean(ms) / 1e3) / 1e12
+    res = {"workload": wl.name, "value": round(units / tmax, 4), "unit": "TFLOP/s",
+           "ms_per_step": round(tmax * 1e3 / steps, 4), "steps": steps,
+           "config": {"workload": wl.name, "pass": "backward (dQ, dK, dV, dlm)", "B": wl.B,
+                      "L": wl.L, "H": wl.H, "Hkv": wl.Hkv, "d": wl.d, "S": wl.S,
+                      "topk": wl.topk, "own_chunk": wl.own_chunk, "landmarks": wl.landmarks,
+                      "dtype": wl.dtype},
+           "roofline": {"kernel": "bwd_row + bwd_key + sort + reduce (whole call)",
+                        "bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 1),
+                        "unit": "TFLOP/s", "frac": round(ach / peak, 5), "traffic": None,
+                        "algorithmic_flops_per_launch": flops,
+                        "peak_source": "FP32 CUDA-core peak: 148 SMs x 128 lanes x 2 flop x "
+                                       "%.0f MHz" % peaks.get("sm_max_mhz", 1965.0)},
+           "clocks": clk.summary(), "gpu_launches": launches}
+    del x, dO, dQ, dK, dV, dlm, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, dist, rank, world):
     import torch
 
@@ -407,6 +494,9 @@ def run_ours(args, dist, rank, world):
                 r, _ = bench_prefill(args, name, dev, peaks, rank, dist, max(5, args.steps // 2), 3)
                 r.pop("flops_per_step", None)
                 res[key] = r
+    if args.extra:
+        res["backward_train"] = bench_backward(args, "train_prefill_bf16", dev, peaks, rank, dist,
+                                               max(3, args.steps // 4), 3)
     if args.decode:
         names = [args.decode_workload]
         if args.extra and "batched_decode_bf16" not in names:

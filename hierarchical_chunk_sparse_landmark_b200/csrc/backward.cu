@@ -33,7 +33,8 @@
 namespace hsa {
 
 constexpr int kSegRows = 1024;          // query rows (entry x head) per key segment
-constexpr int kKeyThreads = 256;        // 64 keys x 4 quarters of d
+constexpr int kKeyThreads = 512;        // 64 keys x 8 lanes over d
+constexpr int kKeyLanes = kKeyThreads / 64;
 constexpr int kScanThreads2 = 1024;
 
 // A selection entry counts when it names a chunk before the token's own chunk
@@ -59,6 +60,9 @@ __device__ __forceinline__ float lm_at(const void *lm, int lm_bf16, int64_t i) {
 }
 
 // ---------------------------------------------------------------- row-centric
+// One pass over the selected chunks: the fusion weights depend only on q and
+// the landmarks, so they come first; then every chunk is staged once and its
+// dw_k and da_k (hence its dq terms) follow from its own softmax.
 template <typename T, int D>
 __global__ void __launch_bounds__(512)
 bwd_row_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
@@ -85,6 +89,7 @@ bwd_row_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
         qs[e] = to_f32(Q[(row * H + (int64_t)g * G) * D + e]);
         dos[e] = to_f32(dO[(row * H + (int64_t)g * G) * D + e]);
     }
+    __syncthreads();
     const int64_t bg = (int64_t)b * Hkv + g;
     const T *Kbg = K + bg * L * D;
     const T *Vbg = V + bg * L * D;
@@ -92,21 +97,43 @@ bwd_row_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
     const int h = g * G + warp;
     const float *qh = qs + warp * D, *doh = dos + warp * D;
     const int64_t c_t = t / S;
-    const int n_items = topk + (own_chunk ? 1 : 0);
 
-    // Chunk `it` staged in shared memory; returns its key count (0: skip).
-    auto stage = [&](int it, int64_t &first, int32_t &ci) -> int {
+    // fusion logits z_k = scale q.l_{i_k} and weights w = softmax over the
+    // valid slots (lane k keeps slot k)
+    float zk = -INFINITY;
+    bool vk = false;
+    for (int it = 0; it < topk; ++it) {
+        const int32_t ci = ip[it];
+        if (!sel_ok(ci, t, S, Nc)) {
+            if (ci >= 0 && threadIdx.x == 0) atomicOr(status, kFlagBadIdx);
+            continue;
+        }
+        float a = 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            a = fmaf(qh[lane + 32 * r], lm_at(lm, lm_bf16, (bg * Nc + ci) * D + lane + 32 * r), a);
+        const float z = scale * warp_sum(a);
+        if (lane == it) { zk = z; vk = true; }
+    }
+    const float m = warp_max(vk ? zk : -INFINITY);
+    const float ew = vk ? expf(zk - m) : 0.f;
+    const float sw = warp_sum(ew);
+    const float wk = vk ? ew / sw : 0.f;
+
+    float dq[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) dq[r] = 0.f;
+    float dwk = 0.f;
+    const int n_items = topk + (own_chunk ? 1 : 0);
+    for (int it = 0; it < n_items; ++it) {
+        int64_t first;
         int nk;
         if (it < topk) {
-            ci = ip[it];
-            if (!sel_ok(ci, t, S, Nc)) {
-                if (ci >= 0 && threadIdx.x == 0) atomicOr(status, kFlagBadIdx);
-                return 0;
-            }
+            const int32_t ci = ip[it];
+            if (!sel_ok(ci, t, S, Nc)) continue;   // uniform across the block
             first = (int64_t)ci * S;
             nk = S;
         } else {
-            ci = -1;
             first = c_t * S;
             nk = (int)(t - first + 1);
         }
@@ -120,17 +147,13 @@ bwd_row_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
                 *reinterpret_cast<const uint4 *>(Vbg + (first + r) * D + c);
         }
         __syncthreads();
-        return nk;
-    };
-    // this lane's keys j = lane, lane + 32: logits scale q.k_j, u_j = dO.v_j, the
-    // normalised p_j and dw = p.u
-    auto chunk_softmax = [&](int nk, float (&p)[2], float (&u)[2]) -> float {
-        float s[2];
+        // keys j = lane, lane + 32: s_j = scale q.k_j, u_j = dO.v_j
+        float sj[2], uj[2];
 #pragma unroll
         for (int w2 = 0; w2 < 2; ++w2) {
             const int j = lane + 32 * w2;
-            s[w2] = -INFINITY;
-            u[w2] = 0.f;
+            sj[w2] = -INFINITY;
+            uj[w2] = 0.f;
             if (j < nk) {
                 float a = 0.f, c = 0.f;
 #pragma unroll 4
@@ -144,76 +167,40 @@ bwd_row_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
                         c = fmaf(doh[x + e], fv[e], c);
                     }
                 }
-                s[w2] = scale * a;
-                u[w2] = c;
+                sj[w2] = scale * a;
+                uj[w2] = c;
             }
         }
-        const float mx = warp_max(fmaxf(s[0], s[1]));
+        const float mx = warp_max(fmaxf(sj[0], sj[1]));
+        float p[2];
 #pragma unroll
-        for (int w2 = 0; w2 < 2; ++w2) p[w2] = lane + 32 * w2 < nk ? expf(s[w2] - mx) : 0.f;
-        const float den = warp_sum(p[0] + p[1]);
-        const float inv = 1.f / den;
+        for (int w2 = 0; w2 < 2; ++w2) p[w2] = lane + 32 * w2 < nk ? expf(sj[w2] - mx) : 0.f;
+        const float inv = 1.f / warp_sum(p[0] + p[1]);
         p[0] *= inv;
         p[1] *= inv;
-        return warp_sum(p[0] * u[0] + p[1] * u[1]);
-    };
-
-    // pass 1: dw_k and the fusion logits z_k (lane k keeps slot k's values)
-    float zk = -INFINITY, dwk = 0.f, dw_own = 0.f;
-    bool vk = false;
-    for (int it = 0; it < n_items; ++it) {
-        int64_t first;
-        int32_t ci;
-        const int nk = stage(it, first, ci);
-        if (nk == 0) continue;                                     // uniform across the block
-        float p[2], u[2];
-        const float dw = chunk_softmax(nk, p, u);
-        if (it < topk) {
-            float a = 0.f;
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-                a = fmaf(qh[lane + 32 * r], lm_at(lm, lm_bf16, (bg * Nc + ci) * D + lane + 32 * r), a);
-            const float z = scale * warp_sum(a);
-            if (lane == it) { zk = z; dwk = dw; vk = true; }
-        } else {
-            dw_own = dw;
-        }
-    }
-    // fusion weights over the valid slots and dz = w (dw - sum w dw)
-    const float m = warp_max(vk ? zk : -INFINITY);
-    const float ew = vk ? expf(zk - m) : 0.f;
-    const float sw = warp_sum(ew);
-    const float wk = vk ? ew / sw : 0.f;
-    const float dsum = warp_sum(wk * dwk);
-    const float dzk = wk * (dwk - dsum);
-    if (lane < topk) coef[(row * H + h) * topk + lane] = make_float2(wk, dzk);
-
-    // pass 2: dq = scale (sum_kj da_kj k_j + sum_k dz_k l_k)
-    float dq[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) dq[r] = 0.f;
-    for (int it = 0; it < n_items; ++it) {
-        int64_t first;
-        int32_t ci;
-        const int nk = stage(it, first, ci);
-        if (nk == 0) continue;
-        float p[2], u[2];
-        const float dw = chunk_softmax(nk, p, u);
+        const float dw = warp_sum(p[0] * uj[0] + p[1] * uj[1]);
         const float a = it < topk ? __shfl_sync(0xffffffffu, wk, it) : 1.f;
+        if (it < topk && lane == it) dwk = dw;
         float da[2];
 #pragma unroll
-        for (int w2 = 0; w2 < 2; ++w2) da[w2] = scale * a * p[w2] * (u[w2] - dw);
+        for (int w2 = 0; w2 < 2; ++w2) da[w2] = scale * a * p[w2] * (uj[w2] - dw);
         for (int j = 0; j < nk; ++j) {
             const float dj = __shfl_sync(0xffffffffu, da[j >> 5], j & 31);
 #pragma unroll
             for (int r = 0; r < R; ++r) dq[r] = fmaf(dj, to_f32(ks[j * RS + lane + 32 * r]), dq[r]);
         }
-        if (it < topk) {
-            const float dz = scale * __shfl_sync(0xffffffffu, dzk, it);
+    }
+    // dz = w (dw - sum w dw); dq += scale sum_k dz_k l_k
+    const float dsum = warp_sum(wk * dwk);
+    const float dzk = wk * (dwk - dsum);
+    if (lane < topk) coef[(row * H + h) * topk + lane] = make_float2(wk, dzk);
+    for (int it = 0; it < topk; ++it) {
+        const int32_t ci = ip[it];
+        if (!sel_ok(ci, t, S, Nc)) continue;
+        const float dz = scale * __shfl_sync(0xffffffffu, dzk, it);
 #pragma unroll
-            for (int r = 0; r < R; ++r)
-                dq[r] = fmaf(dz, lm_at(lm, lm_bf16, (bg * Nc + ci) * D + lane + 32 * r), dq[r]);
-        }
+        for (int r = 0; r < R; ++r)
+            dq[r] = fmaf(dz, lm_at(lm, lm_bf16, (bg * Nc + ci) * D + lane + 32 * r), dq[r]);
     }
     float *dqh = dQ + (row * H + h) * (int64_t)D;
 #pragma unroll
@@ -376,28 +363,33 @@ bwd_scatter_kernel(const int32_t *__restrict__ idx, int Hkv, int64_t L, int S, i
 }
 
 // ---------------------------------------------------------------- key-centric
-// One block per segment; thread (key j = tid / 4, quarter qd = tid % 4) owns
-// d elements qd*D/4 .. of key j's dK and dV.  Rows (entry, head) go 8 at a
-// time: scores and u over the thread's quarter, reduced across the quarter,
-// then the chunk softmax of each row across the block.
+// One block per segment; thread (key j = tid / 8, lane part qd = tid % 8) owns
+// the d elements qd, qd + 8, qd + 16, ... of key j's dK and dV.  Key rows are
+// staged with a stride of D + 8 floats, so the 32 lanes of a warp (4 keys x 8
+// parts) read 32 different banks; a row element is read by the 4 lanes of one
+// part at once (a broadcast).  Rows (entry, head) go 8 at a time: scores and
+// u over the thread's part, summed across the 8 parts, then the chunk softmax
+// of each row across the block.
 template <typename T, int D>
-__global__ void __launch_bounds__(kKeyThreads)
+__global__ void __launch_bounds__(kKeyThreads, 1)
 bwd_key_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
                const T *__restrict__ dO, const float2 *__restrict__ coef,
                const int32_t *__restrict__ entries, const int4 *__restrict__ segs,
                const int32_t *__restrict__ nseg_p, int H, int Hkv, int64_t L, int S,
                int64_t NcAll, int topk, float scale, float *__restrict__ part) {
-    constexpr int X = D / 4;
+    constexpr int X = D / kKeyLanes;
+    constexpr int KS = D + kKeyLanes;              // staged key row stride (floats)
+    constexpr int NW = kKeyThreads / 32;
     constexpr int NR = 8;                          // rows per batch
     constexpr int VEC = Vec16<T>::N;
     const int64_t sidx = blockIdx.x;
     if (sidx >= *nseg_p) return;
     extern __shared__ float4 smem4[];
-    float *Ks = reinterpret_cast<float *>(smem4);  // [64][D]
-    float *Vs = Ks + 64 * D;                       // [64][D]
-    float *qr = Vs + 64 * D;                       // [NR][D]
+    float *Ks = reinterpret_cast<float *>(smem4);  // [64][KS]
+    float *Vs = Ks + 64 * KS;                      // [64][KS]
+    float *qr = Vs + 64 * KS;                      // [NR][D]
     float *dor = qr + NR * D;                      // [NR][D]
-    float *red = dor + NR * D;                     // [3][8 warps][NR]
+    float *red = dor + NR * D;                     // [3][NW][NR]
     __shared__ int64_t rt[NR];
     __shared__ int rh[NR], rnk[NR];
     __shared__ float rw[NR], rdz[NR];
@@ -423,11 +415,12 @@ bwd_key_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
         }
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            Ks[j * D + x + e] = fk[e];
-            Vs[j * D + x + e] = fv[e];
+            Ks[j * KS + x + e] = fk[e];
+            Vs[j * KS + x + e] = fv[e];
         }
     }
-    const int j = tid >> 2, x0 = (tid & 3) * X;
+    const int j = tid / kKeyLanes, qd = tid % kKeyLanes;
+    const float *kj = Ks + j * KS + qd, *vj = Vs + j * KS + qd;
     float dk[X], dv[X], dl = 0.f;
 #pragma unroll
     for (int x = 0; x < X; ++x) dk[x] = dv[x] = 0.f;
@@ -478,74 +471,82 @@ bwd_key_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
         __syncthreads();
         float s[NR], u[NR];
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            float a = 0.f, cc = 0.f;
+        for (int r = 0; r < NR; ++r) s[r] = u[r] = 0.f;
+        // d outer, rows inner: the 2 x NR partial sums and one key / value
+        // element are all that is live
 #pragma unroll
-            for (int x = 0; x < X; ++x) {
-                a = fmaf(qr[r * D + x0 + x], Ks[j * D + x0 + x], a);
-                cc = fmaf(dor[r * D + x0 + x], Vs[j * D + x0 + x], cc);
+        for (int x = 0; x < X; ++x) {
+            const float kx = kj[kKeyLanes * x], vx = vj[kKeyLanes * x];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                s[r] = fmaf(qr[r * D + qd + kKeyLanes * x], kx, s[r]);
+                u[r] = fmaf(dor[r * D + qd + kKeyLanes * x], vx, u[r]);
             }
-            a += __shfl_xor_sync(0xffffffffu, a, 1);
-            a += __shfl_xor_sync(0xffffffffu, a, 2);
-            cc += __shfl_xor_sync(0xffffffffu, cc, 1);
-            cc += __shfl_xor_sync(0xffffffffu, cc, 2);
-            s[r] = j < rnk[r] ? scale * a : -INFINITY;
-            u[r] = cc;
+            asm volatile("" ::: "memory");   // keep each step's loads in its step (registers)
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+#pragma unroll
+            for (int o = 1; o < kKeyLanes; o <<= 1) {
+                s[r] += __shfl_xor_sync(0xffffffffu, s[r], o);
+                u[r] += __shfl_xor_sync(0xffffffffu, u[r], o);
+            }
+            s[r] = j < rnk[r] ? scale * s[r] : -INFINITY;
         }
         // block-wide softmax of each row over the 64 keys
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
             float m = s[r];
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+#pragma unroll
+            for (int o = kKeyLanes; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (lane == 0) red[warp * NR + r] = m;
         }
         __syncthreads();
-        float e_[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
             float m = red[r];
 #pragma unroll
-            for (int w2 = 1; w2 < kKeyThreads / 32; ++w2) m = fmaxf(m, red[w2 * NR + r]);
-            e_[r] = j < rnk[r] ? expf(s[r] - m) : 0.f;
-            float z = e_[r], zu = e_[r] * u[r];
+            for (int w2 = 1; w2 < NW; ++w2) m = fmaxf(m, red[w2 * NR + r]);
+            asm volatile("" ::: "memory");   // one row's loads at a time (registers)
+            s[r] = j < rnk[r] ? expf(s[r] - m) : 0.f;       // s now holds e = exp(s - max)
+            float z = s[r], zu = s[r] * u[r];
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) {
+            for (int o = kKeyLanes; o < 32; o <<= 1) {
                 z += __shfl_xor_sync(0xffffffffu, z, o);
                 zu += __shfl_xor_sync(0xffffffffu, zu, o);
             }
-            // lanes 4 apart hold the warp's 8 keys of one quarter: lane 0 has
-            // the warp's sums, one term per key
+            // lanes kKeyLanes apart hold the warp's keys of one part: lane 0
+            // has the warp's sums, one term per key
             if (lane == 0) {
-                red[(8 + warp) * NR + r] = z;
-                red[(16 + warp) * NR + r] = zu;
+                red[(NW + warp) * NR + r] = z;
+                red[(2 * NW + warp) * NR + r] = zu;
             }
         }
         __syncthreads();
-        float da[NR], wp[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
             float z = 0.f, zu = 0.f;
 #pragma unroll
-            for (int w2 = 0; w2 < kKeyThreads / 32; ++w2) {
-                z += red[(8 + w2) * NR + r];
-                zu += red[(16 + w2) * NR + r];
+            for (int w2 = 0; w2 < NW; ++w2) {
+                z += red[(NW + w2) * NR + r];
+                zu += red[(2 * NW + w2) * NR + r];
             }
-            const float p = e_[r] / z, dw = zu / z;
-            da[r] = scale * rw[r] * p * (u[r] - dw);
-            wp[r] = rw[r] * p;
+            asm volatile("" ::: "memory");
+            const float p = s[r] / z, dw = zu / z;
+            s[r] = scale * rw[r] * p * (u[r] - dw);          // da
+            u[r] = rw[r] * p;                                // w p
         }
 #pragma unroll
         for (int x = 0; x < X; ++x) {
             float a = dk[x], v = dv[x];
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
-                a = fmaf(da[r], qr[r * D + x0 + x], a);
-                v = fmaf(wp[r], dor[r * D + x0 + x], v);
+                a = fmaf(s[r], qr[r * D + qd + kKeyLanes * x], a);
+                v = fmaf(u[r], dor[r * D + qd + kKeyLanes * x], v);
             }
             dk[x] = a;
             dv[x] = v;
+            asm volatile("" ::: "memory");
         }
         if (!own && tid < D) {
 #pragma unroll
@@ -555,8 +556,8 @@ bwd_key_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
     float *pk = part + sidx * (int64_t)(129 * D);
 #pragma unroll
     for (int x = 0; x < X; ++x) {
-        pk[j * D + x0 + x] = dk[x];
-        pk[64 * D + j * D + x0 + x] = dv[x];
+        pk[j * D + qd + kKeyLanes * x] = dk[x];
+        pk[64 * D + j * D + qd + kKeyLanes * x] = dv[x];
     }
     if (tid < D) pk[128 * D + tid] = dl;
 }
@@ -690,7 +691,8 @@ static cudaError_t launch_backward_t(const BwdArgs &a, const BwdLayout &p, cudaS
     }
     // 3. per-segment dK / dV / dl partials
     {
-        const size_t smem = sizeof(float) * (2 * 64 * D + 2 * 8 * D + 3 * 8 * 8);
+        const size_t smem =
+            sizeof(float) * (2 * 64 * (D + kKeyLanes) + 2 * 8 * D + 3 * (kKeyThreads / 32) * 8);
         auto kern = bwd_key_kernel<T, D>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
