@@ -8,7 +8,7 @@ workloads used by the tests and the benchmark.
 """
 from ._binding import (HSAError, check, decode, decode_context_parallel, decode_cp_attend,
                        decode_cp_candidates, decode_cp_combine, decode_cp_merge, decode_noalloc,
-                       decode_workspace_size,
+                       decode_ragged, decode_workspace_size, landmarks_append,
                        landmarks, last_call_kernels, last_call_launches, lib, path_overrides,
                        prefill, prefill_backward, prefill_backward_workspace_size,
                        prefill_varlen, prefill_varlen_workspace_size,
@@ -17,7 +17,7 @@ from ._binding import (HSAError, check, decode, decode_context_parallel, decode_
 
 __all__ = ["HSAError", "check", "decode", "decode_context_parallel", "decode_cp_attend",
            "decode_cp_candidates", "decode_cp_combine", "decode_cp_merge", "decode_noalloc",
-           "decode_workspace_size", "landmarks",
+           "decode_ragged", "decode_workspace_size", "landmarks", "landmarks_append",
            "last_call_kernels", "last_call_launches", "lib", "path_overrides", "prefill",
            "prefill_backward", "prefill_backward_workspace_size", "prefill_varlen", "prefill_varlen_workspace_size", "prefill_workspace_size", "selftest_wait_expiry", "set_stage_events", "status_string",
            "workspace"]

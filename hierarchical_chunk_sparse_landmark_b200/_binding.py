@@ -34,7 +34,8 @@ EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",
             "hsa_last_call_kernels", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
             "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
             "hsa_prefill_variant", "hsa_prefill_varlen_workspace_size", "hsa_prefill_varlen",
-            "hsa_prefill_backward_workspace_size", "hsa_prefill_backward")
+            "hsa_prefill_backward_workspace_size", "hsa_prefill_backward", "hsa_decode_ragged",
+            "hsa_landmarks_append")
 
 
 class Variant(ctypes.Structure):
@@ -76,6 +77,10 @@ def _declare(lib):
     lib.hsa_decode_workspace_size.restype = sz
     lib.hsa_decode.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, i32, f32,
                                vp, vp, vp, sz, vp]
+    lib.hsa_decode_ragged.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
+                                      i32, f32, vp, vp, vp, vp, sz, vp]
+    lib.hsa_landmarks_append.argtypes = [vp, i32, vp, i32, i32, i32, i64, i32, i32, vp, vp, i32,
+                                         vp]
     lib.hsa_check.argtypes = [vp, vp]
     lib.hsa_selftest_wait_expiry.argtypes = [vp, sz, i64, vp]
     lib.hsa_decode_noalloc.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32,
@@ -98,7 +103,8 @@ def _declare(lib):
               "hsa_set_stage_events", "hsa_last_call_launches", "hsa_decode_noalloc",
               "hsa_selftest_wait_expiry", "hsa_set_path_overrides", "hsa_decode_cp_candidates",
               "hsa_decode_cp_merge", "hsa_decode_cp_attend", "hsa_decode_cp_combine",
-              "hsa_prefill_variant", "hsa_prefill_varlen", "hsa_prefill_backward"):
+              "hsa_prefill_variant", "hsa_prefill_varlen", "hsa_prefill_backward",
+              "hsa_decode_ragged", "hsa_landmarks_append"):
         getattr(lib, n).restype = i32
     return lib
 
@@ -346,6 +352,52 @@ def decode(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.0, out=N
                           _stream(dev))
     _check(st, "hsa_decode")
     return out, _opt(idx_out)
+
+
+def decode_ragged(q, K, V, lm, lens, *, S: int = 64, topk: int = 8, scale: float = 0.0,
+                  out=None, idx_out=None, ws=None):
+    """hsa_decode over caches of different lengths: sequence b holds lens[b]
+    (int32 [B] on the device) of the Lmax = K.shape[2] allocated tokens and
+    retrieves among its first lens[b] // S chunks.  Returns (O, idx)."""
+    for n, t in (("q", q), ("K", K), ("V", V), ("lm", lm), ("lens", lens)):
+        _dev(t, n)
+    B, H, d = q.shape
+    _, Hkv, Lmax, _ = K.shape
+    if lens.dtype != torch.int32 or lens.shape != (B,):
+        raise ValueError("lens must be int32 [B]")
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is True:
+        idx_out = torch.empty(B, Hkv, topk, dtype=torch.int32, device=dev)
+    nbytes = decode_workspace_size(B, H, Hkv, Lmax, d, S, topk)
+    if ws is None:
+        ws = workspace(nbytes, dev, ("decode", B * Hkv))
+    st = lib().hsa_decode_ragged(_ptr(q), _ptr(K), _ptr(V), _dtype_code(q), _ptr(lm),
+                                 _dtype_code(lm), B, H, Hkv, Lmax, d, S, topk, float(scale),
+                                 _ptr(lens), _ptr(out), _ptr(_opt(idx_out)), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(dev))
+    _check(st, "hsa_decode_ragged")
+    return out, _opt(idx_out)
+
+
+def landmarks_append(K, lm, len_before, len_after, *, S: int = 64, max_new_chunks: int = 1):
+    """Write the DHSA landmarks of the chunks completed while each cache grew
+    from len_before[b] to len_after[b] tokens into lm [B, Hkv, Lmax//S, d]
+    (fp32 or bf16), leaving every other row as it is."""
+    for n, t in (("K", K), ("lm", lm), ("len_before", len_before), ("len_after", len_after)):
+        _dev(t, n)
+    B, Hkv, Lmax, d = K.shape
+    if lm.shape != (B, Hkv, Lmax // S, d):
+        raise ValueError(f"lm must be [B, Hkv, Lmax//S, d] = {(B, Hkv, Lmax // S, d)}")
+    for t in (len_before, len_after):
+        if t.dtype != torch.int32 or t.shape != (B,):
+            raise ValueError("lengths must be int32 [B]")
+    _check(lib().hsa_landmarks_append(_ptr(K), _dtype_code(K), _ptr(lm), _dtype_code(lm), B, Hkv,
+                                      Lmax, d, S, _ptr(len_before), _ptr(len_after),
+                                      int(max_new_chunks), _stream(K.device)),
+           "hsa_landmarks_append")
+    return lm
 
 
 def decode_noalloc(q, K, V, lm, *, S: int = 64, topk: int = 8, scale: float = 0.0, out=None,

@@ -23,6 +23,9 @@ cudaError_t launch_attend_simt(const void *Q, const void *K, const void *V, bool
                                void *O, cudaStream_t st);
 cudaError_t launch_varlen_setup(const int32_t *bounds, int64_t n, int64_t L, int32_t *bs,
                                 int32_t *tok_chunk, unsigned *status, cudaStream_t st);
+cudaError_t launch_landmarks_append(const void *K, bool bf16, void *lm, bool lm_bf16, int B,
+                                    int Hkv, int64_t Lmax, int d, int S, const int32_t *len0,
+                                    const int32_t *len1, int max_new_chunks, cudaStream_t st);
 cudaError_t launch_landmarks_varlen(const void *K, bool bf16, float *lm, int B, int Hkv, int64_t L,
                                     int d, const int32_t *bounds, int64_t n, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const void *Kc, const void *Vc, bool bf16,
@@ -500,10 +503,15 @@ size_t hsa_decode_workspace_size(int B, int H, int Hkv, int64_t Lc, int d, int S
     return decode_layout(B, Hkv, Lc, S, topk).total;
 }
 
-hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
-                        const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t Lc,
-                        int d, int S, int topk, float scale, void *O, int32_t *idx_out,
-                        void *workspace, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// hsa_decode and hsa_decode_ragged: lens = null, every sequence sees Lc tokens.
+hsa_status_t decode_impl(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                         const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t Lc,
+                         int d, int S, int topk, float scale, const int32_t *lens, void *O,
+                         int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream) {
     hsa_status_t s = check_shape(B, H, Hkv, Lc, d, S, topk);
     if (s != HSA_OK) return s;
     if (!dtype_ok(dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
@@ -531,7 +539,9 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
     if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
     char *ws = (char *)workspace;
     stage_mark(0, st);
-    const DecodeShard whole = {0, nullptr, nullptr, nullptr, nullptr, nullptr};
+    DecodeShard whole = {0, nullptr, nullptr, nullptr, nullptr, nullptr};
+    whole.lens = lens;
+    whole.S = S;
     hsa_status_t r = from_cuda(launch_decode(q, Kc, Vc, dt == HSA_BF16, lm, lm_dt == HSA_BF16, B, H, Hkv,
                                    Lc, d, S, topk, scale, lay.splits, lay.at(ws), O,
                                    idx_out, whole, 0, nullptr, st));
@@ -539,6 +549,52 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
     t_kernels = r == HSA_OK ? (unsigned)(HSA_K_DECODE_SCAN | HSA_K_DECODE_ATTEND) : 0u;
     stage_mark(1, st);
     return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                        const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv, int64_t Lc,
+                        int d, int S, int topk, float scale, void *O, int32_t *idx_out,
+                        void *workspace, size_t ws_bytes, void *stream) {
+    return decode_impl(q, Kc, Vc, dt, lm, lm_dt, B, H, Hkv, Lc, d, S, topk, scale, nullptr, O,
+                       idx_out, workspace, ws_bytes, stream);
+}
+
+hsa_status_t hsa_decode_ragged(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                               const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                               int64_t Lmax, int d, int S, int topk, float scale,
+                               const int32_t *lens, void *O, int32_t *idx_out, void *workspace,
+                               size_t ws_bytes, void *stream) {
+    if (!lens || !aligned16(lens)) return HSA_ERR_INVALID_ARG;
+    return decode_impl(q, Kc, Vc, dt, lm, lm_dt, B, H, Hkv, Lmax, d, S, topk, scale, lens, O,
+                       idx_out, workspace, ws_bytes, stream);
+}
+
+hsa_status_t hsa_landmarks_append(const void *K, hsa_dtype_t k_dt, void *lm, hsa_dtype_t lm_dt,
+                                  int B, int Hkv, int64_t Lmax, int d, int S,
+                                  const int32_t *len_before, const int32_t *len_after,
+                                  int max_new_chunks, void *stream) {
+    hsa_status_t s = check_shape(B, Hkv, Hkv, Lmax, d, S, 1);
+    if (s != HSA_OK) return s;
+    if (!dtype_ok(k_dt) || !dtype_ok(lm_dt)) return HSA_ERR_UNSUPPORTED;
+    if (Lmax % S != 0 || max_new_chunks < 0) return HSA_ERR_INVALID_ARG;
+    t_launches = 0;
+    t_kernels = 0;
+    if (Lmax == 0) return HSA_OK;
+    const void *ptrs[] = {K, lm, len_before, len_after};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
+    const cudaError_t e = launch_landmarks_append(K, k_dt == HSA_BF16, lm, lm_dt == HSA_BF16, B,
+                                                  Hkv, Lmax, d, S, len_before, len_after,
+                                                  max_new_chunks, (cudaStream_t)stream);
+    if (e == cudaSuccess) {
+        t_launches = 1;
+        t_kernels = HSA_K_LANDMARKS;
+    }
+    return from_cuda(e);
 }
 
 hsa_status_t hsa_decode_cp_candidates(const void *q, hsa_dtype_t dt, const void *lm,

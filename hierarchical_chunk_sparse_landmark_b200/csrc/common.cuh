@@ -273,6 +273,9 @@ struct DecodeShard {
     float *cand_score;     // [B*Hkv*topk] or null: the shard's top-K scores (scan)
     int32_t *cand_idx;     // [B*Hkv*topk] or null: their global chunk indices (-1: none)
     float *m, *Z, *acc;    // [B*H], [B*H], [B*H*d] or null: fusion state instead of O (attend)
+    // ragged batch: sequence b sees its first lens[b] / S chunks (null: all of them)
+    const int32_t *lens = nullptr;
+    int S = 0;
 };
 
 // Bytes at the head of a decode workspace that must be zero before a call

@@ -104,10 +104,19 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
     const int g = (int)(bg % Hkv);
     const int G = H / Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t nunits = (Nc + ROWS - 1) / ROWS;
     const TL *lm_bg = lm + bg * Nc * D;
     const int KP = pow2_at_least(topk);
     grid_dep_wait();            // inputs and workspace may come from the previous kernel
+    // chunks this sequence sees: all Nc, or its first lens[b] / S (ragged batch;
+    // a length outside 0 .. Nc*S is flagged and clamped)
+    int64_t nvis = Nc;
+    if (sh.lens) {
+        const int64_t len = sh.lens[b];
+        if ((len < 0 || len > Nc * sh.S) && split == 0 && g == 0 && tid == 0)
+            atomicOr(ws.status, kFlagBadBounds);
+        nvis = len < 0 ? 0 : len > Nc * sh.S ? Nc : len / sh.S;
+    }
+    const int64_t nunits = (nvis + ROWS - 1) / ROWS;
 
     if (tid == 0) {
         for (int i = 0; i < kScanStages; ++i) {
@@ -146,7 +155,7 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
                 }
                 u_next = (int64_t)atomicAdd(ws.next_unit + bg, 1u);
                 const int64_t row0 = u * ROWS;
-                const int64_t left = Nc - row0;
+                const int64_t left = nvis - row0;
                 const uint32_t bytes = (uint32_t)((left < ROWS ? left : ROWS) * ROW_BYTES);
                 unit_of[slot] = u;
                 tc::mbar_expect_tx(&full[slot], bytes);
@@ -188,7 +197,7 @@ decode_scan_kernel(const T *__restrict__ q, const TL *__restrict__ lm, int H, in
             const int64_t unit = unit_of[slot];
             if (unit < 0) break;
             const int64_t row0 = unit * ROWS;
-            const int rows_here = (int)(Nc - row0 < ROWS ? Nc - row0 : ROWS);
+            const int rows_here = (int)(nvis - row0 < ROWS ? nvis - row0 : ROWS);
             const uint8_t *stage = ring + slot * kStageBytes;
 #pragma unroll
             for (int it = 0; it < ITER; ++it) {

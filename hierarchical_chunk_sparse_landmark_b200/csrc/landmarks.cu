@@ -81,6 +81,72 @@ cudaError_t launch_landmarks(const void *K, bool bf16, float *lm, int B, int Hkv
                     : launch_landmarks_t<float, 64>(K, lm, B, Hkv, L, st);
 }
 
+// ---------------------------------------------------------------- incremental update
+// Landmarks of the chunks that completed while a cache grew from len0[b] to
+// len1[b] tokens: chunks len0[b]/S .. len1[b]/S - 1 of sequence b (lengths
+// clamped to 0 .. Lmax).  One warp per chunk, lanes over 16-byte column
+// slices, 32 / (D / VEC) rows per step; partial rows folded by shuffles.
+template <typename T, typename TL, int D>
+__global__ void __launch_bounds__(256)
+landmarks_append_kernel(const T *__restrict__ K, TL *__restrict__ lm, int Hkv, int64_t Lmax,
+                        int S, const int32_t *__restrict__ len0, const int32_t *__restrict__ len1) {
+    constexpr int VEC = Vec16<T>::N;
+    constexpr int LPR = D / VEC;                              // lanes per row slice
+    constexpr int RPS = 32 / LPR;                             // rows per warp step
+    const int64_t bg = blockIdx.x;
+    const int64_t b = bg / Hkv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t Nmax = Lmax / S;
+    auto clampl = [&](int64_t v) { return v < 0 ? (int64_t)0 : v > Lmax ? Lmax : v; };
+    const int64_t lo = clampl(len0[b]) / S, hi = clampl(len1[b]) / S;
+    const int col = (lane % LPR) * VEC, r0 = lane / LPR;
+    const float f = rsqrtf((float)S);                         // sqrt(S) * (sum / S)
+    for (int64_t c = lo + (int64_t)blockIdx.y * 8 + warp; c < hi; c += (int64_t)gridDim.y * 8) {
+        const T *src = K + (bg * Lmax + c * S) * D + col;
+        float acc[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+        for (int r = r0; r < S; r += RPS) {
+            float v[VEC];
+            Vec16<T>::unpack(ld_stream16(src + (int64_t)r * D), v);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] += v[e];
+        }
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        if (lane < LPR) {
+            TL *dst = lm + (bg * Nmax + c) * D + col;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) dst[e] = from_f32<TL>(acc[e] * f);
+        }
+    }
+}
+
+cudaError_t launch_landmarks_append(const void *K, bool bf16, void *lm, bool lm_bf16, int B,
+                                    int Hkv, int64_t Lmax, int d, int S, const int32_t *len0,
+                                    const int32_t *len1, int max_new_chunks, cudaStream_t st) {
+    const int64_t pairs = (int64_t)B * Hkv;
+    if (pairs == 0 || Lmax / S == 0) return cudaSuccess;
+    int ny = (max_new_chunks + 7) / 8;
+    if (ny < 1) ny = 1;
+    if (ny > 1024) ny = 1024;
+    const dim3 grid((unsigned)pairs, (unsigned)ny);
+    using bf = __nv_bfloat16;
+#define HSA_APPEND(T, TL, DD) \
+    landmarks_append_kernel<T, TL, DD><<<grid, 256, 0, st>>>((const T *)K, (TL *)lm, Hkv, Lmax, S, len0, len1)
+    if (bf16) {
+        if (lm_bf16) { if (d == 128) HSA_APPEND(bf, bf, 128); else HSA_APPEND(bf, bf, 64); }
+        else { if (d == 128) HSA_APPEND(bf, float, 128); else HSA_APPEND(bf, float, 64); }
+    } else {
+        if (lm_bf16) { if (d == 128) HSA_APPEND(float, bf, 128); else HSA_APPEND(float, bf, 64); }
+        else { if (d == 128) HSA_APPEND(float, float, 128); else HSA_APPEND(float, float, 64); }
+    }
+#undef HSA_APPEND
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- variable-length chunks
 // Checks the boundaries (0 = b_0 < b_1 < ... < b_n = L, no chunk longer than
 // 64 tokens) in one block and stores the verdict in bs[n + 1].  Wrong

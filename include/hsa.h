@@ -86,6 +86,26 @@ enum {
 };
 
 /*
+ * hsa_landmarks_append -- incremental landmark update for growing caches: the
+ * DHSA landmarks (sqrt(S) * mean of the chunk's keys, as hsa_landmarks) of the
+ * chunks that became complete while sequence b grew from len_before[b] to
+ * len_after[b] tokens, i.e. chunks floor(len_before[b]/S) ..
+ * floor(len_after[b]/S) - 1; no other landmark row is touched.
+ *   K           [B, Hkv, Lmax, d]      k_dt, the cache (Lmax % S == 0)
+ *   lm          [B, Hkv, Lmax/S, d]    lm_dt: fp32, or bf16 (rounded to
+ *                                      nearest even; the form hsa_decode
+ *                                      streams fastest)
+ *   len_before, len_after  [B] int32, DEVICE; clamped to 0 .. Lmax
+ *   max_new_chunks  a bound on the new chunks of one sequence, used only to
+ *                   size the grid (any value >= 0 gives the same result)
+ * One warp per new chunk; K read once per new chunk.
+ */
+hsa_status_t hsa_landmarks_append(const void *K, hsa_dtype_t k_dt, void *lm, hsa_dtype_t lm_dt,
+                                  int B, int Hkv, int64_t Lmax, int d, int S,
+                                  const int32_t *len_before, const int32_t *len_after,
+                                  int max_new_chunks, void *stream);
+
+/*
  * hsa_landmarks -- DHSA landmarks: l[b,g,i] = sqrt(S) * mean of the S keys of
  * chunk i (Dynamic Hierarchical Sparse Attention review, "What carries the
  * argument": chunk representation sqrt(|C|) times the mean key).
@@ -289,6 +309,27 @@ hsa_status_t hsa_decode(const void *q, const void *Kc, const void *Vc, hsa_dtype
                         void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * hsa_decode_ragged -- hsa_decode over a batch of caches of different lengths
+ * (ragged batch): sequence b holds lens[b] tokens of a cache allocated for
+ * Lmax (Lmax % S == 0, the row stride of Kc, Vc and lm) and its new query
+ * retrieves among its first floor(lens[b] / S) chunks, the complete ones (HSA
+ * "Methodology in Plain English": the query retrieves among the chunks
+ * before it; the incomplete chunk holding the newest tokens is the sliding
+ * window's, as in hsa_decode).  A sequence with no complete chunk gets O = 0
+ * and an all -1 selection.
+ *   lens     [B] int32, DEVICE (16-byte aligned); a length outside 0 .. Lmax
+ *            is clamped and makes hsa_check return HSA_ERR_INVALID_ARG
+ * Everything else, including the workspace (hsa_decode_workspace_size with
+ * Lc = Lmax), is hsa_decode's.  The scan reads only each sequence's visible
+ * landmark rows.
+ */
+hsa_status_t hsa_decode_ragged(const void *q, const void *Kc, const void *Vc, hsa_dtype_t dt,
+                               const void *lm, hsa_dtype_t lm_dt, int B, int H, int Hkv,
+                               int64_t Lmax, int d, int S, int topk, float scale,
+                               const int32_t *lens, void *O, int32_t *idx_out, void *workspace,
+                               size_t ws_bytes, void *stream);
+
+/*
  * hsa_decode_noalloc -- hsa_decode for callers that cannot allocate device
  * memory.  (The pages describe no such call; it is an interface convenience
  * of this library.)  Some callers cannot hand hsa_decode a workspace: a
@@ -400,8 +441,9 @@ hsa_status_t hsa_selftest_wait_expiry(void *workspace, size_t ws_bytes, int64_t 
  * hsa_check -- synchronises `stream`, then reads the status word at the head
  * of `workspace` (the one given to the preceding hsa_prefill / hsa_decode).
  * Returns HSA_ERR_TIMEOUT if a device-side bounded wait gave up,
- * HSA_ERR_INVALID_ARG if hsa_prefill_varlen found its chunk boundaries wrong
- * or hsa_prefill_backward a selection entry that names no visible chunk
+ * HSA_ERR_INVALID_ARG if hsa_prefill_varlen found its chunk boundaries wrong,
+ * hsa_decode_ragged a length outside 0 .. Lmax or hsa_prefill_backward a
+ * selection entry that names no visible chunk
  * (either clears the word), HSA_ERR_CUDA if the stream reports an error,
  * HSA_OK otherwise.
  * With workspace = NULL it reads the status word of hsa_decode_noalloc's
