@@ -209,18 +209,75 @@ def kernel_source_hash(files) -> str:
 
 def measured_traffic(kernel: str, src_files, key: str = "dram_bytes_per_launch",
                      workload: str | None = None) -> float | None:
-    """Per-launch DRAM bytes (`key`: read + write, or the write part alone)
-    from the committed ncu summary, if it was taken on the current source of
-    that kernel and, when `workload` is given, on that workload (else None)."""
+    """Per-launch DRAM bytes (`key`: read + write, or the write part alone) of
+    `kernel` on `workload` from the committed ncu summary (entry
+    "kernel:workload"), if it was taken on the current source of that kernel
+    (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(kernel)
+    d = json.load(open(p)).get(f"{kernel}:{workload}")
     if not d or d.get("source_hash") != kernel_source_hash(src_files):
         return None
-    if workload is not None and d.get("workload", "").split(" ")[0] != workload:
-        return None
     return d.get(key)
+
+
+# kernel families of the roofline lines: ncu kernel-name pattern, source files
+TRAFFIC_FAMILIES = {
+    "attend_tc": (("attend_tc_kernel",), ["attend_tc.cu"]),
+    "attend_simt": (("attend_simt_kernel",), ["attend_simt.cu"]),
+    "decode": (("decode_scan_kernel", "decode_attend_kernel"), ["decode.cu"]),
+    "landmarks": (("landmarks_kernel",), ["landmarks.cu"]),
+}
+
+
+def traffic_from_ncu(csv_path: str, workload: str, families: str = "",
+                     out_path: str | None = None) -> dict:
+    """Per-launch DRAM bytes of each kernel family from an ncu CSV of one
+    workload (metrics dram__bytes_read.sum and dram__bytes_write.sum, one row
+    per launch and metric): the median launch of every kernel of the family,
+    summed over the family's kernels (the decode call is its scan plus its
+    attend kernel).  Merged into profiles/traffic.json under "family:workload"
+    with the hash of the family's current source.  `families` (comma-separated)
+    limits the families taken from this CSV (a command can run two workloads)."""
+    import csv
+    import statistics as st
+    per = {}
+    hdr = None
+    for r in csv.reader(open(csv_path)):
+        if r and r[0] == "ID":
+            hdr = r
+            continue
+        if not hdr or len(r) != len(hdr):
+            continue
+        d = dict(zip(hdr, r))
+        name = d["Kernel Name"].split("(")[0].split("<")[0].split("::")[-1].strip().split(" ")[-1]
+        if d["Metric Name"] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            val = float(d["Metric Value"].replace(",", ""))
+            unit = d.get("Metric Unit", "byte").lower()
+            val *= {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9}.get(unit, 1)
+            per.setdefault((name, d["ID"]), {})[d["Metric Name"]] = val
+    out_path = out_path or os.path.join(ROOT, "profiles", "traffic.json")
+    table = json.load(open(out_path)) if os.path.exists(out_path) else {}
+    wanted = [f for f in families.split(",") if f] or list(TRAFFIC_FAMILIES)
+    for fam, (kernels, files) in TRAFFIC_FAMILIES.items():
+        if fam not in wanted or not all(any(k == n for (n, _) in per) for k in kernels):
+            continue
+        rd = wr = 0.0
+        for k in kernels:
+            launches = [v for (n, _), v in per.items() if n == k]
+            rd += st.median(v.get("dram__bytes_read.sum", 0.0) for v in launches)
+            wr += st.median(v.get("dram__bytes_write.sum", 0.0) for v in launches)
+        table[f"{fam}:{workload}"] = {
+            "source_hash": kernel_source_hash([ATTN_SRC + f for f in files]),
+            "dram_bytes_per_launch": rd + wr, "dram_write_bytes_per_launch": wr,
+            "workload": workload, "kernels": list(kernels),
+            "note": "dram__bytes_read.sum + dram__bytes_write.sum, median launch per kernel "
+                    "(ncu --clock-control none, one pass)"}
+    with open(out_path, "w") as f:
+        json.dump(table, f, indent=2, sort_keys=True)
+        f.write("\n")
+    return table
 
 
 # ----------------------------------------------------------------------------- dist
@@ -868,9 +925,16 @@ def main(argv=None):
     ap.add_argument("--no-extra", dest="extra", action="store_false",
                     help="leave out the lines of the other workloads (train-shape and fp32 "
                          "prefill, batched decode)")
+    ap.add_argument("--traffic-from-ncu", nargs=3, metavar=("CSV", "WORKLOAD", "FAMILIES"),
+                    help="write the per-launch DRAM bytes of the kernel FAMILIES (comma-"
+                         "separated: attend_tc, attend_simt, decode, landmarks) in an ncu CSV "
+                         "of WORKLOAD into profiles/traffic.json and exit")
     ap.add_argument("--decode-workload", default="decode_32m_bf16",
                     help="decode workload of the decode line (decode_32m_bf16, batched_decode_bf16)")
     args = ap.parse_args(argv)
+    if args.traffic_from_ncu:
+        traffic_from_ncu(*args.traffic_from_ncu)
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
