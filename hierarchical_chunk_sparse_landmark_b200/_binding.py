@@ -24,7 +24,7 @@ HSA_F32, HSA_BF16 = 0, 1
 K_LANDMARKS, K_SPLIT_LANDMARKS, K_SELECT_TC_ONE_TILE, K_SELECT_TC_MULTI_TILE = 1, 2, 4, 8
 K_SELECT_SIMT, K_WORK_LISTS, K_ATTEND_TC, K_FUSE, K_ATTEND_SIMT = 16, 32, 64, 128, 256
 K_DECODE_SCAN, K_DECODE_ATTEND, K_DECODE_CP_MERGE, K_DECODE_CP_COMBINE = 512, 1024, 2048, 4096
-K_BACKWARD = 8192
+K_BACKWARD, K_BACKWARD_TC = 8192, 16384
 PATH_SIMT_PREFILL, PATH_SIMT_SELECT, PATH_MULTI_TILE_SELECT = 1, 2, 4
 
 EXPORTED = ("hsa_landmarks", "hsa_prefill_workspace_size", "hsa_prefill",

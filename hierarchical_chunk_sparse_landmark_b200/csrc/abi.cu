@@ -715,7 +715,8 @@ size_t hsa_prefill_backward_workspace_size(int B, int H, int Hkv, int64_t L, int
                                            int topk, int dhsa) {
     if (check_shape(B, H, Hkv, L, d, S, topk) != HSA_OK) return 0;
     if (L >= ((int64_t)1 << 26) || (int64_t)B * Hkv * L * topk >= (int64_t)INT32_MAX) return 0;
-    return bwd_layout(B, H, Hkv, L, d, S, topk, dhsa != 0).total;
+    // room for the tensor-core path whenever the shape could take it (bf16 inputs)
+    return bwd_layout(B, H, Hkv, L, d, S, topk, dhsa != 0, H / Hkv == 8 && d == 128).total;
 }
 
 hsa_status_t hsa_prefill_backward(const void *Q, const void *K, const void *V, hsa_dtype_t dt,
@@ -740,7 +741,8 @@ hsa_status_t hsa_prefill_backward(const void *Q, const void *K, const void *V, h
         if (!p || !aligned16(p)) return HSA_ERR_INVALID_ARG;
     const bool dhsa = lm == nullptr;
     if (!dhsa && (!aligned16(lm) || !dlm || !aligned16(dlm))) return HSA_ERR_INVALID_ARG;
-    const BwdLayout lay = bwd_layout(B, H, Hkv, L, d, S, topk, dhsa);
+    const bool tc = backward_tc_supported(dt == HSA_BF16, H / Hkv, d) && !force_simt_path();
+    const BwdLayout lay = bwd_layout(B, H, Hkv, L, d, S, topk, dhsa, tc);
     if (ws_bytes < lay.total) return HSA_ERR_WORKSPACE;
     if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
     cudaStream_t st = (cudaStream_t)stream;
@@ -765,8 +767,10 @@ hsa_status_t hsa_prefill_backward(const void *Q, const void *K, const void *V, h
     }
     const cudaError_t e = launch_backward(a, lay, st);
     if (e == cudaSuccess) {
-        t_launches += lay.Nc > 0 ? 6 : 4;     // row, [hist], scan, [scatter], key, reduce
-        t_kernels |= HSA_K_BACKWARD;
+        // CUDA cores: row, [hist], scan, [scatter], key, reduce; tensor cores: weights,
+        // [hist], scan, [scatter], key (tcgen05), row finish, dl, reduce
+        t_launches += (tc ? 6 : 4) + (lay.Nc > 0 ? 2 : 0);
+        t_kernels |= HSA_K_BACKWARD | (tc ? (unsigned)HSA_K_BACKWARD_TC : 0u);
     }
     stage_mark(1, st);
     return from_cuda(e);

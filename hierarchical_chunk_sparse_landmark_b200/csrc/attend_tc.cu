@@ -54,6 +54,7 @@
 #include "attend_tc.h"
 #include "common.cuh"
 #include "tc.cuh"
+#include "tmap.cuh"
 
 namespace hsa {
 
@@ -736,68 +737,6 @@ fuse_kernel(const __half *__restrict__ part, const __half *__restrict__ own,
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)ptr;
-    }
-    return fn;
-}
-
-// 2D bf16 view [rows, D] with 128-byte swizzled boxes of 64 columns x box_rows.
-static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-    const cuuint32_t es[2] = {1u, 1u};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
-
-// 3-D bf16 view of two planes [2][rows, D]: one box (64, 1, 2) brings a row's
-// 64-column block from both planes as two consecutive 128B-swizzled rows.
-static bool make_map_planes(CUtensorMap *m, const void *base, uint64_t rows, int D) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, 2u};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-    const cuuint32_t box[3] = {64u, 1u, 2u};
-    const cuuint32_t es[3] = {1u, 1u, 1u};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
-
-// 3-D bf16 view of [rows, D] (D = 128) as (64 columns, rows, 2 halves of d),
-// strides 2*D and 128 bytes: one box (64, G, 2) brings all of an entry's G
-// rows, both halves, as two 128B-swizzled [G x 128 B] blocks.
-static bool make_map_q3d(CUtensorMap *m, const void *base, uint64_t rows, int D, int G) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(D / 64)};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, 128u};
-    const cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)(D / 64)};
-    const cuuint32_t es[3] = {1u, 1u, 1u};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
-
 template <int D, int G>
 static cudaError_t launch_attend_tc_t(const TcLaunch &a, cudaStream_t st, cudaEvent_t mid) {
     using C = TcCfg<D, G>;

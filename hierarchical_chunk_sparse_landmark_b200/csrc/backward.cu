@@ -602,8 +602,18 @@ bwd_reduce_kernel(const float *__restrict__ part, const int32_t *__restrict__ ch
 }
 
 // ---------------------------------------------------------------- host side
-BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, bool dhsa) {
+cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, const void *dO,
+                               const void *lm, bool lm_bf16, const int32_t *idx, int B, int H,
+                               int Hkv, int64_t L, int S, int64_t Nc, int64_t NcAll, int topk,
+                               int own_chunk, float scale, float2 *coef, float *dw, float *dqp,
+                               const int4 *segs, const int32_t *nseg, const int32_t *entries,
+                               float *part, int64_t max_seg, unsigned *status, float *dQ,
+                               int phase, cudaStream_t st);
+
+BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, bool dhsa,
+                     bool tc) {
     BwdLayout p;
+    p.tc = tc;
     const int G = H / Hkv;
     p.BG = (int64_t)B * Hkv;
     p.Nc = L / S;
@@ -631,6 +641,13 @@ BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, b
     off = align_up(off + 2 * sizeof(int32_t) * (size_t)(p.BG * p.NcAll), 256);
     p.part_off = off;
     off = align_up(off + sizeof(float) * 129 * (size_t)d * (size_t)p.max_seg, 256);
+    p.dw_off = p.dqp_off = off;
+    if (tc) {                // dw per (row, slot) and the dQ partial rows, own chunk last
+        p.dw_off = off;
+        off = align_up(off + sizeof(float) * (size_t)B * L * H * (topk + 1), 256);
+        p.dqp_off = off;
+        off = align_up(off + sizeof(float) * (size_t)B * L * H * (topk + 1) * d, 256);
+    }
     p.total = off;
     return p;
 }
@@ -650,8 +667,15 @@ static cudaError_t launch_backward_t(const BwdArgs &a, const BwdLayout &p, cudaS
     unsigned *status = (unsigned *)ws;
     constexpr int VEC = Vec16<T>::N;
 
-    // 1. dQ and the per-slot coefficients
-    {
+    // 1. dQ and the per-slot coefficients (CUDA cores), or the fusion weights
+    //    alone (tensor-core path: dQ comes from the key pass)
+    if (p.tc) {
+        cudaError_t e = launch_backward_tc(a.Q, a.K, a.V, a.dO, a.lm, a.lm_bf16 != 0, a.idx, a.B,
+                                           a.H, a.Hkv, a.L, a.S, p.Nc, p.NcAll, a.topk,
+                                           a.own_chunk, a.scale, coef, nullptr, nullptr, nullptr,
+                                           nullptr, nullptr, nullptr, 0, status, a.dQ, 0, st);
+        if (e != cudaSuccess) return e;
+    } else {
         const size_t smem = sizeof(float) * 2 * G * D + 2 * sizeof(T) * 64 * (D + VEC);
         auto kern = bwd_row_kernel<T, D>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -690,7 +714,13 @@ static cudaError_t launch_backward_t(const BwdArgs &a, const BwdLayout &p, cudaS
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 3. per-segment dK / dV / dl partials
-    {
+    if (p.tc) {
+        e = launch_backward_tc(a.Q, a.K, a.V, a.dO, a.lm, a.lm_bf16 != 0, a.idx, a.B, a.H, a.Hkv,
+                               a.L, a.S, p.Nc, p.NcAll, a.topk, a.own_chunk, a.scale, coef,
+                               (float *)(ws + p.dw_off), (float *)(ws + p.dqp_off), segs, nseg,
+                               entries, part, p.max_seg, status, a.dQ, 1, st);
+        if (e != cudaSuccess) return e;
+    } else {
         const size_t smem =
             sizeof(float) * (2 * 64 * (D + kKeyLanes) + 2 * 8 * D + 3 * (kKeyThreads / 32) * 8);
         auto kern = bwd_key_kernel<T, D>;

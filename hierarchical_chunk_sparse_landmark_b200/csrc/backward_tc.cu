@@ -1,0 +1,512 @@
+// backward_tc.cu -- the prefill backward on the 5th-generation tensor cores
+// (bf16 inputs, G = 8 query heads per KV group, d = 128).
+//
+// Same gradients as backward.cu (HiLS Attention abstract: the retrieval scores
+// are learned end to end; the selection is held fixed), organised around the
+// forward's chunk tiles: a tile is one chunk's 64 keys/values and up to 16
+// entries (token, slot) that selected it, 8 query-head rows each, so 128 rows.
+// Per tile, with w the row's fusion weight (1 for the own chunk):
+//
+//   S  = Q.K^T, U = dO.V^T            M = 128 rows, N = 64 keys, K = d   (TMEM)
+//   p  = softmax_j(scale S) (causal mask on own tiles), dw = sum_j p_j U_j
+//   dS = scale w p (U - dw), wP = w p   (bf16, written to shared memory)
+//   dV^T += dO^T . wP,  dK^T += Q^T . dS  M = d, N = 64, K = 128 rows (TMEM,
+//                                         accumulated over the segment's tiles)
+//   dQp  = dS . K                       M = 128 rows, N = d, K = 64 keys
+//
+// The transposed products read the Q / dO / K tiles already in shared memory
+// as MN-major operands (no copy).  One block (4 warps, thread = tile row =
+// TMEM lane) per segment of a chunk's sorted entry list (at most 8 tiles) or
+// per own chunk (at most 4 tiles of 16 tokens); K and V are loaded once per
+// segment.  dw and the dQ partial rows of every (row, slot) go to global
+// memory; bwd_rowfin_kernel then forms dz = w (dw - sum w dw), sums the dQ
+// partials and adds scale sum dz l; bwd_dl_kernel forms each segment's
+// landmark gradient scale sum dz q; the ordered reduction of backward.cu adds
+// the segments.  All in a fixed order: bit-reproducible.
+//
+// Precision: P and dS enter the second products as bf16 (as P does in the
+// forward), so gradients carry ~2^-9 relative rounding per term.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+#include "tmap.cuh"
+
+namespace hsa {
+
+namespace {
+
+constexpr int kBtThreads = 128;
+constexpr long long kBtWait = 4000000000LL;       // SM cycles (about 2 s)
+constexpr int BT_D = 128, BT_G = 8, BT_EPT = 16;  // d, heads per entry, entries per tile
+// shared memory, offsets from a 1024-byte aligned base
+constexpr int OFF_Q = 0;                   // [16 entries][2 halves of d][8 rows][128 B]
+constexpr int OFF_DO = OFF_Q + 32768;      // same layout
+constexpr int OFF_K = OFF_DO + 32768;      // [2 halves][64 keys][128 B]
+constexpr int OFF_V = OFF_K + 16384;
+constexpr int OFF_DS = OFF_V + 16384;      // [128 rows][64 keys] bf16, 128B-swizzled
+constexpr int OFF_WP = OFF_DS + 16384;
+constexpr int OFF_BAR = OFF_WP + 16384;    // two mbarriers, TMEM address, abort flag
+constexpr int BT_SMEM = 1024 + OFF_BAR + 64;
+// TMEM columns (fp32)
+constexpr uint32_t COL_S = 0, COL_U = 64, COL_DQ = 128, COL_DV = 256, COL_DK = 320;
+constexpr uint32_t BT_TMEM_COLS = 512;
+
+struct BtParams {
+    const int4 *segs;
+    const int32_t *nseg;
+    const int32_t *entries;
+    const float2 *coef;      // [B*L*H][topk]: .x = w (written by bwd_coefw_kernel)
+    float *dw;               // [B*L*H][topk+1]: dw of every (row, slot); slot topk = own
+    float *dqp;              // [B*L*Hkv][topk+1][G][D]: dQ partial rows
+    float *part;             // per segment: dK [64][D], dV [64][D], dl [D]
+    unsigned *status;
+    int64_t L, NcAll;
+    int H, Hkv, topk, S;
+    float scale;
+};
+
+__device__ __forceinline__ bool bt_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!tc::mbar_try_wait(bar, parity)) {
+        if (*abort || clock64() - t0 > kBtWait) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kBtThreads, 1)
+bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const BtParams p) {
+    constexpr int D = BT_D, G = BT_G;
+    const int64_t sidx = blockIdx.x;
+    if (sidx >= *p.nseg) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *tma_bar = (uint64_t *)(sm + OFF_BAR), *mma_bar = tma_bar + 1;
+    uint32_t *s_tmem = (uint32_t *)(mma_bar + 1);
+    volatile int *s_abort = (volatile int *)(s_tmem + 1);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+    const int4 sg = p.segs[sidx];
+    const int64_t q = sg.x;
+    const int64_t bg = q / p.NcAll, c = q % p.NcAll;
+    const int64_t b = bg / p.Hkv;
+    const int g = (int)(bg % p.Hkv);
+    const int own = sg.w;
+    const int64_t L = p.L;
+    const int64_t first = c * p.S;
+    const int nkc = (int)(L - first < p.S ? L - first : p.S);
+    const int H = p.H, topk = p.topk;
+
+    // rows of entries a tile does not fill are read by the transposed
+    // products (times zero): they must hold finite values
+    for (int i = tid; i < 65536 / 16; i += kBtThreads)
+        reinterpret_cast<uint4 *>(sm + OFF_Q)[i] = make_uint4(0u, 0u, 0u, 0u);
+    tc::fence_proxy_async_smem();
+    if (warp == 0) {
+        tc::tmem_alloc(s_tmem, BT_TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(tma_bar, 1);
+        tc::mbar_init(mma_bar, 1);
+        *s_abort = 0;
+        tc::fence_barrier_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+    uint32_t ptma = 0, pmma = 0;
+
+    // K and V of the chunk, once per segment
+    const int krow = (int)(bg * L + first);
+    if (tid == 0) {
+        tc::mbar_expect_tx(tma_bar, 2u * 16384u);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+            tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, tma_bar, kb * 64, krow);
+            tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, tma_bar, kb * 64, krow);
+        }
+    }
+    // every wait's outcome is made block-uniform, so that all threads leave
+    // the tile loop together on a timeout
+    bool ok = __syncthreads_and(bt_wait(tma_bar, ptma, s_abort)) != 0;
+    ptma ^= 1u;
+
+    // descriptors (bytes >> 4 in the start field; a K step moves the start)
+    const uint32_t IDESC_SU = tc::idesc_bf16_f32(128, 64, false, false);
+    const uint32_t IDESC_T = tc::idesc_bf16_f32(128, 64, true, true);     // M = d, N = keys
+    const uint32_t IDESC_DQ = tc::idesc_bf16_f32(128, D, true, false);    // B = K, MN-major
+    const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q), 16, 2048);     // rows x d
+    const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO), 16, 2048);
+    const uint64_t bK = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);     // keys x d
+    const uint64_t bV = tc::sdesc_sw128(tc::smem_u32(sm + OFF_V), 16, 1024);
+    const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q), 1024, 2048);   // (d, rows)
+    const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO), 1024, 2048);
+    const uint64_t bDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16384, 1024);  // (keys, rows)
+    const uint64_t bWP = tc::sdesc_sw128(tc::smem_u32(sm + OFF_WP), 16384, 1024);
+    const uint64_t aDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16, 1024);     // rows x keys
+    const uint64_t bKt = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 8192, 1024);    // (d, keys)
+
+    const int e = tid >> 3, h = tid & 7;          // this thread's row: entry e, head h
+    const int n_units = own ? nkc : sg.z;          // tokens (own) or entries of the segment
+    const int ntiles = (n_units + BT_EPT - 1) / BT_EPT;
+    for (int ti = 0; ti < ntiles && ok; ++ti) {
+        const int u = ti * BT_EPT + e;
+        const bool valid = u < n_units;
+        int64_t t = -1;
+        int slot = topk;
+        if (valid) {
+            if (own) {
+                t = first + u;
+            } else {
+                const int32_t code = p.entries[sg.y + u];
+                t = code >> 5;
+                slot = code & 31;
+            }
+        }
+        const int nvalid = n_units - ti * BT_EPT < BT_EPT ? n_units - ti * BT_EPT : BT_EPT;
+        if (tid == 0) tc::mbar_expect_tx(tma_bar, (uint32_t)nvalid * 2u * 2048u);
+        __syncthreads();
+        if (valid && h == 0) {        // one 3-D box per entry: its 8 head rows, both halves
+            const int qrow = (int)((b * L + t) * H + (int64_t)g * G);
+            tc::tma_load_3d(sm + OFF_Q + e * 2048, &tmQ, tma_bar, 0, qrow, 0);
+            tc::tma_load_3d(sm + OFF_DO + e * 2048, &tmO, tma_bar, 0, qrow, 0);
+        }
+        if (!__syncthreads_and(bt_wait(tma_bar, ptma, s_abort))) { ok = false; break; }
+        ptma ^= 1u;
+        // S = Q.K^T and U = dO.V^T
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (kb | kk) ? 1u : 0u;
+                    tc::mma_bf16(tmem + COL_S, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                                 bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                    tc::mma_bf16(tmem + COL_U, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                                 bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                }
+            tc::mma_commit(mma_bar);
+        }
+        if (!__syncthreads_and(bt_wait(mma_bar, pmma, s_abort))) { ok = false; break; }
+        pmma ^= 1u;
+        tc::fence_after_sync();
+        // this row's chunk softmax, dw, dS and w p
+        float s[64], uu[64];
+        {
+            float tmp[32];
+            tc::tmem_ld32(tmem + lane_off + COL_S, tmp);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] = tmp[j];
+            tc::tmem_ld32(tmem + lane_off + COL_S + 32, tmp);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[32 + j] = tmp[j];
+            tc::tmem_ld32(tmem + lane_off + COL_U, tmp);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) uu[j] = tmp[j];
+            tc::tmem_ld32(tmem + lane_off + COL_U + 32, tmp);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) uu[32 + j] = tmp[j];
+            tc::tmem_wait_ld();
+        }
+        const int nk = own ? (valid ? (int)(t - first) + 1 : 64) : 64;
+        const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
+        const float w = !valid ? 0.f : own ? 1.f : p.coef[hrow * topk + slot].x;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) mx = j < nk ? fmaxf(mx, s[j]) : mx;
+        float z = 0.f, zu = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+            const float ej = j < nk ? expf(p.scale * (s[j] - mx)) : 0.f;
+            s[j] = ej;
+            z += ej;
+            zu = fmaf(ej, uu[j], zu);
+        }
+        const float inv = 1.f / z;
+        const float dwv = zu * inv;
+        if (valid) p.dw[hrow * (topk + 1) + slot] = dwv;
+        const float fds = valid ? p.scale * w * inv : 0.f, fwp = valid ? w * inv : 0.f;
+#pragma unroll
+        for (int cch = 0; cch < 8; ++cch) {
+            uint32_t ds4[4], wp4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = cch * 8 + 2 * i;
+                ds4[i] = pack2_bf16(fds * s[j] * (uu[j] - dwv), fds * s[j + 1] * (uu[j + 1] - dwv));
+                wp4[i] = pack2_bf16(fwp * s[j], fwp * s[j + 1]);
+            }
+            const uint32_t off = tc::sw128_offset(tid, cch);
+            *reinterpret_cast<uint4 *>(sm + OFF_DS + off) = make_uint4(ds4[0], ds4[1], ds4[2], ds4[3]);
+            *reinterpret_cast<uint4 *>(sm + OFF_WP + off) = make_uint4(wp4[0], wp4[1], wp4[2], wp4[3]);
+        }
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        // dV^T += dO^T . wP, dK^T += Q^T . dS (over the tile's 128 rows), dQp = dS . K
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t acc = (ti > 0 || ks > 0) ? 1u : 0u;
+                tc::mma_bf16(tmem + COL_DV, tO + (uint64_t)((ks * 4096) >> 4),
+                             bWP + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+                tc::mma_bf16(tmem + COL_DK, tQ + (uint64_t)((ks * 4096) >> 4),
+                             bDS + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + COL_DQ, aDS + (uint64_t)((kk * 32) >> 4),
+                             bKt + (uint64_t)((kk * 2048) >> 4), IDESC_DQ, kk > 0 ? 1u : 0u);
+            tc::mma_commit(mma_bar);
+        }
+        if (!__syncthreads_and(bt_wait(mma_bar, pmma, s_abort))) { ok = false; break; }
+        pmma ^= 1u;
+        tc::fence_after_sync();
+        // this row's dQ partial
+        float *dst = valid ? p.dqp + ((((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h) * (int64_t)D
+                           : nullptr;
+#pragma unroll 1
+        for (int cb = 0; cb < D / 32; ++cb) {
+            float v[32];
+            tc::tmem_ld32(tmem + lane_off + COL_DQ + cb * 32, v);
+            tc::tmem_wait_ld();
+            if (valid) {
+                float4 *d4 = reinterpret_cast<float4 *>(dst + cb * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();          // TMEM dQ and the Q / dO tiles are free for the next tile
+        tc::fence_after_sync();
+    }
+    // the segment's dK and dV partials (thread = element of d), dl is written by bwd_dl_kernel
+    float *pk = p.part + sidx * (int64_t)(129 * D);
+    if (ok) {
+#pragma unroll 1
+        for (int cb = 0; cb < 2; ++cb) {
+            float vk[32], vv[32];
+            tc::tmem_ld32(tmem + lane_off + COL_DK + cb * 32, vk);
+            tc::tmem_ld32(tmem + lane_off + COL_DV + cb * 32, vv);
+            tc::tmem_wait_ld();
+            const bool any = ntiles > 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                pk[(cb * 32 + j) * D + tid] = any ? vk[j] : 0.f;
+                pk[64 * D + (cb * 32 + j) * D + tid] = any ? vv[j] : 0.f;
+            }
+        }
+    } else {
+        if (tid == 0) atomicOr(p.status, kFlagTimeout);
+        // let copies and MMAs that may still be in flight land before exiting
+        const long long t0 = clock64();
+        while (clock64() - t0 < 20000000) { }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, BT_TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- CUDA-core companions
+// Fusion weights w = softmax over the valid slots of scale q.l (one warp per
+// query row (t, h), lane k keeps slot k), written to coef[.].x.
+template <typename TL>
+__global__ void __launch_bounds__(256)
+bwd_coefw_kernel(const __nv_bfloat16 *__restrict__ Q, const TL *__restrict__ lm,
+                 const int32_t *__restrict__ idx, int64_t rows, int H, int Hkv, int64_t L, int S,
+                 int64_t Nc, int topk, float scale, float2 *__restrict__ coef,
+                 unsigned *__restrict__ status) {
+    constexpr int D = BT_D, R = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t hrow = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (hrow >= rows) return;
+    const int64_t bt = hrow / H;
+    const int h = (int)(hrow % H);
+    const int G = H / Hkv, g = h / G;
+    const int64_t b = bt / L, t = bt % L;
+    const int64_t bg = b * Hkv + g;
+    float qv[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) qv[r] = __bfloat162float(Q[hrow * D + lane + 32 * r]);
+    const int32_t *ip = idx + (bt * Hkv + g) * topk;
+    float zk = -INFINITY;
+    bool vk = false;
+    for (int k = 0; k < topk; ++k) {
+        const int32_t ci = ip[k];
+        const bool ok = ci >= 0 && (int64_t)ci < Nc && (int64_t)ci < t / S;
+        if (!ok) {
+            if (ci >= 0 && lane == 0 && h % G == 0) atomicOr(status, kFlagBadIdx);
+            continue;
+        }
+        float a = 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) a = fmaf(qv[r], to_f32(lm[(bg * Nc + ci) * D + lane + 32 * r]), a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == k) { zk = scale * a; vk = true; }
+    }
+    float m = vk ? zk : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ew = vk ? expf(zk - m) : 0.f;
+    float sw = ew;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
+    if (lane < topk) coef[hrow * topk + lane] = make_float2(vk ? ew / sw : 0.f, 0.f);
+}
+
+// Per query row: dz = w (dw - sum w dw) (to coef[.].y), and
+// dQ = sum of the row's dQ partials over its valid slots and the own chunk
+// + scale sum_k dz_k l_k.
+template <typename TL>
+__global__ void __launch_bounds__(256)
+bwd_rowfin_kernel(const TL *__restrict__ lm, const int32_t *__restrict__ idx,
+                  const float *__restrict__ dw, const float *__restrict__ dqp, int64_t rows, int H,
+                  int Hkv, int64_t L, int S, int64_t Nc, int topk, int own_chunk, float scale,
+                  float2 *__restrict__ coef, float *__restrict__ dQ) {
+    constexpr int D = BT_D, R = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t hrow = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (hrow >= rows) return;
+    const int64_t bt = hrow / H;
+    const int h = (int)(hrow % H);
+    const int G = H / Hkv, g = h / G, hh = h % G;
+    const int64_t b = bt / L, t = bt % L;
+    const int64_t bg = b * Hkv + g;
+    const int32_t *ip = idx + (bt * Hkv + g) * topk;
+    const int32_t ci_l = lane < topk ? ip[lane] : -1;
+    const bool vk = lane < topk && ci_l >= 0 && (int64_t)ci_l < Nc && (int64_t)ci_l < t / S;
+    const float wk = vk ? coef[hrow * topk + lane].x : 0.f;
+    const float dwk = vk ? dw[hrow * (topk + 1) + lane] : 0.f;
+    float dsum = wk * dwk;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+    const float dzk = wk * (dwk - dsum);
+    if (lane < topk) coef[hrow * topk + lane] = make_float2(wk, dzk);
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    const float *qp = dqp + ((bt * Hkv + g) * (topk + 1)) * (int64_t)(G * D) + hh * D;
+    for (int k = 0; k < topk; ++k) {
+        if (!__shfl_sync(0xffffffffu, vk ? 1 : 0, k)) continue;
+        const float dz = scale * __shfl_sync(0xffffffffu, dzk, k);
+        const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            acc[r] += qp[(int64_t)k * G * D + lane + 32 * r] +
+                      dz * to_f32(lm[(bg * Nc + ci) * D + lane + 32 * r]);
+    }
+    if (own_chunk) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] += qp[(int64_t)topk * G * D + lane + 32 * r];
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) dQ[hrow * D + lane + 32 * r] = acc[r];
+}
+
+// Landmark-gradient partial of each entry segment, dl = scale sum_rows dz q
+// (thread = element of d); own-chunk segments carry none.
+__global__ void __launch_bounds__(BT_D)
+bwd_dl_kernel(const __nv_bfloat16 *__restrict__ Q, const float2 *__restrict__ coef,
+              const int32_t *__restrict__ entries, const int4 *__restrict__ segs,
+              const int32_t *__restrict__ nseg_p, int H, int Hkv, int64_t L, int64_t NcAll,
+              int topk, float scale, float *__restrict__ part) {
+    constexpr int D = BT_D;
+    const int64_t sidx = blockIdx.x;
+    if (sidx >= *nseg_p) return;
+    const int4 sg = segs[sidx];
+    const int64_t bg = (int64_t)sg.x / NcAll;
+    const int64_t b = bg / Hkv;
+    const int g = (int)(bg % Hkv);
+    const int G = H / Hkv;
+    const int d = threadIdx.x;
+    float acc = 0.f;
+    if (!sg.w) {
+        for (int u = 0; u < sg.z; ++u) {
+            const int32_t code = entries[sg.y + u];
+            const int64_t t = code >> 5;
+            const int slot = code & 31;
+            const int64_t r0 = (b * L + t) * H + (int64_t)g * G;
+#pragma unroll 8
+            for (int hh = 0; hh < G; ++hh)
+                acc = fmaf(coef[(r0 + hh) * topk + slot].y, __bfloat162float(Q[(r0 + hh) * D + d]), acc);
+        }
+    }
+    part[sidx * (int64_t)(129 * D) + 128 * D + d] = scale * acc;
+}
+
+// ---------------------------------------------------------------- host side
+bool backward_tc_supported(bool bf16, int G, int d) {
+    return bf16 && G == BT_G && d == BT_D && encode_fn() != nullptr;
+}
+
+cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, const void *dO,
+                               const void *lm, bool lm_bf16, const int32_t *idx, int B, int H,
+                               int Hkv, int64_t L, int S, int64_t Nc, int64_t NcAll, int topk,
+                               int own_chunk, float scale, float2 *coef, float *dw, float *dqp,
+                               const int4 *segs, const int32_t *nseg, const int32_t *entries,
+                               float *part, int64_t max_seg, unsigned *status, float *dQ,
+                               int phase, cudaStream_t st) {
+    const int64_t rows = (int64_t)B * L * H;
+    const unsigned rblocks = (unsigned)((rows + 7) / 8);
+    cudaError_t e;
+    if (phase == 0) {            // fusion weights (before the key pass)
+        if (lm_bf16)
+            bwd_coefw_kernel<__nv_bfloat16><<<rblocks, 256, 0, st>>>(
+                (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)lm, idx, rows, H, Hkv, L, S, Nc,
+                topk, scale, coef, status);
+        else
+            bwd_coefw_kernel<float><<<rblocks, 256, 0, st>>>(
+                (const __nv_bfloat16 *)Q, (const float *)lm, idx, rows, H, Hkv, L, S, Nc, topk,
+                scale, coef, status);
+        return cudaGetLastError();
+    }
+    CUtensorMap mq, mo, mk, mv;
+    if (!make_map_q3d(&mq, Q, (uint64_t)rows, BT_D, BT_G) ||
+        !make_map_q3d(&mo, dO, (uint64_t)rows, BT_D, BT_G) ||
+        !make_map(&mk, K, (uint64_t)B * Hkv * L, BT_D, 64) ||
+        !make_map(&mv, V, (uint64_t)B * Hkv * L, BT_D, 64))
+        return cudaErrorInvalidValue;
+    BtParams p;
+    p.segs = segs; p.nseg = nseg; p.entries = entries; p.coef = coef; p.dw = dw; p.dqp = dqp;
+    p.part = part; p.status = status; p.L = L; p.NcAll = NcAll; p.H = H; p.Hkv = Hkv;
+    p.topk = topk; p.S = S; p.scale = scale;
+    e = cudaFuncSetAttribute(bwd_key_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BT_SMEM);
+    if (e != cudaSuccess) return e;
+    bwd_key_tc_kernel<<<(unsigned)max_seg, kBtThreads, BT_SMEM, st>>>(mq, mo, mk, mv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (lm_bf16)
+        bwd_rowfin_kernel<__nv_bfloat16><<<rblocks, 256, 0, st>>>(
+            (const __nv_bfloat16 *)lm, idx, dw, dqp, rows, H, Hkv, L, S, Nc, topk, own_chunk, scale,
+            coef, dQ);
+    else
+        bwd_rowfin_kernel<float><<<rblocks, 256, 0, st>>>(
+            (const float *)lm, idx, dw, dqp, rows, H, Hkv, L, S, Nc, topk, own_chunk, scale, coef,
+            dQ);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_dl_kernel<<<(unsigned)max_seg, BT_D, 0, st>>>((const __nv_bfloat16 *)Q, coef, entries, segs,
+                                                     nseg, H, Hkv, L, NcAll, topk, scale, part);
+    return cudaGetLastError();
+}
+
+}  // namespace hsa

@@ -286,11 +286,14 @@ __host__ __device__ constexpr size_t decode_zero_head(int64_t B, int64_t Hkv) {
 
 // Prefill backward (backward.cu): workspace layout and arguments.
 struct BwdLayout {
+    bool tc;                 // the tensor-core key pass (backward_tc.cu)
     int64_t BG, Nc, NcAll, TB, NTB, E, max_seg;
     size_t lm_off, coef_off, cnt_off, cnt_bytes, entries_off, segs_off, nseg_off, cseg_off,
-        part_off, total;
+        part_off, dw_off, dqp_off, total;
 };
-BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, bool dhsa);
+BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, bool dhsa,
+                     bool tc);
+bool backward_tc_supported(bool bf16, int G, int d);
 struct BwdArgs {
     const void *Q, *K, *V, *dO, *lm;
     int lm_bf16, bf16, dhsa;

@@ -184,10 +184,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major,
+                                                      bool a_mn_major = false) {
     return (1u << 4)                               // D format fp32
            | (1u << 7)                             // A format bf16
            | (1u << 10)                            // B format bf16
+           | ((a_mn_major ? 1u : 0u) << 15)        // A major-ness
            | ((b_mn_major ? 1u : 0u) << 16)        // B major-ness
            | ((uint32_t)(N >> 3) << 17)            // N / 8
            | ((uint32_t)(M >> 4) << 24);           // M / 16

@@ -75,12 +75,13 @@ enum {
     HSA_K_DECODE_ATTEND = 1u << 10,       /* decode attend + fusion (or a shard's fusion state) */
     HSA_K_DECODE_CP_MERGE = 1u << 11,     /* global top-K over the shards' candidates */
     HSA_K_DECODE_CP_COMBINE = 1u << 12,   /* O from the shards' fusion states */
-    HSA_K_BACKWARD = 1u << 13             /* prefill gradients (hsa_prefill_backward) */
+    HSA_K_BACKWARD = 1u << 13,            /* prefill gradients (hsa_prefill_backward) */
+    HSA_K_BACKWARD_TC = 1u << 14          /* ... with the tensor-core key pass */
 };
 
 /* Path overrides (hsa_set_path_overrides). */
 enum {
-    HSA_PATH_SIMT_PREFILL = 1,            /* prefill on CUDA cores even where tensor cores apply */
+    HSA_PATH_SIMT_PREFILL = 1,            /* prefill (and its backward) on CUDA cores even where tensor cores apply */
     HSA_PATH_SIMT_SELECT = 2,             /* selection on CUDA cores even where tensor cores apply */
     HSA_PATH_MULTI_TILE_SELECT = 4        /* the multi-tile tensor-core selection at any length */
 };
@@ -253,10 +254,14 @@ hsa_status_t hsa_prefill_varlen(const void *Q, const void *K, const void *V, hsa
  *   dlm      [B, Hkv, L/S, d]   fp32, written; required when lm is given,
  *                               ignored (may be NULL) in DHSA mode
  * Gradients accumulate in fp32 in a fixed order: the results are
- * bit-reproducible run to run.  CUDA cores throughout: a row pass (dQ and the
- * fusion coefficients), a stable sort of the selection by chunk, a per-chunk
- * key pass (dK, dV, dlm partials over segments of at most 1024 query rows)
- * and an ordered reduction.  Supports L < 2^26 and B*Hkv*L*topk < 2^31
+ * bit-reproducible run to run.  Two paths: bf16 inputs with G = 8 and d = 128
+ * run the key pass on the tensor cores (per chunk tile S = Q.K^T, U = dO.V^T,
+ * then dV^T += dO^T.(w P), dK^T += Q^T.dS and the dQ partial dS.K, with P and
+ * dS rounded to bf16 as the forward rounds P: ~2^-9 relative per term);
+ * every other shape (or HSA_PATH_SIMT_PREFILL) runs on CUDA cores in fp32: a
+ * row pass (dQ and the fusion coefficients) and a key pass.  Both sort the
+ * selection by chunk (stable), cut it into segments of at most 1024 query
+ * rows and add the segments' partials in order.  Supports L < 2^26 and B*Hkv*L*topk < 2^31
  * (else HSA_ERR_UNSUPPORTED); workspace from
  * hsa_prefill_backward_workspace_size (dhsa = 1 when lm will be NULL), no
  * zero-fill needed.  All buffers 16-byte aligned.
