@@ -443,7 +443,8 @@ def bench_prefill(args, name, dev, peaks, rank, dist, steps, warmup, keep_inputs
 def bench_backward(args, name, dev, peaks, rank, dist, steps, warmup):
     """Time hsa_prefill_backward on one workload (the forward's selection held
     fixed, computed once outside the timed region; L2 flushed between calls).
-    CUDA cores end to end, so the roofline is the FP32 CUDA-core peak."""
+    The roofline is the bf16 tensor peak when the key pass ran on the tensor
+    cores, else the FP32 CUDA-core peak."""
     import torch
 
     import hierarchical_chunk_sparse_landmark_b200 as hsa
@@ -493,7 +494,9 @@ def bench_backward(args, name, dev, peaks, rank, dist, steps, warmup):
     ms = [e[0].elapsed_time(e[1]) for e in ev]
     flops = backward_flops(wl)
     units, tmax = aggregate(dist, flops * steps / 1e12, sum(ms) / 1e3, dev)
-    peak = fp32_simt_peak_tflops(peaks)
+    tc_path = bool(hsa.last_call_kernels() & 16384)          # HSA_K_BACKWARD_TC
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) if tc_path \
+        else fp32_simt_peak_tflops(peaks)
     ach = flops / (statistics.mean(ms) / 1e3) / 1e12
     res = {"workload": wl.name, "value": round(units / tmax, 4), "unit": "TFLOP/s",
            "ms_per_step": round(tmax * 1e3 / steps, 4), "steps": steps,
@@ -501,11 +504,14 @@ def bench_backward(args, name, dev, peaks, rank, dist, steps, warmup):
                       "L": wl.L, "H": wl.H, "Hkv": wl.Hkv, "d": wl.d, "S": wl.S,
                       "topk": wl.topk, "own_chunk": wl.own_chunk, "landmarks": wl.landmarks,
                       "dtype": wl.dtype},
-           "roofline": {"kernel": "bwd_row + bwd_key + sort + reduce (whole call)",
-                        "bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 1),
-                        "unit": "TFLOP/s", "frac": round(ach / peak, 5), "traffic": None,
-                        "algorithmic_flops_per_launch": flops,
-                        "peak_source": "FP32 CUDA-core peak: 148 SMs x 128 lanes x 2 flop x "
+           "roofline": {"kernel": ("weights + sort + bwd_key_tc (tcgen05) + row finish + dl + "
+                                   "reduce (whole call)") if tc_path else
+                                  "bwd_row + sort + bwd_key + reduce (whole call)",
+                        "bound": "tensor" if tc_path else "alu", "achieved": round(ach, 3),
+                        "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(ach / peak, 5),
+                        "traffic": None, "algorithmic_flops_per_launch": flops,
+                        "peak_source": (peaks["source"] + " bf16 burst") if tc_path else
+                                       "FP32 CUDA-core peak: 148 SMs x 128 lanes x 2 flop x "
                                        "%.0f MHz" % peaks.get("sm_max_mhz", 1965.0)},
            "clocks": clk.summary(), "gpu_launches": launches}
     del x, dO, dQ, dK, dV, dlm, flush

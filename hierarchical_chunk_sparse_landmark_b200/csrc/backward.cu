@@ -28,6 +28,8 @@
 //                     dl (d) of its chunk in registers -> per-segment partials
 //   bwd_reduce_kernel sums each chunk's partials in segment order into dK, dV
 //                     (every row written once) and the landmark gradient
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace hsa {
@@ -605,7 +607,7 @@ bwd_reduce_kernel(const float *__restrict__ part, const int32_t *__restrict__ ch
 cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, const void *dO,
                                const void *lm, bool lm_bf16, const int32_t *idx, int B, int H,
                                int Hkv, int64_t L, int S, int64_t Nc, int64_t NcAll, int topk,
-                               int own_chunk, float scale, float2 *coef, float *dw, float *dqp,
+                               int own_chunk, float scale, float2 *coef, float *dw, __half *dqp,
                                const int4 *segs, const int32_t *nseg, const int32_t *entries,
                                float *part, int64_t max_seg, unsigned *status, float *dQ,
                                int phase, cudaStream_t st);
@@ -618,8 +620,16 @@ BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, b
     p.BG = (int64_t)B * Hkv;
     p.Nc = L / S;
     p.NcAll = (L + S - 1) / S;
-    p.TB = L > 256 * 1024 ? (L + 255) / 256 : 1024;
-    p.NTB = (L + p.TB - 1) / p.TB;
+    // token blocks of the stable scatter: about 256 warps over the (b, g) pairs,
+    // at least 64 tokens each, the count matrix BG x Nc x NTB kept small for
+    // the one-block scan
+    int64_t ntb = (256 + p.BG - 1) / p.BG;
+    const int64_t max_ntb = (L + 63) / 64;
+    if (ntb > max_ntb) ntb = max_ntb;
+    if (ntb < 1) ntb = 1;
+    while (ntb > 1 && p.BG * p.Nc * ntb > 131072) ntb = (ntb + 1) / 2;
+    p.TB = (L + ntb - 1) / ntb;
+    p.NTB = p.TB > 0 ? (L + p.TB - 1) / p.TB : 1;
     p.E = kSegRows / G;
     const int64_t n_entries = p.BG * L * topk;
     p.max_seg = p.BG * p.NcAll + p.BG * p.Nc + (n_entries + p.E - 1) / p.E;
@@ -646,7 +656,7 @@ BwdLayout bwd_layout(int B, int H, int Hkv, int64_t L, int d, int S, int topk, b
         p.dw_off = off;
         off = align_up(off + sizeof(float) * (size_t)B * L * H * (topk + 1), 256);
         p.dqp_off = off;
-        off = align_up(off + sizeof(float) * (size_t)B * L * H * (topk + 1) * d, 256);
+        off = align_up(off + sizeof(__half) * (size_t)B * L * H * (topk + 1) * d, 256);
     }
     p.total = off;
     return p;
@@ -717,7 +727,7 @@ static cudaError_t launch_backward_t(const BwdArgs &a, const BwdLayout &p, cudaS
     if (p.tc) {
         e = launch_backward_tc(a.Q, a.K, a.V, a.dO, a.lm, a.lm_bf16 != 0, a.idx, a.B, a.H, a.Hkv,
                                a.L, a.S, p.Nc, p.NcAll, a.topk, a.own_chunk, a.scale, coef,
-                               (float *)(ws + p.dw_off), (float *)(ws + p.dqp_off), segs, nseg,
+                               (float *)(ws + p.dw_off), (__half *)(ws + p.dqp_off), segs, nseg,
                                entries, part, p.max_seg, status, a.dQ, 1, st);
         if (e != cudaSuccess) return e;
     } else {

@@ -28,6 +28,7 @@
 // forward), so gradients carry ~2^-9 relative rounding per term.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -40,17 +41,21 @@ namespace {
 constexpr int kBtThreads = 128;
 constexpr long long kBtWait = 4000000000LL;       // SM cycles (about 2 s)
 constexpr int BT_D = 128, BT_G = 8, BT_EPT = 16;  // d, heads per entry, entries per tile
-// shared memory, offsets from a 1024-byte aligned base
-constexpr int OFF_Q = 0;                   // [16 entries][2 halves of d][8 rows][128 B]
-constexpr int OFF_DO = OFF_Q + 32768;      // same layout
-constexpr int OFF_K = OFF_DO + 32768;      // [2 halves][64 keys][128 B]
+// shared memory, offsets from a 1024-byte aligned base: two buffers of the
+// tile's Q and dO rows, so the next tile's rows load during this tile's work
+constexpr int QBUF = 32768;                // [16 entries][2 halves of d][8 rows][128 B]
+constexpr int OFF_Q = 0;                   // Q[2]
+constexpr int OFF_DO = OFF_Q + 2 * QBUF;   // dO[2]
+constexpr int OFF_K = OFF_DO + 2 * QBUF;   // [2 halves][64 keys][128 B]
 constexpr int OFF_V = OFF_K + 16384;
 constexpr int OFF_DS = OFF_V + 16384;      // [128 rows][64 keys] bf16, 128B-swizzled
 constexpr int OFF_WP = OFF_DS + 16384;
-constexpr int OFF_BAR = OFF_WP + 16384;    // two mbarriers, TMEM address, abort flag
-constexpr int BT_SMEM = 1024 + OFF_BAR + 64;
-// TMEM columns (fp32)
-constexpr uint32_t COL_S = 0, COL_U = 64, COL_DQ = 128, COL_DV = 256, COL_DK = 320;
+constexpr int OFF_BAR = OFF_WP + 16384;    // mbarriers, TMEM address, abort flag
+constexpr int BT_SMEM = 1024 + OFF_BAR + 128;
+// TMEM columns (fp32): S and U twice (the next tile's products run during this
+// tile's epilogue), the dQ partial, and the segment's dV^T and dK^T
+constexpr uint32_t COL_SU = 0;             // buffer i: S at 128 i, U at 128 i + 64
+constexpr uint32_t COL_DQ = 256, COL_DV = 384, COL_DK = 448;
 constexpr uint32_t BT_TMEM_COLS = 512;
 
 struct BtParams {
@@ -59,7 +64,7 @@ struct BtParams {
     const int32_t *entries;
     const float2 *coef;      // [B*L*H][topk]: .x = w (written by bwd_coefw_kernel)
     float *dw;               // [B*L*H][topk+1]: dw of every (row, slot); slot topk = own
-    float *dqp;              // [B*L*Hkv][topk+1][G][D]: dQ partial rows
+    __half *dqp;             // [B*L*Hkv][topk+1][G][D]: dQ partial rows (fp16)
     float *part;             // per segment: dK [64][D], dV [64][D], dl [D]
     unsigned *status;
     int64_t L, NcAll;
@@ -86,6 +91,13 @@ __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
 
 }  // namespace
 
+// A tile's row of this thread: entry e = tid / 8 of the tile, head h = tid % 8.
+struct BtRow {
+    int64_t t;
+    int slot;
+    bool valid;
+};
+
 __global__ void __launch_bounds__(kBtThreads, 1)
 bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -95,8 +107,9 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (sidx >= *p.nseg) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t *tma_bar = (uint64_t *)(sm + OFF_BAR), *mma_bar = tma_bar + 1;
-    uint32_t *s_tmem = (uint32_t *)(mma_bar + 1);
+    uint64_t *bars = (uint64_t *)(sm + OFF_BAR);
+    uint64_t *kv_bar = bars, *tma_bar = bars + 1, *su_bar = bars + 3, *o_bar = bars + 5;
+    uint32_t *s_tmem = (uint32_t *)(bars + 6);
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
     const int tid = threadIdx.x, warp = tid >> 5;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -111,10 +124,30 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int64_t first = c * p.S;
     const int nkc = (int)(L - first < p.S ? L - first : p.S);
     const int H = p.H, topk = p.topk;
+    const int e = tid >> 3, h = tid & 7;
+    const int n_units = own ? nkc : sg.z;          // tokens (own) or entries of the segment
+    const int ntiles = (n_units + BT_EPT - 1) / BT_EPT;
+    auto row_of = [&](int ti) -> BtRow {
+        BtRow r;
+        const int u = ti * BT_EPT + e;
+        r.valid = u < n_units;
+        r.t = -1;
+        r.slot = topk;
+        if (r.valid) {
+            if (own) {
+                r.t = first + u;
+            } else {
+                const int32_t code = p.entries[sg.y + u];
+                r.t = code >> 5;
+                r.slot = code & 31;
+            }
+        }
+        return r;
+    };
 
     // rows of entries a tile does not fill are read by the transposed
     // products (times zero): they must hold finite values
-    for (int i = tid; i < 65536 / 16; i += kBtThreads)
+    for (int i = tid; i < 4 * QBUF / 16; i += kBtThreads)
         reinterpret_cast<uint4 *>(sm + OFF_Q)[i] = make_uint4(0u, 0u, 0u, 0u);
     tc::fence_proxy_async_smem();
     if (warp == 0) {
@@ -122,8 +155,7 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(tma_bar, 1);
-        tc::mbar_init(mma_bar, 1);
+        for (int i = 0; i < 6; ++i) tc::mbar_init(&bars[i], 1);
         *s_abort = 0;
         tc::fence_barrier_init();
     }
@@ -131,111 +163,113 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    uint32_t ptma = 0, pmma = 0;
+    uint32_t ptma[2] = {0u, 0u}, psu[2] = {0u, 0u}, po = 0u;
 
-    // K and V of the chunk, once per segment
-    const int krow = (int)(bg * L + first);
-    if (tid == 0) {
-        tc::mbar_expect_tx(tma_bar, 2u * 16384u);
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-            tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, tma_bar, kb * 64, krow);
-            tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, tma_bar, kb * 64, krow);
+    // Q / dO rows of tile ti into buffer ti % 2 (one 3-D box per entry: its 8
+    // head rows, both halves of d); the caller has made the buffer free
+    auto load_rows = [&](int ti, const BtRow &r) {
+        const int buf = ti & 1;
+        const int nvalid = n_units - ti * BT_EPT < BT_EPT ? n_units - ti * BT_EPT : BT_EPT;
+        if (tid == 0) tc::mbar_expect_tx(&tma_bar[buf], (uint32_t)nvalid * 2u * 2048u);
+        __syncthreads();
+        if (r.valid && h == 0) {
+            const int qrow = (int)((b * L + r.t) * H + (int64_t)g * G);
+            tc::tma_load_3d(sm + OFF_Q + buf * QBUF + e * 2048, &tmQ, &tma_bar[buf], 0, qrow, 0);
+            tc::tma_load_3d(sm + OFF_DO + buf * QBUF + e * 2048, &tmO, &tma_bar[buf], 0, qrow, 0);
         }
-    }
-    // every wait's outcome is made block-uniform, so that all threads leave
-    // the tile loop together on a timeout
-    bool ok = __syncthreads_and(bt_wait(tma_bar, ptma, s_abort)) != 0;
-    ptma ^= 1u;
-
+    };
     // descriptors (bytes >> 4 in the start field; a K step moves the start)
     const uint32_t IDESC_SU = tc::idesc_bf16_f32(128, 64, false, false);
     const uint32_t IDESC_T = tc::idesc_bf16_f32(128, 64, true, true);     // M = d, N = keys
     const uint32_t IDESC_DQ = tc::idesc_bf16_f32(128, D, true, false);    // B = K, MN-major
-    const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q), 16, 2048);     // rows x d
-    const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO), 16, 2048);
     const uint64_t bK = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);     // keys x d
     const uint64_t bV = tc::sdesc_sw128(tc::smem_u32(sm + OFF_V), 16, 1024);
-    const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q), 1024, 2048);   // (d, rows)
-    const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO), 1024, 2048);
     const uint64_t bDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16384, 1024);  // (keys, rows)
     const uint64_t bWP = tc::sdesc_sw128(tc::smem_u32(sm + OFF_WP), 16384, 1024);
     const uint64_t aDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16, 1024);     // rows x keys
     const uint64_t bKt = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 8192, 1024);    // (d, keys)
-
-    const int e = tid >> 3, h = tid & 7;          // this thread's row: entry e, head h
-    const int n_units = own ? nkc : sg.z;          // tokens (own) or entries of the segment
-    const int ntiles = (n_units + BT_EPT - 1) / BT_EPT;
-    for (int ti = 0; ti < ntiles && ok; ++ti) {
-        const int u = ti * BT_EPT + e;
-        const bool valid = u < n_units;
-        int64_t t = -1;
-        int slot = topk;
-        if (valid) {
-            if (own) {
-                t = first + u;
-            } else {
-                const int32_t code = p.entries[sg.y + u];
-                t = code >> 5;
-                slot = code & 31;
+    // S = Q.K^T and U = dO.V^T of tile ti (thread 0)
+    auto issue_su = [&](int ti) {
+        const int buf = ti & 1;
+        const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 16, 2048);
+        const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 16, 2048);
+        const uint32_t ds = tmem + COL_SU + 128u * (uint32_t)buf;
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (kb | kk) ? 1u : 0u;
+                tc::mma_bf16(ds, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                             bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                tc::mma_bf16(ds + 64, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                             bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
             }
-        }
-        const int nvalid = n_units - ti * BT_EPT < BT_EPT ? n_units - ti * BT_EPT : BT_EPT;
-        if (tid == 0) tc::mbar_expect_tx(tma_bar, (uint32_t)nvalid * 2u * 2048u);
-        __syncthreads();
-        if (valid && h == 0) {        // one 3-D box per entry: its 8 head rows, both halves
-            const int qrow = (int)((b * L + t) * H + (int64_t)g * G);
-            tc::tma_load_3d(sm + OFF_Q + e * 2048, &tmQ, tma_bar, 0, qrow, 0);
-            tc::tma_load_3d(sm + OFF_DO + e * 2048, &tmO, tma_bar, 0, qrow, 0);
-        }
-        if (!__syncthreads_and(bt_wait(tma_bar, ptma, s_abort))) { ok = false; break; }
-        ptma ^= 1u;
-        // S = Q.K^T and U = dO.V^T
-        if (tid == 0) {
-            tc::fence_after_sync();
+        tc::mma_commit(&su_bar[buf]);
+    };
+
+    // K and V of the chunk (once per segment) and the first tile's rows
+    const int krow = (int)(bg * L + first);
+    if (tid == 0) {
+        tc::mbar_expect_tx(kv_bar, 2u * 16384u);
 #pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t acc = (kb | kk) ? 1u : 0u;
-                    tc::mma_bf16(tmem + COL_S, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
-                                 bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
-                    tc::mma_bf16(tmem + COL_U, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
-                                 bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
-                }
-            tc::mma_commit(mma_bar);
+        for (int kb = 0; kb < 2; ++kb) {
+            tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, kv_bar, kb * 64, krow);
+            tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, kv_bar, kb * 64, krow);
         }
-        if (!__syncthreads_and(bt_wait(mma_bar, pmma, s_abort))) { ok = false; break; }
-        pmma ^= 1u;
+    }
+    BtRow cur = row_of(0);
+    bool ok = true;
+    if (ntiles > 0) {
+        load_rows(0, cur);
+        // every wait's outcome is made block-uniform, so that all threads
+        // leave the tile loop together on a timeout
+        ok = __syncthreads_and(bt_wait(kv_bar, 0u, s_abort) && bt_wait(&tma_bar[0], 0u, s_abort)) != 0;
+        ptma[0] ^= 1u;
+        if (ok && tid == 0) issue_su(0);
+    }
+    for (int ti = 0; ti < ntiles && ok; ++ti) {
+        const int buf = ti & 1, nb = buf ^ 1;
+        const bool more = ti + 1 < ntiles;
+        const BtRow nxt = more ? row_of(ti + 1) : cur;
+        if (more) load_rows(ti + 1, nxt);        // buffer nb: tile ti - 1 is done with it
+        const bool valid = cur.valid;
+        const int64_t t = cur.t;
+        const int slot = cur.slot;
+        const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
+        const float w = !valid ? 0.f : own ? 1.f : p.coef[hrow * topk + slot].x;   // before the wait
+        if (!__syncthreads_and(bt_wait(&su_bar[buf], psu[buf], s_abort))) { ok = false; break; }
+        psu[buf] ^= 1u;
         tc::fence_after_sync();
         // this row's chunk softmax, dw, dS and w p
         float s[64], uu[64];
         {
             float tmp[32];
-            tc::tmem_ld32(tmem + lane_off + COL_S, tmp);
+            const uint32_t ts = tmem + lane_off + COL_SU + 128u * (uint32_t)buf;
+            tc::tmem_ld32(ts, tmp);
 #pragma unroll
             for (int j = 0; j < 32; ++j) s[j] = tmp[j];
-            tc::tmem_ld32(tmem + lane_off + COL_S + 32, tmp);
+            tc::tmem_ld32(ts + 32, tmp);
 #pragma unroll
             for (int j = 0; j < 32; ++j) s[32 + j] = tmp[j];
-            tc::tmem_ld32(tmem + lane_off + COL_U, tmp);
+            tc::tmem_ld32(ts + 64, tmp);
 #pragma unroll
             for (int j = 0; j < 32; ++j) uu[j] = tmp[j];
-            tc::tmem_ld32(tmem + lane_off + COL_U + 32, tmp);
+            tc::tmem_ld32(ts + 96, tmp);
 #pragma unroll
             for (int j = 0; j < 32; ++j) uu[32 + j] = tmp[j];
             tc::tmem_wait_ld();
         }
         const int nk = own ? (valid ? (int)(t - first) + 1 : 64) : 64;
-        const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
-        const float w = !valid ? 0.f : own ? 1.f : p.coef[hrow * topk + slot].x;
         float mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 64; ++j) mx = j < nk ? fmaxf(mx, s[j]) : mx;
+        // exp(scale (s - max)) as 2^(scale log2(e) (s - max)) on the MUFU unit
+        const float sl2 = p.scale * 1.4426950408889634f, ml2 = -sl2 * mx;
         float z = 0.f, zu = 0.f;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-            const float ej = j < nk ? expf(p.scale * (s[j] - mx)) : 0.f;
+            const float ej = j < nk ? tc::ex2_approx(fmaf(s[j], sl2, ml2)) : 0.f;
             s[j] = ej;
             z += ej;
             zu = fmaf(ej, uu[j], zu);
@@ -263,6 +297,8 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         // dV^T += dO^T . wP, dK^T += Q^T . dS (over the tile's 128 rows), dQp = dS . K
         if (tid == 0) {
             tc::fence_after_sync();
+            const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 1024, 2048);
+            const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 1024, 2048);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t acc = (ti > 0 || ks > 0) ? 1u : 0u;
@@ -275,28 +311,43 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + COL_DQ, aDS + (uint64_t)((kk * 32) >> 4),
                              bKt + (uint64_t)((kk * 2048) >> 4), IDESC_DQ, kk > 0 ? 1u : 0u);
-            tc::mma_commit(mma_bar);
+            tc::mma_commit(o_bar);
         }
-        if (!__syncthreads_and(bt_wait(mma_bar, pmma, s_abort))) { ok = false; break; }
-        pmma ^= 1u;
+        // the next tile's S and U run during this tile's epilogue
+        if (more) {
+            if (!__syncthreads_and(bt_wait(&tma_bar[nb], ptma[nb], s_abort))) { ok = false; break; }
+            ptma[nb] ^= 1u;
+            if (tid == 0) issue_su(ti + 1);
+        }
+        if (!__syncthreads_and(bt_wait(o_bar, po, s_abort))) { ok = false; break; }
+        po ^= 1u;
         tc::fence_after_sync();
-        // this row's dQ partial
-        float *dst = valid ? p.dqp + ((((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h) * (int64_t)D
-                           : nullptr;
+        // this row's dQ partial (fp16: 2^-11 relative, below the bf16 rounding
+        // of dS it already carries)
+        __half *dst = valid ? p.dqp + ((((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h) * (int64_t)D
+                            : nullptr;
 #pragma unroll 1
         for (int cb = 0; cb < D / 32; ++cb) {
             float v[32];
             tc::tmem_ld32(tmem + lane_off + COL_DQ + cb * 32, v);
             tc::tmem_wait_ld();
             if (valid) {
-                float4 *d4 = reinterpret_cast<float4 *>(dst + cb * 32);
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + cb * 32);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    __half2 h0 = __floats2half2_rn(v[8 * i], v[8 * i + 1]);
+                    __half2 h1 = __floats2half2_rn(v[8 * i + 2], v[8 * i + 3]);
+                    __half2 h2 = __floats2half2_rn(v[8 * i + 4], v[8 * i + 5]);
+                    __half2 h3 = __floats2half2_rn(v[8 * i + 6], v[8 * i + 7]);
+                    d4[i] = make_uint4(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1),
+                                       *reinterpret_cast<uint32_t *>(&h2), *reinterpret_cast<uint32_t *>(&h3));
+                }
             }
         }
         tc::fence_before_sync();
-        __syncthreads();          // TMEM dQ and the Q / dO tiles are free for the next tile
+        __syncthreads();          // TMEM dQ and the dS / wP tiles are free for the next tile
         tc::fence_after_sync();
+        cur = nxt;
     }
     // the segment's dK and dV partials (thread = element of d), dl is written by bwd_dl_kernel
     float *pk = p.part + sidx * (int64_t)(129 * D);
@@ -328,14 +379,15 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
 // ---------------------------------------------------------------- CUDA-core companions
 // Fusion weights w = softmax over the valid slots of scale q.l (one warp per
-// query row (t, h), lane k keeps slot k), written to coef[.].x.
+// query row (t, h), lane k keeps slot k), written to coef[.].x.  A row's slot
+// indices come in one load and all its landmark rows' loads go out together.
 template <typename TL>
 __global__ void __launch_bounds__(256)
 bwd_coefw_kernel(const __nv_bfloat16 *__restrict__ Q, const TL *__restrict__ lm,
                  const int32_t *__restrict__ idx, int64_t rows, int H, int Hkv, int64_t L, int S,
                  int64_t Nc, int topk, float scale, float2 *__restrict__ coef,
                  unsigned *__restrict__ status) {
-    constexpr int D = BT_D, R = D / 32;
+    constexpr int D = BT_D, R = D / 32, KMAX = 32;
     const int lane = threadIdx.x & 31;
     const int64_t hrow = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (hrow >= rows) return;
@@ -347,22 +399,23 @@ bwd_coefw_kernel(const __nv_bfloat16 *__restrict__ Q, const TL *__restrict__ lm,
     float qv[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) qv[r] = __bfloat162float(Q[hrow * D + lane + 32 * r]);
-    const int32_t *ip = idx + (bt * Hkv + g) * topk;
+    const int32_t ci_l = lane < topk ? idx[(bt * Hkv + g) * topk + lane] : -1;
+    const bool vk = ci_l >= 0 && (int64_t)ci_l < Nc && (int64_t)ci_l < t / S;
+    if (lane < topk && ci_l >= 0 && !vk && h % G == 0) atomicOr(status, kFlagBadIdx);
+    const unsigned vmask = __ballot_sync(0xffffffffu, vk);
     float zk = -INFINITY;
-    bool vk = false;
-    for (int k = 0; k < topk; ++k) {
-        const int32_t ci = ip[k];
-        const bool ok = ci >= 0 && (int64_t)ci < Nc && (int64_t)ci < t / S;
-        if (!ok) {
-            if (ci >= 0 && lane == 0 && h % G == 0) atomicOr(status, kFlagBadIdx);
-            continue;
-        }
+#pragma unroll 4
+    for (int k = 0; k < KMAX; ++k) {
+        if (k >= topk) break;
+        if (!((vmask >> k) & 1u)) continue;
+        const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
+        const TL *lr = lm + (bg * Nc + ci) * D + lane;
         float a = 0.f;
 #pragma unroll
-        for (int r = 0; r < R; ++r) a = fmaf(qv[r], to_f32(lm[(bg * Nc + ci) * D + lane + 32 * r]), a);
+        for (int r = 0; r < R; ++r) a = fmaf(qv[r], to_f32(lr[32 * r]), a);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == k) { zk = scale * a; vk = true; }
+        if (lane == k) zk = scale * a;
     }
     float m = vk ? zk : -INFINITY;
 #pragma unroll
@@ -380,7 +433,7 @@ bwd_coefw_kernel(const __nv_bfloat16 *__restrict__ Q, const TL *__restrict__ lm,
 template <typename TL>
 __global__ void __launch_bounds__(256)
 bwd_rowfin_kernel(const TL *__restrict__ lm, const int32_t *__restrict__ idx,
-                  const float *__restrict__ dw, const float *__restrict__ dqp, int64_t rows, int H,
+                  const float *__restrict__ dw, const __half *__restrict__ dqp, int64_t rows, int H,
                   int Hkv, int64_t L, int S, int64_t Nc, int topk, int own_chunk, float scale,
                   float2 *__restrict__ coef, float *__restrict__ dQ) {
     constexpr int D = BT_D, R = D / 32;
@@ -405,32 +458,35 @@ bwd_rowfin_kernel(const TL *__restrict__ lm, const int32_t *__restrict__ idx,
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    const float *qp = dqp + ((bt * Hkv + g) * (topk + 1)) * (int64_t)(G * D) + hh * D;
+    const __half *qp = dqp + ((bt * Hkv + g) * (topk + 1)) * (int64_t)(G * D) + hh * D;
     for (int k = 0; k < topk; ++k) {
         if (!__shfl_sync(0xffffffffu, vk ? 1 : 0, k)) continue;
         const float dz = scale * __shfl_sync(0xffffffffu, dzk, k);
         const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
 #pragma unroll
         for (int r = 0; r < R; ++r)
-            acc[r] += qp[(int64_t)k * G * D + lane + 32 * r] +
+            acc[r] += __half2float(qp[(int64_t)k * G * D + lane + 32 * r]) +
                       dz * to_f32(lm[(bg * Nc + ci) * D + lane + 32 * r]);
     }
     if (own_chunk) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[r] += qp[(int64_t)topk * G * D + lane + 32 * r];
+        for (int r = 0; r < R; ++r) acc[r] += __half2float(qp[(int64_t)topk * G * D + lane + 32 * r]);
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) dQ[hrow * D + lane + 32 * r] = acc[r];
 }
 
-// Landmark-gradient partial of each entry segment, dl = scale sum_rows dz q
-// (thread = element of d); own-chunk segments carry none.
-__global__ void __launch_bounds__(BT_D)
+// Landmark-gradient partial of each entry segment, dl = scale sum_rows dz q:
+// four groups of D threads (thread = element of d) take every fourth entry,
+// then add their sums in group order; own-chunk segments carry none.
+constexpr int kDlGroups = 4;
+__global__ void __launch_bounds__(BT_D * kDlGroups)
 bwd_dl_kernel(const __nv_bfloat16 *__restrict__ Q, const float2 *__restrict__ coef,
               const int32_t *__restrict__ entries, const int4 *__restrict__ segs,
               const int32_t *__restrict__ nseg_p, int H, int Hkv, int64_t L, int64_t NcAll,
               int topk, float scale, float *__restrict__ part) {
     constexpr int D = BT_D;
+    __shared__ float red[kDlGroups][D];
     const int64_t sidx = blockIdx.x;
     if (sidx >= *nseg_p) return;
     const int4 sg = segs[sidx];
@@ -438,20 +494,32 @@ bwd_dl_kernel(const __nv_bfloat16 *__restrict__ Q, const float2 *__restrict__ co
     const int64_t b = bg / Hkv;
     const int g = (int)(bg % Hkv);
     const int G = H / Hkv;
-    const int d = threadIdx.x;
+    const int d = threadIdx.x % D, grp = threadIdx.x / D;
     float acc = 0.f;
     if (!sg.w) {
-        for (int u = 0; u < sg.z; ++u) {
+        for (int u = grp; u < sg.z; u += kDlGroups) {
             const int32_t code = entries[sg.y + u];
             const int64_t t = code >> 5;
             const int slot = code & 31;
             const int64_t r0 = (b * L + t) * H + (int64_t)g * G;
-#pragma unroll 8
-            for (int hh = 0; hh < G; ++hh)
-                acc = fmaf(coef[(r0 + hh) * topk + slot].y, __bfloat162float(Q[(r0 + hh) * D + d]), acc);
+            float dz[BT_G], qv[BT_G];
+#pragma unroll
+            for (int hh = 0; hh < BT_G; ++hh) {
+                dz[hh] = coef[(r0 + hh) * topk + slot].y;
+                qv[hh] = __bfloat162float(Q[(r0 + hh) * D + d]);
+            }
+#pragma unroll
+            for (int hh = 0; hh < BT_G; ++hh) acc = fmaf(dz[hh], qv[hh], acc);
         }
     }
-    part[sidx * (int64_t)(129 * D) + 128 * D + d] = scale * acc;
+    red[grp][d] = acc;
+    __syncthreads();
+    if (grp == 0) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kDlGroups; ++i) s += red[i][d];
+        part[sidx * (int64_t)(129 * D) + 128 * D + d] = scale * s;
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -462,7 +530,7 @@ bool backward_tc_supported(bool bf16, int G, int d) {
 cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, const void *dO,
                                const void *lm, bool lm_bf16, const int32_t *idx, int B, int H,
                                int Hkv, int64_t L, int S, int64_t Nc, int64_t NcAll, int topk,
-                               int own_chunk, float scale, float2 *coef, float *dw, float *dqp,
+                               int own_chunk, float scale, float2 *coef, float *dw, __half *dqp,
                                const int4 *segs, const int32_t *nseg, const int32_t *entries,
                                float *part, int64_t max_seg, unsigned *status, float *dQ,
                                int phase, cudaStream_t st) {
@@ -504,7 +572,7 @@ cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, cons
             (const float *)lm, idx, dw, dqp, rows, H, Hkv, L, S, Nc, topk, own_chunk, scale, coef,
             dQ);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dl_kernel<<<(unsigned)max_seg, BT_D, 0, st>>>((const __nv_bfloat16 *)Q, coef, entries, segs,
+    bwd_dl_kernel<<<(unsigned)max_seg, BT_D * kDlGroups, 0, st>>>((const __nv_bfloat16 *)Q, coef, entries, segs,
                                                      nseg, H, Hkv, L, NcAll, topk, scale, part);
     return cudaGetLastError();
 }
