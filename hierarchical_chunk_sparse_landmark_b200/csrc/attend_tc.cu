@@ -317,6 +317,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             decode_tile(p, d, tl);
             return (!tl.own && lane < tl.n) ? __ldg(p.entries + tl.first + lane) : 0;
         };
+        // a window's query rows are re-read by every tile of their entries: keep
+        // them in L2 ahead of the chunk outputs streaming out (those go evict-first)
+        uint64_t pol_q;
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_q));
         int4 d_cur = load_desc(0), d_nxt = load_desc(1);
         int32_t code_cur = load_code(d_cur);
         for (int64_t u = 0; u < my_u; ++u) {
@@ -359,12 +363,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (lane < d0.n) {
                 const int qrow = (int)((bq * L + (int64_t)(c0 >> 5)) * H + (int64_t)gq * G);
                 if (p.q3d) {
-                    tc::tma_load_3d(sQ(q) + lane * (C::KB * G * 128), &tmQ, &qk_full[q], 0, qrow, 0);
+                    tc::tma_load_3d_hint(sQ(q) + lane * (C::KB * G * 128), &tmQ, &qk_full[q], 0, qrow, 0,
+                                         pol_q);
                 } else {
 #pragma unroll
                     for (int kb = 0; kb < C::KB; ++kb)
-                        tc::tma_load_2d(sQ(q) + kb * (128 * 128) + lane * G * 128, &tmQ, &qk_full[q],
-                                        kb * 64, qrow);
+                        tc::tma_load_2d_hint(sQ(q) + kb * (128 * 128) + lane * G * 128, &tmQ, &qk_full[q],
+                                             kb * 64, qrow, pol_q);
                 }
             }
 
