@@ -926,6 +926,8 @@ def main(argv=None):
                          "single-GPU prefill; train_prefill_bf16; tiny_prefill_f32)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the prefill backward on --workload and print its line")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extra", dest="extra", action="store_false",
@@ -967,7 +969,11 @@ def main(argv=None):
         dist = td
     else:
         torch.cuda.set_device(0)
-    res = run_ours(args, dist, rank, world)
+    if args.backward_only:       # diagnostic: the backward line alone (profiling commands)
+        res = bench_backward(args, args.workload, torch.device("cuda", torch.cuda.current_device()),
+                             load_peaks(), rank, dist, args.steps, args.warmup)
+    else:
+        res = run_ours(args, dist, rank, world)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if dist is not None:
