@@ -15,10 +15,11 @@
 //   dQp  = dS . K                       M = 128 rows, N = d, K = 64 keys
 //
 // The transposed products read the Q / dO / K tiles already in shared memory
-// as MN-major operands (no copy).  One block (4 warps, thread = tile row =
-// TMEM lane) per segment of a chunk's sorted entry list (at most 8 tiles) or
-// per own chunk (at most 4 tiles of 16 tokens); K and V are loaded once per
-// segment.  dw and the dQ partial rows of every (row, slot) go to global
+// as MN-major operands (no copy).  One persistent block per SM (8 warps; the
+// two threads of a tile row -- one TMEM lane -- take keys 0-31 and 32-63)
+// walks the segments of the chunks' sorted entry lists (at most 8 tiles each)
+// and the own chunks (at most 4 tiles of 16 tokens); K and V are loaded once
+// per segment.  dw and the dQ partial rows of every (row, slot) go to global
 // memory; bwd_rowfin_kernel then forms dz = w (dw - sum w dw), sums the dQ
 // partials and adds scale sum dz l; bwd_dl_kernel forms each segment's
 // landmark gradient scale sum dz q; the ordered reduction of backward.cu adds
@@ -38,7 +39,7 @@ namespace hsa {
 
 namespace {
 
-constexpr int kBtThreads = 128;
+constexpr int kBtThreads = 256;            // two threads per tile row: keys 0-31, 32-63
 constexpr long long kBtWait = 4000000000LL;       // SM cycles (about 2 s)
 constexpr int BT_D = 128, BT_G = 8, BT_EPT = 16;  // d, heads per entry, entries per tile
 // shared memory, offsets from a 1024-byte aligned base: two buffers of the
@@ -50,7 +51,10 @@ constexpr int OFF_K = OFF_DO + 2 * QBUF;   // [2 halves][64 keys][128 B]
 constexpr int OFF_V = OFF_K + 16384;
 constexpr int OFF_DS = OFF_V + 16384;      // [128 rows][64 keys] bf16, 128B-swizzled
 constexpr int OFF_WP = OFF_DS + 16384;
-constexpr int OFF_BAR = OFF_WP + 16384;    // mbarriers, TMEM address, abort flag
+constexpr int STG_ROW = 272;               // staged dQ row: 256 B + 16 (no bank conflicts)
+constexpr int OFF_RED = OFF_DS + 128 * STG_ROW;   // (dS, wP and the dQ staging overlap) then
+                                                  // [3][2 halves][128 rows] fp32: row max, sums
+constexpr int OFF_BAR = OFF_RED + 3 * 2 * 128 * 4;   // mbarriers, TMEM address, abort flag
 constexpr int BT_SMEM = 1024 + OFF_BAR + 128;
 // TMEM columns (fp32): S and U twice (the next tile's products run during this
 // tile's epilogue), the dQ partial, and the segment's dV^T and dK^T
@@ -91,7 +95,8 @@ __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
 
 }  // namespace
 
-// A tile's row of this thread: entry e = tid / 8 of the tile, head h = tid % 8.
+// A tile's row of this thread: entry e = (tid % 128) / 8 of the tile, head
+// h = tid % 8; threads tid and tid + 128 share the row (keys 0-31 and 32-63).
 struct BtRow {
     int64_t t;
     int slot;
@@ -103,8 +108,8 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const BtParams p) {
     constexpr int D = BT_D, G = BT_G;
-    const int64_t sidx = blockIdx.x;
-    if (sidx >= *p.nseg) return;
+    const int64_t nseg = *p.nseg;
+    if ((int64_t)blockIdx.x >= nseg) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t *bars = (uint64_t *)(sm + OFF_BAR);
@@ -112,38 +117,12 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     uint32_t *s_tmem = (uint32_t *)(bars + 6);
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-
-    const int4 sg = p.segs[sidx];
-    const int64_t q = sg.x;
-    const int64_t bg = q / p.NcAll, c = q % p.NcAll;
-    const int64_t b = bg / p.Hkv;
-    const int g = (int)(bg % p.Hkv);
-    const int own = sg.w;
+    const int rt = tid & 127, hf = tid >> 7;          // tile row (TMEM lane), key half
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float *red = (float *)(sm + OFF_RED);
+    const int e = rt >> 3, h = rt & 7;
     const int64_t L = p.L;
-    const int64_t first = c * p.S;
-    const int nkc = (int)(L - first < p.S ? L - first : p.S);
     const int H = p.H, topk = p.topk;
-    const int e = tid >> 3, h = tid & 7;
-    const int n_units = own ? nkc : sg.z;          // tokens (own) or entries of the segment
-    const int ntiles = (n_units + BT_EPT - 1) / BT_EPT;
-    auto row_of = [&](int ti) -> BtRow {
-        BtRow r;
-        const int u = ti * BT_EPT + e;
-        r.valid = u < n_units;
-        r.t = -1;
-        r.slot = topk;
-        if (r.valid) {
-            if (own) {
-                r.t = first + u;
-            } else {
-                const int32_t code = p.entries[sg.y + u];
-                r.t = code >> 5;
-                r.slot = code & 31;
-            }
-        }
-        return r;
-    };
 
     // rows of entries a tile does not fill are read by the transposed
     // products (times zero): they must hold finite values
@@ -163,22 +142,8 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    uint32_t ptma[2] = {0u, 0u}, psu[2] = {0u, 0u}, po = 0u;
-
-    // Q / dO rows of tile ti into buffer ti % 2 (one 3-D box per entry: its 8
-    // head rows, both halves of d); the caller has made the buffer free
-    auto load_rows = [&](int ti, const BtRow &r) {
-        const int buf = ti & 1;
-        const int nvalid = n_units - ti * BT_EPT < BT_EPT ? n_units - ti * BT_EPT : BT_EPT;
-        if (tid == 0) tc::mbar_expect_tx(&tma_bar[buf], (uint32_t)nvalid * 2u * 2048u);
-        __syncthreads();
-        if (r.valid && h == 0) {
-            const int qrow = (int)((b * L + r.t) * H + (int64_t)g * G);
-            tc::tma_load_3d(sm + OFF_Q + buf * QBUF + e * 2048, &tmQ, &tma_bar[buf], 0, qrow, 0);
-            tc::tma_load_3d(sm + OFF_DO + buf * QBUF + e * 2048, &tmO, &tma_bar[buf], 0, qrow, 0);
-        }
-    };
-    // descriptors (bytes >> 4 in the start field; a K step moves the start)
+    uint32_t pkv = 0u, ptma[2] = {0u, 0u}, psu[2] = {0u, 0u}, po = 0u;
+    // descriptors of the fixed tiles (bytes >> 4 in the start field; a K step moves the start)
     const uint32_t IDESC_SU = tc::idesc_bf16_f32(128, 64, false, false);
     const uint32_t IDESC_T = tc::idesc_bf16_f32(128, 64, true, true);     // M = d, N = keys
     const uint32_t IDESC_DQ = tc::idesc_bf16_f32(128, D, true, false);    // B = K, MN-major
@@ -188,151 +153,210 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint64_t bWP = tc::sdesc_sw128(tc::smem_u32(sm + OFF_WP), 16384, 1024);
     const uint64_t aDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16, 1024);     // rows x keys
     const uint64_t bKt = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 8192, 1024);    // (d, keys)
-    // S = Q.K^T and U = dO.V^T of tile ti (thread 0)
-    auto issue_su = [&](int ti) {
-        const int buf = ti & 1;
-        const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 16, 2048);
-        const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 16, 2048);
-        const uint32_t ds = tmem + COL_SU + 128u * (uint32_t)buf;
-        tc::fence_after_sync();
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (kb | kk) ? 1u : 0u;
-                tc::mma_bf16(ds, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
-                             bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
-                tc::mma_bf16(ds + 64, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
-                             bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
-            }
-        tc::mma_commit(&su_bar[buf]);
-    };
-
-    // K and V of the chunk (once per segment) and the first tile's rows
-    const int krow = (int)(bg * L + first);
-    if (tid == 0) {
-        tc::mbar_expect_tx(kv_bar, 2u * 16384u);
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-            tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, kv_bar, kb * 64, krow);
-            tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, kv_bar, kb * 64, krow);
-        }
-    }
-    BtRow cur = row_of(0);
     bool ok = true;
-    if (ntiles > 0) {
-        load_rows(0, cur);
-        // every wait's outcome is made block-uniform, so that all threads
-        // leave the tile loop together on a timeout
-        ok = __syncthreads_and(bt_wait(kv_bar, 0u, s_abort) && bt_wait(&tma_bar[0], 0u, s_abort)) != 0;
-        ptma[0] ^= 1u;
-        if (ok && tid == 0) issue_su(0);
-    }
-    for (int ti = 0; ti < ntiles && ok; ++ti) {
-        const int buf = ti & 1, nb = buf ^ 1;
-        const bool more = ti + 1 < ntiles;
-        const BtRow nxt = more ? row_of(ti + 1) : cur;
-        if (more) load_rows(ti + 1, nxt);        // buffer nb: tile ti - 1 is done with it
-        const bool valid = cur.valid;
-        const int64_t t = cur.t;
-        const int slot = cur.slot;
-        const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
-        const float w = !valid ? 0.f : own ? 1.f : p.coef[hrow * topk + slot].x;   // before the wait
-        if (!__syncthreads_and(bt_wait(&su_bar[buf], psu[buf], s_abort))) { ok = false; break; }
-        psu[buf] ^= 1u;
-        tc::fence_after_sync();
-        // this row's chunk softmax, dw, dS and w p
-        float s[64], uu[64];
-        {
-            float tmp[32];
-            const uint32_t ts = tmem + lane_off + COL_SU + 128u * (uint32_t)buf;
-            tc::tmem_ld32(ts, tmp);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = tmp[j];
-            tc::tmem_ld32(ts + 32, tmp);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[32 + j] = tmp[j];
-            tc::tmem_ld32(ts + 64, tmp);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) uu[j] = tmp[j];
-            tc::tmem_ld32(ts + 96, tmp);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) uu[32 + j] = tmp[j];
-            tc::tmem_wait_ld();
-        }
-        const int nk = own ? (valid ? (int)(t - first) + 1 : 64) : 64;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) mx = j < nk ? fmaxf(mx, s[j]) : mx;
-        // exp(scale (s - max)) as 2^(scale log2(e) (s - max)) on the MUFU unit
-        const float sl2 = p.scale * 1.4426950408889634f, ml2 = -sl2 * mx;
-        float z = 0.f, zu = 0.f;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-            const float ej = j < nk ? tc::ex2_approx(fmaf(s[j], sl2, ml2)) : 0.f;
-            s[j] = ej;
-            z += ej;
-            zu = fmaf(ej, uu[j], zu);
-        }
-        const float inv = 1.f / z;
-        const float dwv = zu * inv;
-        if (valid) p.dw[hrow * (topk + 1) + slot] = dwv;
-        const float fds = valid ? p.scale * w * inv : 0.f, fwp = valid ? w * inv : 0.f;
-#pragma unroll
-        for (int cch = 0; cch < 8; ++cch) {
-            uint32_t ds4[4], wp4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = cch * 8 + 2 * i;
-                ds4[i] = pack2_bf16(fds * s[j] * (uu[j] - dwv), fds * s[j + 1] * (uu[j + 1] - dwv));
-                wp4[i] = pack2_bf16(fwp * s[j], fwp * s[j + 1]);
+
+    // persistent: this block takes segments blockIdx.x, + gridDim.x, ...
+    for (int64_t sidx = blockIdx.x; sidx < nseg && ok; sidx += gridDim.x) {
+        const int4 sg = p.segs[sidx];
+        const int64_t q = sg.x;
+        const int64_t bg = q / p.NcAll, c = q % p.NcAll;
+        const int64_t b = bg / p.Hkv;
+        const int g = (int)(bg % p.Hkv);
+        const int own = sg.w;
+        const int64_t first = c * p.S;
+        const int nkc = (int)(L - first < p.S ? L - first : p.S);
+        const int n_units = own ? nkc : sg.z;      // tokens (own) or entries of the segment
+        const int ntiles = (n_units + BT_EPT - 1) / BT_EPT;
+        auto row_of = [&](int ti) -> BtRow {
+            BtRow r;
+            const int u = ti * BT_EPT + e;
+            r.valid = u < n_units;
+            r.t = -1;
+            r.slot = topk;
+            if (r.valid) {
+                if (own) {
+                    r.t = first + u;
+                } else {
+                    const int32_t code = p.entries[sg.y + u];
+                    r.t = code >> 5;
+                    r.slot = code & 31;
+                }
             }
-            const uint32_t off = tc::sw128_offset(tid, cch);
-            *reinterpret_cast<uint4 *>(sm + OFF_DS + off) = make_uint4(ds4[0], ds4[1], ds4[2], ds4[3]);
-            *reinterpret_cast<uint4 *>(sm + OFF_WP + off) = make_uint4(wp4[0], wp4[1], wp4[2], wp4[3]);
-        }
-        tc::fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        // dV^T += dO^T . wP, dK^T += Q^T . dS (over the tile's 128 rows), dQp = dS . K
-        if (tid == 0) {
+            return r;
+        };
+        // Q / dO rows of tile ti into buffer ti % 2 (one 3-D box per entry: its
+        // 8 head rows, both halves of d); the caller has made the buffer free
+        auto load_rows = [&](int ti, const BtRow &r) {
+            const int buf = ti & 1;
+            const int nvalid = n_units - ti * BT_EPT < BT_EPT ? n_units - ti * BT_EPT : BT_EPT;
+            if (tid == 0) tc::mbar_expect_tx(&tma_bar[buf], (uint32_t)nvalid * 2u * 2048u);
+            __syncthreads();
+            if (r.valid && h == 0 && hf == 0) {
+                const int qrow = (int)((b * L + r.t) * H + (int64_t)g * G);
+                tc::tma_load_3d(sm + OFF_Q + buf * QBUF + e * 2048, &tmQ, &tma_bar[buf], 0, qrow, 0);
+                tc::tma_load_3d(sm + OFF_DO + buf * QBUF + e * 2048, &tmO, &tma_bar[buf], 0, qrow, 0);
+            }
+        };
+        // S = Q.K^T and U = dO.V^T of tile ti (thread 0)
+        auto issue_su = [&](int ti) {
+            const int buf = ti & 1;
+            const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 16, 2048);
+            const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 16, 2048);
+            const uint32_t ds = tmem + COL_SU + 128u * (uint32_t)buf;
             tc::fence_after_sync();
-            const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 1024, 2048);
-            const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 1024, 2048);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t acc = (ti > 0 || ks > 0) ? 1u : 0u;
-                tc::mma_bf16(tmem + COL_DV, tO + (uint64_t)((ks * 4096) >> 4),
-                             bWP + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
-                tc::mma_bf16(tmem + COL_DK, tQ + (uint64_t)((ks * 4096) >> 4),
-                             bDS + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (kb | kk) ? 1u : 0u;
+                    tc::mma_bf16(ds, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                                 bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                    tc::mma_bf16(ds + 64, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                                 bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                }
+            tc::mma_commit(&su_bar[buf]);
+        };
+        // entry codes are read two tiles ahead and fusion weights one tile
+        // ahead, so neither load's latency sits on a tile's critical path
+        auto weight_of = [&](const BtRow &r) -> float {
+            if (!r.valid) return 0.f;
+            if (own) return 1.f;
+            return p.coef[((b * L + r.t) * H + (int64_t)g * G + h) * topk + r.slot].x;
+        };
+
+        // K and V of the chunk (the previous segment's products are done with
+        // them) and the first tile's rows
+        const int krow = (int)(bg * L + first);
+        if (tid == 0) {
+            tc::mbar_expect_tx(kv_bar, 2u * 16384u);
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+                tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, kv_bar, kb * 64, krow);
+                tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, kv_bar, kb * 64, krow);
             }
+        }
+        BtRow cur = row_of(0);
+        BtRow nxt = ntiles > 1 ? row_of(1) : cur;
+        float w_cur = weight_of(cur);
+        if (ntiles > 0) load_rows(0, cur);
+        if (ntiles > 1) load_rows(1, nxt);     // the rows of tile ti + 2 load during tile ti
+        // every wait's outcome is made block-uniform, so that all threads
+        // leave the loops together on a timeout
+        ok = __syncthreads_and(bt_wait(kv_bar, pkv, s_abort) &&
+                               (ntiles == 0 || bt_wait(&tma_bar[0], ptma[0], s_abort))) != 0;
+        pkv ^= 1u;
+        if (ntiles > 0) ptma[0] ^= 1u;
+        if (ok && ntiles > 0 && tid == 0) issue_su(0);
+        for (int ti = 0; ti < ntiles && ok; ++ti) {
+            const int buf = ti & 1, nb = buf ^ 1;
+            const bool more = ti + 1 < ntiles;
+            const BtRow nxt2 = ti + 2 < ntiles ? row_of(ti + 2) : nxt;
+            const float w_nxt = more ? weight_of(nxt) : 0.f;
+            // the dS / wP tiles double as the staging of the previous tile's dQ
+            // rows: its bulk stores must have read them before they are rewritten
+            if (hf == 0) tc::bulk_wait_read_all();
+            const bool valid = cur.valid;
+            const int64_t t = cur.t;
+            const int slot = cur.slot;
+            const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
+            const float w = w_cur;
+            if (!__syncthreads_and(bt_wait(&su_bar[buf], psu[buf], s_abort))) { ok = false; break; }
+            psu[buf] ^= 1u;
+            tc::fence_after_sync();
+            // this row's chunk softmax, dw, dS and w p over this thread's 32
+            // keys (j0 .. j0+31); the row max and the two sums are combined
+            // with the other half through shared memory
+            const int j0 = hf * 32;
+            float s[32], uu[32];
+            {
+                const uint32_t ts = tmem + lane_off + COL_SU + 128u * (uint32_t)buf + (uint32_t)j0;
+                tc::tmem_ld32(ts, s);
+                tc::tmem_ld32(ts + 64, uu);
+                tc::tmem_wait_ld();
+            }
+            const int nk = own ? (valid ? (int)(t - first) + 1 : 64) : 64;
+            float mx = -INFINITY;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + COL_DQ, aDS + (uint64_t)((kk * 32) >> 4),
-                             bKt + (uint64_t)((kk * 2048) >> 4), IDESC_DQ, kk > 0 ? 1u : 0u);
-            tc::mma_commit(o_bar);
-        }
-        // the next tile's S and U run during this tile's epilogue
-        if (more) {
-            if (!__syncthreads_and(bt_wait(&tma_bar[nb], ptma[nb], s_abort))) { ok = false; break; }
-            ptma[nb] ^= 1u;
-            if (tid == 0) issue_su(ti + 1);
-        }
-        if (!__syncthreads_and(bt_wait(o_bar, po, s_abort))) { ok = false; break; }
-        po ^= 1u;
-        tc::fence_after_sync();
-        // this row's dQ partial (fp16: 2^-11 relative, below the bf16 rounding
-        // of dS it already carries)
-        __half *dst = valid ? p.dqp + ((((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h) * (int64_t)D
-                            : nullptr;
+            for (int j = 0; j < 32; ++j) mx = j0 + j < nk ? fmaxf(mx, s[j]) : mx;
+            red[hf * 128 + rt] = mx;
+            __syncthreads();
+            mx = fmaxf(red[rt], red[128 + rt]);
+            // exp(scale (s - max)) as 2^(scale log2(e) (s - max)) on the MUFU unit
+            const float sl2 = p.scale * 1.4426950408889634f, ml2 = -sl2 * mx;
+            float z = 0.f, zu = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float ej = j0 + j < nk ? tc::ex2_approx(fmaf(s[j], sl2, ml2)) : 0.f;
+                s[j] = ej;
+                z += ej;
+                zu = fmaf(ej, uu[j], zu);
+            }
+            red[256 + hf * 128 + rt] = z;
+            red[512 + hf * 128 + rt] = zu;
+            __syncthreads();
+            z = red[256 + rt] + red[384 + rt];
+            zu = red[512 + rt] + red[640 + rt];
+            const float inv = 1.f / z;
+            const float dwv = zu * inv;
+            if (valid && hf == 0) p.dw[hrow * (topk + 1) + slot] = dwv;
+            const float fds = valid ? p.scale * w * inv : 0.f, fwp = valid ? w * inv : 0.f;
+#pragma unroll
+            for (int cq = 0; cq < 4; ++cq) {
+                uint32_t ds4[4], wp4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int j = cq * 8 + 2 * i;
+                    ds4[i] = pack2_bf16(fds * s[j] * (uu[j] - dwv), fds * s[j + 1] * (uu[j + 1] - dwv));
+                    wp4[i] = pack2_bf16(fwp * s[j], fwp * s[j + 1]);
+                }
+                const uint32_t off = tc::sw128_offset(rt, hf * 4 + cq);
+                *reinterpret_cast<uint4 *>(sm + OFF_DS + off) = make_uint4(ds4[0], ds4[1], ds4[2], ds4[3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_WP + off) = make_uint4(wp4[0], wp4[1], wp4[2], wp4[3]);
+            }
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            __syncthreads();
+            // dV^T += dO^T . wP, dK^T += Q^T . dS (over the tile's 128 rows), dQp = dS . K
+            if (tid == 0) {
+                tc::fence_after_sync();
+                const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 1024, 2048);
+                const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 1024, 2048);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t acc = (ti > 0 || ks > 0) ? 1u : 0u;
+                    tc::mma_bf16(tmem + COL_DV, tO + (uint64_t)((ks * 4096) >> 4),
+                                 bWP + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+                    tc::mma_bf16(tmem + COL_DK, tQ + (uint64_t)((ks * 4096) >> 4),
+                                 bDS + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + COL_DQ, aDS + (uint64_t)((kk * 32) >> 4),
+                                 bKt + (uint64_t)((kk * 2048) >> 4), IDESC_DQ, kk > 0 ? 1u : 0u);
+                tc::mma_commit(o_bar);
+            }
+            // the next tile's S and U run during this tile's epilogue
+            if (more) {
+                if (!__syncthreads_and(bt_wait(&tma_bar[nb], ptma[nb], s_abort))) { ok = false; break; }
+                ptma[nb] ^= 1u;
+                if (tid == 0) issue_su(ti + 1);
+            }
+            if (!__syncthreads_and(bt_wait(o_bar, po, s_abort))) { ok = false; break; }
+            po ^= 1u;
+            tc::fence_after_sync();
+            // this tile's products are done with its Q / dO buffer: the rows of
+            // tile ti + 2 load into it while the epilogue runs
+            if (ti + 2 < ntiles) load_rows(ti + 2, nxt2);
+            // this row's dQ partial (fp16: 2^-11 relative, below the bf16
+            // rounding of dS it already carries), each half 64 columns, staged
+            // over the dS / wP tiles one 256-byte row per 272 bytes
+            uint8_t *stg = sm + OFF_DS + rt * STG_ROW;
 #pragma unroll 1
-        for (int cb = 0; cb < D / 32; ++cb) {
-            float v[32];
-            tc::tmem_ld32(tmem + lane_off + COL_DQ + cb * 32, v);
-            tc::tmem_wait_ld();
-            if (valid) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + cb * 32);
+            for (int cb = hf * 2; cb < hf * 2 + 2; ++cb) {
+                float v[32];
+                tc::tmem_ld32(tmem + lane_off + COL_DQ + cb * 32, v);
+                tc::tmem_wait_ld();
+                uint4 *d4 = reinterpret_cast<uint4 *>(stg + cb * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     __half2 h0 = __floats2half2_rn(v[8 * i], v[8 * i + 1]);
@@ -343,17 +367,25 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                                        *reinterpret_cast<uint32_t *>(&h2), *reinterpret_cast<uint32_t *>(&h3));
                 }
             }
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            __syncthreads();          // TMEM dQ free for the next tile; the staging is complete
+            tc::fence_after_sync();
+            if (valid && hf == 0) {              // one bulk store per row: 256 bytes
+                __half *dst = p.dqp + ((((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h) * (int64_t)D;
+                tc::bulk_store(dst, stg, 256u);
+                tc::bulk_commit();
+            }
+            cur = nxt;
+            nxt = nxt2;
+            w_cur = w_nxt;
         }
-        tc::fence_before_sync();
-        __syncthreads();          // TMEM dQ and the dS / wP tiles are free for the next tile
-        tc::fence_after_sync();
-        cur = nxt;
-    }
-    // the segment's dK and dV partials (thread = element of d), dl is written by bwd_dl_kernel
-    float *pk = p.part + sidx * (int64_t)(129 * D);
-    if (ok) {
-#pragma unroll 1
-        for (int cb = 0; cb < 2; ++cb) {
+        if (!ok) break;
+        // the segment's dK and dV partials (thread = element of d; each half
+        // 32 keys); dl is written by bwd_dl_kernel
+        {
+            float *pk = p.part + sidx * (int64_t)(129 * D);
+            const int cb = hf;
             float vk[32], vv[32];
             tc::tmem_ld32(tmem + lane_off + COL_DK + cb * 32, vk);
             tc::tmem_ld32(tmem + lane_off + COL_DV + cb * 32, vv);
@@ -361,11 +393,16 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             const bool any = ntiles > 0;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                pk[(cb * 32 + j) * D + tid] = any ? vk[j] : 0.f;
-                pk[64 * D + (cb * 32 + j) * D + tid] = any ? vv[j] : 0.f;
+                pk[(cb * 32 + j) * D + rt] = any ? vk[j] : 0.f;
+                pk[64 * D + (cb * 32 + j) * D + rt] = any ? vv[j] : 0.f;
             }
         }
-    } else {
+        tc::fence_before_sync();
+        __syncthreads();          // TMEM dK / dV free for the next segment
+        tc::fence_after_sync();
+    }
+    if (hf == 0) tc::bulk_wait_all();      // this thread's dQ stores are complete
+    if (!ok) {
         if (tid == 0) atomicOr(p.status, kFlagTimeout);
         // let copies and MMAs that may still be in flight land before exiting
         const long long t0 = clock64();
@@ -561,7 +598,11 @@ cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, cons
     e = cudaFuncSetAttribute(bwd_key_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              BT_SMEM);
     if (e != cudaSuccess) return e;
-    bwd_key_tc_kernel<<<(unsigned)max_seg, kBtThreads, BT_SMEM, st>>>(mq, mo, mk, mv, p);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = max_seg < (int64_t)sms ? max_seg : (int64_t)sms;   // persistent
+    bwd_key_tc_kernel<<<(unsigned)grid, kBtThreads, BT_SMEM, st>>>(mq, mo, mk, mv, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (lm_bf16)
         bwd_rowfin_kernel<__nv_bfloat16><<<rblocks, 256, 0, st>>>(
