@@ -649,7 +649,15 @@ static cudaError_t launch_decode_t(const void *q, const void *lm, const void *Kc
     auto kern = decode_attend_kernel<T, TL, D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int C = topk < kAttMaxCluster ? topk : kAttMaxCluster;
+    // clusters of up to 8 blocks (one slot each) while 8 blocks per (b, g)
+    // fit in about two waves; with more (b, g) pairs, 4 blocks of two slots
+    // each place more easily and run faster (measured: batched decode
+    // 69 -> 64.5 us; a single long sequence prefers 8)
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int cmax = (int64_t)B * Hkv * kAttMaxCluster <= 2 * (int64_t)sms ? kAttMaxCluster : 4;
+    const int C = topk < cmax ? topk : cmax;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)C, (unsigned)(B * Hkv));
     cfg.blockDim = dim3(kAttThreads);

@@ -331,6 +331,17 @@ def test_decode_small(oracle_lib, dtype, d, H, Hkv, topk):
     assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
 
 
+@pytest.mark.parametrize("topk", [8, 5, 3])
+def test_decode_many_sequences_smaller_clusters(oracle_lib, topk):
+    # 40 sequences x 2 groups x 8 blocks exceed two waves: the attend kernel runs
+    # clusters of 4 blocks, each taking two slots (one when topk <= 4)
+    wl = Workload("dec", "decode", "bf16", B=40, L=64 * 120, H=16, Hkv=2, d=128, topk=topk,
+                  seed=90 + topk)
+    x = make_decode_inputs(wl, DEV)
+    rep, _ = decode_parity(oracle_lib, wl, x)
+    assert rep.ok, rep.summary() + "\n" + "\n".join(rep.failures[:10])
+
+
 def test_decode_fewer_chunks_than_topk(oracle_lib):
     wl = Workload("dec", "decode", "bf16", B=2, L=64 * 5, H=16, Hkv=2, d=128, topk=8)
     x = make_decode_inputs(wl, DEV)
