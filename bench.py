@@ -560,6 +560,7 @@ def run_ours(args, dist, rank, world):
     if args.extra:
         res["backward_train"] = bench_backward(args, "train_prefill_bf16", dev, peaks, rank, dist,
                                                max(3, args.steps // 4), 3)
+        res["backward_long"] = bench_backward(args, "long_prefill_bf16", dev, peaks, rank, dist, 3, 3)
     if args.decode:
         names = [args.decode_workload]
         if args.extra and "batched_decode_bf16" not in names:

@@ -161,3 +161,21 @@ def test_backward_tensor_core_long_chunk_lists():
     # 40 chunks, top-8, G = 8: chunk 0's entries span several segments of 8 tiles
     wl = Workload("bwd", "prefill", "bf16", B=1, L=64 * 40, H=8, Hkv=1, d=128, topk=8, seed=77)
     backward_parity(wl, lm_mode="input")
+
+
+def test_backward_long_sequence_paths_agree():
+    # 512 chunks, DHSA landmarks: long per-chunk entry lists (chunk 0 is selected by
+    # thousands of tokens) on both paths; the CUDA-core path is the fp32 reference
+    wl = Workload("bwd", "prefill", "bf16", B=1, L=32768, H=16, Hkv=2, d=128, topk=8, seed=123)
+    x = make_prefill_inputs(wl.with_(landmarks="dhsa"), DEV)
+    _, idx, _ = hsa.prefill(x["Q"], x["K"], x["V"], None, topk=8, idx_out=True)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(5)
+    dO = torch.randn(x["Q"].shape, generator=g, device=DEV).to(torch.bfloat16)
+    tc = hsa.prefill_backward(x["Q"], x["K"], x["V"], idx, dO, None)
+    assert hsa.last_call_kernels() & B.K_BACKWARD_TC
+    with hsa.path_overrides(B.PATH_SIMT_PREFILL):
+        ref = hsa.prefill_backward(x["Q"], x["K"], x["V"], idx, dO, None)
+    hsa.check()
+    for name, a, r in zip(("dQ", "dK", "dV"), tc[:3], ref[:3]):
+        _close(name, a, _f64(r), RTOL_TC)
