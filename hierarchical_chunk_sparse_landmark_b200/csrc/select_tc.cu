@@ -163,18 +163,17 @@ __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, in
 #pragma unroll
         for (int c = 0; c < 32; ++c) stage[c * 128 + r] = sc[c];
     }
+    // Branch-free trips: a key below every held one leaves the list as it is
+    // (insert_key then keeps every slot), so neither the score test nor the
+    // key test is needed, and the threshold is refreshed once at the end.
+    // (With the tests, every trip paid two divergent branches and a key-to-
+    // score conversion on its dependency chain: ~400-500 cycles a trip.)
     while (mask) {
         const int c = __ffs(mask) - 1;
         mask &= mask - 1;
-        const float sv = scale * stage[c * 128 + r];
-        if (sv >= tf) {
-            const uint64_t x = make_key(sv, c0 + c);
-            if (x > v[KP - 1]) {
-                insert_key<KP>(v, x);
-                tf = key_score(v[KP - 1]);
-            }
-        }
+        insert_key<KP>(v, make_key(scale * stage[c * 128 + r], c0 + c));
     }
+    tf = key_score(v[KP - 1]);
 }
 
 // The top-K runs in two groups of four warps (thread = token = TMEM lane),
