@@ -22,11 +22,14 @@
 //   warp 0      producer  (TMA of landmark tiles, two stages)
 //   warp 1      MMA issuer (one score tile per landmark tile, two TMEM buffers)
 //   warps 2-9   top-K     (thread = token = TMEM lane: causal mask, a sorted
-//                          register list of 64-bit keys, insertion only past
-//                          the current K-th key; two groups of four warps over
-//                          alternate 32-column blocks, lists merged at the end)
-// (warps 10-11 only help build qbar; the first two landmark tiles are requested
-// before that, so their loads overlap it.)
+//                          register list of (score, chunk) pairs, insertion
+//                          only past the current K-th score; two groups of
+//                          four warps over alternate 32-column blocks, lists
+//                          merged at the end)
+//   warps 10-11 L2 prefetch of the query rows of the block likely to start a
+//               wave later, so that its qbar loads hit L2
+// (the first two landmark tiles are requested before qbar is built, so their
+// loads overlap it.)
 // select_tc_half_kernel takes the case where every chunk fits one score tile
 // (Nc <= 128): qbar built per 64-column block of d into one buffer, two blocks
 // per SM (see the comment above it).
@@ -104,42 +107,103 @@ __device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-// Insert key x (distinct from every key held) into the sorted list v of KP
-// keys, dropping the smallest.  The KP comparisons are independent of each
-// other and every slot takes its new value from its own and its upper
-// neighbour's comparison, so the insertion is a few dependent steps, not a
-// chain through the whole list.
+// A token's running top-K: scores s[0] >= s[1] >= ... (scaled group scores)
+// and their chunk indices; empty slots hold (-inf, -1).  The order is score
+// descending, then chunk index ascending (a total order: indices are distinct).
 template <int KP>
-__device__ __forceinline__ void insert_key(uint64_t (&v)[KP], uint64_t x) {
-    bool gt[KP];
+struct TopList {
+    float s[KP];
+    int32_t i[KP];
+    __device__ __forceinline__ void clear() {
 #pragma unroll
-    for (int i = 0; i < KP; ++i) gt[i] = v[i] > x;
+        for (int k = 0; k < KP; ++k) {
+            s[k] = -INFINITY;
+            i[k] = -1;
+        }
+    }
+    // above[k]: slot k ranks above the new entry and keeps what it holds;
+    // the first other slot takes the new entry and every later one its upper
+    // neighbour's.  The KP comparisons are independent of each other, so the
+    // insertion is a few dependent steps, not a chain through the list; an
+    // entry that ranks below every held one leaves the list as it is.
+    __device__ __forceinline__ void place(const bool (&above)[KP], float xs, int32_t xi) {
 #pragma unroll
-    for (int i = KP - 1; i > 0; --i) v[i] = gt[i] ? v[i] : (gt[i - 1] ? x : v[i - 1]);
-    v[0] = gt[0] ? v[0] : x;
-}
+        for (int k = KP - 1; k > 0; --k) {
+            s[k] = above[k] ? s[k] : (above[k - 1] ? xs : s[k - 1]);
+            i[k] = above[k] ? i[k] : (above[k - 1] ? xi : i[k - 1]);
+        }
+        s[0] = above[0] ? s[0] : xs;
+        i[0] = above[0] ? i[0] : xi;
+    }
+    // Insert chunk xi whose index is above every held one (the columns of a
+    // row arrive in index order): a held entry of equal score ranks first, so
+    // a single float comparison per slot decides.
+    __device__ __forceinline__ void insert_later(float xs, int32_t xi) {
+        bool above[KP];
+#pragma unroll
+        for (int k = 0; k < KP; ++k) above[k] = s[k] >= xs;
+        place(above, xs, xi);
+    }
+    // Insert an entry of any index (merging two lists).
+    __device__ __forceinline__ void insert_any(float xs, int32_t xi) {
+        bool above[KP];
+#pragma unroll
+        for (int k = 0; k < KP; ++k) above[k] = s[k] > xs || (s[k] == xs && (uint32_t)i[k] < (uint32_t)xi);
+        place(above, xs, xi);
+    }
+};
 
 // One 32-column block of a token's scores (chunks c0 .. c0+31, of which the
-// first `lim` are visible) into its sorted list v of KP 64-bit keys (score
-// bits, ~index).  The lane first marks its candidates -- unscaled scores at or
-// above its current K-th score divided by the scale, a bound loosened by 1e-6
-// so that no column whose scaled score reaches it is missed; the exact test
-// follows -- then takes them one per loop trip from its own 32-float row of
-// `stage` (shared memory, column-major so the rows of a warp's lanes share no
-// bank): the warp runs as many trips as its busiest lane needs, instead of
-// the insertion at every column where any lane has a candidate.  Candidates
-// are taken in column order and the keys order (score, then lower index)
-// totally, so the result does not depend on the order.
+// first `lim` are visible) into its running top-K v.  The lane first marks
+// its candidates -- unscaled scores at or above its current K-th score divided
+// by the scale, a bound loosened by 1e-6 so that no column whose scaled score
+// reaches it is missed; the exact test follows -- then takes them one per
+// loop trip from its own 32-float row of `stage` (shared memory, column-major
+// so the rows of a warp's lanes share no bank): the warp runs as many trips as
+// its busiest lane needs, instead of the insertion at every column where any
+// lane has a candidate.  Candidates are taken in column order, so each enters
+// after every lower index.
+// Sorts eight values into descending order (a 19-comparator network).
+__device__ __forceinline__ void sort8_desc(float (&a)[8]) {
+    constexpr int P[19][2] = {{0, 2}, {1, 3}, {4, 6}, {5, 7}, {0, 4}, {1, 5}, {2, 6},
+                              {3, 7}, {0, 1}, {2, 3}, {4, 5}, {6, 7}, {2, 4}, {3, 5},
+                              {1, 4}, {3, 6}, {1, 2}, {3, 4}, {5, 6}};
+#pragma unroll
+    for (int e = 0; e < 19; ++e) {
+        const float hi = fmaxf(a[P[e][0]], a[P[e][1]]), lo = fminf(a[P[e][0]], a[P[e][1]]);
+        a[P[e][0]] = hi;
+        a[P[e][1]] = lo;
+    }
+}
+// A lower bound on the 8th largest of the 64 scores x, y: the 8th largest of
+// the 16 maxima of 4-column groups (eight distinct scores, each at or above
+// it).  With both groups' maxima sorted, the 8 largest of the union are
+// max(a[i], b[7-i]), so the bound is their minimum.
+__device__ __forceinline__ float eighth_bound64(const float (&x)[32], const float (&y)[32]) {
+    float a[8], b[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        a[q] = fmaxf(fmaxf(x[4 * q], x[4 * q + 1]), fmaxf(x[4 * q + 2], x[4 * q + 3]));
+        b[q] = fmaxf(fmaxf(y[4 * q], y[4 * q + 1]), fmaxf(y[4 * q + 2], y[4 * q + 3]));
+    }
+    sort8_desc(a);
+    sort8_desc(b);
+    float t = INFINITY;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t = fminf(t, fmaxf(a[q], b[7 - q]));
+    return t;
+}
 __device__ __forceinline__ int visible_in_block(int64_t nvis, int64_t c0) {
     const int64_t n = nvis - c0;
     return n <= 0 ? 0 : n >= 32 ? 32 : (int)n;
 }
 template <int KP>
 __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, int lim, float scale,
-                                           uint64_t (&v)[KP], float &tf, float *stage, int r) {
+                                           TopList<KP> &v, float &tf, float *stage, int r,
+                                           float floor) {
     const float tq = tf / scale;                                // scale > 0
-    float tr = tq - fabsf(tq) * 1e-6f;                          // -inf stays -inf
-    if (tf == -INFINITY && lim == 32 && KP < 32) {
+    float tr = fmaxf(tq - fabsf(tq) * 1e-6f, floor);            // -inf stays -inf
+    if (tr == -INFINITY && lim == 32 && KP < 32) {
         // empty list, full block: the smallest of the maxima of KP groups of
         // 32/KP columns is a lower bound on the KP-th largest of the 32 (each
         // group holds a score at or above it), so only scores at or above it
@@ -163,30 +227,29 @@ __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, in
 #pragma unroll
         for (int c = 0; c < 32; ++c) stage[c * 128 + r] = sc[c];
     }
-    // Branch-free trips: a key below every held one leaves the list as it is
-    // (insert_key then keeps every slot), so neither the score test nor the
-    // key test is needed, and the threshold is refreshed once at the end.
-    // (With the tests, every trip paid two divergent branches and a key-to-
-    // score conversion on its dependency chain: ~400-500 cycles a trip.)
+    // Branch-free trips: an entry below every held one leaves the list as it
+    // is, so no score test is needed, and the threshold is refreshed once at
+    // the end.
     while (mask) {
         const int c = __ffs(mask) - 1;
         mask &= mask - 1;
-        insert_key<KP>(v, make_key(scale * stage[c * 128 + r], c0 + c));
+        v.insert_later(scale * stage[c * 128 + r], (int32_t)c0 + c);
     }
-    tf = key_score(v[KP - 1]);
+    tf = v.s[KP - 1];
 }
 
 // The top-K runs in two groups of four warps (thread = token = TMEM lane),
-// each over alternate 32-column blocks of the scores into its own sorted list;
-// group 1 leaves its list in shared memory (`lists`, [KP][128] keys) and group
-// 0 folds it into its own.  Keys are distinct (they hold the chunk index), so
-// the result is the K largest keys of the token whatever the split.
+// each over alternate 32-column blocks of the scores into its own list;
+// group 1 leaves its list in shared memory (`lists`: [KP][128] scores, then
+// [KP][128] indices) and group 0 folds it into its own under the total order,
+// so the result is the token's top K whatever the split.
 template <int KP>
-__device__ __forceinline__ void merge_keys(uint64_t (&v)[KP], const uint64_t *lists, int r) {
+__device__ __forceinline__ void merge_lists(TopList<KP> &v, const float *lists, int r) {
+    const int32_t *li = reinterpret_cast<const int32_t *>(lists + KP * 128);
 #pragma unroll
     for (int j = 0; j < KP; ++j) {
-        const uint64_t x = lists[j * 128 + r];
-        if (x > v[KP - 1]) insert_key<KP>(v, x);
+        const int32_t xi = li[j * 128 + r];
+        if (xi >= 0) v.insert_any(lists[j * 128 + r], xi);
     }
 }
 
@@ -367,7 +430,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
     } else if (warp < 10) {
         // ------------------------------------------------------------ top-K
         // group 0 (warps 2-5) takes the 32-column blocks 0 and 2 of every
-        // score tile, group 1 (warps 6-9) blocks 1 and 3 (see merge_keys)
+        // score tile, group 1 (warps 6-9) blocks 1 and 3 (see merge_lists)
         const int q4 = warp & 3;
         const int hg = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;
@@ -375,10 +438,9 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int64_t t = t0 + r;                              // selection row
         const int64_t nvis = t < Lsel ? chunk_of(p.ch, t * R) : 0;
-        uint64_t v[KP];
-#pragma unroll
-        for (int i = 0; i < KP; ++i) v[i] = 0ull;
-        float tf = -INFINITY;                                  // score of v[KP-1]
+        TopList<KP> v;
+        v.clear();
+        float tf = -INFINITY;                                  // score of v's K-th entry
         for (int n = 0; n < ntiles; ++n) {
             const int s = n & 1;
             // warp-uniform outcome: the TMEM loads below are .sync.aligned
@@ -397,30 +459,56 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_constant
                 if (two) tc::tmem_ld32(tmem + s * C::N + (hg + 2) * 32 + lane_off, sc1);
                 tc::tmem_wait_ld();
                 const int64_t c0 = (int64_t)n * C::N + hg * 32;
-                topk_block<KP>(sc0, c0, visible_in_block(nvis, c0), p.scale, v, tf, stage, r);
-                if (two)
-                    topk_block<KP>(sc1, c0 + 64, visible_in_block(nvis, c0 + 64), p.scale, v, tf,
-                                   stage, r);
+                const int lim0 = visible_in_block(nvis, c0);
+                const int lim1 = two ? visible_in_block(nvis, c0 + 64) : 0;
+                float floor = -INFINITY;
+                if (KP == 8 && tf == -INFINITY && lim1 == 32) floor = eighth_bound64(sc0, sc1);
+                topk_block<KP>(sc0, c0, lim0, p.scale, v, tf, stage, r, floor);
+                if (two) topk_block<KP>(sc1, c0 + 64, lim1, p.scale, v, tf, stage, r, floor);
             }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&tfree[s]);
         }
         // the landmark stages are dead once the last tile's scores are in TMEM
-        uint64_t *lists = reinterpret_cast<uint64_t *>(sB(0));
+        float *lists = reinterpret_cast<float *>(sB(0));
         if (hg == 1) {
 #pragma unroll
-            for (int k = 0; k < KP; ++k) lists[k * 128 + r] = v[k];
+            for (int k = 0; k < KP; ++k) {
+                lists[k * 128 + r] = v.s[k];
+                reinterpret_cast<int32_t *>(lists + KP * 128)[k * 128 + r] = v.i[k];
+            }
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");     // the two top-K groups
         if (hg == 0 && t < Lsel) {
-            merge_keys<KP>(v, lists, r);
+            merge_lists<KP>(v, lists, r);
             // the row's selection serves its R tokens
             for (int j = 0; j < R && t * R + j < L; ++j) {
                 int32_t *dst = p.idx + ((b * L + t * R + j) * p.Hkv + g) * p.topk;
 #pragma unroll
                 for (int k = 0; k < KP; ++k)
-                    if (k < p.topk) dst[k] = key_index(v[k]);
+                    if (k < p.topk) dst[k] = v.i[k];
+            }
+        }
+    } else if (R == 1) {
+        // warps 10-11: warm L2 with the query rows of the block that will
+        // most likely start on some SM a wave later (one block per SM, blocks
+        // placed in launch order), so its qbar loads come from L2
+        uint32_t nsm;
+        asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
+        const int64_t lin = (int64_t)blockIdx.y * gridDim.x + blockIdx.x + nsm;
+        if (lin < (int64_t)gridDim.x * gridDim.y) {
+            const int tbn = ntb - 1 - (int)(lin % gridDim.x);
+            const int64_t bgn = lin / gridDim.x;
+            const int64_t bn = bgn / p.Hkv;
+            const int gn = (int)(bgn % p.Hkv);
+            for (int rr = tid - 10 * 32; rr < C::M; rr += 64) {
+                const int64_t t = (int64_t)tbn * C::M + rr;
+                if (t < L) {
+                    const __nv_bfloat16 *src = (const __nv_bfloat16 *)p.Q + ((bn * L + t) * p.H + (int64_t)gn * G) * D;
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"((uint32_t)(G * D * 2))
+                                 : "memory");
+                }
             }
         }
     }
@@ -615,10 +703,9 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int64_t t = t0 + r;                              // selection row
         const int64_t nvis = t < Lsel ? chunk_of(p.ch, t * R) : 0;
-        uint64_t v[KP];
-#pragma unroll
-        for (int i = 0; i < KP; ++i) v[i] = 0ull;
-        float tf = -INFINITY;                                  // score of v[KP-1]
+        TopList<KP> v;
+        v.clear();
+        float tf = -INFINITY;                                  // score of v's K-th entry
         // warp-uniform outcome: the TMEM loads below are .sync.aligned
         if (__all_sync(0xffffffffu, ok && sel_wait(tfull, 0u, s_abort))) {
             tc::fence_after_sync();
@@ -636,17 +723,19 @@ select_tc_half_kernel(const __grid_constant__ CUtensorMap tmL0, const __grid_con
                 if (two) tc::tmem_ld32(tmem + (cb + 1) * 32 + lane_off, sc1);
                 tc::tmem_wait_ld();
                 const int64_t c0 = (int64_t)cb * 32;
-                topk_block<KP>(sc0, c0, visible_in_block(nvis, c0), p.scale, v, tf, (float *)sA, r);
-                if (two)
-                    topk_block<KP>(sc1, c0 + 32, visible_in_block(nvis, c0 + 32), p.scale, v, tf,
-                                   (float *)sA, r);
+                const int lim0 = visible_in_block(nvis, c0);
+                const int lim1 = two ? visible_in_block(nvis, c0 + 32) : 0;
+                float floor = -INFINITY;
+                if (KP == 8 && tf == -INFINITY && lim1 == 32) floor = eighth_bound64(sc0, sc1);
+                topk_block<KP>(sc0, c0, lim0, p.scale, v, tf, (float *)sA, r, floor);
+                if (two) topk_block<KP>(sc1, c0 + 32, lim1, p.scale, v, tf, (float *)sA, r, floor);
             }
             tc::fence_before_sync();
             for (int j = 0; j < R && t < Lsel && t * R + j < L; ++j) {
                 int32_t *dst = p.idx + ((b * L + t * R + j) * p.Hkv + g) * p.topk;
 #pragma unroll
                 for (int k = 0; k < KP; ++k)
-                    if (k < p.topk) dst[k] = key_index(v[k]);
+                    if (k < p.topk) dst[k] = v.i[k];
             }
         }
     }
