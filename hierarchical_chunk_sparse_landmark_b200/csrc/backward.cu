@@ -567,7 +567,10 @@ bwd_key_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__rest
 // Sums each chunk's segment partials in segment order: dK, dV rows of the
 // chunk (every row of the output written once, zeros where nothing
 // contributed), the landmark gradient (dlm) or, for DHSA landmarks, dl / sqrt(S)
-// folded into every key of the chunk.
+// folded into every key of the chunk.  Grid: chunks x kReduceSlices; a block
+// takes a slice of the chunk's 16-byte groups of key elements, so a chunk with
+// many segments (one selected by most tokens) spreads over several SMs.
+constexpr int kReduceSlices = 8;
 template <int D>
 __global__ void __launch_bounds__(256)
 bwd_reduce_kernel(const float *__restrict__ part, const int32_t *__restrict__ chunk_seg_beg,
@@ -586,20 +589,29 @@ bwd_reduce_kernel(const float *__restrict__ part, const int32_t *__restrict__ ch
         float a = 0.f;
         for (int s = 0; s < ns; ++s) a += part[(sb + s) * (int64_t)(129 * D) + 128 * D + tid];
         dls[tid] = a;
-        if (!dhsa && c < Nc) dlm[(bg * Nc + c) * D + tid] = a;
+        if (blockIdx.y == 0 && !dhsa && c < Nc) dlm[(bg * Nc + c) * D + tid] = a;
     }
     __syncthreads();
     const float fold = (dhsa && c < Nc) ? rsqrtf((float)S) : 0.f;
-    for (int i = tid; i < nkc * D; i += blockDim.x) {
-        float a = 0.f, v = 0.f;
+    const int n4 = nkc * D / 4;
+    float4 *dk4 = reinterpret_cast<float4 *>(dK + (bg * L + first) * D);
+    float4 *dv4 = reinterpret_cast<float4 *>(dV + (bg * L + first) * D);
+    for (int i4 = blockIdx.y * blockDim.x + tid; i4 < n4; i4 += kReduceSlices * blockDim.x) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), v = a;
+#pragma unroll 4
         for (int s = 0; s < ns; ++s) {
-            const float *pk = part + (sb + s) * (int64_t)(129 * D);
-            a += pk[i];
-            v += pk[64 * D + i];
+            const float4 *pk = reinterpret_cast<const float4 *>(part + (sb + s) * (int64_t)(129 * D));
+            const float4 x = pk[i4], y = pk[16 * D + i4];
+            a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+            v.x += y.x; v.y += y.y; v.z += y.z; v.w += y.w;
         }
-        a = fmaf(fold, dls[i % D], a);
-        dK[(bg * L + first) * D + i] = a;
-        dV[(bg * L + first) * D + i] = v;
+        const int col = (4 * i4) % D;
+        a.x = fmaf(fold, dls[col], a.x);
+        a.y = fmaf(fold, dls[col + 1], a.y);
+        a.z = fmaf(fold, dls[col + 2], a.z);
+        a.w = fmaf(fold, dls[col + 3], a.w);
+        dk4[i4] = a;
+        dv4[i4] = v;
     }
 }
 
@@ -743,7 +755,7 @@ static cudaError_t launch_backward_t(const BwdArgs &a, const BwdLayout &p, cudaS
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 4. ordered reduction into dK, dV, dlm
-    bwd_reduce_kernel<D><<<(unsigned)(p.BG * p.NcAll), 256, 0, st>>>(
+    bwd_reduce_kernel<D><<<dim3((unsigned)(p.BG * p.NcAll), kReduceSlices), 256, 0, st>>>(
         part, cseg_beg, cseg_n, a.L, a.S, p.Nc, p.NcAll, a.dhsa, a.dK, a.dV, a.dlm);
     return cudaGetLastError();
 }

@@ -415,147 +415,259 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 }
 
 // ---------------------------------------------------------------- CUDA-core companions
-// Fusion weights w = softmax over the valid slots of scale q.l (one warp per
-// query row (t, h), lane k keeps slot k), written to coef[.].x.  A row's slot
-// indices come in one load and all its landmark rows' loads go out together.
+// The companions work per (b, t, g), one warp each: the G = 8 heads of a token
+// share its slots, so the landmark rows and slot indices are read once for all
+// eight, and the (t, g) blocks of Q, dw, coef and the dQ partials are
+// contiguous, so every load is a coalesced 8- or 16-byte one.
+
+// Four or eight consecutive landmark elements as fp32 (one load, or two for
+// eight fp32 values).
+template <typename TL> __device__ __forceinline__ void lm_load4(const TL *p, float (&v)[4]);
+template <> __device__ __forceinline__ void lm_load4<float>(const float *p, float (&v)[4]) {
+    const float4 u = *reinterpret_cast<const float4 *>(p);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+}
+template <> __device__ __forceinline__ void lm_load4<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+template <typename TL> __device__ __forceinline__ void lm_load8(const TL *p, float (&v)[8]) {
+    float a[4], b[4];
+    lm_load4<TL>(p, a);
+    lm_load4<TL>(p + 4, b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[i] = a[i];
+        v[4 + i] = b[i];
+    }
+}
+template <> __device__ __forceinline__ void lm_load8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[8]) {
+    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4 *>(p), v);
+}
+
+// Fusion weights w = softmax over the valid slots of scale q_h . l_k, written
+// to coef[.].x.  Lane l holds elements 4l .. 4l+3 of the eight heads' queries
+// and, for a group of four slots, of their four landmark rows: 32 partial dot
+// products (slot-major), which five halving exchanges reduce over the warp so
+// that lane l ends with the logit of slot 4i + l/8, head l%8.  A head's
+// softmax then runs over the four lanes that share l%8 and over the groups.
 template <typename TL>
 __global__ void __launch_bounds__(256)
 bwd_coefw_kernel(const __nv_bfloat16 *__restrict__ Q, const TL *__restrict__ lm,
-                 const int32_t *__restrict__ idx, int64_t rows, int H, int Hkv, int64_t L, int S,
+                 const int32_t *__restrict__ idx, int64_t pairs, int H, int Hkv, int64_t L, int S,
                  int64_t Nc, int topk, float scale, float2 *__restrict__ coef,
                  unsigned *__restrict__ status) {
-    constexpr int D = BT_D, R = D / 32, KMAX = 32;
+    constexpr int D = BT_D, G = BT_G, NGR = 8;    // topk <= 32: up to eight groups of four slots
     const int lane = threadIdx.x & 31;
-    const int64_t hrow = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (hrow >= rows) return;
-    const int64_t bt = hrow / H;
-    const int h = (int)(hrow % H);
-    const int G = H / Hkv, g = h / G;
+    const int64_t tg = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);     // (b, t, g)
+    if (tg >= pairs) return;
+    const int g = (int)(tg % Hkv);
+    const int64_t bt = tg / Hkv;
     const int64_t b = bt / L, t = bt % L;
     const int64_t bg = b * Hkv + g;
-    float qv[R];
+    const int64_t hrow0 = bt * H + (int64_t)g * G;
+    float qv[G][4];
 #pragma unroll
-    for (int r = 0; r < R; ++r) qv[r] = __bfloat162float(Q[hrow * D + lane + 32 * r]);
-    const int32_t ci_l = lane < topk ? idx[(bt * Hkv + g) * topk + lane] : -1;
-    const bool vk = ci_l >= 0 && (int64_t)ci_l < Nc && (int64_t)ci_l < t / S;
-    if (lane < topk && ci_l >= 0 && !vk && h % G == 0) atomicOr(status, kFlagBadIdx);
-    const unsigned vmask = __ballot_sync(0xffffffffu, vk);
-    float zk = -INFINITY;
-#pragma unroll 4
-    for (int k = 0; k < KMAX; ++k) {
-        if (k >= topk) break;
-        if (!((vmask >> k) & 1u)) continue;
-        const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
-        const TL *lr = lm + (bg * Nc + ci) * D + lane;
-        float a = 0.f;
-#pragma unroll
-        for (int r = 0; r < R; ++r) a = fmaf(qv[r], to_f32(lr[32 * r]), a);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == k) zk = scale * a;
+    for (int hh = 0; hh < G; ++hh) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(Q + (hrow0 + hh) * D + 4 * lane);
+        qv[hh][0] = __uint_as_float(u.x << 16); qv[hh][1] = __uint_as_float(u.x & 0xffff0000u);
+        qv[hh][2] = __uint_as_float(u.y << 16); qv[hh][3] = __uint_as_float(u.y & 0xffff0000u);
     }
-    float m = vk ? zk : -INFINITY;
+    const int32_t ci_l = lane < topk ? idx[tg * topk + lane] : -1;
+    const bool vk = ci_l >= 0 && (int64_t)ci_l < Nc && (int64_t)ci_l < t / S;
+    if (lane < topk && ci_l >= 0 && !vk) atomicOr(status, kFlagBadIdx);
+    const unsigned vmask = __ballot_sync(0xffffffffu, vk);
+    float z[NGR];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float ew = vk ? expf(zk - m) : 0.f;
-    float sw = ew;
+    for (int gi = 0; gi < NGR; ++gi) {
+        z[gi] = -INFINITY;
+        if (gi * 4 >= topk) continue;                          // warp-uniform
+        float v[32];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
-    if (lane < topk) coef[hrow * topk + lane] = make_float2(vk ? ew / sw : 0.f, 0.f);
+        for (int kk = 0; kk < 4; ++kk) {
+            const int k = gi * 4 + kk;
+            const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
+            float lv[4] = {0.f, 0.f, 0.f, 0.f};
+            if ((vmask >> k) & 1u) lm_load4<TL>(lm + (bg * Nc + ci) * D + 4 * lane, lv);
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh)
+                v[kk * G + hh] = fmaf(qv[hh][3], lv[3], fmaf(qv[hh][2], lv[2], fmaf(qv[hh][1], lv[1], qv[hh][0] * lv[0])));
+        }
+        // after the exchange with offset o a lane keeps the half of its values
+        // whose index bit matches its lane bit o, adding the partner's copy
+#pragma unroll
+        for (int st = 0; st < 5; ++st) {
+            const int o = 16 >> st;
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < o; ++i) {
+                const float send = up ? v[i] : v[i + o];
+                const float keep = up ? v[i + o] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        if ((vmask >> (gi * 4 + (lane >> 3))) & 1u) z[gi] = scale * v[0];
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int gi = 0; gi < NGR; ++gi) m = fmaxf(m, z[gi]);
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    float ew[NGR], sw = 0.f;
+#pragma unroll
+    for (int gi = 0; gi < NGR; ++gi) {
+        ew[gi] = z[gi] > -INFINITY ? expf(z[gi] - m) : 0.f;
+        sw += ew[gi];
+    }
+    sw += __shfl_xor_sync(0xffffffffu, sw, 8);
+    sw += __shfl_xor_sync(0xffffffffu, sw, 16);
+    float2 *cr = coef + (hrow0 + (lane & 7)) * topk;
+#pragma unroll
+    for (int gi = 0; gi < NGR; ++gi) {
+        const int k = gi * 4 + (lane >> 3);
+        if (k < topk) cr[k] = make_float2(z[gi] > -INFINITY ? ew[gi] / sw : 0.f, 0.f);
+    }
 }
 
-// Per query row: dz = w (dw - sum w dw) (to coef[.].y), and
-// dQ = sum of the row's dQ partials over its valid slots and the own chunk
-// + scale sum_k dz_k l_k.
+// Per (b, t, g): dz = w (dw - sum w dw) per head and slot (to coef[.].y), and
+// each head's dQ = the sum of its dQ partials over the valid slots and the own
+// chunk + scale sum_k dz_k l_k.  The partials of (t, g) are one [slot][G][D]
+// fp16 block: lane l reads the 16-byte pieces l + 32 j (j < 4) of a slot, i.e.
+// elements 8 (l % 16) .. +8 of head 2j + l / 16.
 template <typename TL>
 __global__ void __launch_bounds__(256)
 bwd_rowfin_kernel(const TL *__restrict__ lm, const int32_t *__restrict__ idx,
-                  const float *__restrict__ dw, const __half *__restrict__ dqp, int64_t rows, int H,
-                  int Hkv, int64_t L, int S, int64_t Nc, int topk, int own_chunk, float scale,
-                  float2 *__restrict__ coef, float *__restrict__ dQ) {
-    constexpr int D = BT_D, R = D / 32;
+                  const float *__restrict__ dw, const __half *__restrict__ dqp, int64_t pairs,
+                  int H, int Hkv, int64_t L, int S, int64_t Nc, int topk, int own_chunk,
+                  float scale, float2 *__restrict__ coef, float *__restrict__ dQ) {
+    constexpr int D = BT_D, G = BT_G;
     const int lane = threadIdx.x & 31;
-    const int64_t hrow = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (hrow >= rows) return;
-    const int64_t bt = hrow / H;
-    const int h = (int)(hrow % H);
-    const int G = H / Hkv, g = h / G, hh = h % G;
+    const int64_t tg = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);     // (b, t, g)
+    if (tg >= pairs) return;
+    const int g = (int)(tg % Hkv);
+    const int64_t bt = tg / Hkv;
     const int64_t b = bt / L, t = bt % L;
     const int64_t bg = b * Hkv + g;
-    const int32_t *ip = idx + (bt * Hkv + g) * topk;
-    const int32_t ci_l = lane < topk ? ip[lane] : -1;
+    const int64_t hrow0 = bt * H + (int64_t)g * G;
+    const int32_t ci_l = lane < topk ? idx[tg * topk + lane] : -1;
     const bool vk = lane < topk && ci_l >= 0 && (int64_t)ci_l < Nc && (int64_t)ci_l < t / S;
-    const float wk = vk ? coef[hrow * topk + lane].x : 0.f;
-    const float dwk = vk ? dw[hrow * (topk + 1) + lane] : 0.f;
-    float dsum = wk * dwk;
+    const unsigned vmask = __ballot_sync(0xffffffffu, vk);
+    // lane k: dz of slot k for every head
+    float wk[G], dwk[G], dzr[G];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-    const float dzk = wk * (dwk - dsum);
-    if (lane < topk) coef[hrow * topk + lane] = make_float2(wk, dzk);
-    float acc[R];
+    for (int hh = 0; hh < G; ++hh) {
+        wk[hh] = vk ? coef[(hrow0 + hh) * topk + lane].x : 0.f;
+        dwk[hh] = vk ? dw[(hrow0 + hh) * (topk + 1) + lane] : 0.f;
+    }
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    const __half *qp = dqp + ((bt * Hkv + g) * (topk + 1)) * (int64_t)(G * D) + hh * D;
+    for (int hh = 0; hh < G; ++hh) {
+        float dsum = wk[hh] * dwk[hh];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+        dzr[hh] = wk[hh] * (dwk[hh] - dsum);
+        if (lane < topk) coef[(hrow0 + hh) * topk + lane] = make_float2(wk[hh], dzr[hh]);
+    }
+    const int hs = lane >> 4, d0 = 8 * (lane & 15);
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+    const uint4 *qp = reinterpret_cast<const uint4 *>(dqp + tg * (int64_t)(topk + 1) * (G * D)) + lane;
     for (int k = 0; k < topk; ++k) {
-        if (!__shfl_sync(0xffffffffu, vk ? 1 : 0, k)) continue;
-        const float dz = scale * __shfl_sync(0xffffffffu, dzk, k);
+        if (!((vmask >> k) & 1u)) continue;                  // warp-uniform
         const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
+        uint4 raw[4];
 #pragma unroll
-        for (int r = 0; r < R; ++r)
-            acc[r] += __half2float(qp[(int64_t)k * G * D + lane + 32 * r]) +
-                      dz * to_f32(lm[(bg * Nc + ci) * D + lane + 32 * r]);
+        for (int j = 0; j < 4; ++j) raw[j] = qp[(int64_t)k * (G * D / 8) + 32 * j];
+        float lv[8];
+        lm_load8<TL>(lm + (bg * Nc + ci) * D + d0, lv);
+        float dzk[G];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) dzk[hh] = scale * __shfl_sync(0xffffffffu, dzr[hh], k);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float dz = hs ? dzk[2 * j + 1] : dzk[2 * j];
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[j]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h2[e]);
+                acc[j][2 * e] += f.x + dz * lv[2 * e];
+                acc[j][2 * e + 1] += f.y + dz * lv[2 * e + 1];
+            }
+        }
     }
     if (own_chunk) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[r] += __half2float(qp[(int64_t)topk * G * D + lane + 32 * r]);
+        for (int j = 0; j < 4; ++j) {
+            const uint4 r = qp[(int64_t)topk * (G * D / 8) + 32 * j];
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&r);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h2[e]);
+                acc[j][2 * e] += f.x;
+                acc[j][2 * e + 1] += f.y;
+            }
+        }
     }
 #pragma unroll
-    for (int r = 0; r < R; ++r) dQ[hrow * D + lane + 32 * r] = acc[r];
+    for (int j = 0; j < 4; ++j) {
+        float4 *dst = reinterpret_cast<float4 *>(dQ + (hrow0 + 2 * j + hs) * D + d0);
+        dst[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+        dst[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+    }
 }
 
-// Landmark-gradient partial of each entry segment, dl = scale sum_rows dz q:
-// four groups of D threads (thread = element of d) take every fourth entry,
-// then add their sums in group order; own-chunk segments carry none.
-constexpr int kDlGroups = 4;
-__global__ void __launch_bounds__(BT_D * kDlGroups)
+// Landmark-gradient partial of each entry segment, dl = scale sum over its
+// entries' head rows of dz q: one block per segment, warp w takes the entries
+// w, w + 8, ... (lane l: elements 4l .. 4l+3 of the eight head rows, one
+// 8-byte load each; lanes 0-7 load the entry's eight dz and broadcast them);
+// the warps' sums are added in warp order.  Own-chunk segments carry none.
+constexpr int kDlWarps = 8;
+__global__ void __launch_bounds__(32 * kDlWarps)
 bwd_dl_kernel(const __nv_bfloat16 *__restrict__ Q, const float2 *__restrict__ coef,
               const int32_t *__restrict__ entries, const int4 *__restrict__ segs,
               const int32_t *__restrict__ nseg_p, int H, int Hkv, int64_t L, int64_t NcAll,
               int topk, float scale, float *__restrict__ part) {
-    constexpr int D = BT_D;
-    __shared__ float red[kDlGroups][D];
+    constexpr int D = BT_D, G = BT_G;
+    __shared__ float red[kDlWarps][D];
     const int64_t sidx = blockIdx.x;
     if (sidx >= *nseg_p) return;
     const int4 sg = segs[sidx];
     const int64_t bg = (int64_t)sg.x / NcAll;
     const int64_t b = bg / Hkv;
     const int g = (int)(bg % Hkv);
-    const int G = H / Hkv;
-    const int d = threadIdx.x % D, grp = threadIdx.x / D;
-    float acc = 0.f;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (!sg.w) {
-        for (int u = grp; u < sg.z; u += kDlGroups) {
+#pragma unroll 2
+        for (int u = warp; u < sg.z; u += kDlWarps) {
             const int32_t code = entries[sg.y + u];
-            const int64_t t = code >> 5;
-            const int slot = code & 31;
-            const int64_t r0 = (b * L + t) * H + (int64_t)g * G;
-            float dz[BT_G], qv[BT_G];
+            const int64_t r0 = (b * L + (code >> 5)) * H + (int64_t)g * G;
+            const float dzl = lane < G ? coef[(r0 + lane) * topk + (code & 31)].y : 0.f;
+            uint2 qr[G];
 #pragma unroll
-            for (int hh = 0; hh < BT_G; ++hh) {
-                dz[hh] = coef[(r0 + hh) * topk + slot].y;
-                qv[hh] = __bfloat162float(Q[(r0 + hh) * D + d]);
+            for (int hh = 0; hh < G; ++hh)
+                qr[hh] = *reinterpret_cast<const uint2 *>(Q + (r0 + hh) * D + 4 * lane);
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+                const float dz = __shfl_sync(0xffffffffu, dzl, hh);
+                acc[0] = fmaf(dz, __uint_as_float(qr[hh].x << 16), acc[0]);
+                acc[1] = fmaf(dz, __uint_as_float(qr[hh].x & 0xffff0000u), acc[1]);
+                acc[2] = fmaf(dz, __uint_as_float(qr[hh].y << 16), acc[2]);
+                acc[3] = fmaf(dz, __uint_as_float(qr[hh].y & 0xffff0000u), acc[3]);
             }
-#pragma unroll
-            for (int hh = 0; hh < BT_G; ++hh) acc = fmaf(dz[hh], qv[hh], acc);
         }
     }
-    red[grp][d] = acc;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) red[warp][4 * lane + e] = acc[e];
     __syncthreads();
-    if (grp == 0) {
+    if (threadIdx.x < D) {
         float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < kDlGroups; ++i) s += red[i][d];
-        part[sidx * (int64_t)(129 * D) + 128 * D + d] = scale * s;
+        for (int w = 0; w < kDlWarps; ++w) s += red[w][threadIdx.x];
+        part[sidx * (int64_t)(129 * D) + 128 * D + threadIdx.x] = scale * s;
     }
 }
 
@@ -572,16 +684,17 @@ cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, cons
                                float *part, int64_t max_seg, unsigned *status, float *dQ,
                                int phase, cudaStream_t st) {
     const int64_t rows = (int64_t)B * L * H;
-    const unsigned rblocks = (unsigned)((rows + 7) / 8);
+    const int64_t pairs = (int64_t)B * L * Hkv;              // one warp per (b, t, g)
+    const unsigned rblocks = (unsigned)((pairs + 7) / 8);
     cudaError_t e;
     if (phase == 0) {            // fusion weights (before the key pass)
         if (lm_bf16)
             bwd_coefw_kernel<__nv_bfloat16><<<rblocks, 256, 0, st>>>(
-                (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)lm, idx, rows, H, Hkv, L, S, Nc,
+                (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)lm, idx, pairs, H, Hkv, L, S, Nc,
                 topk, scale, coef, status);
         else
             bwd_coefw_kernel<float><<<rblocks, 256, 0, st>>>(
-                (const __nv_bfloat16 *)Q, (const float *)lm, idx, rows, H, Hkv, L, S, Nc, topk,
+                (const __nv_bfloat16 *)Q, (const float *)lm, idx, pairs, H, Hkv, L, S, Nc, topk,
                 scale, coef, status);
         return cudaGetLastError();
     }
@@ -606,14 +719,14 @@ cudaError_t launch_backward_tc(const void *Q, const void *K, const void *V, cons
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (lm_bf16)
         bwd_rowfin_kernel<__nv_bfloat16><<<rblocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)lm, idx, dw, dqp, rows, H, Hkv, L, S, Nc, topk, own_chunk, scale,
+            (const __nv_bfloat16 *)lm, idx, dw, dqp, pairs, H, Hkv, L, S, Nc, topk, own_chunk, scale,
             coef, dQ);
     else
         bwd_rowfin_kernel<float><<<rblocks, 256, 0, st>>>(
-            (const float *)lm, idx, dw, dqp, rows, H, Hkv, L, S, Nc, topk, own_chunk, scale, coef,
+            (const float *)lm, idx, dw, dqp, pairs, H, Hkv, L, S, Nc, topk, own_chunk, scale, coef,
             dQ);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dl_kernel<<<(unsigned)max_seg, BT_D * kDlGroups, 0, st>>>((const __nv_bfloat16 *)Q, coef, entries, segs,
+    bwd_dl_kernel<<<(unsigned)max_seg, 32 * kDlWarps, 0, st>>>((const __nv_bfloat16 *)Q, coef, entries, segs,
                                                      nseg, H, Hkv, L, NcAll, topk, scale, part);
     return cudaGetLastError();
 }
