@@ -39,7 +39,8 @@ namespace hsa {
 
 namespace {
 
-constexpr int kBtThreads = 256;            // two threads per tile row: keys 0-31, 32-63
+constexpr int kBtThreads = 288;            // 8 compute warps (two threads per tile row:
+                                           // keys 0-31, 32-63) and an issuer warp
 constexpr long long kBtWait = 4000000000LL;       // SM cycles (about 2 s)
 constexpr int BT_D = 128, BT_G = 8, BT_EPT = 16;  // d, heads per entry, entries per tile
 // shared memory, offsets from a 1024-byte aligned base: two buffers of the
@@ -51,9 +52,7 @@ constexpr int OFF_K = OFF_DO + 2 * QBUF;   // [2 halves][64 keys][128 B]
 constexpr int OFF_V = OFF_K + 16384;
 constexpr int OFF_DS = OFF_V + 16384;      // [128 rows][64 keys] bf16, 128B-swizzled
 constexpr int OFF_WP = OFF_DS + 16384;
-constexpr int STG_ROW = 272;               // staged dQ row: 256 B + 16 (no bank conflicts)
-constexpr int OFF_RED = OFF_DS + 128 * STG_ROW;   // (dS, wP and the dQ staging overlap) then
-                                                  // [3][2 halves][128 rows] fp32: row max, sums
+constexpr int OFF_RED = OFF_WP + 16384;    // [3][2 halves][128 rows] fp32: row max, sums
 constexpr int OFF_BAR = OFF_RED + 3 * 2 * 128 * 4;   // mbarriers, TMEM address, abort flag
 constexpr int BT_SMEM = 1024 + OFF_BAR + 128;
 // TMEM columns (fp32): S and U twice (the next tile's products run during this
@@ -103,6 +102,55 @@ struct BtRow {
     bool valid;
 };
 
+// One segment: chunk c of (b, g), its entries (or its own tokens) in tiles of
+// BT_EPT.
+struct BtSeg {
+    int64_t bg, b, c, first;
+    int g, own, n_units, ntiles;
+    int32_t ebase;
+};
+__device__ __forceinline__ BtSeg bt_segment(const BtParams &p, int64_t sidx) {
+    const int4 sg = p.segs[sidx];
+    BtSeg s;
+    const int64_t q = sg.x;
+    s.bg = q / p.NcAll;
+    s.c = q % p.NcAll;
+    s.b = s.bg / p.Hkv;
+    s.g = (int)(s.bg % p.Hkv);
+    s.own = sg.w;
+    s.first = s.c * p.S;
+    const int nkc = (int)(p.L - s.first < p.S ? p.L - s.first : p.S);
+    s.n_units = s.own ? nkc : sg.z;      // tokens (own) or entries of the segment
+    s.ntiles = (s.n_units + BT_EPT - 1) / BT_EPT;
+    s.ebase = sg.y;
+    return s;
+}
+
+// Barrier 1 over the eight compute warps (the issuer warp is not in it), with
+// the AND of the threads' votes, so that a timeout is seen by all of them.
+__device__ __forceinline__ bool cbar_and(bool v) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.and.pred q, 1, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Roles: warps 0-7 compute (two threads per tile row: softmax, dS and w P,
+// the dQ partial epilogue, the segment's dK / dV readout); warp 8 issues
+// (lane 0 the MMAs, lanes 0-15 the row loads of their entries).  Per tile
+// the issuer runs S and U of the next tile on the tensor pipe while the
+// compute warps take this tile's softmax, then this tile's dV^T, dK^T and dQ
+// products once the softmax has written dS and w P; the compute warps meet it
+// only at the mbarriers below.
+//   su_bar[buf]  S, U of a tile complete          (issuer -> compute)
+//   ds_full      dS, w P of a tile written        (compute, one arrive per warp -> issuer)
+//   o_bar        dV^T, dK^T, dQ of a tile done    (issuer -> both)
+//   seg_free     dK^T / dV^T of a segment read    (compute, per warp -> issuer)
+constexpr int kBtCompute = 256;
+constexpr int kBtIssuer = 8;               // warp index of the issuer
+
 __global__ void __launch_bounds__(kBtThreads, 1)
 bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -114,13 +162,10 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t *bars = (uint64_t *)(sm + OFF_BAR);
     uint64_t *kv_bar = bars, *tma_bar = bars + 1, *su_bar = bars + 3, *o_bar = bars + 5;
-    uint32_t *s_tmem = (uint32_t *)(bars + 6);
+    uint64_t *ds_full = bars + 6, *seg_free = bars + 7;
+    uint32_t *s_tmem = (uint32_t *)(bars + 8);
     volatile int *s_abort = (volatile int *)(s_tmem + 1);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int rt = tid & 127, hf = tid >> 7;          // tile row (TMEM lane), key half
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    float *red = (float *)(sm + OFF_RED);
-    const int e = rt >> 3, h = rt & 7;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t L = p.L;
     const int H = p.H, topk = p.topk;
 
@@ -135,6 +180,8 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) tc::mbar_init(&bars[i], 1);
+        tc::mbar_init(ds_full, kBtCompute / 32);
+        tc::mbar_init(seg_free, kBtCompute / 32);
         *s_abort = 0;
         tc::fence_barrier_init();
     }
@@ -142,267 +189,291 @@ bwd_key_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    uint32_t pkv = 0u, ptma[2] = {0u, 0u}, psu[2] = {0u, 0u}, po = 0u;
-    // descriptors of the fixed tiles (bytes >> 4 in the start field; a K step moves the start)
-    const uint32_t IDESC_SU = tc::idesc_bf16_f32(128, 64, false, false);
-    const uint32_t IDESC_T = tc::idesc_bf16_f32(128, 64, true, true);     // M = d, N = keys
-    const uint32_t IDESC_DQ = tc::idesc_bf16_f32(128, D, true, false);    // B = K, MN-major
-    const uint64_t bK = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);     // keys x d
-    const uint64_t bV = tc::sdesc_sw128(tc::smem_u32(sm + OFF_V), 16, 1024);
-    const uint64_t bDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16384, 1024);  // (keys, rows)
-    const uint64_t bWP = tc::sdesc_sw128(tc::smem_u32(sm + OFF_WP), 16384, 1024);
-    const uint64_t aDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16, 1024);     // rows x keys
-    const uint64_t bKt = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 8192, 1024);    // (d, keys)
     bool ok = true;
 
-    // persistent: this block takes segments blockIdx.x, + gridDim.x, ...
-    for (int64_t sidx = blockIdx.x; sidx < nseg && ok; sidx += gridDim.x) {
-        const int4 sg = p.segs[sidx];
-        const int64_t q = sg.x;
-        const int64_t bg = q / p.NcAll, c = q % p.NcAll;
-        const int64_t b = bg / p.Hkv;
-        const int g = (int)(bg % p.Hkv);
-        const int own = sg.w;
-        const int64_t first = c * p.S;
-        const int nkc = (int)(L - first < p.S ? L - first : p.S);
-        const int n_units = own ? nkc : sg.z;      // tokens (own) or entries of the segment
-        const int ntiles = (n_units + BT_EPT - 1) / BT_EPT;
-        auto row_of = [&](int ti) -> BtRow {
-            BtRow r;
-            const int u = ti * BT_EPT + e;
-            r.valid = u < n_units;
-            r.t = -1;
-            r.slot = topk;
-            if (r.valid) {
-                if (own) {
-                    r.t = first + u;
-                } else {
-                    const int32_t code = p.entries[sg.y + u];
-                    r.t = code >> 5;
-                    r.slot = code & 31;
+    if (warp == kBtIssuer) {
+        // ------------------------------------------------------------ issuer
+        const uint32_t IDESC_SU = tc::idesc_bf16_f32(128, 64, false, false);
+        const uint32_t IDESC_T = tc::idesc_bf16_f32(128, 64, true, true);     // M = d, N = keys
+        const uint32_t IDESC_DQ = tc::idesc_bf16_f32(128, D, true, false);    // B = K, MN-major
+        // descriptors of the fixed tiles (bytes >> 4 in the start field; a K step moves the start)
+        const uint64_t bK = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 16, 1024);     // keys x d
+        const uint64_t bV = tc::sdesc_sw128(tc::smem_u32(sm + OFF_V), 16, 1024);
+        const uint64_t bDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16384, 1024);  // (keys, rows)
+        const uint64_t bWP = tc::sdesc_sw128(tc::smem_u32(sm + OFF_WP), 16384, 1024);
+        const uint64_t aDS = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DS), 16, 1024);     // rows x keys
+        const uint64_t bKt = tc::sdesc_sw128(tc::smem_u32(sm + OFF_K), 8192, 1024);    // (d, keys)
+        uint32_t pkv = 0u, ptma[2] = {0u, 0u}, pds = 0u, po = 0u, pfree = 0u;
+        bool dkdv_held = false;          // the compute warps still have to read a segment's dK / dV
+        for (int64_t sidx = blockIdx.x; sidx < nseg && ok; sidx += gridDim.x) {
+            const BtSeg sg = bt_segment(p, sidx);
+            // Q / dO rows of tile ti into buffer ti % 2 (one 3-D box per entry:
+            // its 8 head rows, both halves of d); the buffer's readers are done
+            auto load_rows = [&](int ti) {
+                const int buf = ti & 1;
+                const int nvalid = sg.n_units - ti * BT_EPT < BT_EPT ? sg.n_units - ti * BT_EPT : BT_EPT;
+                if (lane == 0) tc::mbar_expect_tx(&tma_bar[buf], (uint32_t)nvalid * 2u * 2048u);
+                __syncwarp();
+                if (lane < nvalid) {
+                    const int u = ti * BT_EPT + lane;
+                    const int64_t t = sg.own ? sg.first + u : (int64_t)(p.entries[sg.ebase + u] >> 5);
+                    const int qrow = (int)((sg.b * L + t) * H + (int64_t)sg.g * G);
+                    tc::tma_load_3d(sm + OFF_Q + buf * QBUF + lane * 2048, &tmQ, &tma_bar[buf], 0, qrow, 0);
+                    tc::tma_load_3d(sm + OFF_DO + buf * QBUF + lane * 2048, &tmO, &tma_bar[buf], 0, qrow, 0);
                 }
-            }
-            return r;
-        };
-        // Q / dO rows of tile ti into buffer ti % 2 (one 3-D box per entry: its
-        // 8 head rows, both halves of d); the caller has made the buffer free
-        auto load_rows = [&](int ti, const BtRow &r) {
-            const int buf = ti & 1;
-            const int nvalid = n_units - ti * BT_EPT < BT_EPT ? n_units - ti * BT_EPT : BT_EPT;
-            if (tid == 0) tc::mbar_expect_tx(&tma_bar[buf], (uint32_t)nvalid * 2u * 2048u);
-            __syncthreads();
-            if (r.valid && h == 0 && hf == 0) {
-                const int qrow = (int)((b * L + r.t) * H + (int64_t)g * G);
-                tc::tma_load_3d(sm + OFF_Q + buf * QBUF + e * 2048, &tmQ, &tma_bar[buf], 0, qrow, 0);
-                tc::tma_load_3d(sm + OFF_DO + buf * QBUF + e * 2048, &tmO, &tma_bar[buf], 0, qrow, 0);
-            }
-        };
-        // S = Q.K^T and U = dO.V^T of tile ti (thread 0)
-        auto issue_su = [&](int ti) {
-            const int buf = ti & 1;
-            const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 16, 2048);
-            const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 16, 2048);
-            const uint32_t ds = tmem + COL_SU + 128u * (uint32_t)buf;
-            tc::fence_after_sync();
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t acc = (kb | kk) ? 1u : 0u;
-                    tc::mma_bf16(ds, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
-                                 bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
-                    tc::mma_bf16(ds + 64, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
-                                 bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
-                }
-            tc::mma_commit(&su_bar[buf]);
-        };
-        // entry codes are read two tiles ahead and fusion weights one tile
-        // ahead, so neither load's latency sits on a tile's critical path
-        auto weight_of = [&](const BtRow &r) -> float {
-            if (!r.valid) return 0.f;
-            if (own) return 1.f;
-            return p.coef[((b * L + r.t) * H + (int64_t)g * G + h) * topk + r.slot].x;
-        };
-
-        // K and V of the chunk (the previous segment's products are done with
-        // them) and the first tile's rows
-        const int krow = (int)(bg * L + first);
-        if (tid == 0) {
-            tc::mbar_expect_tx(kv_bar, 2u * 16384u);
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb) {
-                tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, kv_bar, kb * 64, krow);
-                tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, kv_bar, kb * 64, krow);
-            }
-        }
-        BtRow cur = row_of(0);
-        BtRow nxt = ntiles > 1 ? row_of(1) : cur;
-        float w_cur = weight_of(cur);
-        if (ntiles > 0) load_rows(0, cur);
-        if (ntiles > 1) load_rows(1, nxt);     // the rows of tile ti + 2 load during tile ti
-        // every wait's outcome is made block-uniform, so that all threads
-        // leave the loops together on a timeout
-        ok = __syncthreads_and(bt_wait(kv_bar, pkv, s_abort) &&
-                               (ntiles == 0 || bt_wait(&tma_bar[0], ptma[0], s_abort))) != 0;
-        pkv ^= 1u;
-        if (ntiles > 0) ptma[0] ^= 1u;
-        if (ok && ntiles > 0 && tid == 0) issue_su(0);
-        for (int ti = 0; ti < ntiles && ok; ++ti) {
-            const int buf = ti & 1, nb = buf ^ 1;
-            const bool more = ti + 1 < ntiles;
-            const BtRow nxt2 = ti + 2 < ntiles ? row_of(ti + 2) : nxt;
-            const float w_nxt = more ? weight_of(nxt) : 0.f;
-            // the dS / wP tiles double as the staging of the previous tile's dQ
-            // rows: its bulk stores must have read them before they are rewritten
-            if (hf == 0) tc::bulk_wait_read_all();
-            const bool valid = cur.valid;
-            const int64_t t = cur.t;
-            const int slot = cur.slot;
-            const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
-            const float w = w_cur;
-            if (!__syncthreads_and(bt_wait(&su_bar[buf], psu[buf], s_abort))) { ok = false; break; }
-            psu[buf] ^= 1u;
-            tc::fence_after_sync();
-            // this row's chunk softmax, dw, dS and w p over this thread's 32
-            // keys (j0 .. j0+31); the row max and the two sums are combined
-            // with the other half through shared memory
-            const int j0 = hf * 32;
-            float s[32], uu[32];
-            {
-                const uint32_t ts = tmem + lane_off + COL_SU + 128u * (uint32_t)buf + (uint32_t)j0;
-                tc::tmem_ld32(ts, s);
-                tc::tmem_ld32(ts + 64, uu);
-                tc::tmem_wait_ld();
-            }
-            const int nk = own ? (valid ? (int)(t - first) + 1 : 64) : 64;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) mx = j0 + j < nk ? fmaxf(mx, s[j]) : mx;
-            red[hf * 128 + rt] = mx;
-            __syncthreads();
-            mx = fmaxf(red[rt], red[128 + rt]);
-            // exp(scale (s - max)) as 2^(scale log2(e) (s - max)) on the MUFU unit
-            const float sl2 = p.scale * 1.4426950408889634f, ml2 = -sl2 * mx;
-            float z = 0.f, zu = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float ej = j0 + j < nk ? tc::ex2_approx(fmaf(s[j], sl2, ml2)) : 0.f;
-                s[j] = ej;
-                z += ej;
-                zu = fmaf(ej, uu[j], zu);
-            }
-            red[256 + hf * 128 + rt] = z;
-            red[512 + hf * 128 + rt] = zu;
-            __syncthreads();
-            z = red[256 + rt] + red[384 + rt];
-            zu = red[512 + rt] + red[640 + rt];
-            const float inv = 1.f / z;
-            const float dwv = zu * inv;
-            if (valid && hf == 0) p.dw[hrow * (topk + 1) + slot] = dwv;
-            const float fds = valid ? p.scale * w * inv : 0.f, fwp = valid ? w * inv : 0.f;
-#pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-                uint32_t ds4[4], wp4[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int j = cq * 8 + 2 * i;
-                    ds4[i] = pack2_bf16(fds * s[j] * (uu[j] - dwv), fds * s[j + 1] * (uu[j + 1] - dwv));
-                    wp4[i] = pack2_bf16(fwp * s[j], fwp * s[j + 1]);
-                }
-                const uint32_t off = tc::sw128_offset(rt, hf * 4 + cq);
-                *reinterpret_cast<uint4 *>(sm + OFF_DS + off) = make_uint4(ds4[0], ds4[1], ds4[2], ds4[3]);
-                *reinterpret_cast<uint4 *>(sm + OFF_WP + off) = make_uint4(wp4[0], wp4[1], wp4[2], wp4[3]);
-            }
-            tc::fence_proxy_async_smem();
-            tc::fence_before_sync();
-            __syncthreads();
-            // dV^T += dO^T . wP, dK^T += Q^T . dS (over the tile's 128 rows), dQp = dS . K
-            if (tid == 0) {
+            };
+            // S = Q.K^T and U = dO.V^T of tile ti
+            auto issue_su = [&](int ti) {
+                const int buf = ti & 1;
+                const uint64_t aQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 16, 2048);
+                const uint64_t aO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 16, 2048);
+                const uint32_t ds = tmem + COL_SU + 128u * (uint32_t)buf;
                 tc::fence_after_sync();
-                const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 1024, 2048);
-                const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 1024, 2048);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t acc = (ti > 0 || ks > 0) ? 1u : 0u;
-                    tc::mma_bf16(tmem + COL_DV, tO + (uint64_t)((ks * 4096) >> 4),
-                                 bWP + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
-                    tc::mma_bf16(tmem + COL_DK, tQ + (uint64_t)((ks * 4096) >> 4),
-                                 bDS + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+                for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t acc = (kb | kk) ? 1u : 0u;
+                        tc::mma_bf16(ds, aQ + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                                     bK + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                        tc::mma_bf16(ds + 64, aO + (uint64_t)((kb * 1024 + kk * 32) >> 4),
+                                     bV + (uint64_t)((kb * 8192 + kk * 32) >> 4), IDESC_SU, acc);
+                    }
+                tc::mma_commit(&su_bar[buf]);
+            };
+            // K and V of the chunk (every product of the previous segment is
+            // complete: its last o_bar was waited below) and the first rows
+            const int krow = (int)(sg.bg * L + sg.first);
+            if (lane == 0) {
+                tc::mbar_expect_tx(kv_bar, 2u * 16384u);
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+                    tc::tma_load_2d(sm + OFF_K + kb * 8192, &tmK, kv_bar, kb * 64, krow);
+                    tc::tma_load_2d(sm + OFF_V + kb * 8192, &tmV, kv_bar, kb * 64, krow);
                 }
+            }
+            if (sg.ntiles > 0) load_rows(0);
+            if (sg.ntiles > 1) load_rows(1);
+            ok = bt_wait(kv_bar, pkv, s_abort) && (sg.ntiles == 0 || bt_wait(&tma_bar[0], ptma[0], s_abort));
+            ok = __all_sync(0xffffffffu, ok);
+            pkv ^= 1u;
+            if (sg.ntiles > 0) ptma[0] ^= 1u;
+            if (!ok) break;
+            if (sg.ntiles > 0 && lane == 0) issue_su(0);
+            for (int ti = 0; ti < sg.ntiles; ++ti) {
+                const int buf = ti & 1, nb = buf ^ 1;
+                // the segment's first dV^T / dK^T products overwrite the
+                // accumulators of the previous one: its readout must be done
+                if (ti == 0 && dkdv_held) {
+                    if (!__all_sync(0xffffffffu, bt_wait(seg_free, pfree, s_abort))) { ok = false; break; }
+                    pfree ^= 1u;
+                    dkdv_held = false;
+                }
+                if (!__all_sync(0xffffffffu, bt_wait(ds_full, pds, s_abort))) { ok = false; break; }
+                pds ^= 1u;
+                // dV^T += dO^T . wP, dK^T += Q^T . dS (over the tile's 128 rows), dQp = dS . K
+                if (lane == 0) {
+                    tc::fence_after_sync();
+                    const uint64_t tQ = tc::sdesc_sw128(tc::smem_u32(sm + OFF_Q + buf * QBUF), 1024, 2048);
+                    const uint64_t tO = tc::sdesc_sw128(tc::smem_u32(sm + OFF_DO + buf * QBUF), 1024, 2048);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + COL_DQ, aDS + (uint64_t)((kk * 32) >> 4),
-                                 bKt + (uint64_t)((kk * 2048) >> 4), IDESC_DQ, kk > 0 ? 1u : 0u);
-                tc::mma_commit(o_bar);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t acc = (ti > 0 || ks > 0) ? 1u : 0u;
+                        tc::mma_bf16(tmem + COL_DV, tO + (uint64_t)((ks * 4096) >> 4),
+                                     bWP + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+                        tc::mma_bf16(tmem + COL_DK, tQ + (uint64_t)((ks * 4096) >> 4),
+                                     bDS + (uint64_t)((ks * 2048) >> 4), IDESC_T, acc);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tmem + COL_DQ, aDS + (uint64_t)((kk * 32) >> 4),
+                                     bKt + (uint64_t)((kk * 2048) >> 4), IDESC_DQ, kk > 0 ? 1u : 0u);
+                    tc::mma_commit(o_bar);
+                }
+                // the next tile's S and U: behind this tile's products on the
+                // tensor pipe, so they run during this tile's epilogue
+                if (ti + 1 < sg.ntiles) {
+                    if (!__all_sync(0xffffffffu, bt_wait(&tma_bar[nb], ptma[nb], s_abort))) { ok = false; break; }
+                    ptma[nb] ^= 1u;
+                    if (lane == 0) issue_su(ti + 1);
+                }
+                // this tile's products are done with its Q / dO buffer: the rows
+                // of tile ti + 2 load into it
+                if (!__all_sync(0xffffffffu, bt_wait(o_bar, po, s_abort))) { ok = false; break; }
+                po ^= 1u;
+                if (ti + 2 < sg.ntiles) load_rows(ti + 2);
             }
-            // the next tile's S and U run during this tile's epilogue
-            if (more) {
-                if (!__syncthreads_and(bt_wait(&tma_bar[nb], ptma[nb], s_abort))) { ok = false; break; }
-                ptma[nb] ^= 1u;
-                if (tid == 0) issue_su(ti + 1);
-            }
-            if (!__syncthreads_and(bt_wait(o_bar, po, s_abort))) { ok = false; break; }
-            po ^= 1u;
-            tc::fence_after_sync();
-            // this tile's products are done with its Q / dO buffer: the rows of
-            // tile ti + 2 load into it while the epilogue runs
-            if (ti + 2 < ntiles) load_rows(ti + 2, nxt2);
-            // this row's dQ partial (fp16: 2^-11 relative, below the bf16
-            // rounding of dS it already carries), each half 64 columns, staged
-            // over the dS / wP tiles one 256-byte row per 272 bytes
-            uint8_t *stg = sm + OFF_DS + rt * STG_ROW;
+            if (sg.ntiles > 0) dkdv_held = true;
+        }
+    } else {
+        // ------------------------------------------------------------ compute
+        const int rt = tid & 127, hf = tid >> 7;          // tile row (TMEM lane), key half
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        float *red = (float *)(sm + OFF_RED);
+        const int e = rt >> 3, h = rt & 7;
+        uint32_t psu[2] = {0u, 0u}, po = 0u;
+        for (int64_t sidx = blockIdx.x; sidx < nseg && ok; sidx += gridDim.x) {
+            const BtSeg sg = bt_segment(p, sidx);
+            const int64_t b = sg.b;
+            const int g = sg.g;
+            auto row_of = [&](int ti) -> BtRow {
+                BtRow r;
+                const int u = ti * BT_EPT + e;
+                r.valid = u < sg.n_units;
+                r.t = -1;
+                r.slot = topk;
+                if (r.valid) {
+                    if (sg.own) {
+                        r.t = sg.first + u;
+                    } else {
+                        const int32_t code = p.entries[sg.ebase + u];
+                        r.t = code >> 5;
+                        r.slot = code & 31;
+                    }
+                }
+                return r;
+            };
+            // entry codes are read two tiles ahead and fusion weights one tile
+            // ahead, so neither load's latency sits on a tile's critical path
+            auto weight_of = [&](const BtRow &r) -> float {
+                if (!r.valid) return 0.f;
+                if (sg.own) return 1.f;
+                return p.coef[((b * L + r.t) * H + (int64_t)g * G + h) * topk + r.slot].x;
+            };
+            BtRow cur = row_of(0);
+            BtRow nxt = sg.ntiles > 1 ? row_of(1) : cur;
+            float w_cur = weight_of(cur);
+            for (int ti = 0; ti < sg.ntiles; ++ti) {
+                const int buf = ti & 1;
+                const bool more = ti + 1 < sg.ntiles;
+                const BtRow nxt2 = ti + 2 < sg.ntiles ? row_of(ti + 2) : nxt;
+                const float w_nxt = more ? weight_of(nxt) : 0.f;
+                const bool valid = cur.valid;
+                const int64_t t = cur.t;
+                const int slot = cur.slot;
+                const int64_t hrow = valid ? (b * L + t) * H + (int64_t)g * G + h : 0;
+                const float w = w_cur;
+                if (!cbar_and(bt_wait(&su_bar[buf], psu[buf], s_abort))) { ok = false; break; }
+                psu[buf] ^= 1u;
+                tc::fence_after_sync();
+                // this row's chunk softmax, dw, dS and w p over this thread's 32
+                // keys (j0 .. j0+31); the row max and the two sums are combined
+                // with the other half through shared memory
+                const int j0 = hf * 32;
+                float s[32], uu[32];
+                {
+                    const uint32_t ts = tmem + lane_off + COL_SU + 128u * (uint32_t)buf + (uint32_t)j0;
+                    tc::tmem_ld32(ts, s);
+                    tc::tmem_ld32(ts + 64, uu);
+                    tc::tmem_wait_ld();
+                }
+                const int nk = sg.own ? (valid ? (int)(t - sg.first) + 1 : 64) : 64;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mx = j0 + j < nk ? fmaxf(mx, s[j]) : mx;
+                red[hf * 128 + rt] = mx;
+                cbar();
+                mx = fmaxf(red[rt], red[128 + rt]);
+                // exp(scale (s - max)) as 2^(scale log2(e) (s - max)) on the MUFU unit
+                const float sl2 = p.scale * 1.4426950408889634f, ml2 = -sl2 * mx;
+                float z = 0.f, zu = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float ej = j0 + j < nk ? tc::ex2_approx(fmaf(s[j], sl2, ml2)) : 0.f;
+                    s[j] = ej;
+                    z += ej;
+                    zu = fmaf(ej, uu[j], zu);
+                }
+                red[256 + hf * 128 + rt] = z;
+                red[512 + hf * 128 + rt] = zu;
+                cbar();
+                z = red[256 + rt] + red[384 + rt];
+                zu = red[512 + rt] + red[640 + rt];
+                const float inv = 1.f / z;
+                const float dwv = zu * inv;
+                if (valid && hf == 0) p.dw[hrow * (topk + 1) + slot] = dwv;
+                const float fds = valid ? p.scale * w * inv : 0.f, fwp = valid ? w * inv : 0.f;
+#pragma unroll
+                for (int cq = 0; cq < 4; ++cq) {
+                    uint32_t ds4[4], wp4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int j = cq * 8 + 2 * i;
+                        ds4[i] = pack2_bf16(fds * s[j] * (uu[j] - dwv), fds * s[j + 1] * (uu[j + 1] - dwv));
+                        wp4[i] = pack2_bf16(fwp * s[j], fwp * s[j + 1]);
+                    }
+                    const uint32_t off = tc::sw128_offset(rt, hf * 4 + cq);
+                    *reinterpret_cast<uint4 *>(sm + OFF_DS + off) = make_uint4(ds4[0], ds4[1], ds4[2], ds4[3]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_WP + off) = make_uint4(wp4[0], wp4[1], wp4[2], wp4[3]);
+                }
+                // dS and w P are complete for this warp; the S / U slot is read
+                tc::fence_proxy_async_smem();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(ds_full);
+                if (!cbar_and(bt_wait(o_bar, po, s_abort))) { ok = false; break; }
+                po ^= 1u;
+                tc::fence_after_sync();
+                // this row's dQ partial (fp16: 2^-11 relative, below the bf16
+                // rounding of dS it already carries), each half 64 columns,
+                // straight from registers: a lane's 32-byte pieces are whole
+                // sectors, so no staging and no bulk copies
+                const int64_t qrow = valid ? (((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h : 0;
+                __half *dst = p.dqp + qrow * D;
 #pragma unroll 1
-            for (int cb = hf * 2; cb < hf * 2 + 2; ++cb) {
-                float v[32];
-                tc::tmem_ld32(tmem + lane_off + COL_DQ + cb * 32, v);
-                tc::tmem_wait_ld();
-                uint4 *d4 = reinterpret_cast<uint4 *>(stg + cb * 64);
+                for (int cb = hf * 2; cb < hf * 2 + 2; ++cb) {
+                    float v[32];
+                    tc::tmem_ld32(tmem + lane_off + COL_DQ + cb * 32, v);
+                    tc::tmem_wait_ld();
+                    if (valid) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    __half2 h0 = __floats2half2_rn(v[8 * i], v[8 * i + 1]);
-                    __half2 h1 = __floats2half2_rn(v[8 * i + 2], v[8 * i + 3]);
-                    __half2 h2 = __floats2half2_rn(v[8 * i + 4], v[8 * i + 5]);
-                    __half2 h3 = __floats2half2_rn(v[8 * i + 6], v[8 * i + 7]);
-                    d4[i] = make_uint4(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1),
-                                       *reinterpret_cast<uint32_t *>(&h2), *reinterpret_cast<uint32_t *>(&h3));
+                        for (int hq = 0; hq < 2; ++hq) {
+                            uint32_t w8[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                __half2 hv = __floats2half2_rn(v[16 * hq + 2 * i], v[16 * hq + 2 * i + 1]);
+                                w8[i] = *reinterpret_cast<uint32_t *>(&hv);
+                            }
+                            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                                         :: "l"(dst + cb * 32 + hq * 16), "r"(w8[0]), "r"(w8[1]), "r"(w8[2]),
+                                            "r"(w8[3]), "r"(w8[4]), "r"(w8[5]), "r"(w8[6]), "r"(w8[7])
+                                         : "memory");
+                        }
+                    }
+                }
+                cur = nxt;
+                nxt = nxt2;
+                w_cur = w_nxt;
+            }
+            if (!ok) break;
+            // the segment's dK and dV partials (thread = element of d; each half
+            // 32 keys); dl is written by bwd_dl_kernel
+            {
+                float *pk = p.part + sidx * (int64_t)(129 * D);
+                const int cb = hf;
+                const bool any = sg.ntiles > 0;
+                float vk[32], vv[32];
+                if (any) {
+                    tc::tmem_ld32(tmem + lane_off + COL_DK + cb * 32, vk);
+                    tc::tmem_ld32(tmem + lane_off + COL_DV + cb * 32, vv);
+                    tc::tmem_wait_ld();
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    pk[(cb * 32 + j) * D + rt] = any ? vk[j] : 0.f;
+                    pk[64 * D + (cb * 32 + j) * D + rt] = any ? vv[j] : 0.f;
+                }
+                if (any) {                   // TMEM dK / dV free for the next segment
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(seg_free);
                 }
             }
-            tc::fence_proxy_async_smem();
-            tc::fence_before_sync();
-            __syncthreads();          // TMEM dQ free for the next tile; the staging is complete
-            tc::fence_after_sync();
-            if (valid && hf == 0) {              // one bulk store per row: 256 bytes
-                __half *dst = p.dqp + ((((b * L + t) * p.Hkv + g) * (topk + 1) + slot) * G + h) * (int64_t)D;
-                tc::bulk_store(dst, stg, 256u);
-                tc::bulk_commit();
-            }
-            cur = nxt;
-            nxt = nxt2;
-            w_cur = w_nxt;
         }
-        if (!ok) break;
-        // the segment's dK and dV partials (thread = element of d; each half
-        // 32 keys); dl is written by bwd_dl_kernel
-        {
-            float *pk = p.part + sidx * (int64_t)(129 * D);
-            const int cb = hf;
-            float vk[32], vv[32];
-            tc::tmem_ld32(tmem + lane_off + COL_DK + cb * 32, vk);
-            tc::tmem_ld32(tmem + lane_off + COL_DV + cb * 32, vv);
-            tc::tmem_wait_ld();
-            const bool any = ntiles > 0;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                pk[(cb * 32 + j) * D + rt] = any ? vk[j] : 0.f;
-                pk[64 * D + (cb * 32 + j) * D + rt] = any ? vv[j] : 0.f;
-            }
-        }
-        tc::fence_before_sync();
-        __syncthreads();          // TMEM dK / dV free for the next segment
-        tc::fence_after_sync();
     }
-    if (hf == 0) tc::bulk_wait_all();      // this thread's dQ stores are complete
-    if (!ok) {
+    if (!ok) *s_abort = 1;
+    __syncthreads();
+    if (*s_abort) {
         if (tid == 0) atomicOr(p.status, kFlagTimeout);
         // let copies and MMAs that may still be in flight land before exiting
         const long long t0 = clock64();
