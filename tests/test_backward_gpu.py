@@ -157,6 +157,16 @@ def test_backward_tensor_core_path_agrees_with_cuda_cores(lm_mode, own):
             _close(name, a, _f64(r), RTOL_TC)
 
 
+@pytest.mark.parametrize("topk", [12, 29])
+def test_backward_tensor_core_more_than_eight_slots(topk):
+    # the fusion-weight kernel takes slots in groups of four and the row
+    # finish loops over every slot: K above eight spans several groups
+    wl = Workload("bwd", "prefill", "bf16", B=1, L=64 * 34 + 9, H=16, Hkv=2, d=128, topk=topk,
+                  seed=60 + topk)
+    backward_parity(wl, lm_mode="input")
+    backward_parity(wl.with_(seed=61 + topk), lm_mode="dhsa")
+
+
 def test_backward_tensor_core_long_chunk_lists():
     # 40 chunks, top-8, G = 8: chunk 0's entries span several segments of 8 tiles
     wl = Workload("bwd", "prefill", "bf16", B=1, L=64 * 40, H=8, Hkv=1, d=128, topk=8, seed=77)
