@@ -646,14 +646,34 @@ bwd_rowfin_kernel(const TL *__restrict__ lm, const int32_t *__restrict__ idx,
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
     const uint4 *qp = reinterpret_cast<const uint4 *>(dqp + tg * (int64_t)(topk + 1) * (G * D)) + lane;
-    for (int k = 0; k < topk; ++k) {
-        if (!((vmask >> k) & 1u)) continue;                  // warp-uniform
-        const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
-        uint4 raw[4];
+    // the own chunk's partials and the next valid slot's loads go out before
+    // the current slot is added (the slots are still added in index order)
+    uint4 ro[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) raw[j] = qp[(int64_t)k * (G * D / 8) + 32 * j];
-        float lv[8];
-        lm_load8<TL>(lm + (bg * Nc + ci) * D + d0, lv);
+    for (int j = 0; j < 4; ++j)
+        ro[j] = own_chunk ? qp[(int64_t)topk * (G * D / 8) + 32 * j] : make_uint4(0u, 0u, 0u, 0u);
+    auto load_slot = [&](int k, uint4 (&r)[4], float (&l)[8]) {
+        const int32_t ci = __shfl_sync(0xffffffffu, ci_l, k);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = qp[(int64_t)k * (G * D / 8) + 32 * j];
+        lm_load8<TL>(lm + (bg * Nc + ci) * D + d0, l);
+    };
+    unsigned rest = vmask;                                   // warp-uniform
+    int k = rest ? __ffs(rest) - 1 : -1;
+    uint4 raw[4];
+    float lv[8];
+    if (k >= 0) {
+        rest &= rest - 1;
+        load_slot(k, raw, lv);
+    }
+    while (k >= 0) {
+        const int kn = rest ? __ffs(rest) - 1 : -1;
+        uint4 rawn[4];
+        float lvn[8];
+        if (kn >= 0) {
+            rest &= rest - 1;
+            load_slot(kn, rawn, lvn);
+        }
         float dzk[G];
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) dzk[hh] = scale * __shfl_sync(0xffffffffu, dzr[hh], k);
@@ -668,12 +688,18 @@ bwd_rowfin_kernel(const TL *__restrict__ lm, const int32_t *__restrict__ idx,
                 acc[j][2 * e + 1] += f.y + dz * lv[2 * e + 1];
             }
         }
+        k = kn;
+        if (kn >= 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) raw[j] = rawn[j];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) lv[e] = lvn[e];
+        }
     }
     if (own_chunk) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint4 r = qp[(int64_t)topk * (G * D / 8) + 32 * j];
-            const __half2 *h2 = reinterpret_cast<const __half2 *>(&r);
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&ro[j]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __half22float2(h2[e]);
