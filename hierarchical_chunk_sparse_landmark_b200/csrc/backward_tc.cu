@@ -15,8 +15,9 @@
 //   dQp  = dS . K                       M = 128 rows, N = d, K = 64 keys
 //
 // The transposed products read the Q / dO / K tiles already in shared memory
-// as MN-major operands (no copy).  One persistent block per SM (8 warps; the
-// two threads of a tile row -- one TMEM lane -- take keys 0-31 and 32-63)
+// as MN-major operands (no copy).  One persistent block per SM (8 compute
+// warps, the two threads of a tile row -- one TMEM lane -- taking keys 0-31
+// and 32-63, and an issuer warp for the MMAs and row loads; see the kernel)
 // walks the segments of the chunks' sorted entry lists (at most 8 tiles each)
 // and the own chunks (at most 4 tiles of 16 tokens); K and V are loaded once
 // per segment.  dw and the dQ partial rows of every (row, slot) go to global
