@@ -201,8 +201,12 @@ template <int KP>
 __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, int lim, float scale,
                                            TopList<KP> &v, float &tf, float *stage, int r,
                                            float floor) {
+    // every bound is loosened by 1e-6 of its size: an unscaled score just
+    // below a bound can round to the same scaled score as one at the bound
+    // and then rank above it on its lower index, so it stays a candidate
+    // (-inf stays -inf)
     const float tq = tf / scale;                                // scale > 0
-    float tr = fmaxf(tq - fabsf(tq) * 1e-6f, floor);            // -inf stays -inf
+    float tr = fmaxf(tq - fabsf(tq) * 1e-6f, floor - fabsf(floor) * 1e-6f);
     if (tr == -INFINITY && lim == 32 && KP < 32) {
         // empty list, full block: the smallest of the maxima of KP groups of
         // 32/KP columns is a lower bound on the KP-th largest of the 32 (each
@@ -217,7 +221,7 @@ __device__ __forceinline__ void topk_block(const float (&sc)[32], int64_t c0, in
             for (int c = 1; c < GS; ++c) m = fmaxf(m, sc[g0 + c]);
             bound = fminf(bound, m);
         }
-        tr = bound;
+        tr = bound - fabsf(bound) * 1e-6f;
     }
     uint32_t mask = 0;
 #pragma unroll
