@@ -149,7 +149,7 @@ PrefillLayout prefill_layout(int B, int H, int Hkv, int64_t L, int d, int S, int
     off = align_up(off + sizeof(float) * (size_t)B * Hkv * Nc * d, 256);
     p.tokc_off = off;                // chunk of every token (variable-length chunks)
     if (varlen) off = align_up(off + sizeof(int32_t) * (size_t)L, 256);
-    p.bnds_off = off;                // checked boundaries + verdict (variable-length chunks)
+    p.bnds_off = off;                // checked boundaries + outcome (variable-length chunks)
     if (varlen) off = align_up(off + sizeof(int32_t) * (size_t)(Nc + 2), 256);
     p.tc = tc_shape_ok(B, H, Hkv, L, d, topk);
     p.W = p.NW = p.cap = 0;
